@@ -1,0 +1,434 @@
+"""Pins for the CPU oracle: it is checked against what the pages and the mathematics fix, never
+against itself.  Each test names the passage or the property it rests on."""
+import itertools
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    out = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            out.append([c.strip() for c in line.split("|")])
+    return out
+
+
+def f16(a):
+    return np.asarray(a, dtype=np.float16)
+
+
+# ----------------------------------------------------------------------------- check_24
+
+def test_toy_vectors(oracle):
+    """'Two half-zero vectors produce different pattern answers': A passes both groups, B
+    fails its first group, the extra zeros of B's second group repair nothing, and both are
+    50% zero overall."""
+    for name, vec, passes, nfail, zfrac in _rows("toy_vectors.txt"):
+        v = f16([float(x) for x in vec.split(",")]).reshape(1, -1)
+        p, n = oracle.check_24(v, oracle.F16, oracle.MATMUL)
+        assert p.ravel().tolist() == [int(x) for x in passes.split(",")], name
+        assert n == int(nfail), name
+        assert np.mean(v == 0) == float(zfrac), name
+
+
+@pytest.mark.parametrize("zeros,expect", [(0, 0), (1, 0), (2, 1), (3, 1), (4, 1)])
+def test_at_least_two_zeros(oracle, zeros, expect):
+    """'at least two zeros per four-entry group' (the operation section): 2, 3, 4 zeros pass."""
+    for pos in itertools.combinations(range(4), zeros):
+        g = f16([1.5, -2.0, 3.0, 4.0])
+        g[list(pos)] = 0
+        p, n = oracle.check_24(g.reshape(1, 4), oracle.F16)
+        assert p[0, 0] == expect and n == 1 - expect
+
+
+def test_zero_semantics(oracle):
+    """Both signed zeros count as zero; NaN and subnormals are not zero."""
+    cases = [([0.0, -0.0, 1.0, 1.0], 1), ([np.nan, 0.0, 1.0, 1.0], 0),
+             ([6e-8, 0.0, 1.0, 1.0], 0)]
+    for vals, expect in cases:
+        for dt, cast in ((oracle.F16, f16),
+                         (oracle.BF16, lambda a: synth.f32_to_bf16_bits(np.float32(a))),
+                         (oracle.F32, lambda a: np.asarray(a, np.float32))):
+            p, _ = oracle.check_24(cast(vals).reshape(1, 4), dt)
+            assert p[0, 0] == expect, (vals, dt)
+
+
+def test_conv_groups_run_along_c(oracle):
+    """'For Convolution weights [K,C,R,S] ... groups run along input channels C at each fixed
+    output channel and kernel position': the pass map equals the matmul check of the
+    [K, R, S, C] permuted view, re-indexed to [K, C/4, R, S]."""
+    g = synth.rng(3)
+    w = synth.structured_edge(g, 8 * 3 * 2, 12, "f16").reshape(8, 3, 2, 12)  # [K,R,S,C]
+    conv = np.ascontiguousarray(w.transpose(0, 3, 1, 2))                     # [K,C,R,S]
+    p_conv, n_conv = oracle.check_24(conv, oracle.F16, oracle.CONV)
+    p_mm, n_mm = oracle.check_24(np.ascontiguousarray(w), oracle.F16, oracle.MATMUL)
+    assert p_conv.shape == (8, 3, 3, 2)
+    assert np.array_equal(p_conv, p_mm.transpose(0, 3, 1, 2))
+    assert n_conv == n_mm
+    # flattening the conv tensor along its last axis would group the wrong entries
+    p_flat, _ = oracle.check_24(conv.reshape(8, -1), oracle.F16, oracle.MATMUL)
+    assert p_flat.size == p_conv.size and not np.array_equal(p_flat.ravel(), p_conv.ravel())
+
+
+def test_conv_c_not_multiple_of_four_rejected(oracle):
+    with pytest.raises(oracle.OracleError):
+        oracle.check_24(np.zeros((2, 6, 3, 3), np.float16), oracle.F16, oracle.CONV)
+    with pytest.raises(oracle.OracleError):
+        oracle.check_24(np.zeros((2, 6), np.float16), oracle.F16, oracle.MATMUL)
+
+
+def test_conv_fail5_generator_counts(oracle):
+    d = synth.conv_fail5(shape=(16, 16, 3, 3))
+    G = 16 * 4 * 9
+    p, n = oracle.check_24(d["W"], oracle.F16, oracle.CONV)
+    assert n == round(0.05 * G)
+    assert np.array_equal(np.flatnonzero(p.ravel() == 0), d["failing"])
+
+
+# ----------------------------------------------------------------------------- prune
+
+def _brute_keep(mags):
+    """All C(4,2) choices; keep the one with the largest sum of magnitudes, ties -> the
+    lexicographically smallest ascending pair."""
+    best, bsum = None, -1.0
+    for pair in itertools.combinations(range(4), 2):
+        s = mags[pair[0]] + mags[pair[1]]
+        if s > bsum:
+            best, bsum = pair, s
+    return best
+
+
+def test_prune_brute_force(oracle):
+    """Magnitude pruning to 2 of 4 ('What 2:4 actually is'; ties to the lower index) equals
+    brute-force enumeration of the six 2-of-4 choices.  fp16 magnitudes make every pair sum
+    exact in fp64, so the enumeration decides ties exactly."""
+    g = synth.rng(11)
+    w = synth.structured_edge(g, 64, 256, "f16")
+    vals, meta = oracle.compress_24(w, oracle.F16)
+    pr = oracle.prune_24(w, oracle.F16)
+    mags = np.abs(w.astype(np.float64)).reshape(-1, 4)
+    nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()[: mags.shape[0]]
+    for gi in range(mags.shape[0]):
+        i0, i1 = _brute_keep(mags[gi])
+        assert (nib[gi] & 3, nib[gi] >> 2) == (i0, i1), gi
+        row = pr.reshape(-1, 4)[gi].view(np.uint16)
+        src = w.reshape(-1, 4)[gi].view(np.uint16)
+        for i in range(4):
+            assert row[i] == (src[i] if i in (i0, i1) else 0)
+
+
+def test_prune_exhaustive_small_alphabet(oracle):
+    """Every group over the magnitudes {0, 1, 2} with both signs (6^4 groups)."""
+    alphabet = [0.0, -0.0, 1.0, -1.0, 2.0, -2.0]
+    groups = np.array(list(itertools.product(alphabet, repeat=4)), dtype=np.float16)
+    vals, meta = oracle.compress_24(groups.reshape(1, -1), oracle.F16)
+    nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()
+    for gi, grp in enumerate(groups.astype(np.float64)):
+        i0, i1 = _brute_keep(np.abs(grp))
+        assert (nib[gi] & 3, nib[gi] >> 2) == (i0, i1)
+
+
+def test_prune_ties_and_zeros(oracle):
+    """[0,0,5,0] keeps indices 0 and 2 (reading: exactly two kept, zeros by the tie rule);
+    equal magnitudes of opposite sign tie on magnitude, the lower index wins."""
+    cases = {(0, 0, 5, 0): (0, 2), (1, 1, 1, 1): (0, 1), (-2, 1, 2, 1): (0, 2),
+             (1, -3, 3, 0): (1, 2), (0, 0, 0, 7): (0, 3)}
+    for vals, pair in cases.items():
+        v, m = oracle.compress_24(f16(vals).reshape(1, 4), oracle.F16)
+        assert (m[0] & 3, m[0] >> 2) == pair, vals
+        assert np.array_equal(v.ravel().astype(np.float64), np.array(vals, np.float64)[list(pair)])
+
+
+def test_prune_nan_is_largest(oracle):
+    v, m = oracle.compress_24(f16([np.nan, 1, 2, 3]).reshape(1, 4), oracle.F16)
+    assert (m[0] & 3, m[0] >> 2) == (0, 3)
+
+
+def test_prune_fp32_bf16_order(oracle):
+    """Magnitude order follows the value, for every storage type (|w| bit patterns are
+    monotone in |w|)."""
+    g = synth.rng(5)
+    x = synth.normal(g, (32, 64))
+    for dt, st in ((oracle.F32, "f32"), (oracle.BF16, "bf16")):
+        w = synth.as_storage(x, st)
+        _, meta = oracle.compress_24(w, dt)
+        wf = synth.bf16_bits_to_f32(w) if st == "bf16" else w
+        mags = np.abs(wf.astype(np.float64)).reshape(-1, 4)
+        nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()
+        order = np.argsort(-mags, axis=1, kind="stable")[:, :2]
+        order.sort(axis=1)
+        assert np.array_equal(nib & 3, order[:, 0]) and np.array_equal(nib >> 2, order[:, 1])
+
+
+def test_roundtrip_and_meta_legal(oracle):
+    """decompress(compress(W)) == prune(W) bitwise; every nibble is one of the six ascending
+    index pairs; the pruned tensor passes the check in every group."""
+    g = synth.rng(7)
+    for dt, st in ((oracle.F16, "f16"), (oracle.BF16, "bf16"), (oracle.F32, "f32")):
+        w = synth.structured_edge(g, 24, 96, st)
+        vals, meta = oracle.compress_24(w, dt)
+        back = oracle.decompress_24(vals, meta, dt, w.shape)
+        pr = oracle.prune_24(w, dt)
+        assert np.array_equal(back.view(np.uint8), pr.view(np.uint8))
+        nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()
+        assert set(np.unique(nib).tolist()) <= {0x4, 0x8, 0xC, 0x9, 0xD, 0xE}
+        p, n = oracle.check_24(pr, dt)
+        assert n == 0 and p.all()
+
+
+def test_conv_roundtrip(oracle):
+    g = synth.rng(8)
+    w = synth.structured_edge(g, 4 * 8, 3 * 3, "f16").reshape(4, 8, 3, 3)
+    vals, meta = oracle.compress_24(w, oracle.F16, oracle.CONV)
+    assert vals.shape == (4, 4, 3, 3) and meta.size == 4 * 2 * 9 // 2
+    back = oracle.decompress_24(vals, meta, oracle.F16, w.shape, oracle.CONV)
+    assert np.array_equal(back.view(np.uint16), oracle.prune_24(w, oracle.F16, oracle.CONV).view(np.uint16))
+    # the conv prune equals the matmul prune of the [K,R,S,C] view
+    mm = np.ascontiguousarray(w.transpose(0, 2, 3, 1))
+    pr_mm = oracle.prune_24(mm, oracle.F16).transpose(0, 3, 1, 2)
+    assert np.array_equal(back.view(np.uint16), np.ascontiguousarray(pr_mm).view(np.uint16))
+
+
+def test_decompress_rejects_illegal_nibble(oracle):
+    with pytest.raises(oracle.OracleError):
+        oracle.decompress_24(np.zeros(2, np.float16), np.array([0x5], np.uint8), oracle.F16, (4,))
+
+
+def test_storage_bits_per_weight(oracle):
+    """'The byte saving is about a quarter, not a half': sizes of what the oracle emits."""
+    expect = {r[0]: float(r[1]) for r in _rows("bits_per_weight.txt")}
+    N, K = 64, 256
+    w = synth.draw(synth.rng(1), (N, K), "f16")
+    vals, meta = oracle.compress_24(w, oracle.F16)
+    assert (vals.nbytes + meta.nbytes) * 8 / (N * K) == expect["fp16_sparse24"]
+    assert w.nbytes * 8 / (N * K) == expect["fp16_dense"]
+    codes, scales, _ = oracle.nvfp4_encode(w, oracle.F16)
+    dense_bits = (codes.nbytes + scales.nbytes) * 8 / (N * K)
+    assert dense_bits == expect["nvfp4_dense"]
+    vcodes, vscales, _ = oracle.nvfp4_encode(vals, oracle.F16)
+    sparse_bits = (vcodes.nbytes + vscales.nbytes + meta.nbytes) * 8 / (N * K)
+    assert sparse_bits == expect["nvfp4_sparse24"]
+    assert abs((1 - sparse_bits / dense_bits) - expect["saving_nvfp4"]) < 0.005
+
+
+# ----------------------------------------------------------------------------- NVFP4
+
+def test_byte_counts_of_real_tensors(oracle):
+    """'Bit-exact check against lyf's ModelOpt output': packed / block-scale / global-scale
+    byte counts.  The out_proj-sized tensor is encoded for real; all three rows check the
+    packed : scales = 8 : 1 accounting."""
+    for name, rows, cols, packed, scl, glob in _rows("nvfp4_byte_counts.txt"):
+        rows, cols = int(rows), int(cols)
+        assert rows * cols // 2 == int(packed) and rows * cols // 16 == int(scl), name
+        if name == "out_proj":
+            t = np.zeros((rows, cols), dtype=np.uint16)
+            codes, scales, ts = oracle.nvfp4_encode(t, oracle.BF16)
+            assert codes.nbytes == int(packed) and scales.nbytes == int(scl)
+            assert np.float32(ts).nbytes == int(glob)
+
+
+def test_e2m1_against_ml_dtypes(oracle):
+    """E2M1 decode and round-to-nearest-even (saturating) agree with ml_dtypes' float4_e2m1fn,
+    an independent implementation of the format, over every code and every midpoint."""
+    lib_vals = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    ours = np.array([oracle.e2m1_value(c) for c in range(16)])
+    assert np.array_equal(ours, lib_vals) and np.array_equal(np.signbit(ours), np.signbit(lib_vals))
+    pos = lib_vals[:8]
+    probes = np.concatenate([pos, (pos[1:] + pos[:-1]) / 2, pos + 0.01, pos - 0.01,
+                             [6.5, 7.0, 7.5, 100.0, 1e30]])
+    probes = probes[probes >= 0]
+    lib_codes = probes.astype(np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    for x, c in zip(probes, lib_codes):
+        assert oracle.e2m1_round(x) == int(c), x
+
+
+def test_e4m3_against_ml_dtypes(oracle):
+    """E4M3 decode of all 256 codes and RNE of every midpoint and random in-range values agree
+    with ml_dtypes' float8_e4m3fn; above 448 the oracle saturates (satfinite)."""
+    lib_vals = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    ours = np.array([oracle.e4m3_value(c) for c in range(256)])
+    nan = np.isnan(lib_vals)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], lib_vals[~nan])
+    pos = lib_vals[:127]
+    mids = (pos[1:] + pos[:-1]) / 2
+    rnd = synth.rng(2).uniform(0, 448, 4000)
+    tiny = synth.rng(3).uniform(0, 2.0 ** -6, 2000)
+    probes = np.concatenate([pos, mids, rnd, tiny]).astype(np.float32)
+    lib_codes = probes.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    for x, c in zip(probes, lib_codes):
+        assert oracle.e4m3_round(float(x)) == int(c), x
+    for x in (448.0, 455.0, 464.0, 1e6):
+        assert oracle.e4m3_round(x) == 0x7E
+
+
+def _codes_nibbles(codes):
+    return np.stack([codes & 0xF, codes >> 4], -1).reshape(codes.shape[0], -1)
+
+
+def test_nvfp4_error_bound(oracle):
+    """Every code is the nearest E2M1 point to |t| / (dec(sb) s_t) (the format's rounding
+    bound: at most half a grid step away), and the block scale maps the block maximum close to
+    6 (within E4M3's relative half step, 1/16)."""
+    g = synth.rng(4)
+    x = synth.normal(g, (16, 128)) * np.exp(synth.normal(g, (16, 1)))  # rows of varied scale
+    t = synth.as_storage(x, "bf16")
+    codes, scales, ts = oracle.nvfp4_encode(t, oracle.BF16)
+    tf = synth.bf16_bits_to_f32(t).astype(np.float64)
+    assert np.float32(ts) == np.float32(np.float32(np.abs(tf).max()) / np.float32(2688.0))
+    sb = np.array([[oracle.e4m3_value(c) for c in row] for row in scales])
+    nib = _codes_nibbles(codes)
+    grid = np.array([oracle.e2m1_value(c) for c in range(8)])
+    q = np.abs(tf) / (np.repeat(sb, 16, axis=1) * np.float64(ts))
+    dist = np.abs(grid[nib & 7] - q)
+    step = np.where(q < 2, 0.5, np.where(q < 4, 1.0, 2.0))
+    assert np.all(dist <= step / 2 + 1e-6)
+    assert np.array_equal(nib >> 3, np.signbit(tf).astype(np.int64))
+    bmax = np.abs(tf).reshape(16, -1, 16).max(-1)
+    ratio = bmax / (sb * 6 * np.float64(ts))
+    assert np.all(np.abs(ratio - 1) <= 1 / 16 + 1e-6)
+
+
+def test_nvfp4_negative_zero_kept(oracle):
+    """'keeping FP4 negative zero' (the bit-exact check): a negative value that rounds to zero,
+    and -0 itself, keep the sign bit."""
+    t = np.zeros((1, 16), np.float32)
+    t[0, 0] = 1.0
+    t[0, 1] = -1e-9
+    t[0, 2] = -0.0
+    codes, scales, ts = oracle.nvfp4_encode(t, oracle.F32)
+    nib = _codes_nibbles(codes)[0]
+    assert nib[1] == 0x8 and nib[2] == 0x8 and nib[3] == 0x0
+    assert nib[0] == 0x7 and scales[0, 0] == 0x7E  # 1.0 -> 6 * 448 * s_t
+
+
+def test_nvfp4_all_zero_and_supplied_scale(oracle):
+    t = np.zeros((2, 32), np.float32)
+    t[1, 5] = -0.0
+    codes, scales, ts = oracle.nvfp4_encode(t, oracle.F32)
+    assert ts == 0 and not scales.any() and _codes_nibbles(codes)[1, 5] == 8
+    x = synth.normal(synth.rng(9), (4, 64)).astype(np.float32)
+    own = oracle.nvfp4_encode(x, oracle.F32)
+    shared = oracle.nvfp4_encode(x, oracle.F32, tensor_scale=float(own[2]))
+    assert all(np.array_equal(a, b) for a, b in zip(own[:2], shared[:2]))
+    # a shared scale taken from a larger partner tensor ('The shared global scale') changes
+    # the block scales of this one but not its sizes
+    big = oracle.nvfp4_encode(x, oracle.F32, tensor_scale=float(own[2]) * 8)
+    assert big[2] == np.float32(own[2]) * 8 and not np.array_equal(big[1], own[1])
+    # a scale far too small saturates codes at 6 and block scales at 448
+    tiny = oracle.nvfp4_encode(x, oracle.F32, tensor_scale=float(own[2]) / 1e4)
+    assert (tiny[1] == 0x7E).all()
+
+
+def test_nvfp4_requantisation_is_stable(oracle):
+    """'Bit-exact check': decode, re-quantise, compare byte for byte -> packed codes and block
+    scales identical; the re-estimated global scale may move by about one ULP (decoding
+    cannot recover the original extremes).  Checked with fp32 and bf16 decodes."""
+    g = synth.rng(10)
+    for trial in range(4):
+        x = synth.normal(g, (32, 256)) * (0.02 if trial % 2 else 1.0)
+        t = synth.as_storage(x, "bf16")
+        codes, scales, ts = oracle.nvfp4_encode(t, oracle.BF16)
+        dec = oracle.nvfp4_decode(codes, scales, ts)
+        re32 = oracle.nvfp4_encode(dec.astype(np.float32), oracle.F32)
+        assert np.array_equal(re32[0], codes) and np.array_equal(re32[1], scales)
+        assert abs(int(np.float32(re32[2]).view(np.int32)) - int(np.float32(ts).view(np.int32))) <= 1
+        re16 = oracle.nvfp4_encode(synth.as_storage(dec, "bf16"), oracle.BF16)
+        assert np.array_equal(re16[0], codes) and np.array_equal(re16[1], scales)
+
+
+def test_amax_survives_pruning(oracle):
+    """The largest |w| of every group is always kept, so the tensor scale of the compressed
+    values equals the tensor scale of the dense weight."""
+    g = synth.rng(12)
+    w = synth.draw(g, (64, 512), "bf16", 0.02)
+    vals, _ = oracle.compress_24(w, oracle.BF16)
+    assert oracle.nvfp4_tensor_scale(vals, oracle.BF16) == oracle.nvfp4_tensor_scale(w, oracle.BF16)
+
+
+# ----------------------------------------------------------------------------- GEMM
+
+def test_gemm_matches_library_matmul(oracle):
+    g = synth.rng(13)
+    X = synth.normal(g, (7, 40))
+    W = synth.normal(g, (9, 40))
+    Y, S = oracle.gemm(X, W)
+    assert np.allclose(Y, X @ W.T, rtol=1e-13, atol=1e-13)
+    assert np.allclose(S, np.abs(X) @ np.abs(W).T, rtol=1e-13)
+    # orientation: a one-hot X row selects column k of W, i.e. Y[m, n] = W[n, k]
+    E = np.zeros((1, 40))
+    E[0, 3] = 1.0
+    assert np.array_equal(oracle.gemm(E, W)[0][0], W[:, 3])
+
+
+def test_sparse_gemm_equals_dense_on_pruned(oracle):
+    """Summing over kept entries via the metadata equals the dense sum over the pruned weight
+    exactly in fp64 (the pruned entries are exact zeros)."""
+    g = synth.rng(14)
+    w = synth.draw(g, (24, 64), "f16")
+    x = synth.draw(g, (5, 64), "f16")
+    vals, meta = oracle.compress_24(w, oracle.F16)
+    pruned = oracle.prune_24(w, oracle.F16)
+    X = oracle.to_double(x, oracle.F16)
+    Ys, Ss = oracle.gemm_sparse(X, oracle.to_double(vals, oracle.F16), meta)
+    Yd, Sd = oracle.gemm(X, oracle.to_double(pruned, oracle.F16))
+    assert np.array_equal(Ys, Yd) and np.array_equal(Ss, Sd)
+    assert np.allclose(Yd, X @ oracle.to_double(pruned, oracle.F16).T, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_gemm_nvfp4_values(oracle):
+    """Sparse NVFP4 (reading: one block scale per 16 stored values): the product with decoded
+    values through the metadata equals the dense product with the decompressed decode."""
+    g = synth.rng(15)
+    w = synth.draw(g, (16, 128), "bf16", 0.02)
+    x = synth.draw(g, (3, 128), "bf16")
+    vals, meta = oracle.compress_24(w, oracle.BF16)
+    c, s, ts = oracle.nvfp4_encode(vals, oracle.BF16)
+    V = oracle.nvfp4_decode(c, s, ts)
+    Wd = np.zeros((16, 128))
+    nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()
+    for gi in range(16 * 32):
+        n, j = divmod(gi, 32)
+        Wd[n, 4 * j + (nib[gi] & 3)] = V[n, 2 * j]
+        Wd[n, 4 * j + (nib[gi] >> 2)] = V[n, 2 * j + 1]
+    X = oracle.to_double(x, oracle.BF16)
+    Ys, _ = oracle.gemm_sparse(X, V, meta)
+    assert np.allclose(Ys, X @ Wd.T, rtol=1e-12, atol=1e-15)
+
+
+def test_moe_matches_per_token_matmul(oracle):
+    g = synth.rng(16)
+    E, N, K, T, topk = 6, 8, 32, 5, 3
+    W = synth.normal(g, (E, N, K))
+    X = synth.normal(g, (T, K))
+    r = synth.routing_topk(g, T, E, topk)
+    Y, S = oracle.moe(X, r, W)
+    for t in range(T):
+        for s in range(topk):
+            assert np.allclose(Y[t, s], W[r[t, s]] @ X[t], rtol=1e-13, atol=1e-13)
+            assert np.allclose(S[t, s], np.abs(W[r[t, s]]) @ np.abs(X[t]), rtol=1e-13)
+    with pytest.raises(oracle.OracleError):
+        oracle.moe(X, np.full((T, topk), E, np.int32), W)
+
+
+def test_routing_generator_distinct():
+    g = synth.rng(0)
+    r = synth.routing_topk(g, 200, 512, 10)
+    assert all(len(set(row)) == 10 for row in r.tolist())
+    assert r.min() >= 0 and r.max() < 512
+
+
+def test_tolerance_rule(oracle):
+    ok = oracle.within_tolerance(np.array([1.0005, 0.0, 1e-9]), np.array([1.0, 0.0, 0.0]),
+                                 np.array([1.0, 0.0, 0.0]))
+    assert ok.tolist() == [True, True, False]
