@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the 2:4-sparse vs dense NVFP4 pipeline on the decode-shaped workload.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+
+    check_24(W) -> prune_compress_24(W) -> quantize_nvfp4(W) -> quantize_nvfp4(values)
+    -> gemm_dense(X, W_nvfp4) -> gemm_sparse24(X, values_nvfp4 + meta)
+
+Workload: X bf16 [8, 5120] N(0, 1), W bf16 [5120, 5120] N(0, 0.02) (the decode shape of the
+pages' NVFP4 decode kernels, hidden width 5120).  Inputs live in HBM before timing starts and
+rotate over 4 seeded input sets (about 440 MB in total, well beyond the 126 MB L2), so each
+step reads its weight from DRAM.
+
+Each stage is captured once per input set as a CUDA graph; the timed loop replays the stage
+graphs and records a CUDA event after each stage, which gives the per-stage device time inside
+the timed region.  `value` is the whole step's algorithmic HBM traffic divided by the step
+time (GB/s); the GEMV comparison (dense vs 2:4 sparse: TFLOP/s, GB/s, speedup) is in `gemv`.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --impl reference the CPU oracle (oracle/, plain scalar C) is timed on the host cores on
+a bounded row sample of the same workload: that arm is a reported baseline, not the target.
+Under torchrun every rank runs an independent replica (no collective on the data path);
+rank 0 prints the JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, K = 8, 5120, 5120
+METRIC = "2:4-sparse vs dense GEMM eff. TFLOP/s & HBM GB/s per shape; sparse/dense speedup"
+WORKLOAD = ("decode_nvfp4: X bf16 [8,5120] N(0,1), W bf16 [5120,5120] N(0,0.02); step = "
+            "check_24 + prune_compress_24 + quantize_nvfp4(W) + quantize_nvfp4(values) + "
+            "gemm_dense(X,W_nvfp4) + gemm_sparse24(X,values_nvfp4,meta)")
+STAGES = ("check_24", "prune_compress_24", "quantize_w", "quantize_values", "gemm_dense",
+          "gemm_sparse24")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def stage_bytes(rows: int = N) -> dict:
+    """Algorithmic bytes each stage must move for `rows` weight rows (each operand once; the
+    NVFP4 quantiser reads its input twice because the tensor amax must be known before any
+    block is encoded)."""
+    w = rows * K * 2                      # bf16 weight
+    v = rows * K // 2 * 2                 # kept values, bf16
+    meta = rows * K // 8
+    x = M * K * 2
+    y = M * rows * 4
+    codes_w, scales_w = rows * K // 2, rows * K // 16
+    codes_v, scales_v = rows * K // 4, rows * K // 32
+    return {
+        "check_24": w + rows * K // 4 + 4,
+        "prune_compress_24": w + v + meta,
+        "quantize_w": 2 * w + codes_w + scales_w + 4,
+        "quantize_values": 2 * v + codes_v + scales_v + 4,
+        "gemm_dense": codes_w + scales_w + 4 + x + y,
+        "gemm_sparse24": codes_v + scales_v + 4 + meta + x + y,
+    }
+
+
+def gemv_flops(rows: int = N) -> float:
+    return 2.0 * M * rows * K  # dense-equivalent for both GEMVs
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(kernel_stage: str):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_stage)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, rec["source"])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if sha != rec["source_sha"]:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def run_ours(args, rank: int, world: int, dist) -> dict | None:
+    import torch
+
+    import fp16_gemm_b200 as sp
+    import synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    bf16 = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    sets = []
+    for i in range(args.sets):
+        d = synth.decode_nvfp4(seed=i)
+        s = {"x": bf16(d["X"]), "w": bf16(d["W"])}
+        s["pass"] = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+        s["nfail"] = torch.empty(1, dtype=torch.int32, device=dev)
+        s["v"] = torch.empty((N, K // 2), dtype=torch.bfloat16, device=dev)
+        s["m"] = torch.empty(N * K // 8, dtype=torch.uint8, device=dev)
+        s["wq"] = sp.NVFP4Tensor(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                                 torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
+                                 torch.empty(1, dtype=torch.float32, device=dev))
+        s["vq"] = sp.NVFP4Tensor(torch.empty((N, K // 4), dtype=torch.uint8, device=dev),
+                                 torch.empty((N, K // 32), dtype=torch.uint8, device=dev),
+                                 torch.empty(1, dtype=torch.float32, device=dev))
+        s["yd"] = torch.empty((M, N), dtype=torch.float32, device=dev)
+        s["ys"] = torch.empty((M, N), dtype=torch.float32, device=dev)
+        sets.append(s)
+    ws = torch.empty(sp.quantize_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+
+    def stage_fns(s):
+        sparse_w = sp.Sparse24(s["vq"], s["m"])
+        return [
+            lambda: sp.check_24(s["w"], pass_out=s["pass"], n_fail_out=s["nfail"]),
+            lambda: sp.prune_compress_24(s["w"], values_out=s["v"], meta_out=s["m"]),
+            lambda: sp.quantize_nvfp4(s["w"], out=s["wq"], workspace=ws),
+            lambda: sp.quantize_nvfp4(s["v"], out=s["vq"], workspace=ws),
+            lambda: sp.gemm_dense(s["x"], s["wq"], out=s["yd"]),
+            lambda: sp.gemm_sparse24(s["x"], sparse_w, K, out=s["ys"]),
+        ]
+
+    # eager warm-up (also caches the SM count before capture)
+    for s in sets:
+        for f in stage_fns(s):
+            f()
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
+
+    # capture one graph per (set, stage)
+    graphs = []
+    n0 = sp.kernel_launches()
+    cap = torch.cuda.Stream()
+    for s in sets:
+        row = []
+        for f in stage_fns(s):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                f()
+            row.append(g)
+        graphs.append(row)
+    launches_per_step = (sp.kernel_launches() - n0) // len(sets)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def run_steps(n, events=None, offset=0):
+        for j in range(n):
+            row = graphs[(offset + j) % len(graphs)]
+            for si, g in enumerate(row):
+                g.replay()
+                if events is not None:
+                    events[j][si + 1].record(stream)
+
+    run_steps(args.warmup)
+    torch.cuda.synchronize()
+
+    # per-step, per-stage events (fresh objects: nothing is overwritten before it is read)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+           for _ in range(args.steps)]
+    for j in range(args.steps):
+        evs[j][0] = evs[j - 1][-1] if j > 0 else torch.cuda.Event(enable_timing=True)
+    t_start = evs[0][0]
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    host0 = time.perf_counter()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_start.record(stream)
+        run_steps(args.steps, evs, offset=args.warmup)
+        host_enqueue = time.perf_counter() - host0
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t_end = evs[-1][-1]
+    total_ms = t_start.elapsed_time(t_end)
+    stage_ms = [sum(evs[j][si].elapsed_time(evs[j][si + 1]) for j in range(args.steps)) / args.steps
+                for si in range(len(STAGES))]
+
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    bytes_ = stage_bytes()
+    step_bytes = sum(bytes_.values())
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    s0 = sets[0]
+    d0 = synth.decode_nvfp4(seed=0)
+    hx = torch.from_numpy(d0["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hw = torch.from_numpy(d0["W"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hyd = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    hys = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    hnf = torch.empty(1, dtype=torch.int32).pin_memory()
+    fns = stage_fns(s0)
+
+    def e2e_step():
+        s0["x"].copy_(hx, non_blocking=True)
+        s0["w"].copy_(hw, non_blocking=True)
+        for f in fns:
+            f()
+        hyd.copy_(s0["yd"], non_blocking=True)
+        hys.copy_(s0["ys"], non_blocking=True)
+        hnf.copy_(s0["nfail"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    # results are still correct after all the replays (cheap sanity, outside timing)
+    assert sp.last_device_error() == sp.OK
+    assert int(hnf.item()) == N * K // 4  # raw normal weights: every group fails the check
+
+    if rank != 0:
+        return None
+
+    peak, peak_kind = peaks()
+    stages = {}
+    for name, ms in zip(STAGES, stage_ms):
+        gbs = bytes_[name] / (ms * 1e-3) / 1e9
+        stages[name] = {"us": round(ms * 1e3, 3), "bytes": bytes_[name], "GB/s": round(gbs, 1),
+                        "frac_hbm": round(gbs / peak, 3)}
+    dom = max(STAGES, key=lambda n: stages[n]["us"])
+    rec = traffic_record(dom)
+    achieved = stages[dom]["GB/s"]
+    gd, gs = stages["gemm_dense"], stages["gemm_sparse24"]
+    fl = gemv_flops()
+    return {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "sets": args.sets,
+                   "l2": f"{args.sets} rotating input sets (~{args.sets * 111} MB) > 126 MB L2",
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
+        "gemv": {
+            "dense": {"us": gd["us"], "TFLOP/s": round(fl / (gd["us"] * 1e-6) / 1e12, 2),
+                      "GB/s": gd["GB/s"], "bytes": gd["bytes"]},
+            "sparse24": {"us": gs["us"], "TFLOP/s (dense-equiv)": round(fl / (gs["us"] * 1e-6) / 1e12, 2),
+                         "GB/s": gs["GB/s"], "bytes": gs["bytes"]},
+            "sparse_dense_speedup": round(gd["us"] / gs["us"], 3),
+            "arith_intensity_flop_per_byte": {"dense": round(fl / gd["bytes"], 1),
+                                              "sparse24": round(fl / gs["bytes"], 1)},
+        },
+        "stages": stages,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 3),
+                     "traffic": None if rec is None else rec["traffic_bytes_per_launch"]},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "steps": args.e2e_steps,
+                "h2d_bytes_per_step": hx.numel() * 2 + hw.numel() * 2,
+                "d2h_bytes_per_step": hyd.numel() * 4 + hys.numel() * 4 + 4},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": int(launches_per_step),
+        "host_enqueue_ms": round(host_enqueue * 1e3, 2),
+        "clocks": clk.summary(),
+    }
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def oracle_pipeline(X, Wrows):
+    """One pass of the pipeline in the CPU oracle over a row sample of W."""
+    import oracle
+    od = oracle.BF16
+    oracle.check_24(Wrows, od)
+    V, meta = oracle.compress_24(Wrows, od)
+    cw, sw, tw = oracle.nvfp4_encode(Wrows, od)
+    cv, sv, tv = oracle.nvfp4_encode(V, od)
+    Xd = oracle.to_double(X, od)
+    oracle.gemm(Xd, oracle.nvfp4_decode(cw, sw, tw))
+    oracle.gemm_sparse(Xd, oracle.nvfp4_decode(cv, sv, tv), meta)
+
+
+def cpu_baseline(budget_s: float, steps: int = 1):
+    """Times the oracle on bounded row samples; returns (GB/s, seconds, rows per step, cores)."""
+    import oracle
+    import synth
+    d = synth.decode_nvfp4(seed=0)
+    X, W = d["X"], d["W"]
+    cores = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle_pipeline(X, np.ascontiguousarray(W[:32]))
+    per_row = (time.perf_counter() - t0) / 32
+    rows = int(max(8, min(N, budget_s / max(per_row, 1e-9) / steps)) // 8 * 8)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        r0 = (i * rows) % (N - rows + 1)
+        oracle_pipeline(X, np.ascontiguousarray(W[r0:r0 + rows]))
+    dt = time.perf_counter() - t0
+    gbs = steps * sum(stage_bytes(rows).values()) / dt / 1e9
+    return gbs, dt, rows, cores
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sets", type=int, default=4)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        # the CPU oracle on the host cores; under torchrun only rank 0 works
+        if rank != 0:
+            return
+        budget = 90.0
+        per_step_budget = budget / max(1, args.steps + args.warmup)
+        gbs, dt, rows, cores = cpu_baseline(per_step_budget * args.steps, steps=args.steps)
+        sample = f"{rows} of {N} weight rows per step (rotating), all stages, {args.steps} steps"
+        line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K},
+                "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+
+    # CPU baseline first (rank 0, N=1 only), before any GPU work forks anything
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, dt, rows, cores = cpu_baseline(args.cpu_budget)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} of {N} weight rows, all six stages once ({dt:.1f} s)"}
+
+    line = run_ours(args, rank, world, dist)
+    if line is not None:
+        line["cpu_baseline"] = cpu
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

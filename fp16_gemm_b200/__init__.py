@@ -1,0 +1,329 @@
+"""Python binding of libsp24 (the C ABI declared in include/sp24.h).
+
+Argument marshalling only: every step of the pipeline runs in the CUDA kernels of
+``libsp24.so``.  PyTorch supplies device memory and the current stream.  There is no CPU path:
+the functions accept CUDA tensors only and raise when the library cannot be loaded.
+
+Pipeline ([P1] "NVFP4 vs 2:4 sparse: where the other half of the petaflop went",
+[P2] "Sparse GPU FLOPS Need the Right Zeros in the Right Places", [P5] "NVFP4 Without FP4
+Hardware"):
+
+    check_24 -> prune_compress_24 -> quantize_nvfp4 -> gemm_dense / gemm_sparse24
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import NamedTuple, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsp24.so")
+
+# status codes (include/sp24.h)
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, \
+    ERR_DEVICE_TIMEOUT, ERR_WORKSPACE = range(9)
+F16, BF16, F32, NVFP4 = 0, 1, 2, 3
+OP_MATMUL, OP_CONV = 0, 1
+ALGO_AUTO, ALGO_SKINNY, ALGO_TILED = 0, 1, 2
+
+EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_24",
+           "sp24_prune_compress_24", "sp24_decompress_24", "sp24_quantize_nvfp4_workspace_size",
+           "sp24_quantize_nvfp4", "sp24_dequantize_nvfp4", "sp24_gemm_workspace_size",
+           "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
+           "sp24_last_device_error")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SP24Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.sp24_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+class _Operand(ctypes.Structure):
+    _fields_ = [("format", ctypes.c_int32), ("data", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p)]
+
+
+class _SparseOperand(ctypes.Structure):
+    _fields_ = [("format", ctypes.c_int32), ("values", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("meta", ctypes.c_void_p)]
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libsp24.so (building it in-tree first if it is missing or older than a source)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            from . import build as _build
+            if _build.stale():
+                _build.build()
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+            L.sp24_status_string.restype = ctypes.c_char_p
+            L.sp24_status_string.argtypes = [I]
+            L.sp24_sizes.argtypes = [I, I, P, I, P, P, P, P, P]
+            L.sp24_check_24.argtypes = [P, I, I, P, I, P, P, P]
+            L.sp24_prune_compress_24.argtypes = [P, I, I, P, I, P, P, P]
+            L.sp24_decompress_24.argtypes = [P, P, I, I, P, I, P, P]
+            L.sp24_quantize_nvfp4_workspace_size.argtypes = [I64, I64, P]
+            L.sp24_quantize_nvfp4.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, P]
+            L.sp24_dequantize_nvfp4.argtypes = [P, P, P, I64, I64, I, P, P]
+            L.sp24_gemm_workspace_size.argtypes = [I, I, I, I64, I64, I64, I, P]
+            L.sp24_gemm_dense.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand), I64,
+                                          I64, I64, P, P, I64, I, P]
+            L.sp24_gemm_sparse24.argtypes = [ctypes.POINTER(_Operand),
+                                             ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P,
+                                             I64, I, P]
+            L.sp24_last_device_error.argtypes = [P]
+            L.sp24_kernel_launches.restype = I64
+            L.sp24_kernel_launches.argtypes = []
+            _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------- marshalling
+
+_DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+_TORCH = {F16: torch.float16, BF16: torch.bfloat16, F32: torch.float32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape(shape) -> ctypes.Array:
+    arr = (ctypes.c_int64 * 4)()
+    for i, s in enumerate(shape):
+        arr[i] = int(s)
+    return arr
+
+
+def _call(fn: str, *args) -> None:
+    st = getattr(lib(), fn)(*args)
+    if st != OK:
+        raise SP24Error(st, fn)
+
+
+def _groups(op: int, shape) -> int:
+    shape = tuple(int(s) for s in shape)
+    if op == OP_MATMUL:
+        n = 1
+        for s in shape:
+            n *= s
+        return n // 4
+    K, C, R, S = shape
+    return K * (C // 4) * R * S
+
+
+def group_shape(op: int, shape) -> tuple:
+    shape = tuple(int(s) for s in shape)
+    if op == OP_MATMUL:
+        return shape[:-1] + (shape[-1] // 4,)
+    K, C, R, S = shape
+    return (K, C // 4, R, S)
+
+
+def values_shape(op: int, shape) -> tuple:
+    shape = tuple(int(s) for s in shape)
+    if op == OP_MATMUL:
+        return shape[:-1] + (shape[-1] // 2,)
+    K, C, R, S = shape
+    return (K, C // 2, R, S)
+
+
+class NVFP4Tensor(NamedTuple):
+    """codes uint8 [rows, cols/2], scales uint8 [rows, cols/16], tensor_scale fp32 [1]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tensor_scale: torch.Tensor
+
+
+class Sparse24(NamedTuple):
+    """A 2:4-compressed weight [N, K]: values ([N, K/2] 16-bit, or NVFP4 of them) + meta."""
+    values: object  # torch.Tensor (16-bit) or NVFP4Tensor
+    meta: torch.Tensor
+
+
+# ---------------------------------------------------------------------------- a1 .. a3
+
+def check_24(w: torch.Tensor, op: int = OP_MATMUL, pass_out=None, n_fail_out=None, stream=None):
+    """Per-group eligibility (uint8 0/1) and the failing-group count (int32 [1], device)."""
+    _cuda(w, "w")
+    if pass_out is None:
+        pass_out = torch.empty(group_shape(op, w.shape), dtype=torch.uint8, device=w.device)
+    if n_fail_out is None:
+        n_fail_out = torch.empty(1, dtype=torch.int32, device=w.device)
+    _call("sp24_check_24", _ptr(w), _dtype_code(w), op, _shape(w.shape), w.dim(),
+          _ptr(pass_out), _ptr(n_fail_out), _stream(stream))
+    return pass_out, n_fail_out
+
+
+def prune_compress_24(w: torch.Tensor, op: int = OP_MATMUL, values_out=None, meta_out=None,
+                      stream=None):
+    """(values, meta): kept entries [.., K/2] (or [K, C/2, R, S]) and the nibble stream."""
+    _cuda(w, "w")
+    if values_out is None:
+        values_out = torch.empty(values_shape(op, w.shape), dtype=w.dtype, device=w.device)
+    if meta_out is None:
+        meta_out = torch.empty((_groups(op, w.shape) + 1) // 2, dtype=torch.uint8, device=w.device)
+    _call("sp24_prune_compress_24", _ptr(w), _dtype_code(w), op, _shape(w.shape), w.dim(),
+          _ptr(values_out), _ptr(meta_out), _stream(stream))
+    return values_out, meta_out
+
+
+def decompress_24(values: torch.Tensor, meta: torch.Tensor, shape, op: int = OP_MATMUL,
+                  out=None, stream=None):
+    _cuda(values, "values")
+    _cuda(meta, "meta")
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=values.dtype, device=values.device)
+    _call("sp24_decompress_24", _ptr(values), _ptr(meta), _dtype_code(values), op, _shape(shape),
+          len(shape), _ptr(out), _stream(stream))
+    return out
+
+
+def quantize_workspace_bytes(rows: int, cols: int) -> int:
+    n = ctypes.c_int64(0)
+    _call("sp24_quantize_nvfp4_workspace_size", rows, cols, ctypes.byref(n))
+    return n.value
+
+
+def quantize_nvfp4(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None, out=None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> NVFP4Tensor:
+    """NVFP4 of a 2-D tensor; `tensor_scale` (fp32 [1], device) shares a scale across tensors."""
+    _cuda(t, "t")
+    if t.dim() != 2:
+        raise ValueError("quantize_nvfp4 wants a 2-D tensor")
+    R, L = t.shape
+    if out is None:
+        out = NVFP4Tensor(torch.empty((R, L // 2), dtype=torch.uint8, device=t.device),
+                          torch.empty((R, L // 16), dtype=torch.uint8, device=t.device),
+                          torch.empty(1, dtype=torch.float32, device=t.device))
+    if workspace is None and tensor_scale is None:
+        workspace = torch.empty(quantize_workspace_bytes(R, L), dtype=torch.uint8, device=t.device)
+    _call("sp24_quantize_nvfp4", _ptr(t), _dtype_code(t), R, L, _ptr(tensor_scale),
+          _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), _ptr(workspace),
+          0 if workspace is None else workspace.numel(), _stream(stream))
+    return out
+
+
+def dequantize_nvfp4(q: NVFP4Tensor, dtype=torch.float32, stream=None) -> torch.Tensor:
+    R, L2 = q.codes.shape
+    out = torch.empty((R, 2 * L2), dtype=dtype, device=q.codes.device)
+    _call("sp24_dequantize_nvfp4", _ptr(q.codes), _ptr(q.scales), _ptr(q.tensor_scale), R, 2 * L2,
+          _DT[dtype], _ptr(out), _stream(stream))
+    return out
+
+
+# ---------------------------------------------------------------------------- a4 .. a6
+
+def _operand(t) -> _Operand:
+    if isinstance(t, NVFP4Tensor):
+        return _Operand(NVFP4, t.codes.data_ptr(), t.scales.data_ptr(), t.tensor_scale.data_ptr())
+    _cuda(t, "operand")
+    return _Operand(_dtype_code(t), t.data_ptr(), None, None)
+
+
+def _rows_k(t) -> tuple:
+    if isinstance(t, NVFP4Tensor):
+        return t.codes.shape[0], 2 * t.codes.shape[1]
+    return t.shape[0], t.shape[1]
+
+
+def gemm_workspace_bytes(x, w, sparse: bool, M: int, N: int, K: int, algo: int = ALGO_AUTO) -> int:
+    xf = NVFP4 if isinstance(x, NVFP4Tensor) else _DT[x.dtype]
+    wv = w.values if sparse else w
+    wf = NVFP4 if isinstance(wv, NVFP4Tensor) else _DT[wv.dtype]
+    n = ctypes.c_int64(0)
+    _call("sp24_gemm_workspace_size", xf, wf, int(sparse), M, N, K, algo, ctypes.byref(n))
+    return n.value
+
+
+def gemm_dense(x, w, out=None, algo: int = ALGO_AUTO, workspace=None, stream=None) -> torch.Tensor:
+    """Y[M, N] fp32 = x[M, K] @ w[N, K]^T; x, w: 16-bit tensors or NVFP4Tensor."""
+    M, K = _rows_k(x)
+    N, Kw = _rows_k(w)
+    if K != Kw:
+        raise ValueError(f"K mismatch: {K} vs {Kw}")
+    dev = (x.codes if isinstance(x, NVFP4Tensor) else x).device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws_bytes = gemm_workspace_bytes(x, w, False, M, N, K, algo)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    xo, wo = _operand(x), _operand(w)
+    _call("sp24_gemm_dense", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out),
+          _ptr(workspace), 0 if workspace is None else workspace.numel(), algo, _stream(stream))
+    return out
+
+
+def gemm_sparse24(x, w: Sparse24, K: int, out=None, algo: int = ALGO_AUTO, workspace=None,
+                  stream=None) -> torch.Tensor:
+    """The same product with w 2:4-compressed (values 16-bit or NVFP4 + meta)."""
+    M, Kx = _rows_k(x)
+    if Kx != K:
+        raise ValueError(f"K mismatch: {Kx} vs {K}")
+    v = w.values
+    if isinstance(v, NVFP4Tensor):
+        N = v.codes.shape[0]
+        wo = _SparseOperand(NVFP4, v.codes.data_ptr(), v.scales.data_ptr(),
+                            v.tensor_scale.data_ptr(), w.meta.data_ptr())
+    else:
+        _cuda(v, "values")
+        N = v.shape[0]
+        wo = _SparseOperand(_dtype_code(v), v.data_ptr(), None, None, w.meta.data_ptr())
+    dev = w.meta.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws_bytes = gemm_workspace_bytes(x, w, True, M, N, K, algo)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    xo = _operand(x)
+    _call("sp24_gemm_sparse24", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out),
+          _ptr(workspace), 0 if workspace is None else workspace.numel(), algo, _stream(stream))
+    return out
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process (host-side count)."""
+    return int(lib().sp24_kernel_launches())
+
+
+def last_device_error(stream=None) -> int:
+    return int(lib().sp24_last_device_error(_stream(stream)))
+
+
+def sizes(op: int, dtype: int, shape) -> dict:
+    """Host-side size arithmetic of the compressed and NVFP4 forms (no device access)."""
+    out = [ctypes.c_int64(0) for _ in range(5)]
+    _call("sp24_sizes", op, dtype, _shape(shape), len(shape), *[ctypes.byref(o) for o in out])
+    keys = ("groups", "values_bytes", "meta_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes")
+    return {k: o.value for k, o in zip(keys, out)}

@@ -1,0 +1,221 @@
+// C ABI entry points that are not tied to one kernel family: status strings, size queries,
+// GEMM argument checking and dispatch, device error word.
+#include <string.h>
+
+#include "sp24_internal.cuh"
+
+#include <atomic>
+
+namespace sp24 {
+
+static std::atomic<int64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+bool is16(int f) { return f == SP24_F16 || f == SP24_BF16; }
+
+// Common checks of the x operand; fills the x part of p.
+int prep_x(const sp24_operand* x, int64_t M, int64_t K, SkinnyParams* p) {
+  if (!x) return SP24_ERR_INVALID_ARG;
+  if (x->format == SP24_NVFP4) {
+    if (K % 32) return SP24_ERR_SHAPE;
+    if (M > 0 && K > 0 && (!x->data || !x->scales || !x->tensor_scale)) return SP24_ERR_INVALID_ARG;
+    p->x_fmt = X_Q4;
+  } else if (is16(x->format)) {
+    if (K % 8) return SP24_ERR_SHAPE;
+    if (M > 0 && K > 0 && !x->data) return SP24_ERR_INVALID_ARG;
+    if (!aligned(x->data, 16)) return SP24_ERR_ALIGN;
+    p->x_fmt = X_16;
+  } else {
+    return SP24_ERR_DTYPE;
+  }
+  p->x = x->data;
+  p->x_scales = x->scales;
+  p->x_ts = x->tensor_scale;
+  return SP24_OK;
+}
+
+// MMA type: 16-bit x decides; 16-bit w must agree; NVFP4 x with NVFP4 w -> bf16.
+int mma_type(int xf, int wf, int* t16) {
+  if (is16(xf) && is16(wf) && xf != wf) return SP24_ERR_DTYPE;
+  *t16 = is16(xf) ? xf : (is16(wf) ? wf : SP24_BF16);
+  return SP24_OK;
+}
+
+// Runs the skinny kernel over M in slabs of 64 rows (one launch per slab).
+int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
+  const int64_t M = p.M;
+  for (int64_t m0 = 0; m0 < M; m0 += 64) {
+    SkinnyParams q = p;
+    q.M = M - m0 < 64 ? M - m0 : 64;
+    q.y = p.y + m0 * p.N;
+    if (p.x_fmt == X_16) {
+      q.x = reinterpret_cast<const uint8_t*>(p.x) + m0 * p.K * 2;
+    } else {
+      q.x = reinterpret_cast<const uint8_t*>(p.x) + m0 * p.K / 2;
+      q.x_scales = p.x_scales + m0 * p.K / 16;
+    }
+    int st = skinny_gemm(wf, t16, q, s);
+    if (st) return st;
+  }
+  return SP24_OK;
+}
+
+}  // namespace
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" const char* sp24_status_string(int status) {
+  switch (status) {
+    case SP24_OK: return "ok";
+    case SP24_ERR_INVALID_ARG: return "invalid argument";
+    case SP24_ERR_SHAPE: return "shape violates the operation's rule";
+    case SP24_ERR_DTYPE: return "element type not accepted";
+    case SP24_ERR_ALIGN: return "pointer misaligned";
+    case SP24_ERR_UNSUPPORTED: return "unsupported combination";
+    case SP24_ERR_CUDA: return "CUDA runtime error";
+    case SP24_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SP24_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int sp24_abi_version(void) { return 1; }
+
+extern "C" int sp24_sizes(int op, int dtype, const int64_t* shape, int ndim, int64_t* groups,
+                          int64_t* values_bytes, int64_t* meta_bytes, int64_t* nvfp4_codes_bytes,
+                          int64_t* nvfp4_scales_bytes) {
+  int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  if (!shape || ndim < 1 || ndim > 4) return SP24_ERR_INVALID_ARG;
+  int64_t n = 1;
+  for (int d = 0; d < ndim; ++d) {
+    if (shape[d] < 0) return SP24_ERR_SHAPE;
+    n *= shape[d];
+  }
+  int64_t G;
+  if (op == SP24_OP_MATMUL) {
+    if (shape[ndim - 1] % 4) return SP24_ERR_SHAPE;
+    G = n / 4;
+  } else if (op == SP24_OP_CONV) {
+    if (ndim != 4 || shape[1] % 4) return SP24_ERR_SHAPE;
+    G = shape[0] * (shape[1] / 4) * shape[2] * shape[3];
+  } else {
+    return SP24_ERR_INVALID_ARG;
+  }
+  if (groups) *groups = G;
+  if (values_bytes) *values_bytes = 2 * G * eb;
+  if (meta_bytes) *meta_bytes = (G + 1) / 2;
+  int64_t L = shape[ndim - 1];
+  bool q = op == SP24_OP_MATMUL && L % 16 == 0;
+  if (nvfp4_codes_bytes) *nvfp4_codes_bytes = q ? n / 2 : 0;
+  if (nvfp4_scales_bytes) *nvfp4_scales_bytes = q ? n / 16 : 0;
+  return SP24_OK;
+}
+
+extern "C" int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, int64_t M,
+                                        int64_t N, int64_t K, int algo, int64_t* bytes) {
+  (void)x_format; (void)w_format; (void)sparse; (void)M; (void)N; (void)K; (void)algo;
+  if (!bytes) return SP24_ERR_INVALID_ARG;
+  *bytes = 0;
+  return SP24_OK;
+}
+
+extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int64_t M, int64_t N,
+                               int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                               int algo, void* stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (!x || !w) return SP24_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
+  if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
+  SkinnyParams p;
+  memset(&p, 0, sizeof(p));
+  int st = prep_x(x, M, K, &p);
+  if (st) return st;
+  int t16;
+  st = mma_type(x->format, w->format, &t16);
+  if (st) return st;
+  int wf;
+  if (is16(w->format)) {
+    wf = W_D16;
+    p.w_row_bytes = K * 2;
+  } else if (w->format == SP24_NVFP4) {
+    if (K % 32) return SP24_ERR_SHAPE;
+    wf = W_DQ4;
+    p.w_row_bytes = K / 2;
+    p.scale_row_bytes = K / 16;
+    if (N > 0 && K > 0 && (!w->scales || !w->tensor_scale)) return SP24_ERR_INVALID_ARG;
+  } else {
+    return SP24_ERR_DTYPE;
+  }
+  if (M == 0 || N == 0) return SP24_OK;
+  if (!y) return SP24_ERR_INVALID_ARG;
+  if (K > 0 && !w->data) return SP24_ERR_INVALID_ARG;
+  if (!aligned(w->data, 16)) return SP24_ERR_ALIGN;
+  if (algo == SP24_ALGO_TILED) return SP24_ERR_UNSUPPORTED;
+  p.w = reinterpret_cast<const uint8_t*>(w->data);
+  p.w_scales = w->scales;
+  p.w_ts = w->tensor_scale;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.y = y;
+  return run_skinny(wf, t16, p, as_stream(stream));
+}
+
+extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M,
+                                  int64_t N, int64_t K, float* y, void* workspace,
+                                  int64_t workspace_bytes, int algo, void* stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (!x || !w) return SP24_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
+  if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
+  SkinnyParams p;
+  memset(&p, 0, sizeof(p));
+  int st = prep_x(x, M, K, &p);
+  if (st) return st;
+  int t16;
+  st = mma_type(x->format, w->format, &t16);
+  if (st) return st;
+  int wf;
+  if (is16(w->format)) {
+    if (K % 16) return SP24_ERR_SHAPE;
+    wf = W_S16;
+    p.w_row_bytes = K;  // K/2 values of 2 bytes
+  } else if (w->format == SP24_NVFP4) {
+    if (K % 64) return SP24_ERR_SHAPE;
+    wf = W_SQ4;
+    p.w_row_bytes = K / 4;
+    p.scale_row_bytes = K / 32;
+    if (N > 0 && K > 0 && (!w->scales || !w->tensor_scale)) return SP24_ERR_INVALID_ARG;
+  } else {
+    return SP24_ERR_DTYPE;
+  }
+  p.meta_row_bytes = K / 8;
+  if (M == 0 || N == 0) return SP24_OK;
+  if (!y) return SP24_ERR_INVALID_ARG;
+  if (K > 0 && (!w->values || !w->meta)) return SP24_ERR_INVALID_ARG;
+  if (!aligned(w->values, 16) || !aligned(w->meta, 8)) return SP24_ERR_ALIGN;
+  if (algo == SP24_ALGO_TILED) return SP24_ERR_UNSUPPORTED;
+  p.w = reinterpret_cast<const uint8_t*>(w->values);
+  p.w_scales = w->scales;
+  p.w_ts = w->tensor_scale;
+  p.meta = w->meta;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.y = y;
+  return run_skinny(wf, t16, p, as_stream(stream));
+}
+
+extern "C" int64_t sp24_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+extern "C" int sp24_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SP24_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(int)) != cudaSuccess) return SP24_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int)) != cudaSuccess) return SP24_ERR_CUDA;
+  return v;
+}

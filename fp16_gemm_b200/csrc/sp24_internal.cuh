@@ -1,0 +1,85 @@
+// Internal helpers shared by the libsp24 translation units (device code for sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sp24.h"
+
+namespace sp24 {
+
+// Device error word of this library (one per device, across all kernels): a kernel that
+// detects a problem it cannot report otherwise (a bounded wait that ran out, an illegal
+// nibble) stores a status here; sp24_last_device_error() reads and clears it.
+extern __device__ int g_dev_error;
+
+__device__ __forceinline__ void set_dev_error(int code) { atomicCAS(&g_dev_error, 0, code); }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Host-side count of kernels this library has launched (diagnostics: sp24_kernel_launches).
+void count_launch(int n = 1);
+
+// Status of the launches just issued; every launch site calls this once per kernel launched.
+inline int launch_status(int kernels = 1) {
+  count_launch(kernels);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+}
+
+inline int elem_bytes(int dtype) {
+  switch (dtype) {
+    case SP24_F16:
+    case SP24_BF16:
+      return 2;
+    case SP24_F32:
+      return 4;
+    default:
+      return 0;
+  }
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Number of SMs of the current device (cached per process; B200 has 148).
+int sm_count();
+
+// Magnitude bits of a 16- or 32-bit float pattern: monotone in |value| for non-NaN values.
+__device__ __forceinline__ uint32_t mag16(uint32_t h) { return h & 0x7fffu; }
+__device__ __forceinline__ uint32_t mag32(uint32_t f) { return f & 0x7fffffffu; }
+
+// Streaming 16-byte global load that bypasses L1 allocation (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ------------------------------------------------------------------ skinny GEMM interface
+enum { W_D16 = 0, W_S16 = 1, W_DQ4 = 2, W_SQ4 = 3 };  // weight formats
+enum { X_16 = 0, X_Q4 = 1 };                          // activation formats
+
+struct SkinnyParams {
+  const void* x;            // 16-bit [M, K] or NVFP4 codes [M, K/2]
+  const uint8_t* x_scales;  // NVFP4 x: [M, K/16]
+  const float* x_ts;        // NVFP4 x: tensor scale (device)
+  int x_fmt;
+  const uint8_t* w;         // values / codes, row-major
+  const uint8_t* w_scales;  // NVFP4 block scales
+  const float* w_ts;        // NVFP4 tensor scale (device)
+  const uint8_t* meta;      // 2:4 nibble stream, K/8 bytes per row
+  int64_t M, N, K;
+  int64_t w_row_bytes, scale_row_bytes, meta_row_bytes;
+  float* y;
+  int chunks_total;         // filled by skinny_gemm
+  bool accumulate;          // filled by skinny_gemm
+};
+
+// Launches the skinny kernel for M <= 64 (wf: W_*, t16: SP24_F16 / SP24_BF16 MMA type).
+int skinny_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
+
+}  // namespace sp24

@@ -1,0 +1,249 @@
+// a3: NVFP4 block quantisation and its decode.
+//
+// [P5] "NVFP4 Without FP4 Hardware", sections "Convert BF16 to NVFP4 yourself" (4-bit E2M1
+// values, one E4M3 scale per 16 values, one fp32 global scale per tensor) and "The shared
+// global scale" (one scale shared by a group of tensors, taken from the max absolute value).
+//
+// Two HBM-bound passes: (1) amax of |T| into a scratch word (warp/block max, one atomicMax
+// per block on the float's bit pattern, which orders non-negative floats); (2) encode: one
+// thread per 16-entry block, 32 bytes (16-bit input) read and 9 bytes written.  Every scale
+// and code decision is an IEEE fp32 operation with round-to-nearest-even, written with the
+// explicit __fdiv_rn / __fmul_rn intrinsics so no contraction or approximation can change a
+// rounding; the E4M3 and E2M1 roundings use the hardware's RNE + satfinite conversions.
+#include "sp24_internal.cuh"
+
+namespace sp24 {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int DT>
+__device__ __forceinline__ float to_f32(uint32_t bits16) {
+  if (DT == SP24_BF16) return __uint_as_float(bits16 << 16);
+  return __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+// 16 entries of a block as fp32 (exact: f16 and bf16 embed in fp32).
+template <int DT>
+__device__ __forceinline__ void load_block(const void* t, int64_t blk, float (&v)[16]) {
+  if (DT == SP24_F32) {
+    const uint4* p = reinterpret_cast<const uint4*>(t) + blk * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 x = ldg_stream16(p + q);
+      v[4 * q + 0] = __uint_as_float(x.x);
+      v[4 * q + 1] = __uint_as_float(x.y);
+      v[4 * q + 2] = __uint_as_float(x.z);
+      v[4 * q + 3] = __uint_as_float(x.w);
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(t) + blk * 2;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint4 x = ldg_stream16(p + q);
+      uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * q + 2 * i] = to_f32<DT>(w[i] & 0xffffu);
+        v[8 * q + 2 * i + 1] = to_f32<DT>(w[i] >> 16);
+      }
+    }
+  }
+}
+
+// E4M3 code of x >= 0: round to nearest even, values beyond 448 saturate to 448.
+__device__ __forceinline__ uint32_t e4m3_rne_satfinite(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xffu;  // the second source lands in the low byte
+}
+
+// fp32 value of an E4M3 code (exact).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h2;
+  uint16_t c = (uint16_t)code;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
+}
+
+// Two E2M1 magnitude codes (x_lo, x_hi >= 0) packed as lo | hi << 4, RNE, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1x2_rne_satfinite(float x_lo, float x_hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(x_hi), "f"(x_lo));
+  return r & 0xffu;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ t, int64_t nblk,
+                                                        unsigned int* __restrict__ amax_bits) {
+  float m = 0.0f;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+    float v[16];
+    load_block<DT>(t, b, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+  }
+  unsigned int u = __float_as_uint(m);
+  u = __reduce_max_sync(0xffffffffu, u);
+  __shared__ unsigned int wmax[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = u;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    unsigned int x = threadIdx.x < kThreads / 32 ? wmax[threadIdx.x] : 0u;
+    x = __reduce_max_sync(0xffffffffu, x);
+    if (threadIdx.x == 0 && x) atomicMax(amax_bits, x);
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads) encode_kernel(const void* __restrict__ t, int64_t nblk,
+                                                          const float* __restrict__ ts_in,
+                                                          const unsigned int* __restrict__ amax_bits,
+                                                          uint2* __restrict__ codes,
+                                                          uint8_t* __restrict__ scales,
+                                                          float* __restrict__ ts_out) {
+  // tensor scale: supplied, or amax / 2688 (2688 = 6 * 448)
+  const float s_t = ts_in ? *ts_in : __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
+  const float d = __fmul_rn(s_t, 6.0f);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+    float v[16];
+    load_block<DT>(t, b, v);
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+    uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
+    const float sc = __fmul_rn(e4m3_value(sb), s_t);
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      float q0 = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
+      float q1 = sc != 0.0f ? __fdiv_rn(fabsf(v[i + 1]), sc) : 0.0f;
+      uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
+      byte |= (__float_as_uint(v[i]) >> 31) << 3;       // sign of the low entry
+      byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;   // sign of the high entry
+      packed[i / 8] |= byte << (8 * ((i % 8) / 2));
+    }
+    codes[b] = make_uint2(packed[0], packed[1]);
+    scales[b] = (uint8_t)sb;
+  }
+}
+
+// One byte (two entries) per thread; value computed in fp64 (exact) and rounded once.
+template <int OUT>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const uint8_t* __restrict__ codes,
+                                                          const uint8_t* __restrict__ scales,
+                                                          const float* __restrict__ ts,
+                                                          int64_t nbytes, void* __restrict__ out) {
+  const double s_t = (double)*ts;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbytes; i += stride) {
+    uint32_t byte = codes[i];
+    double sb = (double)e4m3_value(scales[i / 8]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t c = (byte >> (4 * h)) & 0xf;
+      uint32_t mag = c & 7, e = mag >> 1, m = mag & 1;
+      double a = e == 0 ? 0.5 * m : (double)(1 << (e - 1)) * (1.0 + 0.5 * m);
+      double val = (c & 8 ? -a : a) * sb * s_t;
+      int64_t idx = 2 * i + h;
+      if (OUT == SP24_F32) reinterpret_cast<float*>(out)[idx] = (float)val;
+      else if (OUT == SP24_BF16) reinterpret_cast<__nv_bfloat16*>(out)[idx] = __double2bfloat16(val);
+      else reinterpret_cast<__half*>(out)[idx] = __double2half(val);
+    }
+  }
+}
+
+int grid_for(int64_t items) {
+  int64_t blocks = (items + kThreads - 1) / kThreads;
+  int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
+constexpr int64_t kQuantWorkspace = 256;
+
+}  // namespace
+
+// Shared by the quantisation entry points: validates and launches amax (unless a tensor
+// scale is supplied) and encode.  `amax_word` is 4 bytes of zero-initialisable scratch.
+int quantize_nvfp4_launch(const void* t, int dtype, int64_t rows, int64_t cols,
+                          const float* ts_in, uint8_t* codes, uint8_t* scales, float* ts_out,
+                          unsigned int* amax_word, cudaStream_t s) {
+  int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  if (rows < 0 || cols < 0 || cols % 16) return SP24_ERR_SHAPE;
+  if (!ts_out) return SP24_ERR_INVALID_ARG;
+  const int64_t nblk = rows * cols / 16;
+  if (nblk > 0 && (!t || !codes || !scales)) return SP24_ERR_INVALID_ARG;
+  if (nblk > 0 && (!aligned(t, 16) || !aligned(codes, 8))) return SP24_ERR_ALIGN;
+  int nl = 1;  // encode always runs
+  if (!ts_in) {
+    if (!amax_word) return SP24_ERR_WORKSPACE;
+    if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return SP24_ERR_CUDA;
+    if (nblk > 0) {
+      if (dtype == SP24_F32) amax_kernel<SP24_F32><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
+      else if (dtype == SP24_BF16) amax_kernel<SP24_BF16><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
+      else amax_kernel<SP24_F16><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
+      ++nl;
+    }
+  }
+  // launched even when nblk == 0 so that tensor_scale_out is written
+  int g = grid_for(nblk > 0 ? nblk : 1);
+  if (dtype == SP24_F32)
+    encode_kernel<SP24_F32><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+  else if (dtype == SP24_BF16)
+    encode_kernel<SP24_BF16><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+  else
+    encode_kernel<SP24_F16><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+  return launch_status(nl);
+}
+
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" int sp24_quantize_nvfp4_workspace_size(int64_t rows, int64_t cols, int64_t* bytes) {
+  if (!bytes) return SP24_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || cols % 16) return SP24_ERR_SHAPE;
+  *bytes = kQuantWorkspace;
+  return SP24_OK;
+}
+
+extern "C" int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
+                                   const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                   float* tensor_scale_out, void* workspace,
+                                   int64_t workspace_bytes, void* stream) {
+  unsigned int* amax_word = nullptr;
+  if (!tensor_scale_in) {
+    if (!workspace || workspace_bytes < kQuantWorkspace) return SP24_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
+    amax_word = reinterpret_cast<unsigned int*>(workspace);
+  }
+  return quantize_nvfp4_launch(t, dtype, rows, cols, tensor_scale_in, codes, scales,
+                               tensor_scale_out, amax_word, as_stream(stream));
+}
+
+extern "C" int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,
+                                     const float* tensor_scale, int64_t rows, int64_t cols,
+                                     int out_dtype, void* out, void* stream) {
+  if (rows < 0 || cols < 0 || cols % 16) return SP24_ERR_SHAPE;
+  if (!elem_bytes(out_dtype)) return SP24_ERR_DTYPE;
+  int64_t nbytes = rows * cols / 2;
+  if (nbytes == 0) return SP24_OK;
+  if (!codes || !scales || !tensor_scale || !out) return SP24_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (out_dtype == SP24_F32)
+    decode_kernel<SP24_F32><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+  else if (out_dtype == SP24_BF16)
+    decode_kernel<SP24_BF16><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+  else
+    decode_kernel<SP24_F16><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+  return launch_status();
+}

@@ -1,0 +1,429 @@
+// a1 / a2: 2:4 eligibility check, magnitude pruning + compression, decompression.
+//
+// [P2] "Sparse GPU FLOPS Need the Right Zeros in the Right Places", sections "The operation
+// determines which four entries belong together" and "Two half-zero vectors produce different
+// pattern answers"; [P1] "NVFP4 vs 2:4 sparse: where the other half of the petaflop went",
+// section "What 2:4 actually is".
+//
+// These kernels are HBM-bound streams.  For the matmul layout (groups of four consecutive
+// entries) every thread owns whole groups: one 16-byte load holds two 16-bit groups or one
+// fp32 group, consecutive threads take consecutive 16-byte vectors (each warp load is 512
+// contiguous bytes), and the top-2 choice is made in registers with six compares, so no
+// cross-lane exchange is needed.  Conv weights [K, C, R, S] put the four members of a group
+// R*S entries apart; those kernels take one group (or one pair of groups) per thread and
+// read through the read-only cache, which still moves each input byte from DRAM once.
+#include "sp24_internal.cuh"
+
+namespace sp24 {
+
+__device__ int g_dev_error = 0;
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------------ group arithmetic
+
+// Bit mask of the two kept members of a group (|w| descending, index ascending): member i is
+// kept when fewer than two members precede it.  A lower-index member precedes on >=, a higher
+// one only on >.
+__device__ __forceinline__ uint32_t keep_mask(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
+  uint32_t r0 = (m1 > m0) + (m2 > m0) + (m3 > m0);
+  uint32_t r1 = (m0 >= m1) + (m2 > m1) + (m3 > m1);
+  uint32_t r2 = (m0 >= m2) + (m1 >= m2) + (m3 > m2);
+  uint32_t r3 = (m0 >= m3) + (m1 >= m3) + (m2 >= m3);
+  return (r0 < 2) | ((r1 < 2) << 1) | ((r2 < 2) << 2) | ((r3 < 2) << 3);
+}
+
+// nibble = i0 | i1 << 2 of a keep mask with exactly two bits set
+__device__ __forceinline__ uint32_t mask_nibble(uint32_t mask) {
+  uint32_t i0 = __ffs(mask) - 1;
+  uint32_t i1 = 31 - __clz(mask);
+  return i0 | (i1 << 2);
+}
+
+// One 16-bit group held as two words (lo = e0 | e1 << 16, hi = e2 | e3 << 16).
+struct Group16 {
+  uint32_t nib;   // kept indices
+  uint32_t kept;  // v0 | v1 << 16
+};
+
+__device__ __forceinline__ Group16 prune16(uint32_t lo, uint32_t hi) {
+  uint32_t m = keep_mask(mag16(lo), mag16(lo >> 16), mag16(hi), mag16(hi >> 16));
+  Group16 g;
+  g.nib = mask_nibble(m);
+  uint32_t i0 = g.nib & 3, i1 = g.nib >> 2;
+  uint32_t sel = (2 * i0) | ((2 * i0 + 1) << 4) | ((2 * i1) << 8) | ((2 * i1 + 1) << 12);
+  g.kept = __byte_perm(lo, hi, sel);
+  return g;
+}
+
+__device__ __forceinline__ int zeros16(uint32_t lo, uint32_t hi) {
+  return (mag16(lo) == 0) + (mag16(lo >> 16) == 0) + (mag16(hi) == 0) + (mag16(hi >> 16) == 0);
+}
+
+__device__ __forceinline__ int zeros32(uint4 v) {
+  return (mag32(v.x) == 0) + (mag32(v.y) == 0) + (mag32(v.z) == 0) + (mag32(v.w) == 0);
+}
+
+__device__ __forceinline__ void count_fails(int fails, int32_t* n_fail) {
+  if (!n_fail) return;
+  int s = __reduce_add_sync(0xffffffffu, fails);
+  if ((threadIdx.x & 31) == 0 && s) atomicAdd(n_fail, s);
+}
+
+// ------------------------------------------------------------------ matmul layout, vector path
+
+// Groups 2v, 2v+1 (16-bit) or group v (fp32) per 16-byte vector v.  Every lane of a warp runs
+// the same number of iterations so the final warp reduction sees all lanes.
+template <int EB>
+__global__ void __launch_bounds__(kThreads) check24_vec(const uint4* __restrict__ w, int64_t nv,
+                                                        uint8_t* __restrict__ pass,
+                                                        int32_t* __restrict__ n_fail) {
+  int fails = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~int64_t(31);
+  for (int64_t base = warp0; base < nv; base += stride) {
+    int64_t v = base + (threadIdx.x & 31);
+    if (v < nv) {
+      uint4 x = ldg_stream16(w + v);
+      if (EB == 2) {
+        int ok0 = zeros16(x.x, x.y) >= 2, ok1 = zeros16(x.z, x.w) >= 2;
+        fails += 2 - ok0 - ok1;
+        reinterpret_cast<uint16_t*>(pass)[v] = (uint16_t)(ok0 | (ok1 << 8));
+      } else {
+        int ok = zeros32(x) >= 2;
+        fails += 1 - ok;
+        pass[v] = (uint8_t)ok;
+      }
+    }
+  }
+  count_fails(fails, n_fail);
+}
+
+template <int EB>
+__global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict__ w, int64_t nv,
+                                                        uint2* __restrict__ values,
+                                                        uint8_t* __restrict__ meta) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~int64_t(31);
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = warp0; base < nv; base += stride) {
+    int64_t v = base + lane;
+    bool live = v < nv;
+    uint4 x = live ? ldg_stream16(w + v) : make_uint4(0, 0, 0, 0);
+    if (EB == 2) {
+      if (live) {
+        Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
+        values[v] = make_uint2(a.kept, b.kept);
+        meta[v] = (uint8_t)(a.nib | (b.nib << 4));
+      }
+    } else {
+      uint32_t m = keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w));
+      uint32_t nib = mask_nibble(m);
+      uint32_t e[4] = {x.x, x.y, x.z, x.w};
+      uint32_t i0 = nib & 3, i1 = nib >> 2;
+      uint32_t v0 = i0 == 0 ? e[0] : (i0 == 1 ? e[1] : e[2]);
+      uint32_t v1 = i1 == 3 ? e[3] : (i1 == 2 ? e[2] : e[1]);
+      // the partner group v^1 lives in lane^1 (the warp's first vector index is even)
+      uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+      if (live) {
+        values[v] = make_uint2(v0, v1);
+        bool partner_live = (v ^ 1) < nv;
+        if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (partner_live ? other << 4 : 0u));
+      }
+    }
+  }
+}
+
+// Inverse of prune24_vec for 16-bit data: two groups per thread.
+__global__ void __launch_bounds__(kThreads) decompress24_vec16(const uint2* __restrict__ values,
+                                                               const uint8_t* __restrict__ meta,
+                                                               int64_t nv, uint4* __restrict__ w) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
+    uint2 kv = values[v];
+    uint32_t mb = meta[v];
+    uint32_t out[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t nib = (mb >> (4 * h)) & 0xf;
+      uint32_t i0 = nib & 3, i1 = nib >> 2;
+      uint32_t kept = h ? kv.y : kv.x;
+      if (i0 >= i1) {
+        set_dev_error(SP24_ERR_INVALID_ARG);
+        kept = 0;
+      }
+      // byte selectors: slot i takes v0 (bytes 0,1), v1 (bytes 2,3) or zero (bytes 4,5)
+      auto sel = [&](uint32_t i) -> uint32_t { return i == i0 ? 0x10u : (i == i1 ? 0x32u : 0x54u); };
+      out[2 * h] = __byte_perm(kept, 0u, sel(0) | (sel(1) << 8));
+      out[2 * h + 1] = __byte_perm(kept, 0u, sel(2) | (sel(3) << 8));
+    }
+    w[v] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// ------------------------------------------------------------------ generic (any layout) path
+
+struct Layout {
+  int op;
+  int64_t C, RS;  // conv: channels and R*S
+};
+
+// Element index of member i of group g.
+__device__ __forceinline__ int64_t member(const Layout& L, int64_t g, int i) {
+  if (L.op == SP24_OP_MATMUL) return g * 4 + i;
+  int64_t rs = g % L.RS, kj = g / L.RS;
+  int64_t j = kj % (L.C / 4), k = kj / (L.C / 4);
+  return (k * L.C + 4 * j + i) * L.RS + rs;
+}
+
+// Index of stored value t of group g.
+__device__ __forceinline__ int64_t slot(const Layout& L, int64_t g, int t) {
+  if (L.op == SP24_OP_MATMUL) return g * 2 + t;
+  int64_t rs = g % L.RS, kj = g / L.RS;
+  int64_t j = kj % (L.C / 4), k = kj / (L.C / 4);
+  return (k * (L.C / 2) + 2 * j + t) * L.RS + rs;
+}
+
+template <int EB>
+__device__ __forceinline__ uint32_t load_elem(const void* p, int64_t i) {
+  if (EB == 2) return __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+  return __ldg(reinterpret_cast<const unsigned int*>(p) + i);
+}
+
+template <int EB>
+__device__ __forceinline__ void store_elem(void* p, int64_t i, uint32_t v) {
+  if (EB == 2) reinterpret_cast<uint16_t*>(p)[i] = (uint16_t)v;
+  else reinterpret_cast<uint32_t*>(p)[i] = v;
+}
+
+template <int EB>
+__device__ __forceinline__ uint32_t magb(uint32_t x) {
+  return EB == 2 ? mag16(x) : mag32(x);
+}
+
+template <int EB>
+__global__ void __launch_bounds__(kThreads) check24_any(const void* __restrict__ w, Layout L,
+                                                        int64_t g0, int64_t G,
+                                                        uint8_t* __restrict__ pass,
+                                                        int32_t* __restrict__ n_fail) {
+  int fails = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t warp0 = g0 + (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~int64_t(31));
+  for (int64_t base = warp0; base < G; base += stride) {
+    int64_t g = base + (threadIdx.x & 31);
+    if (g < G) {
+      int z = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) z += magb<EB>(load_elem<EB>(w, member(L, g, i))) == 0;
+      pass[g] = (uint8_t)(z >= 2);
+      fails += z < 2;
+    }
+  }
+  count_fails(fails, n_fail);
+}
+
+// One pair of groups (one meta byte) per thread.
+template <int EB>
+__global__ void __launch_bounds__(kThreads) prune24_any(const void* __restrict__ w, Layout L,
+                                                        int64_t p0, int64_t G,
+                                                        void* __restrict__ values,
+                                                        uint8_t* __restrict__ meta) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t P = (G + 1) / 2;
+  for (int64_t p = p0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < P; p += stride) {
+    uint32_t byte = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int64_t g = 2 * p + h;
+      if (g >= G) break;
+      uint32_t e[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) e[i] = load_elem<EB>(w, member(L, g, i));
+      uint32_t nib = mask_nibble(keep_mask(magb<EB>(e[0]), magb<EB>(e[1]), magb<EB>(e[2]), magb<EB>(e[3])));
+      uint32_t i0 = nib & 3, i1 = nib >> 2;
+      store_elem<EB>(values, slot(L, g, 0), i0 == 0 ? e[0] : (i0 == 1 ? e[1] : e[2]));
+      store_elem<EB>(values, slot(L, g, 1), i1 == 3 ? e[3] : (i1 == 2 ? e[2] : e[1]));
+      byte |= nib << (4 * h);
+    }
+    meta[p] = (uint8_t)byte;
+  }
+}
+
+template <int EB>
+__global__ void __launch_bounds__(kThreads) decompress24_any(const void* __restrict__ values,
+                                                             const uint8_t* __restrict__ meta,
+                                                             Layout L, int64_t g0, int64_t G,
+                                                             void* __restrict__ w) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t g = g0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < G; g += stride) {
+    uint32_t nib = (meta[g >> 1] >> (4 * (g & 1))) & 0xf;
+    uint32_t i0 = nib & 3, i1 = nib >> 2;
+    bool legal = i0 < i1;
+    if (!legal) set_dev_error(SP24_ERR_INVALID_ARG);
+    uint32_t v0 = load_elem<EB>(values, slot(L, g, 0)), v1 = load_elem<EB>(values, slot(L, g, 1));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t v = 0;
+      if (legal && i == (int)i0) v = v0;
+      if (legal && i == (int)i1) v = v1;
+      store_elem<EB>(w, member(L, g, i), v);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+int grid_for(int64_t items) {
+  int64_t blocks = (items + kThreads - 1) / kThreads;
+  int64_t cap = (int64_t)sm_count() * 8;  // grid-stride beyond 8 blocks per SM
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
+// Validates (op, shape, ndim) and returns the group count and layout.
+int parse_shape(int op, const int64_t* shape, int ndim, int64_t* G, Layout* L) {
+  if (!shape || ndim < 1 || ndim > 4) return SP24_ERR_INVALID_ARG;
+  for (int d = 0; d < ndim; ++d)
+    if (shape[d] < 0) return SP24_ERR_SHAPE;
+  L->op = op;
+  L->C = 0;
+  L->RS = 1;
+  if (op == SP24_OP_MATMUL) {
+    if (shape[ndim - 1] % 4) return SP24_ERR_SHAPE;
+    int64_t n = 1;
+    for (int d = 0; d < ndim; ++d) n *= shape[d];
+    *G = n / 4;
+    return SP24_OK;
+  }
+  if (op == SP24_OP_CONV) {
+    if (ndim != 4 || shape[1] % 4) return SP24_ERR_SHAPE;
+    L->C = shape[1];
+    L->RS = shape[2] * shape[3];
+    *G = shape[0] * (shape[1] / 4) * L->RS;
+    return SP24_OK;
+  }
+  return SP24_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+int sm_count() {
+  static int cached = 0;
+  if (!cached) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+      cached = n;
+    else
+      return 148;
+  }
+  return cached;
+}
+
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" int sp24_check_24(const void* w, int dtype, int op, const int64_t* shape, int ndim,
+                             uint8_t* pass, int32_t* n_fail, void* stream) {
+  int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  int64_t G;
+  Layout L;
+  int st = parse_shape(op, shape, ndim, &G, &L);
+  if (st) return st;
+  if (G > 0 && (!w || !pass)) return SP24_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (n_fail && cudaMemsetAsync(n_fail, 0, sizeof(int32_t), s) != cudaSuccess) return SP24_ERR_CUDA;
+  if (G == 0) return launch_status(0);
+  int nl = 0;
+  int64_t g_done = 0;
+  if (op == SP24_OP_MATMUL && aligned(w, 16) && aligned(pass, eb == 2 ? 2 : 1)) {
+    int64_t nv = G * 4 * eb / 16;  // whole 16-byte vectors
+    if (nv > 0) {
+      if (eb == 2)
+        check24_vec<2><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+      else
+        check24_vec<4><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+      ++nl;
+      g_done = nv * 16 / (4 * eb);
+    }
+  }
+  if (g_done < G) {
+    if (eb == 2)
+      check24_any<2><<<grid_for(G - g_done), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
+    else
+      check24_any<4><<<grid_for(G - g_done), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
+    ++nl;
+  }
+  return launch_status(nl);
+}
+
+extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const int64_t* shape,
+                                      int ndim, void* values, uint8_t* meta, void* stream) {
+  int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  int64_t G;
+  Layout L;
+  int st = parse_shape(op, shape, ndim, &G, &L);
+  if (st) return st;
+  if (G == 0) return SP24_OK;
+  if (!w || !values || !meta) return SP24_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int nl = 0;
+  int64_t p_done = 0;  // meta bytes (group pairs) already written
+  if (op == SP24_OP_MATMUL && aligned(w, 16) && aligned(values, 8)) {
+    int64_t nv = G * 4 * eb / 16;
+    if (eb == 4) nv &= ~int64_t(1);  // whole meta bytes only
+    if (nv > 0) {
+      if (eb == 2)
+        prune24_vec<2><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+      else
+        prune24_vec<4><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+      ++nl;
+      p_done = (nv * 16 / (4 * eb)) / 2;
+    }
+  }
+  if (2 * p_done < G) {
+    int64_t rest = (G + 1) / 2 - p_done;
+    if (eb == 2)
+      prune24_any<2><<<grid_for(rest), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
+    else
+      prune24_any<4><<<grid_for(rest), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
+    ++nl;
+  }
+  return launch_status(nl);
+}
+
+extern "C" int sp24_decompress_24(const void* values, const uint8_t* meta, int dtype, int op,
+                                  const int64_t* shape, int ndim, void* w_out, void* stream) {
+  int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  int64_t G;
+  Layout L;
+  int st = parse_shape(op, shape, ndim, &G, &L);
+  if (st) return st;
+  if (G == 0) return SP24_OK;
+  if (!values || !meta || !w_out) return SP24_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int nl = 0;
+  int64_t g_done = 0;
+  if (op == SP24_OP_MATMUL && eb == 2 && aligned(values, 8) && aligned(w_out, 16)) {
+    int64_t nv = G / 2;
+    if (nv > 0) {
+      decompress24_vec16<<<grid_for(nv), kThreads, 0, s>>>((const uint2*)values, meta, nv, (uint4*)w_out);
+      ++nl;
+    }
+    g_done = 2 * nv;
+  }
+  if (g_done < G) {
+    if (eb == 2)
+      decompress24_any<2><<<grid_for(G - g_done), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
+    else
+      decompress24_any<4><<<grid_for(G - g_done), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
+    ++nl;
+  }
+  return launch_status(nl);
+}

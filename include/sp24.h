@@ -1,0 +1,188 @@
+/*
+ * sp24.h -- C ABI of libsp24: 2:4 structured sparsity and NVFP4 against dense GEMM on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources (pages, by title; section names in quotes):
+ *   [P1] "NVFP4 vs 2:4 sparse: where the other half of the petaflop went" (robertz.co)
+ *   [P2] "Sparse GPU FLOPS Need the Right Zeros in the Right Places" (leviathansystems.co)
+ *   [P5] "NVFP4 Without FP4 Hardware" (ai-muninn.com)
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must point to memory of the current CUDA device;
+ *     `shape` arrays and the operand structs are host memory and are read before the call
+ *     returns.  The caller owns every buffer; the library never allocates device memory.
+ *   - Tensors are dense and row-major (C order).  GEMM operands are K-contiguous.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and returns a status.  Argument errors are detected on the host and return a
+ *     status without launching anything.  SP24_ERR_CUDA reports a failed launch.  Kernels
+ *     never trap: a device-side wait that runs out of time sets a device error word, which
+ *     sp24_last_device_error() reports.
+ *   - No call falls back to the CPU.
+ */
+#ifndef SP24_H_
+#define SP24_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ----------------------------------------------------------------------- status codes */
+enum {
+  SP24_OK = 0,
+  SP24_ERR_INVALID_ARG = 1,   /* null pointer, unknown enum value, bad operand struct */
+  SP24_ERR_SHAPE = 2,         /* shape violates the operation's rule (e.g. C % 4 != 0) */
+  SP24_ERR_DTYPE = 3,         /* element type not accepted by this call */
+  SP24_ERR_ALIGN = 4,         /* a pointer is not aligned as the call requires */
+  SP24_ERR_UNSUPPORTED = 5,   /* valid request that no kernel of this build serves */
+  SP24_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
+  SP24_ERR_DEVICE_TIMEOUT = 7,/* a bounded device-side wait gave up */
+  SP24_ERR_WORKSPACE = 8      /* workspace missing or smaller than the size query says */
+};
+
+/* ----------------------------------------------------------------------- enums */
+/* element types */
+enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3 };
+
+/* The operation a weight belongs to decides which four entries form a group ([P2] "The
+ * operation determines which four entries belong together"). */
+enum {
+  SP24_OP_MATMUL = 0, /* W[..., K]: groups of four consecutive entries along the last axis K */
+  SP24_OP_CONV = 1    /* W[K, C, R, S]: groups along input channels C at fixed (k, r, s);
+                         C % 4 == 0 */
+};
+
+/* GEMM kernel choice (SP24_ALGO_AUTO picks by shape). */
+enum { SP24_ALGO_AUTO = 0, SP24_ALGO_SKINNY = 1, SP24_ALGO_TILED = 2 };
+
+/* ----------------------------------------------------------------------- operands */
+/* A dense GEMM operand with `rows` rows of K entries.
+ *   format SP24_F16 / SP24_BF16: data -> [rows, K] elements.
+ *   format SP24_NVFP4 ([P5] "Convert BF16 to NVFP4 yourself": 4-bit E2M1 values, one E4M3
+ *   scale per 16 values, one fp32 tensor scale):
+ *       data -> [rows, K/2] bytes of packed E2M1 codes (entry 2i in the low nibble),
+ *       scales -> [rows, K/16] E4M3 block scales, tensor_scale -> one fp32 (device).
+ * Decoded value = E2M1(code) * E4M3(scale) * tensor_scale. */
+typedef struct {
+  int32_t format;
+  const void* data;
+  const uint8_t* scales;
+  const float* tensor_scale;
+} sp24_operand;
+
+/* A 2:4-compressed weight W[N, K] ([P1] "What 2:4 actually is": two kept values per group of
+ * four plus a 2-bit index for each).
+ *   meta -> [N, K/8] bytes: one nibble per group, i0 | i1 << 2 with i0 < i1 the kept indices,
+ *           groups in natural order, the even group in the low nibble.
+ *   format SP24_F16 / SP24_BF16: values -> [N, K/2] kept entries in ascending index order.
+ *   format SP24_NVFP4: the kept values [N, K/2] quantised as an NVFP4 tensor:
+ *           values -> [N, K/4] packed codes, scales -> [N, K/32] (one per 16 stored values),
+ *           tensor_scale -> one fp32 (device). */
+typedef struct {
+  int32_t format;
+  const void* values;
+  const uint8_t* scales;
+  const float* tensor_scale;
+  const uint8_t* meta;
+} sp24_sparse_operand;
+
+/* ----------------------------------------------------------------------- host helpers */
+const char* sp24_status_string(int status);
+int sp24_abi_version(void);
+
+/* Sizes of what the pipeline produces for a tensor (host only, no device access).
+ * groups: groups of four along the reduction axis; values_bytes / meta_bytes: compressed
+ * form; nvfp4_codes_bytes / nvfp4_scales_bytes: dense NVFP4 of the tensor viewed as
+ * [numel / L, L] with L its last axis (matmul only; 0 for conv).  Any output may be NULL. */
+int sp24_sizes(int op, int dtype, const int64_t* shape, int ndim, int64_t* groups,
+               int64_t* values_bytes, int64_t* meta_bytes, int64_t* nvfp4_codes_bytes,
+               int64_t* nvfp4_scales_bytes);
+
+/* ----------------------------------------------------------------------- a1: eligibility */
+/* [P2] "The operation determines which four entries belong together", "Two half-zero vectors
+ * produce different pattern answers": a group passes when at least two of its four entries
+ * are zero (+0 or -0; NaN is not zero); groups are judged one by one.
+ *   w      device, dtype F16/BF16/F32, shape [rows..., K] (MATMUL, ndim 1..4, K % 4 == 0)
+ *          or [K, C, R, S] (CONV, C % 4 == 0).
+ *   pass   device uint8, one byte (0/1) per group, group axis replacing K (MATMUL) or laid
+ *          out [K, C/4, R, S] (CONV).
+ *   n_fail device int32 or NULL: receives the number of failing groups (overwritten). */
+int sp24_check_24(const void* w, int dtype, int op, const int64_t* shape, int ndim,
+                  uint8_t* pass, int32_t* n_fail, void* stream);
+
+/* ----------------------------------------------------------------------- a2: prune/compress */
+/* [P1] "What 2:4 actually is": magnitude pruning to two of four and compression.  Kept = the
+ * two entries first in the order (|w| descending, index ascending), |w| compared as the
+ * magnitude bit pattern (NaN above +inf).
+ *   values device, same dtype as w: [rows, K/2] (MATMUL) or [K, C/2, R, S] (CONV), kept
+ *          entries copied bit for bit in ascending index order.
+ *   meta   device, ceil(groups / 2) bytes, nibble stream as in sp24_sparse_operand. */
+int sp24_prune_compress_24(const void* w, int dtype, int op, const int64_t* shape, int ndim,
+                           void* values, uint8_t* meta, void* stream);
+
+/* Inverse of compression: w_out (device, dtype, `shape`) receives the kept values at their
+ * indices and +0 elsewhere.  Nibbles must be legal (i0 < i1); an illegal nibble yields +0 in
+ * its group and sets the device error word (SP24_ERR_INVALID_ARG). */
+int sp24_decompress_24(const void* values, const uint8_t* meta, int dtype, int op,
+                       const int64_t* shape, int ndim, void* w_out, void* stream);
+
+/* ----------------------------------------------------------------------- a3: NVFP4 */
+/* [P5] "Convert BF16 to NVFP4 yourself", "The shared global scale": quantise T[rows, cols]
+ * (cols % 16 == 0) to NVFP4.
+ *   s_t  = tensor_scale_in ? *tensor_scale_in : amax(|T|) / 2688   (2688 = 6 * 448)
+ *   block scale sb = E4M3_rne_satfinite(bmax / (s_t * 6)) per 16 consecutive entries of a row
+ *   code = sign(t) << 3 | E2M1_rne_satfinite(|t| / (E4M3(sb) * s_t))  (0 when that divisor is 0)
+ * every step an IEEE fp32 operation; negative zero keeps its sign bit.
+ *   t                 device, F16/BF16/F32, [rows, cols]
+ *   tensor_scale_in   device fp32 or NULL (NULL: derive from amax; else a shared scale,
+ *                     finite and >= 0)
+ *   codes             device, [rows, cols/2] bytes;  scales: device, [rows, cols/16] bytes
+ *   tensor_scale_out  device fp32 (may equal tensor_scale_in)
+ *   workspace         device, >= sp24_quantize_nvfp4_workspace_size() bytes, 16-byte
+ *                     aligned; contents are scratch.  Non-finite inputs give unspecified codes. */
+int sp24_quantize_nvfp4_workspace_size(int64_t rows, int64_t cols, int64_t* bytes);
+int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
+                        const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                        float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
+                        void* stream);
+
+/* Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
+ * (F16/BF16/F32). */
+int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,
+                          const float* tensor_scale, int64_t rows, int64_t cols, int out_dtype,
+                          void* out, void* stream);
+
+/* ----------------------------------------------------------------------- a4-a6: GEMM */
+/* Y[m, n] = sum_k x[m, k] * w[n, k] with fp32 accumulation, Y fp32 [M, N] row-major (device).
+ * x: M rows (F16, BF16 or NVFP4); w: N rows (F16, BF16 or NVFP4).  16-bit x and 16-bit w
+ * must have the same type; NVFP4 w is decoded in-kernel to x's type (bf16 when x is NVFP4).
+ * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
+ * aligned.  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
+ * workspace: device scratch of sp24_gemm_workspace_size() bytes (may be NULL when 0). */
+int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, int64_t M, int64_t N,
+                             int64_t K, int algo, int64_t* bytes);
+int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int64_t M, int64_t N,
+                    int64_t K, float* y, void* workspace, int64_t workspace_bytes, int algo,
+                    void* stream);
+
+/* [P2] "The mechanism needs both values and their positions": the same product with w in
+ * 2:4-compressed form; only kept entries are multiplied.  K alignment: 16-bit values K % 16,
+ * NVFP4 values K % 64. */
+int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M,
+                       int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                       int algo, void* stream);
+
+/* ----------------------------------------------------------------------- diagnostics */
+/* Number of kernels this library has launched in this process (host-side counter, all
+ * devices and streams).  For accounting in benchmarks; memsets are not counted. */
+int64_t sp24_kernel_launches(void);
+
+/* Synchronises `stream`, then returns and clears the device error word of the current device
+ * (SP24_OK when no kernel reported a problem). */
+int sp24_last_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SP24_H_ */

@@ -1,0 +1,112 @@
+"""CPU tests of the C ABI: the library builds and loads, exports every declared entry point, and
+rejects bad arguments on the host without touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp16_gemm_b200 as sp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sp24.h")).read()
+    return sorted(set(re.findall(r"\b(sp24_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = sp.lib()
+    names = declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(sp.EXPORTS) | (set(names) - set(sp.EXPORTS))
+    for n in sp.EXPORTS:
+        assert n in names, f"binding lists {n} but the header does not declare it"
+
+
+def test_status_strings_and_version():
+    L = sp.lib()
+    assert L.sp24_abi_version() == 1
+    for st in range(9):
+        assert L.sp24_status_string(st)
+    assert L.sp24_status_string(999) == b"unknown status"
+
+
+def test_sizes_match_the_pages_byte_counts():
+    """'Bit-exact check against lyf's ModelOpt output': packed / scale bytes of three tensors."""
+    for shape, packed, scl in (((12288, 5120), 31457280, 3932160), ((5120, 6144), 15728640, 1966080),
+                               ((17408, 5120), 44564480, 5570560)):
+        s = sp.sizes(sp.OP_MATMUL, sp.BF16, shape)
+        assert s["nvfp4_codes_bytes"] == packed and s["nvfp4_scales_bytes"] == scl
+
+
+def test_sizes_bits_per_weight():
+    """'The byte saving is about a quarter, not a half': 2 kept values + 2-bit indices."""
+    N, K = 5120, 5120
+    d = sp.sizes(sp.OP_MATMUL, sp.F16, (N, K))
+    assert d["groups"] == N * K // 4
+    assert (d["values_bytes"] + d["meta_bytes"]) * 8 / (N * K) == 9.0
+    v = sp.sizes(sp.OP_MATMUL, sp.F16, (N, K // 2))
+    dense = (d["nvfp4_codes_bytes"] + d["nvfp4_scales_bytes"]) * 8 / (N * K)
+    sparse = (v["nvfp4_codes_bytes"] + v["nvfp4_scales_bytes"] + d["meta_bytes"]) * 8 / (N * K)
+    assert dense == 4.5 and sparse == 3.25
+
+
+def test_conv_sizes_and_shape_rules():
+    s = sp.sizes(sp.OP_CONV, sp.F16, (256, 256, 3, 3))
+    assert s["groups"] == 147456 and s["values_bytes"] == 256 * 128 * 9 * 2 and s["meta_bytes"] == 73728
+    with pytest.raises(sp.SP24Error) as e:
+        sp.sizes(sp.OP_CONV, sp.F16, (2, 6, 3, 3))
+    assert e.value.status == sp.ERR_SHAPE
+
+
+def _raw(fn, *args):
+    return getattr(sp.lib(), fn)(*args)
+
+
+def test_host_validation_without_launch():
+    """Bad arguments come back as status codes before any CUDA call (works with no GPU)."""
+    shp = (ctypes.c_int64 * 4)(2, 6, 3, 3)
+    assert _raw("sp24_check_24", None, sp.F16, sp.OP_CONV, shp, 4, None, None, None) == sp.ERR_SHAPE
+    assert _raw("sp24_check_24", None, 7, sp.OP_MATMUL, shp, 2, None, None, None) == sp.ERR_DTYPE
+    shp2 = (ctypes.c_int64 * 4)(4, 8, 0, 0)
+    assert _raw("sp24_check_24", None, sp.F16, 5, shp2, 2, None, None, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_check_24", None, sp.F16, sp.OP_MATMUL, shp2, 2, None, None, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_prune_compress_24", None, sp.BF16, sp.OP_MATMUL, (ctypes.c_int64 * 4)(4, 6), 2,
+                None, None, None) == sp.ERR_SHAPE
+    n = ctypes.c_int64(0)
+    assert _raw("sp24_quantize_nvfp4_workspace_size", 4, 24, ctypes.byref(n)) == sp.ERR_SHAPE
+    assert _raw("sp24_quantize_nvfp4", None, sp.F32, 4, 24, None, None, None, None, None, 0, None) == sp.ERR_WORKSPACE
+    assert _raw("sp24_dequantize_nvfp4", None, None, None, 4, 24, sp.F32, None, None) == sp.ERR_SHAPE
+
+
+def test_gemm_argument_errors():
+    x = sp._Operand(sp.F16, 16, None, None)
+    w = sp._Operand(sp.BF16, 16, None, None)
+    L = sp.lib()
+    args = lambda M, N, K: (M, N, K, None, None, 0, sp.ALGO_AUTO, None)
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w), *args(8, 8, 64)) == sp.ERR_DTYPE
+    w16 = sp._Operand(sp.F16, 16, None, None)
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w16), *args(8, 8, 60)) == sp.ERR_SHAPE
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w16), *args(-1, 8, 64)) == sp.ERR_SHAPE
+    xm = sp._Operand(sp.F16, 8, None, None)  # misaligned
+    assert L.sp24_gemm_dense(ctypes.byref(xm), ctypes.byref(w16), *args(8, 8, 64)) == sp.ERR_ALIGN
+    q = sp._Operand(sp.NVFP4, 16, None, None)  # NVFP4 without scales
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(q), *args(8, 8, 64)) == sp.ERR_INVALID_ARG
+    sw = sp._SparseOperand(sp.F16, 16, None, None, 16)
+    assert L.sp24_gemm_sparse24(ctypes.byref(x), ctypes.byref(sw), *args(8, 8, 40)) == sp.ERR_SHAPE
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w16), 0, 8, 64, None, None, 0, 9, None) == sp.ERR_INVALID_ARG
+    # empty problems are no-ops that need no device
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w16), *args(0, 8, 64)) == sp.OK
+    assert L.sp24_gemm_sparse24(ctypes.byref(x), ctypes.byref(sw), *args(8, 0, 64)) == sp.OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        sp.check_24(torch.zeros(4, 8, dtype=torch.float16))
+    with pytest.raises(ValueError):
+        sp.quantize_nvfp4(torch.zeros(4, 16))

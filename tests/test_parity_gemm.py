@@ -1,0 +1,117 @@
+"""GPU parity of the dense and 2:4-sparse GEMM/GEMV against the oracle's fp64 GEMM on decoded
+operands: |y - y_ref| <= 1e-3 * sum_k |x||w| per output.  Each side runs the whole pipeline
+(prune -> compress -> NVFP4) from the same seeded inputs on its own."""
+import numpy as np
+import pytest
+import torch
+
+import fp16_gemm_b200 as sp
+import oracle
+import synth
+from helpers import ORACLE_DT, assert_gemm_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+REL = 1e-3  # the tolerance the method's statement fixes for GEMM outputs
+
+
+def make_case(xfmt, wfmt, M, N, K, seed, w_sigma=1.0):
+    """Raw inputs: x and w drawn in a 16-bit source type (bf16 for NVFP4 operands)."""
+    g = synth.rng(seed)
+    xsrc = "f16" if xfmt == "f16" else "bf16"
+    wsrc = "f16" if wfmt == "f16" or (wfmt == "nvfp4" and xfmt == "f16") else "bf16"
+    if xfmt == "nvfp4":
+        wsrc = "bf16"
+    X = synth.draw(g, (M, K), xsrc)
+    W = synth.draw(g, (N, K), wsrc, w_sigma)
+    return X, xsrc, W, wsrc
+
+
+def oracle_side(X, xsrc, xfmt, W, wsrc, wfmt, sparse):
+    if xfmt == "nvfp4":
+        c, s, ts = oracle.nvfp4_encode(X, ORACLE_DT[xsrc])
+        Xd = oracle.nvfp4_decode(c, s, ts)
+    else:
+        Xd = oracle.to_double(X, ORACLE_DT[xsrc])
+    od = ORACLE_DT[wsrc]
+    if sparse:
+        V, meta = oracle.compress_24(W, od)
+        if wfmt == "nvfp4":
+            c, s, ts = oracle.nvfp4_encode(V, od)
+            Vd = oracle.nvfp4_decode(c, s, ts)
+        else:
+            Vd = oracle.to_double(V, od)
+        return oracle.gemm_sparse(Xd, Vd, meta)
+    if wfmt == "nvfp4":
+        c, s, ts = oracle.nvfp4_encode(W, od)
+        Wd = oracle.nvfp4_decode(c, s, ts)
+    else:
+        Wd = oracle.to_double(W, od)
+    return oracle.gemm(Xd, Wd)
+
+
+def gpu_side(X, xsrc, xfmt, W, wsrc, wfmt, sparse, algo=sp.ALGO_AUTO):
+    x = to_dev(X, xsrc)
+    if xfmt == "nvfp4":
+        x = sp.quantize_nvfp4(x)
+    w = to_dev(W, wsrc)
+    K = W.shape[1]
+    if sparse:
+        v, m = sp.prune_compress_24(w)
+        if wfmt == "nvfp4":
+            v = sp.quantize_nvfp4(v)
+        return sp.gemm_sparse24(x, sp.Sparse24(v, m.view(W.shape[0], K // 8)), K, algo=algo)
+    if wfmt == "nvfp4":
+        w = sp.quantize_nvfp4(w)
+    return sp.gemm_dense(x, w, algo=algo)
+
+
+FORMATS = [("f16", "f16"), ("bf16", "bf16"), ("bf16", "nvfp4"), ("f16", "nvfp4"), ("nvfp4", "nvfp4")]
+SHAPES = [(16, 256, 512), (1, 64, 256), (5, 72, 384), (33, 130, 640), (64, 96, 1024), (100, 64, 512)]
+
+
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+@pytest.mark.parametrize("fmt", FORMATS, ids=lambda f: f"x{f[0]}-w{f[1]}")
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_gemm_parity(fmt, shape, sparse):
+    xfmt, wfmt = fmt
+    M, N, K = shape
+    X, xs, W, ws = make_case(xfmt, wfmt, M, N, K, seed=M * 1000 + N + K)
+    Y, S = oracle_side(X, xs, xfmt, W, ws, wfmt, sparse)
+    y = gpu_side(X, xs, xfmt, W, ws, wfmt, sparse)
+    assert_gemm_close(y, Y, S, REL)
+    assert sp.last_device_error() == sp.OK
+
+
+def test_fp16_toy_sparse_vs_dense_on_pruned():
+    """W fp16 [256, 512], X fp16 [16, 512]: check -> prune -> compress -> sparse GEMM, against
+    the dense GEMM on the pruned W, both on the GPU and against the oracle."""
+    d = synth.fp16_toy()
+    X, W = d["X"], d["W"]
+    x, w = to_dev(X, "f16"), to_dev(W, "f16")
+    p, n = sp.check_24(w)
+    assert int(n.item()) == oracle.check_24(W, oracle.F16)[1]
+    v, m = sp.prune_compress_24(w)
+    y_sp = sp.gemm_sparse24(x, sp.Sparse24(v, m), 512)
+    y_dn = sp.gemm_dense(x, sp.decompress_24(v, m, W.shape))
+    Y, S = oracle.gemm(oracle.to_double(X, oracle.F16),
+                       oracle.to_double(oracle.prune_24(W, oracle.F16), oracle.F16))
+    assert_gemm_close(y_sp, Y, S)
+    assert_gemm_close(y_dn, Y, S)
+
+
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+def test_decode_workload_full_size(sparse):
+    """bf16 x [8, 5120], NVFP4 w [5120, 5120] (N(0, 0.02)), every output checked."""
+    d = synth.decode_nvfp4()
+    Y, S = oracle_side(d["X"], "bf16", "bf16", d["W"], "bf16", "nvfp4", sparse)
+    y = gpu_side(d["X"], "bf16", "bf16", d["W"], "bf16", "nvfp4", sparse)
+    assert_gemm_close(y, Y, S)
+
+
+def test_k_zero_writes_zeros():
+    x = torch.zeros((4, 0), dtype=torch.float16, device="cuda")
+    w = torch.zeros((8, 0), dtype=torch.float16, device="cuda")
+    y = torch.full((4, 8), 7.0, device="cuda")
+    sp.gemm_dense(x, w, out=y)
+    assert not y.any()

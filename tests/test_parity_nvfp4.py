@@ -1,0 +1,106 @@
+"""GPU parity of a3 (NVFP4 quantisation): codes, block scales and tensor scale bit-exact against
+the oracle on the same seeded inputs; decode against the oracle's fp64 decode."""
+import numpy as np
+import pytest
+import torch
+
+import fp16_gemm_b200 as sp
+import oracle
+import synth
+from helpers import ORACLE_DT, f64_to_bf16_bits, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(t_np, dtype, ts=None):
+    od = ORACLE_DT[dtype]
+    c_ref, s_ref, ts_ref = oracle.nvfp4_encode(t_np, od, ts)
+    t = to_dev(t_np, dtype)
+    ts_dev = None if ts is None else torch.tensor([ts], dtype=torch.float32, device="cuda")
+    q = sp.quantize_nvfp4(t, tensor_scale=ts_dev)
+    torch.cuda.synchronize()
+    assert np.float32(q.tensor_scale.item()).view(np.uint32) == np.float32(ts_ref).view(np.uint32)
+    s = to_host(q.scales)
+    c = to_host(q.codes)
+    bad_s = np.argwhere(s != s_ref)
+    assert bad_s.size == 0, f"{len(bad_s)} scale mismatches, first {bad_s[:3].tolist()}"
+    bad_c = np.argwhere(c != c_ref)
+    assert bad_c.size == 0, f"{len(bad_c)} code mismatches, first {bad_c[:3].tolist()}"
+    return q, (c_ref, s_ref, ts_ref)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (64, 512), (129, 1040)])
+def test_random_rows_of_varied_scale(dtype, shape):
+    g = synth.rng(shape[0] * 31 + shape[1])
+    x = synth.normal(g, shape) * np.exp(2 * synth.normal(g, (shape[0], 1)))
+    _compare(synth.as_storage(x, dtype), dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_subnormal_block_scales(dtype):
+    """Blocks far below the tensor max get E4M3 subnormal scales (and E2M1 half steps)."""
+    g = synth.rng(5)
+    x = synth.normal(g, (16, 256))
+    x[:, :128] *= 1e-3
+    x[0, 0] = 40.0
+    x[3, 16:32] = 0.0
+    _compare(synth.as_storage(x, dtype), dtype)
+
+
+def test_fp32_tiny_tensor_scale():
+    """amax ~1e-36: the tensor scale is an fp32 subnormal; no flush to zero on the GPU."""
+    x = synth.normal(synth.rng(6), (4, 64)).astype(np.float32) * np.float32(1e-37)
+    _compare(x, "f32")
+
+
+def test_supplied_shared_scale_and_saturation():
+    x = synth.normal(synth.rng(7), (8, 128)).astype(np.float32)
+    ts = float(oracle.nvfp4_encode(x, oracle.F32)[2])
+    _compare(x, "f32", ts)
+    _compare(x, "f32", ts * 8)        # scale of a larger partner tensor
+    _compare(x, "f32", ts / 1000.0)   # saturating: codes at 6, scales at 448
+
+
+def test_zeros_and_negative_zero():
+    x = np.zeros((2, 32), np.float32)
+    x[1, 3] = -0.0
+    x[0, 5] = -1e-9
+    x[0, 6] = 1.0
+    q, _ = _compare(x, "f32")
+    z = np.zeros((2, 32), np.float32)
+    z[0, 1] = -0.0
+    _compare(z, "f32")
+
+
+def test_decode_workload_dense_and_sparse():
+    """The decode workload's weight, bf16 [5120, 5120] N(0, 0.02): dense NVFP4, and NVFP4 of its
+    2:4-compressed values [5120, 2560] (one scale per 16 stored values)."""
+    w_np = synth.decode_nvfp4()["W"]
+    _compare(w_np, "bf16")
+    v_np, _ = oracle.compress_24(w_np, oracle.BF16)
+    q, ref = _compare(v_np, "bf16")
+    # amax survives pruning: the two tensor scales agree
+    assert ref[2] == oracle.nvfp4_encode(w_np, oracle.BF16)[2]
+
+
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16, torch.float16])
+def test_dequantize(out):
+    x = synth.normal(synth.rng(8), (24, 160)).astype(np.float32)
+    c, s, ts = oracle.nvfp4_encode(x, oracle.F32)
+    ref = oracle.nvfp4_decode(c, s, ts)
+    q = sp.NVFP4Tensor(to_dev(c, "u8"), to_dev(s, "u8"),
+                       torch.tensor([ts], dtype=torch.float32, device="cuda"))
+    d = to_host(sp.dequantize_nvfp4(q, out))
+    if out == torch.float32:
+        assert np.array_equal(d.view(np.uint32), ref.astype(np.float32).view(np.uint32))
+    elif out == torch.float16:
+        assert np.array_equal(d.view(np.uint16), ref.astype(np.float16).view(np.uint16))
+    else:
+        assert np.array_equal(d, f64_to_bf16_bits(ref))
+
+
+def test_empty_tensor_writes_scale():
+    t = torch.empty((0, 32), dtype=torch.bfloat16, device="cuda")
+    q = sp.quantize_nvfp4(t)
+    assert q.codes.numel() == 0 and float(q.tensor_scale.item()) == 0.0
