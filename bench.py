@@ -11,9 +11,10 @@ pages' NVFP4 decode kernels, hidden width 5120).  Inputs live in HBM before timi
 rotate over 4 seeded input sets (about 440 MB in total, well beyond the 126 MB L2), so each
 step reads its weight from DRAM.
 
-Each stage is captured once per input set as a CUDA graph; the timed loop replays the stage
-graphs and records a CUDA event after each stage, which gives the per-stage device time inside
-the timed region.  `value` is the whole step's algorithmic HBM traffic divided by the step
+The timed steps are captured in windows of up to 16 consecutive steps, one CUDA graph per
+window, with an external CUDA event record node after every stage; the timed region replays
+each window once, so the per-stage device times come from the timed region itself and the host
+pays one graph launch per window.  `value` is the whole step's algorithmic HBM traffic divided by the step
 time (GB/s); the GEMV comparison (dense vs 2:4 sparse: TFLOP/s, GB/s, speedup) is in `gemv`.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -204,56 +205,57 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     torch.cuda.synchronize()
     assert sp.last_device_error() == sp.OK
 
-    # capture one graph per (set, stage)
-    graphs = []
+    # Timed steps are captured in windows of U consecutive steps, one CUDA graph per window, each
+    # stage followed by an external event record node (its own event objects, so nothing is
+    # overwritten before it is read).  Replaying a window costs one graph launch on the host.
+    U = max(u for u in range(1, 17) if args.steps % u == 0)
+    n_win = args.steps // U
     n0 = sp.kernel_launches()
     cap = torch.cuda.Stream()
-    for s in sets:
-        row = []
-        for f in stage_fns(s):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
-                f()
-            row.append(g)
-        graphs.append(row)
-    launches_per_step = (sp.kernel_launches() - n0) // len(sets)
+    windows = []
+    for wi in range(n_win):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(1 + U * len(STAGES))]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            evs[0].record()
+            for j in range(U):
+                fns = stage_fns(sets[(wi * U + j) % len(sets)])
+                for si, f in enumerate(fns):
+                    f()
+                    evs[1 + j * len(STAGES) + si].record()
+        windows.append((g, evs))
+    launches_per_step = (sp.kernel_launches() - n0) // args.steps
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-
-    def run_steps(n, events=None, offset=0):
-        for j in range(n):
-            row = graphs[(offset + j) % len(graphs)]
-            for si, g in enumerate(row):
-                g.replay()
-                if events is not None:
-                    events[j][si + 1].record(stream)
-
-    run_steps(args.warmup)
+    # warm-up: the first W steps' windows (rounded up to whole windows)
+    for wi in range(min(n_win, (args.warmup + U - 1) // U)):
+        windows[wi][0].replay()
     torch.cuda.synchronize()
 
-    # per-step, per-stage events (fresh objects: nothing is overwritten before it is read)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
-           for _ in range(args.steps)]
-    for j in range(args.steps):
-        evs[j][0] = evs[j - 1][-1] if j > 0 else torch.cuda.Event(enable_timing=True)
-    t_start = evs[0][0]
-
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     host0 = time.perf_counter()
     with ClockSampler(torch.cuda.current_device()) as clk:
         t_start.record(stream)
-        run_steps(args.steps, evs, offset=args.warmup)
+        for g, _ in windows:
+            g.replay()
+        t_end.record(stream)
         host_enqueue = time.perf_counter() - host0
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    t_end = evs[-1][-1]
     total_ms = t_start.elapsed_time(t_end)
-    stage_ms = [sum(evs[j][si].elapsed_time(evs[j][si + 1]) for j in range(args.steps)) / args.steps
-                for si in range(len(STAGES))]
+    stage_ms = [0.0] * len(STAGES)
+    for _, evs in windows:
+        for j in range(U):
+            for si in range(len(STAGES)):
+                k = 1 + j * len(STAGES) + si
+                stage_ms[si] += evs[k - 1].elapsed_time(evs[k])
+    stage_ms = [v / args.steps for v in stage_ms]
 
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)

@@ -56,10 +56,51 @@ int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
       q.x = reinterpret_cast<const uint8_t*>(p.x) + m0 * p.K / 2;
       q.x_scales = p.x_scales + m0 * p.K / 16;
     }
-    int st = skinny_gemm(wf, t16, q, s);
+    int st = skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s) : skinny_gemm(wf, t16, q, s);
     if (st) return st;
   }
   return SP24_OK;
+}
+
+int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace of the tiled path: 16-bit copies of the operands that are not 16-bit already.
+int64_t tiled_workspace(int x_fmt, int wf, int64_t M, int64_t N, int64_t K) {
+  int64_t b = 0;
+  if (wf != W_D16) b += round256(N * K * 2);
+  if (x_fmt == X_Q4) b += round256(M * K * 2);
+  return b;
+}
+
+// Tiled (tcgen05) path: expand what is not plain 16-bit into the workspace, then one GEMM.
+int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes, cudaStream_t s) {
+  const int64_t need = tiled_workspace(p.x_fmt, wf, p.M, p.N, p.K);
+  if (need > 0 && (!ws || ws_bytes < need)) return SP24_ERR_WORKSPACE;
+  if (need > 0 && !aligned(ws, 256)) return SP24_ERR_ALIGN;
+  const bool bf = t16 == SP24_BF16;
+  uint8_t* cur = reinterpret_cast<uint8_t*>(ws);
+  const void* w16 = p.w;
+  if (wf != W_D16) {
+    int st = expand_w16(wf, bf, p.w, p.w_scales, p.meta, p.N, p.K, reinterpret_cast<uint16_t*>(cur), s);
+    if (st) return st;
+    w16 = cur;
+    cur += round256(p.N * p.K * 2);
+  }
+  const void* x16 = p.x;
+  if (p.x_fmt == X_Q4) {
+    int st = expand_w16(W_DQ4, bf, reinterpret_cast<const uint8_t*>(p.x), p.x_scales, nullptr, p.M, p.K,
+                        reinterpret_cast<uint16_t*>(cur), s);
+    if (st) return st;
+    x16 = cur;
+  }
+  const float* sa = (wf == W_DQ4 || wf == W_SQ4) ? p.w_ts : nullptr;
+  const float* sb = p.x_fmt == X_Q4 ? p.x_ts : nullptr;
+  return tc_gemm_f16(x16, w16, p.M, p.N, p.K, bf, p.y, sa, sb, s);
+}
+
+int dispatch(int wf, int t16, const SkinnyParams& p, int algo, void* ws, int64_t ws_bytes, cudaStream_t s) {
+  if (algo == SP24_ALGO_SKINNY || (algo == SP24_ALGO_AUTO && p.M <= 64)) return run_skinny(wf, t16, p, s);
+  return run_tiled(wf, t16, p, ws, ws_bytes, s);
 }
 
 }  // namespace
@@ -117,16 +158,21 @@ extern "C" int sp24_sizes(int op, int dtype, const int64_t* shape, int ndim, int
 
 extern "C" int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, int64_t M,
                                         int64_t N, int64_t K, int algo, int64_t* bytes) {
-  (void)x_format; (void)w_format; (void)sparse; (void)M; (void)N; (void)K; (void)algo;
   if (!bytes) return SP24_ERR_INVALID_ARG;
-  *bytes = 0;
+  if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
+  if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
+  if (!(is16(x_format) || x_format == SP24_NVFP4) || !(is16(w_format) || w_format == SP24_NVFP4))
+    return SP24_ERR_DTYPE;
+  const int wf = sparse ? (is16(w_format) ? W_S16 : W_SQ4) : (is16(w_format) ? W_D16 : W_DQ4);
+  const int xf = x_format == SP24_NVFP4 ? X_Q4 : X_16;
+  const bool tiled = algo == SP24_ALGO_TILED || (algo == SP24_ALGO_AUTO && M > 64);
+  *bytes = tiled ? tiled_workspace(xf, wf, M, N, K) : 0;
   return SP24_OK;
 }
 
 extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int64_t M, int64_t N,
                                int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                                int algo, void* stream) {
-  (void)workspace; (void)workspace_bytes;
   if (!x || !w) return SP24_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
   if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
@@ -154,7 +200,6 @@ extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int
   if (!y) return SP24_ERR_INVALID_ARG;
   if (K > 0 && !w->data) return SP24_ERR_INVALID_ARG;
   if (!aligned(w->data, 16)) return SP24_ERR_ALIGN;
-  if (algo == SP24_ALGO_TILED) return SP24_ERR_UNSUPPORTED;
   p.w = reinterpret_cast<const uint8_t*>(w->data);
   p.w_scales = w->scales;
   p.w_ts = w->tensor_scale;
@@ -162,13 +207,12 @@ extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int
   p.N = N;
   p.K = K;
   p.y = y;
-  return run_skinny(wf, t16, p, as_stream(stream));
+  return dispatch(wf, t16, p, algo, workspace, workspace_bytes, as_stream(stream));
 }
 
 extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M,
                                   int64_t N, int64_t K, float* y, void* workspace,
                                   int64_t workspace_bytes, int algo, void* stream) {
-  (void)workspace; (void)workspace_bytes;
   if (!x || !w) return SP24_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
   if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
@@ -198,7 +242,6 @@ extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_opera
   if (!y) return SP24_ERR_INVALID_ARG;
   if (K > 0 && (!w->values || !w->meta)) return SP24_ERR_INVALID_ARG;
   if (!aligned(w->values, 16) || !aligned(w->meta, 8)) return SP24_ERR_ALIGN;
-  if (algo == SP24_ALGO_TILED) return SP24_ERR_UNSUPPORTED;
   p.w = reinterpret_cast<const uint8_t*>(w->values);
   p.w_scales = w->scales;
   p.w_ts = w->tensor_scale;
@@ -207,7 +250,7 @@ extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_opera
   p.N = N;
   p.K = K;
   p.y = y;
-  return run_skinny(wf, t16, p, as_stream(stream));
+  return dispatch(wf, t16, p, algo, workspace, workspace_bytes, as_stream(stream));
 }
 
 extern "C" int64_t sp24_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }

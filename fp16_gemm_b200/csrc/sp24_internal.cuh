@@ -82,4 +82,17 @@ struct SkinnyParams {
 // Launches the skinny kernel for M <= 64 (wf: W_*, t16: SP24_F16 / SP24_BF16 MMA type).
 int skinny_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 
+// Shared-memory staged skinny kernel (bulk copies + native 2:4 MMA); supported() checks the
+// alignment its bulk copies need.
+bool skinny2_supported(int wf, const SkinnyParams& p);
+int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
+
+// Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
+int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,
+                const float* scale_a, const float* scale_b, cudaStream_t s);
+
+// Expands an NVFP4 (W_DQ4) or 2:4-compressed (W_S16 / W_SQ4) operand into exact 16-bit values.
+int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta,
+               int64_t rows, int64_t K, uint16_t* out, cudaStream_t s);
+
 }  // namespace sp24

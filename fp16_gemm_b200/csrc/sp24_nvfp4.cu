@@ -77,16 +77,27 @@ __device__ __forceinline__ uint32_t e2m1x2_rne_satfinite(float x_lo, float x_hi)
   return r & 0xffu;
 }
 
+// Blocks handled per loop iteration by one thread (their loads are issued together).
+constexpr int kBlocksPerIter = 2;
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ t, int64_t nblk,
                                                         unsigned int* __restrict__ amax_bits) {
   float m = 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
-    float v[16];
-    load_block<DT>(t, b, v);
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += kBlocksPerIter * stride) {
+    float v[kBlocksPerIter][16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    for (int u = 0; u < kBlocksPerIter; ++u) {
+      if (b + u * stride < nblk) load_block<DT>(t, b + u * stride, v[u]);
+      else
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[u][i] = 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBlocksPerIter; ++u)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[u][i]));
   }
   unsigned int u = __float_as_uint(m);
   u = __reduce_max_sync(0xffffffffu, u);
@@ -98,6 +109,28 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
     x = __reduce_max_sync(0xffffffffu, x);
     if (threadIdx.x == 0 && x) atomicMax(amax_bits, x);
   }
+}
+
+// Encodes one 16-entry block given the tensor scale s_t and d = s_t * 6.
+__device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, float d, uint2* codes,
+                                             uint8_t* scales, int64_t b) {
+  float bmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+  uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
+  const float sc = __fmul_rn(e4m3_value(sb), s_t);
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    float q0 = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
+    float q1 = sc != 0.0f ? __fdiv_rn(fabsf(v[i + 1]), sc) : 0.0f;
+    uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
+    byte |= (__float_as_uint(v[i]) >> 31) << 3;       // sign of the low entry
+    byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;   // sign of the high entry
+    packed[i / 8] |= byte << (8 * ((i % 8) / 2));
+  }
+  codes[b] = make_uint2(packed[0], packed[1]);
+  scales[b] = (uint8_t)sb;
 }
 
 template <int DT>
@@ -112,26 +145,14 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const void* __restrict
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
   const float d = __fmul_rn(s_t, 6.0f);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
-    float v[16];
-    load_block<DT>(t, b, v);
-    float bmax = 0.0f;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += kBlocksPerIter * stride) {
+    float v[kBlocksPerIter][16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-    uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
-    const float sc = __fmul_rn(e4m3_value(sb), s_t);
-    uint32_t packed[2] = {0u, 0u};
+    for (int u = 0; u < kBlocksPerIter; ++u)
+      if (b + u * stride < nblk) load_block<DT>(t, b + u * stride, v[u]);
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      float q0 = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
-      float q1 = sc != 0.0f ? __fdiv_rn(fabsf(v[i + 1]), sc) : 0.0f;
-      uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
-      byte |= (__float_as_uint(v[i]) >> 31) << 3;       // sign of the low entry
-      byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;   // sign of the high entry
-      packed[i / 8] |= byte << (8 * ((i % 8) / 2));
-    }
-    codes[b] = make_uint2(packed[0], packed[1]);
-    scales[b] = (uint8_t)sb;
+    for (int u = 0; u < kBlocksPerIter; ++u)
+      if (b + u * stride < nblk) encode_block(v[u], s_t, d, codes, scales, b + u * stride);
   }
 }
 

@@ -76,23 +76,34 @@ __device__ __forceinline__ void count_fails(int fails, int32_t* n_fail) {
 
 // Groups 2v, 2v+1 (16-bit) or group v (fp32) per 16-byte vector v.  Every lane of a warp runs
 // the same number of iterations so the final warp reduction sees all lanes.
+// Each thread keeps kUnroll independent 16-byte loads in flight (vectors base + lane + i*stride),
+// enough bytes per SM to cover DRAM latency at full bandwidth.
+constexpr int kUnroll = 4;
+
 template <int EB>
 __global__ void __launch_bounds__(kThreads) check24_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint8_t* __restrict__ pass,
                                                         int32_t* __restrict__ n_fail) {
   int fails = 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~int64_t(31);
-  for (int64_t base = warp0; base < nv; base += stride) {
-    int64_t v = base + (threadIdx.x & 31);
-    if (v < nv) {
-      uint4 x = ldg_stream16(w + v);
+  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t base = t0; base - (threadIdx.x & 31) < nv; base += kUnroll * stride) {
+    uint4 x[kUnroll];
+#pragma unroll
+    for (int i = 0; i < kUnroll; ++i) {
+      const int64_t v = base + i * stride;
+      x[i] = v < nv ? ldg_stream16(w + v) : make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+    }
+#pragma unroll
+    for (int i = 0; i < kUnroll; ++i) {
+      const int64_t v = base + i * stride;
+      if (v >= nv) continue;
       if (EB == 2) {
-        int ok0 = zeros16(x.x, x.y) >= 2, ok1 = zeros16(x.z, x.w) >= 2;
+        int ok0 = zeros16(x[i].x, x[i].y) >= 2, ok1 = zeros16(x[i].z, x[i].w) >= 2;
         fails += 2 - ok0 - ok1;
         reinterpret_cast<uint16_t*>(pass)[v] = (uint16_t)(ok0 | (ok1 << 8));
       } else {
-        int ok = zeros32(x) >= 2;
+        int ok = zeros32(x[i]) >= 2;
         fails += 1 - ok;
         pass[v] = (uint8_t)ok;
       }
@@ -106,31 +117,37 @@ __global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict_
                                                         uint2* __restrict__ values,
                                                         uint8_t* __restrict__ meta) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~int64_t(31);
-  const int lane = threadIdx.x & 31;
-  for (int64_t base = warp0; base < nv; base += stride) {
-    int64_t v = base + lane;
-    bool live = v < nv;
-    uint4 x = live ? ldg_stream16(w + v) : make_uint4(0, 0, 0, 0);
-    if (EB == 2) {
-      if (live) {
-        Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
-        values[v] = make_uint2(a.kept, b.kept);
-        meta[v] = (uint8_t)(a.nib | (b.nib << 4));
-      }
-    } else {
-      uint32_t m = keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w));
-      uint32_t nib = mask_nibble(m);
-      uint32_t e[4] = {x.x, x.y, x.z, x.w};
-      uint32_t i0 = nib & 3, i1 = nib >> 2;
-      uint32_t v0 = i0 == 0 ? e[0] : (i0 == 1 ? e[1] : e[2]);
-      uint32_t v1 = i1 == 3 ? e[3] : (i1 == 2 ? e[2] : e[1]);
-      // the partner group v^1 lives in lane^1 (the warp's first vector index is even)
-      uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
-      if (live) {
-        values[v] = make_uint2(v0, v1);
-        bool partner_live = (v ^ 1) < nv;
-        if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (partner_live ? other << 4 : 0u));
+  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t base = t0; base - (threadIdx.x & 31) < nv; base += kUnroll * stride) {
+    uint4 x[kUnroll];
+#pragma unroll
+    for (int i = 0; i < kUnroll; ++i) {
+      const int64_t v = base + i * stride;
+      x[i] = v < nv ? ldg_stream16(w + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kUnroll; ++i) {
+      const int64_t v = base + i * stride;
+      const bool live = v < nv;
+      if (EB == 2) {
+        if (live) {
+          Group16 a = prune16(x[i].x, x[i].y), b = prune16(x[i].z, x[i].w);
+          values[v] = make_uint2(a.kept, b.kept);
+          meta[v] = (uint8_t)(a.nib | (b.nib << 4));
+        }
+      } else {
+        uint32_t m = keep_mask(mag32(x[i].x), mag32(x[i].y), mag32(x[i].z), mag32(x[i].w));
+        uint32_t nib = mask_nibble(m);
+        uint32_t i0 = nib & 3, i1 = nib >> 2;
+        uint32_t v0 = i0 == 0 ? x[i].x : (i0 == 1 ? x[i].y : x[i].z);
+        uint32_t v1 = i1 == 3 ? x[i].w : (i1 == 2 ? x[i].z : x[i].y);
+        // the partner group v^1 lives in lane^1 (each warp's first vector index is even)
+        uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+        if (live) {
+          values[v] = make_uint2(v0, v1);
+          bool partner_live = (v ^ 1) < nv;
+          if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (partner_live ? other << 4 : 0u));
+        }
       }
     }
   }

@@ -1,0 +1,478 @@
+// a6: skinny (decode-shaped, M <= 64) dense and 2:4-sparse GEMM, shared-memory staged.
+//
+// [P5] "NVFP4 Without FP4 Hardware", "Why NVFP4 helps without FP4 hardware": a decode step
+// reads every weight once, so the GEMV is bound by the weight read and the 4-bit values are
+// unpacked inside the kernel.  [P2] "Sparse GPU FLOPS Need the Right Zeros in the Right
+// Places", "The mechanism needs both values and their positions": the 2:4 path hands the kept
+// values and their 2-bit positions to the sparse tensor-core MMA, which selects the matching
+// activations itself.
+//
+// CTA = 4 warps = 64 weight rows x one K-slice of KC logical entries.
+//   1. Lanes issue one cp.async.bulk per weight row (values/codes, NVFP4 block scales, 2:4
+//      nibbles) into padded shared-memory rows, all completing on one mbarrier; the whole
+//      slice is in flight at once without costing registers.
+//   2. Meanwhile the CTA stages x[M, slice] into shared memory in MMA-fragment order with
+//      16-byte loads, so every B fragment is one conflict-free shared load.
+//   3. Each warp owns 16 rows: it reads its A fragments from shared memory (row pitches chosen
+//      so the reads are bank-conflict free), decodes NVFP4 to 16 bits in registers, and issues
+//      mma.m16n8k16 (dense) or mma.sp m16n8k32 (2:4, metadata from the nibble stream).
+//   4. K-slices are reduced into y with fp32 atomics (y zeroed first) when there are several.
+//
+// Dense layouts: a lane reads a contiguous 16-byte piece of a row per chunk and the K order
+// inside the chunk is permuted (x is staged with the same permutation).  2:4 layouts: the
+// hardware wants lane (g, c) to supply the kept pair of MMA groups c and c+4 of rows g, g+8,
+// and takes the nibbles of groups 0-3 / 4-7 of rows g | g+8 from lanes c = 0 / 1; with the
+// identity group order inside each 32-wide K window those nibbles are the low / high halves of
+// one 32-bit word of each row's nibble stream.
+#include "sp24_internal.cuh"
+#include "sp24_tc.cuh"
+
+namespace sp24 {
+namespace {
+
+using tc::mbar_arrive_expect_tx;
+using tc::mbar_init;
+using tc::mbar_wait;
+using tc::smem_u32;
+
+constexpr int kWarps = 4;
+constexpr int kRows = kWarps * 16;
+
+// Per format: logical K per slice, bytes per row per slice of each array, shared row pitches.
+template <int WF>
+struct F2;
+template <>
+struct F2<W_D16> {  // 16-bit dense: 8 values (16 B) per lane piece, chunk = 32 K
+  static constexpr int KC = 256, CHUNK = 32, STEPS = 2;
+  static constexpr int VB = KC * 2;
+  static constexpr int VP = VB + 64, SP = 0, MP = 0;
+};
+template <>
+struct F2<W_DQ4> {  // NVFP4 dense: 32 codes (16 B) per lane piece, chunk = 128 K
+  static constexpr int KC = 512, CHUNK = 128, STEPS = 8;
+  static constexpr int VB = KC / 2, SB = KC / 16;
+  static constexpr int VP = VB + 64, SP = SB + 16, MP = 0;
+};
+template <>
+struct F2<W_S16> {  // 16-bit 2:4: windows of 32 K (8 groups, 32 B of values)
+  static constexpr int KC = 512, CHUNK = 32, STEPS = 1;
+  static constexpr int VB = KC, MB = KC / 8;
+  static constexpr int VP = VB + 16, SP = 0, MP = MB + 16;
+};
+template <>
+struct F2<W_SQ4> {  // NVFP4 2:4: windows of 32 K (8 groups, 8 B of codes, one block scale)
+  static constexpr int KC = 1024, CHUNK = 32, STEPS = 1;
+  static constexpr int VB = KC / 4, SB = KC / 32, MB = KC / 8;
+  static constexpr int VP = VB + 16, SP = SB + 16, MP = MB + 16;
+};
+
+template <int WF>
+__host__ __device__ constexpr bool sparse_fmt() { return WF == W_S16 || WF == W_SQ4; }
+
+// Bytes of x fragments per (chunk or window, step, token tile): 32 lanes x 8 B (k16 MMA) or
+// x 16 B (k32 sparse MMA).
+template <int WF>
+__host__ __device__ constexpr int frag_bytes() { return sparse_fmt<WF>() ? 512 : 256; }
+
+template <int WF, int NT>
+struct Smem2 {
+  using C = F2<WF>;
+  static constexpr int XB = (C::KC / C::CHUNK) * C::STEPS * NT * frag_bytes<WF>();
+  static constexpr int OFF_V = XB;
+  static constexpr int OFF_S = OFF_V + kRows * C::VP;
+  static constexpr int OFF_M = OFF_S + kRows * C::SP;
+  static constexpr int TOTAL = OFF_M + kRows * C::MP;
+};
+
+template <typename T>
+struct P2;
+template <>
+struct P2<__nv_bfloat16> {  // 16-bit pattern of E2M1(code) * 2^-126
+  static constexpr uint32_t MAG = 0x01C001C0u;
+  static constexpr int MAGPOS = 6;
+  static constexpr float FOLD = 0x1p118f;
+};
+template <>
+struct P2<__half> {  // 16-bit pattern of E2M1(code) * 2^-14
+  static constexpr uint32_t MAG = 0x0E000E00u;
+  static constexpr int MAGPOS = 9;
+  static constexpr float FOLD = 0x1p6f;
+};
+
+__device__ __forceinline__ uint32_t shl2(uint32_t x, int n) { return n >= 0 ? x << n : x >> (-n); }
+
+// Nibbles i and i+4 of w -> 16-bit pair of E2M1 patterns.
+template <typename T>
+__device__ __forceinline__ uint32_t fp4_pair_i4(uint32_t w, int i) {
+  return (shl2(w, P2<T>::MAGPOS - 4 * i) & P2<T>::MAG) | (shl2(w, 12 - 4 * i) & 0x80008000u);
+}
+
+// The byte at bits [8bb, 8bb+8) of w (two consecutive codes) -> 16-bit pair (lo, hi).
+template <typename T>
+__device__ __forceinline__ uint32_t fp4_pair_byte(uint32_t w, int bb) {
+  const uint32_t x = w >> (8 * bb);
+  constexpr int P = P2<T>::MAGPOS;
+  return ((x << P) & (7u << P)) | ((x << 12) & 0x8000u) | ((x << (P + 12)) & (7u << (P + 16))) |
+         ((x << 24) & 0x80000000u);
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  } else {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ uint16_t to_bits16(float f) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    __nv_bfloat16 v = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&v);
+  } else {
+    __half v = __float2half_rn(f);
+    return *reinterpret_cast<uint16_t*>(&v);
+  }
+}
+
+// Two E4M3 block scales (low bytes of code2) -> two packed multipliers E4M3 * FOLD (exact).
+template <typename T>
+__device__ __forceinline__ void scale_pair(uint32_t code2, uint32_t& s0, uint32_t& s1) {
+  uint32_t h2;
+  const uint16_t c = (uint16_t)code2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+  const uint32_t a = to_bits16<T>(__half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu))) * P2<T>::FOLD);
+  const uint32_t b = to_bits16<T>(__half2float(__ushort_as_half((unsigned short)(h2 >> 16))) * P2<T>::FOLD);
+  s0 = a | (a << 16);
+  s1 = b | (b << 16);
+}
+
+template <typename T>
+__device__ __forceinline__ void mma_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint2 b) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+}
+
+// Sparse m16n8k32 with ordered metadata (kept indices ascending in each group), selector 0.
+template <typename T>
+__device__ __forceinline__ void mma_sp_k32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint4 b, uint32_t e) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    asm volatile(
+        "mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, 0x0;"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(e));
+  else
+    asm volatile(
+        "mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, 0x0;"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(e));
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// x[n, k] as 16-bit bits of T (0 outside the matrix); NVFP4 x decoded to E2M1 * E4M3.
+template <typename T>
+__device__ __forceinline__ uint32_t xval(const SkinnyParams& p, int64_t n, int64_t k) {
+  if (n >= p.M || k >= p.K) return 0;
+  if (p.x_fmt == X_16) return __ldg(reinterpret_cast<const unsigned short*>(p.x) + n * p.K + k);
+  const uint8_t* codes = reinterpret_cast<const uint8_t*>(p.x);
+  const uint32_t c = (codes[(n * p.K + k) >> 1] >> (4 * (k & 1))) & 0xf;
+  const uint32_t mag = c & 7, e = mag >> 1, m = mag & 1;
+  const float a = e == 0 ? 0.5f * m : (float)(1 << (e - 1)) * (1.0f + 0.5f * m);
+  uint32_t h2;
+  const uint16_t sc = p.x_scales[(n * p.K + k) >> 4];
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(sc));
+  const float v = a * __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
+  return to_bits16<T>(c & 8 ? -v : v);
+}
+
+// Eight consecutive x entries [k, k+8) of token n as four packed 16-bit pairs.
+template <typename T>
+__device__ __forceinline__ uint4 xoct(const SkinnyParams& p, int64_t n, int64_t k) {
+  if (p.x_fmt == X_16 && n < p.M && k + 8 <= p.K)
+    return __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
+  uint32_t v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = xval<T>(p, n, k + i);
+  return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
+}
+
+template <int WF, typename T, int NT>
+__global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams p) {
+  using C = F2<WF>;
+  using L = Smem2<WF, NT>;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  const int64_t row0 = (int64_t)blockIdx.x * kRows;
+  const int64_t k0 = (int64_t)blockIdx.y * C::KC;
+  const int64_t kv = p.K - k0 < C::KC ? p.K - k0 : C::KC;  // valid logical K in this slice
+  const int rows_v = (int)(p.N - row0 < kRows ? p.N - row0 : kRows);
+
+  // ---- 1. bulk copies of the weight slice (thread r < rows_v copies row r)
+  const uint32_t vbytes = (uint32_t)(WF == W_D16 ? kv * 2 : WF == W_DQ4 ? kv / 2 : WF == W_S16 ? kv : kv / 4);
+  const uint32_t sbytes = (uint32_t)(WF == W_DQ4 ? kv / 16 : WF == W_SQ4 ? kv / 32 : 0);
+  const uint32_t mbytes = (uint32_t)(sparse_fmt<WF>() ? kv / 8 : 0);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_arrive_expect_tx(&bar, (uint32_t)rows_v * (vbytes + sbytes + mbytes));
+  __syncthreads();
+  if (threadIdx.x < rows_v) {
+    const int64_t r = row0 + threadIdx.x;
+    bulk_g2s(sm + L::OFF_V + threadIdx.x * C::VP, p.w + r * p.w_row_bytes + (WF == W_D16 ? k0 * 2 : WF == W_DQ4 ? k0 / 2 : WF == W_S16 ? k0 : k0 / 4), vbytes, &bar);
+    if (sbytes)
+      bulk_g2s(sm + L::OFF_S + threadIdx.x * C::SP, p.w_scales + r * p.scale_row_bytes + (WF == W_DQ4 ? k0 / 16 : k0 / 32), sbytes, &bar);
+    if (mbytes) bulk_g2s(sm + L::OFF_M + threadIdx.x * C::MP, p.meta + r * p.meta_row_bytes + k0 / 8, mbytes, &bar);
+  }
+  // Fill what no copy writes: the tail of each row when the slice is short, and whole rows
+  // past N.  Values become +0 (uninitialised bits could be NaN, and NaN * 0 is NaN) and
+  // nibbles the legal pair (0, 1).  The regions are disjoint from the copies' destinations.
+  if (kv < C::KC || rows_v < kRows) {
+    for (int i = threadIdx.x; i < kRows * (C::VP / 4); i += blockDim.x) {
+      const int r = i / (C::VP / 4), off = (i % (C::VP / 4)) * 4;
+      if (r >= rows_v || off >= (int)vbytes) *reinterpret_cast<uint32_t*>(sm + L::OFF_V + r * C::VP + off) = 0u;
+    }
+    if constexpr (C::SP > 0)
+      for (int i = threadIdx.x; i < kRows * C::SP; i += blockDim.x)
+        if (i / C::SP >= rows_v || i % C::SP >= (int)sbytes) sm[L::OFF_S + i] = 0;
+    if constexpr (C::MP > 0)
+      for (int i = threadIdx.x; i < kRows * C::MP; i += blockDim.x)
+        if (i / C::MP >= rows_v || i % C::MP >= (int)mbytes) sm[L::OFF_M + i] = 0x44;
+  }
+
+  // ---- 2. stage x in fragment order
+  constexpr int NCH = C::KC / C::CHUNK;
+  if constexpr (!sparse_fmt<WF>()) {
+    // entry (ch, s, t, lane): 8 bytes = x[8t+g][k0 + ch*CHUNK + LV*c + kslot(s, 0..3)]
+    constexpr int LV = C::CHUNK / 4;
+    uint2* xs = reinterpret_cast<uint2*>(sm);
+    // one thread per (ch, t, lane, s-pair): 8 consecutive k of the lane piece -> two entries
+    constexpr int PAIRS = C::STEPS / 2 > 0 ? C::STEPS / 2 : 1;
+    const int items = NCH * NT * 32 * (LV / 8);
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int oct = it % (LV / 8), ln = (it / (LV / 8)) % 32, t = (it / (LV / 8) / 32) % NT,
+                ch = it / (LV / 8) / 32 / NT;
+      const int gg = ln >> 2, cc = ln & 3;
+      const int64_t kb = k0 + (int64_t)ch * C::CHUNK + LV * cc + 8 * oct;
+      const uint4 v = xoct<T>(p, 8 * t + gg, kb);
+      // the octet covers steps 2*oct and 2*oct+1 of this lane piece
+      uint2 e0, e1;
+      if (WF == W_DQ4) {  // slots (0,4,1,5) and (2,6,3,7) of the octet
+        e0 = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
+        e1 = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+      } else {  // slots 0..3 and 4..7
+        e0 = make_uint2(v.x, v.y);
+        e1 = make_uint2(v.z, v.w);
+      }
+      const int s0 = 2 * oct;
+      xs[((ch * C::STEPS + s0) * NT + t) * 32 + ln] = e0;
+      xs[((ch * C::STEPS + s0 + 1) * NT + t) * 32 + ln] = e1;
+      (void)PAIRS;
+    }
+  } else {
+    // entry (win, t, lane): 16 bytes = x[8t+g][k0 + 32*win + 2c + 8i + {0,1}], i = 0..3
+    uint4* xs = reinterpret_cast<uint4*>(sm);
+    const int items = NCH * NT * 32;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int ln = it % 32, t = (it / 32) % NT, win = it / 32 / NT;
+      const int gg = ln >> 2, cc = ln & 3;
+      const int64_t n = 8 * t + gg;
+      const int64_t kb = k0 + 32 * win + 2 * cc;
+      uint32_t w4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t k = kb + 8 * i;
+        if (p.x_fmt == X_16 && n < p.M && k + 2 <= p.K)
+          w4[i] = __ldg(reinterpret_cast<const unsigned int*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
+        else
+          w4[i] = xval<T>(p, n, k) | (xval<T>(p, n, k + 1) << 16);
+      }
+      xs[it] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0);
+  if (!ok) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+  const int rg = warp * 16 + g;  // local rows rg, rg + 8
+  const uint8_t* vrow0 = sm + L::OFF_V + rg * C::VP;
+  const uint8_t* vrow1 = vrow0 + 8 * C::VP;
+  const int nch = (int)((kv + C::CHUNK - 1) / C::CHUNK);
+
+  if (ok) {
+    if constexpr (!sparse_fmt<WF>()) {
+      const uint2* xs = reinterpret_cast<const uint2*>(sm);
+#pragma unroll 2
+      for (int ch = 0; ch < nch; ++ch) {
+        const uint4 r0 = *reinterpret_cast<const uint4*>(vrow0 + ch * 64 + 16 * c);
+        const uint4 r1 = *reinterpret_cast<const uint4*>(vrow1 + ch * 64 + 16 * c);
+        uint32_t sc[2][2];
+        if (WF == W_DQ4) {
+          const uint32_t s0 = *reinterpret_cast<const uint16_t*>(sm + L::OFF_S + rg * C::SP + ch * 8 + 2 * c);
+          const uint32_t s1 = *reinterpret_cast<const uint16_t*>(sm + L::OFF_S + (rg + 8) * C::SP + ch * 8 + 2 * c);
+          scale_pair<T>(s0, sc[0][0], sc[0][1]);
+          scale_pair<T>(s1, sc[1][0], sc[1][1]);
+        }
+        const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+        for (int s = 0; s < C::STEPS; ++s) {
+          uint32_t a0, a1, a2, a3;
+          if (WF == W_D16) {
+            a0 = w0[2 * s];
+            a2 = w0[2 * s + 1];
+            a1 = w1[2 * s];
+            a3 = w1[2 * s + 1];
+          } else {
+            const int q = s >> 1, i0 = 2 * (s & 1), hb = s >> 2;
+            a0 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0), sc[0][hb]);
+            a2 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0 + 1), sc[0][hb]);
+            a1 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0), sc[1][hb]);
+            a3 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0 + 1), sc[1][hb]);
+          }
+#pragma unroll
+          for (int t = 0; t < NT; ++t) mma_k16<T>(acc[t], a0, a1, a2, a3, xs[((ch * C::STEPS + s) * NT + t) * 32 + lane]);
+        }
+      }
+    } else {
+      const uint4* xs = reinterpret_cast<const uint4*>(sm);
+      const uint8_t* mrow0 = sm + L::OFF_M + rg * C::MP;
+      const uint8_t* mrow1 = mrow0 + 8 * C::MP;
+#pragma unroll 4
+      for (int win = 0; win < nch; ++win) {
+        // metadata: word `win` of each row's nibble stream; lanes c = 0 / 1 pass the low / high
+        // halves (groups 0-3 / 4-7) of rows g | g+8
+        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(mrow0 + 4 * win);
+        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(mrow1 + 4 * win);
+        const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
+        uint32_t a0, a1, a2, a3;
+        if (WF == W_S16) {  // kept pair of group c / c+4: 4-byte words 8*win + c (+4)
+          a0 = *reinterpret_cast<const uint32_t*>(vrow0 + 32 * win + 4 * c);
+          a2 = *reinterpret_cast<const uint32_t*>(vrow0 + 32 * win + 4 * c + 16);
+          a1 = *reinterpret_cast<const uint32_t*>(vrow1 + 32 * win + 4 * c);
+          a3 = *reinterpret_cast<const uint32_t*>(vrow1 + 32 * win + 4 * c + 16);
+        } else {  // codes: bytes 8*win + c (+4); one block scale per window
+          const uint2 v0 = *reinterpret_cast<const uint2*>(vrow0 + 8 * win);
+          const uint2 v1 = *reinterpret_cast<const uint2*>(vrow1 + 8 * win);
+          uint32_t s0, s1, unused;
+          scale_pair<T>(sm[L::OFF_S + rg * C::SP + win], s0, unused);
+          scale_pair<T>(sm[L::OFF_S + (rg + 8) * C::SP + win], s1, unused);
+          const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));  // bytes c, c+4 -> [0], [1]
+          const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
+          a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+          a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+          a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+          a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) mma_sp_k32<T>(acc[t], a0, a1, a2, a3, xs[(win * NT + t) * 32 + lane], e);
+      }
+    }
+  }
+
+  // ---- 4. epilogue: rows row0 + rg (+8), tokens 8t + 2c (+1)
+  float scale = 1.0f;
+  if (WF == W_DQ4 || WF == W_SQ4) scale = 256.0f * *p.w_ts;
+  if (p.x_fmt == X_Q4) scale *= *p.x_ts;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t n = 8 * t + 2 * c + (q & 1);
+      const int64_t r = row0 + rg + ((q & 2) ? 8 : 0);
+      if (n < p.M && r < p.N) {
+        float* dst = p.y + n * p.N + r;
+        const float v = acc[t][q] * scale;
+        if (p.accumulate) atomicAdd(dst, v);
+        else *dst = v;
+      }
+    }
+  }
+}
+
+template <int WF, typename T>
+int launch2(const SkinnyParams& p, int nt, cudaStream_t s) {
+  using C = F2<WF>;
+  dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)((p.K + C::KC - 1) / C::KC));
+#define SP24_L2(NTV)                                                                                        \
+  {                                                                                                         \
+    auto kern = skinny2_kernel<WF, T, NTV>;                                                                 \
+    constexpr int smem = Smem2<WF, NTV>::TOTAL;                                                             \
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+      return SP24_ERR_CUDA;                                                                                 \
+    kern<<<grid, kWarps * 32, smem, s>>>(p);                                                                \
+  }
+  switch (nt) {
+    case 1: SP24_L2(1) break;
+    case 2: SP24_L2(2) break;
+    case 4: SP24_L2(4) break;
+    case 8: SP24_L2(8) break;
+    default: return SP24_ERR_UNSUPPORTED;
+  }
+#undef SP24_L2
+  return launch_status();
+}
+
+}  // namespace
+
+// True when the shared-memory staged skinny kernel can take this problem: every row slice of
+// every array starts 16-byte aligned and has a 16-byte multiple length.
+bool skinny2_supported(int wf, const SkinnyParams& p) {
+  if (p.M > 64 || p.K == 0) return false;
+  if (!aligned(p.w, 16)) return false;
+  switch (wf) {
+    case W_D16: return p.K % 8 == 0;
+    case W_DQ4: return p.K % 256 == 0 && aligned(p.w_scales, 16);
+    case W_S16: return p.K % 128 == 0 && aligned(p.meta, 16);
+    case W_SQ4: return p.K % 512 == 0 && aligned(p.w_scales, 16) && aligned(p.meta, 16);
+  }
+  return false;
+}
+
+int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s) {
+  const int kc = wf == W_D16 ? F2<W_D16>::KC : wf == W_DQ4 ? F2<W_DQ4>::KC : wf == W_S16 ? F2<W_S16>::KC : F2<W_SQ4>::KC;
+  const int64_t slices = (p.K + kc - 1) / kc;
+  p.accumulate = slices > 1;
+  if (p.accumulate && cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  const int nt = p.M <= 8 ? 1 : p.M <= 16 ? 2 : p.M <= 32 ? 4 : 8;
+  const bool bf = t16 == SP24_BF16;
+  switch (wf) {
+    case W_D16: return bf ? launch2<W_D16, __nv_bfloat16>(p, nt, s) : launch2<W_D16, __half>(p, nt, s);
+    case W_DQ4: return bf ? launch2<W_DQ4, __nv_bfloat16>(p, nt, s) : launch2<W_DQ4, __half>(p, nt, s);
+    case W_S16: return bf ? launch2<W_S16, __nv_bfloat16>(p, nt, s) : launch2<W_S16, __half>(p, nt, s);
+    case W_SQ4: return bf ? launch2<W_SQ4, __nv_bfloat16>(p, nt, s) : launch2<W_SQ4, __half>(p, nt, s);
+  }
+  return SP24_ERR_UNSUPPORTED;
+}
+
+}  // namespace sp24

@@ -115,3 +115,68 @@ def test_k_zero_writes_zeros():
     y = torch.full((4, 8), 7.0, device="cuda")
     sp.gemm_dense(x, w, out=y)
     assert not y.any()
+
+
+ALGO_SHAPES = [(16, 256, 512), (130, 200, 640), (512, 384, 1024)]
+
+
+@pytest.mark.parametrize("algo", [sp.ALGO_SKINNY, sp.ALGO_TILED], ids=["skinny", "tiled"])
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+@pytest.mark.parametrize("fmt", FORMATS, ids=lambda f: f"x{f[0]}-w{f[1]}")
+@pytest.mark.parametrize("shape", ALGO_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_gemm_both_kernels(fmt, shape, sparse, algo):
+    """The skinny (warp-MMA) and the tiled (tcgen05) kernels on the same problems, with token
+    and weight-row tails that do not fill a tile."""
+    xfmt, wfmt = fmt
+    M, N, K = shape
+    X, xs, W, ws = make_case(xfmt, wfmt, M, N, K, seed=M * 7 + N * 3 + K)
+    Y, S = oracle_side(X, xs, xfmt, W, ws, wfmt, sparse)
+    y = gpu_side(X, xs, xfmt, W, ws, wfmt, sparse, algo=algo)
+    assert_gemm_close(y, Y, S, REL)
+    assert sp.last_device_error() == sp.OK
+
+
+def _sampled(xfmt, wfmt, sparse, M, N, K, rows, seed=0, w_sigma=1.0):
+    X, xs, W, ws = make_case(xfmt, wfmt, M, N, K, seed=seed, w_sigma=w_sigma)
+    y = gpu_side(X, xs, xfmt, W, ws, wfmt, sparse)
+    torch.cuda.synchronize()
+    # the oracle on a seeded subset of output rows (x quantisation is per tensor, so NVFP4 x is
+    # encoded whole and the sampled rows decoded from it)
+    if xfmt == "nvfp4":
+        c, s, ts = oracle.nvfp4_encode(X, ORACLE_DT[xs])
+        Xd = oracle.nvfp4_decode(c[rows], s[rows], ts)
+    else:
+        Xd = oracle.to_double(np.ascontiguousarray(X[rows]), ORACLE_DT[xs])
+    od = ORACLE_DT[ws]
+    if sparse:
+        V, meta = oracle.compress_24(W, od)
+        if wfmt == "nvfp4":
+            c, s, ts = oracle.nvfp4_encode(V, od)
+            Vd = oracle.nvfp4_decode(c, s, ts)
+        else:
+            Vd = oracle.to_double(V, od)
+        Y, S = oracle.gemm_sparse(Xd, Vd, meta)
+    else:
+        if wfmt == "nvfp4":
+            c, s, ts = oracle.nvfp4_encode(W, od)
+            Wd = oracle.nvfp4_decode(c, s, ts)
+        else:
+            Wd = oracle.to_double(W, od)
+        Y, S = oracle.gemm(Xd, Wd)
+    assert_gemm_close(y[torch.as_tensor(rows, device=y.device)], Y, S)
+
+
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+def test_prefill_w4a4_4096_sampled(sparse):
+    """NVFP4 x and w at M = N = K = 4096 (the prefill shape), 24 sampled token rows x all 4096
+    outputs checked against the oracle."""
+    rows = np.sort(synth.rng(77).choice(4096, 24, replace=False))
+    _sampled("nvfp4", "nvfp4", sparse, 4096, 4096, 4096, rows)
+
+
+@pytest.mark.parametrize("M", [1024, 16384])
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+def test_fp16_msweep_sampled(M, sparse):
+    """FP16 W [5120, 5120] and X [M, 5120] of the M sweep, sampled token rows."""
+    rows = np.sort(synth.rng(M).choice(M, 8, replace=False))
+    _sampled("f16", "f16", sparse, M, 5120, 5120, rows, seed=5)
