@@ -33,7 +33,7 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_prune_compress_24", "sp24_decompress_24", "sp24_quantize_nvfp4_workspace_size",
            "sp24_quantize_nvfp4", "sp24_dequantize_nvfp4", "sp24_gemm_workspace_size",
            "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
-           "sp24_last_device_error")
+           "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
             L.sp24_quantize_nvfp4_workspace_size.argtypes = [I64, I64, P]
             L.sp24_quantize_nvfp4.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, P]
             L.sp24_dequantize_nvfp4.argtypes = [P, P, P, I64, I64, I, P, P]
+            L.sp24_quantize_nvfp4_noalloc.argtypes = [P, I, I64, I64, P, P, P, P, P]
             L.sp24_gemm_workspace_size.argtypes = [I, I, I, I64, I64, I64, I, P]
             L.sp24_gemm_dense.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand), I64,
                                           I64, I64, P, P, I64, I, P]
@@ -232,6 +233,24 @@ def quantize_nvfp4(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None,
     _call("sp24_quantize_nvfp4", _ptr(t), _dtype_code(t), R, L, _ptr(tensor_scale),
           _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), _ptr(workspace),
           0 if workspace is None else workspace.numel(), _stream(stream))
+    return out
+
+
+def quantize_nvfp4_noalloc(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None, out=None,
+                           stream=None) -> NVFP4Tensor:
+    """quantize_nvfp4 without a workspace: the library's own per-device scratch is used, so the
+    call needs no device allocation (for callers that cannot allocate, e.g. during graph
+    capture).  Calls whose GPU work overlaps race on that scratch."""
+    _cuda(t, "t")
+    if t.dim() != 2:
+        raise ValueError("quantize_nvfp4_noalloc wants a 2-D tensor")
+    R, L = t.shape
+    if out is None:
+        out = NVFP4Tensor(torch.empty((R, L // 2), dtype=torch.uint8, device=t.device),
+                          torch.empty((R, L // 16), dtype=torch.uint8, device=t.device),
+                          torch.empty(1, dtype=torch.float32, device=t.device))
+    _call("sp24_quantize_nvfp4_noalloc", _ptr(t), _dtype_code(t), R, L, _ptr(tensor_scale),
+          _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), _stream(stream))
     return out
 
 

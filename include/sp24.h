@@ -147,6 +147,22 @@ int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
                         float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
                         void* stream);
 
+/* The same quantisation for callers that cannot allocate device memory (code running inside a
+ * CUDA graph capture where cudaMalloc is not allowed, runtimes that only hand out fixed operand
+ * buffers, plugins that must not touch the allocator).  No counterpart on the source pages: it
+ * is a property of this library, not of the method.
+ *   Arguments as sp24_quantize_nvfp4, without the workspace.  The scratch is a 256-byte
+ *   __device__ array inside the library, one per device, kept until the process exits; the
+ *   quantiser needs 4 bytes of it (the amax word) for every tensor shape, and a request needing
+ *   more than 256 bytes returns SP24_ERR_WORKSPACE.  The first call on each device looks up the
+ *   array's device address; make that first call before any stream capture begins.  The call
+ *   allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).  All calls on a
+ *   device share the array: each call clears the amax word first, and calls whose GPU work can
+ *   overlap (different streams without ordering) race on it. */
+int sp24_quantize_nvfp4_noalloc(const void* t, int dtype, int64_t rows, int64_t cols,
+                                const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                float* tensor_scale_out, void* stream);
+
 /* Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
  * (F16/BF16/F32). */
 int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,
