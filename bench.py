@@ -395,6 +395,135 @@ def cpu_baseline(budget_s: float, steps: int = 1):
     return gbs, dt, rows, cores
 
 
+# ------------------------------------------------------------------------------ per-shape sweep
+
+def run_sweep(args) -> None:
+    """One JSON line per (workload, shape, dense|sparse24): GEMM time on prepared operands, with
+    enough rotating weight copies that each launch reads its operands from DRAM."""
+    import torch
+
+    import fp16_gemm_b200 as sp
+    import synth
+
+    torch.cuda.set_device(0)
+    peak_hbm, kind = peaks()
+    peak_bf16 = 1717.8
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak_bf16 = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        kind = "fallback"
+        peak_bf16 = 1590.0
+    # tensor peaks per pipe: measured bf16 dense; FP4 dense = bf16 x 4 (nominal 9 / 2.25 PF);
+    # 2:4 sparse pipes count dense-equivalent FLOPs at twice the dense rate
+    tensor_peak = {"f16": peak_bf16, "f16.sp": 2 * peak_bf16, "nvfp4": 4 * peak_bf16}
+    dev = torch.device("cuda", 0)
+    t16 = lambda a, d: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if d == "bf16"
+                        else torch.from_numpy(a)).to(dev)
+
+    def timeit(fn, reps=20):
+        for _ in range(3):
+            fn(0)
+        torch.cuda.synchronize()
+        times = []
+        for r in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(r)
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(times)
+
+    def clone_op(o):
+        if isinstance(o, torch.Tensor):
+            return o.clone()
+        return type(o)(*[clone_op(t) for t in o])
+
+    def op_bytes(t):
+        if isinstance(t, sp.NVFP4Tensor):
+            return t.codes.numel() + t.scales.numel() + 4
+        if isinstance(t, sp.Sparse24):
+            return op_bytes(t.values) + t.meta.numel()
+        return t.numel() * t.element_size()
+
+    def case(workload, M, N, K, xdt, wdt, X, W):
+        """X, W numpy storage; xdt in {f16,bf16,nvfp4}; wdt in {f16,bf16,nvfp4}."""
+        x = t16(X, "f16" if xdt == "f16" else "bf16")
+        if xdt == "nvfp4":
+            x = sp.quantize_nvfp4(x)
+        w16 = t16(W, "f16" if wdt == "f16" or (wdt == "nvfp4" and xdt == "f16") else "bf16")
+        v, m = sp.prune_compress_24(w16)
+        wd = sp.decompress_24(v, m, w16.shape) if wdt != "nvfp4" else w16  # dense on pruned W
+        dense = sp.quantize_nvfp4(w16) if wdt == "nvfp4" else wd
+        sparse = sp.Sparse24(sp.quantize_nvfp4(v) if wdt == "nvfp4" else v, m)
+        res = {}
+        for name, wop in (("dense", dense), ("sparse24", sparse)):
+            wb = op_bytes(wop)
+            copies = max(1, min(8, int(256e6 // max(wb, 1))))
+            wops = [wop] + [clone_op(wop) for _ in range(copies - 1)]
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            if name == "dense":
+                ws_b = sp.gemm_workspace_bytes(x, wop, False, M, N, K)
+                ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev)
+                fn = lambda r: sp.gemm_dense(x, wops[r % copies], out=y, workspace=ws if ws_b else None)
+            else:
+                ws_b = sp.gemm_workspace_bytes(x, wop, True, M, N, K)
+                ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev)
+                fn = lambda r: sp.gemm_sparse24(x, wops[r % copies], K, out=y, workspace=ws if ws_b else None)
+            us = timeit(fn)
+            byts = op_bytes(x) + wb + M * N * 4
+            flops = 2.0 * M * N * K
+            ai = flops / byts
+            pipe = ("nvfp4" if xdt == "nvfp4" and wdt == "nvfp4" and name == "dense" else
+                    "f16.sp" if name == "sparse24" else "f16")
+            ridge = tensor_peak[pipe] * 1e12 / (peak_hbm * 1e9)
+            tflops = flops / (us * 1e-6) / 1e12
+            gbs = byts / (us * 1e-6) / 1e9
+            bound = "hbm" if ai < ridge else "tensor"
+            frac = gbs / peak_hbm if bound == "hbm" else tflops / tensor_peak[pipe]
+            res[name] = {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(gbs, 1),
+                         "bytes": byts, "AI": round(ai, 1), "bound": bound, "pipe": pipe,
+                         "frac": round(frac, 3)}
+        line = {"sweep": workload, "M": M, "N": N, "K": K, "x": xdt, "w": wdt, **res,
+                "sparse_dense_speedup": round(res["dense"]["us"] / res["sparse24"]["us"], 3),
+                "peaks": {"hbm_gbs": peak_hbm, "tensor_tflops": tensor_peak, "kind": kind}}
+        print(json.dumps(line), flush=True)
+
+    d = synth.fp16_toy()
+    case("fp16_toy", 16, 256, 512, "f16", "f16", d["X"], d["W"])
+    d = synth.decode_nvfp4()
+    case("decode_w4a16", 8, 5120, 5120, "bf16", "nvfp4", d["X"], d["W"])
+    d = synth.prefill_w4a4()
+    case("prefill_w4a4", 4096, 4096, 4096, "nvfp4", "nvfp4", d["X"], d["W"])
+    g = synth.rng(0)
+    W16 = synth.draw(g, (5120, 5120), "f16")
+    Wb = synth.draw(synth.rng(0), (5120, 5120), "bf16")
+    for Mv in (1, 16, 128, 1024, 4096, 16384):
+        X16 = synth.draw(synth.rng(Mv), (Mv, 5120), "f16")
+        case("msweep_fp16", Mv, 5120, 5120, "f16", "f16", X16, W16)
+        Xb = synth.draw(synth.rng(Mv), (Mv, 5120), "bf16")
+        case("msweep_nvfp4_w4a16", Mv, 5120, 5120, "bf16", "nvfp4", Xb, Wb)
+        case("msweep_nvfp4_w4a4", Mv, 5120, 5120, "nvfp4", "nvfp4", Xb, Wb)
+    # conv eligibility check + compression (fp16 [256, 256, 3, 3], 5% failing groups), one
+    # tensor and a batch of 512 such tensors as one [512*256, 256, 3, 3] launch
+    c = synth.conv_fail5()
+    for batch in (1, 512):
+        wc = t16(np.ascontiguousarray(np.broadcast_to(c["W"], (batch,) + c["W"].shape)).reshape(
+            (batch * 256, 256, 3, 3)), "f16")
+        pass_ = torch.empty((batch * 256, 64, 3, 3), dtype=torch.uint8, device=dev)
+        nf = torch.empty(1, dtype=torch.int32, device=dev)
+        vals = torch.empty((batch * 256, 128, 3, 3), dtype=torch.float16, device=dev)
+        meta = torch.empty(batch * 256 * 64 * 9 // 2, dtype=torch.uint8, device=dev)
+        us_c = timeit(lambda r: sp.check_24(wc, sp.OP_CONV, pass_out=pass_, n_fail_out=nf))
+        us_p = timeit(lambda r: sp.prune_compress_24(wc, sp.OP_CONV, values_out=vals, meta_out=meta))
+        nb = wc.numel() * 2
+        print(json.dumps({"sweep": "conv_check_compress", "tensors": batch, "shape": [batch * 256, 256, 3, 3],
+                          "check": {"us": round(us_c, 3), "GB/s": round((nb + pass_.numel()) / us_c / 1e3, 1)},
+                          "compress": {"us": round(us_p, 3), "GB/s": round((nb + vals.numel() * 2 + meta.numel()) / us_p / 1e3, 1)},
+                          "n_fail": int(nf.item())}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,7 +534,11 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -64,23 +64,51 @@ int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
 
 int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
 
-// Workspace of the tiled path: 16-bit copies of the operands that are not 16-bit already.
+// True when a 2:4 weight takes the native sparse tensor-core kernel (16-byte nibble rows).
+bool native_sparse(int wf, int64_t K) { return (wf == W_S16 || wf == W_SQ4) && K % 128 == 0; }
+
+// True when NVFP4 x times NVFP4 w takes the native block-scaled FP4 kernel (256-wide K stages,
+// 16-byte aligned scale rows).
+bool native_nvfp4(int x_fmt, int wf, const SkinnyParams& p) {
+  return x_fmt == X_Q4 && wf == W_DQ4 && p.K % 256 == 0 && aligned(p.x, 16) && aligned(p.w, 16) &&
+         aligned(p.x_scales, 16) && aligned(p.w_scales, 16);
+}
+
+// Workspace of the tiled path: 16-bit copies of the operands that are not 16-bit already
+// (NVFP4 2:4 values decoded to 16 bits for the native sparse kernel; otherwise the weight
+// expanded to a dense 16-bit matrix).
 int64_t tiled_workspace(int x_fmt, int wf, int64_t M, int64_t N, int64_t K) {
+  if (x_fmt == X_Q4 && wf == W_DQ4 && K % 256 == 0) return 0;  // native NVFP4 kernel
   int64_t b = 0;
-  if (wf != W_D16) b += round256(N * K * 2);
+  if (native_sparse(wf, K)) {
+    if (wf == W_SQ4) b += round256(N * K);  // N x K/2 values of 2 bytes
+  } else if (wf != W_D16) {
+    b += round256(N * K * 2);
+  }
   if (x_fmt == X_Q4) b += round256(M * K * 2);
   return b;
 }
 
-// Tiled (tcgen05) path: expand what is not plain 16-bit into the workspace, then one GEMM.
+// Tiled (tcgen05) path: decode what is not plain 16-bit into the workspace, then one GEMM.
 int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes, cudaStream_t s) {
+  // NVFP4 x with NVFP4 w: both stay 4-bit, the tensor core applies the block scales
+  if (native_nvfp4(p.x_fmt, wf, p))
+    return tc_gemm_nvfp4(reinterpret_cast<const uint8_t*>(p.x), p.x_scales, p.x_ts, p.w, p.w_scales, p.w_ts,
+                         p.M, p.N, p.K, p.y, s);
   const int64_t need = tiled_workspace(p.x_fmt, wf, p.M, p.N, p.K);
   if (need > 0 && (!ws || ws_bytes < need)) return SP24_ERR_WORKSPACE;
   if (need > 0 && !aligned(ws, 256)) return SP24_ERR_ALIGN;
   const bool bf = t16 == SP24_BF16;
+  const bool sp_native = native_sparse(wf, p.K);
   uint8_t* cur = reinterpret_cast<uint8_t*>(ws);
   const void* w16 = p.w;
-  if (wf != W_D16) {
+  if (sp_native && wf == W_SQ4) {
+    // kept values only: [N, K/2] NVFP4 -> 16-bit E2M1 * E4M3
+    int st = expand_w16(W_DQ4, bf, p.w, p.w_scales, nullptr, p.N, p.K / 2, reinterpret_cast<uint16_t*>(cur), s);
+    if (st) return st;
+    w16 = cur;
+    cur += round256(p.N * p.K);
+  } else if (!sp_native && wf != W_D16) {
     int st = expand_w16(wf, bf, p.w, p.w_scales, p.meta, p.N, p.K, reinterpret_cast<uint16_t*>(cur), s);
     if (st) return st;
     w16 = cur;
@@ -95,6 +123,7 @@ int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes
   }
   const float* sa = (wf == W_DQ4 || wf == W_SQ4) ? p.w_ts : nullptr;
   const float* sb = p.x_fmt == X_Q4 ? p.x_ts : nullptr;
+  if (sp_native) return tc_gemm_f16_sparse(x16, w16, p.meta, p.M, p.N, p.K, bf, p.y, sa, sb, s);
   return tc_gemm_f16(x16, w16, p.M, p.N, p.K, bf, p.y, sa, sb, s);
 }
 

@@ -48,6 +48,29 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t ro
   return r == CUDA_SUCCESS ? SP24_OK : SP24_ERR_CUDA;
 }
 
+// Byte tensor [rows, cols] with row pitch `pitch_bytes`, box (box_cols x box_rows), no swizzle.
+int make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                       uint32_t box_cols, uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return SP24_ERR_CUDA;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (!aligned(base, 16) || pitch_bytes % 16) return SP24_ERR_ALIGN;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SP24_OK : SP24_ERR_CUDA;
+}
+
 namespace {
 
 using namespace tc;
@@ -188,6 +211,359 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, c
   return launch_status();
 }
 
+// ------------------------------------------------------------------ 2:4 sparse tcgen05 GEMM
+//
+// [P2] "The mechanism needs both values and their positions": the kept values are the A operand
+// (128 rows x 64 stored values = 128 logical K per stage) and the positions travel as metadata
+// in TMEM.  Per stage the producer also loads the 16 nibble-stream bytes of each of the 128
+// rows; warp 6 rewrites them into the tcgen05 metadata layout (TMEM lane l holds, for rows
+// m = 16*(l/16) + l%8 and m + 8, the nibbles of groups 4*((l/8)%2) .. +3 of each 32-wide K
+// window, one 32-bit column per window: the low half for row m, the high half for row m + 8),
+// the MMA thread moves that 2 KB tile into 4 TMEM columns with tcgen05.cp and issues four
+// tcgen05.mma.sp (K = 32 logical each) on it.
+constexpr int kSpBN = 128, kSpStages = 4;
+constexpr uint32_t kSpA = kBM * 128;           // 128 rows x 64 stored 16-bit values
+constexpr uint32_t kSpB = kSpBN * 128;         // one 64-wide K half of B (two per stage)
+constexpr uint32_t kSpM = kBM * 16;            // raw nibble rows (16 B each)
+constexpr uint32_t kSpStage = kSpA + 2 * kSpB + 2 * kSpM;
+constexpr size_t kSpSmem = (size_t)kSpStages * kSpStage + 1024;
+constexpr int kSpCols = 256;                   // TMEM: 128 accumulator + 16 metadata columns
+
+template <bool BF16>
+__global__ void __launch_bounds__(224, 1)
+    gemm_f16sp_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmE, const TcParams p) {
+  constexpr int S = kSpStages, BN = kSpBN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // stage s: [A 16 KB][B0 16 KB][B1 16 KB][raw nibbles 2 KB][tcgen05 metadata 2 KB]
+  auto sA = [&](int s) { return smem + s * kSpStage; };
+  auto sB = [&](int s, int h) { return smem + s * kSpStage + kSpA + h * kSpB; };
+  auto sMr = [&](int s) { return smem + s * kSpStage + kSpA + 2 * kSpB; };
+  auto sMe = [&](int s) { return smem + s * kSpStage + kSpA + 2 * kSpB + kSpM; };
+  __shared__ uint64_t full_bar[S], meta_bar[S], empty_bar[S], tfull_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int aborted;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int n0 = blockIdx.y * BN;
+  const int KB = (p.K + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&meta_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&tfull_bar, 1);
+    aborted = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmE);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base, kSpCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], kSpA + 2 * kSpB + kSpM);
+        tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 64, m0);        // stored values
+        tma_load_2d(sB(s, 0), &tmB, &full_bar[s], kb * 128, n0);     // logical K [0, 64)
+        tma_load_2d(sB(s, 1), &tmB, &full_bar[s], kb * 128 + 64, n0);
+        tma_load_2d(sMr(s), &tmE, &full_bar[s], kb * 16, m0);        // 16 nibble bytes per row
+        ++issued;
+      }
+      for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
+        mbar_wait(&full_bar[kb % S], (kb / S) & 1);
+    }
+  } else if (warp == 6) {
+    // metadata rewrite: lane handles TMEM lanes l = lane + 32 i
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (kb / S) & 1;
+      if (!mbar_wait(&full_bar[s], ph) || *(volatile int*)&aborted) {
+        aborted = 1;
+        break;
+      }
+      const uint8_t* raw = sMr(s);
+      uint8_t* out = sMe(s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int l = lane + 32 * i;
+        const int m = 16 * (l / 16) + (l % 8), half = (l / 8) % 2;
+        const uint4 lo = *reinterpret_cast<const uint4*>(raw + 16 * m);        // row m, 16 bytes
+        const uint4 hi = *reinterpret_cast<const uint4*>(raw + 16 * (m + 8));  // row m + 8
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)  // window t: bytes 4t + 2*half (+1) of each row
+          o[t] = __byte_perm(wl[t], wh[t], half ? 0x7632 : 0x5410);
+        *reinterpret_cast<uint4*>(out + 16 * l) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&meta_bar[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(kBM, BN, BF16, true);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&full_bar[s], ph) || !mbar_wait(&meta_bar[s], ph) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ecol = tmem + BN + 4 * s;
+        tmem_cp_128x128b(ecol, desc_rows16_noswizzle(smem_u32(sMe(s))));
+        const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {  // K window t: A + 32 B, B half t/2 + 64 B * (t%2)
+          const uint64_t b = desc_kmajor_sw128(smem_u32(sB(s, t >> 1))) + 4 * (t & 1);
+          umma_f16_sp(tmem, a0 + 2 * t, b, ecol + t, idesc, (kb | t) != 0);
+        }
+        umma_commit(&empty_bar[s]);
+      }
+      umma_commit(&tfull_bar);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = m0 + 32 * q + lane;
+    if (!mbar_wait(&tfull_bar, 0)) {
+      aborted = 1;
+    } else {
+      tc_fence_after();
+      float scale = 1.0f;
+      if (p.scale_a) scale *= *p.scale_a;
+      if (p.scale_b) scale *= *p.scale_b;
+#pragma unroll 1
+      for (int j = 0; j < BN / 32; ++j) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * j, v);
+        if (row < p.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = n0 + 32 * j + i;
+            if (tok < p.M) p.y[(int64_t)tok * p.N + row] = v[i] * scale;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && aborted) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kSpCols);
+  }
+}
+
+// ------------------------------------------------------------------ W4A4: native NVFP4 GEMM
+//
+// [P1] "NVFP4 vs 2:4 sparse", "The ladder, top to bottom": the measured dense NVFP4 GEMM at 4096
+// cubed is the pages' kernel ceiling.  Here both operands stay packed E2M1 in shared memory
+// (TMA, 128-byte swizzle: 256 K per row) and the tensor core applies the E4M3 block scales from
+// TMEM (tcgen05.mma kind::mxf4nvf4.block_scale.block16, K = 64 per instruction).  Per stage
+// (256 K) the producer also loads each row's 16 scale bytes; warp 6 rewrites them into 128-row x
+// 4-scale tiles (row r at byte 16*(r%32) + 4*(r/32)), one tile per MMA and per 128 rows, which
+// the MMA thread copies into TMEM with tcgen05.cp.32x128b.warpx4 (lanes 0-31, repeated in every
+// lane quarter).  The tensor scales s_w * s_x multiply the accumulator in the epilogue.
+constexpr int kQStages = 3;
+
+template <int BN>
+struct QCfg {
+  static constexpr uint32_t A = kBM * 128;        // 128 rows x 256 FP4
+  static constexpr uint32_t B = BN * 128;
+  static constexpr uint32_t SFA = kBM * 16;       // raw scale rows (16 per 256 K)
+  static constexpr uint32_t SFB = BN * 16;
+  static constexpr uint32_t STAGE = A + B + 2 * SFA + 2 * SFB;
+  static constexpr size_t SMEM = (size_t)kQStages * STAGE + 1024;
+  static constexpr int SFA_COLS = 16;             // 4 MMAs x 4 columns
+  static constexpr int SFB_COLS = 4 * (BN / 32);  // 4 MMAs x BN/32 columns
+  static constexpr int COLS = BN + kQStages * (SFA_COLS + SFB_COLS) <= 256 ? 256 : 512;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(224, 1)
+    gemm_nvfp4_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                         const TcParams p) {
+  using C = QCfg<BN>;
+  constexpr int S = kQStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  auto sA = [&](int s) { return smem + s * C::STAGE; };
+  auto sB = [&](int s) { return smem + s * C::STAGE + C::A; };
+  auto sSAr = [&](int s) { return smem + s * C::STAGE + C::A + C::B; };
+  auto sSAt = [&](int s) { return smem + s * C::STAGE + C::A + C::B + C::SFA; };
+  auto sSBr = [&](int s) { return smem + s * C::STAGE + C::A + C::B + 2 * C::SFA; };
+  auto sSBt = [&](int s) { return smem + s * C::STAGE + C::A + C::B + 2 * C::SFA + C::SFB; };
+  __shared__ uint64_t full_bar[S], sf_bar[S], empty_bar[S], tfull_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int aborted;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int n0 = blockIdx.y * BN;
+  const int KB = (p.K + 255) / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&sf_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&tfull_bar, 1);
+    aborted = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSA);
+    prefetch_tmap(&tmSB);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base, C::COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], C::A + C::B + C::SFA + C::SFB);
+        tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 128, m0);   // 128 bytes = 256 codes
+        tma_load_2d(sB(s), &tmB, &full_bar[s], kb * 128, n0);
+        tma_load_2d(sSAr(s), &tmSA, &full_bar[s], kb * 16, m0); // 16 scales per row
+        tma_load_2d(sSBr(s), &tmSB, &full_bar[s], kb * 16, n0);
+        ++issued;
+      }
+      for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
+        mbar_wait(&full_bar[kb % S], (kb / S) & 1);
+    }
+  } else if (warp == 6) {
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (kb / S) & 1;
+      if (!mbar_wait(&full_bar[s], ph) || *(volatile int*)&aborted) {
+        aborted = 1;
+        break;
+      }
+      // tile (j, g) = MMA j, rows 128 g .. 128 g + 127: word of row r at index 4 * (r % 32) + r / 32
+      auto rewrite = [&](const uint8_t* raw, uint8_t* tiles, int groups) {
+        for (int g = 0; g < groups; ++g) {
+          uint4 w[4];
+#pragma unroll
+          for (int rq = 0; rq < 4; ++rq) w[rq] = *reinterpret_cast<const uint4*>(raw + 16 * (128 * g + 32 * rq + lane));
+          const uint32_t col[4][4] = {{w[0].x, w[1].x, w[2].x, w[3].x}, {w[0].y, w[1].y, w[2].y, w[3].y},
+                                      {w[0].z, w[1].z, w[2].z, w[3].z}, {w[0].w, w[1].w, w[2].w, w[3].w}};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(tiles + 512 * (j * groups + g) + 16 * lane) =
+                make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
+        }
+      };
+      rewrite(sSAr(s), sSAt(s), 1);
+      rewrite(sSBr(s), sSBt(s), BN / 128);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sf_bar[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_nvfp4(kBM, BN);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&full_bar[s], ph) || !mbar_wait(&sf_bar[s], ph) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sfa0 = tmem + BN + s * (C::SFA_COLS + C::SFB_COLS);
+        const uint32_t sfb0 = sfa0 + C::SFA_COLS;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSAt(s) + 512 * j)));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+            tmem_cp_32x128b_x4(sfb0 + (BN / 32) * j + 4 * g,
+                               desc_rows16_noswizzle(smem_u32(sSBt(s) + 512 * (j * (BN / 128) + g))));
+        }
+        const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
+        const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB(s)));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)  // K = 64 codes = 32 bytes = 2 descriptor units
+          umma_nvfp4(tmem, a0 + 2 * j, b0 + 2 * j, idesc, sfa0 + 4 * j, sfb0 + (BN / 32) * j, (kb | j) != 0);
+        umma_commit(&empty_bar[s]);
+      }
+      umma_commit(&tfull_bar);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = m0 + 32 * q + lane;
+    if (!mbar_wait(&tfull_bar, 0)) {
+      aborted = 1;
+    } else {
+      tc_fence_after();
+      float scale = 1.0f;
+      if (p.scale_a) scale *= *p.scale_a;
+      if (p.scale_b) scale *= *p.scale_b;
+#pragma unroll 1
+      for (int j = 0; j < BN / 32; ++j) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * j, v);
+        if (row < p.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = n0 + 32 * j + i;
+            if (tok < p.M) p.y[(int64_t)tok * p.N + row] = v[i] * scale;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && aborted) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::COLS);
+  }
+}
+
+template <int BN>
+int launch_nvfp4(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa, const CUtensorMap& sb,
+                 const TcParams& p, cudaStream_t s) {
+  auto kern = gemm_nvfp4_tc_kernel<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QCfg<BN>::SMEM) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  dim3 grid((unsigned)((p.N + kBM - 1) / kBM), (unsigned)((p.M + BN - 1) / BN));
+  kern<<<grid, 224, QCfg<BN>::SMEM, s>>>(a, b, sa, sb, p);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ weight expansion to 16-bit
 
 // Dense NVFP4 ([rows, K/2] codes, [rows, K/16] scales) or 2:4-compressed weights (16-bit values
@@ -242,6 +618,47 @@ __global__ void __launch_bounds__(256) expand_w16_kernel(const uint8_t* __restri
 }
 
 }  // namespace
+
+// Native 2:4 tensor-core GEMM on 16-bit kept values: y = (*sa)(*sb) x w^T with w given by
+// values [N, K/2] and its nibble stream [N, K/8].  Needs K % 128 == 0 (16-byte nibble rows).
+int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, int64_t M, int64_t N,
+                       int64_t K, bool bf16, float* y, const float* scale_a, const float* scale_b,
+                       cudaStream_t s) {
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 128) return SP24_ERR_UNSUPPORTED;
+  CUtensorMap ta, tb, te;
+  int st = make_tmap_2d(&ta, values, 2, N, K / 2, K, 64, kBM);
+  if (st) return st;
+  st = make_tmap_2d(&tb, x, 2, M, K, K * 2, 64, kSpBN);
+  if (st) return st;
+  st = make_tmap_2d_plain(&te, meta, N, K / 8, K / 8, 16, kBM);
+  if (st) return st;
+  TcParams p{(int)M, (int)N, (int)K, y, scale_a, scale_b};
+  auto kern = bf16 ? gemm_f16sp_tc_kernel<true> : gemm_f16sp_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpSmem) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  dim3 grid((unsigned)((N + kBM - 1) / kBM), (unsigned)((M + kSpBN - 1) / kSpBN));
+  kern<<<grid, 224, kSpSmem, s>>>(ta, tb, te, p);
+  return launch_status();
+}
+
+// Native NVFP4 x NVFP4 GEMM: y = s_w s_x sum_k dec(x) dec(w) with both operands packed E2M1 +
+// E4M3 scales per 16 (K % 256 == 0, so every 256-wide stage holds 16 whole scale bytes per row).
+int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* wc, const uint8_t* wsc,
+                  const float* w_ts, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t s) {
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 256) return SP24_ERR_UNSUPPORTED;
+  const int BN = M > 128 ? 256 : 128;
+  CUtensorMap ta, tb, tsa, tsb;
+  int st = make_tmap_2d(&ta, wc, 1, N, K / 2, K / 2, 128, kBM);
+  if (st) return st;
+  st = make_tmap_2d(&tb, xc, 1, M, K / 2, K / 2, 128, BN);
+  if (st) return st;
+  st = make_tmap_2d_plain(&tsa, wsc, N, K / 16, K / 16, 16, kBM);
+  if (st) return st;
+  st = make_tmap_2d_plain(&tsb, xs, M, K / 16, K / 16, 16, BN);
+  if (st) return st;
+  TcParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts};
+  return BN == 256 ? launch_nvfp4<256>(ta, tb, tsa, tsb, p, s) : launch_nvfp4<128>(ta, tb, tsa, tsb, p, s);
+}
 
 // Expands an NVFP4 / 2:4 operand of `rows` rows into 16-bit [rows, K] at `out` (workspace).
 int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta, int64_t rows,

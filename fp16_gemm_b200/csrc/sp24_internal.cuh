@@ -46,6 +46,18 @@ inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintp
 // Number of SMs of the current device (cached per process; B200 has 148).
 int sm_count();
 
+// Grid for a grid-stride kernel: the blocks needed, capped at one full wave (as many blocks as
+// the occupancy calculator says fit on all SMs at once), so no block waits for a second wave.
+template <typename Kern>
+int full_wave_grid(Kern kernel, int threads, int64_t blocks_needed) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = (int64_t)per_sm * sm_count();
+  if (blocks_needed < 1) blocks_needed = 1;
+  return (int)(blocks_needed < cap ? blocks_needed : cap);
+}
+
 // Magnitude bits of a 16- or 32-bit float pattern: monotone in |value| for non-NaN values.
 __device__ __forceinline__ uint32_t mag16(uint32_t h) { return h & 0x7fffu; }
 __device__ __forceinline__ uint32_t mag32(uint32_t f) { return f & 0x7fffffffu; }
@@ -90,6 +102,15 @@ int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 // Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,
                 const float* scale_a, const float* scale_b, cudaStream_t s);
+
+// Native 2:4 tensor-core GEMM (tcgen05.mma.sp) on 16-bit kept values + nibble stream; K % 128.
+int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, int64_t M, int64_t N,
+                       int64_t K, bool bf16, float* y, const float* scale_a, const float* scale_b,
+                       cudaStream_t s);
+
+// Native NVFP4 x NVFP4 tensor-core GEMM (tcgen05 kind::mxf4nvf4, block16 E4M3 scales); K % 256.
+int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* wc, const uint8_t* wsc,
+                  const float* w_ts, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t s);
 
 // Expands an NVFP4 (W_DQ4) or 2:4-compressed (W_S16 / W_SQ4) operand into exact 16-bit values.
 int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta,

@@ -181,12 +181,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const uint8_t* __restr
   }
 }
 
-int grid_for(int64_t items) {
-  int64_t blocks = (items + kThreads - 1) / kThreads;
-  int64_t cap = (int64_t)sm_count() * 8;
-  if (blocks > cap) blocks = cap;
-  return (int)(blocks < 1 ? 1 : blocks);
-}
+int64_t blocks_for(int64_t items) { return (items + kThreads - 1) / kThreads; }
 
 constexpr int64_t kQuantWorkspace = 256;
 
@@ -209,20 +204,19 @@ int quantize_nvfp4_launch(const void* t, int dtype, int64_t rows, int64_t cols,
     if (!amax_word) return SP24_ERR_WORKSPACE;
     if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return SP24_ERR_CUDA;
     if (nblk > 0) {
-      if (dtype == SP24_F32) amax_kernel<SP24_F32><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
-      else if (dtype == SP24_BF16) amax_kernel<SP24_BF16><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
-      else amax_kernel<SP24_F16><<<grid_for(nblk), kThreads, 0, s>>>(t, nblk, amax_word);
+      if (dtype == SP24_F32) amax_kernel<SP24_F32><<<full_wave_grid(amax_kernel<SP24_F32>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
+      else if (dtype == SP24_BF16) amax_kernel<SP24_BF16><<<full_wave_grid(amax_kernel<SP24_BF16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
+      else amax_kernel<SP24_F16><<<full_wave_grid(amax_kernel<SP24_F16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
       ++nl;
     }
   }
   // launched even when nblk == 0 so that tensor_scale_out is written
-  int g = grid_for(nblk > 0 ? nblk : 1);
   if (dtype == SP24_F32)
-    encode_kernel<SP24_F32><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_F32><<<full_wave_grid(encode_kernel<SP24_F32>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   else if (dtype == SP24_BF16)
-    encode_kernel<SP24_BF16><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_BF16><<<full_wave_grid(encode_kernel<SP24_BF16>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   else
-    encode_kernel<SP24_F16><<<g, kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_F16><<<full_wave_grid(encode_kernel<SP24_F16>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   return launch_status(nl);
 }
 
@@ -261,10 +255,10 @@ extern "C" int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales
   if (!codes || !scales || !tensor_scale || !out) return SP24_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   if (out_dtype == SP24_F32)
-    decode_kernel<SP24_F32><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+    decode_kernel<SP24_F32><<<full_wave_grid(decode_kernel<SP24_F32>, kThreads, blocks_for(nbytes)), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
   else if (out_dtype == SP24_BF16)
-    decode_kernel<SP24_BF16><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+    decode_kernel<SP24_BF16><<<full_wave_grid(decode_kernel<SP24_BF16>, kThreads, blocks_for(nbytes)), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
   else
-    decode_kernel<SP24_F16><<<grid_for(nbytes), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
+    decode_kernel<SP24_F16><<<full_wave_grid(decode_kernel<SP24_F16>, kThreads, blocks_for(nbytes)), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);
   return launch_status();
 }

@@ -292,12 +292,7 @@ __global__ void __launch_bounds__(kThreads) decompress24_any(const void* __restr
 
 // ------------------------------------------------------------------ host side
 
-int grid_for(int64_t items) {
-  int64_t blocks = (items + kThreads - 1) / kThreads;
-  int64_t cap = (int64_t)sm_count() * 8;  // grid-stride beyond 8 blocks per SM
-  if (blocks > cap) blocks = cap;
-  return (int)(blocks < 1 ? 1 : blocks);
-}
+int64_t blocks_for(int64_t items) { return (items + kThreads - 1) / kThreads; }
 
 // Validates (op, shape, ndim) and returns the group count and layout.
 int parse_shape(int op, const int64_t* shape, int ndim, int64_t* G, Layout* L) {
@@ -361,18 +356,18 @@ extern "C" int sp24_check_24(const void* w, int dtype, int op, const int64_t* sh
     int64_t nv = G * 4 * eb / 16;  // whole 16-byte vectors
     if (nv > 0) {
       if (eb == 2)
-        check24_vec<2><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+        check24_vec<2><<<full_wave_grid(check24_vec<2>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
       else
-        check24_vec<4><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+        check24_vec<4><<<full_wave_grid(check24_vec<4>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
       ++nl;
       g_done = nv * 16 / (4 * eb);
     }
   }
   if (g_done < G) {
     if (eb == 2)
-      check24_any<2><<<grid_for(G - g_done), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
+      check24_any<2><<<full_wave_grid(check24_any<2>, kThreads, blocks_for(G - g_done)), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
     else
-      check24_any<4><<<grid_for(G - g_done), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
+      check24_any<4><<<full_wave_grid(check24_any<4>, kThreads, blocks_for(G - g_done)), kThreads, 0, s>>>(w, L, g_done, G, pass, n_fail);
     ++nl;
   }
   return launch_status(nl);
@@ -396,9 +391,9 @@ extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const in
     if (eb == 4) nv &= ~int64_t(1);  // whole meta bytes only
     if (nv > 0) {
       if (eb == 2)
-        prune24_vec<2><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+        prune24_vec<2><<<full_wave_grid(prune24_vec<2>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
       else
-        prune24_vec<4><<<grid_for(nv), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+        prune24_vec<4><<<full_wave_grid(prune24_vec<4>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
       ++nl;
       p_done = (nv * 16 / (4 * eb)) / 2;
     }
@@ -406,9 +401,9 @@ extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const in
   if (2 * p_done < G) {
     int64_t rest = (G + 1) / 2 - p_done;
     if (eb == 2)
-      prune24_any<2><<<grid_for(rest), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
+      prune24_any<2><<<full_wave_grid(prune24_any<2>, kThreads, blocks_for(rest)), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
     else
-      prune24_any<4><<<grid_for(rest), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
+      prune24_any<4><<<full_wave_grid(prune24_any<4>, kThreads, blocks_for(rest)), kThreads, 0, s>>>(w, L, p_done, G, values, meta);
     ++nl;
   }
   return launch_status(nl);
@@ -430,16 +425,16 @@ extern "C" int sp24_decompress_24(const void* values, const uint8_t* meta, int d
   if (op == SP24_OP_MATMUL && eb == 2 && aligned(values, 8) && aligned(w_out, 16)) {
     int64_t nv = G / 2;
     if (nv > 0) {
-      decompress24_vec16<<<grid_for(nv), kThreads, 0, s>>>((const uint2*)values, meta, nv, (uint4*)w_out);
+      decompress24_vec16<<<full_wave_grid(decompress24_vec16, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint2*)values, meta, nv, (uint4*)w_out);
       ++nl;
     }
     g_done = 2 * nv;
   }
   if (g_done < G) {
     if (eb == 2)
-      decompress24_any<2><<<grid_for(G - g_done), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
+      decompress24_any<2><<<full_wave_grid(decompress24_any<2>, kThreads, blocks_for(G - g_done)), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
     else
-      decompress24_any<4><<<grid_for(G - g_done), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
+      decompress24_any<4><<<full_wave_grid(decompress24_any<4>, kThreads, blocks_for(G - g_done)), kThreads, 0, s>>>(values, meta, L, g_done, G, w_out);
     ++nl;
   }
   return launch_status(nl);

@@ -93,9 +93,10 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor of kind::f16 with fp32 accumulation, both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16) {
-  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+// Instruction descriptor of kind::f16 with fp32 accumulation, both operands K-major; bit 2
+// marks a sparse (2:4) A operand.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool sparse = false) {
+  return (sparse ? 1u << 2 : 0u) | (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -107,6 +108,63 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Sparse (2:4) MMA, kind::f16: A holds the kept values (M x K/2), metadata in TMEM at `e_tmem`.
+__device__ __forceinline__ void umma_f16_sp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Block-scaled FP4 MMA (kind::mxf4nvf4, one E4M3 scale per 16 K): A and B are packed E2M1 in
+// shared memory, the scale factors of A and B in TMEM at `sfa` / `sfb`.
+__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 scales, K = 64), K-major.
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Copies 32 rows x 128 bits from shared memory into TMEM lanes 0-31 of 4 columns and repeats
+// them in the other three lane quarters (the layout block-scale factors are read from).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Copies 128 TMEM lanes x 128 bits (4 columns) from shared memory described by `sdesc`.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled tile of 16-byte rows stored back to back (8-row core
+// matrices 128 B apart): the source form of tcgen05.cp.128x128b.
+__device__ __forceinline__ uint64_t desc_rows16_noswizzle(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3fffu);
+  d |= static_cast<uint64_t>(2048u >> 4) << 16;  // LBO (one core-matrix column: unused)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // SBO: next 8-row core matrix
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;  // layout type 0: no swizzle
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy (TMA,
+// tcgen05.cp, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far has completed.

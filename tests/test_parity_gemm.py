@@ -117,7 +117,7 @@ def test_k_zero_writes_zeros():
     assert not y.any()
 
 
-ALGO_SHAPES = [(16, 256, 512), (130, 200, 640), (512, 384, 1024)]
+ALGO_SHAPES = [(16, 256, 512), (130, 200, 640), (512, 384, 1024), (200, 136, 192)]
 
 
 @pytest.mark.parametrize("algo", [sp.ALGO_SKINNY, sp.ALGO_TILED], ids=["skinny", "tiled"])
@@ -129,6 +129,8 @@ def test_gemm_both_kernels(fmt, shape, sparse, algo):
     and weight-row tails that do not fill a tile."""
     xfmt, wfmt = fmt
     M, N, K = shape
+    if K % 64 and (wfmt == "nvfp4" or xfmt == "nvfp4"):
+        pytest.skip("NVFP4 2:4 operands need K % 64")
     X, xs, W, ws = make_case(xfmt, wfmt, M, N, K, seed=M * 7 + N * 3 + K)
     Y, S = oracle_side(X, xs, xfmt, W, ws, wfmt, sparse)
     y = gpu_side(X, xs, xfmt, W, ws, wfmt, sparse, algo=algo)
