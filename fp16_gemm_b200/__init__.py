@@ -33,7 +33,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_prune_compress_24", "sp24_decompress_24", "sp24_quantize_nvfp4_workspace_size",
            "sp24_quantize_nvfp4", "sp24_dequantize_nvfp4", "sp24_gemm_workspace_size",
            "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
-           "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc")
+           "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc", "sp24_gemm_grouped_workspace_size",
+           "sp24_gemm_grouped")
 
 _lock = threading.Lock()
 _lib = None
@@ -84,6 +85,9 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P,
                                              I64, I, P]
             L.sp24_last_device_error.argtypes = [P]
+            L.sp24_gemm_grouped_workspace_size.argtypes = [I64, I, I64, P]
+            L.sp24_gemm_grouped.argtypes = [ctypes.POINTER(_Operand), P, I64, I, ctypes.POINTER(_Operand),
+                                             ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -328,6 +332,40 @@ def gemm_sparse24(x, w: Sparse24, K: int, out=None, algo: int = ALGO_AUTO, works
     xo = _operand(x)
     _call("sp24_gemm_sparse24", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out),
           _ptr(workspace), 0 if workspace is None else workspace.numel(), algo, _stream(stream))
+    return out
+
+
+def grouped_workspace_bytes(T: int, topk: int, E: int) -> int:
+    n = ctypes.c_int64(0)
+    _call("sp24_gemm_grouped_workspace_size", T, topk, E, ctypes.byref(n))
+    return n.value
+
+
+def gemm_grouped(x, routing: torch.Tensor, w, E: int, N: int, K: int, out=None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """Routed-expert GEMM: Y[t, s, :] = x[t] @ W[routing[t, s]]^T with the E experts stacked as
+    one [E*N, K] operand (16-bit tensor, NVFP4Tensor, or Sparse24 of those)."""
+    _cuda(routing, "routing")
+    T, topk = routing.shape
+    dev = routing.device
+    if out is None:
+        out = torch.empty((T, topk, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(grouped_workspace_bytes(T, topk, E), dtype=torch.uint8, device=dev)
+    xo = _operand(x)
+    if isinstance(w, Sparse24):
+        v = w.values
+        if isinstance(v, NVFP4Tensor):
+            so = _SparseOperand(NVFP4, v.codes.data_ptr(), v.scales.data_ptr(), v.tensor_scale.data_ptr(),
+                                w.meta.data_ptr())
+        else:
+            so = _SparseOperand(_dtype_code(v), v.data_ptr(), None, None, w.meta.data_ptr())
+        dense_p, sparse_p = None, ctypes.byref(so)
+    else:
+        do = _operand(w)
+        dense_p, sparse_p = ctypes.byref(do), None
+    _call("sp24_gemm_grouped", ctypes.byref(xo), _ptr(routing), T, topk, dense_p, sparse_p, E, N, K,
+          _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
     return out
 
 

@@ -334,7 +334,10 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {  // K window t: A + 32 B, B half t/2 + 64 B * (t%2)
           const uint64_t b = desc_kmajor_sw128(smem_u32(sB(s, t >> 1))) + 4 * (t & 1);
-          umma_f16_sp(tmem, a0 + 2 * t, b, ecol + t, idesc, (kb | t) != 0);
+          // the metadata address must be even: an odd column is named by the even one below
+          // it plus the descriptor's sparse-id2 field
+          const uint32_t e = ecol + t;
+          umma_f16_sp(tmem, a0 + 2 * t, b, e & ~1u, idesc | (e & 1u), (kb | t) != 0);
         }
         umma_commit(&empty_bar[s]);
       }

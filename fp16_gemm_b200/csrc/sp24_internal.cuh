@@ -49,9 +49,9 @@ int sm_count();
 // Grid for a grid-stride kernel: the blocks needed, capped at one full wave (as many blocks as
 // the occupancy calculator says fit on all SMs at once), so no block waits for a second wave.
 template <typename Kern>
-int full_wave_grid(Kern kernel, int threads, int64_t blocks_needed) {
+int full_wave_grid(Kern kernel, int threads, int64_t blocks_needed, size_t dyn_smem = 0) {
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess || per_sm < 1)
     per_sm = 1;
   const int64_t cap = (int64_t)per_sm * sm_count();
   if (blocks_needed < 1) blocks_needed = 1;
@@ -89,6 +89,11 @@ struct SkinnyParams {
   float* y;
   int chunks_total;         // filled by skinny_gemm
   bool accumulate;          // filled by skinny_gemm
+  // grouped (routed-expert) mode: blockIdx.z picks a token tile of one expert
+  const int32_t* perm;      // [T * topk] flat (token * topk + slot) entries grouped by expert
+  const int32_t* tiles;     // [max_tiles][3] = expert, first perm index, token count (<= 64)
+  int topk;
+  int64_t expert_rows;      // weight rows per expert (N)
 };
 
 // Launches the skinny kernel for M <= 64 (wf: W_*, t16: SP24_F16 / SP24_BF16 MMA type).
@@ -98,6 +103,8 @@ int skinny_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 // alignment its bulk copies need.
 bool skinny2_supported(int wf, const SkinnyParams& p);
 int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
+// Grouped variant: one launch over max_tiles token tiles (tile table and perm on the device).
+int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStream_t s);
 
 // Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,

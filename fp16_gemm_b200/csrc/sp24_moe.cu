@@ -1,0 +1,239 @@
+// a7: routed-expert (MoE) grouped GEMM, dense and 2:4 sparse.
+//
+// [P1] "NVFP4 vs 2:4 sparse", "Concurrency, not sparsity, is the lever": tokens are routed top-10
+// to 512 experts and every touched expert's weights are read once per step; section "Where it
+// is supported in software" notes that no 2:4 grouped GEMM existed for such a model.
+//
+// Y[t, s, n] = sum_k x[t, k] W[e, n, k] with e = routing[t, s].  Steps, all on the device:
+//   1. route_count:   histogram of expert ids (atomic adds into counts[E]);
+//   2. route_scan:    one CTA turns counts into offsets (exclusive scan) and a table of token
+//                     tiles (expert, first index, count <= 64);
+//   3. route_scatter: each (t, s) takes a slot of its expert's range (perm = t * topk + s);
+//   4. the staged skinny kernel in grouped mode: grid (64-row weight blocks, K slices, tiles),
+//      each CTA gathering its tile's x rows by index and adding into Y[t, s, :].
+// The order of tokens inside an expert's range depends on atomic arrival, but every output is a
+// complete sum for one (t, s), so the result does not.
+#include "sp24_internal.cuh"
+
+namespace sp24 {
+namespace {
+
+constexpr int kTile = 64;
+
+__global__ void route_count(const int32_t* __restrict__ routing, int64_t n, int64_t E, int32_t* __restrict__ counts) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t e = routing[i];
+    if (e < 0 || e >= E) {
+      set_dev_error(SP24_ERR_INVALID_ARG);
+      continue;
+    }
+    atomicAdd(&counts[e], 1);
+  }
+}
+
+// Single CTA of 1024 threads: block-wide exclusive scans over E experts in chunks of 1024.
+__global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ counts, int64_t E,
+                                                   int32_t* __restrict__ offsets, int32_t* __restrict__ tiles,
+                                                   int64_t max_tiles) {
+  __shared__ int32_t warp_sum[2][32];
+  __shared__ int32_t carry[2];
+  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t base = 0; base < E; base += 1024) {
+    const int64_t e = base + threadIdx.x;
+    const int32_t cnt = e < E ? counts[e] : 0;
+    const int32_t nt = (cnt + kTile - 1) / kTile;
+    // inclusive warp scans of (cnt, nt)
+    int32_t a = cnt, b = nt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t ya = __shfl_up_sync(0xffffffffu, a, d), yb = __shfl_up_sync(0xffffffffu, b, d);
+      if (lane >= d) {
+        a += ya;
+        b += yb;
+      }
+    }
+    if (lane == 31) {
+      warp_sum[0][warp] = a;
+      warp_sum[1][warp] = b;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int32_t wa = warp_sum[0][lane], wb = warp_sum[1][lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t ya = __shfl_up_sync(0xffffffffu, wa, d), yb = __shfl_up_sync(0xffffffffu, wb, d);
+        if (lane >= d) {
+          wa += ya;
+          wb += yb;
+        }
+      }
+      warp_sum[0][lane] = wa;  // inclusive over warps
+      warp_sum[1][lane] = wb;
+    }
+    __syncthreads();
+    const int32_t pre_a = carry[0] + (warp ? warp_sum[0][warp - 1] : 0) + a - cnt;  // exclusive
+    const int32_t pre_b = carry[1] + (warp ? warp_sum[1][warp - 1] : 0) + b - nt;
+    if (e < E) {
+      offsets[e] = pre_a;
+      for (int32_t j = 0; j < nt && pre_b + j < max_tiles; ++j) {
+        int32_t* t = tiles + 3 * (int64_t)(pre_b + j);
+        t[0] = (int32_t)e;
+        t[1] = pre_a + kTile * j;
+        t[2] = cnt - kTile * j < kTile ? cnt - kTile * j : kTile;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) {
+      carry[0] = pre_a + cnt;
+      carry[1] = pre_b + nt;
+    }
+    __syncthreads();
+  }
+  // unused tile slots get count 0 (those CTAs exit at once)
+  for (int64_t i = carry[1] + threadIdx.x; i < max_tiles; i += blockDim.x) tiles[3 * i + 2] = 0;
+}
+
+__global__ void route_scatter(const int32_t* __restrict__ routing, int64_t n, int64_t E,
+                              const int32_t* __restrict__ offsets, int32_t* __restrict__ fill,
+                              int32_t* __restrict__ perm) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t e = routing[i];
+    if (e < 0 || e >= E) continue;
+    perm[offsets[e] + atomicAdd(&fill[e], 1)] = (int32_t)i;
+  }
+}
+
+struct MoeWs {
+  int32_t *counts, *fill, *offsets, *tiles, *perm;
+  int64_t max_tiles, bytes;
+};
+
+MoeWs moe_layout(void* base, int64_t T, int topk, int64_t E) {
+  MoeWs w{};
+  const int64_t n = T * topk;
+  w.max_tiles = (n + kTile - 1) / kTile + E;
+  auto r16 = [](int64_t b) { return (b + 15) / 16 * 16; };
+  int64_t off = 0;
+  uint8_t* p = reinterpret_cast<uint8_t*>(base);
+  w.counts = reinterpret_cast<int32_t*>(p + off);
+  off += r16(4 * E);
+  w.fill = reinterpret_cast<int32_t*>(p + off);
+  off += r16(4 * E);
+  w.offsets = reinterpret_cast<int32_t*>(p + off);
+  off += r16(4 * E);
+  w.tiles = reinterpret_cast<int32_t*>(p + off);
+  off += r16(12 * w.max_tiles);
+  w.perm = reinterpret_cast<int32_t*>(p + off);
+  off += r16(4 * n);
+  w.bytes = off;
+  return w;
+}
+
+bool is16(int f) { return f == SP24_F16 || f == SP24_BF16; }
+
+}  // namespace
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" int sp24_gemm_grouped_workspace_size(int64_t T, int topk, int64_t E, int64_t* bytes) {
+  if (!bytes) return SP24_ERR_INVALID_ARG;
+  if (T < 0 || topk < 0 || E <= 0) return SP24_ERR_SHAPE;
+  *bytes = moe_layout(nullptr, T, topk, E).bytes;
+  return SP24_OK;
+}
+
+extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, int64_t T, int topk,
+                                 const sp24_operand* w_dense, const sp24_sparse_operand* w_sparse, int64_t E,
+                                 int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                                 void* stream) {
+  if (!x || (!w_dense == !w_sparse)) return SP24_ERR_INVALID_ARG;
+  if (T < 0 || topk < 0 || E <= 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
+  if (E > INT32_MAX || T * topk > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  const int64_t n = T * topk;
+  if (n == 0 || N == 0) return SP24_OK;
+  if (!routing || !y) return SP24_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(y, 0, (size_t)(n * N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
+  if (K == 0) return SP24_OK;
+
+  SkinnyParams p{};
+  // activations
+  if (x->format == SP24_NVFP4) {
+    if (K % 32 || !x->data || !x->scales || !x->tensor_scale) return SP24_ERR_INVALID_ARG;
+    p.x_fmt = X_Q4;
+  } else if (is16(x->format)) {
+    if (K % 8 || !x->data) return SP24_ERR_INVALID_ARG;
+    if (!aligned(x->data, 16)) return SP24_ERR_ALIGN;
+    p.x_fmt = X_16;
+  } else {
+    return SP24_ERR_DTYPE;
+  }
+  p.x = x->data;
+  p.x_scales = x->scales;
+  p.x_ts = x->tensor_scale;
+  // expert weights, stacked [E * N, K]
+  int wf, wformat;
+  if (w_dense) {
+    wformat = w_dense->format;
+    if (is16(wformat)) {
+      wf = W_D16;
+      p.w_row_bytes = K * 2;
+    } else if (wformat == SP24_NVFP4) {
+      wf = W_DQ4;
+      p.w_row_bytes = K / 2;
+      p.scale_row_bytes = K / 16;
+      if (!w_dense->scales || !w_dense->tensor_scale) return SP24_ERR_INVALID_ARG;
+    } else {
+      return SP24_ERR_DTYPE;
+    }
+    p.w = reinterpret_cast<const uint8_t*>(w_dense->data);
+    p.w_scales = w_dense->scales;
+    p.w_ts = w_dense->tensor_scale;
+  } else {
+    wformat = w_sparse->format;
+    if (is16(wformat)) {
+      wf = W_S16;
+      p.w_row_bytes = K;
+    } else if (wformat == SP24_NVFP4) {
+      wf = W_SQ4;
+      p.w_row_bytes = K / 4;
+      p.scale_row_bytes = K / 32;
+      if (!w_sparse->scales || !w_sparse->tensor_scale) return SP24_ERR_INVALID_ARG;
+    } else {
+      return SP24_ERR_DTYPE;
+    }
+    p.w = reinterpret_cast<const uint8_t*>(w_sparse->values);
+    p.w_scales = w_sparse->scales;
+    p.w_ts = w_sparse->tensor_scale;
+    p.meta = w_sparse->meta;
+    p.meta_row_bytes = K / 8;
+  }
+  if (!p.w || (w_sparse && !p.meta)) return SP24_ERR_INVALID_ARG;
+  if (is16(x->format) && is16(wformat) && x->format != wformat) return SP24_ERR_DTYPE;
+  const int t16 = is16(x->format) ? x->format : (is16(wformat) ? wformat : SP24_BF16);
+  p.N = N;
+  p.K = K;
+  p.y = y;
+  p.M = kTile;
+  if (!skinny2_supported(wf, p)) return SP24_ERR_UNSUPPORTED;
+
+  MoeWs ws = moe_layout(workspace, T, topk, E);
+  if (!workspace || workspace_bytes < ws.bytes) return SP24_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
+  const size_t zero_bytes = (size_t)(reinterpret_cast<uint8_t*>(ws.offsets) - reinterpret_cast<uint8_t*>(ws.counts));
+  if (cudaMemsetAsync(ws.counts, 0, zero_bytes, s) != cudaSuccess) return SP24_ERR_CUDA;  // counts + fill
+  const int blocks = (int)((n + 255) / 256 < (int64_t)sm_count() * 4 ? (n + 255) / 256 : (int64_t)sm_count() * 4);
+  route_count<<<blocks, 256, 0, s>>>(routing, n, E, ws.counts);
+  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles);
+  route_scatter<<<blocks, 256, 0, s>>>(routing, n, E, ws.offsets, ws.fill, ws.perm);
+  int st = launch_status(3);
+  if (st) return st;
+  p.perm = ws.perm;
+  p.tiles = ws.tiles;
+  p.topk = topk;
+  p.expert_rows = N;
+  return skinny2_grouped(wf, t16, p, ws.max_tiles, s);
+}

@@ -11,6 +11,7 @@
 // explicit __fdiv_rn / __fmul_rn intrinsics so no contraction or approximation can change a
 // rounding; the E4M3 and E2M1 roundings use the hardware's RNE + satfinite conversions.
 #include "sp24_internal.cuh"
+#include "sp24_stream.cuh"
 
 namespace sp24 {
 namespace {
@@ -77,28 +78,68 @@ __device__ __forceinline__ uint32_t e2m1x2_rne_satfinite(float x_lo, float x_hi)
   return r & 0xffu;
 }
 
-// Blocks handled per loop iteration by one thread (their loads are issued together).
-constexpr int kBlocksPerIter = 2;
+// Streaming ring: 4 stages of 16 KB per CTA (512 blocks of 16 16-bit entries, or 256 fp32).
+constexpr int kChunk = 16384, kStages = 4;
+constexpr size_t kRingBytes = (size_t)kChunk * kStages;
+
+// 16 entries of a block from shared memory as fp32.
+template <int DT>
+__device__ __forceinline__ void smem_block(const uint8_t* p, float (&v)[16]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  if (DT == SP24_F32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 x = q[i];
+      v[4 * i + 0] = __uint_as_float(x.x);
+      v[4 * i + 1] = __uint_as_float(x.y);
+      v[4 * i + 2] = __uint_as_float(x.z);
+      v[4 * i + 3] = __uint_as_float(x.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 x = q[i];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[8 * i + 2 * k] = to_f32<DT>(w[k] & 0xffffu);
+        v[8 * i + 2 * k + 1] = to_f32<DT>(w[k] >> 16);
+      }
+    }
+  }
+}
+
+template <int DT>
+constexpr int block_bytes() { return DT == SP24_F32 ? 64 : 32; }
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ t, int64_t nblk,
                                                         unsigned int* __restrict__ amax_bits) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  constexpr int BB = block_bytes<DT>();
   float m = 0.0f;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += kBlocksPerIter * stride) {
-    float v[kBlocksPerIter][16];
+  stream::for_each_chunk<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(t), nblk * BB, ring, [&](const uint8_t* chunk, int64_t, int bytes) {
+        // any 16-byte vector order will do for a max: consecutive threads, consecutive vectors
+        const uint4* cv = reinterpret_cast<const uint4*>(chunk);
+        const int nvec = bytes / 16;
 #pragma unroll
-    for (int u = 0; u < kBlocksPerIter; ++u) {
-      if (b + u * stride < nblk) load_block<DT>(t, b + u * stride, v[u]);
-      else
+        for (int q = 0; q < kChunk / 16 / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          if (j >= nvec) continue;
+          const uint4 x = cv[j];
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[u][i] = 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < kBlocksPerIter; ++u)
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[u][i]));
-  }
+          for (int k = 0; k < 4; ++k) {
+            if (DT == SP24_F32) {
+              m = fmaxf(m, fabsf(__uint_as_float(w[k])));
+            } else {
+              m = fmaxf(m, fabsf(to_f32<DT>(w[k] & 0xffffu)));
+              m = fmaxf(m, fabsf(to_f32<DT>(w[k] >> 16)));
+            }
+          }
+        }
+      });
   unsigned int u = __float_as_uint(m);
   u = __reduce_max_sync(0xffffffffu, u);
   __shared__ unsigned int wmax[kThreads / 32];
@@ -140,20 +181,25 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const void* __restrict
                                                           uint2* __restrict__ codes,
                                                           uint8_t* __restrict__ scales,
                                                           float* __restrict__ ts_out) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  constexpr int BB = block_bytes<DT>();
   // tensor scale: supplied, or amax / 2688 (2688 = 6 * 448)
   const float s_t = ts_in ? *ts_in : __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
   const float d = __fmul_rn(s_t, 6.0f);
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += kBlocksPerIter * stride) {
-    float v[kBlocksPerIter][16];
+  stream::for_each_chunk<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(t), nblk * BB, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
+        const int nb = bytes / BB;
+        const int64_t b0 = c * (kChunk / BB);
 #pragma unroll
-    for (int u = 0; u < kBlocksPerIter; ++u)
-      if (b + u * stride < nblk) load_block<DT>(t, b + u * stride, v[u]);
-#pragma unroll
-    for (int u = 0; u < kBlocksPerIter; ++u)
-      if (b + u * stride < nblk) encode_block(v[u], s_t, d, codes, scales, b + u * stride);
-  }
+        for (int q = 0; q < kChunk / BB / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          if (j >= nb) continue;
+          float v[16];
+          smem_block<DT>(chunk + j * BB, v);
+          encode_block(v, s_t, d, codes, scales, b0 + j);
+        }
+      });
 }
 
 // One byte (two entries) per thread; value computed in fp64 (exact) and rounded once.
@@ -183,6 +229,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const uint8_t* __restr
 
 int64_t blocks_for(int64_t items) { return (items + kThreads - 1) / kThreads; }
 
+// Grid of a streaming kernel over `bytes` of input: one CTA per chunk, capped at a full wave
+// (at least one CTA, so that the encode kernel also writes the tensor scale of an empty tensor).
+template <typename Kern>
+int ring_grid(Kern k, int64_t bytes) {
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingBytes);
+  return full_wave_grid(k, kThreads, (bytes + kChunk - 1) / kChunk, kRingBytes);
+}
+
 constexpr int64_t kQuantWorkspace = 256;
 
 }  // namespace
@@ -204,19 +258,19 @@ int quantize_nvfp4_launch(const void* t, int dtype, int64_t rows, int64_t cols,
     if (!amax_word) return SP24_ERR_WORKSPACE;
     if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return SP24_ERR_CUDA;
     if (nblk > 0) {
-      if (dtype == SP24_F32) amax_kernel<SP24_F32><<<full_wave_grid(amax_kernel<SP24_F32>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
-      else if (dtype == SP24_BF16) amax_kernel<SP24_BF16><<<full_wave_grid(amax_kernel<SP24_BF16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
-      else amax_kernel<SP24_F16><<<full_wave_grid(amax_kernel<SP24_F16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(t, nblk, amax_word);
+      if (dtype == SP24_F32) amax_kernel<SP24_F32><<<ring_grid(amax_kernel<SP24_F32>, nblk * ((SP24_F32) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, amax_word);
+      else if (dtype == SP24_BF16) amax_kernel<SP24_BF16><<<ring_grid(amax_kernel<SP24_BF16>, nblk * ((SP24_BF16) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, amax_word);
+      else amax_kernel<SP24_F16><<<ring_grid(amax_kernel<SP24_F16>, nblk * ((SP24_F16) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, amax_word);
       ++nl;
     }
   }
   // launched even when nblk == 0 so that tensor_scale_out is written
   if (dtype == SP24_F32)
-    encode_kernel<SP24_F32><<<full_wave_grid(encode_kernel<SP24_F32>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_F32><<<ring_grid(encode_kernel<SP24_F32>, nblk * ((SP24_F32) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   else if (dtype == SP24_BF16)
-    encode_kernel<SP24_BF16><<<full_wave_grid(encode_kernel<SP24_BF16>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_BF16><<<ring_grid(encode_kernel<SP24_BF16>, nblk * ((SP24_BF16) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   else
-    encode_kernel<SP24_F16><<<full_wave_grid(encode_kernel<SP24_F16>, kThreads, blocks_for(nblk > 0 ? nblk : 1)), kThreads, 0, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
+    encode_kernel<SP24_F16><<<ring_grid(encode_kernel<SP24_F16>, nblk * ((SP24_F16) == SP24_F32 ? 64 : 32)), kThreads, kRingBytes, s>>>(t, nblk, ts_in, amax_word, (uint2*)codes, scales, ts_out);
   return launch_status(nl);
 }
 

@@ -13,6 +13,7 @@
 // R*S entries apart; those kernels take one group (or one pair of groups) per thread and
 // read through the read-only cache, which still moves each input byte from DRAM once.
 #include "sp24_internal.cuh"
+#include "sp24_stream.cuh"
 
 namespace sp24 {
 
@@ -76,39 +77,37 @@ __device__ __forceinline__ void count_fails(int fails, int32_t* n_fail) {
 
 // Groups 2v, 2v+1 (16-bit) or group v (fp32) per 16-byte vector v.  Every lane of a warp runs
 // the same number of iterations so the final warp reduction sees all lanes.
-// Each thread keeps kUnroll independent 16-byte loads in flight (vectors base + lane + i*stride),
-// enough bytes per SM to cover DRAM latency at full bandwidth.
-constexpr int kUnroll = 4;
+// Streaming ring: 4 stages of 16 KB per CTA (1024 vectors of 16 bytes, 4 per thread).
+constexpr int kChunk = 16384, kStages = 4;
+constexpr size_t kRingBytes = (size_t)kChunk * kStages;
 
 template <int EB>
 __global__ void __launch_bounds__(kThreads) check24_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint8_t* __restrict__ pass,
                                                         int32_t* __restrict__ n_fail) {
+  extern __shared__ __align__(128) uint8_t ring[];
   int fails = 0;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  for (int64_t base = t0; base - (threadIdx.x & 31) < nv; base += kUnroll * stride) {
-    uint4 x[kUnroll];
+  stream::for_each_chunk<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(w), nv * 16, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
+        const uint4* cv = reinterpret_cast<const uint4*>(chunk);
+        const int nvec = bytes / 16;
+        const int64_t v0 = c * (kChunk / 16);
 #pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
-      const int64_t v = base + i * stride;
-      x[i] = v < nv ? ldg_stream16(w + v) : make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-    }
-#pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
-      const int64_t v = base + i * stride;
-      if (v >= nv) continue;
-      if (EB == 2) {
-        int ok0 = zeros16(x[i].x, x[i].y) >= 2, ok1 = zeros16(x[i].z, x[i].w) >= 2;
-        fails += 2 - ok0 - ok1;
-        reinterpret_cast<uint16_t*>(pass)[v] = (uint16_t)(ok0 | (ok1 << 8));
-      } else {
-        int ok = zeros32(x[i]) >= 2;
-        fails += 1 - ok;
-        pass[v] = (uint8_t)ok;
-      }
-    }
-  }
+        for (int q = 0; q < kChunk / 16 / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          if (j >= nvec) continue;
+          const uint4 x = cv[j];
+          if (EB == 2) {
+            const int ok0 = zeros16(x.x, x.y) >= 2, ok1 = zeros16(x.z, x.w) >= 2;
+            fails += 2 - ok0 - ok1;
+            reinterpret_cast<uint16_t*>(pass)[v0 + j] = (uint16_t)(ok0 | (ok1 << 8));
+          } else {
+            const int ok = zeros32(x) >= 2;
+            fails += 1 - ok;
+            pass[v0 + j] = (uint8_t)ok;
+          }
+        }
+      });
   count_fails(fails, n_fail);
 }
 
@@ -116,41 +115,39 @@ template <int EB>
 __global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint2* __restrict__ values,
                                                         uint8_t* __restrict__ meta) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  for (int64_t base = t0; base - (threadIdx.x & 31) < nv; base += kUnroll * stride) {
-    uint4 x[kUnroll];
+  extern __shared__ __align__(128) uint8_t ring[];
+  stream::for_each_chunk<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(w), nv * 16, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
+        const uint4* cv = reinterpret_cast<const uint4*>(chunk);
+        const int nvec = bytes / 16;
+        const int64_t v0 = c * (kChunk / 16);
 #pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
-      const int64_t v = base + i * stride;
-      x[i] = v < nv ? ldg_stream16(w + v) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < kUnroll; ++i) {
-      const int64_t v = base + i * stride;
-      const bool live = v < nv;
-      if (EB == 2) {
-        if (live) {
-          Group16 a = prune16(x[i].x, x[i].y), b = prune16(x[i].z, x[i].w);
-          values[v] = make_uint2(a.kept, b.kept);
-          meta[v] = (uint8_t)(a.nib | (b.nib << 4));
+        for (int q = 0; q < kChunk / 16 / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          const bool live = j < nvec;
+          const uint4 x = live ? cv[j] : make_uint4(0, 0, 0, 0);
+          const int64_t v = v0 + j;
+          if (EB == 2) {
+            if (live) {
+              const Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
+              values[v] = make_uint2(a.kept, b.kept);
+              meta[v] = (uint8_t)(a.nib | (b.nib << 4));
+            }
+          } else {
+            const uint32_t nib = mask_nibble(keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w)));
+            const uint32_t i0 = nib & 3, i1 = nib >> 2;
+            const uint32_t e0 = i0 == 0 ? x.x : (i0 == 1 ? x.y : x.z);
+            const uint32_t e1 = i1 == 3 ? x.w : (i1 == 2 ? x.z : x.y);
+            // the partner group (v ^ 1) is in lane ^ 1: j and v have the parity of threadIdx.x
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+            if (live) {
+              values[v] = make_uint2(e0, e1);
+              const bool partner_live = (j ^ 1) < nvec;
+              if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (partner_live ? other << 4 : 0u));
+            }
+          }
         }
-      } else {
-        uint32_t m = keep_mask(mag32(x[i].x), mag32(x[i].y), mag32(x[i].z), mag32(x[i].w));
-        uint32_t nib = mask_nibble(m);
-        uint32_t i0 = nib & 3, i1 = nib >> 2;
-        uint32_t v0 = i0 == 0 ? x[i].x : (i0 == 1 ? x[i].y : x[i].z);
-        uint32_t v1 = i1 == 3 ? x[i].w : (i1 == 2 ? x[i].z : x[i].y);
-        // the partner group v^1 lives in lane^1 (each warp's first vector index is even)
-        uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
-        if (live) {
-          values[v] = make_uint2(v0, v1);
-          bool partner_live = (v ^ 1) < nv;
-          if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (partner_live ? other << 4 : 0u));
-        }
-      }
-    }
-  }
+      });
 }
 
 // Inverse of prune24_vec for 16-bit data: two groups per thread.
@@ -294,6 +291,13 @@ __global__ void __launch_bounds__(kThreads) decompress24_any(const void* __restr
 
 int64_t blocks_for(int64_t items) { return (items + kThreads - 1) / kThreads; }
 
+// Grid of a streaming kernel over nv 16-byte vectors: one CTA per chunk, capped at a full wave.
+template <typename Kern>
+int ring_grid(Kern k, int64_t nv) {
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingBytes);
+  return full_wave_grid(k, kThreads, (nv * 16 + kChunk - 1) / kChunk, kRingBytes);
+}
+
 // Validates (op, shape, ndim) and returns the group count and layout.
 int parse_shape(int op, const int64_t* shape, int ndim, int64_t* G, Layout* L) {
   if (!shape || ndim < 1 || ndim > 4) return SP24_ERR_INVALID_ARG;
@@ -356,9 +360,9 @@ extern "C" int sp24_check_24(const void* w, int dtype, int op, const int64_t* sh
     int64_t nv = G * 4 * eb / 16;  // whole 16-byte vectors
     if (nv > 0) {
       if (eb == 2)
-        check24_vec<2><<<full_wave_grid(check24_vec<2>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+        check24_vec<2><<<ring_grid(check24_vec<2>, nv), kThreads, kRingBytes, s>>>((const uint4*)w, nv, pass, n_fail);
       else
-        check24_vec<4><<<full_wave_grid(check24_vec<4>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, pass, n_fail);
+        check24_vec<4><<<ring_grid(check24_vec<4>, nv), kThreads, kRingBytes, s>>>((const uint4*)w, nv, pass, n_fail);
       ++nl;
       g_done = nv * 16 / (4 * eb);
     }
@@ -391,9 +395,9 @@ extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const in
     if (eb == 4) nv &= ~int64_t(1);  // whole meta bytes only
     if (nv > 0) {
       if (eb == 2)
-        prune24_vec<2><<<full_wave_grid(prune24_vec<2>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+        prune24_vec<2><<<ring_grid(prune24_vec<2>, nv), kThreads, kRingBytes, s>>>((const uint4*)w, nv, (uint2*)values, meta);
       else
-        prune24_vec<4><<<full_wave_grid(prune24_vec<4>, kThreads, blocks_for(nv)), kThreads, 0, s>>>((const uint4*)w, nv, (uint2*)values, meta);
+        prune24_vec<4><<<ring_grid(prune24_vec<4>, nv), kThreads, kRingBytes, s>>>((const uint4*)w, nv, (uint2*)values, meta);
       ++nl;
       p_done = (nv * 16 / (4 * eb)) / 2;
     }

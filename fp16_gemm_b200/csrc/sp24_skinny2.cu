@@ -191,10 +191,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// x[n, k] as 16-bit bits of T (0 outside the matrix); NVFP4 x decoded to E2M1 * E4M3.
+// x[n, k] as 16-bit bits of T (0 outside the matrix); NVFP4 x decoded to E2M1 * E4M3.  `n` is
+// the x row already mapped (grouped mode: the routed token), `live` says whether the tile row
+// exists.
 template <typename T>
-__device__ __forceinline__ uint32_t xval(const SkinnyParams& p, int64_t n, int64_t k) {
-  if (n >= p.M || k >= p.K) return 0;
+__device__ __forceinline__ uint32_t xval(const SkinnyParams& p, int64_t n, int64_t k, bool live = true) {
+  if (!live || k >= p.K) return 0;
   if (p.x_fmt == X_16) return __ldg(reinterpret_cast<const unsigned short*>(p.x) + n * p.K + k);
   const uint8_t* codes = reinterpret_cast<const uint8_t*>(p.x);
   const uint32_t c = (codes[(n * p.K + k) >> 1] >> (4 * (k & 1))) & 0xf;
@@ -209,24 +211,36 @@ __device__ __forceinline__ uint32_t xval(const SkinnyParams& p, int64_t n, int64
 
 // Eight consecutive x entries [k, k+8) of token n as four packed 16-bit pairs.
 template <typename T>
-__device__ __forceinline__ uint4 xoct(const SkinnyParams& p, int64_t n, int64_t k) {
-  if (p.x_fmt == X_16 && n < p.M && k + 8 <= p.K)
+__device__ __forceinline__ uint4 xoct(const SkinnyParams& p, int64_t n, int64_t k, bool live) {
+  if (p.x_fmt == X_16 && live && k + 8 <= p.K)
     return __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
   uint32_t v[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = xval<T>(p, n, k + i);
+  for (int i = 0; i < 8; ++i) v[i] = xval<T>(p, n, k + i, live);
   return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
 }
 
-template <int WF, typename T, int NT>
-__global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams p) {
+template <int WF, typename T, int NT, bool GROUPED>
+__global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
   using C = F2<WF>;
   using L = Smem2<WF, NT>;
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
+  __shared__ int32_t rows_of[GROUPED ? 64 : 1];  // grouped: flat (token, slot) of each tile row
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
+  if constexpr (GROUPED) {
+    // tile = (expert, first perm index, count): rebase w / scales / meta on the expert's rows
+    const int32_t* tl = p.tiles + 3 * (int64_t)blockIdx.z;
+    const int32_t e = tl[0], first = tl[1], cnt = tl[2];
+    if (cnt <= 0) return;
+    p.M = cnt;
+    p.w += (int64_t)e * p.expert_rows * p.w_row_bytes;
+    if (p.w_scales) p.w_scales += (int64_t)e * p.expert_rows * p.scale_row_bytes;
+    if (p.meta) p.meta += (int64_t)e * p.expert_rows * p.meta_row_bytes;
+    if (threadIdx.x < 64) rows_of[threadIdx.x] = threadIdx.x < cnt ? p.perm[first + threadIdx.x] : 0;
+  }
   const int64_t row0 = (int64_t)blockIdx.x * kRows;
   const int64_t k0 = (int64_t)blockIdx.y * C::KC;
   const int64_t kv = p.K - k0 < C::KC ? p.K - k0 : C::KC;  // valid logical K in this slice
@@ -240,7 +254,7 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams
     mbar_init(&bar, 1);
     tc::fence_mbar_init();
   }
-  __syncthreads();
+  __syncthreads();  // also publishes rows_of
   if (threadIdx.x == 0) mbar_arrive_expect_tx(&bar, (uint32_t)rows_v * (vbytes + sbytes + mbytes));
   __syncthreads();
   if (threadIdx.x < rows_v) {
@@ -280,7 +294,9 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams
                 ch = it / (LV / 8) / 32 / NT;
       const int gg = ln >> 2, cc = ln & 3;
       const int64_t kb = k0 + (int64_t)ch * C::CHUNK + LV * cc + 8 * oct;
-      const uint4 v = xoct<T>(p, 8 * t + gg, kb);
+      const int nrow = 8 * t + gg;
+      const int64_t xr = GROUPED ? (nrow < p.M ? rows_of[nrow] / p.topk : 0) : nrow;
+      const uint4 v = xoct<T>(p, xr, kb, nrow < p.M);
       // the octet covers steps 2*oct and 2*oct+1 of this lane piece
       uint2 e0, e1;
       if (WF == W_DQ4) {  // slots (0,4,1,5) and (2,6,3,7) of the octet
@@ -302,16 +318,18 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
       const int ln = it % 32, t = (it / 32) % NT, win = it / 32 / NT;
       const int gg = ln >> 2, cc = ln & 3;
-      const int64_t n = 8 * t + gg;
+      const int nrow = 8 * t + gg;
+      const bool live = nrow < p.M;
+      const int64_t n = GROUPED ? (live ? rows_of[nrow] / p.topk : 0) : nrow;
       const int64_t kb = k0 + 32 * win + 2 * cc;
       uint32_t w4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int64_t k = kb + 8 * i;
-        if (p.x_fmt == X_16 && n < p.M && k + 2 <= p.K)
+        if (p.x_fmt == X_16 && live && k + 2 <= p.K)
           w4[i] = __ldg(reinterpret_cast<const unsigned int*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
         else
-          w4[i] = xval<T>(p, n, k) | (xval<T>(p, n, k + 1) << 16);
+          w4[i] = xval<T>(p, n, k, live) | (xval<T>(p, n, k + 1, live) << 16);
       }
       xs[it] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
@@ -410,7 +428,8 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams
       const int64_t n = 8 * t + 2 * c + (q & 1);
       const int64_t r = row0 + rg + ((q & 2) ? 8 : 0);
       if (n < p.M && r < p.N) {
-        float* dst = p.y + n * p.N + r;
+        const int64_t orow = GROUPED ? (int64_t)rows_of[n] : n;
+        float* dst = p.y + orow * p.N + r;
         const float v = acc[t][q] * scale;
         if (p.accumulate) atomicAdd(dst, v);
         else *dst = v;
@@ -419,13 +438,13 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(const SkinnyParams
   }
 }
 
-template <int WF, typename T>
-int launch2(const SkinnyParams& p, int nt, cudaStream_t s) {
+template <int WF, typename T, bool GROUPED = false>
+int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
   using C = F2<WF>;
-  dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)((p.K + C::KC - 1) / C::KC));
+  dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)((p.K + C::KC - 1) / C::KC), tiles);
 #define SP24_L2(NTV)                                                                                        \
   {                                                                                                         \
-    auto kern = skinny2_kernel<WF, T, NTV>;                                                                 \
+    auto kern = skinny2_kernel<WF, T, NTV, GROUPED>;                                                        \
     constexpr int smem = Smem2<WF, NTV>::TOTAL;                                                             \
     if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
       return SP24_ERR_CUDA;                                                                                 \
@@ -443,6 +462,25 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s) {
 }
 
 }  // namespace
+
+// Grouped launch: grid.z = max_tiles token tiles (<= 64 tokens each, NT = 8); y must be zeroed
+// by the caller when K spans several slices (results are accumulated).
+int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStream_t s) {
+  if (max_tiles <= 0) return SP24_OK;
+  if (max_tiles > 65535) return SP24_ERR_UNSUPPORTED;
+  const int kc = wf == W_D16 ? F2<W_D16>::KC : wf == W_DQ4 ? F2<W_DQ4>::KC : wf == W_S16 ? F2<W_S16>::KC : F2<W_SQ4>::KC;
+  p.accumulate = (p.K + kc - 1) / kc > 1;
+  p.M = 64;
+  const bool bf = t16 == SP24_BF16;
+  const unsigned z = (unsigned)max_tiles;
+  switch (wf) {
+    case W_D16: return bf ? launch2<W_D16, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_D16, __half, true>(p, 8, s, z);
+    case W_DQ4: return bf ? launch2<W_DQ4, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_DQ4, __half, true>(p, 8, s, z);
+    case W_S16: return bf ? launch2<W_S16, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_S16, __half, true>(p, 8, s, z);
+    case W_SQ4: return bf ? launch2<W_SQ4, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_SQ4, __half, true>(p, 8, s, z);
+  }
+  return SP24_ERR_UNSUPPORTED;
+}
 
 // True when the shared-memory staged skinny kernel can take this problem: every row slice of
 // every array starts 16-byte aligned and has a 16-byte multiple length.

@@ -189,6 +189,24 @@ int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int6
                        int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                        int algo, void* stream);
 
+/* ----------------------------------------------------------------------- a7: routed experts */
+/* [P1] "Concurrency, not sparsity, is the lever": tokens routed top-k to E experts.
+ *   Y[t, s, n] = sum_k x[t, k] W[e, n, k],  e = routing[t, s]   (fp32 [T, topk, N], device)
+ *   x        T rows (F16, BF16 or NVFP4), as for sp24_gemm_dense.
+ *   routing  device int32 [T, topk]; ids outside [0, E) set the device error word
+ *            (SP24_ERR_INVALID_ARG) and leave their outputs 0.
+ *   weights  the E experts stacked as one [E*N, K] operand: exactly one of w_dense
+ *            (16-bit or NVFP4; NVFP4 experts share one tensor scale, [P5] "The shared global
+ *            scale") or w_sparse (2:4-compressed, stacked [E*N, K/2] values + [E*N, K/8] meta).
+ *   K alignment: NVFP4 dense K % 256, NVFP4 2:4 K % 512, 16-bit K % 8 (2:4: K % 128).
+ *   workspace: sp24_gemm_grouped_workspace_size() bytes, 16-byte aligned (routing histogram,
+ *   offsets, token tiles, permutation). */
+int sp24_gemm_grouped_workspace_size(int64_t T, int topk, int64_t E, int64_t* bytes);
+int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, int64_t T, int topk,
+                      const sp24_operand* w_dense, const sp24_sparse_operand* w_sparse, int64_t E,
+                      int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                      void* stream);
+
 /* ----------------------------------------------------------------------- diagnostics */
 /* Number of kernels this library has launched in this process (host-side counter, all
  * devices and streams).  For accounting in benchmarks; memsets are not counted. */

@@ -95,8 +95,12 @@ def routing_topk(g: np.random.Generator, T: int, E: int, topk: int) -> np.ndarra
 
 def moe(seed: int = SEED, E: int = 512, N: int = 512, K: int = 2048, T: int = 4096,
         topk: int = 10):
+    """Expert weights are drawn one expert after the other from the stream (the same numbers a
+    single [E, N, K] draw gives), which keeps the float64 temporary at one expert."""
     g = rng(seed)
-    W = draw(g, (E, N, K), "bf16", 0.02)
+    W = np.empty((E, N, K), dtype=np.uint16)
+    for e in range(E):
+        W[e] = draw(g, (N, K), "bf16", 0.02)
     X = draw(g, (T, K), "bf16")
     routing = routing_topk(g, T, E, topk)
     return {"W": W, "X": X, "routing": routing}

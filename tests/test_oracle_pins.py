@@ -432,3 +432,12 @@ def test_tolerance_rule(oracle):
     ok = oracle.within_tolerance(np.array([1.0005, 0.0, 1e-9]), np.array([1.0, 0.0, 0.0]),
                                  np.array([1.0, 0.0, 0.0]))
     assert ok.tolist() == [True, True, False]
+
+
+def test_moe_generator_matches_one_draw():
+    """Drawing experts one by one continues the same stream: identical to one [E, N, K] draw."""
+    d = synth.moe(E=3, N=4, K=16, T=5, topk=2)
+    g = synth.rng(0)
+    W = synth.draw(g, (3, 4, 16), "bf16", 0.02)
+    X = synth.draw(g, (5, 16), "bf16")
+    assert np.array_equal(d["W"], W) and np.array_equal(d["X"], X)
