@@ -422,17 +422,25 @@ def run_sweep(args) -> None:
                         else torch.from_numpy(a)).to(dev)
 
     def timeit(fn, reps=20):
-        for _ in range(3):
-            fn(0)
+        """Median over 5 replays of a CUDA graph of `reps` back-to-back launches (rotating
+        operand copies), per launch in microseconds: no host time between launches."""
+        for r in range(3):
+            fn(r)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream()):
+            for r in range(reps):
+                fn(r)
+        g.replay()
         torch.cuda.synchronize()
         times = []
-        for r in range(reps):
+        for _ in range(5):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fn(r)
+            g.replay()
             b.record()
             torch.cuda.synchronize()
-            times.append(a.elapsed_time(b) * 1e3)
+            times.append(a.elapsed_time(b) * 1e3 / reps)
         return statistics.median(times)
 
     def clone_op(o):
@@ -524,6 +532,43 @@ def run_sweep(args) -> None:
                           "n_fail": int(nf.item())}), flush=True)
 
 
+def run_ncu_target() -> None:
+    """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode
+    pipeline on the decode workload, W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096)."""
+    import torch
+
+    import fp16_gemm_b200 as sp
+    import synth
+
+    torch.cuda.set_device(0)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    d = synth.decode_nvfp4()
+    x, w = bf(d["X"]), bf(d["W"])
+    for _ in range(2):
+        sp.check_24(w)
+        v, m = sp.prune_compress_24(w)
+        wq, vq = sp.quantize_nvfp4(w), sp.quantize_nvfp4(v)
+        sp.gemm_dense(x, wq)
+        sp.gemm_sparse24(x, sp.Sparse24(vq, m), K)
+    d = synth.prefill_w4a4()
+    xq, w = sp.quantize_nvfp4(bf(d["X"])), bf(d["W"])
+    v, m = sp.prune_compress_24(w)
+    wq, vq = sp.quantize_nvfp4(w), sp.quantize_nvfp4(v)
+    for _ in range(2):
+        sp.gemm_dense(xq, wq)
+        sp.gemm_sparse24(xq, sp.Sparse24(vq, m), 4096)
+    g = synth.rng(0)
+    w16 = torch.from_numpy(synth.draw(g, (5120, 5120), "f16")).cuda()
+    x16 = torch.from_numpy(synth.draw(g, (4096, 5120), "f16")).cuda()
+    v, m = sp.prune_compress_24(w16)
+    for _ in range(2):
+        sp.gemm_dense(x16, w16)
+        sp.gemm_sparse24(x16, sp.Sparse24(v, m), 5120)
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
+    print("ncu target done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -535,9 +580,13 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
+    ap.add_argument("--ncu-target", action="store_true", help="run each kernel once, untimed")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.ncu_target:
+        run_ncu_target()
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

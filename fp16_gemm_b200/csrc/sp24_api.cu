@@ -56,7 +56,9 @@ int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
       q.x = reinterpret_cast<const uint8_t*>(p.x) + m0 * p.K / 2;
       q.x_scales = p.x_scales + m0 * p.K / 16;
     }
-    int st = skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s) : skinny_gemm(wf, t16, q, s);
+    int st = decode_supported(wf, q)    ? decode_gemv(wf, t16, q, s)
+             : skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s)
+                                        : skinny_gemm(wf, t16, q, s);
     if (st) return st;
   }
   return SP24_OK;

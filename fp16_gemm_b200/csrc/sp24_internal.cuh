@@ -1,6 +1,7 @@
 // Internal helpers shared by the libsp24 translation units (device code for sm_100a).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -103,6 +104,14 @@ int skinny_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 // alignment its bulk copies need.
 bool skinny2_supported(int wf, const SkinnyParams& p);
 int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
+// Persistent decode GEMV for NVFP4 weights (dense / 2:4) at M <= 8 (TMA-fed, one CTA per SM).
+bool decode_supported(int wf, const SkinnyParams& p);
+int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s);
+// 2-D TMA maps (defined with the tensor-core GEMMs): 128-byte swizzled, and unswizzled bytes.
+int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                 uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows);
+int make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                       uint32_t box_cols, uint32_t box_rows);
 // Grouped variant: one launch over max_tiles token tiles (tile table and perm on the device).
 int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStream_t s);
 

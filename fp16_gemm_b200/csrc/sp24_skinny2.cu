@@ -461,6 +461,256 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
   return launch_status();
 }
 
+// ------------------------------------------------------------------ persistent decode GEMV (M <= 8)
+//
+// One CTA per SM: a producer warp streams 16-row weight units (2-D TMA: codes with the 128-byte
+// swizzle, block scales and 2:4 nibbles unswizzled) through a ring of shared-memory slots, and 8
+// consumer warps take the units round-robin.  x (M <= 8 tokens) is staged once per CTA for the
+// whole K in fragment order.  Units are spread evenly over all CTAs (each CTA a contiguous range
+// in tile-major order), so every SM streams the same number of bytes; a warp's partial sums of a
+// 16-row tile are added into one of four shared tile buffers, and the last warp of the CTA to
+// finish a tile adds the buffer into y (zeroed first) with one atomic per output.
+//
+// MMA row m of a warp reads tile row prow(m) = (m/2) + 4 (m%2) (+8 for m >= 8): in every group of
+// 8 lanes sharing a shared-memory phase, the two rows then sit 4 rows apart, so the 128-byte
+// swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)) puts their pieces in disjoint
+// halves of the banks.
+constexpr int kDecConsumers = 8;
+constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+
+template <int WF>
+struct U3;
+template <>
+struct U3<W_DQ4> {  // 256 K per unit: codes 16 x 128 B, scales 16 x 16 B
+  static constexpr int UK = 256, CODES = 2048, SCALES = 256, META = 0, SLOT = 3072, SLOTS = 24;
+};
+template <>
+struct U3<W_SQ4> {  // 512 K per unit: codes 16 x 128 B, scales 16 x 16 B, nibbles 16 x 64 B
+  static constexpr int UK = 512, CODES = 2048, SCALES = 256, META = 1024, SLOT = 4096, SLOTS = 16;
+};
+
+__device__ __forceinline__ int prow(int m) { return (m & 8) + ((m & 7) >> 1) + 4 * (m & 1); }
+
+template <int WF, typename T>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_gemv_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
+                       const __grid_constant__ CUtensorMap tmM, const SkinnyParams p) {
+  using U = U3<WF>;
+  constexpr int S = U::SLOTS;
+  extern __shared__ uint8_t dsm[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+  uint8_t* slots = base;                              // S x SLOT, 1024-aligned
+  uint8_t* xs = base + S * U::SLOT;                   // x fragments, 16 * K bytes
+  __shared__ uint64_t full_bar[S], empty_bar[S];
+  __shared__ float tbuf[4][16][8];
+  __shared__ int tdone[4];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t upr = p.K / U::UK;                    // units per 16-row tile
+  const int64_t U_all = ((p.N + 15) / 16) * upr;
+  const int64_t ub = U_all * blockIdx.x / gridDim.x, ue = U_all * (blockIdx.x + 1) / gridDim.x;
+  const int nunits = (int)(ue - ub);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      tc::mbar_init(&full_bar[i], 1);
+      tc::mbar_init(&empty_bar[i], 1);
+    }
+    tc::fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 4 * 16 * 8; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
+  if (threadIdx.x < 4) tdone[threadIdx.x] = 0;
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---- producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmC);
+      tc::prefetch_tmap(&tmS);
+      if (U::META) tc::prefetch_tmap(&tmM);
+      for (int i = 0; i < nunits; ++i) {
+        const int sl = i % S;
+        if (!mbar_wait(&empty_bar[sl], ((i / S) & 1) ^ 1)) {
+          set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+          break;
+        }
+        const int64_t u = ub + i, tile = u / upr, kp = u % upr;
+        uint8_t* d = slots + sl * U::SLOT;
+        mbar_arrive_expect_tx(&full_bar[sl], U::CODES + U::SCALES + U::META);
+        tc::tma_load_2d(d, &tmC, &full_bar[sl], (int)(kp * 128), (int)(tile * 16));
+        tc::tma_load_2d(d + U::CODES, &tmS, &full_bar[sl], (int)(kp * 16), (int)(tile * 16));
+        if (U::META) tc::tma_load_2d(d + U::CODES + U::SCALES, &tmM, &full_bar[sl], (int)(kp * 64), (int)(tile * 16));
+      }
+    }
+    return;
+  }
+
+  // ---- x for the whole K, fragment order (all consumer threads)
+  const int ct = threadIdx.x - 32, nct = blockDim.x - 32;
+  if (WF == W_DQ4) {
+    // entry (chunk, step, lane) of 8 bytes; one item = 8 consecutive k of a lane piece
+    uint2* xf = reinterpret_cast<uint2*>(xs);
+    const int items = (int)(p.K / 128) * 32 * 4;
+    for (int it = ct; it < items; it += nct) {
+      const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
+      const int gg = ln >> 2, cc = ln & 3;
+      const int64_t kb = (int64_t)ch * 128 + 32 * cc + 8 * oct;
+      const uint4 v = xoct<T>(p, gg, kb, gg < p.M);
+      xf[(ch * 8 + 2 * oct) * 32 + ln] = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
+      xf[(ch * 8 + 2 * oct + 1) * 32 + ln] = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+    }
+  } else {
+    // entry (window, lane) of 16 bytes: x[g][32 w + 2c + 8i + {0,1}], i = 0..3
+    uint4* xf = reinterpret_cast<uint4*>(xs);
+    const int items = (int)(p.K / 32) * 32;
+    for (int it = ct; it < items; it += nct) {
+      const int ln = it & 31, w = it >> 5;
+      const int gg = ln >> 2, cc = ln & 3;
+      uint32_t q4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t k = 32 * (int64_t)w + 2 * cc + 8 * i;
+        q4[i] = xval<T>(p, gg, k, gg < p.M) | (xval<T>(p, gg, k + 1, gg < p.M) << 16);
+      }
+      xf[it] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(nct) : "memory");  // consumers only
+
+  // ---- consumers
+  const int cw = warp - 1;
+  const int g = lane >> 2, c = lane & 3;
+  const int r0 = prow(g), r1 = prow(g + 8);
+  float scale = 256.0f * *p.w_ts;
+  if (p.x_fmt == X_Q4) scale *= *p.x_ts;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int64_t cur = -1;
+  int cnt = 0;
+
+  auto flush = [&](int64_t tile) {
+    float* b = &tbuf[tile & 3][0][0];
+    atomicAdd(b + r0 * 8 + 2 * c, acc[0]);
+    atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1]);
+    atomicAdd(b + r1 * 8 + 2 * c, acc[2]);
+    atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3]);
+    __threadfence_block();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      const int64_t lo = tile * upr > ub ? tile * upr : ub, hi = (tile + 1) * upr < ue ? (tile + 1) * upr : ue;
+      last = atomicAdd(&tdone[tile & 3], cnt) + cnt == (int)(hi - lo);
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence_block();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = lane + 32 * q, row = e >> 3, tok = e & 7;
+        const int64_t gr = tile * 16 + row;
+        if (tok < p.M && gr < p.N) atomicAdd(p.y + (int64_t)tok * p.N + gr, b[e] * scale);
+        b[e] = 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) tdone[tile & 3] = 0;
+    }
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    cnt = 0;
+  };
+
+  for (int i = cw; i < nunits; i += kDecConsumers) {
+    const int sl = i % S;
+    const int64_t u = ub + i, tile = u / upr, kp = u % upr;
+    if (tile != cur) {
+      if (cur >= 0) flush(cur);
+      cur = tile;
+    }
+    if (!mbar_wait(&full_bar[sl], (i / S) & 1)) {
+      set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+      break;
+    }
+    const uint8_t* d = slots + sl * U::SLOT;
+    const uint8_t* sc = d + U::CODES;
+    if constexpr (WF == W_DQ4) {
+      const uint2* xf = reinterpret_cast<const uint2*>(xs);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int j = 4 * ch + c;
+        const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
+        const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
+        uint32_t s00, s01, s10, s11;
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), s00, s01);
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), s10, s11);
+        const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
+        const int64_t gch = kp * 2 + ch;
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+          const int q = st >> 1, i0 = 2 * (st & 1);
+          const uint32_t sa = st < 4 ? s00 : s01, sb = st < 4 ? s10 : s11;
+          const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0), sa);
+          const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0 + 1), sa);
+          const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0), sb);
+          const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0 + 1), sb);
+          float acc4[4] = {acc[0], acc[1], acc[2], acc[3]};
+          mma_k16<T>(acc4, a0, a1, a2, a3, xf[(gch * 8 + st) * 32 + lane]);
+          acc[0] = acc4[0]; acc[1] = acc4[1]; acc[2] = acc4[2]; acc[3] = acc4[3];
+        }
+      }
+    } else {
+      const uint4* xf = reinterpret_cast<const uint4*>(xs);
+      const uint8_t* me = sc + U::SCALES;
+#pragma unroll 4
+      for (int w = 0; w < 16; ++w) {
+        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * 64 + 4 * w);
+        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * 64 + 4 * w);
+        const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
+        const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * 128 + (((w >> 1) ^ (r0 & 7)) << 4) + 8 * (w & 1));
+        const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * 128 + (((w >> 1) ^ (r1 & 7)) << 4) + 8 * (w & 1));
+        uint32_t s0, s1, unused;
+        scale_pair<T>(sc[r0 * 16 + w], s0, unused);
+        scale_pair<T>(sc[r1 * 16 + w], s1, unused);
+        const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
+        const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
+        const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+        const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+        const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+        const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+        float acc4[4] = {acc[0], acc[1], acc[2], acc[3]};
+        mma_sp_k32<T>(acc4, a0, a1, a2, a3, xf[(kp * 16 + w) * 32 + lane], e);
+        acc[0] = acc4[0]; acc[1] = acc4[1]; acc[2] = acc4[2]; acc[3] = acc4[3];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
+    ++cnt;
+  }
+  if (cur >= 0) flush(cur);
+}
+
+template <int WF, typename T>
+int launch_decode(const SkinnyParams& p, cudaStream_t s) {
+  using U = U3<WF>;
+  CUtensorMap tc_, ts_, tm_;
+  const int64_t cb = WF == W_DQ4 ? p.K / 2 : p.K / 4;
+  int st = make_tmap_2d(&tc_, p.w, 1, p.N, cb, cb, 128, 16);
+  if (st) return st;
+  const int64_t sb = WF == W_DQ4 ? p.K / 16 : p.K / 32;
+  st = make_tmap_2d_plain(&ts_, p.w_scales, p.N, sb, sb, 16, 16);
+  if (st) return st;
+  if (WF == W_SQ4) {
+    st = make_tmap_2d_plain(&tm_, p.meta, p.N, p.K / 8, p.K / 8, 64, 16);
+    if (st) return st;
+  } else {
+    tm_ = ts_;
+  }
+  const size_t smem = 1024 + (size_t)U::SLOTS * U::SLOT + 16 * (size_t)p.K;
+  auto kern = decode_gemv_kernel<WF, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  if (cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
+  kern<<<sm_count(), kDecThreads, smem, s>>>(tc_, ts_, tm_, p);
+  return launch_status();
+}
+
 }  // namespace
 
 // Grouped launch: grid.z = max_tiles token tiles (<= 64 tokens each, NT = 8); y must be zeroed
@@ -479,6 +729,24 @@ int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStre
     case W_S16: return bf ? launch2<W_S16, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_S16, __half, true>(p, 8, s, z);
     case W_SQ4: return bf ? launch2<W_SQ4, __nv_bfloat16, true>(p, 8, s, z) : launch2<W_SQ4, __half, true>(p, 8, s, z);
   }
+  return SP24_ERR_UNSUPPORTED;
+}
+
+// True when the persistent decode kernel takes the problem: NVFP4 weights (dense or 2:4), at most
+// 8 tokens, whole 16-row tiles, K a whole number of units and small enough for x to stay in
+// shared memory (16 K bytes of fragments).
+bool decode_supported(int wf, const SkinnyParams& p) {
+  if (p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0 || p.K > 8192) return false;
+  if (!aligned(p.w, 16) || !aligned(p.w_scales, 16)) return false;
+  if (wf == W_DQ4) return p.K % 256 == 0;
+  if (wf == W_SQ4) return p.K % 512 == 0 && aligned(p.meta, 16);
+  return false;
+}
+
+int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s) {
+  const bool bf = t16 == SP24_BF16;
+  if (wf == W_DQ4) return bf ? launch_decode<W_DQ4, __nv_bfloat16>(p, s) : launch_decode<W_DQ4, __half>(p, s);
+  if (wf == W_SQ4) return bf ? launch_decode<W_SQ4, __nv_bfloat16>(p, s) : launch_decode<W_SQ4, __half>(p, s);
   return SP24_ERR_UNSUPPORTED;
 }
 
