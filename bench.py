@@ -3,8 +3,13 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 
-    check_24(W) -> prune_compress_24(W) -> quantize_nvfp4(W) -> quantize_nvfp4(values)
+    prepare_24(W)                      check + prune/compress + both NVFP4 tensor scales,
+                                       one read of W
+    -> quantize_nvfp4(W, s_w) -> quantize_nvfp4(values, s_v)   encode with those scales
     -> gemm_dense(X, W_nvfp4) -> gemm_sparse24(X, values_nvfp4 + meta)
+
+(the outputs are bit-identical to check_24 -> prune_compress_24 -> quantize_nvfp4(W) ->
+quantize_nvfp4(values), which read W four times).
 
 Workload: X bf16 [8, 5120] N(0, 1), W bf16 [5120, 5120] N(0, 0.02) (the decode shape of the
 pages' NVFP4 decode kernels, hidden width 5120).  Inputs live in HBM before timing starts and
@@ -43,17 +48,17 @@ sys.path.insert(0, ROOT)
 M, N, K = 8, 5120, 5120
 METRIC = "2:4-sparse vs dense GEMM eff. TFLOP/s & HBM GB/s per shape; sparse/dense speedup"
 WORKLOAD = ("decode_nvfp4: X bf16 [8,5120] N(0,1), W bf16 [5120,5120] N(0,0.02); step = "
-            "check_24 + prune_compress_24 + quantize_nvfp4(W) + quantize_nvfp4(values) + "
-            "gemm_dense(X,W_nvfp4) + gemm_sparse24(X,values_nvfp4,meta)")
-STAGES = ("check_24", "prune_compress_24", "quantize_w", "quantize_values", "gemm_dense",
-          "gemm_sparse24")
+            "prepare_24(W: check + prune/compress + tensor scales) + quantize_nvfp4(W) + "
+            "quantize_nvfp4(values) + gemm_dense(X,W_nvfp4) + gemm_sparse24(X,values_nvfp4,meta)")
+STAGES = ("prepare_24", "quantize_w", "quantize_values", "gemm_dense", "gemm_sparse24")
 FALLBACK_HBM_GBS = 6650.0
 
 
 def stage_bytes(rows: int = N) -> dict:
-    """Algorithmic bytes each stage must move for `rows` weight rows (each operand once; the
-    NVFP4 quantiser reads its input twice because the tensor amax must be known before any
-    block is encoded)."""
+    """Algorithmic bytes each stage must move for `rows` weight rows, each operand once: the
+    fused preparation reads W and writes the pass map, the kept values, the nibbles and 24
+    bytes of counts/scales; each encode reads its input (the tensor scale is already known) and
+    writes codes + block scales."""
     w = rows * K * 2                      # bf16 weight
     v = rows * K // 2 * 2                 # kept values, bf16
     meta = rows * K // 8
@@ -62,10 +67,9 @@ def stage_bytes(rows: int = N) -> dict:
     codes_w, scales_w = rows * K // 2, rows * K // 16
     codes_v, scales_v = rows * K // 4, rows * K // 32
     return {
-        "check_24": w + rows * K // 4 + 4,
-        "prune_compress_24": w + v + meta,
-        "quantize_w": 2 * w + codes_w + scales_w + 4,
-        "quantize_values": 2 * v + codes_v + scales_v + 4,
+        "prepare_24": w + rows * K // 4 + v + meta + 24,
+        "quantize_w": w + codes_w + scales_w + 8,
+        "quantize_values": v + codes_v + scales_v + 8,
         "gemm_dense": codes_w + scales_w + 4 + x + y,
         "gemm_sparse24": codes_v + scales_v + 4 + meta + x + y,
     }
@@ -176,6 +180,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         s["nfail"] = torch.empty(1, dtype=torch.int32, device=dev)
         s["v"] = torch.empty((N, K // 2), dtype=torch.bfloat16, device=dev)
         s["m"] = torch.empty(N * K // 8, dtype=torch.uint8, device=dev)
+        s["ts"] = torch.empty(2, dtype=torch.float32, device=dev)
         s["wq"] = sp.NVFP4Tensor(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
                                  torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
                                  torch.empty(1, dtype=torch.float32, device=dev))
@@ -185,15 +190,15 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
         s["yd"] = torch.empty((M, N), dtype=torch.float32, device=dev)
         s["ys"] = torch.empty((M, N), dtype=torch.float32, device=dev)
         sets.append(s)
-    ws = torch.empty(sp.quantize_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+    ws = torch.empty(sp.prepare_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
 
     def stage_fns(s):
         sparse_w = sp.Sparse24(s["vq"], s["m"])
+        prep = sp.Prepared24(s["pass"], s["nfail"], s["v"], s["m"], s["ts"][0:1], s["ts"][1:2])
         return [
-            lambda: sp.check_24(s["w"], pass_out=s["pass"], n_fail_out=s["nfail"]),
-            lambda: sp.prune_compress_24(s["w"], values_out=s["v"], meta_out=s["m"]),
-            lambda: sp.quantize_nvfp4(s["w"], out=s["wq"], workspace=ws),
-            lambda: sp.quantize_nvfp4(s["v"], out=s["vq"], workspace=ws),
+            lambda: sp.prepare_24(s["w"], out=prep, workspace=ws),
+            lambda: sp.quantize_nvfp4(s["w"], tensor_scale=prep.w_tensor_scale, out=s["wq"]),
+            lambda: sp.quantize_nvfp4(s["v"], tensor_scale=prep.v_tensor_scale, out=s["vq"]),
             lambda: sp.gemm_dense(s["x"], s["wq"], out=s["yd"]),
             lambda: sp.gemm_sparse24(s["x"], sparse_w, K, out=s["ys"]),
         ]
@@ -534,7 +539,7 @@ def run_sweep(args) -> None:
 
 def run_ncu_target() -> None:
     """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode
-    pipeline on the decode workload, W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096)."""
+    pipeline on the decode workload: prepare_vec, encode_kernel x2, decode_gemv x2 per pass; W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096)."""
     import torch
 
     import fp16_gemm_b200 as sp
@@ -545,11 +550,9 @@ def run_ncu_target() -> None:
     d = synth.decode_nvfp4()
     x, w = bf(d["X"]), bf(d["W"])
     for _ in range(2):
-        sp.check_24(w)
-        v, m = sp.prune_compress_24(w)
-        wq, vq = sp.quantize_nvfp4(w), sp.quantize_nvfp4(v)
+        _, wq, sw = sp.prepare_nvfp4_24(w)
         sp.gemm_dense(x, wq)
-        sp.gemm_sparse24(x, sp.Sparse24(vq, m), K)
+        sp.gemm_sparse24(x, sw, K)
     d = synth.prefill_w4a4()
     xq, w = sp.quantize_nvfp4(bf(d["X"])), bf(d["W"])
     v, m = sp.prune_compress_24(w)

@@ -34,7 +34,7 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_quantize_nvfp4", "sp24_dequantize_nvfp4", "sp24_gemm_workspace_size",
            "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
            "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc", "sp24_gemm_grouped_workspace_size",
-           "sp24_gemm_grouped")
+           "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24")
 
 _lock = threading.Lock()
 _lib = None
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
             L.sp24_gemm_grouped_workspace_size.argtypes = [I64, I, I64, P]
             L.sp24_gemm_grouped.argtypes = [ctypes.POINTER(_Operand), P, I64, I, ctypes.POINTER(_Operand),
                                              ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
+            L.sp24_prepare_24_workspace_size.argtypes = [I64, I64, P]
+            L.sp24_prepare_24.argtypes = [P, I, I64, I64, P, P, P, P, P, P, P, I64, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -264,6 +266,57 @@ def dequantize_nvfp4(q: NVFP4Tensor, dtype=torch.float32, stream=None) -> torch.
     _call("sp24_dequantize_nvfp4", _ptr(q.codes), _ptr(q.scales), _ptr(q.tensor_scale), R, 2 * L2,
           _DT[dtype], _ptr(out), _stream(stream))
     return out
+
+
+class Prepared24(NamedTuple):
+    """What sp24_prepare_24 produces for a weight W[rows, K]."""
+    pass_map: Optional[torch.Tensor]   # uint8 [rows, K/4] or None
+    n_fail: torch.Tensor               # int32 [1]
+    values: torch.Tensor               # kept entries [rows, K/2], W's dtype
+    meta: torch.Tensor                 # uint8 [rows, K/8] nibble stream
+    w_tensor_scale: torch.Tensor       # fp32 [1]: amax|W| / 2688
+    v_tensor_scale: torch.Tensor       # fp32 [1]: amax|values| / 2688
+
+
+def prepare_workspace_bytes(rows: int, K: int) -> int:
+    n = ctypes.c_int64(0)
+    _call("sp24_prepare_24_workspace_size", rows, K, ctypes.byref(n))
+    return n.value
+
+
+def prepare_24(w: torch.Tensor, with_pass: bool = True, out: Optional[Prepared24] = None,
+               workspace=None, stream=None) -> Prepared24:
+    """check_24 + prune_compress_24 + both NVFP4 tensor scales of a matmul weight w[rows, K]
+    (K % 16 == 0) with one read of w; identical to the separate calls."""
+    _cuda(w, "w")
+    if w.dim() != 2:
+        raise ValueError("prepare_24 wants a 2-D weight")
+    R, K = w.shape
+    dev = w.device
+    if out is None:
+        out = Prepared24(
+            torch.empty((R, K // 4), dtype=torch.uint8, device=dev) if with_pass else None,
+            torch.empty(1, dtype=torch.int32, device=dev),
+            torch.empty((R, K // 2), dtype=w.dtype, device=dev),
+            torch.empty((R, K // 8), dtype=torch.uint8, device=dev),
+            torch.empty(1, dtype=torch.float32, device=dev),
+            torch.empty(1, dtype=torch.float32, device=dev))
+    if workspace is None:
+        workspace = torch.empty(prepare_workspace_bytes(R, K), dtype=torch.uint8, device=dev)
+    _call("sp24_prepare_24", _ptr(w), _dtype_code(w), R, K, _ptr(out.pass_map), _ptr(out.n_fail),
+          _ptr(out.values), _ptr(out.meta), _ptr(out.w_tensor_scale), _ptr(out.v_tensor_scale),
+          _ptr(workspace), workspace.numel(), _stream(stream))
+    return out
+
+
+def prepare_nvfp4_24(w: torch.Tensor, stream=None):
+    """The whole weight side of both GEMM paths: prepare_24, then NVFP4 of w and of its kept
+    values with the tensor scales prepare_24 derived.  Returns (Prepared24, dense NVFP4Tensor,
+    Sparse24 with NVFP4 values)."""
+    p = prepare_24(w, stream=stream)
+    wq = quantize_nvfp4(w, tensor_scale=p.w_tensor_scale, stream=stream)
+    vq = quantize_nvfp4(p.values, tensor_scale=p.v_tensor_scale, stream=stream)
+    return p, wq, Sparse24(vq, p.meta)
 
 
 # ---------------------------------------------------------------------------- a4 .. a6

@@ -67,6 +67,36 @@ __device__ __forceinline__ int zeros32(uint4 v) {
   return (mag32(v.x) == 0) + (mag32(v.y) == 0) + (mag32(v.z) == 0) + (mag32(v.w) == 0);
 }
 
+// |x| of one 16-bit entry of type DT as fp32 (exact).
+template <int DT>
+__device__ __forceinline__ float abs16(uint32_t bits) {
+  if (DT == SP24_BF16) return __uint_as_float((bits & 0x7fffu) << 16);
+  return fabsf(__half2float(__ushort_as_half((unsigned short)(bits & 0xffffu))));
+}
+
+// max(m, |entries of a word|): two 16-bit entries or one fp32.  fmaxf never returns a NaN
+// operand, so NaN entries take no part in a maximum.
+template <int DT>
+__device__ __forceinline__ float max_abs_word(float m, uint32_t w) {
+  if (DT == SP24_F32) return fmaxf(m, fabsf(__uint_as_float(w)));
+  return fmaxf(fmaxf(m, abs16<DT>(w)), abs16<DT>(w >> 16));
+}
+
+// Block-wide max of non-negative floats (ordered like their bit patterns) into *dst with one
+// atomicMax per CTA.
+__device__ __forceinline__ void block_max_to(float m, unsigned int* dst) {
+  __shared__ unsigned int wmax[kThreads / 32];
+  __syncthreads();  // wmax may still be read by an earlier call
+  unsigned int u = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = u;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    unsigned int x = threadIdx.x < kThreads / 32 ? wmax[threadIdx.x] : 0u;
+    x = __reduce_max_sync(0xffffffffu, x);
+    if (threadIdx.x == 0 && x) atomicMax(dst, x);
+  }
+}
+
 __device__ __forceinline__ void count_fails(int fails, int32_t* n_fail) {
   if (!n_fail) return;
   int s = __reduce_add_sync(0xffffffffu, fails);
@@ -148,6 +178,80 @@ __global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict_
           }
         }
       });
+}
+
+// One read of a matmul weight doing the work of check24_vec, prune24_vec and the amax passes of
+// the NVFP4 quantiser for both w and its kept values.  Scratch words (zeroed before the launch):
+// acc[0] = amax|w| bits, acc[1] = amax|kept values| bits, acc[2] = failing groups, acc[3] = CTAs
+// done.  The last CTA to finish writes the fail count and the two NVFP4 tensor scales
+// amax / 2688, computed exactly as the quantiser derives them.
+template <int DT>
+__global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict__ w, int64_t nv,
+                                                        uint8_t* __restrict__ pass, uint2* __restrict__ values,
+                                                        uint8_t* __restrict__ meta, unsigned int* __restrict__ acc,
+                                                        int32_t* __restrict__ n_fail, float* __restrict__ ts_w,
+                                                        float* __restrict__ ts_v) {
+  constexpr int EB = DT == SP24_F32 ? 4 : 2;
+  extern __shared__ __align__(128) uint8_t ring[];
+  int fails = 0;
+  float mw = 0.0f, mv = 0.0f;
+  stream::for_each_chunk<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(w), nv * 16, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
+        const uint4* cv = reinterpret_cast<const uint4*>(chunk);
+        const int nvec = bytes / 16;
+        const int64_t v0 = c * (kChunk / 16);
+#pragma unroll
+        for (int q = 0; q < kChunk / 16 / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          const bool live = j < nvec;
+          const uint4 x = live ? cv[j] : make_uint4(0, 0, 0, 0);
+          const int64_t v = v0 + j;
+          mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.x), x.y);
+          mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.z), x.w);
+          if (EB == 2) {
+            if (live) {
+              const int ok0 = zeros16(x.x, x.y) >= 2, ok1 = zeros16(x.z, x.w) >= 2;
+              fails += 2 - ok0 - ok1;
+              if (pass) reinterpret_cast<uint16_t*>(pass)[v] = (uint16_t)(ok0 | (ok1 << 8));
+              const Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
+              values[v] = make_uint2(a.kept, b.kept);
+              meta[v] = (uint8_t)(a.nib | (b.nib << 4));
+              mv = max_abs_word<DT>(max_abs_word<DT>(mv, a.kept), b.kept);
+            }
+          } else {
+            const uint32_t nib = mask_nibble(keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w)));
+            const uint32_t i0 = nib & 3, i1 = nib >> 2;
+            const uint32_t e0 = i0 == 0 ? x.x : (i0 == 1 ? x.y : x.z);
+            const uint32_t e1 = i1 == 3 ? x.w : (i1 == 2 ? x.z : x.y);
+            // the partner group (v ^ 1) is in lane ^ 1: j and v have the parity of threadIdx.x
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+            if (live) {
+              const int ok = zeros32(x) >= 2;
+              fails += 1 - ok;
+              if (pass) pass[v] = (uint8_t)ok;
+              values[v] = make_uint2(e0, e1);
+              if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (other << 4));  // nv is even
+              mv = max_abs_word<DT>(max_abs_word<DT>(mv, e0), e1);
+            }
+          }
+        }
+      });
+  count_fails(fails, reinterpret_cast<int32_t*>(acc + 2));
+  block_max_to(mw, acc);
+  block_max_to(mv, acc + 1);
+  // last CTA: publish the totals
+  __shared__ int is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(acc + 3, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    __threadfence();
+    const volatile unsigned int* a = acc;
+    if (n_fail) *n_fail = (int32_t)a[2];
+    if (ts_w) *ts_w = __fdiv_rn(__uint_as_float(a[0]), 2688.0f);
+    if (ts_v) *ts_v = __fdiv_rn(__uint_as_float(a[1]), 2688.0f);
+  }
 }
 
 // Inverse of prune24_vec for 16-bit data: two groups per thread.
@@ -442,4 +546,39 @@ extern "C" int sp24_decompress_24(const void* values, const uint8_t* meta, int d
     ++nl;
   }
   return launch_status(nl);
+}
+
+extern "C" int sp24_prepare_24_workspace_size(int64_t rows, int64_t K, int64_t* bytes) {
+  if (!bytes) return SP24_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 16) return SP24_ERR_SHAPE;
+  *bytes = 256;
+  return SP24_OK;
+}
+
+extern "C" int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* pass,
+                               int32_t* n_fail, void* values, uint8_t* meta, float* w_tensor_scale,
+                               float* v_tensor_scale, void* workspace, int64_t workspace_bytes,
+                               void* stream) {
+  const int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  if (rows < 0 || K < 0 || K % 16) return SP24_ERR_SHAPE;
+  const int64_t nv = rows * K * eb / 16;
+  if (nv > 0 && (!w || !values || !meta)) return SP24_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < 256) return SP24_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
+  if (nv > 0 && (!aligned(w, 16) || !aligned(values, 8) || (pass && !aligned(pass, 2)))) return SP24_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  unsigned int* acc = reinterpret_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(acc, 0, 4 * sizeof(unsigned int), s) != cudaSuccess) return SP24_ERR_CUDA;
+  // launched even for an empty weight, so that the count and the scales are written
+  if (dtype == SP24_F32)
+    prepare_vec<SP24_F32><<<ring_grid(prepare_vec<SP24_F32>, nv), kThreads, kRingBytes, s>>>(
+        (const uint4*)w, nv, pass, (uint2*)values, meta, acc, n_fail, w_tensor_scale, v_tensor_scale);
+  else if (dtype == SP24_BF16)
+    prepare_vec<SP24_BF16><<<ring_grid(prepare_vec<SP24_BF16>, nv), kThreads, kRingBytes, s>>>(
+        (const uint4*)w, nv, pass, (uint2*)values, meta, acc, n_fail, w_tensor_scale, v_tensor_scale);
+  else
+    prepare_vec<SP24_F16><<<ring_grid(prepare_vec<SP24_F16>, nv), kThreads, kRingBytes, s>>>(
+        (const uint4*)w, nv, pass, (uint2*)values, meta, acc, n_fail, w_tensor_scale, v_tensor_scale);
+  return launch_status();
 }

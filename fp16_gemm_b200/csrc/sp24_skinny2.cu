@@ -545,34 +545,71 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     return;
   }
 
-  // ---- x for the whole K, fragment order (all consumer threads)
+  // ---- x for the whole K, fragment order (all consumer threads).  Every CTA reads the same x,
+  // so each starts at its own rotation of the items, and each thread issues XB loads before it
+  // stores any: the staging costs a few L2 round trips instead of one per item.
   const int ct = threadIdx.x - 32, nct = blockDim.x - 32;
+  constexpr int XB = 8;
   if (WF == W_DQ4) {
-    // entry (chunk, step, lane) of 8 bytes; one item = 8 consecutive k of a lane piece
+    // item = (chunk, lane, oct): 8 consecutive k of a lane piece -> two 8-byte fragment entries
     uint2* xf = reinterpret_cast<uint2*>(xs);
     const int items = (int)(p.K / 128) * 32 * 4;
-    for (int it = ct; it < items; it += nct) {
-      const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
-      const int gg = ln >> 2, cc = ln & 3;
-      const int64_t kb = (int64_t)ch * 128 + 32 * cc + 8 * oct;
-      const uint4 v = xoct<T>(p, gg, kb, gg < p.M);
-      xf[(ch * 8 + 2 * oct) * 32 + ln] = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
-      xf[(ch * 8 + 2 * oct + 1) * 32 + ln] = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+    const int rot = (int)(((int64_t)blockIdx.x * 1031) % items);
+    for (int base = ct; base < items; base += nct * XB) {
+      uint4 v[XB];
+#pragma unroll
+      for (int b = 0; b < XB; ++b) {
+        int it = base + b * nct;
+        if (it < items) {
+          it = it + rot < items ? it + rot : it + rot - items;
+          const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
+          const int gg = ln >> 2, cc = ln & 3;
+          v[b] = xoct<T>(p, gg, (int64_t)ch * 128 + 32 * cc + 8 * oct, gg < p.M);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < XB; ++b) {
+        int it = base + b * nct;
+        if (it < items) {
+          it = it + rot < items ? it + rot : it + rot - items;
+          const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
+          xf[(ch * 8 + 2 * oct) * 32 + ln] = make_uint2(__byte_perm(v[b].x, v[b].z, 0x5410), __byte_perm(v[b].x, v[b].z, 0x7632));
+          xf[(ch * 8 + 2 * oct + 1) * 32 + ln] = make_uint2(__byte_perm(v[b].y, v[b].w, 0x5410), __byte_perm(v[b].y, v[b].w, 0x7632));
+        }
+      }
     }
   } else {
-    // entry (window, lane) of 16 bytes: x[g][32 w + 2c + 8i + {0,1}], i = 0..3
+    // item = (window w, token g): x[g][32w, 32w + 32) as four octs; the entry of lane 4g + c is
+    // word c of each oct, i.e. x[g][32w + 2c + 8i + {0,1}], i = 0..3
     uint4* xf = reinterpret_cast<uint4*>(xs);
-    const int items = (int)(p.K / 32) * 32;
-    for (int it = ct; it < items; it += nct) {
-      const int ln = it & 31, w = it >> 5;
-      const int gg = ln >> 2, cc = ln & 3;
-      uint32_t q4[4];
+    const int items = (int)(p.K / 32) * 8;
+    const int rot = (int)(((int64_t)blockIdx.x * 257) % items);
+    constexpr int IB = XB / 4;
+    for (int base = ct; base < items; base += nct * IB) {
+      uint4 v[IB][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t k = 32 * (int64_t)w + 2 * cc + 8 * i;
-        q4[i] = xval<T>(p, gg, k, gg < p.M) | (xval<T>(p, gg, k + 1, gg < p.M) << 16);
+      for (int b = 0; b < IB; ++b) {
+        int it = base + b * nct;
+        if (it < items) {
+          it = it + rot < items ? it + rot : it + rot - items;
+          const int gg = it & 7, w = it >> 3;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[b][i] = xoct<T>(p, gg, 32 * (int64_t)w + 8 * i, gg < p.M);
+        }
       }
-      xf[it] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+#pragma unroll
+      for (int b = 0; b < IB; ++b) {
+        int it = base + b * nct;
+        if (it < items) {
+          it = it + rot < items ? it + rot : it + rot - items;
+          const int gg = it & 7, w = it >> 3;
+          uint4* e = xf + w * 32 + 4 * gg;
+          e[0] = make_uint4(v[b][0].x, v[b][1].x, v[b][2].x, v[b][3].x);
+          e[1] = make_uint4(v[b][0].y, v[b][1].y, v[b][2].y, v[b][3].y);
+          e[2] = make_uint4(v[b][0].z, v[b][1].z, v[b][2].z, v[b][3].z);
+          e[3] = make_uint4(v[b][0].w, v[b][1].w, v[b][2].w, v[b][3].w);
+        }
+      }
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(nct) : "memory");  // consumers only
@@ -583,16 +620,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int r0 = prow(g), r1 = prow(g + 8);
   float scale = 256.0f * *p.w_ts;
   if (p.x_fmt == X_Q4) scale *= *p.x_ts;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
   int64_t cur = -1;
   int cnt = 0;
 
   auto flush = [&](int64_t tile) {
     float* b = &tbuf[tile & 3][0][0];
-    atomicAdd(b + r0 * 8 + 2 * c, acc[0]);
-    atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1]);
-    atomicAdd(b + r1 * 8 + 2 * c, acc[2]);
-    atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3]);
+    atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
+    atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
+    atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
+    atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
     __threadfence_block();
     __syncwarp();
     int last = 0;
@@ -614,6 +651,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (lane == 0) tdone[tile & 3] = 0;
     }
     acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    acc2[0] = acc2[1] = acc2[2] = acc2[3] = 0.f;
     cnt = 0;
   };
 
@@ -631,31 +669,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const uint8_t* d = slots + sl * U::SLOT;
     const uint8_t* sc = d + U::CODES;
     if constexpr (WF == W_DQ4) {
+      // the two 128-K chunks of the unit feed two independent accumulator chains
       const uint2* xf = reinterpret_cast<const uint2*>(xs);
+      uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int j = 4 * ch + c;
         const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
         const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
-        uint32_t s00, s01, s10, s11;
-        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), s00, s01);
-        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), s10, s11);
-        const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
-        const int64_t gch = kp * 2 + ch;
+        w0[ch][0] = v0.x; w0[ch][1] = v0.y; w0[ch][2] = v0.z; w0[ch][3] = v0.w;
+        w1[ch][0] = v1.x; w1[ch][1] = v1.y; w1[ch][2] = v1.z; w1[ch][3] = v1.w;
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), sa[ch][0], sa[ch][1]);
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), sb[ch][0], sb[ch][1]);
+      }
 #pragma unroll
-        for (int st = 0; st < 8; ++st) {
-          const int q = st >> 1, i0 = 2 * (st & 1);
-          const uint32_t sa = st < 4 ? s00 : s01, sb = st < 4 ? s10 : s11;
-          const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0), sa);
-          const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[q], i0 + 1), sa);
-          const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0), sb);
-          const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0 + 1), sb);
-          float acc4[4] = {acc[0], acc[1], acc[2], acc[3]};
-          mma_k16<T>(acc4, a0, a1, a2, a3, xf[(gch * 8 + st) * 32 + lane]);
-          acc[0] = acc4[0]; acc[1] = acc4[1]; acc[2] = acc4[2]; acc[3] = acc4[3];
+      for (int st = 0; st < 8; ++st) {
+        const int q = st >> 1, i0 = 2 * (st & 1);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const uint32_t s0 = sa[ch][st >> 2], s1 = sb[ch][st >> 2];
+          const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], i0), s0);
+          const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], i0 + 1), s0);
+          const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], i0), s1);
+          const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], i0 + 1), s1);
+          mma_k16<T>(ch ? acc2 : acc, a0, a1, a2, a3, xf[((kp * 2 + ch) * 8 + st) * 32 + lane]);
         }
       }
     } else {
+      // even and odd windows feed two independent accumulator chains
       const uint4* xf = reinterpret_cast<const uint4*>(xs);
       const uint8_t* me = sc + U::SCALES;
 #pragma unroll 4
@@ -674,9 +715,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
         const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
         const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
-        float acc4[4] = {acc[0], acc[1], acc[2], acc[3]};
-        mma_sp_k32<T>(acc4, a0, a1, a2, a3, xf[(kp * 16 + w) * 32 + lane], e);
-        acc[0] = acc4[0]; acc[1] = acc4[1]; acc[2] = acc4[2]; acc[3] = acc4[3];
+        mma_sp_k32<T>((w & 1) ? acc2 : acc, a0, a1, a2, a3, xf[(kp * 16 + w) * 32 + lane], e);
       }
     }
     __syncwarp();

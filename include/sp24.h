@@ -169,6 +169,30 @@ int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,
                           const float* tensor_scale, int64_t rows, int64_t cols, int out_dtype,
                           void* out, void* stream);
 
+/* ----------------------------------------------------------------------- a1-a3 in one read */
+/* Prepares a matmul weight W[rows, K] (K % 16 == 0) with a single read of W: the outputs equal,
+ * bit for bit, those of
+ *   sp24_check_24(W)            -> pass, n_fail
+ *   sp24_prune_compress_24(W)   -> values [rows, K/2], meta [rows, K/8]
+ * plus the two tensor scales sp24_quantize_nvfp4 derives when given none:
+ *   w_tensor_scale = amax|W| / 2688,  v_tensor_scale = amax|values| / 2688.
+ * Passing those scales to sp24_quantize_nvfp4 (tensor_scale_in) then gives the NVFP4 encodings
+ * of W and of the values without another amax pass, identical to the unscaled calls.  [P1]
+ * "What 2:4 actually is" and [P5] "Convert BF16 to NVFP4 yourself" define the steps; the pages
+ * run them one after the other, this call fuses their reads of W.
+ *   w          device, F16/BF16/F32, 16-byte aligned
+ *   pass       device [rows, K/4] bytes (2-byte aligned) or NULL
+ *   n_fail     device int32 or NULL
+ *   values     device, dtype, [rows, K/2], 8-byte aligned;  meta: device [rows, K/8] bytes
+ *   w_tensor_scale, v_tensor_scale   device fp32 or NULL
+ *   workspace  device, >= sp24_prepare_24_workspace_size() bytes, 16-byte aligned; scratch.
+ * One memset and one streaming kernel; an empty W gives n_fail 0 and scales 0. */
+int sp24_prepare_24_workspace_size(int64_t rows, int64_t K, int64_t* bytes);
+int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* pass,
+                    int32_t* n_fail, void* values, uint8_t* meta, float* w_tensor_scale,
+                    float* v_tensor_scale, void* workspace, int64_t workspace_bytes,
+                    void* stream);
+
 /* ----------------------------------------------------------------------- a4-a6: GEMM */
 /* Y[m, n] = sum_k x[m, k] * w[n, k] with fp32 accumulation, Y fp32 [M, N] row-major (device).
  * x: M rows (F16, BF16 or NVFP4); w: N rows (F16, BF16 or NVFP4).  16-bit x and 16-bit w
