@@ -56,9 +56,11 @@ int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
       q.x = reinterpret_cast<const uint8_t*>(p.x) + m0 * p.K / 2;
       q.x_scales = p.x_scales + m0 * p.K / 16;
     }
-    int st = decode_supported(wf, q)    ? decode_gemv(wf, t16, q, s)
-             : skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s)
-                                        : skinny_gemm(wf, t16, q, s);
+    // the decode kernel declines (SP24_ERR_UNSUPPORTED, nothing launched) when the driver
+    // refuses its x tensor map
+    int st = decode_supported(wf, q) ? decode_gemv(wf, t16, q, s) : SP24_ERR_UNSUPPORTED;
+    if (st == SP24_ERR_UNSUPPORTED)
+      st = skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s) : skinny_gemm(wf, t16, q, s);
     if (st) return st;
   }
   return SP24_OK;

@@ -49,13 +49,31 @@ struct Group16 {
   uint32_t kept;  // v0 | v1 << 16
 };
 
-__device__ __forceinline__ Group16 prune16(uint32_t lo, uint32_t hi) {
-  uint32_t m = keep_mask(mag16(lo), mag16(lo >> 16), mag16(hi), mag16(hi >> 16));
+// Sort keys of a group of four 16-bit entries held as lo = e0 | e1 << 16, hi = e2 | e3 << 16:
+// key = magnitude bits << 2 | (3 - index), so a larger key means a larger |w|, or an equal |w|
+// at a lower index (the pruning order), and the four keys all differ.  A min/max network gives
+// the largest three: k1 and k2 are the kept members, and the group has at least two zeros
+// exactly when k3 < 4 (a magnitude of 0).
+struct Keys4 {
+  uint32_t k1, k2, k3, k4;
+};
+
+__device__ __forceinline__ Keys4 sort_keys16(uint32_t lo, uint32_t hi) {
+  const uint32_t a = ((lo & 0x7fffu) << 2) | 3u, b = ((lo >> 14) & 0x1fffcu) | 2u;
+  const uint32_t c = ((hi & 0x7fffu) << 2) | 1u, d = (hi >> 14) & 0x1fffcu;
+  const uint32_t m01 = max(a, b), n01 = min(a, b), m23 = max(c, d), n23 = min(c, d);
+  const uint32_t x = min(m01, m23), y = max(n01, n23);
+  return Keys4{max(m01, m23), max(x, y), min(x, y), min(n01, n23)};
+}
+
+// Nibble (i0 | i1 << 2, i0 < i1) and kept pair (ascending index) from the two largest keys.
+__device__ __forceinline__ Group16 kept16(const Keys4& k, uint32_t lo, uint32_t hi) {
+  const uint32_t ra = k.k1 & 3u, rb = k.k2 & 3u;      // 3 - index
+  const uint32_t i0 = 3u - max(ra, rb), i1 = 3u - min(ra, rb);
   Group16 g;
-  g.nib = mask_nibble(m);
-  uint32_t i0 = g.nib & 3, i1 = g.nib >> 2;
-  uint32_t sel = (2 * i0) | ((2 * i0 + 1) << 4) | ((2 * i1) << 8) | ((2 * i1 + 1) << 12);
-  g.kept = __byte_perm(lo, hi, sel);
+  g.nib = i0 | (i1 << 2);
+  const uint32_t t = (i0 | (i1 << 8)) * 2u;            // first byte of each kept entry
+  g.kept = __byte_perm(lo, hi, t * 0x11u + 0x1010u);
   return g;
 }
 
@@ -72,6 +90,12 @@ template <int DT>
 __device__ __forceinline__ float abs16(uint32_t bits) {
   if (DT == SP24_BF16) return __uint_as_float((bits & 0x7fffu) << 16);
   return fabsf(__half2float(__ushort_as_half((unsigned short)(bits & 0xffffu))));
+}
+
+// |w| of the 16-bit entry behind a sort key, as fp32 (exact).
+template <int DT>
+__device__ __forceinline__ float key_to_abs(uint32_t key) {
+  return abs16<DT>(key >> 2);
 }
 
 // max(m, |entries of a word|): two 16-bit entries or one fp32.  fmaxf never returns a NaN
@@ -159,7 +183,8 @@ __global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict_
           const int64_t v = v0 + j;
           if (EB == 2) {
             if (live) {
-              const Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
+              const Group16 a = kept16(sort_keys16(x.x, x.y), x.x, x.y);
+              const Group16 b = kept16(sort_keys16(x.z, x.w), x.z, x.w);
               values[v] = make_uint2(a.kept, b.kept);
               meta[v] = (uint8_t)(a.nib | (b.nib << 4));
             }
@@ -192,9 +217,18 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
                                                         int32_t* __restrict__ n_fail, float* __restrict__ ts_w,
                                                         float* __restrict__ ts_v) {
   constexpr int EB = DT == SP24_F32 ? 4 : 2;
+  // largest key of a non-NaN 16-bit entry: +inf's magnitude, index 0
+  constexpr uint32_t kNaNKey = ((DT == SP24_BF16 ? 0x7f80u : 0x7c00u) << 2) | 3u;
+  auto below_nan = [&](const Keys4& k) {  // largest non-NaN key of a group whose k1 is NaN
+    return k.k2 <= kNaNKey ? k.k2 : (k.k3 <= kNaNKey ? k.k3 : (k.k4 <= kNaNKey ? k.k4 : 0u));
+  };
+  auto kept_below_nan = [&](const Keys4& k) {
+    return k.k1 <= kNaNKey ? k.k1 : (k.k2 <= kNaNKey ? k.k2 : 0u);
+  };
   extern __shared__ __align__(128) uint8_t ring[];
   int fails = 0;
-  float mw = 0.0f, mv = 0.0f;
+  float mw = 0.0f, mv = 0.0f;  // fp32 weights
+  uint32_t kw = 0, kv = 0;     // 16-bit weights: keys
   stream::for_each_chunk<kChunk, kStages>(
       reinterpret_cast<const uint8_t*>(w), nv * 16, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
         const uint4* cv = reinterpret_cast<const uint4*>(chunk);
@@ -206,17 +240,18 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
           const bool live = j < nvec;
           const uint4 x = live ? cv[j] : make_uint4(0, 0, 0, 0);
           const int64_t v = v0 + j;
-          mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.x), x.y);
-          mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.z), x.w);
           if (EB == 2) {
             if (live) {
-              const int ok0 = zeros16(x.x, x.y) >= 2, ok1 = zeros16(x.z, x.w) >= 2;
+              const Keys4 ka = sort_keys16(x.x, x.y), kb = sort_keys16(x.z, x.w);
+              const int ok0 = ka.k3 < 4u, ok1 = kb.k3 < 4u;
               fails += 2 - ok0 - ok1;
               if (pass) reinterpret_cast<uint16_t*>(pass)[v] = (uint16_t)(ok0 | (ok1 << 8));
-              const Group16 a = prune16(x.x, x.y), b = prune16(x.z, x.w);
+              const Group16 a = kept16(ka, x.x, x.y), b = kept16(kb, x.z, x.w);
               values[v] = make_uint2(a.kept, b.kept);
               meta[v] = (uint8_t)(a.nib | (b.nib << 4));
-              mv = max_abs_word<DT>(max_abs_word<DT>(mv, a.kept), b.kept);
+              // amax over non-NaN entries, on keys (magnitude order); NaN sorts highest
+              kw = max(kw, max(ka.k1 <= kNaNKey ? ka.k1 : below_nan(ka), kb.k1 <= kNaNKey ? kb.k1 : below_nan(kb)));
+              kv = max(kv, max(kept_below_nan(ka), kept_below_nan(kb)));
             }
           } else {
             const uint32_t nib = mask_nibble(keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w)));
@@ -231,11 +266,17 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
               if (pass) pass[v] = (uint8_t)ok;
               values[v] = make_uint2(e0, e1);
               if ((v & 1) == 0) meta[v >> 1] = (uint8_t)(nib | (other << 4));  // nv is even
+              mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.x), x.y);
+              mw = max_abs_word<DT>(max_abs_word<DT>(mw, x.z), x.w);
               mv = max_abs_word<DT>(max_abs_word<DT>(mv, e0), e1);
             }
           }
         }
       });
+  if constexpr (EB == 2) {
+    mw = key_to_abs<DT>(kw);
+    mv = key_to_abs<DT>(kv);
+  }
   count_fails(fails, reinterpret_cast<int32_t*>(acc + 2));
   block_max_to(mw, acc);
   block_max_to(mv, acc + 1);

@@ -463,20 +463,24 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
 
 // ------------------------------------------------------------------ persistent decode GEMV (M <= 8)
 //
-// One CTA per SM: a producer warp streams 16-row weight units (2-D TMA: codes with the 128-byte
-// swizzle, block scales and 2:4 nibbles unswizzled) through a ring of shared-memory slots, and 8
-// consumer warps take the units round-robin.  x (M <= 8 tokens) is staged once per CTA for the
-// whole K in fragment order.  Units are spread evenly over all CTAs (each CTA a contiguous range
-// in tile-major order), so every SM streams the same number of bytes; a warp's partial sums of a
-// 16-row tile are added into one of four shared tile buffers, and the last warp of the CTA to
-// finish a tile adds the buffer into y (zeroed first) with one atomic per output.
+// One CTA per SM: a producer warp first loads x (M <= 8 tokens, whole K) with 2-D TMA into
+// shared memory (boxes of 64 k x 8 tokens with the 128-byte swizzle; token rows past M read as
+// zeros), then streams 16-row weight units (codes with the 128-byte swizzle, block scales and
+// 2:4 nibbles unswizzled) through a ring of slots; 16 consumer warps take the units
+// round-robin.  Units are spread evenly over the CTAs (each CTA a contiguous range in
+// tile-major order), so every SM streams the same number of bytes.  A warp adds its partial
+// sums of a 16-row tile into that tile's shared buffer whenever its next unit belongs to another
+// tile; when all units are done the CTA adds its buffers into y (zeroed first) with one atomic
+// per output, which also joins tiles split between neighbouring CTAs.
 //
-// MMA row m of a warp reads tile row prow(m) = (m/2) + 4 (m%2) (+8 for m >= 8): in every group of
-// 8 lanes sharing a shared-memory phase, the two rows then sit 4 rows apart, so the 128-byte
-// swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)) puts their pieces in disjoint
-// halves of the banks.
-constexpr int kDecConsumers = 8;
+// B fragments are read straight from the swizzled x: in every 8-lane shared-memory phase the
+// 16-byte pieces of different tokens sit in different chunks (chunk j of token g at j ^ g), so
+// the reads are conflict free.  MMA row m of a warp reads tile row prow(m) = (m/2) + 4 (m%2)
+// (+8 for m >= 8), which puts the two rows of a phase in disjoint bank halves of the swizzled
+// weight codes.
+constexpr int kDecConsumers = 16;
 constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+constexpr int kDecMaxTiles = 32;  // per-CTA tile buffers (16 rows x 8 tokens fp32 each)
 
 template <int WF>
 struct U3;
@@ -491,47 +495,64 @@ struct U3<W_SQ4> {  // 512 K per unit: codes 16 x 128 B, scales 16 x 16 B, nibbl
 
 __device__ __forceinline__ int prow(int m) { return (m & 8) + ((m & 7) >> 1) + 4 * (m & 1); }
 
+// Byte offset in the swizzled x of token g, column k (k % 8 == 0): box k / 64 of 1 KB, token
+// row of 128 B, 16-byte chunk (k % 64) / 8 stored at chunk ^ g.
+__device__ __forceinline__ uint32_t xoff(int g, int64_t k) {
+  return (uint32_t)((k >> 6) * 1024 + g * 128 + ((((int)(k >> 3) & 7) ^ g) << 4));
+}
+
 template <int WF, typename T>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_gemv_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
-                       const __grid_constant__ CUtensorMap tmM, const SkinnyParams p) {
+                       const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmX,
+                       const SkinnyParams p) {
   using U = U3<WF>;
   constexpr int S = U::SLOTS;
   extern __shared__ uint8_t dsm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
   uint8_t* slots = base;                              // S x SLOT, 1024-aligned
-  uint8_t* xs = base + S * U::SLOT;                   // x fragments, 16 * K bytes
-  __shared__ uint64_t full_bar[S], empty_bar[S];
-  __shared__ float tbuf[4][16][8];
-  __shared__ int tdone[4];
+  uint8_t* xs = base + S * U::SLOT;                   // x, 16 * K bytes, 1024-aligned
+  __shared__ uint64_t full_bar[S], empty_bar[S], x_bar;
+  __shared__ float tbuf[kDecMaxTiles][16][8];
+  __shared__ int issued, abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t upr = p.K / U::UK;                    // units per 16-row tile
   const int64_t U_all = ((p.N + 15) / 16) * upr;
   const int64_t ub = U_all * blockIdx.x / gridDim.x, ue = U_all * (blockIdx.x + 1) / gridDim.x;
   const int nunits = (int)(ue - ub);
+  const int64_t t0 = ub / upr;
+  const int nloc = nunits > 0 ? (int)((ue - 1) / upr - t0 + 1) : 0;  // <= kDecMaxTiles (host check)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       tc::mbar_init(&full_bar[i], 1);
       tc::mbar_init(&empty_bar[i], 1);
     }
+    tc::mbar_init(&x_bar, 1);
+    issued = 0;
+    abort_flag = 0;
     tc::fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < 4 * 16 * 8; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
-  if (threadIdx.x < 4) tdone[threadIdx.x] = 0;
+  for (int i = threadIdx.x; i < nloc * 128; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
   __syncthreads();
 
   if (warp == 0) {
-    // ---- producer
-    if (lane == 0) {
+    // ---- producer: x, then the weight units
+    if (lane == 0 && nunits > 0) {
+      tc::prefetch_tmap(&tmX);
       tc::prefetch_tmap(&tmC);
       tc::prefetch_tmap(&tmS);
       if (U::META) tc::prefetch_tmap(&tmM);
-      for (int i = 0; i < nunits; ++i) {
+      const int nbox = (int)(p.K / 64);
+      mbar_arrive_expect_tx(&x_bar, (uint32_t)nbox * 1024u);
+      for (int b = 0; b < nbox; ++b) tc::tma_load_2d(xs + b * 1024, &tmX, &x_bar, b * 64, 0);
+      int i = 0;
+      for (; i < nunits; ++i) {
         const int sl = i % S;
         if (!mbar_wait(&empty_bar[sl], ((i / S) & 1) ^ 1)) {
           set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+          abort_flag = 1;
           break;
         }
         const int64_t u = ub + i, tile = u / upr, kp = u % upr;
@@ -541,194 +562,130 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         tc::tma_load_2d(d + U::CODES, &tmS, &full_bar[sl], (int)(kp * 16), (int)(tile * 16));
         if (U::META) tc::tma_load_2d(d + U::CODES + U::SCALES, &tmM, &full_bar[sl], (int)(kp * 64), (int)(tile * 16));
       }
+      issued = i;
     }
-    return;
-  }
-
-  // ---- x for the whole K, fragment order (all consumer threads).  Every CTA reads the same x,
-  // so each starts at its own rotation of the items, and each thread issues XB loads before it
-  // stores any: the staging costs a few L2 round trips instead of one per item.
-  const int ct = threadIdx.x - 32, nct = blockDim.x - 32;
-  constexpr int XB = 8;
-  if (WF == W_DQ4) {
-    // item = (chunk, lane, oct): 8 consecutive k of a lane piece -> two 8-byte fragment entries
-    uint2* xf = reinterpret_cast<uint2*>(xs);
-    const int items = (int)(p.K / 128) * 32 * 4;
-    const int rot = (int)(((int64_t)blockIdx.x * 1031) % items);
-    for (int base = ct; base < items; base += nct * XB) {
-      uint4 v[XB];
+  } else if (nunits > 0) {
+    // ---- consumers
+    const int cw = warp - 1;
+    const int g = lane >> 2, c = lane & 3;
+    const int r0 = prow(g), r1 = prow(g + 8);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+    int64_t cur = -1;
+    auto flush = [&]() {
+      float* b = &tbuf[cur - t0][0][0];
+      atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
+      atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
+      atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
+      atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
 #pragma unroll
-      for (int b = 0; b < XB; ++b) {
-        int it = base + b * nct;
-        if (it < items) {
-          it = it + rot < items ? it + rot : it + rot - items;
-          const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
-          const int gg = ln >> 2, cc = ln & 3;
-          v[b] = xoct<T>(p, gg, (int64_t)ch * 128 + 32 * cc + 8 * oct, gg < p.M);
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < XB; ++b) {
-        int it = base + b * nct;
-        if (it < items) {
-          it = it + rot < items ? it + rot : it + rot - items;
-          const int oct = it & 3, ln = (it >> 2) & 31, ch = it >> 7;
-          xf[(ch * 8 + 2 * oct) * 32 + ln] = make_uint2(__byte_perm(v[b].x, v[b].z, 0x5410), __byte_perm(v[b].x, v[b].z, 0x7632));
-          xf[(ch * 8 + 2 * oct + 1) * 32 + ln] = make_uint2(__byte_perm(v[b].y, v[b].w, 0x5410), __byte_perm(v[b].y, v[b].w, 0x7632));
-        }
-      }
-    }
-  } else {
-    // item = (window w, token g): x[g][32w, 32w + 32) as four octs; the entry of lane 4g + c is
-    // word c of each oct, i.e. x[g][32w + 2c + 8i + {0,1}], i = 0..3
-    uint4* xf = reinterpret_cast<uint4*>(xs);
-    const int items = (int)(p.K / 32) * 8;
-    const int rot = (int)(((int64_t)blockIdx.x * 257) % items);
-    constexpr int IB = XB / 4;
-    for (int base = ct; base < items; base += nct * IB) {
-      uint4 v[IB][4];
-#pragma unroll
-      for (int b = 0; b < IB; ++b) {
-        int it = base + b * nct;
-        if (it < items) {
-          it = it + rot < items ? it + rot : it + rot - items;
-          const int gg = it & 7, w = it >> 3;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) v[b][i] = xoct<T>(p, gg, 32 * (int64_t)w + 8 * i, gg < p.M);
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < IB; ++b) {
-        int it = base + b * nct;
-        if (it < items) {
-          it = it + rot < items ? it + rot : it + rot - items;
-          const int gg = it & 7, w = it >> 3;
-          uint4* e = xf + w * 32 + 4 * gg;
-          e[0] = make_uint4(v[b][0].x, v[b][1].x, v[b][2].x, v[b][3].x);
-          e[1] = make_uint4(v[b][0].y, v[b][1].y, v[b][2].y, v[b][3].y);
-          e[2] = make_uint4(v[b][0].z, v[b][1].z, v[b][2].z, v[b][3].z);
-          e[3] = make_uint4(v[b][0].w, v[b][1].w, v[b][2].w, v[b][3].w);
-        }
-      }
-    }
-  }
-  asm volatile("bar.sync 1, %0;" ::"r"(nct) : "memory");  // consumers only
-
-  // ---- consumers
-  const int cw = warp - 1;
-  const int g = lane >> 2, c = lane & 3;
-  const int r0 = prow(g), r1 = prow(g + 8);
-  float scale = 256.0f * *p.w_ts;
-  if (p.x_fmt == X_Q4) scale *= *p.x_ts;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-  int64_t cur = -1;
-  int cnt = 0;
-
-  auto flush = [&](int64_t tile) {
-    float* b = &tbuf[tile & 3][0][0];
-    atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
-    atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
-    atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
-    atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
-    __threadfence_block();
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      const int64_t lo = tile * upr > ub ? tile * upr : ub, hi = (tile + 1) * upr < ue ? (tile + 1) * upr : ue;
-      last = atomicAdd(&tdone[tile & 3], cnt) + cnt == (int)(hi - lo);
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      __threadfence_block();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = lane + 32 * q, row = e >> 3, tok = e & 7;
-        const int64_t gr = tile * 16 + row;
-        if (tok < p.M && gr < p.N) atomicAdd(p.y + (int64_t)tok * p.N + gr, b[e] * scale);
-        b[e] = 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) tdone[tile & 3] = 0;
-    }
-    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-    acc2[0] = acc2[1] = acc2[2] = acc2[3] = 0.f;
-    cnt = 0;
-  };
-
-  for (int i = cw; i < nunits; i += kDecConsumers) {
-    const int sl = i % S;
-    const int64_t u = ub + i, tile = u / upr, kp = u % upr;
-    if (tile != cur) {
-      if (cur >= 0) flush(cur);
-      cur = tile;
-    }
-    if (!mbar_wait(&full_bar[sl], (i / S) & 1)) {
+      for (int q = 0; q < 4; ++q) acc[q] = acc2[q] = 0.f;
+    };
+    bool ok = mbar_wait(&x_bar, 0);
+    if (!ok) {
       set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-      break;
+      abort_flag = 1;
     }
-    const uint8_t* d = slots + sl * U::SLOT;
-    const uint8_t* sc = d + U::CODES;
-    if constexpr (WF == W_DQ4) {
-      // the two 128-K chunks of the unit feed two independent accumulator chains
-      const uint2* xf = reinterpret_cast<const uint2*>(xs);
-      uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int j = 4 * ch + c;
-        const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
-        const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
-        w0[ch][0] = v0.x; w0[ch][1] = v0.y; w0[ch][2] = v0.z; w0[ch][3] = v0.w;
-        w1[ch][0] = v1.x; w1[ch][1] = v1.y; w1[ch][2] = v1.z; w1[ch][3] = v1.w;
-        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), sa[ch][0], sa[ch][1]);
-        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), sb[ch][0], sb[ch][1]);
+    for (int i = cw; ok && i < nunits; i += kDecConsumers) {
+      const int sl = i % S;
+      const int64_t u = ub + i, tile = u / upr, kp = u % upr;
+      if (tile != cur) {
+        if (cur >= 0) flush();
+        cur = tile;
       }
-#pragma unroll
-      for (int st = 0; st < 8; ++st) {
-        const int q = st >> 1, i0 = 2 * (st & 1);
+      if (!mbar_wait(&full_bar[sl], (i / S) & 1)) {
+        set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+        abort_flag = 1;
+        break;
+      }
+      const uint8_t* d = slots + sl * U::SLOT;
+      const uint8_t* sc = d + U::CODES;
+      if constexpr (WF == W_DQ4) {
+        // the unit's two 128-K chunks feed two independent accumulator chains
+        uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          const uint32_t s0 = sa[ch][st >> 2], s1 = sb[ch][st >> 2];
-          const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], i0), s0);
-          const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], i0 + 1), s0);
-          const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], i0), s1);
-          const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], i0 + 1), s1);
-          mma_k16<T>(ch ? acc2 : acc, a0, a1, a2, a3, xf[((kp * 2 + ch) * 8 + st) * 32 + lane]);
+          const int j = 4 * ch + c;
+          const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
+          const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
+          w0[ch][0] = v0.x; w0[ch][1] = v0.y; w0[ch][2] = v0.z; w0[ch][3] = v0.w;
+          w1[ch][0] = v1.x; w1[ch][1] = v1.y; w1[ch][2] = v1.z; w1[ch][3] = v1.w;
+          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), sa[ch][0], sa[ch][1]);
+          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), sb[ch][0], sb[ch][1]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            // x[g][P .. P+8), P = chunk base + 32c + 8q: codes at nibbles (i, i+4) of word q
+            // pair with x entries (i, i+4)
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff(g, kp * 256 + ch * 128 + 32 * c + 8 * q));
+            const uint32_t s0 = sa[ch][q >> 1], s1 = sb[ch][q >> 1];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
+              const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
+              const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h), s0);
+              const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h + 1), s0);
+              const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h), s1);
+              const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h + 1), s1);
+              mma_k16<T>(ch ? acc2 : acc, a0, a1, a2, a3, bx);
+            }
+          }
+        }
+      } else {
+        // even and odd windows feed two independent accumulator chains
+        const uint8_t* me = sc + U::SCALES;
+#pragma unroll 4
+        for (int w = 0; w < 16; ++w) {
+          const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * 64 + 4 * w);
+          const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * 64 + 4 * w);
+          const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
+          const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * 128 + (((w >> 1) ^ (r0 & 7)) << 4) + 8 * (w & 1));
+          const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * 128 + (((w >> 1) ^ (r1 & 7)) << 4) + 8 * (w & 1));
+          uint32_t s0, s1, unused;
+          scale_pair<T>(sc[r0 * 16 + w], s0, unused);
+          scale_pair<T>(sc[r1 * 16 + w], s1, unused);
+          const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
+          const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
+          const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+          const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+          const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+          const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+          // x[g][32w' + 2c + 8i + {0, 1}], i = 0..3: word c of four consecutive 16-byte pieces
+          const int64_t kw = kp * 512 + 32 * w;
+          const uint8_t* xr = xs + 4 * c;
+          const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr + xoff(g, kw)),
+                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 8)),
+                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 16)),
+                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 24)));
+          mma_sp_k32<T>((w & 1) ? acc2 : acc, a0, a1, a2, a3, bx, e);
         }
       }
-    } else {
-      // even and odd windows feed two independent accumulator chains
-      const uint4* xf = reinterpret_cast<const uint4*>(xs);
-      const uint8_t* me = sc + U::SCALES;
-#pragma unroll 4
-      for (int w = 0; w < 16; ++w) {
-        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * 64 + 4 * w);
-        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * 64 + 4 * w);
-        const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
-        const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * 128 + (((w >> 1) ^ (r0 & 7)) << 4) + 8 * (w & 1));
-        const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * 128 + (((w >> 1) ^ (r1 & 7)) << 4) + 8 * (w & 1));
-        uint32_t s0, s1, unused;
-        scale_pair<T>(sc[r0 * 16 + w], s0, unused);
-        scale_pair<T>(sc[r1 * 16 + w], s1, unused);
-        const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
-        const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
-        const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
-        const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
-        const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
-        const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
-        mma_sp_k32<T>((w & 1) ? acc2 : acc, a0, a1, a2, a3, xf[(kp * 16 + w) * 32 + lane], e);
-      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
     }
-    __syncwarp();
-    if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
-    ++cnt;
+    if (cur >= 0) flush();
   }
-  if (cur >= 0) flush(cur);
+  __syncthreads();
+  // a gave-up wait may leave copies in flight: let them land before the CTA's memory goes away
+  if (abort_flag && threadIdx.x == 0) {
+    tc::mbar_wait(&x_bar, 0);
+    for (int i = issued > S ? issued - S : 0; i < issued; ++i) tc::mbar_wait(&full_bar[i % S], (i / S) & 1);
+  }
+  // ---- the CTA's tile sums into y
+  float scale = 256.0f * *p.w_ts;
+  for (int e = threadIdx.x; e < nloc * 128; e += blockDim.x) {
+    const int lt = e >> 7, row = (e >> 3) & 15, tok = e & 7;
+    const int64_t gr = (t0 + lt) * 16 + row;
+    const float v = (&tbuf[0][0][0])[e];
+    if (tok < p.M && gr < p.N && v != 0.0f) atomicAdd(p.y + (int64_t)tok * p.N + gr, v * scale);
+  }
 }
 
 template <int WF, typename T>
 int launch_decode(const SkinnyParams& p, cudaStream_t s) {
   using U = U3<WF>;
-  CUtensorMap tc_, ts_, tm_;
+  CUtensorMap tc_, ts_, tm_, tx_;
   const int64_t cb = WF == W_DQ4 ? p.K / 2 : p.K / 4;
   int st = make_tmap_2d(&tc_, p.w, 1, p.N, cb, cb, 128, 16);
   if (st) return st;
@@ -741,12 +698,14 @@ int launch_decode(const SkinnyParams& p, cudaStream_t s) {
   } else {
     tm_ = ts_;
   }
+  // x rows past M (up to the 8-row box) read as zeros
+  if (make_tmap_2d(&tx_, p.x, 2, p.M, p.K, p.K * 2, 64, 8)) return SP24_ERR_UNSUPPORTED;
   const size_t smem = 1024 + (size_t)U::SLOTS * U::SLOT + 16 * (size_t)p.K;
   auto kern = decode_gemv_kernel<WF, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   if (cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
-  kern<<<sm_count(), kDecThreads, smem, s>>>(tc_, ts_, tm_, p);
+  kern<<<sm_count(), kDecThreads, smem, s>>>(tc_, ts_, tm_, tx_, p);
   return launch_status();
 }
 
@@ -771,15 +730,21 @@ int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStre
   return SP24_ERR_UNSUPPORTED;
 }
 
-// True when the persistent decode kernel takes the problem: NVFP4 weights (dense or 2:4), at most
-// 8 tokens, whole 16-row tiles, K a whole number of units and small enough for x to stay in
-// shared memory (16 K bytes of fragments).
+// True when the persistent decode kernel takes the problem: 16-bit x of at most 8 tokens (TMA
+// rows: 16-byte aligned, K % 64), NVFP4 weights (dense or 2:4) in whole 16-row tiles, K a whole
+// number of units and small enough for x to stay in shared memory (16 K bytes), and at most
+// kDecMaxTiles tiles touched by any CTA.
 bool decode_supported(int wf, const SkinnyParams& p) {
-  if (p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0 || p.K > 8192) return false;
-  if (!aligned(p.w, 16) || !aligned(p.w_scales, 16)) return false;
-  if (wf == W_DQ4) return p.K % 256 == 0;
-  if (wf == W_SQ4) return p.K % 512 == 0 && aligned(p.meta, 16);
-  return false;
+  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0 || p.K > 8192) return false;
+  if (!aligned(p.x, 16) || !aligned(p.w, 16) || !aligned(p.w_scales, 16)) return false;
+  int64_t uk;
+  if (wf == W_DQ4) uk = U3<W_DQ4>::UK;
+  else if (wf == W_SQ4 && aligned(p.meta, 16)) uk = U3<W_SQ4>::UK;
+  else return false;
+  if (p.K % uk) return false;
+  const int64_t upr = p.K / uk, units = (p.N / 16) * upr, grid = sm_count();
+  const int64_t per_cta = (units + grid - 1) / grid;
+  return per_cta / upr + 2 <= kDecMaxTiles;
 }
 
 int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s) {
