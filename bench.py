@@ -536,6 +536,31 @@ def run_sweep(args) -> None:
                           "compress": {"us": round(us_p, 3), "GB/s": round((nb + vals.numel() * 2 + meta.numel()) / us_p / 1e3, 1)},
                           "n_fail": int(nf.item())}), flush=True)
 
+    # routed experts: 4096 tokens x top-10 of 512 experts [512, 2048], bf16 x, NVFP4 experts
+    # (dense, and 2:4 of the same experts); every expert is touched, so each call reads all of
+    # them once (one copy: 302 MB dense / 218 MB 2:4, well beyond L2)
+    d = synth.moe()
+    E, Ne, Ke = d["W"].shape
+    xm = t16(d["X"], "bf16")
+    rt = torch.from_numpy(d["routing"]).to(dev)
+    wm = t16(d["W"].reshape(E * Ne, Ke), "bf16")
+    del d
+    _, wq, sw = sp.prepare_nvfp4_24(wm)
+    del wm
+    ym = torch.empty((rt.shape[0], rt.shape[1], Ne), dtype=torch.float32, device=dev)
+    T, topk = rt.shape
+    fl = 2.0 * T * topk * Ne * Ke
+    xy = T * Ke * 2 + T * topk * Ne * 4 + T * topk * 4
+    line = {"sweep": "moe_grouped", "experts": E, "expert_shape": [Ne, Ke], "tokens": T, "topk": topk,
+            "x": "bf16", "w": "nvfp4"}
+    for name, wop in (("dense", wq), ("sparse24", sw)):
+        us = timeit(lambda r: sp.gemm_grouped(xm, rt, wop, E, Ne, Ke, out=ym), reps=5)
+        byt = op_bytes(wop) + xy
+        line[name] = {"us": round(us, 2), "TFLOP/s": round(fl / us / 1e6, 2), "GB/s": round(byt / us / 1e3, 1),
+                      "bytes": byt, "frac_hbm": round(byt / us / 1e3 / peak_hbm, 3)}
+    line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse24"]["us"], 3)
+    print(json.dumps(line), flush=True)
+
 
 def run_ncu_target() -> None:
     """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(192, 1)
   using C = TcCfg<BN>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = tc::align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * C::A_BYTES;
   __shared__ uint64_t full_bar[S], empty_bar[S], tfull_bar;
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(224, 1)
                          const __grid_constant__ CUtensorMap tmE, const TcParams p) {
   constexpr int S = kSpStages, BN = kSpBN;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = tc::align1024(smem_raw);
   // stage s: [A 16 KB][B0 16 KB][B1 16 KB][raw nibbles 2 KB][tcgen05 metadata 2 KB]
   auto sA = [&](int s) { return smem + s * kSpStage; };
   auto sB = [&](int s, int h) { return smem + s * kSpStage + kSpA + h * kSpB; };
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(224, 1)
   using C = QCfg<BN>;
   constexpr int S = kQStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = tc::align1024(smem_raw);
   auto sA = [&](int s) { return smem + s * C::STAGE; };
   auto sB = [&](int s) { return smem + s * C::STAGE + C::A; };
   auto sSAr = [&](int s) { return smem + s * C::STAGE + C::A + C::B; };

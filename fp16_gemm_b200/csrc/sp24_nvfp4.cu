@@ -153,6 +153,15 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
 }
 
 // Encodes one 16-entry block given the tensor scale s_t and d = s_t * 6.
+//
+// The code of an entry is E2M1_rne(fl(|v| / sc)), and only the side of fl(|v| / sc) relative to
+// E2M1's rounding boundaries (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) matters.  With the block's
+// divisor sc in [2^-100, 2^100], q = RN(|v| * RN(1 / sc)) is within 2.01 ulp of |v| / sc (two
+// roundings of 2^-24 each), so q and fl(|v| / sc) give the same code unless q lies within a few
+// ulps of a boundary.  Every boundary has at most three significant bits, i.e. a zero in the low
+// 21 bits of its fp32 significand; an entry whose q is within 4 ulps of such a value (which also
+// covers the power-of-two boundary 0.25, where the ulp halves) takes the IEEE division instead.
+// The codes are therefore exactly those of the per-entry division, at one multiply per entry.
 __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, float d, uint2* codes,
                                              uint8_t* scales, int64_t b) {
   float bmax = 0.0f;
@@ -160,12 +169,29 @@ __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, fl
   for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
   uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
   const float sc = __fmul_rn(e4m3_value(sb), s_t);
+  float q[16];
+  if (sc >= 0x1p-100f && sc <= 0x1p100f) {
+    const float y = __frcp_rn(sc);
+    uint32_t near = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      q[i] = __fmul_rn(fabsf(v[i]), y);
+      const uint32_t u = __float_as_uint(q[i]);
+      near |= (uint32_t)(((u + 4u) & 0x1fffffu) <= 8u && u != 0u) << i;
+    }
+    if (near) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if ((near >> i) & 1u) q[i] = __fdiv_rn(fabsf(v[i]), sc);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
+  }
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
-    float q0 = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
-    float q1 = sc != 0.0f ? __fdiv_rn(fabsf(v[i + 1]), sc) : 0.0f;
-    uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
+    uint32_t byte = e2m1x2_rne_satfinite(q[i], q[i + 1]);
     byte |= (__float_as_uint(v[i]) >> 31) << 3;       // sign of the low entry
     byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;   // sign of the high entry
     packed[i / 8] |= byte << (8 * ((i % 8) / 2));

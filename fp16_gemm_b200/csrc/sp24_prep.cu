@@ -67,13 +67,14 @@ __device__ __forceinline__ Keys4 sort_keys16(uint32_t lo, uint32_t hi) {
 }
 
 // Nibble (i0 | i1 << 2, i0 < i1) and kept pair (ascending index) from the two largest keys.
+// With r = 3 - index, i0 = 3 - max(r) and i1 = 3 - min(r); the byte-permute selector of the
+// pair is 0x1010 + 0x22 i0 + 0x2200 i1 (bytes 2 i0, 2 i0 + 1, 2 i1, 2 i1 + 1 of lo:hi).
 __device__ __forceinline__ Group16 kept16(const Keys4& k, uint32_t lo, uint32_t hi) {
-  const uint32_t ra = k.k1 & 3u, rb = k.k2 & 3u;      // 3 - index
-  const uint32_t i0 = 3u - max(ra, rb), i1 = 3u - min(ra, rb);
+  const uint32_t ra = k.k1 & 3u, rb = k.k2 & 3u;
+  const uint32_t rh = max(ra, rb), rl = min(ra, rb);
   Group16 g;
-  g.nib = i0 | (i1 << 2);
-  const uint32_t t = (i0 | (i1 << 8)) * 2u;            // first byte of each kept entry
-  g.kept = __byte_perm(lo, hi, t * 0x11u + 0x1010u);
+  g.nib = 15u - rh - 4u * rl;
+  g.kept = __byte_perm(lo, hi, (0x1010u + 0x66u + 0x6600u) - 0x22u * rh - 0x2200u * rl);
   return g;
 }
 
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
   extern __shared__ __align__(128) uint8_t ring[];
   int fails = 0;
   float mw = 0.0f, mv = 0.0f;  // fp32 weights
-  uint32_t kw = 0, kv = 0;     // 16-bit weights: keys
+  uint32_t km = 0, kw = 0, kv = 0;  // 16-bit weights: keys (w and values, w only, values only)
   stream::for_each_chunk<kChunk, kStages>(
       reinterpret_cast<const uint8_t*>(w), nv * 16, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
         const uint4* cv = reinterpret_cast<const uint4*>(chunk);
@@ -249,9 +250,15 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
               const Group16 a = kept16(ka, x.x, x.y), b = kept16(kb, x.z, x.w);
               values[v] = make_uint2(a.kept, b.kept);
               meta[v] = (uint8_t)(a.nib | (b.nib << 4));
-              // amax over non-NaN entries, on keys (magnitude order); NaN sorts highest
-              kw = max(kw, max(ka.k1 <= kNaNKey ? ka.k1 : below_nan(ka), kb.k1 <= kNaNKey ? kb.k1 : below_nan(kb)));
-              kv = max(kv, max(kept_below_nan(ka), kept_below_nan(kb)));
+              // amax over non-NaN entries on keys (magnitude order; NaN sorts highest).  Without
+              // a NaN the largest entry of the vector is kept, so one max serves w and values.
+              const uint32_t top = max(ka.k1, kb.k1);
+              if (top <= kNaNKey) {
+                km = max(km, top);
+              } else {
+                kw = max(kw, max(ka.k1 <= kNaNKey ? ka.k1 : below_nan(ka), kb.k1 <= kNaNKey ? kb.k1 : below_nan(kb)));
+                kv = max(kv, max(kept_below_nan(ka), kept_below_nan(kb)));
+              }
             }
           } else {
             const uint32_t nib = mask_nibble(keep_mask(mag32(x.x), mag32(x.y), mag32(x.z), mag32(x.w)));
@@ -274,8 +281,8 @@ __global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict_
         }
       });
   if constexpr (EB == 2) {
-    mw = key_to_abs<DT>(kw);
-    mv = key_to_abs<DT>(kv);
+    mw = key_to_abs<DT>(max(km, kw));
+    mv = key_to_abs<DT>(max(km, kv));
   }
   count_fails(fails, reinterpret_cast<int32_t*>(acc + 2));
   block_max_to(mw, acc);

@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   using U = U3<WF>;
   constexpr int S = U::SLOTS;
   extern __shared__ uint8_t dsm[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = tc::align1024(dsm);
   uint8_t* slots = base;                              // S x SLOT, 1024-aligned
   uint8_t* xs = base + S * U::SLOT;                   // x, 16 * K bytes, 1024-aligned
   __shared__ uint64_t full_bar[S], empty_bar[S], x_bar;

@@ -66,6 +66,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 
 // 2-D TMA tile load (x = innermost coordinate, in elements) into shared memory, completing
 // `bytes` of transaction count on `bar`.  No cluster multicast.
+// The first 1024-byte aligned address at or after p, a pointer into dynamic shared memory.  The
+// offset is added to p itself (not rebuilt from an integer), so the compiler still knows the
+// result points into shared memory and emits shared loads and stores for it.
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y) {
   asm volatile(

@@ -104,3 +104,37 @@ def test_empty_tensor_writes_scale():
     t = torch.empty((0, 32), dtype=torch.bfloat16, device="cuda")
     q = sp.quantize_nvfp4(t)
     assert q.codes.numel() == 0 and float(q.tensor_scale.item()) == 0.0
+
+
+def _boundary_blocks(seed, nblocks, ts):
+    """fp32 blocks of 16 whose entries sit at, and a few fp32 steps either side of, E2M1's
+    rounding boundaries (0.25 ... 5) times the block's decoded scale: entry 0 fixes the block
+    max (hence the E4M3 block scale), the other 15 are boundary * sc * (1 + k 2^-24).  The block
+    scale sc is worked out the way the method defines it, in fp32, to place the entries; the
+    expected codes still come from the oracle."""
+    g = synth.rng(seed)
+    f32 = np.float32
+    d = f32(f32(ts) * f32(6.0))
+    bounds = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    out = np.zeros((nblocks, 16), np.float32)
+    for b in range(nblocks):
+        target = int(g.integers(1, 127))                     # an E4M3 code with a finite value
+        bmax = f32(6.0 * oracle.e4m3_value(target) * ts)
+        sb = oracle.e4m3_round(float(f32(bmax / d)))
+        sc = f32(f32(oracle.e4m3_value(sb)) * f32(ts))
+        out[b, 0] = bmax
+        m = bounds[g.integers(0, len(bounds), size=15)]
+        k = g.integers(-5, 6, size=15).astype(np.float64)
+        vals = (m * np.float64(sc) * (1.0 + k * 2.0 ** -24)).astype(np.float32)
+        vals = np.minimum(vals, bmax)                        # keep entry 0 the block max
+        sign = np.where(g.random(15) < 0.5, -1.0, 1.0).astype(np.float32)
+        out[b, 1:] = vals * sign
+    return out
+
+
+@pytest.mark.parametrize("ts", [1.0, 3.0517578125e-05, 0.012345, 7.5e-12])
+def test_quotients_at_rounding_boundaries(ts):
+    """Every entry's quotient |t| / sc lies within a few fp32 steps of an E2M1 rounding boundary
+    (including exact ties): the codes must equal the oracle's, which divides entry by entry."""
+    t = _boundary_blocks(int(ts * 1e6) % 9973 + 17, 4096, ts).reshape(256, 256)
+    _compare(t, "f32", ts)
