@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
 // roundings of 2^-24 each), so q and fl(|v| / sc) give the same code unless q lies within a few
 // ulps of a boundary.  Every boundary has at most three significant bits, i.e. a zero in the low
 // 21 bits of its fp32 significand; an entry whose q is within 4 ulps of such a value (which also
-// covers the power-of-two boundary 0.25, where the ulp halves) takes the IEEE division instead.
+// covers the power-of-two boundary 0.25, where the ulp halves) takes the IEEE division instead,
+// together with the other entry of its pair.
 // The codes are therefore exactly those of the per-entry division, at one multiply per entry.
 __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, float d, uint2* codes,
                                              uint8_t* scales, int64_t b) {
@@ -169,29 +170,26 @@ __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, fl
   for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
   uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
   const float sc = __fmul_rn(e4m3_value(sb), s_t);
-  float q[16];
-  if (sc >= 0x1p-100f && sc <= 0x1p100f) {
-    const float y = __frcp_rn(sc);
-    uint32_t near = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      q[i] = __fmul_rn(fabsf(v[i]), y);
-      const uint32_t u = __float_as_uint(q[i]);
-      near |= (uint32_t)(((u + 4u) & 0x1fffffu) <= 8u && u != 0u) << i;
-    }
-    if (near) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if ((near >> i) & 1u) q[i] = __fdiv_rn(fabsf(v[i]), sc);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
-  }
+  const bool fast = sc >= 0x1p-100f && sc <= 0x1p100f;
+  const float y = __frcp_rn(sc);
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
-    uint32_t byte = e2m1x2_rne_satfinite(q[i], q[i + 1]);
+    const float a0 = fabsf(v[i]), a1 = fabsf(v[i + 1]);
+    float q0, q1;
+    if (fast) {
+      q0 = __fmul_rn(a0, y);
+      q1 = __fmul_rn(a1, y);
+      const uint32_t u0 = __float_as_uint(q0), u1 = __float_as_uint(q1);
+      if ((((u0 + 4u) & 0x1fffffu) <= 8u && u0 != 0u) || (((u1 + 4u) & 0x1fffffu) <= 8u && u1 != 0u)) {
+        q0 = __fdiv_rn(a0, sc);  // within 4 ulp of a value with <= 3 significant bits
+        q1 = __fdiv_rn(a1, sc);
+      }
+    } else {
+      q0 = sc != 0.0f ? __fdiv_rn(a0, sc) : 0.0f;
+      q1 = sc != 0.0f ? __fdiv_rn(a1, sc) : 0.0f;
+    }
+    uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
     byte |= (__float_as_uint(v[i]) >> 31) << 3;       // sign of the low entry
     byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;   // sign of the high entry
     packed[i / 8] |= byte << (8 * ((i % 8) / 2));

@@ -280,58 +280,84 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
         if (i / C::MP >= rows_v || i % C::MP >= (int)mbytes) sm[L::OFF_M + i] = 0x44;
   }
 
-  // ---- 2. stage x in fragment order
+  // ---- 2. stage x in fragment order.  Each thread issues XB independent loads before it stores
+  // any, so the staging costs a few L2 round trips rather than one per item.
   constexpr int NCH = C::KC / C::CHUNK;
+  constexpr int XB = 8;
   if constexpr (!sparse_fmt<WF>()) {
     // entry (ch, s, t, lane): 8 bytes = x[8t+g][k0 + ch*CHUNK + LV*c + kslot(s, 0..3)]
     constexpr int LV = C::CHUNK / 4;
     uint2* xs = reinterpret_cast<uint2*>(sm);
-    // one thread per (ch, t, lane, s-pair): 8 consecutive k of the lane piece -> two entries
-    constexpr int PAIRS = C::STEPS / 2 > 0 ? C::STEPS / 2 : 1;
+    // one item per (ch, t, lane, octet): 8 consecutive k of the lane piece -> two entries
     const int items = NCH * NT * 32 * (LV / 8);
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int oct = it % (LV / 8), ln = (it / (LV / 8)) % 32, t = (it / (LV / 8) / 32) % NT,
-                ch = it / (LV / 8) / 32 / NT;
-      const int gg = ln >> 2, cc = ln & 3;
-      const int64_t kb = k0 + (int64_t)ch * C::CHUNK + LV * cc + 8 * oct;
-      const int nrow = 8 * t + gg;
-      const int64_t xr = GROUPED ? (nrow < p.M ? rows_of[nrow] / p.topk : 0) : nrow;
-      const uint4 v = xoct<T>(p, xr, kb, nrow < p.M);
-      // the octet covers steps 2*oct and 2*oct+1 of this lane piece
-      uint2 e0, e1;
-      if (WF == W_DQ4) {  // slots (0,4,1,5) and (2,6,3,7) of the octet
-        e0 = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
-        e1 = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
-      } else {  // slots 0..3 and 4..7
-        e0 = make_uint2(v.x, v.y);
-        e1 = make_uint2(v.z, v.w);
+    for (int base = threadIdx.x; base < items; base += blockDim.x * XB) {
+      uint4 v[XB];
+#pragma unroll
+      for (int b = 0; b < XB; ++b) {
+        const int it = base + b * blockDim.x;
+        if (it < items) {
+          const int oct = it % (LV / 8), ln = (it / (LV / 8)) % 32, t = (it / (LV / 8) / 32) % NT,
+                    ch = it / (LV / 8) / 32 / NT;
+          const int gg = ln >> 2, cc = ln & 3;
+          const int64_t kb = k0 + (int64_t)ch * C::CHUNK + LV * cc + 8 * oct;
+          const int nrow = 8 * t + gg;
+          const int64_t xr = GROUPED ? (nrow < p.M ? rows_of[nrow] / p.topk : 0) : nrow;
+          v[b] = xoct<T>(p, xr, kb, nrow < p.M);
+        }
       }
-      const int s0 = 2 * oct;
-      xs[((ch * C::STEPS + s0) * NT + t) * 32 + ln] = e0;
-      xs[((ch * C::STEPS + s0 + 1) * NT + t) * 32 + ln] = e1;
-      (void)PAIRS;
+#pragma unroll
+      for (int b = 0; b < XB; ++b) {
+        const int it = base + b * blockDim.x;
+        if (it < items) {
+          const int oct = it % (LV / 8), ln = (it / (LV / 8)) % 32, t = (it / (LV / 8) / 32) % NT,
+                    ch = it / (LV / 8) / 32 / NT;
+          // the octet covers steps 2*oct and 2*oct+1 of this lane piece
+          uint2 e0, e1;
+          if (WF == W_DQ4) {  // slots (0,4,1,5) and (2,6,3,7) of the octet
+            e0 = make_uint2(__byte_perm(v[b].x, v[b].z, 0x5410), __byte_perm(v[b].x, v[b].z, 0x7632));
+            e1 = make_uint2(__byte_perm(v[b].y, v[b].w, 0x5410), __byte_perm(v[b].y, v[b].w, 0x7632));
+          } else {  // slots 0..3 and 4..7
+            e0 = make_uint2(v[b].x, v[b].y);
+            e1 = make_uint2(v[b].z, v[b].w);
+          }
+          const int s0 = 2 * oct;
+          xs[((ch * C::STEPS + s0) * NT + t) * 32 + ln] = e0;
+          xs[((ch * C::STEPS + s0 + 1) * NT + t) * 32 + ln] = e1;
+        }
+      }
     }
   } else {
     // entry (win, t, lane): 16 bytes = x[8t+g][k0 + 32*win + 2c + 8i + {0,1}], i = 0..3
     uint4* xs = reinterpret_cast<uint4*>(sm);
     const int items = NCH * NT * 32;
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int ln = it % 32, t = (it / 32) % NT, win = it / 32 / NT;
-      const int gg = ln >> 2, cc = ln & 3;
-      const int nrow = 8 * t + gg;
-      const bool live = nrow < p.M;
-      const int64_t n = GROUPED ? (live ? rows_of[nrow] / p.topk : 0) : nrow;
-      const int64_t kb = k0 + 32 * win + 2 * cc;
-      uint32_t w4[4];
+    constexpr int IB = XB / 4;  // items per batch, four loads each
+    for (int base = threadIdx.x; base < items; base += blockDim.x * IB) {
+      uint32_t w4[IB][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t k = kb + 8 * i;
-        if (p.x_fmt == X_16 && live && k + 2 <= p.K)
-          w4[i] = __ldg(reinterpret_cast<const unsigned int*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
-        else
-          w4[i] = xval<T>(p, n, k, live) | (xval<T>(p, n, k + 1, live) << 16);
+      for (int b = 0; b < IB; ++b) {
+        const int it = base + b * blockDim.x;
+        if (it < items) {
+          const int ln = it % 32, t = (it / 32) % NT, win = it / 32 / NT;
+          const int gg = ln >> 2, cc = ln & 3;
+          const int nrow = 8 * t + gg;
+          const bool live = nrow < p.M;
+          const int64_t n = GROUPED ? (live ? rows_of[nrow] / p.topk : 0) : nrow;
+          const int64_t kb = k0 + 32 * win + 2 * cc;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t k = kb + 8 * i;
+            if (p.x_fmt == X_16 && live && k + 2 <= p.K)
+              w4[b][i] = __ldg(reinterpret_cast<const unsigned int*>(reinterpret_cast<const uint16_t*>(p.x) + n * p.K + k));
+            else
+              w4[b][i] = xval<T>(p, n, k, live) | (xval<T>(p, n, k + 1, live) << 16);
+          }
+        }
       }
-      xs[it] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+#pragma unroll
+      for (int b = 0; b < IB; ++b) {
+        const int it = base + b * blockDim.x;
+        if (it < items) xs[it] = make_uint4(w4[b][0], w4[b][1], w4[b][2], w4[b][3]);
+      }
     }
   }
   __syncthreads();
@@ -518,6 +544,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t upr = p.K / U::UK;                    // units per 16-row tile
+  const int upr32 = (int)upr;
   const int64_t U_all = ((p.N + 15) / 16) * upr;
   const int64_t ub = U_all * blockIdx.x / gridDim.x, ue = U_all * (blockIdx.x + 1) / gridDim.x;
   const int nunits = (int)(ue - ub);
@@ -547,20 +574,27 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int nbox = (int)(p.K / 64);
       mbar_arrive_expect_tx(&x_bar, (uint32_t)nbox * 1024u);
       for (int b = 0; b < nbox; ++b) tc::tma_load_2d(xs + b * 1024, &tmX, &x_bar, b * 64, 0);
-      int i = 0;
+      int i = 0, sl = 0, phase = 0;
+      int tile = (int)(ub / upr), kp = (int)(ub % upr);  // unit ub + i, advanced incrementally
       for (; i < nunits; ++i) {
-        const int sl = i % S;
-        if (!mbar_wait(&empty_bar[sl], ((i / S) & 1) ^ 1)) {
+        if (!mbar_wait(&empty_bar[sl], phase ^ 1)) {
           set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
           abort_flag = 1;
           break;
         }
-        const int64_t u = ub + i, tile = u / upr, kp = u % upr;
         uint8_t* d = slots + sl * U::SLOT;
         mbar_arrive_expect_tx(&full_bar[sl], U::CODES + U::SCALES + U::META);
         tc::tma_load_2d(d, &tmC, &full_bar[sl], (int)(kp * 128), (int)(tile * 16));
         tc::tma_load_2d(d + U::CODES, &tmS, &full_bar[sl], (int)(kp * 16), (int)(tile * 16));
         if (U::META) tc::tma_load_2d(d + U::CODES + U::SCALES, &tmM, &full_bar[sl], (int)(kp * 64), (int)(tile * 16));
+        if (++kp == upr32) {
+          kp = 0;
+          ++tile;
+        }
+        if (++sl == S) {
+          sl = 0;
+          phase ^= 1;
+        }
       }
       issued = i;
     }
@@ -570,7 +604,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int g = lane >> 2, c = lane & 3;
     const int r0 = prow(g), r1 = prow(g + 8);
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-    int64_t cur = -1;
+    int cur = -1;
     auto flush = [&]() {
       float* b = &tbuf[cur - t0][0][0];
       atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
@@ -587,7 +621,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     for (int i = cw; ok && i < nunits; i += kDecConsumers) {
       const int sl = i % S;
-      const int64_t u = ub + i, tile = u / upr, kp = u % upr;
+      const uint32_t u = (uint32_t)(ub + i);             // < 2^31 (host check)
+      const int tile = (int)(u / (uint32_t)upr32), kp = (int)(u - (uint32_t)tile * (uint32_t)upr32);
       if (tile != cur) {
         if (cur >= 0) flush();
         cur = tile;
@@ -743,6 +778,7 @@ bool decode_supported(int wf, const SkinnyParams& p) {
   else return false;
   if (p.K % uk) return false;
   const int64_t upr = p.K / uk, units = (p.N / 16) * upr, grid = sm_count();
+  if (units >= (int64_t(1) << 31)) return false;
   const int64_t per_cta = (units + grid - 1) / grid;
   return per_cta / upr + 2 <= kDecMaxTiles;
 }
