@@ -199,7 +199,9 @@ int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* 
  * must have the same type; NVFP4 w is decoded in-kernel to x's type (bf16 when x is NVFP4).
  * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
  * aligned.  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
- * workspace: device scratch of sp24_gemm_workspace_size() bytes (may be NULL when 0). */
+ * workspace: device scratch of sp24_gemm_workspace_size() bytes (may be NULL when 0).
+ * Kernels that split K across CTAs or warps combine partial sums with fp32 atomics, so two
+ * identical calls may differ in the last bits of an output. */
 int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, int64_t M, int64_t N,
                              int64_t K, int algo, int64_t* bytes);
 int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int64_t M, int64_t N,

@@ -48,8 +48,9 @@ def test_decode_matches_tiled_kernel(sparse):
 
 
 def test_repeated_launches_reuse_no_state():
-    """Two back-to-back calls into the same output: the second result equals the first (the
-    output is cleared by each call and no shared-memory state leaks between launches)."""
+    """Two back-to-back calls, the second into an output pre-filled with 7.0: the results agree
+    to fp32 summation-order noise (the output is cleared by each call and no shared-memory
+    state leaks between launches; partial sums meet through fp32 atomics, whose order varies)."""
     M, N, K = 8, 2048, 1024
     X, xs, W, ws = make_case("bf16", "nvfp4", M, N, K, seed=5, w_sigma=0.02)
     x = torch.from_numpy(X.view("int16")).view(torch.bfloat16).cuda()
@@ -57,4 +58,4 @@ def test_repeated_launches_reuse_no_state():
     y1 = sp.gemm_dense(x, w)
     y2 = sp.gemm_dense(x, w, out=torch.full_like(y1, 7.0))
     torch.cuda.synchronize()
-    assert torch.equal(y1, y2)
+    assert torch.allclose(y1, y2, rtol=1e-5, atol=1e-5)
