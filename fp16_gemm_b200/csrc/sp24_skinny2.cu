@@ -489,229 +489,227 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
 
 // ------------------------------------------------------------------ persistent decode GEMV (M <= 8)
 //
-// One CTA per SM: a producer warp first loads x (M <= 8 tokens, whole K) with 2-D TMA into
-// shared memory (boxes of 64 k x 8 tokens with the 128-byte swizzle; token rows past M read as
-// zeros), then streams 16-row weight units (codes with the 128-byte swizzle, block scales and
-// 2:4 nibbles unswizzled) through a ring of slots; 16 consumer warps take the units
-// round-robin.  Units are spread evenly over the CTAs (each CTA a contiguous range in
-// tile-major order), so every SM streams the same number of bytes.  A warp adds its partial
-// sums of a 16-row tile into that tile's shared buffer whenever its next unit belongs to another
-// tile; when all units are done the CTA adds its buffers into y (zeroed first) with one atomic
-// per output, which also joins tiles split between neighbouring CTAs.
+// One CTA of 16 warps per SM.  All threads first copy x (M <= 8 tokens, whole K) into shared
+// memory with 16-byte cp.async (token rows past M are zeroed).  The weight is cut into units of
+// 16 rows x UK logical k; each CTA takes a contiguous range of units in tile-major order (so
+// every SM streams the same number of bytes) and its warps take the units round-robin.  A warp
+// moves its own units with 16-byte cp.async on the load/store path into a private double
+// buffer, so every warp keeps two units in flight without a producer: one thread issuing TMA
+// requests for a whole SM cannot keep HBM busy when each unit is 16 short rows.  A warp adds its
+// partial sums of a 16-row tile into that tile's shared buffer whenever its next unit belongs to
+// another tile; when all units are done the CTA adds its buffers into y (zeroed first) with one
+// atomic per output, which also joins tiles split between neighbouring CTAs.
 //
-// B fragments are read straight from the swizzled x: in every 8-lane shared-memory phase the
-// 16-byte pieces of different tokens sit in different chunks (chunk j of token g at j ^ g), so
-// the reads are conflict free.  MMA row m of a warp reads tile row prow(m) = (m/2) + 4 (m%2)
-// (+8 for m >= 8), which puts the two rows of a phase in disjoint bank halves of the swizzled
-// weight codes.
-constexpr int kDecConsumers = 16;
-constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+// Layouts in shared memory: codes of a unit as 16 rows of 128 bytes, 16-byte chunk j of row r
+// stored at chunk j ^ (r % 8); x as boxes of 64 k x 8 tokens, chunk j of token g at j ^ g.  In
+// every 8-lane phase the B-fragment reads of different tokens fall in different chunks, and
+// MMA row m reads tile row prow(m) = (m/2) + 4 (m%2) (+8 for m >= 8), which puts the two rows of
+// a phase in disjoint halves of the banks: the shared reads are conflict free.
+constexpr int kDecWarps = 16;
+constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecMaxTiles = 32;  // per-CTA tile buffers (16 rows x 8 tokens fp32 each)
+constexpr int kDecDepth = 2;      // units in flight per warp
 
 template <int WF>
 struct U3;
 template <>
-struct U3<W_DQ4> {  // 256 K per unit: codes 16 x 128 B, scales 16 x 16 B
-  static constexpr int UK = 256, CODES = 2048, SCALES = 256, META = 0, SLOT = 3072, SLOTS = 24;
+struct U3<W_DQ4> {  // 256 k per unit: codes 16 x 128 B, scales 16 x 16 B
+  static constexpr int UK = 256, CODES = 2048, SCALES = 256, META = 0, SLOT = 2304;
 };
 template <>
-struct U3<W_SQ4> {  // 512 K per unit: codes 16 x 128 B, scales 16 x 16 B, nibbles 16 x 64 B
-  static constexpr int UK = 512, CODES = 2048, SCALES = 256, META = 1024, SLOT = 4096, SLOTS = 16;
+struct U3<W_SQ4> {  // 512 k per unit: codes 16 x 128 B, scales 16 x 16 B, nibbles 16 x 64 B
+  static constexpr int UK = 512, CODES = 2048, SCALES = 256, META = 1024, SLOT = 3328;
 };
 
 __device__ __forceinline__ int prow(int m) { return (m & 8) + ((m & 7) >> 1) + 4 * (m & 1); }
 
-// Byte offset in the swizzled x of token g, column k (k % 8 == 0): box k / 64 of 1 KB, token
-// row of 128 B, 16-byte chunk (k % 64) / 8 stored at chunk ^ g.
+// Byte offset in the staged x of token g, column k (k % 8 == 0): box k / 64 of 1 KB, token row of
+// 128 B, 16-byte chunk (k % 64) / 8 stored at chunk ^ g.
 __device__ __forceinline__ uint32_t xoff(int g, int64_t k) {
   return (uint32_t)((k >> 6) * 1024 + g * 128 + ((((int)(k >> 3) & 7) ^ g) << 4));
 }
 
-template <int WF, typename T>
-__global__ void __launch_bounds__(kDecThreads, 1)
-    decode_gemv_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
-                       const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmX,
-                       const SkinnyParams p) {
+// One warp copies unit (tile, kp) into `slot`: codes (four 16-byte pieces per lane, each four
+// consecutive lanes' pieces one 128-byte row segment), block scales and 2:4 nibbles.
+template <int WF>
+__device__ __forceinline__ void issue_unit(uint8_t* slot, const SkinnyParams& p, int tile, int kp, int lane) {
   using U = U3<WF>;
-  constexpr int S = U::SLOTS;
-  extern __shared__ uint8_t dsm[];
-  uint8_t* base = tc::align1024(dsm);
-  uint8_t* slots = base;                              // S x SLOT, 1024-aligned
-  uint8_t* xs = base + S * U::SLOT;                   // x, 16 * K bytes, 1024-aligned
-  __shared__ uint64_t full_bar[S], empty_bar[S], x_bar;
+  const int64_t crow = WF == W_DQ4 ? p.K / 2 : p.K / 4;
+  const uint8_t* cbase = p.w + (int64_t)tile * 16 * crow + kp * 128;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int q = lane + 32 * t, r = q >> 3, j = q & 7;
+    tc::cp_async16(slot + r * 128 + ((j ^ (r & 7)) << 4), cbase + r * crow + j * 16);
+  }
+  if (lane < 16) {
+    const int64_t srow = WF == W_DQ4 ? p.K / 16 : p.K / 32;
+    tc::cp_async16(slot + U::CODES + lane * 16, p.w_scales + ((int64_t)tile * 16 + lane) * srow + kp * 16);
+  }
+  if constexpr (U::META > 0) {
+    const int64_t mrow = p.K / 8;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int q = lane + 32 * t, r = q >> 2, j = q & 3;
+      tc::cp_async16(slot + U::CODES + U::SCALES + r * 64 + j * 16,
+                     p.meta + ((int64_t)tile * 16 + r) * mrow + kp * 64 + j * 16);
+    }
+  }
+}
+
+// Dynamic shared memory of the decode kernel: x (16 K bytes) + every warp's unit buffers.
+template <int WF>
+constexpr size_t decode_smem(int64_t K) {
+  return 16 * (size_t)K + (size_t)kDecWarps * kDecDepth * U3<WF>::SLOT;
+}
+
+template <int WF, typename T>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const SkinnyParams p) {
+  using U = U3<WF>;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t* xs = dsm;                            // 16 * K bytes
+  uint8_t* slots = dsm + 16 * p.K;              // kDecWarps x kDecDepth x SLOT
   __shared__ float tbuf[kDecMaxTiles][16][8];
-  __shared__ int issued, abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t upr = p.K / U::UK;                    // units per 16-row tile
-  const int upr32 = (int)upr;
-  const int64_t U_all = ((p.N + 15) / 16) * upr;
-  const int64_t ub = U_all * blockIdx.x / gridDim.x, ue = U_all * (blockIdx.x + 1) / gridDim.x;
-  const int nunits = (int)(ue - ub);
-  const int64_t t0 = ub / upr;
-  const int nloc = nunits > 0 ? (int)((ue - 1) / upr - t0 + 1) : 0;  // <= kDecMaxTiles (host check)
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      tc::mbar_init(&full_bar[i], 1);
-      tc::mbar_init(&empty_bar[i], 1);
-    }
-    tc::mbar_init(&x_bar, 1);
-    issued = 0;
-    abort_flag = 0;
-    tc::fence_mbar_init();
-  }
+  const int upr = (int)(p.K / U::UK);           // units per 16-row tile
+  const int64_t U_all = (p.N / 16) * upr;       // < 2^31 (host check)
+  const int ub = (int)(U_all * blockIdx.x / gridDim.x), ue = (int)(U_all * (blockIdx.x + 1) / gridDim.x);
+  const int nunits = ue - ub;
+  if (nunits <= 0) return;                      // whole CTA, before any barrier
+  const int t0 = ub / upr;
+  const int nloc = (ue - 1) / upr - t0 + 1;     // <= kDecMaxTiles (host check)
   for (int i = threadIdx.x; i < nloc * 128; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
-  __syncthreads();
 
-  if (warp == 0) {
-    // ---- producer: x, then the weight units
-    if (lane == 0 && nunits > 0) {
-      tc::prefetch_tmap(&tmX);
-      tc::prefetch_tmap(&tmC);
-      tc::prefetch_tmap(&tmS);
-      if (U::META) tc::prefetch_tmap(&tmM);
-      const int nbox = (int)(p.K / 64);
-      mbar_arrive_expect_tx(&x_bar, (uint32_t)nbox * 1024u);
-      for (int b = 0; b < nbox; ++b) tc::tma_load_2d(xs + b * 1024, &tmX, &x_bar, b * 64, 0);
-      int i = 0, sl = 0, phase = 0;
-      int tile = (int)(ub / upr), kp = (int)(ub % upr);  // unit ub + i, advanced incrementally
-      for (; i < nunits; ++i) {
-        if (!mbar_wait(&empty_bar[sl], phase ^ 1)) {
-          set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-          abort_flag = 1;
-          break;
-        }
-        uint8_t* d = slots + sl * U::SLOT;
-        mbar_arrive_expect_tx(&full_bar[sl], U::CODES + U::SCALES + U::META);
-        tc::tma_load_2d(d, &tmC, &full_bar[sl], (int)(kp * 128), (int)(tile * 16));
-        tc::tma_load_2d(d + U::CODES, &tmS, &full_bar[sl], (int)(kp * 16), (int)(tile * 16));
-        if (U::META) tc::tma_load_2d(d + U::CODES + U::SCALES, &tmM, &full_bar[sl], (int)(kp * 64), (int)(tile * 16));
-        if (++kp == upr32) {
-          kp = 0;
-          ++tile;
-        }
-        if (++sl == S) {
-          sl = 0;
-          phase ^= 1;
-        }
-      }
-      issued = i;
-    }
-  } else if (nunits > 0) {
-    // ---- consumers
-    const int cw = warp - 1;
-    const int g = lane >> 2, c = lane & 3;
-    const int r0 = prow(g), r1 = prow(g + 8);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-    int cur = -1;
-    auto flush = [&]() {
-      float* b = &tbuf[cur - t0][0][0];
-      atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
-      atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
-      atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
-      atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
+  // ---- x: one 16-byte piece per (token, 8 k); consecutive threads take consecutive pieces of a row
+  const int64_t kp8 = p.K / 8;
+  const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
+  for (int64_t i = threadIdx.x; i < 8 * kp8; i += blockDim.x) {
+    const int g = (int)(i / kp8);
+    const int64_t k = (i - g * kp8) * 8;
+    uint8_t* dst = xs + xoff(g, k);
+    if (g < p.M)
+      tc::cp_async16(dst, xg + g * p.K + k);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  tc::cp_async_commit();
+
+  // ---- this warp's units: local index warp + kDecWarps * n; the first kDecDepth in flight now
+  uint8_t* wslots = slots + warp * kDecDepth * U::SLOT;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = acc2[q] = 0.f;
-    };
-    bool ok = mbar_wait(&x_bar, 0);
-    if (!ok) {
-      set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-      abort_flag = 1;
+  for (int d = 0; d < kDecDepth; ++d) {
+    const int i = warp + kDecWarps * d;
+    if (i < nunits) {
+      const int u = ub + i, tile = u / upr;
+      issue_unit<WF>(wslots + d * U::SLOT, p, tile, u - tile * upr, lane);
     }
-    for (int i = cw; ok && i < nunits; i += kDecConsumers) {
-      const int sl = i % S;
-      const uint32_t u = (uint32_t)(ub + i);             // < 2^31 (host check)
-      const int tile = (int)(u / (uint32_t)upr32), kp = (int)(u - (uint32_t)tile * (uint32_t)upr32);
-      if (tile != cur) {
-        if (cur >= 0) flush();
-        cur = tile;
+    tc::cp_async_commit();  // possibly empty: keeps the group count uniform
+  }
+  tc::cp_async_wait<kDecDepth>();  // this thread's x pieces have landed
+  __syncthreads();                 // everyone's x pieces and the zeroed buffers are visible
+
+  const int g = lane >> 2, c = lane & 3;
+  const int r0 = prow(g), r1 = prow(g + 8);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+  int cur = -1;
+  auto flush = [&]() {
+    float* b = &tbuf[cur - t0][0][0];
+    atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
+    atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
+    atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
+    atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = acc2[q] = 0.f;
+  };
+  for (int n = 0, i = warp; i < nunits; ++n, i += kDecWarps) {
+    const int u = ub + i, tile = u / upr, kp = u - tile * upr;
+    if (tile != cur) {
+      if (cur >= 0) flush();
+      cur = tile;
+    }
+    tc::cp_async_wait<kDecDepth - 1>();  // this unit's group (all but the newest) has landed
+    __syncwarp();
+    uint8_t* slot = wslots + (n % kDecDepth) * U::SLOT;
+    const uint8_t* d = slot;
+    const uint8_t* sc = d + U::CODES;
+    if constexpr (WF == W_DQ4) {
+      // the unit's two 128-k chunks feed two independent accumulator chains
+      uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int j = 4 * ch + c;
+        const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
+        const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
+        w0[ch][0] = v0.x; w0[ch][1] = v0.y; w0[ch][2] = v0.z; w0[ch][3] = v0.w;
+        w1[ch][0] = v1.x; w1[ch][1] = v1.y; w1[ch][2] = v1.z; w1[ch][3] = v1.w;
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), sa[ch][0], sa[ch][1]);
+        scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), sb[ch][0], sb[ch][1]);
       }
-      if (!mbar_wait(&full_bar[sl], (i / S) & 1)) {
-        set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-        abort_flag = 1;
-        break;
-      }
-      const uint8_t* d = slots + sl * U::SLOT;
-      const uint8_t* sc = d + U::CODES;
-      if constexpr (WF == W_DQ4) {
-        // the unit's two 128-K chunks feed two independent accumulator chains
-        uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          const int j = 4 * ch + c;
-          const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * 128 + ((j ^ (r0 & 7)) << 4));
-          const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * 128 + ((j ^ (r1 & 7)) << 4));
-          w0[ch][0] = v0.x; w0[ch][1] = v0.y; w0[ch][2] = v0.z; w0[ch][3] = v0.w;
-          w1[ch][0] = v1.x; w1[ch][1] = v1.y; w1[ch][2] = v1.z; w1[ch][3] = v1.w;
-          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * 16 + 8 * ch + 2 * c), sa[ch][0], sa[ch][1]);
-          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * 16 + 8 * ch + 2 * c), sb[ch][0], sb[ch][1]);
-        }
+          // x[g][P .. P+8), P = chunk base + 32c + 8q: codes at nibbles (i, i+4) of word q pair
+          // with x entries (i, i+4)
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff(g, kp * 256 + ch * 128 + 32 * c + 8 * q));
+          const uint32_t s0 = sa[ch][q >> 1], s1 = sb[ch][q >> 1];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            // x[g][P .. P+8), P = chunk base + 32c + 8q: codes at nibbles (i, i+4) of word q
-            // pair with x entries (i, i+4)
-            const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff(g, kp * 256 + ch * 128 + 32 * c + 8 * q));
-            const uint32_t s0 = sa[ch][q >> 1], s1 = sb[ch][q >> 1];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
-              const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
-              const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h), s0);
-              const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h + 1), s0);
-              const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h), s1);
-              const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h + 1), s1);
-              mma_k16<T>(ch ? acc2 : acc, a0, a1, a2, a3, bx);
-            }
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
+            const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
+            const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h), s0);
+            const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[ch][q], 2 * h + 1), s0);
+            const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h), s1);
+            const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[ch][q], 2 * h + 1), s1);
+            mma_k16<T>(ch ? acc2 : acc, a0, a1, a2, a3, bx);
           }
         }
-      } else {
-        // even and odd windows feed two independent accumulator chains
-        const uint8_t* me = sc + U::SCALES;
-#pragma unroll 4
-        for (int w = 0; w < 16; ++w) {
-          const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * 64 + 4 * w);
-          const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * 64 + 4 * w);
-          const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
-          const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * 128 + (((w >> 1) ^ (r0 & 7)) << 4) + 8 * (w & 1));
-          const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * 128 + (((w >> 1) ^ (r1 & 7)) << 4) + 8 * (w & 1));
-          uint32_t s0, s1, unused;
-          scale_pair<T>(sc[r0 * 16 + w], s0, unused);
-          scale_pair<T>(sc[r1 * 16 + w], s1, unused);
-          const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
-          const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
-          const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
-          const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
-          const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
-          const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
-          // x[g][32w' + 2c + 8i + {0, 1}], i = 0..3: word c of four consecutive 16-byte pieces
-          const int64_t kw = kp * 512 + 32 * w;
-          const uint8_t* xr = xs + 4 * c;
-          const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr + xoff(g, kw)),
-                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 8)),
-                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 16)),
-                                      *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 24)));
-          mma_sp_k32<T>((w & 1) ? acc2 : acc, a0, a1, a2, a3, bx, e);
-        }
       }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
+    } else {
+      // even and odd windows feed two independent accumulator chains
+      const uint8_t* me = sc + U::SCALES;
+#pragma unroll 4
+      for (int w = 0; w < 16; ++w) {
+        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * 64 + 4 * w);
+        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * 64 + 4 * w);
+        const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
+        const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * 128 + (((w >> 1) ^ (r0 & 7)) << 4) + 8 * (w & 1));
+        const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * 128 + (((w >> 1) ^ (r1 & 7)) << 4) + 8 * (w & 1));
+        uint32_t s0, s1, unused;
+        scale_pair<T>(sc[r0 * 16 + w], s0, unused);
+        scale_pair<T>(sc[r1 * 16 + w], s1, unused);
+        const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
+        const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
+        const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+        const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+        const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+        const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+        // x[g][32w' + 2c + 8i + {0, 1}], i = 0..3: word c of four consecutive 16-byte pieces
+        const int64_t kw = (int64_t)kp * 512 + 32 * w;
+        const uint8_t* xr = xs + 4 * c;
+        const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr + xoff(g, kw)),
+                                    *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 8)),
+                                    *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 16)),
+                                    *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 24)));
+        mma_sp_k32<T>((w & 1) ? acc2 : acc, a0, a1, a2, a3, bx, e);
+      }
     }
-    if (cur >= 0) flush();
+    __syncwarp();  // every lane is done with the slot before it is refilled
+    const int inext = i + kDecWarps * kDecDepth;
+    if (inext < nunits) {
+      const int u2 = ub + inext, t2 = u2 / upr;
+      issue_unit<WF>(slot, p, t2, u2 - t2 * upr, lane);
+    }
+    tc::cp_async_commit();
   }
+  if (cur >= 0) flush();
+  tc::cp_async_wait<0>();  // nothing in flight (the trailing groups are empty)
   __syncthreads();
-  // a gave-up wait may leave copies in flight: let them land before the CTA's memory goes away
-  if (abort_flag && threadIdx.x == 0) {
-    tc::mbar_wait(&x_bar, 0);
-    for (int i = issued > S ? issued - S : 0; i < issued; ++i) tc::mbar_wait(&full_bar[i % S], (i / S) & 1);
-  }
   // ---- the CTA's tile sums into y
-  float scale = 256.0f * *p.w_ts;
+  const float scale = 256.0f * *p.w_ts;
   for (int e = threadIdx.x; e < nloc * 128; e += blockDim.x) {
     const int lt = e >> 7, row = (e >> 3) & 15, tok = e & 7;
-    const int64_t gr = (t0 + lt) * 16 + row;
+    const int64_t gr = (int64_t)(t0 + lt) * 16 + row;
     const float v = (&tbuf[0][0][0])[e];
     if (tok < p.M && gr < p.N && v != 0.0f) atomicAdd(p.y + (int64_t)tok * p.N + gr, v * scale);
   }
@@ -719,28 +717,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 template <int WF, typename T>
 int launch_decode(const SkinnyParams& p, cudaStream_t s) {
-  using U = U3<WF>;
-  CUtensorMap tc_, ts_, tm_, tx_;
-  const int64_t cb = WF == W_DQ4 ? p.K / 2 : p.K / 4;
-  int st = make_tmap_2d(&tc_, p.w, 1, p.N, cb, cb, 128, 16);
-  if (st) return st;
-  const int64_t sb = WF == W_DQ4 ? p.K / 16 : p.K / 32;
-  st = make_tmap_2d_plain(&ts_, p.w_scales, p.N, sb, sb, 16, 16);
-  if (st) return st;
-  if (WF == W_SQ4) {
-    st = make_tmap_2d_plain(&tm_, p.meta, p.N, p.K / 8, p.K / 8, 64, 16);
-    if (st) return st;
-  } else {
-    tm_ = ts_;
-  }
-  // x rows past M (up to the 8-row box) read as zeros
-  if (make_tmap_2d(&tx_, p.x, 2, p.M, p.K, p.K * 2, 64, 8)) return SP24_ERR_UNSUPPORTED;
-  const size_t smem = 1024 + (size_t)U::SLOTS * U::SLOT + 16 * (size_t)p.K;
+  const size_t smem = decode_smem<WF>(p.K);
   auto kern = decode_gemv_kernel<WF, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   if (cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
-  kern<<<sm_count(), kDecThreads, smem, s>>>(tc_, ts_, tm_, tx_, p);
+  kern<<<sm_count(), kDecThreads, smem, s>>>(p);
   return launch_status();
 }
 
@@ -765,18 +747,25 @@ int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStre
   return SP24_ERR_UNSUPPORTED;
 }
 
-// True when the persistent decode kernel takes the problem: 16-bit x of at most 8 tokens (TMA
-// rows: 16-byte aligned, K % 64), NVFP4 weights (dense or 2:4) in whole 16-row tiles, K a whole
-// number of units and small enough for x to stay in shared memory (16 K bytes), and at most
-// kDecMaxTiles tiles touched by any CTA.
+// True when the persistent decode kernel takes the problem: 16-bit x of at most 8 tokens
+// (16-byte aligned rows), NVFP4 weights (dense or 2:4) in whole 16-row tiles, K a whole number of
+// units, x plus the warps' unit buffers within shared memory, and at most kDecMaxTiles tiles
+// touched by any CTA.
 bool decode_supported(int wf, const SkinnyParams& p) {
-  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0 || p.K > 8192) return false;
+  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0) return false;
   if (!aligned(p.x, 16) || !aligned(p.w, 16) || !aligned(p.w_scales, 16)) return false;
   int64_t uk;
-  if (wf == W_DQ4) uk = U3<W_DQ4>::UK;
-  else if (wf == W_SQ4 && aligned(p.meta, 16)) uk = U3<W_SQ4>::UK;
-  else return false;
-  if (p.K % uk) return false;
+  size_t smem;
+  if (wf == W_DQ4) {
+    uk = U3<W_DQ4>::UK;
+    smem = decode_smem<W_DQ4>(p.K);
+  } else if (wf == W_SQ4 && aligned(p.meta, 16)) {
+    uk = U3<W_SQ4>::UK;
+    smem = decode_smem<W_SQ4>(p.K);
+  } else {
+    return false;
+  }
+  if (p.K % uk || smem + sizeof(float) * kDecMaxTiles * 128 > 227 * 1024) return false;
   const int64_t upr = p.K / uk, units = (p.N / 16) * upr, grid = sm_count();
   if (units >= (int64_t(1) << 31)) return false;
   const int64_t per_cta = (units + grid - 1) / grid;

@@ -64,6 +64,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// 16-byte asynchronous global -> shared copy on the load/store path (not the TMA engine), cached
+// in L2 only.  Copies complete in commit-group order: cp_async_wait<N>() returns once at most N
+// of the calling thread's groups are still in flight; other threads see the data after a barrier.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // 2-D TMA tile load (x = innermost coordinate, in elements) into shared memory, completing
 // `bytes` of transaction count on `bar`.  No cluster multicast.
 // The first 1024-byte aligned address at or after p, a pointer into dynamic shared memory.  The
