@@ -78,8 +78,8 @@ __device__ __forceinline__ uint32_t e2m1x2_rne_satfinite(float x_lo, float x_hi)
   return r & 0xffu;
 }
 
-// Streaming ring: 4 stages of 16 KB per CTA (512 blocks of 16 16-bit entries, or 256 fp32).
-constexpr int kChunk = 16384, kStages = 4;
+// Streaming ring: 3 stages of 16 KB per CTA (512 blocks of 16 16-bit entries, or 256 fp32).
+constexpr int kChunk = 16384, kStages = 3;  // 48 KB per CTA: four CTAs per SM
 constexpr size_t kRingBytes = (size_t)kChunk * kStages;
 
 // 16 entries of a block from shared memory as fp32.
@@ -113,7 +113,7 @@ template <int DT>
 constexpr int block_bytes() { return DT == SP24_F32 ? 64 : 32; }
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ t, int64_t nblk,
+__global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ t, int64_t nblk,
                                                         unsigned int* __restrict__ amax_bits) {
   extern __shared__ __align__(128) uint8_t ring[];
   constexpr int BB = block_bytes<DT>();
@@ -199,7 +199,7 @@ __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, fl
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads) encode_kernel(const void* __restrict__ t, int64_t nblk,
+__global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restrict__ t, int64_t nblk,
                                                           const float* __restrict__ ts_in,
                                                           const unsigned int* __restrict__ amax_bits,
                                                           uint2* __restrict__ codes,

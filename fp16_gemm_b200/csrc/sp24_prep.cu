@@ -132,12 +132,12 @@ __device__ __forceinline__ void count_fails(int fails, int32_t* n_fail) {
 
 // Groups 2v, 2v+1 (16-bit) or group v (fp32) per 16-byte vector v.  Every lane of a warp runs
 // the same number of iterations so the final warp reduction sees all lanes.
-// Streaming ring: 4 stages of 16 KB per CTA (1024 vectors of 16 bytes, 4 per thread).
-constexpr int kChunk = 16384, kStages = 4;
+// Streaming ring: 3 stages of 16 KB per CTA (1024 vectors of 16 bytes, 4 per thread).
+constexpr int kChunk = 16384, kStages = 3;  // 48 KB per CTA: four CTAs per SM
 constexpr size_t kRingBytes = (size_t)kChunk * kStages;
 
 template <int EB>
-__global__ void __launch_bounds__(kThreads) check24_vec(const uint4* __restrict__ w, int64_t nv,
+__global__ void __launch_bounds__(kThreads, 4) check24_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint8_t* __restrict__ pass,
                                                         int32_t* __restrict__ n_fail) {
   extern __shared__ __align__(128) uint8_t ring[];
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads) check24_vec(const uint4* __restrict_
 }
 
 template <int EB>
-__global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict__ w, int64_t nv,
+__global__ void __launch_bounds__(kThreads, 4) prune24_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint2* __restrict__ values,
                                                         uint8_t* __restrict__ meta) {
   extern __shared__ __align__(128) uint8_t ring[];
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) prune24_vec(const uint4* __restrict_
 // done.  The last CTA to finish writes the fail count and the two NVFP4 tensor scales
 // amax / 2688, computed exactly as the quantiser derives them.
 template <int DT>
-__global__ void __launch_bounds__(kThreads) prepare_vec(const uint4* __restrict__ w, int64_t nv,
+__global__ void __launch_bounds__(kThreads, 4) prepare_vec(const uint4* __restrict__ w, int64_t nv,
                                                         uint8_t* __restrict__ pass, uint2* __restrict__ values,
                                                         uint8_t* __restrict__ meta, unsigned int* __restrict__ acc,
                                                         int32_t* __restrict__ n_fail, float* __restrict__ ts_w,

@@ -508,7 +508,6 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
 constexpr int kDecWarps = 16;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecMaxTiles = 32;  // per-CTA tile buffers (16 rows x 8 tokens fp32 each)
-constexpr int kDecDepth = 2;      // units in flight per warp
 
 template <int WF>
 struct U3;
@@ -556,13 +555,14 @@ __device__ __forceinline__ void issue_unit(uint8_t* slot, const SkinnyParams& p,
   }
 }
 
-// Dynamic shared memory of the decode kernel: x (16 K bytes) + every warp's unit buffers.
+// Dynamic shared memory of the decode kernel: x (16 K bytes) + every warp's DEPTH unit buffers.
 template <int WF>
-constexpr size_t decode_smem(int64_t K) {
-  return 16 * (size_t)K + (size_t)kDecWarps * kDecDepth * U3<WF>::SLOT;
+constexpr size_t decode_smem(int64_t K, int depth) {
+  return 16 * (size_t)K + (size_t)kDecWarps * depth * U3<WF>::SLOT;
 }
+constexpr size_t kDecSmemMax = 227 * 1024 - sizeof(float) * kDecMaxTiles * 128;
 
-template <int WF, typename T>
+template <int WF, typename T, int kDecDepth>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const SkinnyParams p) {
   using U = U3<WF>;
   extern __shared__ __align__(16) uint8_t dsm[];
@@ -581,14 +581,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
   for (int i = threadIdx.x; i < nloc * 128; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
 
   // ---- x: one 16-byte piece per (token, 8 k); consecutive threads take consecutive pieces of a row
-  const int64_t kp8 = p.K / 8;
+  const int kp8 = (int)(p.K / 8);                // 32-bit index math: K <= 8192 here
   const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
-  for (int64_t i = threadIdx.x; i < 8 * kp8; i += blockDim.x) {
-    const int g = (int)(i / kp8);
-    const int64_t k = (i - g * kp8) * 8;
+  for (int i = threadIdx.x; i < 8 * kp8; i += blockDim.x) {
+    const int g = i / kp8;
+    const int k = (i - g * kp8) * 8;
     uint8_t* dst = xs + xoff(g, k);
     if (g < p.M)
-      tc::cp_async16(dst, xg + g * p.K + k);
+      tc::cp_async16(dst, xg + (int64_t)g * p.K + k);
     else
       *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
   }
@@ -717,8 +717,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
 
 template <int WF, typename T>
 int launch_decode(const SkinnyParams& p, cudaStream_t s) {
-  const size_t smem = decode_smem<WF>(p.K);
-  auto kern = decode_gemv_kernel<WF, T>;
+  // three units in flight per warp when they fit beside x, else two
+  const bool deep = decode_smem<WF>(p.K, 3) <= kDecSmemMax;
+  const size_t smem = decode_smem<WF>(p.K, deep ? 3 : 2);
+  auto kern = deep ? decode_gemv_kernel<WF, T, 3> : decode_gemv_kernel<WF, T, 2>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   if (cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
@@ -758,14 +760,14 @@ bool decode_supported(int wf, const SkinnyParams& p) {
   size_t smem;
   if (wf == W_DQ4) {
     uk = U3<W_DQ4>::UK;
-    smem = decode_smem<W_DQ4>(p.K);
+    smem = decode_smem<W_DQ4>(p.K, 2);
   } else if (wf == W_SQ4 && aligned(p.meta, 16)) {
     uk = U3<W_SQ4>::UK;
-    smem = decode_smem<W_SQ4>(p.K);
+    smem = decode_smem<W_SQ4>(p.K, 2);
   } else {
     return false;
   }
-  if (p.K % uk || smem + sizeof(float) * kDecMaxTiles * 128 > 227 * 1024) return false;
+  if (p.K % uk || smem > kDecSmemMax) return false;
   const int64_t upr = p.K / uk, units = (p.N / 16) * upr, grid = sm_count();
   if (units >= (int64_t(1) << 31)) return false;
   const int64_t per_cta = (units + grid - 1) / grid;
