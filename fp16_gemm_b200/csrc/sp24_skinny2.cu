@@ -555,34 +555,62 @@ __device__ __forceinline__ void issue_unit(uint8_t* slot, const SkinnyParams& p,
   }
 }
 
-// Dynamic shared memory of the decode kernel: x (16 K bytes) + every warp's DEPTH unit buffers.
+// Dynamic shared memory of the decode kernel: the staged x columns (16 bytes per column) and
+// every warp's DEPTH unit buffers.
 template <int WF>
-constexpr size_t decode_smem(int64_t K, int depth) {
-  return 16 * (size_t)K + (size_t)kDecWarps * depth * U3<WF>::SLOT;
+constexpr size_t decode_smem(int64_t xcols, int depth) {
+  return 16 * (size_t)xcols + (size_t)kDecWarps * depth * U3<WF>::SLOT;
 }
 constexpr size_t kDecSmemMax = 227 * 1024 - sizeof(float) * kDecMaxTiles * 128;
 
+// Work split of the decode kernel: k-groups of G units (G divides the units per tile).  A CTA's
+// contiguous unit range must span at most two k-groups and touch at most kDecMaxTiles tiles;
+// the smallest G of at least about 1024 k that satisfies this keeps the staged x small.
+// Returns 0 when no G works; *xcols receives the x columns a CTA stages.
+template <int WF>
+int decode_group(const SkinnyParams& p, int64_t* xcols) {
+  const int64_t uk = U3<WF>::UK, upr = p.K / uk, T = p.N / 16, grid = sm_count();
+  const int64_t per_cta = (T * upr + grid - 1) / grid;
+  const int64_t target = (1024 + uk - 1) / uk;
+  for (int64_t g = 1; g <= upr; ++g) {
+    if (upr % g || (g < target && g < upr)) continue;
+    if (per_cta > T * g || per_cta / g + 3 > kDecMaxTiles) continue;
+    const int64_t cols = (upr / g >= 2 ? 2 * g : g) * uk;
+    if (decode_smem<WF>(cols, 2) > kDecSmemMax) return 0;
+    *xcols = cols;
+    return (int)g;
+  }
+  return 0;
+}
+
 template <int WF, typename T, int kDecDepth>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const SkinnyParams p) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const SkinnyParams p, int G) {
   using U = U3<WF>;
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint8_t* xs = dsm;                            // 16 * K bytes
-  uint8_t* slots = dsm + 16 * p.K;              // kDecWarps x kDecDepth x SLOT
   __shared__ float tbuf[kDecMaxTiles][16][8];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int upr = (int)(p.K / U::UK);           // units per 16-row tile
-  const int64_t U_all = (p.N / 16) * upr;       // < 2^31 (host check)
+  const int NT16 = (int)(p.N / 16), TG = NT16 * G;  // tiles; units per k-group
+  const int64_t U_all = (int64_t)NT16 * upr;         // < 2^31 (host check)
   const int ub = (int)(U_all * blockIdx.x / gridDim.x), ue = (int)(U_all * (blockIdx.x + 1) / gridDim.x);
   const int nunits = ue - ub;
   if (nunits <= 0) return;                      // whole CTA, before any barrier
-  const int t0 = ub / upr;
-  const int nloc = (ue - 1) / upr - t0 + 1;     // <= kDecMaxTiles (host check)
+  // unit u = (k-group kg, tile, kq): kp = kg * G + kq.  A CTA's range spans at most two k-groups
+  // (host check); its tiles get shared-buffer slots: [tf, NT16) of kg_lo, then [0, tl] of kg_hi.
+  const int kg_lo = ub / TG, kg_hi = (ue - 1) / TG;
+  const int tf = (ub - kg_lo * TG) / G, tl = (ue - 1 - kg_hi * TG) / G;
+  const int nlo = kg_lo == kg_hi ? tl - tf + 1 : NT16 - tf;
+  const int nloc = kg_lo == kg_hi ? nlo : nlo + tl + 1;   // <= kDecMaxTiles (host check)
+  const int64_t k0 = (int64_t)kg_lo * G * U::UK;          // x columns staged: [k0, k0 + kx)
+  const int kx = (kg_hi - kg_lo + 1) * G * U::UK;
+  uint8_t* xs = dsm;                            // 16 * kx bytes
+  uint8_t* slots = dsm + 16 * kx;               // kDecWarps x kDecDepth x SLOT
   for (int i = threadIdx.x; i < nloc * 128; i += blockDim.x) (&tbuf[0][0][0])[i] = 0.f;
 
   // ---- x: one 16-byte piece per (token, 8 k); consecutive threads take consecutive pieces of a row
-  const int kp8 = (int)(p.K / 8);                // 32-bit index math: K <= 8192 here
-  const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
+  const int kp8 = kx / 8;
+  const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x) + k0;
   for (int i = threadIdx.x; i < 8 * kp8; i += blockDim.x) {
     const int g = i / kp8;
     const int k = (i - g * kp8) * 8;
@@ -593,6 +621,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
       *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
   }
   tc::cp_async_commit();
+  auto unit_at = [&](int u, int& slot, int& tile, int& kp) {
+    const int kg = u / TG, rem = u - kg * TG;
+    tile = rem / G;
+    kp = kg * G + (rem - tile * G);
+    slot = kg == kg_lo ? tile - tf : nlo + tile;
+  };
 
   // ---- this warp's units: local index warp + kDecWarps * n; the first kDecDepth in flight now
   uint8_t* wslots = slots + warp * kDecDepth * U::SLOT;
@@ -600,8 +634,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
   for (int d = 0; d < kDecDepth; ++d) {
     const int i = warp + kDecWarps * d;
     if (i < nunits) {
-      const int u = ub + i, tile = u / upr;
-      issue_unit<WF>(wslots + d * U::SLOT, p, tile, u - tile * upr, lane);
+      int sl, tile, kp;
+      unit_at(ub + i, sl, tile, kp);
+      issue_unit<WF>(wslots + d * U::SLOT, p, tile, kp, lane);
     }
     tc::cp_async_commit();  // possibly empty: keeps the group count uniform
   }
@@ -613,7 +648,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
   float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
   int cur = -1;
   auto flush = [&]() {
-    float* b = &tbuf[cur - t0][0][0];
+    float* b = &tbuf[cur][0][0];
     atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
     atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
     atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
@@ -622,10 +657,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
     for (int q = 0; q < 4; ++q) acc[q] = acc2[q] = 0.f;
   };
   for (int n = 0, i = warp; i < nunits; ++n, i += kDecWarps) {
-    const int u = ub + i, tile = u / upr, kp = u - tile * upr;
-    if (tile != cur) {
+    int slt, tile, kp;
+    unit_at(ub + i, slt, tile, kp);
+    if (slt != cur) {
       if (cur >= 0) flush();
-      cur = tile;
+      cur = slt;
     }
     tc::cp_async_wait<kDecDepth - 1>();  // this unit's group (all but the newest) has landed
     __syncwarp();
@@ -651,7 +687,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
         for (int ch = 0; ch < 2; ++ch) {
           // x[g][P .. P+8), P = chunk base + 32c + 8q: codes at nibbles (i, i+4) of word q pair
           // with x entries (i, i+4)
-          const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff(g, kp * 256 + ch * 128 + 32 * c + 8 * q));
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff(g, kp * 256 - k0 + ch * 128 + 32 * c + 8 * q));
           const uint32_t s0 = sa[ch][q >> 1], s1 = sb[ch][q >> 1];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -685,7 +721,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
         const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
         const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
         // x[g][32w' + 2c + 8i + {0, 1}], i = 0..3: word c of four consecutive 16-byte pieces
-        const int64_t kw = (int64_t)kp * 512 + 32 * w;
+        const int64_t kw = (int64_t)kp * 512 - k0 + 32 * w;
         const uint8_t* xr = xs + 4 * c;
         const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr + xoff(g, kw)),
                                     *reinterpret_cast<const uint32_t*>(xr + xoff(g, kw + 8)),
@@ -697,8 +733,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
     __syncwarp();  // every lane is done with the slot before it is refilled
     const int inext = i + kDecWarps * kDecDepth;
     if (inext < nunits) {
-      const int u2 = ub + inext, t2 = u2 / upr;
-      issue_unit<WF>(slot, p, t2, u2 - t2 * upr, lane);
+      int s2, t2, k2;
+      unit_at(ub + inext, s2, t2, k2);
+      issue_unit<WF>(slot, p, t2, k2, lane);
     }
     tc::cp_async_commit();
   }
@@ -709,7 +746,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
   const float scale = 256.0f * *p.w_ts;
   for (int e = threadIdx.x; e < nloc * 128; e += blockDim.x) {
     const int lt = e >> 7, row = (e >> 3) & 15, tok = e & 7;
-    const int64_t gr = (int64_t)(t0 + lt) * 16 + row;
+    const int tile = lt < nlo ? tf + lt : lt - nlo;
+    const int64_t gr = (int64_t)tile * 16 + row;
     const float v = (&tbuf[0][0][0])[e];
     if (tok < p.M && gr < p.N && v != 0.0f) atomicAdd(p.y + (int64_t)tok * p.N + gr, v * scale);
   }
@@ -717,14 +755,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_gemv_kernel(const Skinn
 
 template <int WF, typename T>
 int launch_decode(const SkinnyParams& p, cudaStream_t s) {
+  int64_t xcols = 0;
+  const int G = decode_group<WF>(p, &xcols);
+  if (!G) return SP24_ERR_UNSUPPORTED;
   // three units in flight per warp when they fit beside x, else two
-  const bool deep = decode_smem<WF>(p.K, 3) <= kDecSmemMax;
-  const size_t smem = decode_smem<WF>(p.K, deep ? 3 : 2);
+  const bool deep = decode_smem<WF>(xcols, 3) <= kDecSmemMax;
+  const size_t smem = decode_smem<WF>(xcols, deep ? 3 : 2);
   auto kern = deep ? decode_gemv_kernel<WF, T, 3> : decode_gemv_kernel<WF, T, 2>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   if (cudaMemsetAsync(p.y, 0, (size_t)(p.M * p.N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
-  kern<<<sm_count(), kDecThreads, smem, s>>>(p);
+  kern<<<sm_count(), kDecThreads, smem, s>>>(p, G);
   return launch_status();
 }
 
@@ -751,27 +792,15 @@ int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStre
 
 // True when the persistent decode kernel takes the problem: 16-bit x of at most 8 tokens
 // (16-byte aligned rows), NVFP4 weights (dense or 2:4) in whole 16-row tiles, K a whole number of
-// units, x plus the warps' unit buffers within shared memory, and at most kDecMaxTiles tiles
-// touched by any CTA.
+// units, and a k-group split that fits (decode_group).
 bool decode_supported(int wf, const SkinnyParams& p) {
-  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0) return false;
+  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.N == 0 || p.K == 0) return false;
   if (!aligned(p.x, 16) || !aligned(p.w, 16) || !aligned(p.w_scales, 16)) return false;
-  int64_t uk;
-  size_t smem;
-  if (wf == W_DQ4) {
-    uk = U3<W_DQ4>::UK;
-    smem = decode_smem<W_DQ4>(p.K, 2);
-  } else if (wf == W_SQ4 && aligned(p.meta, 16)) {
-    uk = U3<W_SQ4>::UK;
-    smem = decode_smem<W_SQ4>(p.K, 2);
-  } else {
-    return false;
-  }
-  if (p.K % uk || smem > kDecSmemMax) return false;
-  const int64_t upr = p.K / uk, units = (p.N / 16) * upr, grid = sm_count();
-  if (units >= (int64_t(1) << 31)) return false;
-  const int64_t per_cta = (units + grid - 1) / grid;
-  return per_cta / upr + 2 <= kDecMaxTiles;
+  if ((p.N / 16) * (p.K / 256) >= (int64_t(1) << 31)) return false;
+  int64_t xcols;
+  if (wf == W_DQ4) return p.K % U3<W_DQ4>::UK == 0 && decode_group<W_DQ4>(p, &xcols) > 0;
+  if (wf == W_SQ4) return aligned(p.meta, 16) && p.K % U3<W_SQ4>::UK == 0 && decode_group<W_SQ4>(p, &xcols) > 0;
+  return false;
 }
 
 int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s) {
