@@ -158,11 +158,16 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
 // E2M1's rounding boundaries (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) matters.  With the block's
 // divisor sc in [2^-100, 2^100], q = RN(|v| * RN(1 / sc)) is within 2.01 ulp of |v| / sc (two
 // roundings of 2^-24 each), so q and fl(|v| / sc) give the same code unless q lies within a few
-// ulps of a boundary.  Every boundary has at most three significant bits, i.e. a zero in the low
-// 21 bits of its fp32 significand; an entry whose q is within 4 ulps of such a value (which also
-// covers the power-of-two boundary 0.25, where the ulp halves) takes the IEEE division instead,
-// together with the other entry of its pair.
-// The codes are therefore exactly those of the per-entry division, at one multiply per entry.
+// ulps of a boundary.  Every boundary is a multiple of 0.25: rounding q to the nearest multiple
+// of 0.25 (adding and subtracting 2^21 in fp32) and testing |q - that| < q * 2^-21 (a window of
+// 4 to 8 ulps of q; never true for q = 0) flags every such q.  A pair with a flagged entry takes
+// the IEEE division for both entries.  The codes are therefore exactly those of the per-entry
+// division, at a multiply and four FMA-pipe operations per entry.
+__device__ __forceinline__ bool near_quarter(float q) {
+  const float r = __fadd_rn(__fadd_rn(q, 0x1p21f), -0x1p21f);   // nearest multiple of 0.25
+  return __fmaf_rn(q, 0x1p-21f, -fabsf(__fadd_rn(q, -r))) > 0.0f;
+}
+
 __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, float d, uint2* codes,
                                              uint8_t* scales, int64_t b) {
   float bmax = 0.0f;
@@ -180,9 +185,8 @@ __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, fl
     if (fast) {
       q0 = __fmul_rn(a0, y);
       q1 = __fmul_rn(a1, y);
-      const uint32_t u0 = __float_as_uint(q0), u1 = __float_as_uint(q1);
-      if ((((u0 + 4u) & 0x1fffffu) <= 8u && u0 != 0u) || (((u1 + 4u) & 0x1fffffu) <= 8u && u1 != 0u)) {
-        q0 = __fdiv_rn(a0, sc);  // within 4 ulp of a value with <= 3 significant bits
+      if (near_quarter(q0) || near_quarter(q1)) {
+        q0 = __fdiv_rn(a0, sc);  // within 4 ulp of a multiple of 0.25
         q1 = __fdiv_rn(a1, sc);
       }
     } else {
