@@ -34,7 +34,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_quantize_nvfp4", "sp24_dequantize_nvfp4", "sp24_gemm_workspace_size",
            "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
            "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc", "sp24_gemm_grouped_workspace_size",
-           "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24")
+           "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24",
+           "sp24_quantize_nvfp4_pair")
 
 _lock = threading.Lock()
 _lib = None
@@ -90,6 +91,7 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
             L.sp24_prepare_24_workspace_size.argtypes = [I64, I64, P]
             L.sp24_prepare_24.argtypes = [P, I, I64, I64, P, P, P, P, P, P, P, I64, P]
+            L.sp24_quantize_nvfp4_pair.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, I64, P, P, P, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -242,6 +244,28 @@ def quantize_nvfp4(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None,
     return out
 
 
+def quantize_nvfp4_pair(t0: torch.Tensor, ts0: torch.Tensor, t1: torch.Tensor, ts1: torch.Tensor,
+                        out0=None, out1=None, stream=None):
+    """NVFP4 of two 2-D tensors of one dtype in one launch, each with its supplied tensor scale
+    (fp32 [1], device); identical to quantize_nvfp4(t0, ts0) and quantize_nvfp4(t1, ts1)."""
+    _cuda(t0, "t0")
+    _cuda(t1, "t1")
+    if t0.dim() != 2 or t1.dim() != 2 or t0.dtype != t1.dtype:
+        raise ValueError("quantize_nvfp4_pair wants two 2-D tensors of one dtype")
+    outs = []
+    for t, o in ((t0, out0), (t1, out1)):
+        R, L = t.shape
+        outs.append(o if o is not None else NVFP4Tensor(
+            torch.empty((R, L // 2), dtype=torch.uint8, device=t.device),
+            torch.empty((R, L // 16), dtype=torch.uint8, device=t.device),
+            torch.empty(1, dtype=torch.float32, device=t.device)))
+    a, b = outs
+    _call("sp24_quantize_nvfp4_pair", _ptr(t0), _dtype_code(t0), t0.shape[0], t0.shape[1], _ptr(ts0),
+          _ptr(a.codes), _ptr(a.scales), _ptr(a.tensor_scale), _ptr(t1), t1.shape[0], t1.shape[1],
+          _ptr(ts1), _ptr(b.codes), _ptr(b.scales), _ptr(b.tensor_scale), _stream(stream))
+    return a, b
+
+
 def quantize_nvfp4_noalloc(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None, out=None,
                            stream=None) -> NVFP4Tensor:
     """quantize_nvfp4 without a workspace: the library's own per-device scratch is used, so the
@@ -314,8 +338,7 @@ def prepare_nvfp4_24(w: torch.Tensor, stream=None):
     values with the tensor scales prepare_24 derived.  Returns (Prepared24, dense NVFP4Tensor,
     Sparse24 with NVFP4 values)."""
     p = prepare_24(w, stream=stream)
-    wq = quantize_nvfp4(w, tensor_scale=p.w_tensor_scale, stream=stream)
-    vq = quantize_nvfp4(p.values, tensor_scale=p.v_tensor_scale, stream=stream)
+    wq, vq = quantize_nvfp4_pair(w, p.w_tensor_scale, p.values, p.v_tensor_scale, stream=stream)
     return p, wq, Sparse24(vq, p.meta)
 
 

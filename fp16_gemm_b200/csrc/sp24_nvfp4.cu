@@ -230,6 +230,46 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restr
       });
 }
 
+// Encode pass over two tensors in one launch, each with its supplied tensor scale.
+struct EncodeJob {
+  const void* t;
+  int64_t nblk;
+  const float* ts_in;
+  uint2* codes;
+  uint8_t* scales;
+  float* ts_out;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 4) encode_pair_kernel(EncodeJob ja, EncodeJob jb) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  constexpr int BB = block_bytes<DT>();
+  const float s_a = *ja.ts_in, s_b = *jb.ts_in;
+  __syncthreads();  // every thread has read the scales before ts_out (which may alias) is written
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *ja.ts_out = s_a;
+    *jb.ts_out = s_b;
+  }
+  const float d_a = __fmul_rn(s_a, 6.0f), d_b = __fmul_rn(s_b, 6.0f);
+  stream::for_each_chunk2<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(ja.t), ja.nblk * BB, reinterpret_cast<const uint8_t*>(jb.t),
+      jb.nblk * BB, ring, [&](const uint8_t* chunk, int seg, int64_t c, int bytes) {
+        const int nb = bytes / BB;
+        const int64_t b0 = c * (kChunk / BB);
+        uint2* codes = seg ? jb.codes : ja.codes;
+        uint8_t* scales = seg ? jb.scales : ja.scales;
+        const float s_t = seg ? s_b : s_a, d = seg ? d_b : d_a;
+#pragma unroll
+        for (int q = 0; q < kChunk / BB / kThreads; ++q) {
+          const int j = threadIdx.x + q * kThreads;
+          if (j >= nb) continue;
+          float v[16];
+          smem_block<DT>(chunk + j * BB, v);
+          encode_block(v, s_t, d, codes, scales, b0 + j);
+        }
+      });
+}
+
 // One byte (two entries) per thread; value computed in fp64 (exact) and rounded once.
 template <int OUT>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const uint8_t* __restrict__ codes,
@@ -325,6 +365,32 @@ extern "C" int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64
   }
   return quantize_nvfp4_launch(t, dtype, rows, cols, tensor_scale_in, codes, scales,
                                tensor_scale_out, amax_word, as_stream(stream));
+}
+
+extern "C" int sp24_quantize_nvfp4_pair(const void* t0, int dtype, int64_t rows0, int64_t cols0,
+                                        const float* ts0, uint8_t* codes0, uint8_t* scales0, float* ts_out0,
+                                        const void* t1, int64_t rows1, int64_t cols1, const float* ts1,
+                                        uint8_t* codes1, uint8_t* scales1, float* ts_out1, void* stream) {
+  const int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  if (rows0 < 0 || cols0 < 0 || cols0 % 16 || rows1 < 0 || cols1 < 0 || cols1 % 16) return SP24_ERR_SHAPE;
+  if (!ts0 || !ts1 || !ts_out0 || !ts_out1) return SP24_ERR_INVALID_ARG;
+  const int64_t n0 = rows0 * cols0 / 16, n1 = rows1 * cols1 / 16;
+  if ((n0 > 0 && (!t0 || !codes0 || !scales0)) || (n1 > 0 && (!t1 || !codes1 || !scales1))) return SP24_ERR_INVALID_ARG;
+  if ((n0 > 0 && (!aligned(t0, 16) || !aligned(codes0, 8))) || (n1 > 0 && (!aligned(t1, 16) || !aligned(codes1, 8))))
+    return SP24_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const EncodeJob a{t0, n0, ts0, (uint2*)codes0, scales0, ts_out0};
+  const EncodeJob b{t1, n1, ts1, (uint2*)codes1, scales1, ts_out1};
+  const int64_t bytes = (n0 + n1) * (dtype == SP24_F32 ? 64 : 32);
+  // launched even for empty tensors, so that both tensor scales are written
+  if (dtype == SP24_F32)
+    encode_pair_kernel<SP24_F32><<<ring_grid(encode_pair_kernel<SP24_F32>, bytes), kThreads, kRingBytes, s>>>(a, b);
+  else if (dtype == SP24_BF16)
+    encode_pair_kernel<SP24_BF16><<<ring_grid(encode_pair_kernel<SP24_BF16>, bytes), kThreads, kRingBytes, s>>>(a, b);
+  else
+    encode_pair_kernel<SP24_F16><<<ring_grid(encode_pair_kernel<SP24_F16>, bytes), kThreads, kRingBytes, s>>>(a, b);
+  return launch_status();
 }
 
 extern "C" int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,

@@ -23,15 +23,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// Runs body(stage_ptr, chunk_index, chunk_bytes) over this CTA's chunks of `src` (nbytes, a
-// multiple of 16, src 16-byte aligned).  `ring` must hold S * CHUNK bytes of dynamic shared
+// Runs body(stage_ptr, segment, chunk_index_in_segment, chunk_bytes) over this CTA's chunks of
+// two inputs taken as one sequence: the chunks of `a` (abytes), then those of `b` (bbytes, may
+// be 0).  Chunks c = blockIdx.x, blockIdx.x + gridDim.x, ... of that sequence.  Sizes are
+// multiples of 16, sources 16-byte aligned.  `ring` must hold S * CHUNK bytes of dynamic shared
 // memory, 16-byte aligned.
 template <int CHUNK, int S, class Body>
-__device__ __forceinline__ void for_each_chunk(const uint8_t* __restrict__ src, int64_t nbytes, uint8_t* ring,
-                                               Body&& body) {
+__device__ __forceinline__ void for_each_chunk2(const uint8_t* __restrict__ a, int64_t abytes,
+                                                const uint8_t* __restrict__ b, int64_t bbytes, uint8_t* ring,
+                                                Body&& body) {
   __shared__ uint64_t bars[S];
   __shared__ int abort_flag;
-  const int64_t nchunks = (nbytes + CHUNK - 1) / CHUNK;
+  const int64_t na = (abytes + CHUNK - 1) / CHUNK;
+  const int64_t nchunks = na + (bbytes + CHUNK - 1) / CHUNK;
   const int64_t mine = blockIdx.x < nchunks ? (nchunks - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) tc::mbar_init(&bars[s], 1);
@@ -39,12 +43,21 @@ __device__ __forceinline__ void for_each_chunk(const uint8_t* __restrict__ src, 
     tc::fence_mbar_init();
   }
   __syncthreads();
+  // (segment, byte offset in it, size) of sequence chunk c
+  auto locate = [&](int64_t c, int& seg, int64_t& off, uint32_t& sz) {
+    seg = c >= na;
+    off = (seg ? c - na : c) * (int64_t)CHUNK;
+    const int64_t n = seg ? bbytes : abytes;
+    sz = (uint32_t)(n - off < CHUNK ? n - off : CHUNK);
+  };
   auto issue = [&](int64_t i) {
     const int s = (int)(i % S);
-    const int64_t off = (blockIdx.x + i * gridDim.x) * (int64_t)CHUNK;
-    const uint32_t sz = (uint32_t)(nbytes - off < CHUNK ? nbytes - off : CHUNK);
+    int seg;
+    int64_t off;
+    uint32_t sz;
+    locate(blockIdx.x + i * gridDim.x, seg, off, sz);
     tc::mbar_arrive_expect_tx(&bars[s], sz);
-    bulk_g2s(ring + s * CHUNK, src + off, sz, &bars[s]);
+    bulk_g2s(ring + s * CHUNK, (seg ? b : a) + off, sz, &bars[s]);
   };
   if (threadIdx.x == 0)
     for (int64_t i = 0; i < (mine < S ? mine : S); ++i) issue(i);
@@ -53,9 +66,11 @@ __device__ __forceinline__ void for_each_chunk(const uint8_t* __restrict__ src, 
     const int s = (int)(i % S);
     const bool ok = tc::mbar_wait(&bars[s], (uint32_t)((i / S) & 1));
     if (!ok) abort_flag = 1;
-    const int64_t c = blockIdx.x + i * gridDim.x;
-    const int64_t off = c * (int64_t)CHUNK;
-    if (ok) body(ring + s * CHUNK, c, (int)(nbytes - off < CHUNK ? nbytes - off : CHUNK));
+    int seg;
+    int64_t off;
+    uint32_t sz;
+    locate(blockIdx.x + i * gridDim.x, seg, off, sz);
+    if (ok) body(ring + s * CHUNK, seg, off / CHUNK, (int)sz);
     __syncthreads();
     if (abort_flag) break;
     if (threadIdx.x == 0 && i + S < mine) issue(i + S);
@@ -66,6 +81,15 @@ __device__ __forceinline__ void for_each_chunk(const uint8_t* __restrict__ src, 
     const int64_t last = i + S < mine ? i + S : mine;
     for (int64_t j = i; j < last; ++j) tc::mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1));
   }
+}
+
+// Runs body(stage_ptr, chunk_index, chunk_bytes) over this CTA's chunks of `src` (nbytes, a
+// multiple of 16, src 16-byte aligned): chunks c = blockIdx.x, blockIdx.x + gridDim.x, ...
+template <int CHUNK, int S, class Body>
+__device__ __forceinline__ void for_each_chunk(const uint8_t* __restrict__ src, int64_t nbytes, uint8_t* ring,
+                                               Body&& body) {
+  for_each_chunk2<CHUNK, S>(src, nbytes, nullptr, 0, ring,
+                            [&](const uint8_t* stage, int, int64_t c, int bytes) { body(stage, c, bytes); });
 }
 
 }  // namespace stream

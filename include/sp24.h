@@ -163,6 +163,16 @@ int sp24_quantize_nvfp4_noalloc(const void* t, int dtype, int64_t rows, int64_t 
                                 const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
                                 float* tensor_scale_out, void* stream);
 
+/* Two quantisations in one launch (a weight and its 2:4 values, with the tensor scales that
+ * sp24_prepare_24 derived, say): the results equal those of sp24_quantize_nvfp4(t0, ts0) and
+ * sp24_quantize_nvfp4(t1, ts1).  Both tensors have type `dtype`; each tensor scale is required
+ * (device fp32) and is copied to its ts_out (which may be the same pointer).  Shapes, layouts
+ * and alignment as for sp24_quantize_nvfp4; either tensor may be empty.  No workspace. */
+int sp24_quantize_nvfp4_pair(const void* t0, int dtype, int64_t rows0, int64_t cols0,
+                             const float* ts0, uint8_t* codes0, uint8_t* scales0, float* ts_out0,
+                             const void* t1, int64_t rows1, int64_t cols1, const float* ts1,
+                             uint8_t* codes1, uint8_t* scales1, float* ts_out1, void* stream);
+
 /* Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
  * (F16/BF16/F32). */
 int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,

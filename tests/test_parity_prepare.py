@@ -118,3 +118,32 @@ def test_rejected_arguments():
     with pytest.raises(sp.SP24Error) as e:
         sp.prepare_24(buf[1:1 + 4 * 64].view(4, 64))                                # W misaligned
     assert e.value.status == sp.ERR_ALIGN
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_quantize_pair_matches_two_calls_and_oracle(dtype):
+    """One launch encoding two tensors with supplied scales equals two quantize_nvfp4 calls with
+    the same scales, and the oracle's encodings with those scales; an empty second tensor still
+    gets its tensor scale copied."""
+    od = ORACLE_DT[dtype]
+    g = synth.rng(31)
+    a_np = synth.as_storage(synth.normal(g, (70, 320)) * np.exp(synth.normal(g, (70, 1))), dtype)
+    b_np = synth.structured_edge(g, 33, 160, dtype)
+    ts_a = oracle.nvfp4_tensor_scale(a_np, od)
+    ts_b = oracle.nvfp4_tensor_scale(b_np, od) * 2.0  # a shared, larger scale
+    a, b = to_dev(a_np, dtype), to_dev(b_np, dtype)
+    ta = torch.tensor([ts_a], dtype=torch.float32, device="cuda")
+    tb = torch.tensor([ts_b], dtype=torch.float32, device="cuda")
+    qa, qb = sp.quantize_nvfp4_pair(a, ta, b, tb)
+    ra, rb = sp.quantize_nvfp4(a, tensor_scale=ta), sp.quantize_nvfp4(b, tensor_scale=tb)
+    torch.cuda.synchronize()
+    for q, r in ((qa, ra), (qb, rb)):
+        assert torch.equal(q.codes, r.codes) and torch.equal(q.scales, r.scales)
+        assert torch.equal(q.tensor_scale, r.tensor_scale)
+    _same_nvfp4(qa, oracle.nvfp4_encode(a_np, od, ts_a), "first")
+    _same_nvfp4(qb, oracle.nvfp4_encode(b_np, od, float(np.float32(ts_b))), "second")
+    e = torch.empty((0, 32), dtype=a.dtype, device="cuda")
+    qa2, qe = sp.quantize_nvfp4_pair(a, ta, e, tb)
+    torch.cuda.synchronize()
+    assert torch.equal(qa2.codes, ra.codes) and qe.codes.numel() == 0
+    assert qe.tensor_scale.item() == tb.item()
