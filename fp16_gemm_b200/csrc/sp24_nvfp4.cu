@@ -202,6 +202,109 @@ __device__ __forceinline__ void encode_block(const float (&v)[16], float s_t, fl
   scales[b] = (uint8_t)sb;
 }
 
+// ---- 16-bit inputs: codes by counting thresholds, no per-entry division.
+//
+// fl32(a / sc) rounds (RNE, saturating) to an E2M1 code above j exactly when a / sc > T_j, with
+// T_j the boundary between codes j and j + 1 moved half an fp32 ulp to the side its tie goes:
+// away from the odd code (0.25, 1.25, 2.5 and 5 round down on a tie, 0.75, 1.75 and 3.5 up).
+// a / sc never equals T_j (T_j has more significant bits than any ratio of two fp32 values can
+// produce), so for a 16-bit a the test is a >= RU16(T_j * sc), where T_j * sc is exact in fp64.
+// Each CTA tabulates the seven 16-bit thresholds for every E4M3 block-scale code (a zero
+// divisor gets NaN thresholds: every compare fails, code 0), and an entry's code is the number
+// of thresholds it reaches, counted two entries at a time with packed compares and adds.
+__constant__ double kE2M1Bound[7] = {0.25 + 0x1p-26, 0.75 - 0x1p-25, 1.25 + 0x1p-24, 1.75 - 0x1p-24,
+                                     2.5 + 0x1p-23,  3.5 - 0x1p-23,  5.0 + 0x1p-22};
+
+template <int DT>
+struct Pack16;
+template <>
+struct Pack16<SP24_BF16> {
+  static constexpr uint32_t BIAS = 0x43004300u;  // 128.0 twice: 128 + k has k in its low bits
+  static constexpr uint32_t QNAN = 0x7FC07FC0u;
+};
+template <>
+struct Pack16<SP24_F16> {
+  static constexpr uint32_t BIAS = 0x64006400u;  // 1024.0 twice
+  static constexpr uint32_t QNAN = 0x7E007E00u;
+};
+
+template <int DT>
+__device__ __forceinline__ uint32_t ge2(uint32_t a, uint32_t b) {  // 1.0 / 0.0 per half
+  uint32_t r;
+  if (DT == SP24_BF16) asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else asm("set.ge.f16x2.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <int DT>
+__device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if (DT == SP24_BF16) asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <int DT>
+__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {  // NaN loses, as in fmaxf
+  uint32_t r;
+  if (DT == SP24_BF16) asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Smallest 16-bit value of type DT at or above x (x exact in fp64; rounding up twice is rounding
+// up once).
+template <int DT>
+__device__ __forceinline__ uint32_t ru16(double x) {
+  const float f = __double2float_ru(x);
+  if (DT == SP24_BF16) return __bfloat16_as_ushort(__float2bfloat16_ru(f));
+  return __half_as_ushort(__float2half_ru(f));
+}
+
+// tab[8 c + j] = threshold j of block-scale code c, in both halves (j = 7 unused).
+template <int DT>
+__device__ void build_thresholds(float s_t, uint32_t* tab) {
+  for (int i = threadIdx.x; i < 128 * 8; i += blockDim.x) {
+    const int c = i >> 3, j = i & 7;
+    uint32_t v = Pack16<DT>::QNAN;
+    if (j < 7 && c < 127) {
+      const float sc = __fmul_rn(e4m3_value(c), s_t);
+      if (sc != 0.0f) {
+        const uint32_t h = ru16<DT>(kE2M1Bound[j] * (double)sc);
+        v = h | (h << 16);
+      }
+    }
+    tab[i] = v;
+  }
+}
+
+// Encodes one block of 16 16-bit entries (32 bytes at p) with the thresholds of its scale code.
+template <int DT>
+__device__ __forceinline__ void encode_block16(const uint8_t* p, const uint32_t* tab, float d, uint2* codes,
+                                               uint8_t* scales, int64_t b) {
+  const uint4 u0 = reinterpret_cast<const uint4*>(p)[0], u1 = reinterpret_cast<const uint4*>(p)[1];
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  uint32_t a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = w[i] & 0x7fff7fffu;
+  const uint32_t m = max2<DT>(max2<DT>(max2<DT>(a[0], a[1]), max2<DT>(a[2], a[3])),
+                              max2<DT>(max2<DT>(a[4], a[5]), max2<DT>(a[6], a[7])));
+  const float bmax = fmaxf(to_f32<DT>(m & 0xffffu), to_f32<DT>(m >> 16));
+  const uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
+  const uint4 t0 = reinterpret_cast<const uint4*>(tab + 8 * sb)[0];
+  const uint4 t1 = reinterpret_cast<const uint4*>(tab + 8 * sb)[1];
+  const uint32_t th[7] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z};
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t acc = Pack16<DT>::BIAS;
+#pragma unroll
+    for (int j = 0; j < 7; ++j) acc = add2<DT>(acc, ge2<DT>(a[i], th[j]));
+    // codes in bits 0-2 and 16-18, signs of the two entries to bits 3 and 19
+    const uint32_t x = (acc & 0x00070007u) | ((w[i] >> 12) & 0x00080008u);
+    packed[i >> 2] |= ((x | (x >> 12)) & 0xffu) << (8 * (i & 3));
+  }
+  codes[b] = make_uint2(packed[0], packed[1]);
+  scales[b] = (uint8_t)sb;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restrict__ t, int64_t nblk,
                                                           const float* __restrict__ ts_in,
@@ -215,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restr
   const float s_t = ts_in ? *ts_in : __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
   const float d = __fmul_rn(s_t, 6.0f);
+  __shared__ __align__(16) uint32_t tab[DT == SP24_F32 ? 4 : 128 * 8];
+  if constexpr (DT != SP24_F32) build_thresholds<DT>(s_t, tab);  // published by the ring's first barrier
   stream::for_each_chunk<kChunk, kStages>(
       reinterpret_cast<const uint8_t*>(t), nblk * BB, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
         const int nb = bytes / BB;
@@ -223,9 +328,13 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restr
         for (int q = 0; q < kChunk / BB / kThreads; ++q) {
           const int j = threadIdx.x + q * kThreads;
           if (j >= nb) continue;
-          float v[16];
-          smem_block<DT>(chunk + j * BB, v);
-          encode_block(v, s_t, d, codes, scales, b0 + j);
+          if constexpr (DT == SP24_F32) {
+            float v[16];
+            smem_block<DT>(chunk + j * BB, v);
+            encode_block(v, s_t, d, codes, scales, b0 + j);
+          } else {
+            encode_block16<DT>(chunk + j * BB, tab, d, codes, scales, b0 + j);
+          }
         }
       });
 }
@@ -251,6 +360,11 @@ __global__ void __launch_bounds__(kThreads, 4) encode_pair_kernel(EncodeJob ja, 
     *jb.ts_out = s_b;
   }
   const float d_a = __fmul_rn(s_a, 6.0f), d_b = __fmul_rn(s_b, 6.0f);
+  __shared__ __align__(16) uint32_t tab[2][DT == SP24_F32 ? 4 : 128 * 8];
+  if constexpr (DT != SP24_F32) {  // published by the ring's first barrier
+    build_thresholds<DT>(s_a, tab[0]);
+    build_thresholds<DT>(s_b, tab[1]);
+  }
   stream::for_each_chunk2<kChunk, kStages>(
       reinterpret_cast<const uint8_t*>(ja.t), ja.nblk * BB, reinterpret_cast<const uint8_t*>(jb.t),
       jb.nblk * BB, ring, [&](const uint8_t* chunk, int seg, int64_t c, int bytes) {
@@ -263,9 +377,13 @@ __global__ void __launch_bounds__(kThreads, 4) encode_pair_kernel(EncodeJob ja, 
         for (int q = 0; q < kChunk / BB / kThreads; ++q) {
           const int j = threadIdx.x + q * kThreads;
           if (j >= nb) continue;
-          float v[16];
-          smem_block<DT>(chunk + j * BB, v);
-          encode_block(v, s_t, d, codes, scales, b0 + j);
+          if constexpr (DT == SP24_F32) {
+            float v[16];
+            smem_block<DT>(chunk + j * BB, v);
+            encode_block(v, s_t, d, codes, scales, b0 + j);
+          } else {
+            encode_block16<DT>(chunk + j * BB, tab[seg], d, codes, scales, b0 + j);
+          }
         }
       });
 }

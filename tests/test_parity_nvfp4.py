@@ -138,3 +138,14 @@ def test_quotients_at_rounding_boundaries(ts):
     (including exact ties): the codes must equal the oracle's, which divides entry by entry."""
     t = _boundary_blocks(int(ts * 1e6) % 9973 + 17, 4096, ts).reshape(256, 256)
     _compare(t, "f32", ts)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("ts", [0.25, 1.0 / 448, None])
+def test_16bit_entries_on_rounding_boundaries(dtype, ts):
+    """16-bit entries on a quarter grid with a power-of-two block divisor (tensor scale 1/4): many
+    quotients fall exactly on E2M1 rounding boundaries (exact ties) or next to them; the codes
+    must equal the oracle's per-entry division and tie-to-even."""
+    g = synth.rng(41)
+    t = synth.as_storage(np.round(synth.normal(g, (64, 256)) * 8) / 4, dtype)
+    _compare(t, dtype, ts)
