@@ -258,42 +258,27 @@ __device__ __forceinline__ uint32_t ru16(double x) {
   return __half_as_ushort(__float2half_ru(f));
 }
 
-// tab[8 c + j] = threshold j of block-scale code c (16 bits; j = 7 unused).
+// tab[8 c + j] = threshold j of block-scale code c, in both halves (j = 7 unused).
 template <int DT>
-__device__ void build_thresholds(float s_t, uint16_t* tab) {
+__device__ void build_thresholds(float s_t, uint32_t* tab) {
   for (int i = threadIdx.x; i < 128 * 8; i += blockDim.x) {
     const int c = i >> 3, j = i & 7;
-    uint32_t v = Pack16<DT>::QNAN & 0xffffu;
+    uint32_t v = Pack16<DT>::QNAN;
     if (j < 7 && c < 127) {
       const float sc = __fmul_rn(e4m3_value(c), s_t);
-      if (sc != 0.0f) v = ru16<DT>(kE2M1Bound[j] * (double)sc);
+      if (sc != 0.0f) {
+        const uint32_t h = ru16<DT>(kE2M1Bound[j] * (double)sc);
+        v = h | (h << 16);
+      }
     }
-    tab[i] = (uint16_t)v;
+    tab[i] = v;
   }
-}
-
-// E4M3_rne_satfinite(fl(bmax / d)) from yd = RN(1 / d) (0 when d is outside [2^-100, 2^100]).
-// RN(bmax * yd) is within 2.01 ulp of bmax / d; every E4M3 rounding boundary (including the
-// subnormal ones and zero's) has at most five significant bits, i.e. 19 zero low bits of its
-// fp32 significand, so a product within 4 ulps of such a value takes the IEEE division.
-__device__ __forceinline__ uint32_t block_scale_code(float bmax, float d, float yd) {
-  if (d == 0.0f) return 0u;
-  if (yd != 0.0f) {
-    const float q = __fmul_rn(bmax, yd);
-    const uint32_t u = __float_as_uint(q);
-    if (((u + 4u) & 0x7ffffu) > 8u || u == 0u) return e4m3_rne_satfinite(q);
-  }
-  return e4m3_rne_satfinite(__fdiv_rn(bmax, d));
-}
-
-__device__ __forceinline__ float recip_for_scale(float d) {
-  return d >= 0x1p-100f && d <= 0x1p100f ? __frcp_rn(d) : 0.0f;
 }
 
 // Encodes one block of 16 16-bit entries (32 bytes at p) with the thresholds of its scale code.
 template <int DT>
-__device__ __forceinline__ void encode_block16(const uint8_t* p, const uint16_t* tab, float d, float yd,
-                                               uint2* codes, uint8_t* scales, int64_t b) {
+__device__ __forceinline__ void encode_block16(const uint8_t* p, const uint32_t* tab, float d, uint2* codes,
+                                               uint8_t* scales, int64_t b) {
   const uint4 u0 = reinterpret_cast<const uint4*>(p)[0], u1 = reinterpret_cast<const uint4*>(p)[1];
   const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
   uint32_t a[8];
@@ -302,11 +287,10 @@ __device__ __forceinline__ void encode_block16(const uint8_t* p, const uint16_t*
   const uint32_t m = max2<DT>(max2<DT>(max2<DT>(a[0], a[1]), max2<DT>(a[2], a[3])),
                               max2<DT>(max2<DT>(a[4], a[5]), max2<DT>(a[6], a[7])));
   const float bmax = fmaxf(to_f32<DT>(m & 0xffffu), to_f32<DT>(m >> 16));
-  const uint32_t sb = block_scale_code(bmax, d, yd);
-  const uint4 t = *reinterpret_cast<const uint4*>(tab + 8 * sb);  // thresholds 0-6, pairs of halves
-  const uint32_t th[7] = {__byte_perm(t.x, 0, 0x1010), __byte_perm(t.x, 0, 0x3232), __byte_perm(t.y, 0, 0x1010),
-                          __byte_perm(t.y, 0, 0x3232), __byte_perm(t.z, 0, 0x1010), __byte_perm(t.z, 0, 0x3232),
-                          __byte_perm(t.w, 0, 0x1010)};
+  const uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
+  const uint4 t0 = reinterpret_cast<const uint4*>(tab + 8 * sb)[0];
+  const uint4 t1 = reinterpret_cast<const uint4*>(tab + 8 * sb)[1];
+  const uint32_t th[7] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z};
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -333,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restr
   // tensor scale: supplied, or amax / 2688 (2688 = 6 * 448)
   const float s_t = ts_in ? *ts_in : __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
-  const float d = __fmul_rn(s_t, 6.0f), yd = recip_for_scale(d);
-  __shared__ __align__(16) uint16_t tab[DT == SP24_F32 ? 8 : 128 * 8];
+  const float d = __fmul_rn(s_t, 6.0f);
+  __shared__ __align__(16) uint32_t tab[DT == SP24_F32 ? 4 : 128 * 8];
   if constexpr (DT != SP24_F32) build_thresholds<DT>(s_t, tab);  // published by the ring's first barrier
   stream::for_each_chunk<kChunk, kStages>(
       reinterpret_cast<const uint8_t*>(t), nblk * BB, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
@@ -349,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const void* __restr
             smem_block<DT>(chunk + j * BB, v);
             encode_block(v, s_t, d, codes, scales, b0 + j);
           } else {
-            encode_block16<DT>(chunk + j * BB, tab, d, yd, codes, scales, b0 + j);
+            encode_block16<DT>(chunk + j * BB, tab, d, codes, scales, b0 + j);
           }
         }
       });
@@ -376,8 +360,7 @@ __global__ void __launch_bounds__(kThreads, 4) encode_pair_kernel(EncodeJob ja, 
     *jb.ts_out = s_b;
   }
   const float d_a = __fmul_rn(s_a, 6.0f), d_b = __fmul_rn(s_b, 6.0f);
-  const float yd_a = recip_for_scale(d_a), yd_b = recip_for_scale(d_b);
-  __shared__ __align__(16) uint16_t tab[2][DT == SP24_F32 ? 8 : 128 * 8];
+  __shared__ __align__(16) uint32_t tab[2][DT == SP24_F32 ? 4 : 128 * 8];
   if constexpr (DT != SP24_F32) {  // published by the ring's first barrier
     build_thresholds<DT>(s_a, tab[0]);
     build_thresholds<DT>(s_b, tab[1]);
@@ -399,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 4) encode_pair_kernel(EncodeJob ja, 
             smem_block<DT>(chunk + j * BB, v);
             encode_block(v, s_t, d, codes, scales, b0 + j);
           } else {
-            encode_block16<DT>(chunk + j * BB, tab[seg], d, seg ? yd_b : yd_a, codes, scales, b0 + j);
+            encode_block16<DT>(chunk + j * BB, tab[seg], d, codes, scales, b0 + j);
           }
         }
       });
