@@ -82,6 +82,7 @@ struct Smem2 {
   static constexpr int OFF_S = OFF_V + kRows * C::VP;
   static constexpr int OFF_M = OFF_S + kRows * C::SP;
   static constexpr int TOTAL = OFF_M + kRows * C::MP;
+  static constexpr int BYTES = TOTAL + (TOTAL - OFF_V);  // x + two weight buffers
 };
 
 template <typename T>
@@ -183,13 +184,6 @@ __device__ __forceinline__ void mma_sp_k32(float (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(e));
 }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 
 // x[n, k] as 16-bit bits of T (0 outside the matrix); NVFP4 x decoded to E2M1 * E4M3.  `n` is
 // the x row already mapped (grouped mode: the routed token), `live` says whether the tile row
@@ -225,7 +219,6 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
   using C = F2<WF>;
   using L = Smem2<WF, NT>;
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
   __shared__ int32_t rows_of[GROUPED ? 64 : 1];  // grouped: flat (token, slot) of each tile row
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -241,44 +234,64 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
     if (p.meta) p.meta += (int64_t)e * p.expert_rows * p.meta_row_bytes;
     if (threadIdx.x < 64) rows_of[threadIdx.x] = threadIdx.x < cnt ? p.perm[first + threadIdx.x] : 0;
   }
-  const int64_t row0 = (int64_t)blockIdx.x * kRows;
   const int64_t k0 = (int64_t)blockIdx.y * C::KC;
   const int64_t kv = p.K - k0 < C::KC ? p.K - k0 : C::KC;  // valid logical K in this slice
-  const int rows_v = (int)(p.N - row0 < kRows ? p.N - row0 : kRows);
+  const int nrb = (int)((p.N + kRows - 1) / kRows);       // 64-row weight blocks
 
-  // ---- 1. bulk copies of the weight slice (thread r < rows_v copies row r)
+  // ---- 1. weight slices: row block rb into buffer `buf` with 16-byte cp.async, all threads;
+  // each row's pieces are consecutive, so a warp's copies cover whole row segments.
   const uint32_t vbytes = (uint32_t)(WF == W_D16 ? kv * 2 : WF == W_DQ4 ? kv / 2 : WF == W_S16 ? kv : kv / 4);
   const uint32_t sbytes = (uint32_t)(WF == W_DQ4 ? kv / 16 : WF == W_SQ4 ? kv / 32 : 0);
   const uint32_t mbytes = (uint32_t)(sparse_fmt<WF>() ? kv / 8 : 0);
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    tc::fence_mbar_init();
-  }
-  __syncthreads();  // also publishes rows_of
-  if (threadIdx.x == 0) mbar_arrive_expect_tx(&bar, (uint32_t)rows_v * (vbytes + sbytes + mbytes));
-  __syncthreads();
-  if (threadIdx.x < rows_v) {
-    const int64_t r = row0 + threadIdx.x;
-    bulk_g2s(sm + L::OFF_V + threadIdx.x * C::VP, p.w + r * p.w_row_bytes + (WF == W_D16 ? k0 * 2 : WF == W_DQ4 ? k0 / 2 : WF == W_S16 ? k0 : k0 / 4), vbytes, &bar);
-    if (sbytes)
-      bulk_g2s(sm + L::OFF_S + threadIdx.x * C::SP, p.w_scales + r * p.scale_row_bytes + (WF == W_DQ4 ? k0 / 16 : k0 / 32), sbytes, &bar);
-    if (mbytes) bulk_g2s(sm + L::OFF_M + threadIdx.x * C::MP, p.meta + r * p.meta_row_bytes + k0 / 8, mbytes, &bar);
-  }
-  // Fill what no copy writes: the tail of each row when the slice is short, and whole rows
-  // past N.  Values become +0 (uninitialised bits could be NaN, and NaN * 0 is NaN) and
-  // nibbles the legal pair (0, 1).  The regions are disjoint from the copies' destinations.
-  if (kv < C::KC || rows_v < kRows) {
-    for (int i = threadIdx.x; i < kRows * (C::VP / 4); i += blockDim.x) {
-      const int r = i / (C::VP / 4), off = (i % (C::VP / 4)) * 4;
-      if (r >= rows_v || off >= (int)vbytes) *reinterpret_cast<uint32_t*>(sm + L::OFF_V + r * C::VP + off) = 0u;
+  const int64_t voff = WF == W_D16 ? k0 * 2 : WF == W_DQ4 ? k0 / 2 : WF == W_S16 ? k0 : k0 / 4;
+  const int64_t soff = WF == W_DQ4 ? k0 / 16 : k0 / 32, moff = k0 / 8;
+  constexpr int WREG = L::TOTAL - L::OFF_V;  // one buffer: values, scales, nibbles
+  auto load_block = [&](int rb, int buf) {
+    uint8_t* bv = sm + L::OFF_V + buf * WREG;
+    uint8_t* bs = bv + (L::OFF_S - L::OFF_V);
+    uint8_t* bm = bv + (L::OFF_M - L::OFF_V);
+    const int64_t row0 = (int64_t)rb * kRows;
+    const int rows_v = (int)(p.N - row0 < kRows ? p.N - row0 : kRows);
+    const int vp = (int)(vbytes / 16), sp = (int)(sbytes / 16), mp = (int)(mbytes / 16);
+    for (int i = threadIdx.x; i < rows_v * vp; i += blockDim.x) {
+      const int r = i / vp, j = i - r * vp;
+      tc::cp_async16(bv + r * C::VP + 16 * j, p.w + (row0 + r) * p.w_row_bytes + voff + 16 * j);
     }
-    if constexpr (C::SP > 0)
-      for (int i = threadIdx.x; i < kRows * C::SP; i += blockDim.x)
-        if (i / C::SP >= rows_v || i % C::SP >= (int)sbytes) sm[L::OFF_S + i] = 0;
-    if constexpr (C::MP > 0)
-      for (int i = threadIdx.x; i < kRows * C::MP; i += blockDim.x)
-        if (i / C::MP >= rows_v || i % C::MP >= (int)mbytes) sm[L::OFF_M + i] = 0x44;
-  }
+    if constexpr (C::SP > 0) {
+      for (int i = threadIdx.x; i < rows_v * sp; i += blockDim.x) {
+        const int r = i / sp, j = i - r * sp;
+        tc::cp_async16(bs + r * C::SP + 16 * j, p.w_scales + (row0 + r) * p.scale_row_bytes + soff + 16 * j);
+      }
+    }
+    if constexpr (C::MP > 0) {
+      for (int i = threadIdx.x; i < rows_v * mp; i += blockDim.x) {
+        const int r = i / mp, j = i - r * mp;
+        tc::cp_async16(bm + r * C::MP + 16 * j, p.meta + (row0 + r) * p.meta_row_bytes + moff + 16 * j);
+      }
+    }
+    // Fill what no copy writes: the tail of each row when the slice is short, and whole rows
+    // past N.  Values become +0 (uninitialised bits could be NaN, and NaN * 0 is NaN) and
+    // nibbles the legal pair (0, 1).  The regions are disjoint from the copies' destinations.
+    if (kv < C::KC || rows_v < kRows) {
+      for (int i = threadIdx.x; i < kRows * (C::VP / 4); i += blockDim.x) {
+        const int r = i / (C::VP / 4), off = (i % (C::VP / 4)) * 4;
+        if (r >= rows_v || off >= (int)vbytes) *reinterpret_cast<uint32_t*>(bv + r * C::VP + off) = 0u;
+      }
+      if constexpr (C::SP > 0) {
+        for (int i = threadIdx.x; i < kRows * C::SP; i += blockDim.x) {
+          if (i / C::SP >= rows_v || i % C::SP >= (int)sbytes) bs[i] = 0;
+        }
+      }
+      if constexpr (C::MP > 0) {
+        for (int i = threadIdx.x; i < kRows * C::MP; i += blockDim.x) {
+          if (i / C::MP >= rows_v || i % C::MP >= (int)mbytes) bm[i] = 0x44;
+        }
+      }
+    }
+  };
+  __syncthreads();  // publishes rows_of
+  load_block(blockIdx.x, 0);
+  tc::cp_async_commit();
 
   // ---- 2. stage x in fragment order.  Each thread issues XB independent loads before it stores
   // any, so the staging costs a few L2 round trips rather than one per item.
@@ -360,20 +373,25 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
       }
     }
   }
-  __syncthreads();
-  const bool ok = mbar_wait(&bar, 0);
-  if (!ok) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-
-  float acc[NT][4];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
+  // ---- 3. row blocks blockIdx.x, blockIdx.x + gridDim.x, ...: the next block's weights stream
+  // in while this one is multiplied; the staged x serves them all
   const int rg = warp * 16 + g;  // local rows rg, rg + 8
-  const uint8_t* vrow0 = sm + L::OFF_V + rg * C::VP;
-  const uint8_t* vrow1 = vrow0 + 8 * C::VP;
   const int nch = (int)((kv + C::CHUNK - 1) / C::CHUNK);
-
-  if (ok) {
+  const int ntl = (p.M + 7) / 8;  // live token tiles
+  for (int it = 0, rb = blockIdx.x; rb < nrb; ++it, rb += gridDim.x) {
+    if (rb + (int)gridDim.x < nrb) load_block(rb + gridDim.x, (it + 1) & 1);
+    tc::cp_async_commit();
+    tc::cp_async_wait<1>();  // this block's copies (and x's stores, after the barrier)
+    __syncthreads();
+    const int64_t row0 = (int64_t)rb * kRows;
+    uint8_t* const bv = sm + L::OFF_V + (it & 1) * WREG;
+    const uint8_t* vrow0 = bv + rg * C::VP;
+    const uint8_t* vrow1 = vrow0 + 8 * C::VP;
+    const uint8_t* srow = bv + (L::OFF_S - L::OFF_V);
+    float acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  {
     if constexpr (!sparse_fmt<WF>()) {
       const uint2* xs = reinterpret_cast<const uint2*>(sm);
 #pragma unroll 2
@@ -382,8 +400,8 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
         const uint4 r1 = *reinterpret_cast<const uint4*>(vrow1 + ch * 64 + 16 * c);
         uint32_t sc[2][2];
         if (WF == W_DQ4) {
-          const uint32_t s0 = *reinterpret_cast<const uint16_t*>(sm + L::OFF_S + rg * C::SP + ch * 8 + 2 * c);
-          const uint32_t s1 = *reinterpret_cast<const uint16_t*>(sm + L::OFF_S + (rg + 8) * C::SP + ch * 8 + 2 * c);
+          const uint32_t s0 = *reinterpret_cast<const uint16_t*>(srow + rg * C::SP + ch * 8 + 2 * c);
+          const uint32_t s1 = *reinterpret_cast<const uint16_t*>(srow + (rg + 8) * C::SP + ch * 8 + 2 * c);
           scale_pair<T>(s0, sc[0][0], sc[0][1]);
           scale_pair<T>(s1, sc[1][0], sc[1][1]);
         }
@@ -404,12 +422,13 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
             a3 = hmul2u<T>(fp4_pair_i4<T>(w1[q], i0 + 1), sc[1][hb]);
           }
 #pragma unroll
-          for (int t = 0; t < NT; ++t) mma_k16<T>(acc[t], a0, a1, a2, a3, xs[((ch * C::STEPS + s) * NT + t) * 32 + lane]);
+          for (int t = 0; t < NT; ++t)
+            if (t < ntl) mma_k16<T>(acc[t], a0, a1, a2, a3, xs[((ch * C::STEPS + s) * NT + t) * 32 + lane]);
         }
       }
     } else {
       const uint4* xs = reinterpret_cast<const uint4*>(sm);
-      const uint8_t* mrow0 = sm + L::OFF_M + rg * C::MP;
+      const uint8_t* mrow0 = bv + (L::OFF_M - L::OFF_V) + rg * C::MP;
       const uint8_t* mrow1 = mrow0 + 8 * C::MP;
 #pragma unroll 4
       for (int win = 0; win < nch; ++win) {
@@ -428,8 +447,8 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
           const uint2 v0 = *reinterpret_cast<const uint2*>(vrow0 + 8 * win);
           const uint2 v1 = *reinterpret_cast<const uint2*>(vrow1 + 8 * win);
           uint32_t s0, s1, unused;
-          scale_pair<T>(sm[L::OFF_S + rg * C::SP + win], s0, unused);
-          scale_pair<T>(sm[L::OFF_S + (rg + 8) * C::SP + win], s1, unused);
+          scale_pair<T>(srow[rg * C::SP + win], s0, unused);
+          scale_pair<T>(srow[(rg + 8) * C::SP + win], s1, unused);
           const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));  // bytes c, c+4 -> [0], [1]
           const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
           a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
@@ -438,7 +457,8 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
           a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
         }
 #pragma unroll
-        for (int t = 0; t < NT; ++t) mma_sp_k32<T>(acc[t], a0, a1, a2, a3, xs[(win * NT + t) * 32 + lane], e);
+        for (int t = 0; t < NT; ++t)
+          if (t < ntl) mma_sp_k32<T>(acc[t], a0, a1, a2, a3, xs[(win * NT + t) * 32 + lane], e);
       }
     }
   }
@@ -462,16 +482,21 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
       }
     }
   }
+    __syncthreads();  // every warp is done with this buffer before it is refilled
+  }
+  tc::cp_async_wait<0>();
 }
 
 template <int WF, typename T, bool GROUPED = false>
 int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
   using C = F2<WF>;
-  dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)((p.K + C::KC - 1) / C::KC), tiles);
+  // grouped: one CTA walks all of an expert's row blocks, so its token tile's x is staged once
+  const unsigned nrb = (unsigned)((p.N + kRows - 1) / kRows);
+  dim3 grid(GROUPED ? 1u : nrb, (unsigned)((p.K + C::KC - 1) / C::KC), tiles);
 #define SP24_L2(NTV)                                                                                        \
   {                                                                                                         \
     auto kern = skinny2_kernel<WF, T, NTV, GROUPED>;                                                        \
-    constexpr int smem = Smem2<WF, NTV>::TOTAL;                                                             \
+    constexpr int smem = Smem2<WF, NTV>::BYTES;                                                             \
     if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
       return SP24_ERR_CUDA;                                                                                 \
     kern<<<grid, kWarps * 32, smem, s>>>(p);                                                                \
