@@ -82,7 +82,9 @@ struct Smem2 {
   static constexpr int OFF_S = OFF_V + kRows * C::VP;
   static constexpr int OFF_M = OFF_S + kRows * C::SP;
   static constexpr int TOTAL = OFF_M + kRows * C::MP;
-  static constexpr int BYTES = TOTAL + (TOTAL - OFF_V);  // x + two weight buffers
+  static constexpr int WREG = TOTAL - OFF_V;   // one weight buffer
+  // x + one weight buffer (one row block per CTA) or two (grouped: row blocks double-buffered)
+  static constexpr int bytes(bool two) { return TOTAL + (two ? WREG : 0); }
 };
 
 template <typename T>
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
   const uint32_t mbytes = (uint32_t)(sparse_fmt<WF>() ? kv / 8 : 0);
   const int64_t voff = WF == W_D16 ? k0 * 2 : WF == W_DQ4 ? k0 / 2 : WF == W_S16 ? k0 : k0 / 4;
   const int64_t soff = WF == W_DQ4 ? k0 / 16 : k0 / 32, moff = k0 / 8;
-  constexpr int WREG = L::TOTAL - L::OFF_V;  // one buffer: values, scales, nibbles
+  constexpr int WREG = L::WREG;  // one buffer: values, scales, nibbles
   auto load_block = [&](int rb, int buf) {
     uint8_t* bv = sm + L::OFF_V + buf * WREG;
     uint8_t* bs = bv + (L::OFF_S - L::OFF_V);
@@ -379,12 +381,12 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
   const int nch = (int)((kv + C::CHUNK - 1) / C::CHUNK);
   const int ntl = (p.M + 7) / 8;  // live token tiles
   for (int it = 0, rb = blockIdx.x; rb < nrb; ++it, rb += gridDim.x) {
-    if (rb + (int)gridDim.x < nrb) load_block(rb + gridDim.x, (it + 1) & 1);
+    if (GROUPED && rb + (int)gridDim.x < nrb) load_block(rb + gridDim.x, (it + 1) & 1);
     tc::cp_async_commit();
     tc::cp_async_wait<1>();  // this block's copies (and x's stores, after the barrier)
     __syncthreads();
     const int64_t row0 = (int64_t)rb * kRows;
-    uint8_t* const bv = sm + L::OFF_V + (it & 1) * WREG;
+    uint8_t* const bv = sm + L::OFF_V + (GROUPED ? (it & 1) * WREG : 0);
     const uint8_t* vrow0 = bv + rg * C::VP;
     const uint8_t* vrow1 = vrow0 + 8 * C::VP;
     const uint8_t* srow = bv + (L::OFF_S - L::OFF_V);
@@ -467,18 +469,48 @@ __global__ void __launch_bounds__(kWarps * 32) skinny2_kernel(SkinnyParams p) {
   float scale = 1.0f;
   if (WF == W_DQ4 || WF == W_SQ4) scale = 256.0f * *p.w_ts;
   if (p.x_fmt == X_Q4) scale *= *p.x_ts;
+  if (p.accumulate && p.N % 4 == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0) {
+    // partial sums over a K slice: transpose the tile through the (now idle) weight buffer so
+    // that each thread adds four consecutive outputs of one token with one vector atomic
+    constexpr int OP = kRows + 4;  // padded row of the transposed tile (floats)
+    float* ot = reinterpret_cast<float*>(bv);
+    __syncthreads();  // every warp is done reading the weight buffer
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int64_t n = 8 * t + 2 * c + (q & 1);
-      const int64_t r = row0 + rg + ((q & 2) ? 8 : 0);
-      if (n < p.M && r < p.N) {
+    for (int t = 0; t < NT; ++t) {
+      if (t < ntl) {
+        const int n = 8 * t + 2 * c;
+        ot[n * OP + rg] = acc[t][0];
+        ot[(n + 1) * OP + rg] = acc[t][1];
+        ot[n * OP + rg + 8] = acc[t][2];
+        ot[(n + 1) * OP + rg + 8] = acc[t][3];
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.M * (kRows / 4); i += blockDim.x) {
+      const int n = i / (kRows / 4), r = 4 * (i % (kRows / 4));
+      if (row0 + r < p.N) {
         const int64_t orow = GROUPED ? (int64_t)rows_of[n] : n;
-        float* dst = p.y + orow * p.N + r;
-        const float v = acc[t][q] * scale;
-        if (p.accumulate) atomicAdd(dst, v);
-        else *dst = v;
+        const float4 v = *reinterpret_cast<const float4*>(ot + n * OP + r);
+        float* dst = p.y + orow * p.N + row0 + r;
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x * scale),
+                     "f"(v.y * scale), "f"(v.z * scale), "f"(v.w * scale)
+                     : "memory");
+      }
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t n = 8 * t + 2 * c + (q & 1);
+        const int64_t r = row0 + rg + ((q & 2) ? 8 : 0);
+        if (n < p.M && r < p.N) {
+          const int64_t orow = GROUPED ? (int64_t)rows_of[n] : n;
+          float* dst = p.y + orow * p.N + r;
+          const float v = acc[t][q] * scale;
+          if (p.accumulate) atomicAdd(dst, v);
+          else *dst = v;
+        }
       }
     }
   }
@@ -496,7 +528,7 @@ int launch2(const SkinnyParams& p, int nt, cudaStream_t s, unsigned tiles = 1) {
 #define SP24_L2(NTV)                                                                                        \
   {                                                                                                         \
     auto kern = skinny2_kernel<WF, T, NTV, GROUPED>;                                                        \
-    constexpr int smem = Smem2<WF, NTV>::BYTES;                                                             \
+    constexpr int smem = Smem2<WF, NTV>::bytes(GROUPED);                                                    \
     if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
       return SP24_ERR_CUDA;                                                                                 \
     kern<<<grid, kWarps * 32, smem, s>>>(p);                                                                \
