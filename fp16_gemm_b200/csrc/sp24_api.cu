@@ -58,7 +58,9 @@ int run_skinny(int wf, int t16, SkinnyParams p, cudaStream_t s) {
     }
     // the decode kernel declines (SP24_ERR_UNSUPPORTED, nothing launched) when the driver
     // refuses its x tensor map
-    int st = decode_supported(wf, q) ? decode_gemv(wf, t16, q, s) : SP24_ERR_UNSUPPORTED;
+    int st = decode_tile_supported(wf, q) ? decode_tile(wf, t16, q, s)
+             : decode_supported(wf, q)    ? decode_gemv(wf, t16, q, s)
+                                          : SP24_ERR_UNSUPPORTED;
     if (st == SP24_ERR_UNSUPPORTED)
       st = skinny2_supported(wf, q) ? skinny2_gemm(wf, t16, q, s) : skinny_gemm(wf, t16, q, s);
     if (st) return st;

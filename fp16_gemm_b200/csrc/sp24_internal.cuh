@@ -105,6 +105,10 @@ int skinny_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 bool skinny2_supported(int wf, const SkinnyParams& p);
 int skinny2_gemm(int wf, int t16, SkinnyParams p, cudaStream_t s);
 // Persistent decode GEMV for NVFP4 weights (dense / 2:4) at M <= 8 (TMA-fed, one CTA per SM).
+// Whole-tile decode GEMV (M <= 8, NVFP4 weights, at least one 16-row tile per SM): writes y
+// without atomics, so y needs no zeroing.
+bool decode_tile_supported(int wf, const SkinnyParams& p);
+int decode_tile(int wf, int t16, const SkinnyParams& p, cudaStream_t s);
 bool decode_supported(int wf, const SkinnyParams& p);
 int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s);
 // 2-D TMA maps (defined with the tensor-core GEMMs): 128-byte swizzled, and unswizzled bytes.

@@ -26,6 +26,7 @@
 // one 32-bit word of each row's nibble stream.
 #include "sp24_internal.cuh"
 #include "sp24_tc.cuh"
+#include "sp24_stream.cuh"
 
 namespace sp24 {
 namespace {
@@ -826,6 +827,207 @@ int launch_decode(const SkinnyParams& p, cudaStream_t s) {
   return launch_status();
 }
 
+// ------------------------------------------------------------------ decode GEMV, whole tiles per CTA
+//
+// When there are at least as many 16-row tiles as SMs, each CTA owns a contiguous range of whole
+// tiles.  A tile's codes (and block scales, and 2:4 nibbles) over the full K are one contiguous
+// block of memory, so a producer thread fetches each with a single bulk copy into a ring of
+// tile buffers (bulk copies move data efficiently only in large requests), and x arrives as 8
+// bulk-copied rows padded by 16 bytes (so B-fragment reads of different tokens fall in
+// different banks).  16 consumer warps split each tile's K chunks round-robin, add their partial
+// sums into the tile's shared buffer, and release the buffer; at the end the CTA writes its
+// tiles' outputs with plain stores: every output has exactly one writer, so y needs no zeroing
+// and no atomics.  Rows sit unswizzled at a pitch that is a multiple of 128 bytes, so an A read
+// meets a 2-way bank conflict per 8-lane phase.
+constexpr int kTileWarps = 16;
+constexpr int kTileThreads = (kTileWarps + 1) * 32;  // + producer warp
+constexpr int kTileMaxLocal = 32;
+
+template <int WF>
+struct TileGeom {
+  int64_t cb, sb, mb;  // bytes per row: codes, block scales, nibbles
+  __host__ __device__ explicit TileGeom(int64_t K)
+      : cb(WF == W_DQ4 ? K / 2 : K / 4), sb(WF == W_DQ4 ? K / 16 : K / 32), mb(WF == W_SQ4 ? K / 8 : 0) {}
+  __host__ __device__ int64_t bytes() const { return 16 * (cb + sb + mb); }
+};
+
+// Dynamic shared memory: x (8 rows of 2K + 16 bytes), nbuf tile buffers, per-tile sums.
+template <int WF>
+size_t tile_smem(int64_t K, int nbuf, int64_t local_tiles) {
+  return 8 * (size_t)(2 * K + 16) + (size_t)nbuf * TileGeom<WF>(K).bytes() + (size_t)local_tiles * 512;
+}
+
+template <int WF, typename T, int NBUF>
+__global__ void __launch_bounds__(kTileThreads, 1) decode_tile_kernel(const SkinnyParams p) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ uint64_t full_bar[NBUF], empty_bar[NBUF], x_bar;
+  __shared__ int issued, abort_flag;
+  const TileGeom<WF> tg(p.K);
+  const int64_t xp = 2 * p.K + 16;                       // padded x row
+  uint8_t* xs = dsm;
+  uint8_t* bufs = dsm + 8 * xp;
+  float* tbuf = reinterpret_cast<float*>(bufs + NBUF * tg.bytes());  // [local tile][16 rows][8 tokens]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NT16 = (int)(p.N / 16);
+  const int t0 = (int)((int64_t)NT16 * blockIdx.x / gridDim.x), t1 = (int)((int64_t)NT16 * (blockIdx.x + 1) / gridDim.x);
+  const int ntiles = t1 - t0;                             // >= 1 (host: T >= grid), <= kTileMaxLocal
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBUF; ++i) {
+      tc::mbar_init(&full_bar[i], 1);
+      tc::mbar_init(&empty_bar[i], kTileWarps);
+    }
+    tc::mbar_init(&x_bar, 1);
+    issued = 0;
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < ntiles * 128; i += blockDim.x) tbuf[i] = 0.f;
+  // token rows past M: zeros
+  for (int i = threadIdx.x; i < (8 - p.M) * (int)(xp / 16); i += blockDim.x) {
+    const int r = p.M + i / (int)(xp / 16), j = i % (int)(xp / 16);
+    *reinterpret_cast<uint4*>(xs + r * xp + 16 * j) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+
+  if (warp == kTileWarps) {
+    // ---- producer: x rows, then each tile's codes / scales / nibbles, one bulk copy apiece
+    if (lane == 0) {
+      const uint8_t* xg = reinterpret_cast<const uint8_t*>(p.x);
+      tc::mbar_arrive_expect_tx(&x_bar, (uint32_t)(p.M * 2 * p.K));
+      for (int g = 0; g < p.M; ++g) stream::bulk_g2s(xs + g * xp, xg + (int64_t)g * 2 * p.K, (uint32_t)(2 * p.K), &x_bar);
+      int i = 0;
+      for (; i < ntiles; ++i) {
+        const int sl = i % NBUF;
+        if (!mbar_wait(&empty_bar[sl], ((i / NBUF) & 1) ^ 1)) {
+          set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+          abort_flag = 1;
+          break;
+        }
+        uint8_t* d = bufs + sl * tg.bytes();
+        const int64_t row = (int64_t)(t0 + i) * 16;
+        tc::mbar_arrive_expect_tx(&full_bar[sl], (uint32_t)tg.bytes());
+        stream::bulk_g2s(d, p.w + row * tg.cb, (uint32_t)(16 * tg.cb), &full_bar[sl]);
+        stream::bulk_g2s(d + 16 * tg.cb, p.w_scales + row * tg.sb, (uint32_t)(16 * tg.sb), &full_bar[sl]);
+        if (WF == W_SQ4) stream::bulk_g2s(d + 16 * (tg.cb + tg.sb), p.meta + row * tg.mb, (uint32_t)(16 * tg.mb), &full_bar[sl]);
+      }
+      issued = i;
+    }
+  } else {
+    // ---- consumers: chunks (128 k dense, 32-k windows 2:4) of each tile, round-robin over warps
+    const int g = lane >> 2, c = lane & 3;
+    const int r0 = prow(g), r1 = prow(g + 8);
+    const uint8_t* x0 = xs + g * xp;  // this lane's token row
+    const int nq = WF == W_DQ4 ? (int)(p.K / 128) : (int)(p.K / 32);
+    bool ok = mbar_wait(&x_bar, 0);
+    if (!ok) {
+      set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+      abort_flag = 1;
+    }
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const int sl = i % NBUF;
+      if (!mbar_wait(&full_bar[sl], (i / NBUF) & 1)) {
+        set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+        abort_flag = 1;
+        break;
+      }
+      const uint8_t* d = bufs + sl * tg.bytes();
+      const uint8_t* sc = d + 16 * tg.cb;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (WF == W_DQ4) {
+        auto chunk = [&](int q, float(&A)[4]) {
+          // lane piece: codes 32c .. 32c + 31 of chunk q (16 bytes of each row), two block scales
+          const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 64 * q + 16 * c);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 64 * q + 16 * c);
+          uint32_t sa[2], sb[2];
+          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 8 * q + 2 * c), sa[0], sa[1]);
+          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 8 * q + 2 * c), sb[0], sb[1]);
+          const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            // x[g][P .. P+8), P = 128q + 32c + 8qq: codes at nibbles (i, i+4) of word qq pair with
+            // x entries (i, i+4)
+            const uint4 xv = *reinterpret_cast<const uint4*>(x0 + 2 * (128 * q + 32 * c + 8 * qq));
+            const uint32_t s0 = sa[qq >> 1], s1 = sb[qq >> 1];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
+              const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
+              const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[qq], 2 * h), s0);
+              const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[qq], 2 * h + 1), s0);
+              const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[qq], 2 * h), s1);
+              const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[qq], 2 * h + 1), s1);
+              mma_k16<T>(A, a0, a1, a2, a3, bx);
+            }
+          }
+        };
+        for (int q = warp; q < nq; q += 2 * kTileWarps) {
+          chunk(q, acc);
+          if (q + kTileWarps < nq) chunk(q + kTileWarps, acc2);
+        }
+      } else {
+        const uint8_t* me = sc + 16 * tg.sb;
+        auto window = [&](int w, float(&A)[4]) {
+          const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * tg.mb + 4 * w);
+          const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * tg.mb + 4 * w);
+          const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
+          const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * tg.cb + 8 * w);
+          const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * tg.cb + 8 * w);
+          uint32_t s0, s1, unused;
+          scale_pair<T>(sc[r0 * tg.sb + w], s0, unused);
+          scale_pair<T>(sc[r1 * tg.sb + w], s1, unused);
+          const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
+          const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
+          const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+          const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+          const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+          const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+          // x[g][32w + 2c + 8i + {0, 1}], i = 0..3
+          const uint8_t* xr = x0 + 2 * (32 * w) + 4 * c;
+          const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 16),
+                                      *reinterpret_cast<const uint32_t*>(xr + 32), *reinterpret_cast<const uint32_t*>(xr + 48));
+          mma_sp_k32<T>(A, a0, a1, a2, a3, bx, e);
+        };
+        for (int w = warp; w < nq; w += 2 * kTileWarps) {
+          window(w, acc);
+          if (w + kTileWarps < nq) window(w + kTileWarps, acc2);
+        }
+      }
+      float* b = tbuf + i * 128;
+      atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
+      atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
+      atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
+      atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
+    }
+  }
+  __syncthreads();
+  // a gave-up wait may leave copies in flight: let them land before the CTA's memory goes away
+  if (abort_flag && threadIdx.x == kTileWarps * 32) {
+    tc::mbar_wait(&x_bar, 0);
+    for (int i = issued > NBUF ? issued - NBUF : 0; i < issued; ++i) tc::mbar_wait(&full_bar[i % NBUF], (i / NBUF) & 1);
+  }
+  // ---- the CTA's tiles into y, one writer per output
+  const float scale = 256.0f * *p.w_ts;
+  for (int e = threadIdx.x; e < ntiles * 128; e += blockDim.x) {
+    const int lt = e >> 7, row = (e >> 3) & 15, tok = e & 7;
+    if (tok < p.M) p.y[(int64_t)tok * p.N + (int64_t)(t0 + lt) * 16 + row] = tbuf[e] * scale;
+  }
+}
+
+template <int WF, typename T>
+int launch_tile(const SkinnyParams& p, cudaStream_t s) {
+  const int grid = sm_count();
+  const int64_t T16 = p.N / 16, local = (T16 + grid - 1) / grid;
+  const bool three = tile_smem<WF>(p.K, 3, local) <= 227 * 1024 - 256;
+  const size_t smem = tile_smem<WF>(p.K, three ? 3 : 2, local);
+  auto kern = three ? decode_tile_kernel<WF, T, 3> : decode_tile_kernel<WF, T, 2>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  kern<<<grid, kTileThreads, smem, s>>>(p);
+  return launch_status();
+}
+
 }  // namespace
 
 // Grouped launch: grid.z = max_tiles token tiles (<= 64 tokens each, NT = 8); y must be zeroed
@@ -858,6 +1060,28 @@ bool decode_supported(int wf, const SkinnyParams& p) {
   if (wf == W_DQ4) return p.K % U3<W_DQ4>::UK == 0 && decode_group<W_DQ4>(p, &xcols) > 0;
   if (wf == W_SQ4) return aligned(p.meta, 16) && p.K % U3<W_SQ4>::UK == 0 && decode_group<W_SQ4>(p, &xcols) > 0;
   return false;
+}
+
+// True when the whole-tile decode kernel takes the problem: 16-bit x of at most 8 tokens,
+// NVFP4 weights (dense: K % 128; 2:4: K % 32) with at least one 16-row tile per SM and at most
+// kTileMaxLocal tiles per CTA, 16-byte aligned operands, and x plus two tile buffers in shared
+// memory.
+bool decode_tile_supported(int wf, const SkinnyParams& p) {
+  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0) return false;
+  if (!aligned(p.x, 16) || !aligned(p.w, 16) || !aligned(p.w_scales, 16) || !aligned(p.y, 4)) return false;
+  const int64_t T16 = p.N / 16, grid = sm_count(), local = (T16 + grid - 1) / grid;
+  if (T16 < grid || local > kTileMaxLocal) return false;
+  if (wf == W_DQ4) return p.K % 128 == 0 && tile_smem<W_DQ4>(p.K, 2, local) <= 227 * 1024 - 256;
+  if (wf == W_SQ4)
+    return p.K % 32 == 0 && aligned(p.meta, 16) && tile_smem<W_SQ4>(p.K, 2, local) <= 227 * 1024 - 256;
+  return false;
+}
+
+int decode_tile(int wf, int t16, const SkinnyParams& p, cudaStream_t s) {
+  const bool bf = t16 == SP24_BF16;
+  if (wf == W_DQ4) return bf ? launch_tile<W_DQ4, __nv_bfloat16>(p, s) : launch_tile<W_DQ4, __half>(p, s);
+  if (wf == W_SQ4) return bf ? launch_tile<W_SQ4, __nv_bfloat16>(p, s) : launch_tile<W_SQ4, __half>(p, s);
+  return SP24_ERR_UNSUPPORTED;
 }
 
 int decode_gemv(int wf, int t16, const SkinnyParams& p, cudaStream_t s) {
