@@ -934,62 +934,72 @@ __global__ void __launch_bounds__(kTileThreads, 1) decode_tile_kernel(const Skin
       const uint8_t* sc = d + 16 * tg.cb;
       float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (WF == W_DQ4) {
-        auto chunk = [&](int q, float(&A)[4]) {
-          // lane piece: codes 32c .. 32c + 31 of chunk q (16 bytes of each row), two block scales
-          const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 64 * q + 16 * c);
-          const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 64 * q + 16 * c);
-          uint32_t sa[2], sb[2];
-          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 8 * q + 2 * c), sa[0], sa[1]);
-          scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 8 * q + 2 * c), sb[0], sb[1]);
-          const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
+        // chunks q and q + 16 of a warp are decoded step by step into two accumulator chains
+        for (int q = warp; q < nq; q += 2 * kTileWarps) {
+          const bool two = q + kTileWarps < nq;
+          uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qc = u && two ? q + kTileWarps : q;  // a missing second chunk repeats the first, unused
+            const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 64 * qc + 16 * c);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 64 * qc + 16 * c);
+            w0[u][0] = v0.x; w0[u][1] = v0.y; w0[u][2] = v0.z; w0[u][3] = v0.w;
+            w1[u][0] = v1.x; w1[u][1] = v1.y; w1[u][2] = v1.z; w1[u][3] = v1.w;
+            scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 8 * qc + 2 * c), sa[u][0], sa[u][1]);
+            scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 8 * qc + 2 * c), sb[u][0], sb[u][1]);
+          }
 #pragma unroll
           for (int qq = 0; qq < 4; ++qq) {
-            // x[g][P .. P+8), P = 128q + 32c + 8qq: codes at nibbles (i, i+4) of word qq pair with
-            // x entries (i, i+4)
-            const uint4 xv = *reinterpret_cast<const uint4*>(x0 + 2 * (128 * q + 32 * c + 8 * qq));
-            const uint32_t s0 = sa[qq >> 1], s1 = sb[qq >> 1];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
-              const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
-              const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[qq], 2 * h), s0);
-              const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[qq], 2 * h + 1), s0);
-              const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[qq], 2 * h), s1);
-              const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[qq], 2 * h + 1), s1);
-              mma_k16<T>(A, a0, a1, a2, a3, bx);
+            for (int u = 0; u < 2; ++u) {
+              if (u && !two) continue;
+              const int qc = u ? q + kTileWarps : q;
+              // x[g][P .. P+8), P = 128 qc + 32c + 8qq: codes at nibbles (i, i+4) of word qq pair
+              // with x entries (i, i+4)
+              const uint4 xv = *reinterpret_cast<const uint4*>(x0 + 2 * (128 * qc + 32 * c + 8 * qq));
+              const uint32_t s0 = sa[u][qq >> 1], s1 = sb[u][qq >> 1];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
+                const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
+                const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[u][qq], 2 * h), s0);
+                const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[u][qq], 2 * h + 1), s0);
+                const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[u][qq], 2 * h), s1);
+                const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[u][qq], 2 * h + 1), s1);
+                mma_k16<T>(u ? acc2 : acc, a0, a1, a2, a3, bx);
+              }
             }
           }
-        };
-        for (int q = warp; q < nq; q += 2 * kTileWarps) {
-          chunk(q, acc);
-          if (q + kTileWarps < nq) chunk(q + kTileWarps, acc2);
         }
       } else {
+        // window pairs (2v, 2v + 1): 16 bytes of codes and 8 of nibbles per row in one load each,
+        // the two windows into two accumulator chains
         const uint8_t* me = sc + 16 * tg.sb;
-        auto window = [&](int w, float(&A)[4]) {
-          const uint32_t m0 = *reinterpret_cast<const uint32_t*>(me + r0 * tg.mb + 4 * w);
-          const uint32_t m1 = *reinterpret_cast<const uint32_t*>(me + r1 * tg.mb + 4 * w);
-          const uint32_t e = __byte_perm(m0, m1, (c & 1) ? 0x7632 : 0x5410);
-          const uint2 v0 = *reinterpret_cast<const uint2*>(d + r0 * tg.cb + 8 * w);
-          const uint2 v1 = *reinterpret_cast<const uint2*>(d + r1 * tg.cb + 8 * w);
-          uint32_t s0, s1, unused;
-          scale_pair<T>(sc[r0 * tg.sb + w], s0, unused);
-          scale_pair<T>(sc[r1 * tg.sb + w], s1, unused);
-          const uint32_t b0 = __byte_perm(v0.x, v0.y, c | ((c + 4) << 4));
-          const uint32_t b1 = __byte_perm(v1.x, v1.y, c | ((c + 4) << 4));
-          const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
-          const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
-          const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
-          const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
-          // x[g][32w + 2c + 8i + {0, 1}], i = 0..3
-          const uint8_t* xr = x0 + 2 * (32 * w) + 4 * c;
-          const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 16),
-                                      *reinterpret_cast<const uint32_t*>(xr + 32), *reinterpret_cast<const uint32_t*>(xr + 48));
-          mma_sp_k32<T>(A, a0, a1, a2, a3, bx, e);
-        };
-        for (int w = warp; w < nq; w += 2 * kTileWarps) {
-          window(w, acc);
-          if (w + kTileWarps < nq) window(w + kTileWarps, acc2);
+        for (int v = warp; 2 * v < nq; v += kTileWarps) {
+          const uint4 c0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 16 * v);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 16 * v);
+          const uint2 m0 = *reinterpret_cast<const uint2*>(me + r0 * tg.mb + 8 * v);
+          const uint2 m1 = *reinterpret_cast<const uint2*>(me + r1 * tg.mb + 8 * v);
+          const uint32_t sc0 = *reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 2 * v);
+          const uint32_t sc1 = *reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 2 * v);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t e = __byte_perm(u ? m0.y : m0.x, u ? m1.y : m1.x, (c & 1) ? 0x7632 : 0x5410);
+            uint32_t s0, s1, unused;
+            scale_pair<T>((sc0 >> (8 * u)) & 0xffu, s0, unused);
+            scale_pair<T>((sc1 >> (8 * u)) & 0xffu, s1, unused);
+            const uint32_t b0 = __byte_perm(u ? c0.z : c0.x, u ? c0.w : c0.y, c | ((c + 4) << 4));
+            const uint32_t b1 = __byte_perm(u ? c1.z : c1.x, u ? c1.w : c1.y, c | ((c + 4) << 4));
+            const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
+            const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
+            const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
+            const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
+            // x[g][32w + 2c + 8i + {0, 1}], i = 0..3, w = 2v + u
+            const uint8_t* xr = x0 + 2 * (32 * (2 * v + u)) + 4 * c;
+            const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 16),
+                                        *reinterpret_cast<const uint32_t*>(xr + 32), *reinterpret_cast<const uint32_t*>(xr + 48));
+            mma_sp_k32<T>(u ? acc2 : acc, a0, a1, a2, a3, bx, e);
+          }
         }
       }
       float* b = tbuf + i * 128;
@@ -1063,7 +1073,7 @@ bool decode_supported(int wf, const SkinnyParams& p) {
 }
 
 // True when the whole-tile decode kernel takes the problem: 16-bit x of at most 8 tokens,
-// NVFP4 weights (dense: K % 128; 2:4: K % 32) with at least one 16-row tile per SM and at most
+// NVFP4 weights (dense: K % 128; 2:4: K % 64) with at least one 16-row tile per SM and at most
 // kTileMaxLocal tiles per CTA, 16-byte aligned operands, and x plus two tile buffers in shared
 // memory.
 bool decode_tile_supported(int wf, const SkinnyParams& p) {
@@ -1073,7 +1083,7 @@ bool decode_tile_supported(int wf, const SkinnyParams& p) {
   if (T16 < grid || local > kTileMaxLocal) return false;
   if (wf == W_DQ4) return p.K % 128 == 0 && tile_smem<W_DQ4>(p.K, 2, local) <= 227 * 1024 - 256;
   if (wf == W_SQ4)
-    return p.K % 32 == 0 && aligned(p.meta, 16) && tile_smem<W_SQ4>(p.K, 2, local) <= 227 * 1024 - 256;
+    return p.K % 64 == 0 && aligned(p.meta, 16) && tile_smem<W_SQ4>(p.K, 2, local) <= 227 * 1024 - 256;
   return false;
 }
 
