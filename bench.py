@@ -21,7 +21,7 @@ window; the timed region replays each window once, so the host pays one graph la
 window.  An event record node inside a graph costs a few microseconds, so the timed windows
 carry only one pair of events, around the dominant stage of their first step: that kernel's
 launch duration (for `roofline`) is measured inside the timed region.  The per-stage breakdown
-(`stages`) comes from separate windows with an event after every stage, run before timing.
+(`stages`) comes from graphs of back-to-back launches of each stage alone, run before timing.
 `value` is the whole step's algorithmic HBM traffic divided by the step time (GB/s); the GEMV
 comparison (dense vs 2:4 sparse: TFLOP/s, GB/s, speedup) is in `gemv`.
 
@@ -215,36 +215,29 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     cap = torch.cuda.Stream()
     U = max(u for u in range(1, 17) if args.steps % u == 0)
 
-    # Stage breakdown (before the timed region): windows of U steps with an event after every
-    # stage.  An event record node in a graph costs a few microseconds of its own, so these
-    # windows are not used for the step time; they give each stage's share and pick the
-    # dominant stage.
-    br_windows = []
-    for wi in range(2):
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(1 + U * len(STAGES))]
+    # Stage breakdown (before the timed region): each stage alone, U launches back to back over
+    # the rotating input sets in one CUDA graph with events only around the whole graph (an
+    # event record node costs a few microseconds, which would swamp the short kernels).  The
+    # stages run in step order first, so every stage sees the operands the step gives it.
+    stage_ms = []
+    for si in range(len(STAGES)):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            evs[0].record()
             for j in range(U):
-                for si, f in enumerate(stage_fns(sets[(wi * U + j) % len(sets)])):
-                    f()
-                    evs[1 + j * len(STAGES) + si].record()
-        br_windows.append((g, evs))
-    for g, _ in br_windows:
+                stage_fns(sets[j % len(sets)])[si]()
         g.replay()
-    torch.cuda.synchronize()
-    for g, _ in br_windows:  # second replay is the one read
-        g.replay()
-    torch.cuda.synchronize()
-    stage_ms = [0.0] * len(STAGES)
-    for _, evs in br_windows:
-        for j in range(U):
-            for si in range(len(STAGES)):
-                k = 1 + j * len(STAGES) + si
-                stage_ms[si] += evs[k - 1].elapsed_time(evs[k])
-    stage_ms = [v / (2 * U) for v in stage_ms]
+        torch.cuda.synchronize()
+        reps = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()  # the current stream, where replay() launches the graph
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            reps.append(a.elapsed_time(b) / U)
+        stage_ms.append(statistics.median(reps))
+        del g
     dom_i = max(range(len(STAGES)), key=lambda i: stage_ms[i])
-    del br_windows
 
     # Timed steps: windows of U consecutive steps, one CUDA graph per window, with no event
     # between stages except one pair around the dominant stage of the window's first step (that
@@ -381,8 +374,8 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
                                               "sparse24": round(fl / gs["bytes"], 1)},
         },
         "stages": stages,
-        "stages_note": ("per-stage times from event-per-stage windows run before the timed "
-                        "region (each event node adds a few us); the step time has no stage events"),
+        "stages_note": ("per-stage kernel times from graphs of back-to-back launches of each "
+                        "stage alone, run before the timed region; the step time has no stage events"),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 3),
                      "launch_us": round(dom_ms * 1e3, 3), "launches_timed": len(windows),
