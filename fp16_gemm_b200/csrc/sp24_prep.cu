@@ -302,6 +302,51 @@ __global__ void __launch_bounds__(kThreads, 4) prepare_vec(const uint4* __restri
   }
 }
 
+// Conv layout W[K, C, R, S], 16-bit entries: the four channels 4j .. 4j + 3 of output channel k
+// form a contiguous block of 4 RS entries holding the RS groups (k, j, rs); group rs takes
+// entries rs, RS + rs, 2 RS + rs and 3 RS + rs of the block, and groups are numbered
+// (k, j, rs) row-major, i.e. block after block.  Chunks of whole block pairs (ch bytes) stream
+// through the ring; thread t takes groups 2m, 2m + 1 of a chunk (m = t, t + blockDim.x, ...), so
+// every nibble byte has one writer.  PRUNE: kept values to [K, C/2, R, S] and nibbles, else the
+// pass map and fail count.
+template <bool PRUNE>
+__global__ void __launch_bounds__(kThreads, 4) conv24_vec16(const uint16_t* __restrict__ w, int64_t nbytes, int ch,
+                                                             int RS, uint8_t* __restrict__ pass,
+                                                             int32_t* __restrict__ n_fail, uint16_t* __restrict__ values,
+                                                             uint8_t* __restrict__ meta) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  int fails = 0;
+  stream::for_each_chunk_rt<kChunk, kStages>(
+      reinterpret_cast<const uint8_t*>(w), nbytes, ch, ring, [&](const uint8_t* chunk, int64_t c, int bytes) {
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(chunk);
+        const int64_t g0 = c * (ch / 8);  // groups before this chunk (8 bytes of entries per group)
+        const int ng = bytes / 8;         // even: whole block pairs
+        for (int m = threadIdx.x; 2 * m < ng; m += kThreads) {
+          uint32_t nib[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int gi = 2 * m + u, b = gi / RS, rs = gi - b * RS;
+            const uint16_t* blk = e + (int64_t)b * 4 * RS + rs;
+            const uint32_t lo = blk[0] | ((uint32_t)blk[RS] << 16), hi = blk[2 * RS] | ((uint32_t)blk[3 * RS] << 16);
+            const Keys4 k = sort_keys16(lo, hi);
+            if (PRUNE) {
+              const Group16 gr = kept16(k, lo, hi);
+              nib[u] = gr.nib;
+              const int64_t blk_g = g0 / RS + b;  // global block: chunks hold whole blocks
+              values[(2 * blk_g) * RS + rs] = (uint16_t)(gr.kept & 0xffffu);
+              values[(2 * blk_g + 1) * RS + rs] = (uint16_t)(gr.kept >> 16);
+            } else {
+              const int ok = k.k3 < 4u;
+              fails += 1 - ok;
+              pass[g0 + gi] = (uint8_t)ok;
+            }
+          }
+          if (PRUNE) meta[(g0 >> 1) + m] = (uint8_t)(nib[0] | (nib[1] << 4));
+        }
+      });
+  if (!PRUNE) count_fails(fails, n_fail);
+}
+
 // Inverse of prune24_vec for 16-bit data: two groups per thread.
 __global__ void __launch_bounds__(kThreads) decompress24_vec16(const uint2* __restrict__ values,
                                                                const uint8_t* __restrict__ meta,
@@ -335,6 +380,16 @@ struct Layout {
   int op;
   int64_t C, RS;  // conv: channels and R*S
 };
+
+// Chunk bytes for conv24_vec16: whole block pairs (16 RS bytes) up to the ring's stage size, or 0
+// when that path does not apply (an odd number of blocks, or R*S too large).
+int64_t conv_chunk(const Layout& L, int64_t G) {
+  const int64_t unit = 16 * L.RS;
+  const int64_t blocks = G / L.RS;
+  if (L.op != SP24_OP_CONV || unit > kChunk || blocks % 2) return 0;
+  return kChunk / unit * unit;
+}
+
 
 // Element index of member i of group g.
 __device__ __forceinline__ int64_t member(const Layout& L, int64_t g, int i) {
@@ -508,6 +563,14 @@ extern "C" int sp24_check_24(const void* w, int dtype, int op, const int64_t* sh
   if (G == 0) return launch_status(0);
   int nl = 0;
   int64_t g_done = 0;
+  if (op == SP24_OP_CONV && eb == 2 && aligned(w, 16) && conv_chunk(L, G) > 0) {
+    const int ch = (int)conv_chunk(L, G);
+    auto k = conv24_vec16<false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingBytes);
+    const int grid = full_wave_grid(k, kThreads, (G * 8 + ch - 1) / ch, kRingBytes);
+    k<<<grid, kThreads, kRingBytes, s>>>((const uint16_t*)w, G * 8, ch, (int)L.RS, pass, n_fail, nullptr, nullptr);
+    return launch_status(1);
+  }
   if (op == SP24_OP_MATMUL && aligned(w, 16) && aligned(pass, eb == 2 ? 2 : 1)) {
     int64_t nv = G * 4 * eb / 16;  // whole 16-byte vectors
     if (nv > 0) {
@@ -542,6 +605,14 @@ extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const in
   cudaStream_t s = as_stream(stream);
   int nl = 0;
   int64_t p_done = 0;  // meta bytes (group pairs) already written
+  if (op == SP24_OP_CONV && eb == 2 && aligned(w, 16) && aligned(values, 2) && conv_chunk(L, G) > 0) {
+    const int ch = (int)conv_chunk(L, G);
+    auto k = conv24_vec16<true>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingBytes);
+    const int grid = full_wave_grid(k, kThreads, (G * 8 + ch - 1) / ch, kRingBytes);
+    k<<<grid, kThreads, kRingBytes, s>>>((const uint16_t*)w, G * 8, ch, (int)L.RS, nullptr, nullptr, (uint16_t*)values, meta);
+    return launch_status(1);
+  }
   if (op == SP24_OP_MATMUL && aligned(w, 16) && aligned(values, 8)) {
     int64_t nv = G * 4 * eb / 16;
     if (eb == 4) nv &= ~int64_t(1);  // whole meta bytes only

@@ -83,6 +83,49 @@ __device__ __forceinline__ void for_each_chunk2(const uint8_t* __restrict__ a, i
   }
 }
 
+// As for_each_chunk below, with chunks of `ch` bytes (a multiple of 16, at most CHUNK) chosen at
+// run time; stages stay CHUNK bytes apart in `ring`.
+template <int CHUNK, int S, class Body>
+__device__ __forceinline__ void for_each_chunk_rt(const uint8_t* __restrict__ src, int64_t nbytes, int ch,
+                                                  uint8_t* ring, Body&& body) {
+  __shared__ uint64_t bars[S];
+  __shared__ int abort_flag;
+  const int64_t nchunks = (nbytes + ch - 1) / ch;
+  const int64_t mine = blockIdx.x < nchunks ? (nchunks - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) tc::mbar_init(&bars[s], 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  auto size_of = [&](int64_t c) { return (uint32_t)(nbytes - c * ch < ch ? nbytes - c * ch : ch); };
+  auto issue = [&](int64_t i) {
+    const int s = (int)(i % S);
+    const int64_t c = blockIdx.x + i * gridDim.x;
+    const uint32_t sz = size_of(c);
+    tc::mbar_arrive_expect_tx(&bars[s], sz);
+    bulk_g2s(ring + s * CHUNK, src + c * ch, sz, &bars[s]);
+  };
+  if (threadIdx.x == 0)
+    for (int64_t i = 0; i < (mine < S ? mine : S); ++i) issue(i);
+  int64_t i = 0;
+  for (; i < mine; ++i) {
+    const int s = (int)(i % S);
+    const bool ok = tc::mbar_wait(&bars[s], (uint32_t)((i / S) & 1));
+    if (!ok) abort_flag = 1;
+    const int64_t c = blockIdx.x + i * gridDim.x;
+    if (ok) body(ring + s * CHUNK, c, (int)size_of(c));
+    __syncthreads();
+    if (abort_flag) break;
+    if (threadIdx.x == 0 && i + S < mine) issue(i + S);
+  }
+  if (threadIdx.x == 0 && abort_flag) {
+    set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+    const int64_t last = i + S < mine ? i + S : mine;
+    for (int64_t j = i; j < last; ++j) tc::mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1));
+  }
+}
+
 // Runs body(stage_ptr, chunk_index, chunk_bytes) over this CTA's chunks of `src` (nbytes, a
 // multiple of 16, src 16-byte aligned): chunks c = blockIdx.x, blockIdx.x + gridDim.x, ...
 template <int CHUNK, int S, class Body>

@@ -70,7 +70,7 @@ def test_misaligned_views_use_the_generic_path():
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-@pytest.mark.parametrize("shape", [(8, 12, 3, 2), (4, 8, 1, 1), (3, 4, 5, 7)])
+@pytest.mark.parametrize("shape", [(8, 12, 3, 2), (4, 8, 1, 1), (3, 4, 5, 7), (64, 64, 3, 3), (32, 64, 7, 7)])
 def test_conv_layout(dtype, shape):
     K, C, R, S = shape
     od = ORACLE_DT[dtype]
