@@ -7,10 +7,12 @@
 // Y[t, s, n] = sum_k x[t, k] W[e, n, k] with e = routing[t, s].  Steps, all on the device:
 //   1. route_count:   histogram of expert ids (atomic adds into counts[E]);
 //   2. route_scan:    one CTA turns counts into offsets (exclusive scan) and a table of token
-//                     tiles (expert, first index, count <= 64);
+//                     tiles (expert, first index, count <= tile);
 //   3. route_scatter: each (t, s) takes a slot of its expert's range (perm = t * topk + s);
-//   4. the staged skinny kernel in grouped mode: grid (64-row weight blocks, K slices, tiles),
-//      each CTA gathering its tile's x rows by index and adding into Y[t, s, :].
+//   4. NVFP4 experts with 16-bit tokens: the tensor-core kernel over tiles of up to 128 routed
+//      rows, each CTA writing its outputs once; other formats: the staged skinny kernel in
+//      grouped mode over tiles of 64 (grid: 64-row weight blocks, K slices, tiles), each CTA
+//      gathering its tile's x rows by index and adding into Y[t, s, :].
 // The order of tokens inside an expert's range depends on atomic arrival, but every output is a
 // complete sum for one (t, s), so the result does not.
 #include "sp24_internal.cuh"
@@ -18,7 +20,8 @@
 namespace sp24 {
 namespace {
 
-constexpr int kTile = 64;
+constexpr int kTile = 64;     // token tile of the skinny kernel (the smallest tile: sizes the table)
+constexpr int kTileTc = 128;  // token tile of the tensor-core kernel
 
 __global__ void route_count(const int32_t* __restrict__ routing, int64_t n, int64_t E, int32_t* __restrict__ counts) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
@@ -34,7 +37,7 @@ __global__ void route_count(const int32_t* __restrict__ routing, int64_t n, int6
 // Single CTA of 1024 threads: block-wide exclusive scans over E experts in chunks of 1024.
 __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ counts, int64_t E,
                                                    int32_t* __restrict__ offsets, int32_t* __restrict__ tiles,
-                                                   int64_t max_tiles) {
+                                                   int64_t max_tiles, int tile) {
   __shared__ int32_t warp_sum[2][32];
   __shared__ int32_t carry[2];
   if (threadIdx.x == 0) carry[0] = carry[1] = 0;
@@ -43,7 +46,7 @@ __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ c
   for (int64_t base = 0; base < E; base += 1024) {
     const int64_t e = base + threadIdx.x;
     const int32_t cnt = e < E ? counts[e] : 0;
-    const int32_t nt = (cnt + kTile - 1) / kTile;
+    const int32_t nt = (cnt + tile - 1) / tile;
     // inclusive warp scans of (cnt, nt)
     int32_t a = cnt, b = nt;
 #pragma unroll
@@ -80,8 +83,8 @@ __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ c
       for (int32_t j = 0; j < nt && pre_b + j < max_tiles; ++j) {
         int32_t* t = tiles + 3 * (int64_t)(pre_b + j);
         t[0] = (int32_t)e;
-        t[1] = pre_a + kTile * j;
-        t[2] = cnt - kTile * j < kTile ? cnt - kTile * j : kTile;
+        t[1] = pre_a + tile * j;
+        t[2] = cnt - tile * j < tile ? cnt - tile * j : tile;
       }
     }
     __syncthreads();
@@ -95,12 +98,18 @@ __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ c
   for (int64_t i = carry[1] + threadIdx.x; i < max_tiles; i += blockDim.x) tiles[3 * i + 2] = 0;
 }
 
+// Also zeroes the outputs of routed rows with an invalid expert id when `y_zero` is set (the
+// tensor-core path writes every valid output once and clears nothing else beforehand).
 __global__ void route_scatter(const int32_t* __restrict__ routing, int64_t n, int64_t E,
                               const int32_t* __restrict__ offsets, int32_t* __restrict__ fill,
-                              int32_t* __restrict__ perm) {
+                              int32_t* __restrict__ perm, float* __restrict__ y_zero, int64_t N) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int32_t e = routing[i];
-    if (e < 0 || e >= E) continue;
+    if (e < 0 || e >= E) {
+      if (y_zero)
+        for (int64_t c = 0; c < N; ++c) y_zero[i * N + c] = 0.0f;
+      continue;
+    }
     perm[offsets[e] + atomicAdd(&fill[e], 1)] = (int32_t)i;
   }
 }
@@ -156,8 +165,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   if (n == 0 || N == 0) return SP24_OK;
   if (!routing || !y) return SP24_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
-  if (cudaMemsetAsync(y, 0, (size_t)(n * N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
-  if (K == 0) return SP24_OK;
+  if (K == 0) return cudaMemsetAsync(y, 0, (size_t)(n * N) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
 
   SkinnyParams p{};
   // activations
@@ -217,8 +225,12 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.N = N;
   p.K = K;
   p.y = y;
-  p.M = kTile;
-  if (!skinny2_supported(wf, p)) return SP24_ERR_UNSUPPORTED;
+  const bool tc = moe_tc_supported(wf, p.x_fmt, N, K, n / kTileTc + E, p.w, p.w_scales, p.x);
+  const int tile = tc ? kTileTc : kTile;
+  p.M = tile;
+  if (!tc && !skinny2_supported(wf, p)) return SP24_ERR_UNSUPPORTED;
+  // the skinny kernel adds K-slice partial sums into Y; the tensor-core kernel stores each output
+  if (!tc && cudaMemsetAsync(y, 0, (size_t)(n * N) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
 
   MoeWs ws = moe_layout(workspace, T, topk, E);
   if (!workspace || workspace_bytes < ws.bytes) return SP24_ERR_WORKSPACE;
@@ -226,14 +238,17 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   const size_t zero_bytes = (size_t)(reinterpret_cast<uint8_t*>(ws.offsets) - reinterpret_cast<uint8_t*>(ws.counts));
   if (cudaMemsetAsync(ws.counts, 0, zero_bytes, s) != cudaSuccess) return SP24_ERR_CUDA;  // counts + fill
   const int blocks = (int)((n + 255) / 256 < (int64_t)sm_count() * 4 ? (n + 255) / 256 : (int64_t)sm_count() * 4);
+  // tiles of `tile` rows: at most sum_e ceil(c_e / tile) <= n / tile + E of them
+  const int64_t n_tiles = n / tile + E < ws.max_tiles ? n / tile + E : ws.max_tiles;
   route_count<<<blocks, 256, 0, s>>>(routing, n, E, ws.counts);
-  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles);
-  route_scatter<<<blocks, 256, 0, s>>>(routing, n, E, ws.offsets, ws.fill, ws.perm);
+  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles, tile);
+  route_scatter<<<blocks, 256, 0, s>>>(routing, n, E, ws.offsets, ws.fill, ws.perm, tc ? y : nullptr, N);
   int st = launch_status(3);
   if (st) return st;
   p.perm = ws.perm;
   p.tiles = ws.tiles;
   p.topk = topk;
   p.expert_rows = N;
-  return skinny2_grouped(wf, t16, p, ws.max_tiles, s);
+  if (tc) return moe_tc_grouped(t16, p, n_tiles, s);
+  return skinny2_grouped(wf, t16, p, n_tiles, s);
 }

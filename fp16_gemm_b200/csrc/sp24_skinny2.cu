@@ -27,6 +27,7 @@
 #include "sp24_internal.cuh"
 #include "sp24_tc.cuh"
 #include "sp24_stream.cuh"
+#include "sp24_fp4.cuh"
 
 namespace sp24 {
 namespace {
@@ -87,72 +88,6 @@ struct Smem2 {
   // x + one weight buffer (one row block per CTA) or two (grouped: row blocks double-buffered)
   static constexpr int bytes(bool two) { return TOTAL + (two ? WREG : 0); }
 };
-
-template <typename T>
-struct P2;
-template <>
-struct P2<__nv_bfloat16> {  // 16-bit pattern of E2M1(code) * 2^-126
-  static constexpr uint32_t MAG = 0x01C001C0u;
-  static constexpr int MAGPOS = 6;
-  static constexpr float FOLD = 0x1p118f;
-};
-template <>
-struct P2<__half> {  // 16-bit pattern of E2M1(code) * 2^-14
-  static constexpr uint32_t MAG = 0x0E000E00u;
-  static constexpr int MAGPOS = 9;
-  static constexpr float FOLD = 0x1p6f;
-};
-
-__device__ __forceinline__ uint32_t shl2(uint32_t x, int n) { return n >= 0 ? x << n : x >> (-n); }
-
-// Nibbles i and i+4 of w -> 16-bit pair of E2M1 patterns.
-template <typename T>
-__device__ __forceinline__ uint32_t fp4_pair_i4(uint32_t w, int i) {
-  return (shl2(w, P2<T>::MAGPOS - 4 * i) & P2<T>::MAG) | (shl2(w, 12 - 4 * i) & 0x80008000u);
-}
-
-// The byte at bits [8bb, 8bb+8) of w (two consecutive codes) -> 16-bit pair (lo, hi).
-template <typename T>
-__device__ __forceinline__ uint32_t fp4_pair_byte(uint32_t w, int bb) {
-  const uint32_t x = w >> (8 * bb);
-  constexpr int P = P2<T>::MAGPOS;
-  return ((x << P) & (7u << P)) | ((x << 12) & 0x8000u) | ((x << (P + 12)) & (7u << (P + 16))) |
-         ((x << 24) & 0x80000000u);
-}
-
-template <typename T>
-__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
-  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  } else {
-    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ uint16_t to_bits16(float f) {
-  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-    __nv_bfloat16 v = __float2bfloat16_rn(f);
-    return *reinterpret_cast<uint16_t*>(&v);
-  } else {
-    __half v = __float2half_rn(f);
-    return *reinterpret_cast<uint16_t*>(&v);
-  }
-}
-
-// Two E4M3 block scales (low bytes of code2) -> two packed multipliers E4M3 * FOLD (exact).
-template <typename T>
-__device__ __forceinline__ void scale_pair(uint32_t code2, uint32_t& s0, uint32_t& s1) {
-  uint32_t h2;
-  const uint16_t c = (uint16_t)code2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
-  const uint32_t a = to_bits16<T>(__half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu))) * P2<T>::FOLD);
-  const uint32_t b = to_bits16<T>(__half2float(__ushort_as_half((unsigned short)(h2 >> 16))) * P2<T>::FOLD);
-  s0 = a | (a << 16);
-  s1 = b | (b << 16);
-}
 
 template <typename T>
 __device__ __forceinline__ void mma_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -16,6 +16,8 @@ Workloads (the shapes the pages' workloads take; see the design notes for the ma
 * ``moe``:           W bf16 [512, 512, 2048] N(0, 0.02), X bf16 [4096, 2048] N(0, 1), then
                      routing int32 [4096, 10]: ten distinct experts per token, uniform
                      without replacement.
+* ``moe_skewed``:    W bf16 [E, N, K] N(0, 0.02), X [T, K] N(0, 1), routing with given per-expert
+                     row counts in a seeded random order (tile-boundary parity cases).
 * ``msweep``:        W [5120, 5120] then X [M, 5120], N(0, 1), fp16 or bf16.
 * ``conv_fail5``:    W fp16 [256, 256, 3, 3] N(0, 1) with a 2-of-4 zero pattern along C
                      drawn at random per group, then round(5%) of the groups (a seeded
@@ -103,6 +105,22 @@ def moe(seed: int = SEED, E: int = 512, N: int = 512, K: int = 2048, T: int = 40
         W[e] = draw(g, (N, K), "bf16", 0.02)
     X = draw(g, (T, K), "bf16")
     routing = routing_topk(g, T, E, topk)
+    return {"W": W, "X": X, "routing": routing}
+
+
+def moe_skewed(counts, seed: int = SEED, N: int = 256, K: int = 320, topk: int = 2,
+               xdtype: str = "bf16"):
+    """Routing with exactly counts[e] routed rows on expert e: the flat list of expert ids in a
+    seeded random order, reshaped to [T, topk] (T = sum(counts) / topk; a token may meet the
+    same expert twice).  W bf16 [E, N, K] N(0, 0.02), then X [T, K] N(0, 1) in `xdtype`."""
+    counts = list(counts)
+    n = int(sum(counts))
+    assert n % topk == 0
+    g = rng(seed)
+    W = draw(g, (len(counts), N, K), "bf16", 0.02)
+    X = draw(g, (n // topk, K), xdtype)
+    flat = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
+    routing = g.permutation(flat).reshape(n // topk, topk).astype(np.int32)
     return {"W": W, "X": X, "routing": routing}
 
 

@@ -38,7 +38,7 @@ def _expert_sparse_decoded(W_e, wfmt, ts):
 
 def _run(X, W, routing, xfmt, wfmt, sparse, tokens):
     E, N, K = W.shape
-    x = to_dev(X, "bf16")
+    x = to_dev(X, "f16" if xfmt == "f16" else "bf16")
     if xfmt == "nvfp4":
         x = sp.quantize_nvfp4(x)
     w = to_dev(W.reshape(E * N, K), "bf16")
@@ -62,7 +62,7 @@ def _run(X, W, routing, xfmt, wfmt, sparse, tokens):
         c, s, xts = oracle.nvfp4_encode(X, oracle.BF16)
         Xd = oracle.nvfp4_decode(c[tokens], s[tokens], xts)
     else:
-        Xd = oracle.to_double(np.ascontiguousarray(X[tokens]), oracle.BF16)
+        Xd = oracle.to_double(np.ascontiguousarray(X[tokens]), oracle.F16 if xfmt == "f16" else oracle.BF16)
     used = sorted(set(routing[tokens].ravel().tolist()))
     dec = {e: (_expert_sparse_decoded if sparse else _expert_dense_decoded)(np.ascontiguousarray(W[e]), wfmt, ts)
            for e in used}
@@ -101,3 +101,47 @@ def test_moe_rejects_bad_expert_ids():
     y = sp.gemm_grouped(x, r, w, 4, 64, 512)
     assert sp.last_device_error() == sp.ERR_INVALID_ARG
     assert not y[0, 0].any()
+
+
+# Per-expert routed-row counts around the 128-row token tiles and the 16-row MMA granularity of
+# the tensor-core path (NVFP4 experts, 16-bit tokens, N % 128, K % 64): an expert spanning three
+# tiles (128, 128, 44), tiles of 1, 15, 16, 17, 127, 128 and 129 rows, and experts with none.
+SKEW = [300, 1, 0, 15, 16, 17, 127, 0, 128, 129, 1]
+
+
+@pytest.mark.parametrize("xfmt", ["bf16", "f16"])
+@pytest.mark.parametrize("NK", [(256, 320), (128, 64), (384, 128), (128, 2112)],
+                         ids=lambda s: f"N{s[0]}-K{s[1]}")
+def test_moe_tile_boundaries(NK, xfmt):
+    """Every output of skewed routings: 128-row tiles at their edges, K of 1, 2, 5 and 33
+    stages of 64, one to three weight-row blocks of 128, bf16 and f16 tokens."""
+    N, K = NK
+    d = synth.moe_skewed(SKEW, seed=11, N=N, K=K, topk=2, xdtype=xfmt)
+    T = d["X"].shape[0]
+    _run(d["X"], d["W"], d["routing"], xfmt, "nvfp4", False, np.arange(T))
+
+
+def test_moe_single_routed_row():
+    """One token, one expert of eight: a single 16-wide MMA tile with 15 zero-filled rows."""
+    d = synth.moe_skewed([0, 0, 0, 1, 0, 0, 0, 0], seed=12, N=128, K=256, topk=1)
+    _run(d["X"], d["W"], d["routing"], "bf16", "nvfp4", False, np.arange(1))
+
+
+def test_moe_bad_expert_ids_tensor_core_path():
+    """Invalid ids on the tensor-core path (no output memset there): error word set and the
+    invalid rows' outputs zero, the valid rows still right."""
+    d = synth.moe_skewed([40, 40, 48], seed=13, N=128, K=256, topk=2)
+    X, W, routing = d["X"], d["W"], d["routing"].copy()
+    E, N, K = W.shape
+    x = to_dev(X, "bf16")
+    w = sp.quantize_nvfp4(to_dev(W.reshape(E * N, K), "bf16"))
+    bad = routing.copy()
+    bad[0, 1] = E
+    bad[5, 0] = -1
+    r = torch.from_numpy(bad).cuda()
+    y = torch.full((X.shape[0], 2, N), float("nan"), device="cuda")
+    sp.gemm_grouped(x, r, w, E, N, K, out=y)
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.ERR_INVALID_ARG
+    assert not y[0, 1].any() and not y[5, 0].any()
+    assert torch.isfinite(y).all()
