@@ -225,7 +225,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.N = N;
   p.K = K;
   p.y = y;
-  const bool tc = moe_tc_supported(wf, p.x_fmt, N, K, n / kTileTc + E, p.w, p.w_scales, p.x);
+  const bool tc = moe_tc_supported(wf, p.x_fmt, T, E, N, K, n / kTileTc + E, p.w, p.w_scales, p.x);
   const int tile = tc ? kTileTc : kTile;
   p.M = tile;
   if (!tc && !skinny2_supported(wf, p)) return SP24_ERR_UNSUPPORTED;
@@ -249,6 +249,6 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.tiles = ws.tiles;
   p.topk = topk;
   p.expert_rows = N;
-  if (tc) return moe_tc_grouped(t16, p, n_tiles, s);
+  if (tc) return moe_tc_grouped(t16, p, E, T, n_tiles, s);
   return skinny2_grouped(wf, t16, p, n_tiles, s);
 }

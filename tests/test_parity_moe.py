@@ -104,17 +104,18 @@ def test_moe_rejects_bad_expert_ids():
 
 
 # Per-expert routed-row counts around the 128-row token tiles and the 16-row MMA granularity of
-# the tensor-core path (NVFP4 experts, 16-bit tokens, N % 128, K % 64): an expert spanning three
+# the tensor-core path (NVFP4 experts, 16-bit tokens, N % 128, K % 256): an expert spanning three
 # tiles (128, 128, 44), tiles of 1, 15, 16, 17, 127, 128 and 129 rows, and experts with none.
 SKEW = [300, 1, 0, 15, 16, 17, 127, 0, 128, 129, 1]
 
 
 @pytest.mark.parametrize("xfmt", ["bf16", "f16"])
-@pytest.mark.parametrize("NK", [(256, 320), (128, 64), (384, 128), (128, 2112)],
+@pytest.mark.parametrize("NK", [(256, 512), (128, 256), (384, 768), (128, 2304)],
                          ids=lambda s: f"N{s[0]}-K{s[1]}")
 def test_moe_tile_boundaries(NK, xfmt):
-    """Every output of skewed routings: 128-row tiles at their edges, K of 1, 2, 5 and 33
-    stages of 64, one to three weight-row blocks of 128, bf16 and f16 tokens."""
+    """Every output of skewed routings: 128-row tiles at their edges, K of 1, 2, 3 and 9
+    weight boxes of 256 (the last wraps the four-box ring twice), one to three weight-row
+    blocks of 128, bf16 and f16 tokens."""
     N, K = NK
     d = synth.moe_skewed(SKEW, seed=11, N=N, K=K, topk=2, xdtype=xfmt)
     T = d["X"].shape[0]
