@@ -5,14 +5,14 @@
 // one token tile of one expert (up to 128 routed rows) against 128 of the expert's weight rows
 // over the whole K, so every output has one writer and no K slice is reduced through atomics.
 //
-// Roles (K advances in stages of 64; stage i uses slot i % 8 of an x ring in shared memory and
-// of an A ring in tensor memory):
+// Roles (K advances in stages of 64; stage i uses slot i % 10 of an x ring in shared memory and
+// of an A ring in tensor memory; slots are synchronised in pairs):
 //   * TMA warp W loads the raw weights of four stages at a time: the 128 rows' code bytes
 //     (128-byte rows, 128-byte swizzle) and their E4M3 block scales (16-byte rows);
 //   * eight gather warps copy the tile's token rows of x for each stage with 16-byte cp.async
 //     (rows past the tile's count zero-filled) into a 128-byte swizzled K-major tile, the MMA's
-//     B operand, six stages ahead; once a stage has landed they fence the generic proxy against
-//     the async proxy and arrive on its barrier (TMA row gathers move only 512 bytes per
+//     B operand, three stage pairs ahead; once a pair has landed they fence the generic proxy
+//     against the async proxy and arrive on its barrier (TMA row gathers move only 512 bytes per
 //     instruction, and the SM issues TMA instructions far too slowly for that);
 //   * four groups of four converter warps: group g expands stages g, g + 4, g + 8, ... (thread
 //     = weight row): code pairs -> 16-bit values (hardware E2M1 conversion) times the block
@@ -41,9 +41,10 @@ constexpr int kMtRows = 128;      // weight rows per CTA (MMA M)
 constexpr int kMtTok = 128;       // routed rows per token tile (MMA N <= 128)
 constexpr int kMtBK = 64;         // K per stage
 constexpr int kMtBoxK = 256;      // K per weight box (four stages)
-constexpr int kMtBoxes = 4;       // weight boxes in flight (16 stages)
-constexpr int kMtSlots = 8;       // stage slots: x tile in shared memory + A slot in TMEM (i % 8)
-constexpr int kMtDx = kMtSlots - 2;  // x is copied six stages ahead (its slot's MMA i - 2 is done)
+constexpr int kMtBoxes = 3;       // weight boxes in flight (12 stages)
+constexpr int kMtSlots = 10;      // stage slots: x tile in shared memory + A slot in TMEM (i % 10)
+constexpr int kMtPairs = kMtSlots / 2;
+constexpr int kMtDp = kMtPairs - 2;  // x is copied three stage pairs ahead (the slot pair's MMAs, two pairs back, are done)
 constexpr int kMtGroups = 4;      // converter groups
 constexpr int kMtConvWarps = 4 * kMtGroups;
 constexpr int kMtGatherWarps = 8;
@@ -138,9 +139,10 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem;                           // [kMtBoxes][codes 128 x 128 B swizzled | scales 128 x 16 B]
   uint8_t* sX = smem + kMtBoxes * kMtBox;       // [kMtSlots][128 rows x 128 B swizzled]
-  // st_full[s]: stage in slot s has its A (4 converter warps) and its x (8 gather warps);
-  // st_empty[s]: the MMAs that read slot s have completed (commit)
-  __shared__ uint64_t w_full[kMtBoxes], w_empty[kMtBoxes], st_full[kMtSlots], st_empty[kMtSlots], tfull_bar;
+  // Slots are synchronised in pairs (2q, 2q + 1), so the MMA thread waits and commits once per
+  // two stages.  st_full[q]: both stages have their A (4 converter warps each) and their x (8
+  // gather warps each); st_empty[q]: the MMAs that read the pair have completed (commit).
+  __shared__ uint64_t w_full[kMtBoxes], w_empty[kMtBoxes], st_full[kMtPairs], st_empty[kMtPairs], tfull_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int aborted;
   __shared__ int32_t s_perm[kMtTok];
@@ -160,9 +162,9 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       mbar_init(&w_full[s], 1);
       mbar_init(&w_empty[s], kMtConvWarps);
     }
-    for (int s = 0; s < kMtSlots; ++s) {
-      mbar_init(&st_full[s], 4 + kMtGatherWarps);
-      mbar_init(&st_empty[s], 1);
+    for (int q = 0; q < kMtPairs; ++q) {
+      mbar_init(&st_full[q], 2 * 4 + kMtGatherWarps);  // two converter groups, the gather warps once
+      mbar_init(&st_empty[q], 1);
     }
     mbar_init(&tfull_bar, 1);
     aborted = 0;
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       }
       const int as = i % kMtSlots;
       if (i >= kMtSlots &&
-          !__all_sync(0xffffffffu, mbar_wait(&st_empty[as], ((i / kMtSlots) - 1) & 1))) {  // MMA i - 8 done
+          !__all_sync(0xffffffffu, mbar_wait(&st_empty[as >> 1], ((i / kMtSlots) - 1) & 1))) {  // MMA i - 10 done
         aborted = 1;
         break;
       }
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       tmem_st32(a_base + kMtACols * as, a);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st_full[as]);
+      if (lane == 0) mbar_arrive(&st_full[as >> 1]);
     }
 
     // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (weight rows) and accumulator
@@ -242,23 +244,30 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       // The next stage's barrier is tested (without waiting) before this stage's MMAs are
       // issued, so the test's latency overlaps them.
       const uint32_t idesc = idesc_f16(kMtRows, n_mma, kBf16);
+      const uint64_t b_first = desc_kmajor_sw128(smem_u32(sX));
+      const int KP = KB / 2;  // stage pairs (KB is a multiple of 4)
       bool ready = mbar_wait(&st_full[0], 0);
 #pragma unroll 1
-      for (int i = 0; i < KB; ++i) {
-        if (!ready || *(volatile int*)&aborted) {
+      for (int pr = 0; pr < KP; ++pr) {
+        if (!ready) {  // a producer gave up (or the wait ran out): stop issuing
           aborted = 1;
           break;
         }
-        const int s = i % kMtSlots, sn = (i + 1) % kMtSlots;
-        const uint32_t pn = ((i + 1) / kMtSlots) & 1;
-        const bool next = i + 1 < KB && mbar_test_wait(&st_full[sn], pn);
+        const int q = pr % kMtPairs, qn = (pr + 1) % kMtPairs;
+        const uint32_t pn = ((pr + 1) / kMtPairs) & 1;
+        const bool next = pr + 1 < KP && mbar_test_wait(&st_full[qn], pn);
         tc_fence_after();
-        const uint64_t b0 = desc_kmajor_sw128(smem_u32(sX + s * kMtX));
-        const uint32_t a0 = tmem + kMtAccCols + kMtACols * s;
 #pragma unroll
-        for (int k = 0; k < kMtBK / 16; ++k) umma_f16_tmem_a(tmem, a0 + 8 * k, b0 + 2 * k, idesc, (i | k) != 0);
-        umma_commit(&st_empty[s]);
-        ready = i + 1 >= KB || next || mbar_wait(&st_full[sn], pn);
+        for (int h = 0; h < 2; ++h) {
+          const int s = 2 * q + h;
+          const uint64_t b0 = b_first + (uint64_t)(s * (kMtX >> 4));  // descriptor address: 16-byte units
+          const uint32_t a0 = tmem + kMtAccCols + kMtACols * s;
+#pragma unroll
+          for (int k = 0; k < kMtBK / 16; ++k)
+            umma_f16_tmem_a(tmem, a0 + 8 * k, b0 + 2 * k, idesc, (pr | h | k) != 0);
+        }
+        umma_commit(&st_empty[q]);
+        ready = pr + 1 >= KP || next || mbar_wait(&st_full[qn], pn);
       }
       umma_commit(&tfull_bar);  // also after an abort, so the epilogue does not wait in vain
     }
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     }
   } else {
     // ---- token rows: gather thread t copies 16-byte chunk t % 8 of routed rows t / 8 + 32u
-    // (u = 0 .. 3) of each stage, kMtDx stages ahead (rows count .. n_mma - 1 zero-filled)
+    // (u = 0 .. 3) of each stage, kMtDp stage pairs ahead (rows count .. n_mma - 1 zero-filled)
     const int t = tid - 32 * kMtWarpX0, j = t & 7;
     const uint16_t* xrow[4];
     uint32_t xoff[4], xbytes[4];
@@ -303,27 +312,31 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       for (int u = 0; u < 4; ++u)
         if (u < nx) cp_async16_zfill(b + xoff[u], xrow[u] + (int64_t)kx * kMtBK, xbytes[u]);
     };
-    for (int kx = 0; kx < kMtDx; ++kx) {  // the first kMtDx stages: their slots are fresh
-      if (kx < KB) issue(kx);
+    const int KP = KB / 2;
+    for (int pp = 0; pp < kMtDp; ++pp) {  // the first pairs: their slots are fresh
+      if (pp < KP) {
+        issue(2 * pp);
+        issue(2 * pp + 1);
+      }
       cp_async_commit();
     }
 #pragma unroll 1
-    for (int i = 0; i < KB; ++i) {
-      cp_async_wait<kMtDx - 1>();  // this thread's chunks of stage i have landed
+    for (int pr = 0; pr < KP; ++pr) {
+      cp_async_wait<kMtDp - 1>();  // this thread's chunks of stage pair pr have landed
       fence_proxy_async_smem();    // ... and are visible to the MMA's operand reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st_full[i % kMtSlots]);
-      const int kx = i + kMtDx;
-      if (kx < KB) {
-        if (kx >= kMtSlots) {  // the slot's previous stage kx - kMtSlots = i - 2 is multiplied
-          const bool ok =
-              mbar_wait(&st_empty[kx % kMtSlots], ((kx / kMtSlots) - 1) & 1) && !*(volatile int*)&aborted;
+      if (lane == 0) mbar_arrive(&st_full[pr % kMtPairs]);
+      const int pn = pr + kMtDp;
+      if (pn < KP) {
+        if (pn >= kMtPairs) {  // the slot pair's previous pair pn - kMtPairs = pr - 2 is multiplied
+          const bool ok = mbar_wait(&st_empty[pn % kMtPairs], ((pn / kMtPairs) - 1) & 1) && !*(volatile int*)&aborted;
           if (!__all_sync(0xffffffffu, ok)) {
             aborted = 1;
             break;
           }
         }
-        issue(kx);
+        issue(2 * pn);
+        issue(2 * pn + 1);
       }
       cp_async_commit();
     }
