@@ -118,11 +118,12 @@ int make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64
                        uint32_t box_cols, uint32_t box_rows);
 // Grouped variant: one launch over max_tiles token tiles (tile table and perm on the device).
 int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStream_t s);
-// Routed-expert GEMM on the tensor cores for NVFP4 experts and 16-bit tokens: token tiles of up
-// to 128 routed rows (p.tiles, p.perm), 128 weight rows per CTA, tcgen05.mma into TMEM.
+// Routed-expert GEMM on the tensor cores for NVFP4 experts (dense W_DQ4 or 2:4 W_SQ4) and 16-bit
+// tokens: token tiles of up to 128 routed rows (p.tiles, p.perm), 128 weight rows per CTA,
+// tcgen05.mma (.sp for 2:4) into TMEM.
 bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_t K, int64_t max_tiles,
-                      const void* codes, const void* scales, const void* x);
-int moe_tc_grouped(int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s);
+                      const void* codes, const void* scales, const void* meta, const void* x);
+int moe_tc_grouped(int wf, int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s);
 
 // Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,

@@ -9,8 +9,8 @@
 //   2. route_scan:    one CTA turns counts into offsets (exclusive scan) and a table of token
 //                     tiles (expert, first index, count <= tile);
 //   3. route_scatter: each (t, s) takes a slot of its expert's range (perm = t * topk + s);
-//   4. NVFP4 experts with 16-bit tokens: the tensor-core kernel over tiles of up to 128 routed
-//      rows, each CTA writing its outputs once; other formats: the staged skinny kernel in
+//   4. NVFP4 experts (dense or 2:4) with 16-bit tokens: the tensor-core kernel over tiles of up
+//      to 128 routed rows, each CTA writing its outputs once; other formats: the staged skinny kernel in
 //      grouped mode over tiles of 64 (grid: 64-row weight blocks, K slices, tiles), each CTA
 //      gathering its tile's x rows by index and adding into Y[t, s, :].
 // The order of tokens inside an expert's range depends on atomic arrival, but every output is a
@@ -225,7 +225,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.N = N;
   p.K = K;
   p.y = y;
-  const bool tc = moe_tc_supported(wf, p.x_fmt, T, E, N, K, n / kTileTc + E, p.w, p.w_scales, p.x);
+  const bool tc = moe_tc_supported(wf, p.x_fmt, T, E, N, K, n / kTileTc + E, p.w, p.w_scales, p.meta, p.x);
   const int tile = tc ? kTileTc : kTile;
   p.M = tile;
   if (!tc && !skinny2_supported(wf, p)) return SP24_ERR_UNSUPPORTED;
@@ -249,6 +249,6 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.tiles = ws.tiles;
   p.topk = topk;
   p.expert_rows = N;
-  if (tc) return moe_tc_grouped(t16, p, E, T, n_tiles, s);
+  if (tc) return moe_tc_grouped(wf, t16, p, E, T, n_tiles, s);
   return skinny2_grouped(wf, t16, p, n_tiles, s);
 }

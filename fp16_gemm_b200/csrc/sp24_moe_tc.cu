@@ -1,14 +1,18 @@
-// a7 on the tensor cores: routed-expert GEMM with 16-bit tokens and NVFP4 experts (W4A16).
+// a7 on the tensor cores: routed-expert GEMM with 16-bit tokens and NVFP4 experts (W4A16),
+// dense or 2:4-compressed.
 //
 // [P1] "NVFP4 vs 2:4 sparse", "Concurrency, not sparsity, is the lever": every touched expert's
 // weights are read once per step, and the tokens routed to it share that read.  One CTA computes
 // one token tile of one expert (up to 128 routed rows) against 128 of the expert's weight rows
 // over the whole K, so every output has one writer and no K slice is reduced through atomics.
+// [P2] "The mechanism needs both values and their positions": for 2:4 experts the kept values
+// are the MMA's A operand and their positions travel as tcgen05 sparse metadata.
 //
-// Roles (K advances in stages of 64; stage i uses slot i % 10 of an x ring in shared memory and
-// of an A ring in tensor memory; slots are synchronised in pairs):
-//   * TMA warp W loads the raw weights of four stages at a time: the 128 rows' code bytes
-//     (128-byte rows, 128-byte swizzle) and their E4M3 block scales (16-byte rows);
+// Roles (K advances in stages of 64 logical elements; stage i uses slot i % 10 of an x ring in
+// shared memory and of an A ring in tensor memory; slots are synchronised in pairs):
+//   * TMA warp W loads the raw weights of 4 (dense) or 8 (2:4) stages at a time: the 128 rows'
+//     code bytes (128-byte rows, 128-byte swizzle), their E4M3 block scales (16-byte rows) and,
+//     for 2:4, their metadata nibbles (64-byte rows);
 //   * eight gather warps copy the tile's token rows of x for each stage with 16-byte cp.async
 //     (rows past the tile's count zero-filled) into a 128-byte swizzled K-major tile, the MMA's
 //     B operand, three stage pairs ahead; once a pair has landed they fence the generic proxy
@@ -16,14 +20,19 @@
 //     instruction, and the SM issues TMA instructions far too slowly for that);
 //   * four groups of four converter warps: group g expands stages g, g + 4, g + 8, ... (thread
 //     = weight row): code pairs -> 16-bit values (hardware E2M1 conversion) times the block
-//     scale, written with tcgen05.st into the stage's 32-column slot of tensor memory, the MMA's
-//     A operand (lane = weight row, two K elements per column), then arrive on its barrier;
-//   * one thread issues four `tcgen05.mma kind::f16` per stage (M = 128 weight rows, N = the
-//     tile's count rounded up to 16, K = 16, A from TMEM, B from shared memory) into a TMEM
-//     accumulator and commits the slot back to its producers.  An MMA instruction costs the
-//     same for any N up to 64 and little more up to 128, so at ~80 routed rows this thread's own
-//     pace matters: one barrier per stage, tested for the next stage before the current
-//     stage's MMAs are issued;
+//     scale, written with tcgen05.st into the stage's slot of tensor memory, the MMA's A operand
+//     (lane = weight row, two stored values per column: 32 columns dense, 16 for 2:4).  For 2:4
+//     the row's metadata nibbles are regrouped with warp shuffles into the tcgen05 metadata
+//     layout (TMEM lane l carries rows m = 16 (l / 16) + l % 8 and m + 8, the nibbles of groups
+//     4 ((l / 8) % 2) .. + 3 of each 32-wide K window, one column per window: the low half for
+//     row m, the high half for row m + 8) and stored into two columns beside the slot;
+//   * one thread issues the stage's MMAs (M = 128 weight rows, N = the tile's count rounded up
+//     to 16, A from TMEM, B from shared memory): four `tcgen05.mma kind::f16` (K = 16) dense,
+//     two `tcgen05.mma.sp kind::f16` (K = 32 logical) for 2:4, into a TMEM accumulator, and
+//     commits each slot pair back to its producers.  An MMA instruction costs about the same for
+//     any N up to 128, so at ~80 routed rows the instruction count sets the pace and the 2:4
+//     form needs half as many: one barrier per stage pair, tested for the next pair before the
+//     current pair's MMAs are issued;
 //   * after the last stage the converter warps read the accumulator (lane = weight row, column
 //     = routed row) and store y[token, slot, row] * unscale * tensor scale once.
 // Every wait is bounded; on a timeout the CTA records SP24_ERR_DEVICE_TIMEOUT, lets its copies
@@ -39,9 +48,7 @@ using namespace tc;
 
 constexpr int kMtRows = 128;      // weight rows per CTA (MMA M)
 constexpr int kMtTok = 128;       // routed rows per token tile (MMA N <= 128)
-constexpr int kMtBK = 64;         // K per stage
-constexpr int kMtBoxK = 256;      // K per weight box (four stages)
-constexpr int kMtBoxes = 3;       // weight boxes in flight (12 stages)
+constexpr int kMtBK = 64;         // logical K per stage
 constexpr int kMtSlots = 10;      // stage slots: x tile in shared memory + A slot in TMEM (i % 10)
 constexpr int kMtPairs = kMtSlots / 2;
 constexpr int kMtDp = kMtPairs - 2;  // x is copied three stage pairs ahead (the slot pair's MMAs, two pairs back, are done)
@@ -50,16 +57,27 @@ constexpr int kMtConvWarps = 4 * kMtGroups;
 constexpr int kMtGatherWarps = 8;
 constexpr int kMtWarpMma = kMtConvWarps, kMtWarpW = kMtConvWarps + 1, kMtWarpX0 = kMtConvWarps + 2;
 constexpr int kMtThreads = 32 * (kMtWarpX0 + kMtGatherWarps);
-constexpr uint32_t kMtCodeBox = kMtRows * kMtBoxK / 2;    // 16 KB: 128 rows x 128 code bytes
-constexpr uint32_t kMtScaleBox = kMtRows * kMtBoxK / 16;  // 2 KB: 128 rows x 16 scale bytes
-constexpr uint32_t kMtBox = kMtCodeBox + kMtScaleBox;
 constexpr uint32_t kMtX = kMtTok * kMtBK * 2;              // 16 KB
-constexpr size_t kMtSmem = (size_t)kMtBoxes * kMtBox + (size_t)kMtSlots * kMtX + 1024;
 constexpr uint32_t kMtAccCols = 128;                       // fp32 accumulator, one column per routed row
-constexpr uint32_t kMtACols = kMtBK / 2;                   // 32 columns: one stage of A (16-bit pairs)
-constexpr uint32_t kMtCols = 512;                          // accumulator + kMtSlots A slots
-static_assert(kMtAccCols + kMtSlots * kMtACols <= kMtCols, "tensor memory");
-static_assert(kMtSmem <= 227 * 1024, "shared memory");
+constexpr uint32_t kMtCols = 512;
+constexpr uint32_t kMtCodeBox = kMtRows * 128;             // 16 KB: 128 rows x 128 code bytes
+constexpr uint32_t kMtScaleBox = kMtRows * 16;             // 2 KB: 128 rows x 16 scale bytes
+
+// Geometry of the dense (SP = false) and 2:4 (SP = true) weight streams.
+template <bool SP>
+struct MtGeom {
+  static constexpr int kStagesPerBox = SP ? 8 : 4;                 // 128 code bytes per row per box
+  static constexpr int kBoxK = kMtBK * kStagesPerBox;              // logical K per box
+  static constexpr uint32_t kMetaBox = SP ? kMtRows * 64 : 0;      // 128 rows x 64 nibble bytes
+  static constexpr uint32_t kBox = kMtCodeBox + kMtScaleBox + kMetaBox;
+  static constexpr int kBoxes = SP ? 2 : 3;                        // 16 / 12 stages in flight
+  static constexpr uint32_t kACols = SP ? 16 : 32;                 // A columns per stage
+  static constexpr uint32_t kMetaCol0 = kMtAccCols + kMtSlots * kACols;  // 2 metadata columns per slot
+  static constexpr size_t kSmem = (size_t)kBoxes * kBox + (size_t)kMtSlots * kMtX + 1024;
+  static_assert(kMetaCol0 + (SP ? 2 * kMtSlots : 0) <= kMtCols, "tensor memory");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kBox % 1024 == 0, "swizzled boxes stay 1024-byte aligned");
+};
 
 // 16-byte copy that reads `src_bytes` (16 or 0) and zero-fills the rest.
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uint32_t src_bytes) {
@@ -72,6 +90,31 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uin
 __device__ __forceinline__ uint32_t sw128(int r, int j) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
 }
+
+// Sparse (2:4) MMA, kind::f16, with A (the kept values) in tensor memory.
+__device__ __forceinline__ void umma_f16_sp_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                   uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], [%1], %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Stores 16 / 2 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st2_nowait(uint32_t taddr, uint32_t r0, uint32_t r1) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(r0), "r"(r1) : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct MoeTcParams {
   const uint16_t* x;     // [T, K] 16-bit tokens
@@ -104,18 +147,22 @@ __device__ __forceinline__ void e2m1x8_to_16(uint32_t w, uint32_t* h) {
   }
 }
 
-// The four block-scale multipliers of one stage (E4M3 codes in the bytes of `sw`), each in both
-// halves of a word: E4M3 (f16: the products stay exact, at most 6 significant bits between
-// 2^-10 and 2688) or E4M3 * 2^104 (bf16: with the codes at E2M1 * 2^-112 every product is
-// E2M1 * E4M3 * 2^-8, a normal bf16).
-template <typename T>
-__device__ __forceinline__ void block_scales4(uint32_t sw, uint32_t (&m)[4]) {
-  uint32_t lo, hi;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"((uint16_t)(sw & 0xffffu)));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"((uint16_t)(sw >> 16)));
-  const uint32_t h[4] = {lo & 0xffffu, lo >> 16, hi & 0xffffu, hi >> 16};
+// The NS (2 or 4) block-scale multipliers of one stage (E4M3 codes in the low bytes of `sw`),
+// each in both halves of a word: E4M3 (f16: the products stay exact, at most 6 significant bits
+// between 2^-10 and 2688) or E4M3 * 2^104 (bf16: with the codes at E2M1 * 2^-112 every product
+// is E2M1 * E4M3 * 2^-8, a normal bf16).
+template <typename T, int NS>
+__device__ __forceinline__ void block_scales(uint32_t sw, uint32_t (&m)[NS]) {
+  uint32_t h[4];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
+  for (int q = 0; q < NS / 2; ++q) {
+    uint32_t w;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(w) : "h"((uint16_t)(sw >> (16 * q))));
+    h[2 * q] = w & 0xffffu;
+    h[2 * q + 1] = w >> 16;
+  }
+#pragma unroll
+  for (int b = 0; b < NS; ++b) {
     uint32_t v = h[b];
     if constexpr (std::is_same<T, __nv_bfloat16>::value)
       v = to_bits16<T>(__half2float(__ushort_as_half((unsigned short)v)) * 0x1p104f);
@@ -124,25 +171,26 @@ __device__ __forceinline__ void block_scales4(uint32_t sw, uint32_t (&m)[4]) {
 }
 
 // The factor that takes an accumulated product back to x . w: 2^8 for bf16 operands (see
-// block_scales4), 1 for f16, times the experts' tensor scale.
+// block_scales), 1 for f16, times the experts' tensor scale.
 template <typename T>
 constexpr float kMtUnscale = std::is_same<T, __nv_bfloat16>::value ? 256.0f : 1.0f;
 
 // One CTA: token tile blockIdx.y (expert e, rows first .. first + count of the permutation) x
 // weight rows 128 * blockIdx.x .. + 127 of expert e, over all of K.
-template <typename T>
+template <typename T, bool SP>
 __global__ void __launch_bounds__(kMtThreads, 1)
     moe_w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
-                        const MoeTcParams p) {
+                        const __grid_constant__ CUtensorMap tmE, const MoeTcParams p) {
+  using G = MtGeom<SP>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sW = smem;                           // [kMtBoxes][codes 128 x 128 B swizzled | scales 128 x 16 B]
-  uint8_t* sX = smem + kMtBoxes * kMtBox;       // [kMtSlots][128 rows x 128 B swizzled]
+  uint8_t* sW = smem;                        // [kBoxes][codes 128 x 128 B swizzled | scales 128 x 16 B | meta 128 x 64 B]
+  uint8_t* sX = smem + G::kBoxes * G::kBox;  // [kMtSlots][128 rows x 128 B swizzled]
   // Slots are synchronised in pairs (2q, 2q + 1), so the MMA thread waits and commits once per
   // two stages.  st_full[q]: both stages have their A (4 converter warps each) and their x (8
-  // gather warps each); st_empty[q]: the MMAs that read the pair have completed (commit).
-  __shared__ uint64_t w_full[kMtBoxes], w_empty[kMtBoxes], st_full[kMtPairs], st_empty[kMtPairs], tfull_bar;
+  // gather warps, once for the pair); st_empty[q]: the MMAs that read the pair have completed.
+  __shared__ uint64_t w_full[G::kBoxes], w_empty[G::kBoxes], st_full[kMtPairs], st_empty[kMtPairs], tfull_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int aborted;
   __shared__ int32_t s_perm[kMtTok];
@@ -154,11 +202,11 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   const int n_mma = (count + 15) & ~15;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = e * p.N + (int)blockIdx.x * kMtRows;  // stacked weight row (< 2^31)
-  const int KB = p.K / kMtBK;                           // stages (a multiple of 4)
+  const int KB = p.K / kMtBK;                           // stages (a multiple of kStagesPerBox)
 
   if (tid < count) s_perm[tid] = p.perm[first + tid];
   if (tid == 0) {
-    for (int s = 0; s < kMtBoxes; ++s) {
+    for (int s = 0; s < G::kBoxes; ++s) {
       mbar_init(&w_full[s], 1);
       mbar_init(&w_empty[s], kMtConvWarps);
     }
@@ -182,29 +230,65 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     const int g = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qd) << 16;
     const uint32_t a_base = tmem + t_lane + kMtAccCols;
+    const uint32_t e_base = tmem + t_lane + G::kMetaCol0;
+    // metadata regrouping: this lane's TMEM lane carries rows m (lane msrc) and m + 8 (msrc + 8)
+    // of the warp, bytes 2h, 2h + 1 of each 32-wide window
+    const int msrc = 16 * (lane >> 4) + (lane & 7);
+    const uint32_t msel = ((lane >> 3) & 1) ? 0x7632u : 0x5410u;
 #pragma unroll 1
-    for (int i = g, m = 0; i < KB; i += kMtGroups, ++m) {  // stage i = 4m + g: stage g of box m
-      const int bs = m % kMtBoxes;
-      if (!__all_sync(0xffffffffu, mbar_wait(&w_full[bs], (m / kMtBoxes) & 1) && !*(volatile int*)&aborted)) {
+    for (int i = g; i < KB; i += kMtGroups) {
+      const int m = i / G::kStagesPerBox, st = i % G::kStagesPerBox, bs = m % G::kBoxes;
+      if (!__all_sync(0xffffffffu, mbar_wait(&w_full[bs], (m / G::kBoxes) & 1) && !*(volatile int*)&aborted)) {
         aborted = 1;
         break;
       }
-      const uint8_t* box = sW + bs * kMtBox;
-      // this stage's 32 code bytes of row r: 16-byte chunks 2g, 2g + 1 of the swizzled row
-      const uint4 c0 = *reinterpret_cast<const uint4*>(box + r * 128 + (((2 * g) ^ (r & 7)) << 4));
-      const uint4 c1 = *reinterpret_cast<const uint4*>(box + r * 128 + (((2 * g + 1) ^ (r & 7)) << 4));
-      const uint32_t sw = *reinterpret_cast<const uint32_t*>(box + kMtCodeBox + r * 16 + 4 * g);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&w_empty[bs]);  // the warp's raw bytes of this box are in registers
-      uint32_t sc[4];
-      block_scales4<T>(sw, sc);
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      uint32_t a[32];  // column j = K elements 2j, 2j + 1 of the stage
+      const uint8_t* box = sW + bs * G::kBox;
+      uint32_t a[G::kACols];  // column j = stored values 2j, 2j + 1 of the stage
+      uint32_t ecol[2] = {0u, 0u};
+      if constexpr (!SP) {
+        // this stage's 32 code bytes of row r: 16-byte chunks 2st, 2st + 1 of the swizzled row
+        const uint4 c0 = *reinterpret_cast<const uint4*>(box + r * 128 + (((2 * st) ^ (r & 7)) << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(box + r * 128 + (((2 * st + 1) ^ (r & 7)) << 4));
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(box + kMtCodeBox + r * 16 + 4 * st);
+        if (st + kMtGroups >= G::kStagesPerBox) {  // this group's last stage of the box
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&w_empty[bs]);
+        }
+        uint32_t sc[4];
+        block_scales<T, 4>(sw, sc);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int wi = 0; wi < 8; ++wi) {
-        e2m1x8_to_16<T>(words[wi], &a[4 * wi]);
+        for (int wi = 0; wi < 8; ++wi) {
+          e2m1x8_to_16<T>(words[wi], &a[4 * wi]);
 #pragma unroll
-        for (int pq = 0; pq < 4; ++pq) a[4 * wi + pq] = hmul2u<T>(a[4 * wi + pq], sc[wi >> 1]);
+          for (int pq = 0; pq < 4; ++pq) a[4 * wi + pq] = hmul2u<T>(a[4 * wi + pq], sc[wi >> 1]);
+        }
+      } else {
+        // 32 kept values (16 code bytes: chunk st of the swizzled row), 2 block scales, 8 bytes
+        // of metadata (two 32-wide windows of 4 bytes) of row r
+        const uint4 c = *reinterpret_cast<const uint4*>(box + r * 128 + ((st ^ (r & 7)) << 4));
+        const uint32_t sw = *reinterpret_cast<const uint16_t*>(box + kMtCodeBox + r * 16 + 2 * st);
+        const uint2 mw = *reinterpret_cast<const uint2*>(box + kMtCodeBox + kMtScaleBox + r * 64 + 8 * st);
+        if (st + kMtGroups >= G::kStagesPerBox) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&w_empty[bs]);
+        }
+        uint32_t sc[2];
+        block_scales<T, 2>(sw, sc);
+        const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          e2m1x8_to_16<T>(words[wi], &a[4 * wi]);
+#pragma unroll
+          for (int pq = 0; pq < 4; ++pq) a[4 * wi + pq] = hmul2u<T>(a[4 * wi + pq], sc[wi >> 1]);
+        }
+        const uint32_t mwin[2] = {mw.x, mw.y};
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t lo = __shfl_sync(0xffffffffu, mwin[t], msrc);
+          const uint32_t hi = __shfl_sync(0xffffffffu, mwin[t], msrc + 8);
+          ecol[t] = __byte_perm(lo, hi, msel);
+        }
       }
       const int as = i % kMtSlots;
       if (i >= kMtSlots &&
@@ -213,7 +297,13 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         break;
       }
       tc_fence_after();
-      tmem_st32(a_base + kMtACols * as, a);
+      if constexpr (!SP) {
+        tmem_st32(a_base + G::kACols * as, a);
+      } else {
+        tmem_st16_nowait(a_base + G::kACols * as, a);
+        tmem_st2_nowait(e_base + 2 * as, ecol[0], ecol[1]);
+        tmem_wait_st();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&st_full[as >> 1]);
@@ -240,12 +330,11 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     }
   } else if (warp == kMtWarpMma) {
     if (lane == 0) {
-      // ---- MMA issuer: four K = 16 steps per stage, A from TMEM slot i % 8, B from x slot i % 8.
-      // The next stage's barrier is tested (without waiting) before this stage's MMAs are
-      // issued, so the test's latency overlaps them.
-      const uint32_t idesc = idesc_f16(kMtRows, n_mma, kBf16);
+      // ---- MMA issuer.  The next pair's barrier is tested (without waiting) before this
+      // pair's MMAs are issued, so the test's latency overlaps them.
+      const uint32_t idesc = idesc_f16(kMtRows, n_mma, kBf16, SP);
       const uint64_t b_first = desc_kmajor_sw128(smem_u32(sX));
-      const int KP = KB / 2;  // stage pairs (KB is a multiple of 4)
+      const int KP = KB / 2;  // stage pairs
       bool ready = mbar_wait(&st_full[0], 0);
 #pragma unroll 1
       for (int pr = 0; pr < KP; ++pr) {
@@ -261,10 +350,19 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         for (int h = 0; h < 2; ++h) {
           const int s = 2 * q + h;
           const uint64_t b0 = b_first + (uint64_t)(s * (kMtX >> 4));  // descriptor address: 16-byte units
-          const uint32_t a0 = tmem + kMtAccCols + kMtACols * s;
+          const uint32_t a0 = tmem + kMtAccCols + G::kACols * s;
+          if constexpr (!SP) {
 #pragma unroll
-          for (int k = 0; k < kMtBK / 16; ++k)
-            umma_f16_tmem_a(tmem, a0 + 8 * k, b0 + 2 * k, idesc, (pr | h | k) != 0);
+            for (int k = 0; k < kMtBK / 16; ++k)  // K = 16: 8 A columns, 32 bytes of B
+              umma_f16_tmem_a(tmem, a0 + 8 * k, b0 + 2 * k, idesc, (pr | h | k) != 0);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // K = 32 logical: 8 A columns, 64 bytes of B, one metadata column
+              // an odd metadata column is named by the even one below it plus the sparse-id2 field
+              const uint32_t ecl = tmem + G::kMetaCol0 + 2 * s + t;
+              umma_f16_sp_tmem_a(tmem, a0 + 8 * t, b0 + 4 * t, ecl & ~1u, idesc | (ecl & 1u), (pr | h | t) != 0);
+            }
+          }
         }
         umma_commit(&st_empty[q]);
         ready = pr + 1 >= KP || next || mbar_wait(&st_full[qn], pn);
@@ -273,23 +371,25 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     }
   } else if (warp == kMtWarpW) {
     if (lane == 0) {
-      // ---- weight boxes: codes and block scales of four stages per copy pair
+      // ---- weight boxes: codes, block scales (and metadata) of kStagesPerBox stages per copy set
       int issued = 0;
 #pragma unroll 1
-      for (int m = 0; m < KB / 4; ++m) {
-        const int s = m % kMtBoxes;
-        if (!mbar_wait(&w_empty[s], ((m / kMtBoxes) & 1) ^ 1) || *(volatile int*)&aborted) {
+      for (int m = 0; m < KB / G::kStagesPerBox; ++m) {
+        const int s = m % G::kBoxes;
+        if (!mbar_wait(&w_empty[s], ((m / G::kBoxes) & 1) ^ 1) || *(volatile int*)&aborted) {
           aborted = 1;
           break;
         }
-        mbar_arrive_expect_tx(&w_full[s], kMtBox);
-        tma_load_2d(sW + s * kMtBox, &tmC, &w_full[s], m * (kMtBoxK / 2), row0);
-        tma_load_2d(sW + s * kMtBox + kMtCodeBox, &tmS, &w_full[s], m * (kMtBoxK / 16), row0);
+        uint8_t* box = sW + s * G::kBox;
+        mbar_arrive_expect_tx(&w_full[s], G::kBox);
+        tma_load_2d(box, &tmC, &w_full[s], m * 128, row0);
+        tma_load_2d(box + kMtCodeBox, &tmS, &w_full[s], m * 16, row0);
+        if constexpr (SP) tma_load_2d(box + kMtCodeBox + kMtScaleBox, &tmE, &w_full[s], m * 64, row0);
         ++issued;
       }
       // no copy may still be landing in shared memory when the CTA exits
-      for (int m = issued - kMtBoxes > 0 ? issued - kMtBoxes : 0; m < issued; ++m)
-        mbar_wait(&w_full[m % kMtBoxes], (m / kMtBoxes) & 1);
+      for (int m = issued - G::kBoxes > 0 ? issued - G::kBoxes : 0; m < issued; ++m)
+        mbar_wait(&w_full[m % G::kBoxes], (m / G::kBoxes) & 1);
     }
   } else {
     // ---- token rows: gather thread t copies 16-byte chunk t % 8 of routed rows t / 8 + 32u
@@ -351,28 +451,33 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   }
 }
 
-template <typename T>
-int launch_moe_tc(const CUtensorMap& tmC, const CUtensorMap& tmS, const MoeTcParams& p, int64_t n_tiles,
-                  cudaStream_t s) {
-  auto kern = moe_w4a16_tc_kernel<T>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMtSmem) != cudaSuccess)
+template <typename T, bool SP>
+int launch_moe_tc(const CUtensorMap& tmC, const CUtensorMap& tmS, const CUtensorMap& tmE, const MoeTcParams& p,
+                  int64_t n_tiles, cudaStream_t s) {
+  auto kern = moe_w4a16_tc_kernel<T, SP>;
+  const size_t smem = MtGeom<SP>::kSmem;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   dim3 grid((unsigned)(p.N / kMtRows), (unsigned)n_tiles);
-  kern<<<grid, kMtThreads, kMtSmem, s>>>(tmC, tmS, p);
+  kern<<<grid, kMtThreads, smem, s>>>(tmC, tmS, tmE, p);
   return launch_status();
 }
 
 }  // namespace
 
 bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_t K, int64_t max_tiles,
-                      const void* codes, const void* scales, const void* x) {
-  return wf == W_DQ4 && x_fmt == X_16 && T > 0 && T < INT32_MAX && N > 0 && N % kMtRows == 0 &&
-         N / kMtRows <= 65535 && K > 0 && K % kMtBoxK == 0 && K <= INT32_MAX / 2 && E * N <= INT32_MAX &&
-         max_tiles <= 65535 && aligned(codes, 16) && aligned(scales, 16) && aligned(x, 16);
+                      const void* codes, const void* scales, const void* meta, const void* x) {
+  const bool sp = wf == W_SQ4;
+  if (!(wf == W_DQ4 || sp) || x_fmt != X_16) return false;
+  const int64_t box_k = sp ? MtGeom<true>::kBoxK : MtGeom<false>::kBoxK;
+  return T > 0 && T < INT32_MAX && N > 0 && N % kMtRows == 0 && N / kMtRows <= 65535 && K > 0 &&
+         K % box_k == 0 && K <= INT32_MAX / 2 && E * N <= INT32_MAX && max_tiles <= 65535 && aligned(codes, 16) &&
+         aligned(scales, 16) && (!sp || aligned(meta, 16)) && aligned(x, 16);
 }
 
-int moe_tc_grouped(int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s) {
+int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s) {
   if (n_tiles <= 0) return SP24_OK;
+  const bool sparse = wf == W_SQ4;
   MoeTcParams p{};
   p.x = reinterpret_cast<const uint16_t*>(sp.x);
   p.w_ts = sp.w_ts;
@@ -384,12 +489,19 @@ int moe_tc_grouped(int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_
   p.N = (int)sp.N;
   p.K = (int)sp.K;
   const uint64_t rows = (uint64_t)(E * sp.N), K = (uint64_t)sp.K;
-  CUtensorMap tmC, tmS;
-  int st = make_tmap_2d(&tmC, sp.w, 1, rows, K / 2, K / 2, kMtBoxK / 2, kMtRows);  // codes, 128-byte swizzle
-  if (!st) st = make_tmap_2d_plain(&tmS, sp.w_scales, rows, K / 16, K / 16, kMtBoxK / 16, kMtRows);
+  // per row: codes K/2 (dense) or K/4 (2:4) bytes, scales K/16 or K/32, metadata K/8 (2:4)
+  const uint64_t cb = sparse ? K / 4 : K / 2, sb = sparse ? K / 32 : K / 16;
+  CUtensorMap tmC, tmS, tmE;
+  int st = make_tmap_2d(&tmC, sp.w, 1, rows, cb, cb, 128, kMtRows);  // 128-byte swizzle
+  if (!st) st = make_tmap_2d_plain(&tmS, sp.w_scales, rows, sb, sb, 16, kMtRows);
+  if (!st) st = sparse ? make_tmap_2d_plain(&tmE, sp.meta, rows, K / 8, K / 8, 64, kMtRows) : SP24_OK;
   if (st) return st;
-  return t16 == SP24_F16 ? launch_moe_tc<__half>(tmC, tmS, p, n_tiles, s)
-                         : launch_moe_tc<__nv_bfloat16>(tmC, tmS, p, n_tiles, s);
+  if (!sparse) tmE = tmS;  // unused
+  if (sparse)
+    return t16 == SP24_F16 ? launch_moe_tc<__half, true>(tmC, tmS, tmE, p, n_tiles, s)
+                           : launch_moe_tc<__nv_bfloat16, true>(tmC, tmS, tmE, p, n_tiles, s);
+  return t16 == SP24_F16 ? launch_moe_tc<__half, false>(tmC, tmS, tmE, p, n_tiles, s)
+                         : launch_moe_tc<__nv_bfloat16, false>(tmC, tmS, tmE, p, n_tiles, s);
 }
 
 }  // namespace sp24

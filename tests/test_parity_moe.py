@@ -146,3 +146,15 @@ def test_moe_bad_expert_ids_tensor_core_path():
     assert sp.last_device_error() == sp.ERR_INVALID_ARG
     assert not y[0, 1].any() and not y[5, 0].any()
     assert torch.isfinite(y).all()
+
+
+@pytest.mark.parametrize("xfmt", ["bf16", "f16"])
+@pytest.mark.parametrize("NK", [(256, 512), (128, 1024), (384, 2560)], ids=lambda s: f"N{s[0]}-K{s[1]}")
+def test_moe_tile_boundaries_sparse24(NK, xfmt):
+    """2:4-compressed NVFP4 experts on the tensor-core path (tcgen05.mma.sp, metadata regrouped
+    in registers): the same skewed routings, K of 1, 2 and 5 weight boxes of 512 (the last
+    wraps the two-box ring twice), every output checked."""
+    N, K = NK
+    d = synth.moe_skewed(SKEW, seed=21, N=N, K=K, topk=2, xdtype=xfmt)
+    T = d["X"].shape[0]
+    _run(d["X"], d["W"], d["routing"], xfmt, "nvfp4", True, np.arange(T))
