@@ -123,7 +123,9 @@ int skinny2_grouped(int wf, int t16, SkinnyParams p, int64_t max_tiles, cudaStre
 // tcgen05.mma (.sp for 2:4) into TMEM.
 bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_t K, int64_t max_tiles,
                       const void* codes, const void* scales, const void* meta, const void* x);
-int moe_tc_grouped(int wf, int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s);
+// n_tiles bounds the tile table; *n_valid (device) is the number of used tiles, which come first.
+int moe_tc_grouped(int wf, int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles,
+                   const int32_t* n_valid, cudaStream_t s);
 
 // Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,

@@ -37,7 +37,7 @@ __global__ void route_count(const int32_t* __restrict__ routing, int64_t n, int6
 // Single CTA of 1024 threads: block-wide exclusive scans over E experts in chunks of 1024.
 __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ counts, int64_t E,
                                                    int32_t* __restrict__ offsets, int32_t* __restrict__ tiles,
-                                                   int64_t max_tiles, int tile) {
+                                                   int64_t max_tiles, int tile, int32_t* __restrict__ n_tiles) {
   __shared__ int32_t warp_sum[2][32];
   __shared__ int32_t carry[2];
   if (threadIdx.x == 0) carry[0] = carry[1] = 0;
@@ -94,8 +94,9 @@ __global__ void __launch_bounds__(1024) route_scan(const int32_t* __restrict__ c
     }
     __syncthreads();
   }
-  // unused tile slots get count 0 (those CTAs exit at once)
+  // unused tile slots get count 0 (those CTAs exit at once); the used ones come first
   for (int64_t i = carry[1] + threadIdx.x; i < max_tiles; i += blockDim.x) tiles[3 * i + 2] = 0;
+  if (threadIdx.x == 0) *n_tiles = carry[1] < max_tiles ? carry[1] : (int32_t)max_tiles;
 }
 
 // Also zeroes the outputs of routed rows with an invalid expert id when `y_zero` is set (the
@@ -115,7 +116,7 @@ __global__ void route_scatter(const int32_t* __restrict__ routing, int64_t n, in
 }
 
 struct MoeWs {
-  int32_t *counts, *fill, *offsets, *tiles, *perm;
+  int32_t *counts, *fill, *offsets, *n_tiles, *tiles, *perm;
   int64_t max_tiles, bytes;
 };
 
@@ -132,6 +133,8 @@ MoeWs moe_layout(void* base, int64_t T, int topk, int64_t E) {
   off += r16(4 * E);
   w.offsets = reinterpret_cast<int32_t*>(p + off);
   off += r16(4 * E);
+  w.n_tiles = reinterpret_cast<int32_t*>(p + off);
+  off += 16;
   w.tiles = reinterpret_cast<int32_t*>(p + off);
   off += r16(12 * w.max_tiles);
   w.perm = reinterpret_cast<int32_t*>(p + off);
@@ -241,7 +244,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   // tiles of `tile` rows: at most sum_e ceil(c_e / tile) <= n / tile + E of them
   const int64_t n_tiles = n / tile + E < ws.max_tiles ? n / tile + E : ws.max_tiles;
   route_count<<<blocks, 256, 0, s>>>(routing, n, E, ws.counts);
-  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles, tile);
+  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles, tile, ws.n_tiles);
   route_scatter<<<blocks, 256, 0, s>>>(routing, n, E, ws.offsets, ws.fill, ws.perm, tc ? y : nullptr, N);
   int st = launch_status(3);
   if (st) return st;
@@ -249,6 +252,6 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   p.tiles = ws.tiles;
   p.topk = topk;
   p.expert_rows = N;
-  if (tc) return moe_tc_grouped(wf, t16, p, E, T, n_tiles, s);
+  if (tc) return moe_tc_grouped(wf, t16, p, E, T, n_tiles, ws.n_tiles, s);
   return skinny2_grouped(wf, t16, p, n_tiles, s);
 }

@@ -8,8 +8,10 @@
 // [P2] "The mechanism needs both values and their positions": for 2:4 experts the kept values
 // are the MMA's A operand and their positions travel as tcgen05 sparse metadata.
 //
-// Roles (K advances in stages of 64 logical elements; stage i uses slot i % 10 of an x ring in
-// shared memory and of an A ring in tensor memory; slots are synchronised in pairs):
+// The kernel is persistent: each CTA (one per SM) walks a list of items (token tile x 128-row
+// block) and every ring below runs across them.  Roles (K advances in stages of 64 logical
+// elements; stage i of the CTA's sequence uses slot i % 8 (dense) or i % 10 (2:4) of an x ring
+// in shared memory and of an A ring in tensor memory; slots are synchronised in pairs):
 //   * TMA warp W loads the raw weights of 4 (dense) or 8 (2:4) stages at a time: the 128 rows'
 //     code bytes (128-byte rows, 128-byte swizzle), their E4M3 block scales (16-byte rows) and,
 //     for 2:4, their metadata nibbles (64-byte rows);
@@ -33,8 +35,9 @@
 //     any N up to 128, so at ~80 routed rows the instruction count sets the pace and the 2:4
 //     form needs half as many: one barrier per stage pair, tested for the next pair before the
 //     current pair's MMAs are issued;
-//   * after the last stage the converter warps read the accumulator (lane = weight row, column
-//     = routed row) and store y[token, slot, row] * unscale * tensor scale once.
+//   * four epilogue warps read a finished item's accumulator (lane = weight row, column = routed
+//     row) and store y[token, slot, row] * unscale * tensor scale once, while the MMAs fill the
+//     other of two accumulators with the next item.
 // Every wait is bounded; on a timeout the CTA records SP24_ERR_DEVICE_TIMEOUT, lets its copies
 // land, frees its TMEM and returns.
 #include "sp24_fp4.cuh"
@@ -49,16 +52,16 @@ using namespace tc;
 constexpr int kMtRows = 128;      // weight rows per CTA (MMA M)
 constexpr int kMtTok = 128;       // routed rows per token tile (MMA N <= 128)
 constexpr int kMtBK = 64;         // logical K per stage
-constexpr int kMtSlots = 10;      // stage slots: x tile in shared memory + A slot in TMEM (i % 10)
-constexpr int kMtPairs = kMtSlots / 2;
-constexpr int kMtDp = kMtPairs - 2;  // x is copied three stage pairs ahead (the slot pair's MMAs, two pairs back, are done)
 constexpr int kMtGroups = 4;      // converter groups
 constexpr int kMtConvWarps = 4 * kMtGroups;
 constexpr int kMtGatherWarps = 8;
+constexpr int kMtEpiWarps = 4;
 constexpr int kMtWarpMma = kMtConvWarps, kMtWarpW = kMtConvWarps + 1, kMtWarpX0 = kMtConvWarps + 2;
-constexpr int kMtThreads = 32 * (kMtWarpX0 + kMtGatherWarps);
+constexpr int kMtWarpEpi0 = kMtWarpX0 + kMtGatherWarps;
+constexpr int kMtThreads = 32 * (kMtWarpEpi0 + kMtEpiWarps);
+constexpr int kMtMaxItems = 64;   // items per CTA (the host sizes the grid for it)
 constexpr uint32_t kMtX = kMtTok * kMtBK * 2;              // 16 KB
-constexpr uint32_t kMtAccCols = 128;                       // fp32 accumulator, one column per routed row
+constexpr uint32_t kMtAccCols = 128;                       // fp32 accumulator, one column per routed row (two of them)
 constexpr uint32_t kMtCols = 512;
 constexpr uint32_t kMtCodeBox = kMtRows * 128;             // 16 KB: 128 rows x 128 code bytes
 constexpr uint32_t kMtScaleBox = kMtRows * 16;             // 2 KB: 128 rows x 16 scale bytes
@@ -71,10 +74,13 @@ struct MtGeom {
   static constexpr uint32_t kMetaBox = SP ? kMtRows * 64 : 0;      // 128 rows x 64 nibble bytes
   static constexpr uint32_t kBox = kMtCodeBox + kMtScaleBox + kMetaBox;
   static constexpr int kBoxes = SP ? 2 : 3;                        // 16 / 12 stages in flight
+  static constexpr int kSlots = SP ? 10 : 8;                       // stage slots: x tile + A slot (i % kSlots)
   static constexpr uint32_t kACols = SP ? 16 : 32;                 // A columns per stage
-  static constexpr uint32_t kMetaCol0 = kMtAccCols + kMtSlots * kACols;  // 2 metadata columns per slot
-  static constexpr size_t kSmem = (size_t)kBoxes * kBox + (size_t)kMtSlots * kMtX + 1024;
-  static_assert(kMetaCol0 + (SP ? 2 * kMtSlots : 0) <= kMtCols, "tensor memory");
+  static constexpr uint32_t kACol0 = 2 * kMtAccCols;               // after the two accumulators
+  static constexpr uint32_t kMetaCol0 = kACol0 + kSlots * kACols;  // 2 metadata columns per slot
+  static constexpr size_t kSmem = (size_t)kBoxes * kBox + (size_t)kSlots * kMtX + 1024;
+  static_assert(kSlots % 2 == 0 && kSlots >= 6, "slot pairs, copies two pairs behind the MMAs");
+  static_assert(kMetaCol0 + (SP ? 2 * kSlots : 0) <= kMtCols, "tensor memory");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kBox % 1024 == 0, "swizzled boxes stay 1024-byte aligned");
 };
@@ -121,6 +127,7 @@ struct MoeTcParams {
   const float* w_ts;     // tensor scale of the stacked experts
   const int32_t* tiles;  // (expert, first permutation index, count) per token tile
   const int32_t* perm;   // flat (token * topk + slot) of each routed row, grouped by expert
+  const int32_t* n_valid;  // number of used tiles (they come first in the table)
   float* y;              // [T, topk, N]
   int topk;
   int T;
@@ -175,46 +182,60 @@ __device__ __forceinline__ void block_scales(uint32_t sw, uint32_t (&m)[NS]) {
 template <typename T>
 constexpr float kMtUnscale = std::is_same<T, __nv_bfloat16>::value ? 256.0f : 1.0f;
 
-// One CTA: token tile blockIdx.y (expert e, rows first .. first + count of the permutation) x
-// weight rows 128 * blockIdx.x .. + 127 of expert e, over all of K.
+// Persistent: CTA c takes the items c, c + gridDim.x, ... (item = token tile t x row block rb,
+// numbered t * (N / 128) + rb; the used tiles come first) and runs every ring across them, so
+// the next item's copies and conversions overlap this item's MMAs; two TMEM accumulators let the
+// epilogue warps drain one item while the MMAs fill the next.
 template <typename T, bool SP>
 __global__ void __launch_bounds__(kMtThreads, 1)
     moe_w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
                         const __grid_constant__ CUtensorMap tmE, const MoeTcParams p) {
   using G = MtGeom<SP>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int kSlots = G::kSlots, kPairs = kSlots / 2, kDp = kPairs - 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem;                        // [kBoxes][codes 128 x 128 B swizzled | scales 128 x 16 B | meta 128 x 64 B]
-  uint8_t* sX = smem + G::kBoxes * G::kBox;  // [kMtSlots][128 rows x 128 B swizzled]
+  uint8_t* sX = smem + G::kBoxes * G::kBox;  // [kSlots][128 rows x 128 B swizzled]
   // Slots are synchronised in pairs (2q, 2q + 1), so the MMA thread waits and commits once per
   // two stages.  st_full[q]: both stages have their A (4 converter warps each) and their x (8
   // gather warps, once for the pair); st_empty[q]: the MMAs that read the pair have completed.
-  __shared__ uint64_t w_full[G::kBoxes], w_empty[G::kBoxes], st_full[kMtPairs], st_empty[kMtPairs], tfull_bar;
+  // t_full[a]: accumulator a holds a finished item; t_empty[a]: the epilogue has read it.
+  __shared__ uint64_t w_full[G::kBoxes], w_empty[G::kBoxes], st_full[kPairs], st_empty[kPairs];
+  __shared__ uint64_t t_full[2], t_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int aborted;
-  __shared__ int32_t s_perm[kMtTok];
+  __shared__ int32_t s_item[kMtMaxItems][3];  // expert, first permutation index, count
 
-  const int32_t* tile = p.tiles + 3 * (int64_t)blockIdx.y;
-  const int count = tile[2];
-  if (count <= 0) return;  // unused tile slot: the whole CTA leaves before any shared state
-  const int e = tile[0], first = tile[1];
-  const int n_mma = (count + 15) & ~15;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = e * p.N + (int)blockIdx.x * kMtRows;  // stacked weight row (< 2^31)
-  const int KB = p.K / kMtBK;                           // stages (a multiple of kStagesPerBox)
+  const int RB = p.N / kMtRows;
+  const int n_items = *p.n_valid * RB;
+  int nj = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  nj = nj < kMtMaxItems ? nj : kMtMaxItems;  // the host sizes the grid so that this never cuts
+  if (nj == 0) return;  // the whole CTA leaves before any shared state
+  const int KB = p.K / kMtBK;  // stages per item (a multiple of kStagesPerBox)
+  const int KP = KB / 2;
+  auto item_id = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
 
-  if (tid < count) s_perm[tid] = p.perm[first + tid];
+  for (int j = tid; j < nj; j += blockDim.x) {
+    const int32_t* t = p.tiles + 3 * (int64_t)(item_id(j) / RB);
+    s_item[j][0] = t[0];
+    s_item[j][1] = t[1];
+    s_item[j][2] = t[2];
+  }
   if (tid == 0) {
     for (int s = 0; s < G::kBoxes; ++s) {
       mbar_init(&w_full[s], 1);
       mbar_init(&w_empty[s], kMtConvWarps);
     }
-    for (int q = 0; q < kMtPairs; ++q) {
+    for (int q = 0; q < kPairs; ++q) {
       mbar_init(&st_full[q], 2 * 4 + kMtGatherWarps);  // two converter groups, the gather warps once
       mbar_init(&st_empty[q], 1);
     }
-    mbar_init(&tfull_bar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&t_full[a], 1);
+      mbar_init(&t_empty[a], kMtEpiWarps);
+    }
     aborted = 0;
     fence_mbar_init();
   }
@@ -225,18 +246,20 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   const uint32_t tmem = tmem_base;
 
   if (warp < kMtConvWarps) {
-    // ---- converters: group g = warp / 4 expands stages g, g + 4, ...; thread = weight row r
-    // (lane quarter warp % 4, the TMEM lanes this warp may access).
+    // ---- converters: group g = warp / 4 expands stages g, g + 4, ... of the CTA's stage
+    // sequence (all its items, back to back); thread = weight row r (lane quarter warp % 4, the
+    // TMEM lanes this warp may access).
     const int g = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qd) << 16;
-    const uint32_t a_base = tmem + t_lane + kMtAccCols;
+    const uint32_t a_base = tmem + t_lane + G::kACol0;
     const uint32_t e_base = tmem + t_lane + G::kMetaCol0;
     // metadata regrouping: this lane's TMEM lane carries rows m (lane msrc) and m + 8 (msrc + 8)
     // of the warp, bytes 2h, 2h + 1 of each 32-wide window
     const int msrc = 16 * (lane >> 4) + (lane & 7);
     const uint32_t msel = ((lane >> 3) & 1) ? 0x7632u : 0x5410u;
+    const int n_stages = nj * KB;
 #pragma unroll 1
-    for (int i = g; i < KB; i += kMtGroups) {
+    for (int i = g; i < n_stages; i += kMtGroups) {
       const int m = i / G::kStagesPerBox, st = i % G::kStagesPerBox, bs = m % G::kBoxes;
       if (!__all_sync(0xffffffffu, mbar_wait(&w_full[bs], (m / G::kBoxes) & 1) && !*(volatile int*)&aborted)) {
         aborted = 1;
@@ -290,9 +313,9 @@ __global__ void __launch_bounds__(kMtThreads, 1)
           ecol[t] = __byte_perm(lo, hi, msel);
         }
       }
-      const int as = i % kMtSlots;
-      if (i >= kMtSlots &&
-          !__all_sync(0xffffffffu, mbar_wait(&st_empty[as >> 1], ((i / kMtSlots) - 1) & 1))) {  // MMA i - 10 done
+      const int as = i % kSlots;
+      if (i >= kSlots &&
+          !__all_sync(0xffffffffu, mbar_wait(&st_empty[as >> 1], ((i / kSlots) - 1) & 1))) {  // MMA i - kSlots done
         aborted = 1;
         break;
       }
@@ -309,134 +332,181 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       if (lane == 0) mbar_arrive(&st_full[as >> 1]);
     }
 
-    // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (weight rows) and accumulator
-    // columns 32 (w / 4) .. + 31 (routed rows), storing each routed row's 32 outputs at once.
-    if (__all_sync(0xffffffffu, mbar_wait(&tfull_bar, 0))) {
+  }
+  else if (warp == kMtWarpMma) {
+    if (lane == 0) {
+      // ---- MMA issuer over the CTA's stage pairs.  Little scalar work per pair (this thread
+      // shares the SM with thirty busy warps, and the tensor pipe idles while it computes): the
+      // pair loop is unrolled over the slot pairs, so barriers and descriptor offsets are
+      // constants; item bookkeeping happens only at item ends.  The next pair's barrier is
+      // tested (without waiting) before this pair's MMAs are issued, so the test overlaps them.
+      const uint64_t b_first = desc_kmajor_sw128(smem_u32(sX));
+      const uint32_t a_first = tmem + G::kACol0, e_first = tmem + G::kMetaCol0;
+      const int NP = nj * KP;
+      int P = 0, j = 0, lp = 0;
+      uint32_t idesc = idesc_f16(kMtRows, (s_item[0][2] + 15) & ~15, kBf16, SP), d_tmem = tmem;
+      bool ready = mbar_wait(&st_full[0], 0);
+#pragma unroll 1
+      for (int round = 0; P < NP; ++round) {
+#pragma unroll
+        for (int q = 0; q < kPairs; ++q) {
+          if (P < NP) {
+            if (!ready) {  // a producer gave up (or a wait ran out): stop issuing
+              aborted = 1;
+              P = NP;
+              break;
+            }
+            const int qn = (q + 1) % kPairs;
+            const uint32_t pn = (uint32_t)(round + (q + 1 == kPairs)) & 1;  // parity of pair P + 1
+            const bool next = P + 1 < NP && mbar_test_wait(&st_full[qn], pn);
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int sl = 2 * q + h;
+              const uint64_t b0 = b_first + (uint64_t)(sl * (kMtX >> 4));  // descriptor address: 16-byte units
+              const uint32_t a0 = a_first + G::kACols * sl;
+              if constexpr (!SP) {
+#pragma unroll
+                for (int k = 0; k < kMtBK / 16; ++k)  // K = 16: 8 A columns, 32 bytes of B
+                  umma_f16_tmem_a(d_tmem, a0 + 8 * k, b0 + 2 * k, idesc, (lp | h | k) != 0);
+              } else {
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {  // K = 32 logical: 8 A columns, 64 bytes of B, one metadata column
+                  // an odd metadata column is named by the even one below it plus the sparse-id2 field
+                  const uint32_t ecl = e_first + 2 * sl + t;
+                  umma_f16_sp_tmem_a(d_tmem, a0 + 8 * t, b0 + 4 * t, ecl & ~1u, idesc | (ecl & 1u),
+                                     (lp | h | t) != 0);
+                }
+              }
+            }
+            umma_commit(&st_empty[q]);
+            if (++lp == KP) {  // the item is done: hand its accumulator over, set up the next one
+              umma_commit(&t_full[j & 1]);
+              lp = 0;
+              if (++j < nj) {
+                d_tmem = tmem + kMtAccCols * (j & 1);
+                idesc = idesc_f16(kMtRows, (s_item[j][2] + 15) & ~15, kBf16, SP);
+                if (j >= 2 && !mbar_wait(&t_empty[j & 1], ((j >> 1) - 1) & 1)) ready = false;
+              }
+            }
+            if (ready) ready = P + 1 >= NP || next || mbar_wait(&st_full[qn], pn);
+            ++P;
+          }
+        }
+      }
+      if (aborted) {  // let the epilogue warps through (their results are void)
+        umma_commit(&t_full[0]);
+        umma_commit(&t_full[1]);
+      }
+    }
+  } else if (warp >= kMtWarpEpi0) {
+    // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (weight rows) of the item's
+    // accumulator, 32 columns (routed rows) at a time, and stores each routed row's 32 outputs
+    // with one store; then it hands the accumulator back.
+    const int qd = warp & 3;
+    const uint32_t t_lane = static_cast<uint32_t>(32 * qd) << 16;
+    const float scale = kMtUnscale<T> * *p.w_ts;
+#pragma unroll 1
+    for (int j = 0; j < nj; ++j) {
+      const int acc = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&t_full[acc], (j >> 1) & 1) && !*(volatile int*)&aborted)) {
+        aborted = 1;
+        break;
+      }
       tc_fence_after();
-      const int c = warp >> 2;
-      if (32 * c < count) {
-        const int orow = (int)blockIdx.x * kMtRows + r;
-        const float scale = kMtUnscale<T> * *p.w_ts;
+      const int first = s_item[j][1], count = s_item[j][2];
+      const int orow = (item_id(j) % RB) * kMtRows + 32 * qd + lane;
+#pragma unroll 1
+      for (int c = 0; 32 * c < count; ++c) {
         float v[32];
-        tmem_ld32(tmem + t_lane + 32 * c, v);
+        tmem_ld32(tmem + t_lane + kMtAccCols * acc + 32 * c, v);
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) {
           const int i = 32 * c + ii;
-          if (i < count) p.y[(int64_t)s_perm[i] * p.N + orow] = v[ii] * scale;
+          if (i < count) p.y[(int64_t)p.perm[first + i] * p.N + orow] = v[ii] * scale;
         }
       }
-    } else {
-      aborted = 1;
-    }
-  } else if (warp == kMtWarpMma) {
-    if (lane == 0) {
-      // ---- MMA issuer.  The next pair's barrier is tested (without waiting) before this
-      // pair's MMAs are issued, so the test's latency overlaps them.
-      const uint32_t idesc = idesc_f16(kMtRows, n_mma, kBf16, SP);
-      const uint64_t b_first = desc_kmajor_sw128(smem_u32(sX));
-      const int KP = KB / 2;  // stage pairs
-      bool ready = mbar_wait(&st_full[0], 0);
-#pragma unroll 1
-      for (int pr = 0; pr < KP; ++pr) {
-        if (!ready) {  // a producer gave up (or the wait ran out): stop issuing
-          aborted = 1;
-          break;
-        }
-        const int q = pr % kMtPairs, qn = (pr + 1) % kMtPairs;
-        const uint32_t pn = ((pr + 1) / kMtPairs) & 1;
-        const bool next = pr + 1 < KP && mbar_test_wait(&st_full[qn], pn);
-        tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int s = 2 * q + h;
-          const uint64_t b0 = b_first + (uint64_t)(s * (kMtX >> 4));  // descriptor address: 16-byte units
-          const uint32_t a0 = tmem + kMtAccCols + G::kACols * s;
-          if constexpr (!SP) {
-#pragma unroll
-            for (int k = 0; k < kMtBK / 16; ++k)  // K = 16: 8 A columns, 32 bytes of B
-              umma_f16_tmem_a(tmem, a0 + 8 * k, b0 + 2 * k, idesc, (pr | h | k) != 0);
-          } else {
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {  // K = 32 logical: 8 A columns, 64 bytes of B, one metadata column
-              // an odd metadata column is named by the even one below it plus the sparse-id2 field
-              const uint32_t ecl = tmem + G::kMetaCol0 + 2 * s + t;
-              umma_f16_sp_tmem_a(tmem, a0 + 8 * t, b0 + 4 * t, ecl & ~1u, idesc | (ecl & 1u), (pr | h | t) != 0);
-            }
-          }
-        }
-        umma_commit(&st_empty[q]);
-        ready = pr + 1 >= KP || next || mbar_wait(&st_full[qn], pn);
-      }
-      umma_commit(&tfull_bar);  // also after an abort, so the epilogue does not wait in vain
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[acc]);
     }
   } else if (warp == kMtWarpW) {
     if (lane == 0) {
       // ---- weight boxes: codes, block scales (and metadata) of kStagesPerBox stages per copy set
+      const int BPI = KB / G::kStagesPerBox, NB = nj * BPI;
       int issued = 0;
 #pragma unroll 1
-      for (int m = 0; m < KB / G::kStagesPerBox; ++m) {
-        const int s = m % G::kBoxes;
-        if (!mbar_wait(&w_empty[s], ((m / G::kBoxes) & 1) ^ 1) || *(volatile int*)&aborted) {
+      for (int b = 0; b < NB; ++b) {
+        const int j = b / BPI, mb = b - j * BPI, s = b % G::kBoxes;
+        const int row0 = s_item[j][0] * p.N + (item_id(j) % RB) * kMtRows;  // stacked weight row (< 2^31)
+        if (!mbar_wait(&w_empty[s], ((b / G::kBoxes) & 1) ^ 1) || *(volatile int*)&aborted) {
           aborted = 1;
           break;
         }
         uint8_t* box = sW + s * G::kBox;
         mbar_arrive_expect_tx(&w_full[s], G::kBox);
-        tma_load_2d(box, &tmC, &w_full[s], m * 128, row0);
-        tma_load_2d(box + kMtCodeBox, &tmS, &w_full[s], m * 16, row0);
-        if constexpr (SP) tma_load_2d(box + kMtCodeBox + kMtScaleBox, &tmE, &w_full[s], m * 64, row0);
+        tma_load_2d(box, &tmC, &w_full[s], mb * 128, row0);
+        tma_load_2d(box + kMtCodeBox, &tmS, &w_full[s], mb * 16, row0);
+        if constexpr (SP) tma_load_2d(box + kMtCodeBox + kMtScaleBox, &tmE, &w_full[s], mb * 64, row0);
         ++issued;
       }
       // no copy may still be landing in shared memory when the CTA exits
-      for (int m = issued - G::kBoxes > 0 ? issued - G::kBoxes : 0; m < issued; ++m)
-        mbar_wait(&w_full[m % G::kBoxes], (m / G::kBoxes) & 1);
+      for (int b = issued - G::kBoxes > 0 ? issued - G::kBoxes : 0; b < issued; ++b)
+        mbar_wait(&w_full[b % G::kBoxes], (b / G::kBoxes) & 1);
     }
   } else {
     // ---- token rows: gather thread t copies 16-byte chunk t % 8 of routed rows t / 8 + 32u
-    // (u = 0 .. 3) of each stage, kMtDp stage pairs ahead (rows count .. n_mma - 1 zero-filled)
-    const int t = tid - 32 * kMtWarpX0, j = t & 7;
+    // (u = 0 .. 3) of each stage, kDp stage pairs ahead (rows count .. n_mma - 1 zero-filled)
+    const int t = tid - 32 * kMtWarpX0, j8 = t & 7;
     const uint16_t* xrow[4];
     uint32_t xoff[4], xbytes[4];
-    int nx = 0;
+    int nx = 0, cur_j = -1;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = (t >> 3) + 32 * u;
-      xoff[u] = sw128(i, j);
-      xbytes[u] = i < count ? 16u : 0u;
-      xrow[u] = p.x + (i < count ? (int64_t)(s_perm[i] / p.topk) * p.K : 0) + 8 * j;
-      nx += i < n_mma;
-    }
-    auto issue = [&](int kx) {
-      uint8_t* b = sX + (kx % kMtSlots) * kMtX;
+    for (int u = 0; u < 4; ++u) xoff[u] = sw128((t >> 3) + 32 * u, j8);
+    auto issue_pair = [&](int P) {
+      const int j = P / KP, lp = P - j * KP;
+      if (j != cur_j) {  // a new item: its routed rows' token addresses
+        cur_j = j;
+        const int first = s_item[j][1], count = s_item[j][2], n_mma = (count + 15) & ~15;
+        nx = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (u < nx) cp_async16_zfill(b + xoff[u], xrow[u] + (int64_t)kx * kMtBK, xbytes[u]);
-    };
-    const int KP = KB / 2;
-    for (int pp = 0; pp < kMtDp; ++pp) {  // the first pairs: their slots are fresh
-      if (pp < KP) {
-        issue(2 * pp);
-        issue(2 * pp + 1);
+        for (int u = 0; u < 4; ++u) {
+          const int i = (t >> 3) + 32 * u;
+          xbytes[u] = i < count ? 16u : 0u;
+          xrow[u] = p.x + (i < count ? (int64_t)(p.perm[first + i] / p.topk) * p.K : 0) + 8 * j8;
+          nx += i < n_mma;
+        }
       }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint8_t* b = sX + ((2 * P + h) % kSlots) * kMtX;
+        const int64_t kofs = (int64_t)(2 * lp + h) * kMtBK;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (u < nx) cp_async16_zfill(b + xoff[u], xrow[u] + kofs, xbytes[u]);
+      }
+    };
+    const int NP = nj * KP;
+    for (int pp = 0; pp < kDp; ++pp) {  // the first pairs: their slots are fresh
+      if (pp < NP) issue_pair(pp);
       cp_async_commit();
     }
 #pragma unroll 1
-    for (int pr = 0; pr < KP; ++pr) {
-      cp_async_wait<kMtDp - 1>();  // this thread's chunks of stage pair pr have landed
-      fence_proxy_async_smem();    // ... and are visible to the MMA's operand reads
+    for (int P = 0; P < NP; ++P) {
+      cp_async_wait<kDp - 1>();  // this thread's chunks of stage pair P have landed
+      fence_proxy_async_smem();  // ... and are visible to the MMA's operand reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st_full[pr % kMtPairs]);
-      const int pn = pr + kMtDp;
-      if (pn < KP) {
-        if (pn >= kMtPairs) {  // the slot pair's previous pair pn - kMtPairs = pr - 2 is multiplied
-          const bool ok = mbar_wait(&st_empty[pn % kMtPairs], ((pn / kMtPairs) - 1) & 1) && !*(volatile int*)&aborted;
+      if (lane == 0) mbar_arrive(&st_full[P % kPairs]);
+      const int Pn = P + kDp;
+      if (Pn < NP) {
+        if (Pn >= kPairs) {  // the slot pair's previous pair Pn - kPairs = P - 2 is multiplied
+          const bool ok = mbar_wait(&st_empty[Pn % kPairs], ((Pn / kPairs) - 1) & 1) && !*(volatile int*)&aborted;
           if (!__all_sync(0xffffffffu, ok)) {
             aborted = 1;
             break;
           }
         }
-        issue(2 * pn);
-        issue(2 * pn + 1);
+        issue_pair(Pn);
       }
       cp_async_commit();
     }
@@ -453,13 +523,17 @@ __global__ void __launch_bounds__(kMtThreads, 1)
 
 template <typename T, bool SP>
 int launch_moe_tc(const CUtensorMap& tmC, const CUtensorMap& tmS, const CUtensorMap& tmE, const MoeTcParams& p,
-                  int64_t n_tiles, cudaStream_t s) {
+                  int64_t n_items_max, cudaStream_t s) {
   auto kern = moe_w4a16_tc_kernel<T, SP>;
   const size_t smem = MtGeom<SP>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
-  dim3 grid((unsigned)(p.N / kMtRows), (unsigned)n_tiles);
-  kern<<<grid, kMtThreads, smem, s>>>(tmC, tmS, tmE, p);
+  // one CTA per SM, or more when the items would not fit kMtMaxItems per CTA
+  int64_t grid = sm_count();
+  if ((n_items_max + kMtMaxItems - 1) / kMtMaxItems > grid) grid = (n_items_max + kMtMaxItems - 1) / kMtMaxItems;
+  if (grid > n_items_max) grid = n_items_max;
+  if (grid > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, kMtThreads, smem, s>>>(tmC, tmS, tmE, p);
   return launch_status();
 }
 
@@ -470,12 +544,13 @@ bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_
   const bool sp = wf == W_SQ4;
   if (!(wf == W_DQ4 || sp) || x_fmt != X_16) return false;
   const int64_t box_k = sp ? MtGeom<true>::kBoxK : MtGeom<false>::kBoxK;
-  return T > 0 && T < INT32_MAX && N > 0 && N % kMtRows == 0 && N / kMtRows <= 65535 && K > 0 &&
-         K % box_k == 0 && K <= INT32_MAX / 2 && E * N <= INT32_MAX && max_tiles <= 65535 && aligned(codes, 16) &&
-         aligned(scales, 16) && (!sp || aligned(meta, 16)) && aligned(x, 16);
+  return T > 0 && T < INT32_MAX && N > 0 && N % kMtRows == 0 && K > 0 && K % box_k == 0 && K <= INT32_MAX / 2 &&
+         E * N <= INT32_MAX && max_tiles * (N / kMtRows) <= INT32_MAX && aligned(codes, 16) && aligned(scales, 16) &&
+         (!sp || aligned(meta, 16)) && aligned(x, 16);
 }
 
-int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_t n_tiles, cudaStream_t s) {
+int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_t n_tiles,
+                   const int32_t* n_valid, cudaStream_t s) {
   if (n_tiles <= 0) return SP24_OK;
   const bool sparse = wf == W_SQ4;
   MoeTcParams p{};
@@ -483,6 +558,7 @@ int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T
   p.w_ts = sp.w_ts;
   p.tiles = sp.tiles;
   p.perm = sp.perm;
+  p.n_valid = n_valid;
   p.y = sp.y;
   p.topk = sp.topk;
   p.T = (int)T;
@@ -497,11 +573,12 @@ int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T
   if (!st) st = sparse ? make_tmap_2d_plain(&tmE, sp.meta, rows, K / 8, K / 8, 64, kMtRows) : SP24_OK;
   if (st) return st;
   if (!sparse) tmE = tmS;  // unused
+  const int64_t n_items_max = n_tiles * (sp.N / kMtRows);
   if (sparse)
-    return t16 == SP24_F16 ? launch_moe_tc<__half, true>(tmC, tmS, tmE, p, n_tiles, s)
-                           : launch_moe_tc<__nv_bfloat16, true>(tmC, tmS, tmE, p, n_tiles, s);
-  return t16 == SP24_F16 ? launch_moe_tc<__half, false>(tmC, tmS, tmE, p, n_tiles, s)
-                         : launch_moe_tc<__nv_bfloat16, false>(tmC, tmS, tmE, p, n_tiles, s);
+    return t16 == SP24_F16 ? launch_moe_tc<__half, true>(tmC, tmS, tmE, p, n_items_max, s)
+                           : launch_moe_tc<__nv_bfloat16, true>(tmC, tmS, tmE, p, n_items_max, s);
+  return t16 == SP24_F16 ? launch_moe_tc<__half, false>(tmC, tmS, tmE, p, n_items_max, s)
+                         : launch_moe_tc<__nv_bfloat16, false>(tmC, tmS, tmE, p, n_items_max, s);
 }
 
 }  // namespace sp24
