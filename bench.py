@@ -590,7 +590,9 @@ def run_sweep(args) -> None:
 
 def run_ncu_target() -> None:
     """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode
-    pipeline on the decode workload: prepare_vec, encode_kernel x2, decode_gemv x2 per pass; W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096)."""
+    pipeline on the decode workload: prepare_vec, encode_pair_kernel, decode_tile_kernel dense
+    and 2:4 per pass; W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096; then the
+    routed-expert workload once, NVFP4 experts dense and 2:4)."""
     import torch
 
     import fp16_gemm_b200 as sp
@@ -618,6 +620,16 @@ def run_ncu_target() -> None:
     for _ in range(2):
         sp.gemm_dense(x16, w16)
         sp.gemm_sparse24(x16, sp.Sparse24(v, m), 5120)
+    del w16, x16, v, m
+    d = synth.moe()
+    E, Ne, Ke = d["W"].shape
+    xm, rt = bf(d["X"]), torch.from_numpy(d["routing"]).cuda()
+    wm = bf(d["W"].reshape(E * Ne, Ke))
+    del d
+    _, wq, sw = sp.prepare_nvfp4_24(wm)
+    del wm
+    sp.gemm_grouped(xm, rt, wq, E, Ne, Ke)
+    sp.gemm_grouped(xm, rt, sw, E, Ne, Ke)
     torch.cuda.synchronize()
     assert sp.last_device_error() == sp.OK
     print("ncu target done")
