@@ -235,6 +235,9 @@ int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int6
  *            (16-bit or NVFP4; NVFP4 experts share one tensor scale, [P5] "The shared global
  *            scale") or w_sparse (2:4-compressed, stacked [E*N, K/2] values + [E*N, K/8] meta).
  *   K alignment: NVFP4 dense K % 256, NVFP4 2:4 K % 512, 16-bit K % 8 (2:4: K % 128).
+ *   NVFP4 experts (dense or 2:4) with 16-bit x and N % 128 == 0 run on the tensor cores and
+ *   write every output once (the result does not depend on launch order); other cases add
+ *   K-slice partial sums with fp32 atomics.
  *   workspace: sp24_gemm_grouped_workspace_size() bytes, 16-byte aligned (routing histogram,
  *   offsets, token tiles, permutation). */
 int sp24_gemm_grouped_workspace_size(int64_t T, int topk, int64_t E, int64_t* bytes);
