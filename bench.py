@@ -562,6 +562,31 @@ def run_sweep(args) -> None:
                           "compress": {"us": round(us_p, 3), "GB/s": round((nb + vals.numel() * 2 + meta.numel()) / us_p / 1e3, 1)},
                           "n_fail": int(nf.item())}), flush=True)
 
+    # large single-tensor quantisation: a [151936, 4096] bf16 output head (~1.16 GiB -> 0.33 GiB
+    # of codes + scales).  Full call: amax pass + encode pass (the tensor is 10x the L2, so it is
+    # read twice); with a supplied (group-shared) scale: one pass; the group scale alone: one read.
+    Wh = t16(synth.output_head()["W"], "bf16")
+    R, L = Wh.shape
+    qh = sp.quantize_nvfp4(Wh)
+    nb_in, nb_out = Wh.numel() * 2, R * L // 2 + R * L // 16 + 4
+    us_full = timeit(lambda r: sp.quantize_nvfp4(Wh, out=qh), reps=5)
+    ts_h = qh.tensor_scale.clone()
+    us_one = timeit(lambda r: sp.quantize_nvfp4(Wh, tensor_scale=ts_h, out=qh), reps=5)
+    gs_out = torch.empty(1, dtype=torch.float32, device=dev)
+    us_gs = timeit(lambda r: sp.nvfp4_group_tensor_scale([Wh], out=gs_out), reps=5)
+    alg = nb_in + nb_out
+    print(json.dumps({"sweep": "quantize_large", "shape": [R, L], "dtype": "bf16",
+                      "in_bytes": nb_in, "out_bytes": nb_out,
+                      "derived_scale": {"us": round(us_full, 1), "GB/s": round(alg / us_full / 1e3, 1),
+                                        "frac_hbm": round(alg / us_full / 1e3 / peak_hbm, 3),
+                                        "traffic_GB/s": round((2 * nb_in + nb_out) / us_full / 1e3, 1),
+                                        "note": "two reads of the tensor (amax, then encode)"},
+                      "supplied_scale": {"us": round(us_one, 1), "GB/s": round(alg / us_one / 1e3, 1),
+                                         "frac_hbm": round(alg / us_one / 1e3 / peak_hbm, 3)},
+                      "group_scale_only": {"us": round(us_gs, 1), "GB/s": round(nb_in / us_gs / 1e3, 1),
+                                           "frac_hbm": round(nb_in / us_gs / 1e3 / peak_hbm, 3)}}), flush=True)
+    del Wh, qh
+
     # routed experts: 4096 tokens x top-10 of 512 experts [512, 2048], bf16 x, NVFP4 experts
     # (dense, and 2:4 of the same experts); every expert is touched, so each call reads all of
     # them once (one copy: 302 MB dense / 218 MB 2:4, well beyond L2)

@@ -35,7 +35,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_gemm_dense", "sp24_gemm_sparse24", "sp24_kernel_launches",
            "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc", "sp24_gemm_grouped_workspace_size",
            "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24",
-           "sp24_quantize_nvfp4_pair")
+           "sp24_quantize_nvfp4_pair", "sp24_nvfp4_group_tensor_scale_workspace_size",
+           "sp24_nvfp4_group_tensor_scale")
 
 _lock = threading.Lock()
 _lib = None
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             L.sp24_prepare_24_workspace_size.argtypes = [I64, I64, P]
             L.sp24_prepare_24.argtypes = [P, I, I64, I64, P, P, P, P, P, P, P, I64, P]
             L.sp24_quantize_nvfp4_pair.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, I64, P, P, P, P, P]
+            L.sp24_nvfp4_group_tensor_scale_workspace_size.argtypes = [P]
+            L.sp24_nvfp4_group_tensor_scale.argtypes = [P, P, I, I, P, P, I64, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -241,6 +244,32 @@ def quantize_nvfp4(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None,
     _call("sp24_quantize_nvfp4", _ptr(t), _dtype_code(t), R, L, _ptr(tensor_scale),
           _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), _ptr(workspace),
           0 if workspace is None else workspace.numel(), _stream(stream))
+    return out
+
+
+def nvfp4_group_tensor_scale(tensors, out: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One NVFP4 tensor scale (fp32 [1], device) shared by a group of tensors of one dtype:
+    max amax / 2688 over all of them.  Pass it to quantize_nvfp4(t, tensor_scale=...)."""
+    tensors = list(tensors)
+    if not tensors:
+        raise ValueError("nvfp4_group_tensor_scale wants at least one tensor")
+    for i, t in enumerate(tensors):
+        _cuda(t, f"tensors[{i}]")
+        if not t.is_contiguous() or t.dtype != tensors[0].dtype:
+            raise ValueError("nvfp4_group_tensor_scale wants contiguous tensors of one dtype")
+    dev = tensors[0].device
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        nb = ctypes.c_int64(0)
+        _call("sp24_nvfp4_group_tensor_scale_workspace_size", ctypes.byref(nb))
+        workspace = torch.empty(nb.value, dtype=torch.uint8, device=dev)
+    n = len(tensors)
+    ptrs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in tensors])
+    numels = (ctypes.c_int64 * n)(*[t.numel() for t in tensors])
+    _call("sp24_nvfp4_group_tensor_scale", ptrs, numels, n, _dtype_code(tensors[0]), _ptr(out),
+          _ptr(workspace), workspace.numel(), _stream(stream))
     return out
 
 

@@ -173,6 +173,22 @@ int sp24_quantize_nvfp4_pair(const void* t0, int dtype, int64_t rows0, int64_t c
                              const void* t1, int64_t rows1, int64_t cols1, const float* ts1,
                              uint8_t* codes1, uint8_t* scales1, float* ts_out1, void* stream);
 
+/* [P5] "The shared global scale": one tensor scale for a group of tensors that are read
+ * together (q / k / v, gate / up):  s = max_i amax(|T_i|) / 2688, one IEEE fp32 division, the
+ * scale sp24_quantize_nvfp4 derives for the group's entries taken as one tensor.  Quantise each
+ * tensor with sp24_quantize_nvfp4(T_i, tensor_scale_in = s).
+ *   tensors    host array of n device pointers (16-byte aligned when the tensor is not empty)
+ *   numels     host array of n entry counts; numel * element size a multiple of 16 bytes
+ *   dtype      F16, BF16 or F32, shared by the group
+ *   tensor_scale_out  device fp32; n == 0 or all-empty tensors give 0
+ *   workspace  device, >= sp24_nvfp4_group_tensor_scale_workspace_size() bytes, 16-byte
+ *              aligned; scratch.  NaN entries are skipped; an infinity gives an infinite scale.
+ * One launch per 16 tensors plus a one-thread kernel; nothing is allocated. */
+int sp24_nvfp4_group_tensor_scale_workspace_size(int64_t* bytes);
+int sp24_nvfp4_group_tensor_scale(const void* const* tensors, const int64_t* numels, int n,
+                                  int dtype, float* tensor_scale_out, void* workspace,
+                                  int64_t workspace_bytes, void* stream);
+
 /* Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
  * (F16/BF16/F32). */
 int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,

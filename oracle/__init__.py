@@ -204,6 +204,15 @@ def nvfp4_tensor_scale(t: np.ndarray, dtype: int) -> float:
     return float(np.float32(lib().sp24o_nvfp4_tensor_scale(_ptr(t), dtype, t.size)))
 
 
+def nvfp4_group_tensor_scale(tensors, dtype: int) -> float:
+    """One tensor scale for a group of tensors read together ([P5] "The shared global scale"):
+    the scale of the group's entries taken as one tensor, max amax / 2688."""
+    flat = [np.ascontiguousarray(t).ravel() for t in tensors]
+    if not flat or sum(f.size for f in flat) == 0:
+        return 0.0
+    return nvfp4_tensor_scale(np.concatenate([f for f in flat if f.size]), dtype)
+
+
 def nvfp4_encode(t: np.ndarray, dtype: int, tensor_scale: float | None = None):
     """(codes [R, L/2] u8, scales [R, L/16] u8, tensor_scale f32) of a 2-D tensor T[R, L]."""
     t = _bits(t, dtype)

@@ -18,6 +18,10 @@ Workloads (the shapes the pages' workloads take; see the design notes for the ma
                      without replacement.
 * ``moe_skewed``:    W bf16 [E, N, K] N(0, 0.02), X [T, K] N(0, 1), routing with given per-expert
                      row counts in a seeded random order (tile-boundary parity cases).
+* ``output_head``:   W bf16 [151936, 4096] N(0, 0.02) (an output head of ~1.16 GiB: the pages'
+                     large single-tensor quantisation), drawn in row chunks.
+* ``qkv_group``:     Wq [2048, 2048], Wk, Wv [512, 2048] N(0, 0.02), one x40 outlier in Wv (a
+                     group sharing one NVFP4 tensor scale).
 * ``msweep``:        W [5120, 5120] then X [M, 5120], N(0, 1), fp16 or bf16.
 * ``conv_fail5``:    W fp16 [256, 256, 3, 3] N(0, 1) with a 2-of-4 zero pattern along C
                      drawn at random per group, then round(5%) of the groups (a seeded
@@ -106,6 +110,31 @@ def moe(seed: int = SEED, E: int = 512, N: int = 512, K: int = 2048, T: int = 40
     X = draw(g, (T, K), "bf16")
     routing = routing_topk(g, T, E, topk)
     return {"W": W, "X": X, "routing": routing}
+
+
+def output_head(seed: int = SEED, vocab: int = 151936, hidden: int = 4096, sigma: float = 0.02,
+                rows_per_draw: int = 8192):
+    """W bf16 [vocab, hidden] N(0, sigma), drawn in row chunks from one stream (the same numbers
+    a single draw gives) so the float64 temporary stays at one chunk."""
+    g = rng(seed)
+    W = np.empty((vocab, hidden), dtype=np.uint16)
+    for r in range(0, vocab, rows_per_draw):
+        n = min(rows_per_draw, vocab - r)
+        W[r:r + n] = draw(g, (n, hidden), "bf16", sigma)
+    return {"W": W}
+
+
+def qkv_group(seed: int = SEED, hidden: int = 2048, kv: int = 512, dtype: str = "bf16"):
+    """Three projection weights read together: Wq [hidden, hidden], Wk and Wv [kv, hidden],
+    N(0, 0.02), drawn in that order; Wv gets one outlier (x 40 at a seeded place) so the
+    group's largest magnitude sits in the last tensor."""
+    g = rng(seed)
+    Wq = normal(g, (hidden, hidden), 0.02)
+    Wk = normal(g, (kv, hidden), 0.02)
+    Wv = normal(g, (kv, hidden), 0.02)
+    i = int(g.integers(0, Wv.size))
+    Wv.flat[i] *= 40.0
+    return {"Wq": as_storage(Wq, dtype), "Wk": as_storage(Wk, dtype), "Wv": as_storage(Wv, dtype)}
 
 
 def moe_skewed(counts, seed: int = SEED, N: int = 256, K: int = 320, topk: int = 2,

@@ -356,6 +356,42 @@ def test_amax_survives_pruning(oracle):
     assert oracle.nvfp4_tensor_scale(vals, oracle.BF16) == oracle.nvfp4_tensor_scale(w, oracle.BF16)
 
 
+def test_group_tensor_scale_closed_form(oracle):
+    """'The shared global scale': a group's scale comes from the largest |t| of all its tensors.
+    The largest magnitude 2688 = 6 * 448 (exact in bf16) sits in the second tensor, so the
+    group's scale is exactly 1.0 and each tensor alone would get a smaller one."""
+    a = synth.as_storage(np.array([[1.0, -2.0, 0.5, 3.0] * 4]), "bf16")
+    b = synth.as_storage(np.array([[0.0] * 15 + [-2688.0]]), "bf16")
+    assert oracle.nvfp4_group_tensor_scale([a, b], oracle.BF16) == 1.0
+    assert oracle.nvfp4_tensor_scale(a, oracle.BF16) == np.float32(3.0) / np.float32(2688.0)
+    assert oracle.nvfp4_group_tensor_scale([], oracle.BF16) == 0.0
+
+
+def test_group_tensor_scale_is_max_of_members(oracle):
+    """Division by the positive constant 2688 with round-to-nearest is monotone, so the group's
+    scale equals the largest of the members' own scales, for every storage type."""
+    g = synth.rng(41)
+    for dt, od in (("f16", oracle.F16), ("bf16", oracle.BF16), ("f32", oracle.F32)):
+        ts = [synth.draw(g, (int(g.integers(1, 9)), 16 * int(g.integers(1, 5))), dt, float(sig))
+              for sig in (0.02, 1.0, 0.3)]
+        own = [np.float32(oracle.nvfp4_tensor_scale(t, od)) for t in ts]
+        assert oracle.nvfp4_group_tensor_scale(ts, od) == max(own)
+
+
+def test_group_tensor_scale_skips_nan(oracle):
+    """NaN compares false, so it never becomes the maximum (the group scale of the rest)."""
+    x = synth.normal(synth.rng(42), (4, 32)).astype(np.float32)
+    y = x.copy()
+    y[2, 7] = np.nan
+    assert oracle.nvfp4_group_tensor_scale([y, x[:1]], oracle.F32) == oracle.nvfp4_tensor_scale(x, oracle.F32)
+
+
+def test_output_head_generator_matches_one_draw():
+    """Drawing the head in row chunks continues one stream: identical to a single draw."""
+    d = synth.output_head(vocab=10, hidden=16, rows_per_draw=3)
+    assert np.array_equal(d["W"], synth.draw(synth.rng(0), (10, 16), "bf16", 0.02))
+
+
 # ----------------------------------------------------------------------------- GEMM
 
 def test_gemm_matches_library_matmul(oracle):
