@@ -486,6 +486,8 @@ def run_sweep(args) -> None:
             return op_bytes(t.values) + t.meta.numel()
         return t.numel() * t.element_size()
 
+    selections = []
+
     def case(workload, M, N, K, xdt, wdt, X, W):
         """X, W numpy storage; xdt in {f16,bf16,nvfp4}; wdt in {f16,bf16,nvfp4}."""
         x = t16(X, "f16" if xdt == "f16" else "bf16")
@@ -524,8 +526,19 @@ def run_sweep(args) -> None:
             res[name] = {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(gbs, 1),
                          "bytes": byts, "AI": round(ai, 1), "bound": bound, "pipe": pipe,
                          "frac": round(frac, 3)}
+        # the dense / 2:4 choice the library makes for this shape without measuring (its rule
+        # of measured crossovers) against the faster of the two just timed
+        fmt = {"f16": sp.F16, "bf16": sp.BF16, "nvfp4": sp.NVFP4}
+        sp.gemm_choice_reset()
+        rule_sparse = sp.gemm_choice(fmt[xdt], fmt[wdt], M, N, K)[0]
+        faster_sparse = res["sparse24"]["us"] < res["dense"]["us"]
+        chosen = res["sparse24" if rule_sparse else "dense"]["us"]
+        selections.append({"workload": workload, "M": M, "rule": "sparse24" if rule_sparse else "dense",
+                           "faster": "sparse24" if faster_sparse else "dense",
+                           "loss": round(chosen / min(res["dense"]["us"], res["sparse24"]["us"]) - 1.0, 3)})
         line = {"sweep": workload, "M": M, "N": N, "K": K, "x": xdt, "w": wdt, **res,
                 "sparse_dense_speedup": round(res["dense"]["us"] / res["sparse24"]["us"], 3),
+                "selected": "sparse24" if rule_sparse else "dense",
                 "peaks": {"hbm_gbs": peak_hbm, "tensor_tflops": tensor_peak, "kind": kind}}
         print(json.dumps(line), flush=True)
 
@@ -544,6 +557,9 @@ def run_sweep(args) -> None:
         Xb = synth.draw(synth.rng(Mv), (Mv, 5120), "bf16")
         case("msweep_nvfp4_w4a16", Mv, 5120, 5120, "bf16", "nvfp4", Xb, Wb)
         case("msweep_nvfp4_w4a4", Mv, 5120, 5120, "nvfp4", "nvfp4", Xb, Wb)
+    agree = sum(c["rule"] == c["faster"] for c in selections)
+    print(json.dumps({"sweep": "dense_sparse_selection", "shapes": len(selections), "rule_picks_faster": agree,
+                      "worst_loss": max(c["loss"] for c in selections), "cases": selections}), flush=True)
     # conv eligibility check + compression (fp16 [256, 256, 3, 3], 5% failing groups), one
     # tensor and a batch of 512 such tensors as one [512*256, 256, 3, 3] launch
     c = synth.conv_fail5()

@@ -36,7 +36,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_last_device_error", "sp24_quantize_nvfp4_noalloc", "sp24_gemm_grouped_workspace_size",
            "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24",
            "sp24_quantize_nvfp4_pair", "sp24_nvfp4_group_tensor_scale_workspace_size",
-           "sp24_nvfp4_group_tensor_scale")
+           "sp24_nvfp4_group_tensor_scale", "sp24_gemm_select", "sp24_gemm_choice", "sp24_gemm_auto",
+           "sp24_gemm_choice_reset")
 
 _lock = threading.Lock()
 _lib = None
@@ -95,6 +96,13 @@ def lib() -> ctypes.CDLL:
             L.sp24_quantize_nvfp4_pair.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, I64, P, P, P, P, P]
             L.sp24_nvfp4_group_tensor_scale_workspace_size.argtypes = [P]
             L.sp24_nvfp4_group_tensor_scale.argtypes = [P, P, I, I, P, P, I64, P]
+            L.sp24_gemm_select.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand),
+                                           ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, I,
+                                           P, P, P, P]
+            L.sp24_gemm_choice.argtypes = [I, I, I64, I64, I64, P, P]
+            L.sp24_gemm_auto.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand),
+                                         ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P, P]
+            L.sp24_gemm_choice_reset.argtypes = []
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -438,6 +446,66 @@ def gemm_sparse24(x, w: Sparse24, K: int, out=None, algo: int = ALGO_AUTO, works
     _call("sp24_gemm_sparse24", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out),
           _ptr(workspace), 0 if workspace is None else workspace.numel(), algo, _stream(stream))
     return out
+
+
+def _sparse_operand(w: "Sparse24") -> _SparseOperand:
+    v = w.values
+    if isinstance(v, NVFP4Tensor):
+        return _SparseOperand(NVFP4, v.codes.data_ptr(), v.scales.data_ptr(), v.tensor_scale.data_ptr(),
+                              w.meta.data_ptr())
+    _cuda(v, "values")
+    return _SparseOperand(_dtype_code(v), v.data_ptr(), None, None, w.meta.data_ptr())
+
+
+def _both_forms(x, w_dense, w_sparse: "Sparse24"):
+    M, K = _rows_k(x)
+    N, Kw = _rows_k(w_dense)
+    if K != Kw:
+        raise ValueError(f"K mismatch: {K} vs {Kw}")
+    ws = max(gemm_workspace_bytes(x, w_dense, False, M, N, K), gemm_workspace_bytes(x, w_sparse, True, M, N, K))
+    return M, N, K, ws
+
+
+def gemm_choice(x_format: int, w_format: int, M: int, N: int, K: int) -> tuple:
+    """(use_sparse, measured): the dense / 2:4 decision for a shape (host only)."""
+    u, m = ctypes.c_int(0), ctypes.c_int(0)
+    _call("sp24_gemm_choice", x_format, w_format, M, N, K, ctypes.byref(u), ctypes.byref(m))
+    return bool(u.value), bool(m.value)
+
+
+def gemm_choice_reset() -> None:
+    _call("sp24_gemm_choice_reset")
+
+
+def gemm_select(x, w_dense, w_sparse: "Sparse24", reps: int = 10, out=None, workspace=None, stream=None) -> dict:
+    """Times the dense and the 2:4 GEMM of this shape, records the faster one (synchronises)."""
+    M, N, K, ws_bytes = _both_forms(x, w_dense, w_sparse)
+    dev = w_sparse.meta.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    xo, wd, wsp = _operand(x), _operand(w_dense), _sparse_operand(w_sparse)
+    u, td, tsp = ctypes.c_int(0), ctypes.c_float(0), ctypes.c_float(0)
+    _call("sp24_gemm_select", ctypes.byref(xo), ctypes.byref(wd), ctypes.byref(wsp), M, N, K, _ptr(out),
+          _ptr(workspace), 0 if workspace is None else workspace.numel(), reps, ctypes.byref(u),
+          ctypes.byref(td), ctypes.byref(tsp), _stream(stream))
+    return {"use_sparse": bool(u.value), "us_dense": td.value, "us_sparse": tsp.value}
+
+
+def gemm_auto(x, w_dense, w_sparse: "Sparse24", out=None, workspace=None, stream=None):
+    """Y[M, N] from whichever form sp24_gemm_choice names; returns (Y, used_sparse)."""
+    M, N, K, ws_bytes = _both_forms(x, w_dense, w_sparse)
+    dev = w_sparse.meta.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    xo, wd, wsp = _operand(x), _operand(w_dense), _sparse_operand(w_sparse)
+    u = ctypes.c_int(0)
+    _call("sp24_gemm_auto", ctypes.byref(xo), ctypes.byref(wd), ctypes.byref(wsp), M, N, K, _ptr(out),
+          _ptr(workspace), 0 if workspace is None else workspace.numel(), ctypes.byref(u), _stream(stream))
+    return out, bool(u.value)
 
 
 def grouped_workspace_bytes(T: int, topk: int, E: int) -> int:

@@ -241,6 +241,36 @@ int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int6
                        int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                        int algo, void* stream);
 
+/* [P2] "Ask which sparse implementations were actually selected": a 2:4-eligible weight runs
+ * sparse only where that is faster for the problem size; dense may win.  For one weight held
+ * in both forms (w_dense: the pruned weight, 16-bit or NVFP4; w_sparse: its compressed form,
+ * same format):
+ *   sp24_gemm_select  times sp24_gemm_dense and sp24_gemm_sparse24 (algo auto) on `stream`, one
+ *                     warm-up and `reps` timed launches each, writes the faster to *use_sparse
+ *                     and the per-launch times (us, may be NULL), and records the decision for
+ *                     (device, x format, weight format, M, N, K).  Synchronises with the stream;
+ *                     not for use during graph capture.  y receives a result of either form.
+ *   sp24_gemm_choice  (host only) the recorded decision, else a rule of crossovers measured on
+ *                     B200: weights of fewer than 2^20 entries dense (launch-bound); else
+ *                     16-bit weights 2:4 for M <= 2048, NVFP4 weights with 16-bit x 2:4,
+ *                     NVFP4 weights with NVFP4 x dense.  *measured (may be NULL): 1 if recorded.
+ *                     SP24_ERR_DTYPE for format pairs without a 2:4 path.
+ *   sp24_gemm_auto    runs the GEMM sp24_gemm_choice names; *used_sparse (may be NULL) says
+ *                     which.  Asynchronous.
+ *   workspace: at least the larger of the two sp24_gemm_workspace_size() values (algo 0).
+ *   sp24_gemm_choice_reset forgets every recorded decision. */
+int sp24_gemm_select(const sp24_operand* x, const sp24_operand* w_dense,
+                     const sp24_sparse_operand* w_sparse, int64_t M, int64_t N, int64_t K,
+                     float* y, void* workspace, int64_t workspace_bytes, int reps,
+                     int* use_sparse, float* us_dense, float* us_sparse, void* stream);
+int sp24_gemm_choice(int x_format, int w_format, int64_t M, int64_t N, int64_t K,
+                     int* use_sparse, int* measured);
+int sp24_gemm_auto(const sp24_operand* x, const sp24_operand* w_dense,
+                   const sp24_sparse_operand* w_sparse, int64_t M, int64_t N, int64_t K,
+                   float* y, void* workspace, int64_t workspace_bytes, int* used_sparse,
+                   void* stream);
+int sp24_gemm_choice_reset(void);
+
 /* ----------------------------------------------------------------------- a7: routed experts */
 /* [P1] "Concurrency, not sparsity, is the lever": tokens routed top-k to E experts.
  *   Y[t, s, n] = sum_k x[t, k] W[e, n, k],  e = routing[t, s]   (fp32 [T, topk, N], device)
