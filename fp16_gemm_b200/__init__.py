@@ -37,7 +37,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_gemm_grouped", "sp24_prepare_24_workspace_size", "sp24_prepare_24",
            "sp24_quantize_nvfp4_pair", "sp24_nvfp4_group_tensor_scale_workspace_size",
            "sp24_nvfp4_group_tensor_scale", "sp24_gemm_select", "sp24_gemm_choice", "sp24_gemm_auto",
-           "sp24_gemm_choice_reset")
+           "sp24_gemm_choice_reset", "sp24_moe_block_workspace_size", "sp24_moe_block",
+           "sp24_interleave_rows")
 
 _lock = threading.Lock()
 _lib = None
@@ -103,6 +104,11 @@ def lib() -> ctypes.CDLL:
             L.sp24_gemm_auto.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand),
                                          ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P, P]
             L.sp24_gemm_choice_reset.argtypes = []
+            L.sp24_moe_block_workspace_size.argtypes = [I64, I, I64, I64, P]
+            L.sp24_moe_block.argtypes = [ctypes.POINTER(_Operand), P, P, I64, I, ctypes.POINTER(_Operand),
+                                         ctypes.POINTER(_SparseOperand), ctypes.POINTER(_Operand),
+                                         ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
+            L.sp24_interleave_rows.argtypes = [P, P, I64, I64, I64, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -557,3 +563,61 @@ def sizes(op: int, dtype: int, shape) -> dict:
     _call("sp24_sizes", op, dtype, _shape(shape), len(shape), *[ctypes.byref(o) for o in out])
     keys = ("groups", "values_bytes", "meta_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes")
     return {k: o.value for k, o in zip(keys, out)}
+
+
+def _interleave(a: torch.Tensor, b: torch.Tensor, rows: int, block_rows: int = 16, stream=None) -> torch.Tensor:
+    _cuda(a, "a")
+    _cuda(b, "b")
+    if a.shape != b.shape or a.dtype != b.dtype:
+        raise ValueError("interleave wants two tensors of one shape and dtype")
+    row_bytes = a.numel() * a.element_size() // rows
+    out = torch.empty((2 * rows, row_bytes), dtype=torch.uint8, device=a.device)
+    _call("sp24_interleave_rows", _ptr(a), _ptr(b), rows, row_bytes, block_rows, _ptr(out), _stream(stream))
+    return out
+
+
+def pack_gate_up(gate, up, stream=None):
+    """The expert block's gate / up operand: the stacked gate and up weights [E*F, H] (NVFP4Tensor,
+    or Sparse24 of NVFP4Tensor values, sharing one tensor scale) packed in 16-row blocks."""
+    if isinstance(gate, Sparse24):
+        gv, uv = gate.values, up.values
+        rows = gv.codes.shape[0]
+        vals = NVFP4Tensor(_interleave(gv.codes, uv.codes, rows, stream=stream),
+                           _interleave(gv.scales, uv.scales, rows, stream=stream), gv.tensor_scale.clone())
+        return Sparse24(vals, _interleave(gate.meta, up.meta, rows, stream=stream).reshape(-1))
+    rows = gate.codes.shape[0]
+    return NVFP4Tensor(_interleave(gate.codes, up.codes, rows, stream=stream),
+                       _interleave(gate.scales, up.scales, rows, stream=stream), gate.tensor_scale.clone())
+
+
+def moe_block_workspace_bytes(T: int, topk: int, E: int, F: int) -> int:
+    n = ctypes.c_int64(0)
+    _call("sp24_moe_block_workspace_size", T, topk, E, F, ctypes.byref(n))
+    return n.value
+
+
+def moe_block(x: torch.Tensor, routing: torch.Tensor, router_w: torch.Tensor, w_gate_up, w_down, E: int, H: int,
+              F: int, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """y[T, H] fp32 = sum_s r[t, s] * (SiLU(x Wg^T) * (x Wu^T)) Wd^T over the routed experts;
+    w_gate_up from pack_gate_up, w_down [E*H, F]; each an NVFP4Tensor or a Sparse24 of one."""
+    _cuda(routing, "routing")
+    _cuda(router_w, "router_w")
+    T, topk = routing.shape
+    dev = routing.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(moe_block_workspace_bytes(T, topk, E, F), dtype=torch.uint8, device=dev)
+    xo = _operand(x)
+    gd = gs = dd = ds = None
+    if isinstance(w_gate_up, Sparse24):
+        gs = ctypes.byref(_sparse_operand(w_gate_up))
+    else:
+        gd = ctypes.byref(_operand(w_gate_up))
+    if isinstance(w_down, Sparse24):
+        ds = ctypes.byref(_sparse_operand(w_down))
+    else:
+        dd = ctypes.byref(_operand(w_down))
+    _call("sp24_moe_block", ctypes.byref(xo), _ptr(routing), _ptr(router_w), T, topk, gd, gs, dd, ds, E, H, F,
+          _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    return out

@@ -126,6 +126,21 @@ bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_
 // n_tiles bounds the tile table; *n_valid (device) is the number of used tiles, which come first.
 int moe_tc_grouped(int wf, int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles,
                    const int32_t* n_valid, cudaStream_t s);
+// One GEMM of the expert block on the same kernel: epi 1 = gate/up (weights packed in 16-row
+// gate / up blocks, output h = SiLU(gate) * up in x's 16-bit type, routed order), epi 2 = down
+// (x = h rows in routed order, output y[T, N] += router weight * product).
+struct MoeBlockGemm {
+  const uint16_t* x;
+  const uint8_t *codes, *scales, *meta;
+  const float* w_ts;
+  const int32_t *tiles, *perm, *n_valid;
+  float* y;
+  uint16_t* h;
+  const float* router_w;
+  int x_direct, topk;
+  int64_t T, E, N, K, n_tiles;
+};
+int moe_tc_block_gemm(int epi, int wf, int t16, const MoeBlockGemm& g, cudaStream_t s);
 
 // Tensor-core (tcgen05) 16-bit GEMM: y[M, N] = (*scale_a) (*scale_b) x[M, K] w[N, K]^T.
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,

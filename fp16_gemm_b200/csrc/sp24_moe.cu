@@ -255,3 +255,153 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   if (tc) return moe_tc_grouped(wf, t16, p, E, T, n_tiles, ws.n_tiles, s);
   return skinny2_grouped(wf, t16, p, n_tiles, s);
 }
+
+// ------------------------------------------------------------------ expert block (NEXT-3)
+//
+// y[t] = sum_s r[t, s] * (SiLU(x_t Wg_e^T) * (x_t Wu_e^T)) Wd_e^T,  e = routing[t, s]
+// ([P1] "Concurrency, not sparsity, is the lever": the routed experts of a decode step).
+// Routing as for sp24_gemm_grouped (tiles of up to 128 routed rows), then the tensor-core
+// kernel twice: gate/up (weights packed as 16-row gate / up blocks, SwiGLU in the epilogue, h in
+// x's 16-bit type and routed order) and down (h rows read directly, router weight and fp32 add
+// into y in the epilogue).
+
+namespace sp24 {
+namespace {
+
+__global__ void interleave_rows_kernel(const uint4* __restrict__ a, const uint4* __restrict__ b, int64_t out_rows,
+                                       int64_t vec_per_row, int64_t block_rows, uint4* __restrict__ out) {
+  const int64_t n = out_rows * vec_per_row;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / vec_per_row, v = i - r * vec_per_row;
+    const int64_t blk = r / (2 * block_rows), within = r - blk * 2 * block_rows;
+    const int64_t src_row = blk * block_rows + (within % block_rows);
+    out[i] = (within < block_rows ? a : b)[src_row * vec_per_row + v];
+  }
+}
+
+int64_t block_h_bytes(int64_t T, int topk, int64_t F) { return (T * topk * F * 2 + 15) / 16 * 16; }
+
+}  // namespace
+}  // namespace sp24
+
+extern "C" int sp24_interleave_rows(const void* a, const void* b, int64_t rows, int64_t row_bytes,
+                                    int64_t block_rows, void* out, void* stream) {
+  if (rows < 0 || row_bytes < 0 || block_rows <= 0) return SP24_ERR_SHAPE;
+  if (rows % block_rows || row_bytes % 16) return SP24_ERR_SHAPE;
+  if (rows == 0 || row_bytes == 0) return SP24_OK;
+  if (!a || !b || !out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16)) return SP24_ERR_ALIGN;
+  const int64_t n = 2 * rows * (row_bytes / 16);
+  const int64_t blocks = (n + 255) / 256 < (int64_t)sm_count() * 8 ? (n + 255) / 256 : (int64_t)sm_count() * 8;
+  interleave_rows_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(
+      reinterpret_cast<const uint4*>(a), reinterpret_cast<const uint4*>(b), 2 * rows, row_bytes / 16, block_rows,
+      reinterpret_cast<uint4*>(out));
+  return launch_status();
+}
+
+extern "C" int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t F, int64_t* bytes) {
+  if (!bytes) return SP24_ERR_INVALID_ARG;
+  if (T < 0 || topk < 0 || E <= 0 || F < 0) return SP24_ERR_SHAPE;
+  *bytes = moe_layout(nullptr, T, topk, E).bytes + block_h_bytes(T, topk, F);
+  return SP24_OK;
+}
+
+namespace {
+
+// An NVFP4 expert operand (dense or 2:4) of the block: format, pointers, validation.
+struct BlockW {
+  int wf;
+  const uint8_t *codes, *scales, *meta;
+  const float* ts;
+};
+
+int block_weights(const sp24_operand* d, const sp24_sparse_operand* s, BlockW* out) {
+  if (!d == !s) return SP24_ERR_INVALID_ARG;
+  if (d) {
+    if (d->format != SP24_NVFP4) return SP24_ERR_DTYPE;
+    *out = {W_DQ4, reinterpret_cast<const uint8_t*>(d->data), d->scales, nullptr, d->tensor_scale};
+  } else {
+    if (s->format != SP24_NVFP4) return SP24_ERR_DTYPE;
+    *out = {W_SQ4, reinterpret_cast<const uint8_t*>(s->values), s->scales, s->meta, s->tensor_scale};
+    if (!out->meta) return SP24_ERR_INVALID_ARG;
+  }
+  if (!out->codes || !out->scales || !out->ts) return SP24_ERR_INVALID_ARG;
+  return SP24_OK;
+}
+
+}  // namespace
+
+extern "C" int sp24_moe_block(const sp24_operand* x, const int32_t* routing, const float* router_w, int64_t T,
+                              int topk, const sp24_operand* w_gate_up, const sp24_sparse_operand* w_gate_up_sparse,
+                              const sp24_operand* w_down, const sp24_sparse_operand* w_down_sparse, int64_t E,
+                              int64_t H, int64_t F, float* y, void* workspace, int64_t workspace_bytes,
+                              void* stream) {
+  if (!x) return SP24_ERR_INVALID_ARG;
+  if (T < 0 || topk < 0 || E <= 0 || H < 0 || F < 0) return SP24_ERR_SHAPE;
+  if (E > INT32_MAX || T * topk > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  if (!is16(x->format)) return SP24_ERR_DTYPE;
+  BlockW gu, dn;
+  int st = block_weights(w_gate_up, w_gate_up_sparse, &gu);
+  if (!st) st = block_weights(w_down, w_down_sparse, &dn);
+  if (st) return st;
+  const int64_t n = T * topk;
+  cudaStream_t s = as_stream(stream);
+  if (H == 0 || T == 0) return SP24_OK;
+  if (!y) return SP24_ERR_INVALID_ARG;
+  if (n == 0 || F == 0) return cudaMemsetAsync(y, 0, (size_t)(T * H) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  if (!routing || !router_w || !x->data) return SP24_ERR_INVALID_ARG;
+  if (!aligned(x->data, 16)) return SP24_ERR_ALIGN;
+  // gate/up: N = 2F rows per expert, K = H; down: N = H rows per expert, K = F
+  const int64_t bound = n / kTileTc + E;
+  if (!moe_tc_supported(gu.wf, X_16, T, E, 2 * F, H, bound, gu.codes, gu.scales, gu.meta, x->data) ||
+      !moe_tc_supported(dn.wf, X_16, T, E, H, F, bound, dn.codes, dn.scales, dn.meta, x->data))
+    return SP24_ERR_UNSUPPORTED;
+  MoeWs ws = moe_layout(workspace, T, topk, E);
+  if (!workspace || workspace_bytes < ws.bytes + block_h_bytes(T, topk, F)) return SP24_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
+  uint16_t* h = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(workspace) + ws.bytes);
+  const size_t zero_bytes = (size_t)(reinterpret_cast<uint8_t*>(ws.offsets) - reinterpret_cast<uint8_t*>(ws.counts));
+  if (cudaMemsetAsync(ws.counts, 0, zero_bytes, s) != cudaSuccess) return SP24_ERR_CUDA;
+  if (cudaMemsetAsync(y, 0, (size_t)(T * H) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
+  const int blocks = (int)((n + 255) / 256 < (int64_t)sm_count() * 4 ? (n + 255) / 256 : (int64_t)sm_count() * 4);
+  const int64_t n_tiles = bound < ws.max_tiles ? bound : ws.max_tiles;
+  route_count<<<blocks, 256, 0, s>>>(routing, n, E, ws.counts);
+  route_scan<<<1, 1024, 0, s>>>(ws.counts, E, ws.offsets, ws.tiles, ws.max_tiles, kTileTc, ws.n_tiles);
+  route_scatter<<<blocks, 256, 0, s>>>(routing, n, E, ws.offsets, ws.fill, ws.perm, nullptr, 0);
+  st = launch_status(3);
+  if (st) return st;
+  const int t16 = x->format;
+  MoeBlockGemm g{};
+  g.tiles = ws.tiles;
+  g.perm = ws.perm;
+  g.n_valid = ws.n_tiles;
+  g.topk = topk;
+  g.T = T;
+  g.E = E;
+  g.n_tiles = n_tiles;
+  // gate / up -> h
+  g.x = reinterpret_cast<const uint16_t*>(x->data);
+  g.codes = gu.codes;
+  g.scales = gu.scales;
+  g.meta = gu.meta;
+  g.w_ts = gu.ts;
+  g.h = h;
+  g.x_direct = 0;
+  g.N = 2 * F;
+  g.K = H;
+  st = moe_tc_block_gemm(1, gu.wf, t16, g, s);
+  if (st) return st;
+  // down, combined into y
+  g.x = h;
+  g.codes = dn.codes;
+  g.scales = dn.scales;
+  g.meta = dn.meta;
+  g.w_ts = dn.ts;
+  g.h = nullptr;
+  g.y = y;
+  g.router_w = router_w;
+  g.x_direct = 1;
+  g.N = H;
+  g.K = F;
+  return moe_tc_block_gemm(2, dn.wf, t16, g, s);
+}

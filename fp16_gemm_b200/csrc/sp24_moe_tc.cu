@@ -122,17 +122,27 @@ __device__ __forceinline__ void tmem_st2_nowait(uint32_t taddr, uint32_t r0, uin
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Epilogues: the routed-expert GEMM's store, the expert block's gate/up activation, and its
+// router-weighted combine.
+enum { kEpiStore = 0, kEpiGlu = 1, kEpiCombine = 2 };
+
 struct MoeTcParams {
-  const uint16_t* x;     // [T, K] 16-bit tokens
+  const uint16_t* x;     // [T, K] 16-bit tokens; with x_direct, [routed rows, K] in routed order
   const float* w_ts;     // tensor scale of the stacked experts
   const int32_t* tiles;  // (expert, first permutation index, count) per token tile
   const int32_t* perm;   // flat (token * topk + slot) of each routed row, grouped by expert
   const int32_t* n_valid;  // number of used tiles (they come first in the table)
-  float* y;              // [T, topk, N]
+  float* y;              // store: [T, topk, N];  combine: [T, N], accumulated into
+  uint16_t* h;           // glu: [routed rows, N / 2] in routed order, x's 16-bit type
+  const float* router_w; // combine: [T, topk]
+  int x_direct;          // x row of routed row p is row p (else token perm[p] / topk)
   int topk;
   int T;
   int N, K;
 };
+
+// The SwiGLU activation of the expert block: SiLU(g) * u = g / (1 + e^-g) * u, fp32.
+__device__ __forceinline__ float swiglu(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
 
 // Four E2M1 code pairs (the bytes of w, low nibble = lower K index) -> four packed 16-bit pairs
 // of the code values: exact f16 from the hardware conversion; for bf16 the same bits moved
@@ -186,7 +196,7 @@ constexpr float kMtUnscale = std::is_same<T, __nv_bfloat16>::value ? 256.0f : 1.
 // numbered t * (N / 128) + rb; the used tiles come first) and runs every ring across them, so
 // the next item's copies and conversions overlap this item's MMAs; two TMEM accumulators let the
 // epilogue warps drain one item while the MMAs fill the next.
-template <typename T, bool SP>
+template <typename T, bool SP, int EPI>
 __global__ void __launch_bounds__(kMtThreads, 1)
     moe_w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
                         const __grid_constant__ CUtensorMap tmE, const MoeTcParams p) {
@@ -415,15 +425,40 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       }
       tc_fence_after();
       const int first = s_item[j][1], count = s_item[j][2];
-      const int orow = (item_id(j) % RB) * kMtRows + 32 * qd + lane;
+      const int rb = item_id(j) % RB;
+      const int orow = rb * kMtRows + 32 * qd + lane;
 #pragma unroll 1
       for (int c = 0; 32 * c < count; ++c) {
         float v[32];
         tmem_ld32(tmem + t_lane + kMtAccCols * acc + 32 * c, v);
+        if constexpr (EPI == kEpiStore) {
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) {
-          const int i = 32 * c + ii;
-          if (i < count) p.y[(int64_t)p.perm[first + i] * p.N + orow] = v[ii] * scale;
+          for (int ii = 0; ii < 32; ++ii) {
+            const int i = 32 * c + ii;
+            if (i < count) p.y[(int64_t)p.perm[first + i] * p.N + orow] = v[ii] * scale;
+          }
+        } else if constexpr (EPI == kEpiCombine) {
+          // y[t, n] += r[t, s] * (x . w): the slots of a token meet in fp32 adds
+#pragma unroll
+          for (int ii = 0; ii < 32; ++ii) {
+            const int i = 32 * c + ii;
+            if (i < count) {
+              const int pr = p.perm[first + i];
+              atomicAdd(&p.y[(int64_t)(pr / p.topk) * p.N + orow], v[ii] * scale * p.router_w[pr]);
+            }
+          }
+        } else {
+          // gate / up packed in 16-row blocks: lanes 0-15 of this quarter hold gate rows of
+          // features f0 .. f0 + 15, lanes 16-31 the up rows of the same features
+          const int64_t f = (int64_t)rb * (kMtRows / 2) + 16 * qd + (lane & 15);
+          const int64_t F = p.N / 2;
+#pragma unroll
+          for (int ii = 0; ii < 32; ++ii) {
+            const float mine = v[ii] * scale;
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+            const int i = 32 * c + ii;
+            if (lane < 16 && i < count) p.h[(int64_t)(first + i) * F + f] = to_bits16<T>(swiglu(mine, other));
+          }
         }
       }
       tc_fence_before();
@@ -473,7 +508,8 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         for (int u = 0; u < 4; ++u) {
           const int i = (t >> 3) + 32 * u;
           xbytes[u] = i < count ? 16u : 0u;
-          xrow[u] = p.x + (i < count ? (int64_t)(p.perm[first + i] / p.topk) * p.K : 0) + 8 * j8;
+          const int64_t xr = p.x_direct ? (int64_t)(first + i) : (int64_t)(p.perm[first + i] / p.topk);
+          xrow[u] = p.x + (i < count ? xr * p.K : 0) + 8 * j8;
           nx += i < n_mma;
         }
       }
@@ -521,10 +557,10 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   }
 }
 
-template <typename T, bool SP>
+template <typename T, bool SP, int EPI>
 int launch_moe_tc(const CUtensorMap& tmC, const CUtensorMap& tmS, const CUtensorMap& tmE, const MoeTcParams& p,
                   int64_t n_items_max, cudaStream_t s) {
-  auto kern = moe_w4a16_tc_kernel<T, SP>;
+  auto kern = moe_w4a16_tc_kernel<T, SP, EPI>;
   const size_t smem = MtGeom<SP>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
@@ -535,6 +571,16 @@ int launch_moe_tc(const CUtensorMap& tmC, const CUtensorMap& tmS, const CUtensor
   if (grid > INT32_MAX) return SP24_ERR_UNSUPPORTED;
   kern<<<(unsigned)grid, kMtThreads, smem, s>>>(tmC, tmS, tmE, p);
   return launch_status();
+}
+
+template <int EPI>
+int launch_moe_tc_any(bool sparse, int t16, const CUtensorMap& tmC, const CUtensorMap& tmS, const CUtensorMap& tmE,
+                      const MoeTcParams& p, int64_t n_items_max, cudaStream_t s) {
+  if (sparse)
+    return t16 == SP24_F16 ? launch_moe_tc<__half, true, EPI>(tmC, tmS, tmE, p, n_items_max, s)
+                           : launch_moe_tc<__nv_bfloat16, true, EPI>(tmC, tmS, tmE, p, n_items_max, s);
+  return t16 == SP24_F16 ? launch_moe_tc<__half, false, EPI>(tmC, tmS, tmE, p, n_items_max, s)
+                         : launch_moe_tc<__nv_bfloat16, false, EPI>(tmC, tmS, tmE, p, n_items_max, s);
 }
 
 }  // namespace
@@ -548,6 +594,23 @@ bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_
          E * N <= INT32_MAX && max_tiles * (N / kMtRows) <= INT32_MAX && aligned(codes, 16) && aligned(scales, 16) &&
          (!sp || aligned(meta, 16)) && aligned(x, 16);
 }
+
+namespace {
+
+// Tensor maps of a stacked weight operand (dense NVFP4 codes + scales, or 2:4 values + scales +
+// nibbles) with `rows` rows of K logical entries.
+int weight_maps(bool sparse, const uint8_t* codes, const uint8_t* scales, const uint8_t* meta, uint64_t rows,
+                uint64_t K, CUtensorMap* tmC, CUtensorMap* tmS, CUtensorMap* tmE) {
+  // per row: codes K/2 (dense) or K/4 (2:4) bytes, scales K/16 or K/32, metadata K/8 (2:4)
+  const uint64_t cb = sparse ? K / 4 : K / 2, sb = sparse ? K / 32 : K / 16;
+  int st = make_tmap_2d(tmC, codes, 1, rows, cb, cb, 128, kMtRows);  // 128-byte swizzle
+  if (!st) st = make_tmap_2d_plain(tmS, scales, rows, sb, sb, 16, kMtRows);
+  if (!st) st = sparse ? make_tmap_2d_plain(tmE, meta, rows, K / 8, K / 8, 64, kMtRows) : SP24_OK;
+  if (!st && !sparse) *tmE = *tmS;  // unused
+  return st;
+}
+
+}  // namespace
 
 int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T, int64_t n_tiles,
                    const int32_t* n_valid, cudaStream_t s) {
@@ -564,21 +627,35 @@ int moe_tc_grouped(int wf, int t16, const SkinnyParams& sp, int64_t E, int64_t T
   p.T = (int)T;
   p.N = (int)sp.N;
   p.K = (int)sp.K;
-  const uint64_t rows = (uint64_t)(E * sp.N), K = (uint64_t)sp.K;
-  // per row: codes K/2 (dense) or K/4 (2:4) bytes, scales K/16 or K/32, metadata K/8 (2:4)
-  const uint64_t cb = sparse ? K / 4 : K / 2, sb = sparse ? K / 32 : K / 16;
   CUtensorMap tmC, tmS, tmE;
-  int st = make_tmap_2d(&tmC, sp.w, 1, rows, cb, cb, 128, kMtRows);  // 128-byte swizzle
-  if (!st) st = make_tmap_2d_plain(&tmS, sp.w_scales, rows, sb, sb, 16, kMtRows);
-  if (!st) st = sparse ? make_tmap_2d_plain(&tmE, sp.meta, rows, K / 8, K / 8, 64, kMtRows) : SP24_OK;
+  const int st = weight_maps(sparse, sp.w, sp.w_scales, sp.meta, (uint64_t)(E * sp.N), (uint64_t)sp.K, &tmC, &tmS, &tmE);
   if (st) return st;
-  if (!sparse) tmE = tmS;  // unused
-  const int64_t n_items_max = n_tiles * (sp.N / kMtRows);
-  if (sparse)
-    return t16 == SP24_F16 ? launch_moe_tc<__half, true>(tmC, tmS, tmE, p, n_items_max, s)
-                           : launch_moe_tc<__nv_bfloat16, true>(tmC, tmS, tmE, p, n_items_max, s);
-  return t16 == SP24_F16 ? launch_moe_tc<__half, false>(tmC, tmS, tmE, p, n_items_max, s)
-                         : launch_moe_tc<__nv_bfloat16, false>(tmC, tmS, tmE, p, n_items_max, s);
+  return launch_moe_tc_any<kEpiStore>(sparse, t16, tmC, tmS, tmE, p, n_tiles * (sp.N / kMtRows), s);
+}
+
+int moe_tc_block_gemm(int epi, int wf, int t16, const MoeBlockGemm& g, cudaStream_t s) {
+  if (g.n_tiles <= 0) return SP24_OK;
+  const bool sparse = wf == W_SQ4;
+  MoeTcParams p{};
+  p.x = g.x;
+  p.w_ts = g.w_ts;
+  p.tiles = g.tiles;
+  p.perm = g.perm;
+  p.n_valid = g.n_valid;
+  p.y = g.y;
+  p.h = g.h;
+  p.router_w = g.router_w;
+  p.x_direct = g.x_direct;
+  p.topk = g.topk;
+  p.T = (int)g.T;
+  p.N = (int)g.N;
+  p.K = (int)g.K;
+  CUtensorMap tmC, tmS, tmE;
+  const int st = weight_maps(sparse, g.codes, g.scales, g.meta, (uint64_t)(g.E * g.N), (uint64_t)g.K, &tmC, &tmS, &tmE);
+  if (st) return st;
+  const int64_t items = g.n_tiles * (g.N / kMtRows);
+  if (epi == kEpiGlu) return launch_moe_tc_any<kEpiGlu>(sparse, t16, tmC, tmS, tmE, p, items, s);
+  return launch_moe_tc_any<kEpiCombine>(sparse, t16, tmC, tmS, tmE, p, items, s);
 }
 
 }  // namespace sp24

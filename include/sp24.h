@@ -292,6 +292,35 @@ int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, int64_t T, 
                       int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                       void* stream);
 
+/* Expert block of the routed model ([P1] "Concurrency, not sparsity, is the lever"): for each
+ * token t,  y[t] = sum_s r[t, s] * h_ts Wd_e^T  with  h_ts = SiLU(x_t Wg_e^T) * (x_t Wu_e^T),
+ * e = routing[t, s]; SiLU(g) = g / (1 + e^-g).  h is held in x's 16-bit type; y is fp32.
+ *   x          T rows of H entries, F16 or BF16, 16-byte aligned
+ *   routing    device int32 [T, topk];  router_w: device fp32 [T, topk]
+ *   w_gate_up  the E experts' gate and up weights [E * 2F, H], NVFP4, packed by
+ *              sp24_interleave_rows(gate, up, block_rows = 16): rows 32k .. 32k + 15 are gate
+ *              rows 16k .. 16k + 15, rows 32k + 16 .. 32k + 31 the up rows of the same features;
+ *              gate and up share one tensor scale (sp24_nvfp4_group_tensor_scale); exactly one
+ *              of w_gate_up (dense) or w_gate_up_sparse (2:4 values + nibbles, same packing)
+ *   w_down     [E * H, F], NVFP4 dense or 2:4 (w_down_sparse), one of the two
+ *   y          device fp32 [T, H], overwritten
+ *   Shapes: F % 64 and H % 128; dense K (H for gate/up, F for down) % 256, 2:4 K % 512;
+ *   SP24_ERR_UNSUPPORTED otherwise.  Slots of a token are summed with fp32 atomics (the order,
+ *   and so the last bits, may vary between calls).
+ *   workspace: sp24_moe_block_workspace_size() bytes, 16-byte aligned (routing tables and h). */
+int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t F, int64_t* bytes);
+int sp24_moe_block(const sp24_operand* x, const int32_t* routing, const float* router_w, int64_t T,
+                   int topk, const sp24_operand* w_gate_up,
+                   const sp24_sparse_operand* w_gate_up_sparse, const sp24_operand* w_down,
+                   const sp24_sparse_operand* w_down_sparse, int64_t E, int64_t H, int64_t F,
+                   float* y, void* workspace, int64_t workspace_bytes, void* stream);
+
+/* Row interleave: out[2 * rows, row_bytes] takes block_rows rows of a, then block_rows rows of
+ * b, and so on (the gate / up packing of sp24_moe_block).  rows % block_rows == 0, row_bytes % 16
+ * == 0, all pointers device and 16-byte aligned. */
+int sp24_interleave_rows(const void* a, const void* b, int64_t rows, int64_t row_bytes,
+                         int64_t block_rows, void* out, void* stream);
+
 /* ----------------------------------------------------------------------- diagnostics */
 /* Number of kernels this library has launched in this process (host-side counter, all
  * devices and streams).  For accounting in benchmarks; memsets are not counted. */

@@ -296,3 +296,36 @@ def within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, s_ref: np.ndarray, re
     err = np.abs(y_gpu - y_ref)
     ok = np.where(s_ref > 0, err <= rel * s_ref, y_gpu == 0)
     return ok
+
+
+def round_to_16(x: np.ndarray, dtype: int) -> np.ndarray:
+    """fp64 values held in a 16-bit type (round to nearest even; through fp32 for bf16), as fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == F16:
+        return x.astype(np.float16).astype(np.float64)
+    u = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def moe_block(X: np.ndarray, routing: np.ndarray, router_w: np.ndarray, Wg: np.ndarray, Wu: np.ndarray,
+              Wd: np.ndarray, hdtype: int):
+    """(Y, S) of the routed expert block on decoded fp64 operands ([P1] "Concurrency, not sparsity,
+    is the lever"): for each token t and slot s with expert e = routing[t, s],
+    h = SiLU(Wg[e] x_t) * (Wu[e] x_t) held in the 16-bit type `hdtype`, and
+    Y[t] = sum_s router_w[t, s] * Wd[e] h;  S[t] = sum_s |router_w| |Wd[e]| |h| (tolerance scale).
+    X [T, H]; Wg, Wu [E, F, H]; Wd [E, H, F]."""
+    T, topk = routing.shape
+    H = X.shape[1]
+    Y = np.zeros((T, H))
+    S = np.zeros((T, H))
+    for t in range(T):
+        for s in range(topk):
+            e = int(routing[t, s])
+            r = float(router_w[t, s])
+            g = Wg[e] @ X[t]
+            u = Wu[e] @ X[t]
+            h = round_to_16(g / (1.0 + np.exp(-g)) * u, hdtype)
+            Y[t] += r * (Wd[e] @ h)
+            S[t] += abs(r) * (np.abs(Wd[e]) @ np.abs(h))
+    return Y, S

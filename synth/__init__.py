@@ -18,6 +18,8 @@ Workloads (the shapes the pages' workloads take; see the design notes for the ma
                      without replacement.
 * ``moe_skewed``:    W bf16 [E, N, K] N(0, 0.02), X [T, K] N(0, 1), routing with given per-expert
                      row counts in a seeded random order (tile-boundary parity cases).
+* ``moe_block``:     Wg, Wu bf16 [E, F, H], Wd bf16 [E, H, F] N(0, 0.02) expert by expert, X bf16
+                     [T, H] N(0, 1), top-k routing, router weights uniform normalised per token.
 * ``output_head``:   W bf16 [151936, 4096] N(0, 0.02) (an output head of ~1.16 GiB: the pages'
                      large single-tensor quantisation), drawn in row chunks.
 * ``qkv_group``:     Wq [2048, 2048], Wk, Wv [512, 2048] N(0, 0.02), one x40 outlier in Wv (a
@@ -135,6 +137,24 @@ def qkv_group(seed: int = SEED, hidden: int = 2048, kv: int = 512, dtype: str = 
     i = int(g.integers(0, Wv.size))
     Wv.flat[i] *= 40.0
     return {"Wq": as_storage(Wq, dtype), "Wk": as_storage(Wk, dtype), "Wv": as_storage(Wv, dtype)}
+
+
+def moe_block(seed: int = SEED, E: int = 512, H: int = 2048, F: int = 512, T: int = 4096, topk: int = 10):
+    """Expert block: Wg, Wu [E, F, H] and Wd [E, H, F] bf16 N(0, 0.02) (drawn in that order,
+    expert by expert), X bf16 [T, H] N(0, 1), routing [T, topk] (distinct experts per token,
+    uniform), router weights fp32 [T, topk]: uniform draws normalised to sum 1 per token."""
+    g = rng(seed)
+    Wg = np.empty((E, F, H), dtype=np.uint16)
+    Wu = np.empty((E, F, H), dtype=np.uint16)
+    Wd = np.empty((E, H, F), dtype=np.uint16)
+    for W, shape in ((Wg, (F, H)), (Wu, (F, H)), (Wd, (H, F))):
+        for e in range(E):
+            W[e] = draw(g, shape, "bf16", 0.02)
+    X = draw(g, (T, H), "bf16")
+    routing = routing_topk(g, T, E, topk)
+    r = g.random(size=(T, topk))
+    r = (r / r.sum(axis=1, keepdims=True)).astype(np.float32)
+    return {"Wg": Wg, "Wu": Wu, "Wd": Wd, "X": X, "routing": routing, "router_w": r}
 
 
 def moe_skewed(counts, seed: int = SEED, N: int = 256, K: int = 320, topk: int = 2,

@@ -477,3 +477,54 @@ def test_moe_generator_matches_one_draw():
     W = synth.draw(g, (3, 4, 16), "bf16", 0.02)
     X = synth.draw(g, (5, 16), "bf16")
     assert np.array_equal(d["W"], W) and np.array_equal(d["X"], X)
+
+
+# ----------------------------------------------------------------------------- expert block
+
+
+def test_moe_block_hand_example(oracle):
+    """A hand-computed block: x = [1, 2]; gate row [1, 0] gives g = 1, up row [0, 1] gives u = 2,
+    so h = SiLU(1) * 2 = 2 / (1 + e^-1) = 1.46211716..., held in bf16 as 1.4609375 (8 significant
+    bits: 1 + 59/128); down rows [3] and [-1], router weight 0.5: y = [2.19140625, -0.73046875]."""
+    X = np.array([[1.0, 2.0]])
+    Wg = np.array([[[1.0, 0.0]]])
+    Wu = np.array([[[0.0, 1.0]]])
+    Wd = np.array([[[3.0], [-1.0]]])
+    Y, S = oracle.moe_block(X, np.array([[0]]), np.array([[0.5]]), Wg, Wu, Wd, oracle.BF16)
+    assert Y.tolist() == [[2.19140625, -0.73046875]]
+    assert S.tolist() == [[2.19140625, 0.73046875]]
+    # in f16 h keeps 11 bits: 1.4619140625 (1 + 473/1024)
+    Y16, _ = oracle.moe_block(X, np.array([[0]]), np.array([[1.0]]), Wg, Wu, Wd, oracle.F16)
+    assert Y16.tolist() == [[3 * 1.4619140625, -1.4619140625]]
+
+
+def test_moe_block_silu_zero_and_linearity(oracle):
+    """SiLU(0) = 0: a zero gate row silences its feature whatever up and down hold; y is linear in
+    the router weights, and two slots on one expert add."""
+    g = synth.rng(43)
+    X = synth.normal(g, (3, 8))
+    Wg, Wu, Wd = synth.normal(g, (2, 4, 8)), synth.normal(g, (2, 4, 8)), synth.normal(g, (2, 8, 4))
+    Wg0 = Wg.copy()
+    Wg0[:, 1] = 0.0
+    Wd1 = Wd.copy()
+    Wd1[:, :, 1] += 100.0  # only feature 1 reads these columns
+    rt = np.array([[0, 1], [1, 1], [0, 0]])
+    rw = synth.normal(g, (3, 2))
+    a, _ = oracle.moe_block(X, rt, rw, Wg0, Wu, Wd, oracle.F16)
+    b, _ = oracle.moe_block(X, rt, rw, Wg0, Wu, Wd1, oracle.F16)
+    assert np.array_equal(a, b)
+    c, _ = oracle.moe_block(X, rt, 2 * rw, Wg, Wu, Wd, oracle.F16)
+    d, _ = oracle.moe_block(X, rt, rw, Wg, Wu, Wd, oracle.F16)
+    assert np.allclose(c, 2 * d, rtol=1e-15, atol=0)
+    one, _ = oracle.moe_block(X[:1], np.array([[1]]), rw[1:2, :1], Wg, Wu, Wd, oracle.F16)
+    two, _ = oracle.moe_block(X[:1], np.array([[1, 1]]), np.array([[rw[1, 0], rw[1, 0]]]), Wg, Wu, Wd, oracle.F16)
+    assert np.allclose(two, 2 * one, rtol=1e-15, atol=0)
+
+
+def test_round_to_16_against_ml_dtypes(oracle):
+    """The block's 16-bit hold of h: round to nearest even, checked against ml_dtypes' casts."""
+    x = synth.normal(synth.rng(44), 4096) * np.exp(3 * synth.normal(synth.rng(45), 4096))
+    bf = np.asarray(x.astype(np.float32).astype(ml_dtypes.bfloat16), dtype=np.float64)
+    assert np.array_equal(oracle.round_to_16(x, oracle.BF16), bf)
+    assert np.array_equal(oracle.round_to_16(x, oracle.F16), x.astype(np.float16).astype(np.float64))
+
