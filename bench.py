@@ -578,6 +578,46 @@ def run_sweep(args) -> None:
                           "compress": {"us": round(us_p, 3), "GB/s": round((nb + vals.numel() * 2 + meta.numel()) / us_p / 1e3, 1)},
                           "n_fail": int(nf.item())}), flush=True)
 
+    # routed expert block: 512 experts (gate/up [1024, 2048] packed, down [2048, 512]), 4096 bf16
+    # tokens top-10, NVFP4 experts dense or 2:4; FLOPs 6 T topk H F; bytes: weights once, x, y,
+    # h written and read once, the per-slot outputs written and read once (routing tables excluded)
+    d = synth.moe_block()
+    E, F, H = d["Wg"].shape
+    xb = t16(d["X"], "bf16")
+    rtb = torch.from_numpy(d["routing"]).to(dev)
+    rwb = torch.from_numpy(d["router_w"]).to(dev)
+    Tb, kb = rtb.shape
+    wg = t16(d["Wg"].reshape(E * F, H), "bf16")
+    wu = t16(d["Wu"].reshape(E * F, H), "bf16")
+    wdn = t16(d["Wd"].reshape(E * H, F), "bf16")
+    del d
+    tsd = sp.nvfp4_group_tensor_scale([wg, wu])
+    gu_d = sp.pack_gate_up(sp.quantize_nvfp4(wg, tsd), sp.quantize_nvfp4(wu, tsd))
+    dn_d = sp.quantize_nvfp4(wdn)
+    (vg, mg), (vu, mu) = sp.prune_compress_24(wg), sp.prune_compress_24(wu)
+    del wg, wu
+    tss = sp.nvfp4_group_tensor_scale([vg, vu])
+    gu_s = sp.pack_gate_up(sp.Sparse24(sp.quantize_nvfp4(vg, tss), mg), sp.Sparse24(sp.quantize_nvfp4(vu, tss), mu))
+    del vg, vu
+    vd, md = sp.prune_compress_24(wdn)
+    dn_s = sp.Sparse24(sp.quantize_nvfp4(vd), md)
+    del wdn, vd
+    yb = torch.empty((Tb, H), dtype=torch.float32, device=dev)
+    wsb = torch.empty(sp.moe_block_workspace_bytes(Tb, kb, E, H, F), dtype=torch.uint8, device=dev)
+    flb = 6.0 * Tb * kb * H * F
+    xyh = Tb * H * 2 + Tb * H * 4 + 2 * Tb * kb * F * 2 + 2 * Tb * kb * H * 4
+    line = {"sweep": "moe_block", "experts": E, "hidden": H, "inter": F, "tokens": Tb, "topk": kb, "x": "bf16",
+            "w": "nvfp4", "flop": flb}
+    for name, (gop, dop) in (("dense", (gu_d, dn_d)), ("sparse24", (gu_s, dn_s))):
+        us = timeit(lambda r: sp.moe_block(xb, rtb, rwb, gop, dop, E, H, F, out=yb, workspace=wsb), reps=3)
+        byt = op_bytes(gop) + op_bytes(dop) + xyh
+        line[name] = {"us": round(us, 1), "TFLOP/s": round(flb / us / 1e6, 1), "GB/s": round(byt / us / 1e3, 1),
+                      "bytes": byt, "frac_hbm": round(byt / us / 1e3 / peak_hbm, 3),
+                      "frac_tensor": round(flb / us / 1e6 / tensor_peak["f16"], 3)}
+    line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse24"]["us"], 3)
+    print(json.dumps(line), flush=True)
+    del gu_d, dn_d, gu_s, dn_s, xb, yb, wsb
+
     # large single-tensor quantisation: a [151936, 4096] bf16 output head (~1.16 GiB -> 0.33 GiB
     # of codes + scales).  Full call: amax pass + encode pass (the tensor is 10x the L2, so it is
     # read twice); with a supplied (group-shared) scale: one pass; the group scale alone: one read.

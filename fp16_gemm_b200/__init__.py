@@ -104,7 +104,7 @@ def lib() -> ctypes.CDLL:
             L.sp24_gemm_auto.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_Operand),
                                          ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P, P]
             L.sp24_gemm_choice_reset.argtypes = []
-            L.sp24_moe_block_workspace_size.argtypes = [I64, I, I64, I64, P]
+            L.sp24_moe_block_workspace_size.argtypes = [I64, I, I64, I64, I64, P]
             L.sp24_moe_block.argtypes = [ctypes.POINTER(_Operand), P, P, I64, I, ctypes.POINTER(_Operand),
                                          ctypes.POINTER(_SparseOperand), ctypes.POINTER(_Operand),
                                          ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
@@ -590,9 +590,9 @@ def pack_gate_up(gate, up, stream=None):
                        _interleave(gate.scales, up.scales, rows, stream=stream), gate.tensor_scale.clone())
 
 
-def moe_block_workspace_bytes(T: int, topk: int, E: int, F: int) -> int:
+def moe_block_workspace_bytes(T: int, topk: int, E: int, H: int, F: int) -> int:
     n = ctypes.c_int64(0)
-    _call("sp24_moe_block_workspace_size", T, topk, E, F, ctypes.byref(n))
+    _call("sp24_moe_block_workspace_size", T, topk, E, H, F, ctypes.byref(n))
     return n.value
 
 
@@ -607,7 +607,7 @@ def moe_block(x: torch.Tensor, routing: torch.Tensor, router_w: torch.Tensor, w_
     if out is None:
         out = torch.empty((T, H), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = torch.empty(moe_block_workspace_bytes(T, topk, E, F), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(moe_block_workspace_bytes(T, topk, E, H, F), dtype=torch.uint8, device=dev)
     xo = _operand(x)
     gd = gs = dd = ds = None
     if isinstance(w_gate_up, Sparse24):

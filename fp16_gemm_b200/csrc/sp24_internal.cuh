@@ -127,8 +127,8 @@ bool moe_tc_supported(int wf, int x_fmt, int64_t T, int64_t E, int64_t N, int64_
 int moe_tc_grouped(int wf, int t16, const SkinnyParams& p, int64_t E, int64_t T, int64_t n_tiles,
                    const int32_t* n_valid, cudaStream_t s);
 // One GEMM of the expert block on the same kernel: epi 1 = gate/up (weights packed in 16-row
-// gate / up blocks, output h = SiLU(gate) * up in x's 16-bit type, routed order), epi 2 = down
-// (x = h rows in routed order, output y[T, N] += router weight * product).
+// gate / up blocks, output h = SiLU(gate) * up in x's 16-bit type, routed order), epi 0 = down
+// (x = h rows in routed order, output stored as y[T, topk, N]).
 struct MoeBlockGemm {
   const uint16_t* x;
   const uint8_t *codes, *scales, *meta;
@@ -136,7 +136,6 @@ struct MoeBlockGemm {
   const int32_t *tiles, *perm, *n_valid;
   float* y;
   uint16_t* h;
-  const float* router_w;
   int x_direct, topk;
   int64_t T, E, N, K, n_tiles;
 };

@@ -262,8 +262,9 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
 // ([P1] "Concurrency, not sparsity, is the lever": the routed experts of a decode step).
 // Routing as for sp24_gemm_grouped (tiles of up to 128 routed rows), then the tensor-core
 // kernel twice: gate/up (weights packed as 16-row gate / up blocks, SwiGLU in the epilogue, h in
-// x's 16-bit type and routed order) and down (h rows read directly, router weight and fp32 add
-// into y in the epilogue).
+// x's 16-bit type and routed order) and down (h rows read directly, each routed row's output
+// stored once), then a streaming kernel sums each token's slots in order with the router weights
+// (fp32, deterministic).
 
 namespace sp24 {
 namespace {
@@ -280,6 +281,26 @@ __global__ void interleave_rows_kernel(const uint4* __restrict__ a, const uint4*
 }
 
 int64_t block_h_bytes(int64_t T, int topk, int64_t F) { return (T * topk * F * 2 + 15) / 16 * 16; }
+int64_t block_o_bytes(int64_t T, int topk, int64_t H) { return T * topk * H * 4; }
+
+// y[t, n] = sum_s r[t, s] * o[t, s, n], the slots in order (fp32): four outputs per thread.
+__global__ void combine_kernel(const float4* __restrict__ o, const float* __restrict__ r, int64_t T, int topk,
+                               int64_t H4, float4* __restrict__ y) {
+  const int64_t n = T * H4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / H4, c = i - t * H4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < topk; ++s) {
+      const float w = r[t * topk + s];
+      const float4 v = __ldcs(o + (t * topk + s) * H4 + c);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    y[i] = acc;
+  }
+}
 
 }  // namespace
 }  // namespace sp24
@@ -299,10 +320,10 @@ extern "C" int sp24_interleave_rows(const void* a, const void* b, int64_t rows, 
   return launch_status();
 }
 
-extern "C" int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t F, int64_t* bytes) {
+extern "C" int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t H, int64_t F, int64_t* bytes) {
   if (!bytes) return SP24_ERR_INVALID_ARG;
-  if (T < 0 || topk < 0 || E <= 0 || F < 0) return SP24_ERR_SHAPE;
-  *bytes = moe_layout(nullptr, T, topk, E).bytes + block_h_bytes(T, topk, F);
+  if (T < 0 || topk < 0 || E <= 0 || H < 0 || F < 0) return SP24_ERR_SHAPE;
+  *bytes = moe_layout(nullptr, T, topk, E).bytes + block_h_bytes(T, topk, F) + block_o_bytes(T, topk, H);
   return SP24_OK;
 }
 
@@ -357,12 +378,13 @@ extern "C" int sp24_moe_block(const sp24_operand* x, const int32_t* routing, con
       !moe_tc_supported(dn.wf, X_16, T, E, H, F, bound, dn.codes, dn.scales, dn.meta, x->data))
     return SP24_ERR_UNSUPPORTED;
   MoeWs ws = moe_layout(workspace, T, topk, E);
-  if (!workspace || workspace_bytes < ws.bytes + block_h_bytes(T, topk, F)) return SP24_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < ws.bytes + block_h_bytes(T, topk, F) + block_o_bytes(T, topk, H))
+    return SP24_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
   uint16_t* h = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(workspace) + ws.bytes);
+  float* o = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + ws.bytes + block_h_bytes(T, topk, F));
   const size_t zero_bytes = (size_t)(reinterpret_cast<uint8_t*>(ws.offsets) - reinterpret_cast<uint8_t*>(ws.counts));
   if (cudaMemsetAsync(ws.counts, 0, zero_bytes, s) != cudaSuccess) return SP24_ERR_CUDA;
-  if (cudaMemsetAsync(y, 0, (size_t)(T * H) * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
   const int blocks = (int)((n + 255) / 256 < (int64_t)sm_count() * 4 ? (n + 255) / 256 : (int64_t)sm_count() * 4);
   const int64_t n_tiles = bound < ws.max_tiles ? bound : ws.max_tiles;
   route_count<<<blocks, 256, 0, s>>>(routing, n, E, ws.counts);
@@ -391,17 +413,22 @@ extern "C" int sp24_moe_block(const sp24_operand* x, const int32_t* routing, con
   g.K = H;
   st = moe_tc_block_gemm(1, gu.wf, t16, g, s);
   if (st) return st;
-  // down, combined into y
+  // down -> o[t, s, :] (every routed row's output stored once), then the slots combined in order
   g.x = h;
   g.codes = dn.codes;
   g.scales = dn.scales;
   g.meta = dn.meta;
   g.w_ts = dn.ts;
   g.h = nullptr;
-  g.y = y;
-  g.router_w = router_w;
+  g.y = o;
   g.x_direct = 1;
   g.N = H;
   g.K = F;
-  return moe_tc_block_gemm(2, dn.wf, t16, g, s);
+  st = moe_tc_block_gemm(0, dn.wf, t16, g, s);
+  if (st) return st;
+  const int64_t nvec = T * (H / 4);
+  const int64_t cb = (nvec + 255) / 256 < (int64_t)sm_count() * 8 ? (nvec + 255) / 256 : (int64_t)sm_count() * 8;
+  combine_kernel<<<(unsigned)cb, 256, 0, s>>>(reinterpret_cast<const float4*>(o), router_w, T, topk, H / 4,
+                                              reinterpret_cast<float4*>(y));
+  return launch_status();
 }

@@ -59,7 +59,7 @@ constexpr int kMtEpiWarps = 4;
 constexpr int kMtWarpMma = kMtConvWarps, kMtWarpW = kMtConvWarps + 1, kMtWarpX0 = kMtConvWarps + 2;
 constexpr int kMtWarpEpi0 = kMtWarpX0 + kMtGatherWarps;
 constexpr int kMtThreads = 32 * (kMtWarpEpi0 + kMtEpiWarps);
-constexpr int kMtMaxItems = 64;   // items per CTA (the host sizes the grid for it)
+constexpr int kMtMaxItems = 256;  // items per CTA (the host sizes the grid for it)
 constexpr uint32_t kMtX = kMtTok * kMtBK * 2;              // 16 KB
 constexpr uint32_t kMtAccCols = 128;                       // fp32 accumulator, one column per routed row (two of them)
 constexpr uint32_t kMtCols = 512;
@@ -122,9 +122,9 @@ __device__ __forceinline__ void tmem_st2_nowait(uint32_t taddr, uint32_t r0, uin
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Epilogues: the routed-expert GEMM's store, the expert block's gate/up activation, and its
-// router-weighted combine.
-enum { kEpiStore = 0, kEpiGlu = 1, kEpiCombine = 2 };
+// Epilogues: the routed-expert GEMM's store (also the expert block's down projection) and the
+// expert block's gate/up activation.
+enum { kEpiStore = 0, kEpiGlu = 1 };
 
 struct MoeTcParams {
   const uint16_t* x;     // [T, K] 16-bit tokens; with x_direct, [routed rows, K] in routed order
@@ -132,9 +132,8 @@ struct MoeTcParams {
   const int32_t* tiles;  // (expert, first permutation index, count) per token tile
   const int32_t* perm;   // flat (token * topk + slot) of each routed row, grouped by expert
   const int32_t* n_valid;  // number of used tiles (they come first in the table)
-  float* y;              // store: [T, topk, N];  combine: [T, N], accumulated into
+  float* y;              // store: [T, topk, N]
   uint16_t* h;           // glu: [routed rows, N / 2] in routed order, x's 16-bit type
-  const float* router_w; // combine: [T, topk]
   int x_direct;          // x row of routed row p is row p (else token perm[p] / topk)
   int topk;
   int T;
@@ -437,27 +436,21 @@ __global__ void __launch_bounds__(kMtThreads, 1)
             const int i = 32 * c + ii;
             if (i < count) p.y[(int64_t)p.perm[first + i] * p.N + orow] = v[ii] * scale;
           }
-        } else if constexpr (EPI == kEpiCombine) {
-          // y[t, n] += r[t, s] * (x . w): the slots of a token meet in fp32 adds
-#pragma unroll
-          for (int ii = 0; ii < 32; ++ii) {
-            const int i = 32 * c + ii;
-            if (i < count) {
-              const int pr = p.perm[first + i];
-              atomicAdd(&p.y[(int64_t)(pr / p.topk) * p.N + orow], v[ii] * scale * p.router_w[pr]);
-            }
-          }
         } else {
           // gate / up packed in 16-row blocks: lanes 0-15 of this quarter hold gate rows of
-          // features f0 .. f0 + 15, lanes 16-31 the up rows of the same features
+          // features f0 .. f0 + 15, lanes 16-31 the up rows of the same features.  Lanes 0-15
+          // evaluate even tokens, lanes 16-31 odd ones (one exchange per token pair: each half
+          // sends what the other half lacks)
           const int64_t f = (int64_t)rb * (kMtRows / 2) + 16 * qd + (lane & 15);
           const int64_t F = p.N / 2;
+          const bool lo = lane < 16;
 #pragma unroll
-          for (int ii = 0; ii < 32; ++ii) {
-            const float mine = v[ii] * scale;
-            const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-            const int i = 32 * c + ii;
-            if (lane < 16 && i < count) p.h[(int64_t)(first + i) * F + f] = to_bits16<T>(swiglu(mine, other));
+          for (int ii = 0; ii < 32; ii += 2) {
+            const float a = v[ii] * scale, b = v[ii + 1] * scale;
+            const float got = __shfl_xor_sync(0xffffffffu, lo ? b : a, 16);
+            const int i = 32 * c + ii + (lo ? 0 : 1);
+            const float hv = lo ? swiglu(a, got) : swiglu(got, b);  // (gate, up) of token i
+            if (i < count) p.h[(int64_t)(first + i) * F + f] = to_bits16<T>(hv);
           }
         }
       }
@@ -644,7 +637,6 @@ int moe_tc_block_gemm(int epi, int wf, int t16, const MoeBlockGemm& g, cudaStrea
   p.n_valid = g.n_valid;
   p.y = g.y;
   p.h = g.h;
-  p.router_w = g.router_w;
   p.x_direct = g.x_direct;
   p.topk = g.topk;
   p.T = (int)g.T;
@@ -655,7 +647,8 @@ int moe_tc_block_gemm(int epi, int wf, int t16, const MoeBlockGemm& g, cudaStrea
   if (st) return st;
   const int64_t items = g.n_tiles * (g.N / kMtRows);
   if (epi == kEpiGlu) return launch_moe_tc_any<kEpiGlu>(sparse, t16, tmC, tmS, tmE, p, items, s);
-  return launch_moe_tc_any<kEpiCombine>(sparse, t16, tmC, tmS, tmE, p, items, s);
+  if (epi == kEpiStore) return launch_moe_tc_any<kEpiStore>(sparse, t16, tmC, tmS, tmE, p, items, s);
+  return SP24_ERR_INVALID_ARG;
 }
 
 }  // namespace sp24

@@ -305,10 +305,12 @@ int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, int64_t T, 
  *   w_down     [E * H, F], NVFP4 dense or 2:4 (w_down_sparse), one of the two
  *   y          device fp32 [T, H], overwritten
  *   Shapes: F % 64 and H % 128; dense K (H for gate/up, F for down) % 256, 2:4 K % 512;
- *   SP24_ERR_UNSUPPORTED otherwise.  Slots of a token are summed with fp32 atomics (the order,
- *   and so the last bits, may vary between calls).
- *   workspace: sp24_moe_block_workspace_size() bytes, 16-byte aligned (routing tables and h). */
-int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t F, int64_t* bytes);
+ *   SP24_ERR_UNSUPPORTED otherwise.  Each routed row's down output is stored once and a token's
+ *   slots are summed in slot order in fp32 (deterministic).
+ *   workspace: sp24_moe_block_workspace_size() bytes, 16-byte aligned (routing tables, h in
+ *   x's type [T*topk, F], the per-slot outputs fp32 [T, topk, H]). */
+int sp24_moe_block_workspace_size(int64_t T, int topk, int64_t E, int64_t H, int64_t F,
+                                  int64_t* bytes);
 int sp24_moe_block(const sp24_operand* x, const int32_t* routing, const float* router_w, int64_t T,
                    int topk, const sp24_operand* w_gate_up,
                    const sp24_sparse_operand* w_gate_up_sparse, const sp24_operand* w_down,
