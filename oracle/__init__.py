@@ -67,6 +67,10 @@ def lib():
                 getattr(L, f).argtypes = [P, I, I, P, I, P]
             L.sp24o_compress_24.argtypes = [P, I, I, P, I, P, P]
             L.sp24o_decompress_24.argtypes = [P, P, I, I, P, I, P]
+            L.sp24o_check_48.restype = I64
+            L.sp24o_check_48.argtypes = [P, I, I64, I64, P]
+            L.sp24o_compress_48.argtypes = [P, I, I64, I64, P, P]
+            L.sp24o_decompress_48.argtypes = [P, P, I, I64, I64, P]
             L.sp24o_e2m1_value.restype = ctypes.c_double
             L.sp24o_e2m1_value.argtypes = [I]
             L.sp24o_e4m3_value.restype = ctypes.c_double
@@ -180,6 +184,38 @@ def decompress_24(values: np.ndarray, meta: np.ndarray, dtype: int, shape, op: i
     out = np.empty(tuple(shape), dtype=values.dtype)
     _check(lib().sp24o_decompress_24(_ptr(values), _ptr(meta), dtype, op, _ptr(_shape(shape)),
                                      len(shape), _ptr(out)), "decompress_24")
+    return out.view(kind)
+
+
+def check_48(w: np.ndarray, dtype: int):
+    """Pairwise 4:8 eligibility of W[rows, K] (chunks of 8 along K): pass map [rows, K/8], fails."""
+    w = _bits(w, dtype)
+    rows, K = w.shape
+    pass_ = np.zeros((rows, K // 8), dtype=np.uint8)
+    n = lib().sp24o_check_48(_ptr(w), dtype, rows, K, _ptr(pass_))
+    if n < 0:
+        raise OracleError(f"check_48: oracle returned {n}")
+    return pass_, int(n)
+
+
+def compress_48(w: np.ndarray, dtype: int):
+    """(values [rows, K/2] in the caller's storage type, meta nibble stream) of pairwise 4:8."""
+    kind = np.asarray(w).dtype
+    w = _bits(w, dtype)
+    rows, K = w.shape
+    values = np.empty((rows, K // 2), dtype=w.dtype)
+    meta = np.empty((rows * (K // 8) + 1) // 2, dtype=np.uint8)
+    _check(lib().sp24o_compress_48(_ptr(w), dtype, rows, K, _ptr(values), _ptr(meta)), "compress_48")
+    return values.view(kind), meta
+
+
+def decompress_48(values: np.ndarray, meta: np.ndarray, dtype: int, shape):
+    kind = np.asarray(values).dtype
+    values = _bits(values, dtype)
+    meta = np.ascontiguousarray(meta, dtype=np.uint8)
+    rows, K = shape
+    out = np.empty((rows, K), dtype=values.dtype)
+    _check(lib().sp24o_decompress_48(_ptr(values), _ptr(meta), dtype, rows, K, _ptr(out)), "decompress_48")
     return out.view(kind)
 
 

@@ -266,6 +266,101 @@ int sp24o_decompress_24(const void* values, const uint8_t* meta, int dtype, int 
   return O_OK;
 }
 
+/* ---------------------------------------------------------------- pairwise 4:8 */
+
+/* Pairwise 4:8, the sparse pattern of the tensor cores' packed-FP4 kind, per reading R21: along
+ * K, chunks of 8 consecutive entries, each made of four pairs (2j, 2j + 1).  A chunk is eligible
+ * when at most two of its pairs hold a nonzero entry (+0 and -0 are zero).  Pruning keeps the two
+ * pairs of largest score |a| + |b| (one IEEE fp32 addition of the entries' fp32 magnitudes), NaN
+ * scores above every number, ties to the lower pair.  The compressed chunk is its kept pairs in
+ * ascending order (values [rows, K/2]) plus a nibble i0 | i1 << 2 (pair indices, i0 < i1), chunk
+ * 2c of the flat chunk sequence in the low nibble of byte c. */
+
+/* Does pair a (score sa, index ia) come before pair b in the keep order? */
+static int pair_before(float sa, int ia, float sb, int ib) {
+  int na = isnan(sa), nb = isnan(sb);
+  if (na != nb) return na;
+  if (!na && sa != sb) return sa > sb;
+  return ia < ib;
+}
+
+static void kept_pairs48(const void* w, int dtype, int64_t base, int* i0, int* i1) {
+  float sc[4];
+  for (int j = 0; j < 4; ++j) {
+    volatile float a = fabsf(elem_f32(w, dtype, base + 2 * j));
+    volatile float b = fabsf(elem_f32(w, dtype, base + 2 * j + 1));
+    volatile float sum = a + b;
+    sc[j] = sum;
+  }
+  int kept[2], nk = 0;
+  for (int i = 0; i < 4; ++i) {
+    int rank = 0;
+    for (int j = 0; j < 4; ++j)
+      if (j != i && pair_before(sc[j], j, sc[i], i)) rank++;
+    if (rank < 2) kept[nk++] = i;
+  }
+  *i0 = kept[0];
+  *i1 = kept[1];
+}
+
+/* Per-chunk pass map [rows, K/8] (may be NULL); returns the failing-chunk count or -code. */
+int64_t sp24o_check_48(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* pass) {
+  if (!elem_bytes(dtype)) return -O_EDTYPE;
+  if (rows < 0 || K < 0 || K % 8) return -O_ESHAPE;
+  int64_t fails = 0;
+  for (int64_t c = 0; c < rows * (K / 8); ++c) {
+    int nonzero_pairs = 0;
+    for (int j = 0; j < 4; ++j) {
+      uint32_t a = mag_bits(raw_bits(w, dtype, 8 * c + 2 * j), dtype);
+      uint32_t b = mag_bits(raw_bits(w, dtype, 8 * c + 2 * j + 1), dtype);
+      if (a || b) nonzero_pairs++;
+    }
+    int ok = nonzero_pairs <= 2;
+    if (pass) pass[c] = (uint8_t)ok;
+    if (!ok) fails++;
+  }
+  return fails;
+}
+
+int sp24o_compress_48(const void* w, int dtype, int64_t rows, int64_t K, void* values, uint8_t* meta) {
+  if (!elem_bytes(dtype)) return O_EDTYPE;
+  if (rows < 0 || K < 0 || K % 8) return O_ESHAPE;
+  const int64_t C = rows * (K / 8);
+  memset(meta, 0, (size_t)((C + 1) / 2));
+  for (int64_t c = 0; c < C; ++c) {
+    int i0, i1;
+    kept_pairs48(w, dtype, 8 * c, &i0, &i1);
+    put_raw_bits(values, dtype, 4 * c + 0, raw_bits(w, dtype, 8 * c + 2 * i0));
+    put_raw_bits(values, dtype, 4 * c + 1, raw_bits(w, dtype, 8 * c + 2 * i0 + 1));
+    put_raw_bits(values, dtype, 4 * c + 2, raw_bits(w, dtype, 8 * c + 2 * i1));
+    put_raw_bits(values, dtype, 4 * c + 3, raw_bits(w, dtype, 8 * c + 2 * i1 + 1));
+    uint8_t nib = (uint8_t)(i0 | (i1 << 2));
+    meta[c / 2] |= (uint8_t)((c % 2) ? (nib << 4) : nib);
+  }
+  return O_OK;
+}
+
+/* Kept pairs back at their places, +0 elsewhere; a nibble whose pair indices are not strictly
+ * ascending returns O_EARG. */
+int sp24o_decompress_48(const void* values, const uint8_t* meta, int dtype, int64_t rows, int64_t K, void* out) {
+  if (!elem_bytes(dtype)) return O_EDTYPE;
+  if (rows < 0 || K < 0 || K % 8) return O_ESHAPE;
+  for (int64_t c = 0; c < rows * (K / 8); ++c) {
+    int nib = (meta[c / 2] >> ((c % 2) * 4)) & 0xf;
+    int i0 = nib & 3, i1 = nib >> 2;
+    if (i0 >= i1) return O_EARG;
+    for (int j = 0; j < 4; ++j) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v = 0;
+        if (j == i0) v = raw_bits(values, dtype, 4 * c + h);
+        if (j == i1) v = raw_bits(values, dtype, 4 * c + 2 + h);
+        put_raw_bits(out, dtype, 8 * c + 2 * j + h, v);
+      }
+    }
+  }
+  return O_OK;
+}
+
 /* ---------------------------------------------------------------- a3: NVFP4 */
 
 /* E2M1 magnitude codes 0..7 (1 exponent bit pair, 1 mantissa bit, bias 1):

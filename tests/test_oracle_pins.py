@@ -528,3 +528,112 @@ def test_round_to_16_against_ml_dtypes(oracle):
     assert np.array_equal(oracle.round_to_16(x, oracle.BF16), bf)
     assert np.array_equal(oracle.round_to_16(x, oracle.F16), x.astype(np.float16).astype(np.float64))
 
+
+
+# ----------------------------------------------------------------------------- pairwise 4:8
+
+_PAIR_NIBBLES = {0x4, 0x8, 0xC, 0x9, 0xD, 0xE}  # i0 | i1 << 2 for the six pairs i0 < i1
+
+
+def _nibbles(meta, n):
+    return np.stack([meta & 0xF, meta >> 4], 1).ravel()[:n]
+
+
+def test_pairwise48_brute_force(oracle):
+    """Keeping the two pairs of largest |a| + |b| ('What 2:4 actually is': the largest magnitudes
+    survive, here per pair of entries) is the choice, among the six of 2 of 4 pairs, that keeps
+    the most total magnitude.  fp16 entries of distinct pair sums make the maximiser unique, and
+    their fp32 sums are exact."""
+    g = synth.rng(41)
+    w = f16(synth.normal(g, (48, 128)))
+    pair = np.abs(w.astype(np.float64)).reshape(-1, 4, 2).sum(axis=2)
+    vals, meta = oracle.compress_48(w, oracle.F16)
+    nib = _nibbles(meta, pair.shape[0])
+    choices = list(itertools.combinations(range(4), 2))
+    checked = 0
+    for c in range(pair.shape[0]):
+        if len(set(pair[c].tolist())) < 4:
+            continue
+        totals = [pair[c][i] + pair[c][j] for i, j in choices]
+        i0, i1 = choices[int(np.argmax(totals))]
+        assert (nib[c] & 3, nib[c] >> 2) == (i0, i1), c
+        src = w.reshape(-1, 8)[c].view(np.uint16)
+        assert np.array_equal(vals.reshape(-1, 4)[c].view(np.uint16), src[[2 * i0, 2 * i0 + 1, 2 * i1, 2 * i1 + 1]])
+        checked += 1
+    assert checked > 700
+
+
+def test_pairwise48_ties_nan_and_fp32_score(oracle):
+    """Ties go to the lower pair; a NaN pair ranks above every number; the score is one fp32
+    addition, so 1 + 2^-30 ties with 1 (the lower pair wins, although the exact sum is larger)."""
+    cases = {
+        (0, 0, 0, 0, 0, 0, 0, 0): (0, 1),
+        (0, 0, 0, 0, 0, 0, 3, 0): (0, 3),
+        (1, 1, 2, 0, -2, 0, 0, 1): (0, 1),
+        (1, 1, 2, 0, -2, 0, 0, 3): (0, 3),
+        (1, 2, 0, 0, 3, -4, 0.5, 0): (0, 2),
+        (0, 0, 0, 1, 0, 0, 1, 0): (1, 3),
+    }
+    for v, pair in cases.items():
+        _, m = oracle.compress_48(f16(v).reshape(1, 8), oracle.F16)
+        assert (m[0] & 3, m[0] >> 2) == pair, v
+    _, m = oracle.compress_48(f16([1, 1, 0, np.nan, 5, 5, 0, 0]).reshape(1, 8), oracle.F16)
+    assert (m[0] & 3, m[0] >> 2) == (1, 2)
+    _, m = oracle.compress_48(f16([0, 0, np.inf, 0, 1, np.nan, np.inf, 1]).reshape(1, 8), oracle.F16)
+    assert (m[0] & 3, m[0] >> 2) == (1, 2)  # NaN first, then inf against inf + 1 = inf: lower pair
+    x = np.array([1, 0, 1, 2.0 ** -30, 5, 0, 0, 0], np.float32).reshape(1, 8)
+    assert np.float32(1) + np.float32(2.0 ** -30) == np.float32(1)
+    _, m = oracle.compress_48(x, oracle.F32)
+    assert (m[0] & 3, m[0] >> 2) == (0, 2)
+
+
+def test_pairwise48_check(oracle):
+    """A chunk of 8 is eligible when at most two of its four pairs hold a nonzero (-0 is zero);
+    a chunk that passes 2:4 can fail pairwise 4:8 and the other way round."""
+    v = {
+        "two_pairs": ([1, 2, 0, 0, 3, 4, 0, 0], 1),
+        "three_pairs": ([1, 0, 0, 2, 0, 0, 3, 0], 0),
+        "negzero": ([1, 0, -0.0, -0.0, 0, 0, 0, 5], 1),
+        "24_ok_48_fail": ([1, 0, 0, 2, 3, 0, 0, 4], 0),
+        "48_ok_24_fail": ([1, 2, 3, 4, 0, 0, 0, 0], 1),
+    }
+    for name, (x, ok) in v.items():
+        p, n = oracle.check_48(f16(x).reshape(1, 8), oracle.F16)
+        assert p.ravel().tolist() == [ok] and n == 1 - ok, name
+    assert oracle.check_24(f16(v["24_ok_48_fail"][0]).reshape(1, 8), oracle.F16)[1] == 0
+    assert oracle.check_24(f16(v["48_ok_24_fail"][0]).reshape(1, 8), oracle.F16)[1] == 1
+    with pytest.raises(oracle.OracleError):
+        oracle.check_48(f16(np.zeros(12)).reshape(1, 12), oracle.F16)
+
+
+def test_pairwise48_roundtrip(oracle):
+    """decompress(compress(W)) keeps the two chosen pairs bitwise and zeroes the other two; the
+    result passes the check in every chunk; its compress gives back the same values and meta;
+    every nibble names two ascending pairs; values take K/2 and meta K/16 bytes per row."""
+    g = synth.rng(42)
+    for dt, st in ((oracle.F16, "f16"), (oracle.BF16, "bf16"), (oracle.F32, "f32")):
+        w = synth.structured_edge(g, 24, 96, st)
+        vals, meta = oracle.compress_48(w, dt)
+        assert vals.shape == (24, 48) and meta.size == 24 * 96 // 16
+        back = oracle.decompress_48(vals, meta, dt, w.shape)
+        nib = _nibbles(meta, 24 * 12)
+        assert set(np.unique(nib).tolist()) <= _PAIR_NIBBLES
+        bw, sw = back.reshape(-1, 4, 2).view(np.uint8), w.reshape(-1, 4, 2).view(np.uint8)
+        for c in range(nib.size):
+            kept = {nib[c] & 3, nib[c] >> 2}
+            for j in range(4):
+                assert np.array_equal(bw[c, j], sw[c, j] if j in kept else np.zeros_like(sw[c, j]))
+        p, n = oracle.check_48(back, dt)
+        assert n == 0 and p.all()
+        v2, m2 = oracle.compress_48(back, dt)
+        assert np.array_equal(v2.view(np.uint8), vals.view(np.uint8)) and np.array_equal(m2, meta)
+
+
+def test_pairwise48_odd_chunk_count_and_illegal_nibble(oracle):
+    """An odd number of chunks leaves the high nibble of the last meta byte zero; a nibble with
+    pair indices out of order is rejected."""
+    w = f16(np.arange(1, 9)).reshape(1, 8)
+    vals, meta = oracle.compress_48(w, oracle.F16)
+    assert meta.tolist() == [0xE] and vals.astype(np.float64).tolist() == [[5, 6, 7, 8]]
+    with pytest.raises(oracle.OracleError):
+        oracle.decompress_48(vals, np.array([0x6], np.uint8), oracle.F16, (1, 8))
