@@ -641,7 +641,25 @@ def run_sweep(args) -> None:
                                          "frac_hbm": round(alg / us_one / 1e3 / peak_hbm, 3)},
                       "group_scale_only": {"us": round(us_gs, 1), "GB/s": round(nb_in / us_gs / 1e3, 1),
                                            "frac_hbm": round(nb_in / us_gs / 1e3 / peak_hbm, 3)}}), flush=True)
-    del Wh, qh
+    # pairwise 4:8 on the same tensor (check; prune + compress), 2:4 prune + compress beside it
+    pass48 = torch.empty((R, L // 8), dtype=torch.uint8, device=dev)
+    nf48 = torch.empty(1, dtype=torch.int32, device=dev)
+    vals = torch.empty((R, L // 2), dtype=torch.bfloat16, device=dev)
+    meta48 = torch.empty(R * L // 16, dtype=torch.uint8, device=dev)
+    meta24 = torch.empty(R * L // 8, dtype=torch.uint8, device=dev)
+    us_c48 = timeit(lambda r: sp.check_48(Wh, pass_out=pass48, n_fail_out=nf48), reps=5)
+    us_p48 = timeit(lambda r: sp.prune_compress_48(Wh, values_out=vals, meta_out=meta48), reps=5)
+    us_p24 = timeit(lambda r: sp.prune_compress_24(Wh, values_out=vals, meta_out=meta24), reps=5)
+    b_c48 = nb_in + pass48.numel()
+    b_p48, b_p24 = nb_in + nb_in // 2 + meta48.numel(), nb_in + nb_in // 2 + meta24.numel()
+    print(json.dumps({"sweep": "pairwise48", "shape": [R, L], "dtype": "bf16",
+                      "check_48": {"us": round(us_c48, 1), "GB/s": round(b_c48 / us_c48 / 1e3, 1),
+                                   "frac_hbm": round(b_c48 / us_c48 / 1e3 / peak_hbm, 3)},
+                      "prune_compress_48": {"us": round(us_p48, 1), "GB/s": round(b_p48 / us_p48 / 1e3, 1),
+                                            "frac_hbm": round(b_p48 / us_p48 / 1e3 / peak_hbm, 3)},
+                      "prune_compress_24": {"us": round(us_p24, 1), "GB/s": round(b_p24 / us_p24 / 1e3, 1),
+                                            "frac_hbm": round(b_p24 / us_p24 / 1e3 / peak_hbm, 3)}}), flush=True)
+    del Wh, qh, pass48, vals, meta48, meta24
 
     # routed experts: 4096 tokens x top-10 of 512 experts [512, 2048], bf16 x, NVFP4 experts
     # (dense, and 2:4 of the same experts); every expert is touched, so each call reads all of

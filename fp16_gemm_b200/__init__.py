@@ -38,7 +38,7 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_quantize_nvfp4_pair", "sp24_nvfp4_group_tensor_scale_workspace_size",
            "sp24_nvfp4_group_tensor_scale", "sp24_gemm_select", "sp24_gemm_choice", "sp24_gemm_auto",
            "sp24_gemm_choice_reset", "sp24_moe_block_workspace_size", "sp24_moe_block",
-           "sp24_interleave_rows")
+           "sp24_interleave_rows", "sp24_check_48", "sp24_prune_compress_48", "sp24_decompress_48")
 
 _lock = threading.Lock()
 _lib = None
@@ -109,6 +109,9 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(_SparseOperand), ctypes.POINTER(_Operand),
                                          ctypes.POINTER(_SparseOperand), I64, I64, I64, P, P, I64, P]
             L.sp24_interleave_rows.argtypes = [P, P, I64, I64, I64, P, P]
+            L.sp24_check_48.argtypes = [P, I, I64, I64, P, P, P]
+            L.sp24_prune_compress_48.argtypes = [P, I, I64, I64, P, P, P]
+            L.sp24_decompress_48.argtypes = [P, P, I, I64, I64, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -233,6 +236,54 @@ def decompress_24(values: torch.Tensor, meta: torch.Tensor, shape, op: int = OP_
         out = torch.empty(tuple(shape), dtype=values.dtype, device=values.device)
     _call("sp24_decompress_24", _ptr(values), _ptr(meta), _dtype_code(values), op, _shape(shape),
           len(shape), _ptr(out), _stream(stream))
+    return out
+
+
+def _rows_k48(shape) -> tuple:
+    shape = tuple(int(d) for d in shape)
+    if not shape:
+        raise ValueError("pairwise 4:8 needs at least one axis")
+    K = shape[-1]
+    rows = 1
+    for d in shape[:-1]:
+        rows *= d
+    return rows, K
+
+
+def check_48(w: torch.Tensor, pass_out=None, n_fail_out=None, stream=None):
+    """Pairwise 4:8 eligibility per chunk of 8 along K (uint8 0/1, [.., K/8]) and the failing
+    chunk count (int32 [1], device)."""
+    _cuda(w, "w")
+    rows, K = _rows_k48(w.shape)
+    if pass_out is None:
+        pass_out = torch.empty(tuple(w.shape[:-1]) + (K // 8,), dtype=torch.uint8, device=w.device)
+    if n_fail_out is None:
+        n_fail_out = torch.empty(1, dtype=torch.int32, device=w.device)
+    _call("sp24_check_48", _ptr(w), _dtype_code(w), rows, K, _ptr(pass_out), _ptr(n_fail_out), _stream(stream))
+    return pass_out, n_fail_out
+
+
+def prune_compress_48(w: torch.Tensor, values_out=None, meta_out=None, stream=None):
+    """(values [.., K/2], meta): the two kept pairs of every chunk of 8 and the nibble stream."""
+    _cuda(w, "w")
+    rows, K = _rows_k48(w.shape)
+    if values_out is None:
+        values_out = torch.empty(tuple(w.shape[:-1]) + (K // 2,), dtype=w.dtype, device=w.device)
+    if meta_out is None:
+        meta_out = torch.empty((rows * (K // 8) + 1) // 2, dtype=torch.uint8, device=w.device)
+    _call("sp24_prune_compress_48", _ptr(w), _dtype_code(w), rows, K, _ptr(values_out), _ptr(meta_out),
+          _stream(stream))
+    return values_out, meta_out
+
+
+def decompress_48(values: torch.Tensor, meta: torch.Tensor, shape, out=None, stream=None):
+    _cuda(values, "values")
+    _cuda(meta, "meta")
+    rows, K = _rows_k48(shape)
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=values.dtype, device=values.device)
+    _call("sp24_decompress_48", _ptr(values), _ptr(meta), _dtype_code(values), rows, K, _ptr(out),
+          _stream(stream))
     return out
 
 

@@ -127,6 +127,32 @@ int sp24_prune_compress_24(const void* w, int dtype, int op, const int64_t* shap
 int sp24_decompress_24(const void* values, const uint8_t* meta, int dtype, int op,
                        const int64_t* shape, int ndim, void* w_out, void* stream);
 
+/* ----------------------------------------------------------------------- pairwise 4:8 */
+/* The sparse pattern of the tensor cores' packed-FP4 MMA kind, whose sparse unit is a pair of
+ * consecutive entries.  [P1] "What 2:4 actually is" (the largest magnitudes survive), carried
+ * over to pairs.  W is [rows, K] row-major (matmul layout), K % 8 == 0; chunk c is entries
+ * 8c .. 8c + 7 of the flat tensor, i.e. four pairs along K.
+ *   check:     a chunk passes when at most two of its pairs hold a nonzero entry (+0 and -0 are
+ *              zero, NaN is not).  pass: device uint8 [rows, K/8]; n_fail: device int32 or
+ *              NULL (overwritten with the failing-chunk count).
+ *   prune:     keeps the two pairs of largest score |a| + |b| (one IEEE fp32 addition of the
+ *              entries' fp32 magnitudes; a NaN score above every number; ties to the lower
+ *              pair).  values: device, w's dtype, [rows, K/2], the kept pairs bit for bit in
+ *              ascending order; meta: device, ceil(rows * K / 16) bytes, nibble i0 | i1 << 2
+ *              per chunk (i0 < i1), chunk 2c in the low nibble of byte c.
+ *   decompress: w_out (device, [rows, K]) receives the kept pairs at their places and +0
+ *              elsewhere; an illegal nibble (i0 >= i1) yields +0 in its chunk and sets the
+ *              device error word (SP24_ERR_INVALID_ARG).
+ * Pointers need the alignment of their element type (SP24_ERR_ALIGN otherwise); 16-byte
+ * aligned ones take the vector kernels.  K % 8 != 0 or negative sizes: SP24_ERR_SHAPE.  The
+ * caller owns every buffer; all calls are asynchronous on `stream`. */
+int sp24_check_48(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* pass, int32_t* n_fail,
+                  void* stream);
+int sp24_prune_compress_48(const void* w, int dtype, int64_t rows, int64_t K, void* values, uint8_t* meta,
+                           void* stream);
+int sp24_decompress_48(const void* values, const uint8_t* meta, int dtype, int64_t rows, int64_t K,
+                       void* w_out, void* stream);
+
 /* ----------------------------------------------------------------------- a3: NVFP4 */
 /* [P5] "Convert BF16 to NVFP4 yourself", "The shared global scale": quantise T[rows, cols]
  * (cols % 16 == 0) to NVFP4.

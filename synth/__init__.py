@@ -218,3 +218,25 @@ def structured_edge(g: np.random.Generator, rows: int, K: int, dtype: str) -> np
     x = np.where(choice == 2, ties, x)
     x = np.where(choice == 3, np.round(base), x)   # small integers: many equal magnitudes
     return as_storage(x, dtype)
+
+
+def pairwise_edge(g: np.random.Generator, rows: int, K: int, dtype: str) -> np.ndarray:
+    """structured_edge for chunks of 8 along K: a third of the chunks get two of their four pairs
+    zeroed (eligible for pairwise 4:8; zeros of both signs), a sixth one pair; a few entries are
+    NaN or +-inf, and some pairs repeat another pair's magnitudes (score ties)."""
+    x = structured_edge(g, rows, K, "f32").astype(np.float64).reshape(rows, K // 8, 4, 2)
+    kind = g.integers(0, 6, size=(rows, K // 8))
+    order = np.argsort(g.random((rows, K // 8, 4)), axis=2)
+    sign = np.where(g.random((rows, K // 8, 4, 2)) < 0.5, -0.0, 0.0)
+    for z in range(2):
+        drop = (kind < 2) if z == 0 else (kind < 3)
+        hit = (np.arange(4)[None, None, :] == order[:, :, z:z + 1]) & drop[:, :, None]
+        x = np.where(hit[..., None], sign, x)
+    tie = (kind == 4)[:, :, None, None] & (np.arange(4)[None, None, :, None] == 3)
+    x = np.where(tie, -x[:, :, 0:1, :], x)                 # pair 3 repeats pair 0's magnitudes
+    x = x.reshape(rows, K)
+    special = g.random((rows, K))
+    x = np.where(special < 0.002, np.nan, x)
+    x = np.where((special >= 0.002) & (special < 0.004), np.inf, x)
+    x = np.where((special >= 0.004) & (special < 0.006), -np.inf, x)
+    return as_storage(x, dtype)
