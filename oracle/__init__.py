@@ -81,6 +81,8 @@ def lib():
             L.sp24o_nvfp4_tensor_scale.argtypes = [P, I, I64]
             L.sp24o_nvfp4_encode.argtypes = [P, I, I64, I64, P, P, P, P]
             L.sp24o_nvfp4_decode.argtypes = [P, P, ctypes.c_float, I64, I64, P]
+            L.sp24o_nvfp4_encode_blk.argtypes = [P, I, I64, I64, I, P, P, P, P]
+            L.sp24o_nvfp4_decode_blk.argtypes = [P, P, ctypes.c_float, I64, I64, I, P]
             L.sp24o_to_double.argtypes = [P, I, I64, P]
             L.sp24o_gemm.argtypes = [P, P, I64, I64, I64, P, P, I]
             L.sp24o_gemm_sparse.argtypes = [P, P, P, I64, I64, I64, P, P, I]
@@ -249,28 +251,29 @@ def nvfp4_group_tensor_scale(tensors, dtype: int) -> float:
     return nvfp4_tensor_scale(np.concatenate([f for f in flat if f.size]), dtype)
 
 
-def nvfp4_encode(t: np.ndarray, dtype: int, tensor_scale: float | None = None):
-    """(codes [R, L/2] u8, scales [R, L/16] u8, tensor_scale f32) of a 2-D tensor T[R, L]."""
+def nvfp4_encode(t: np.ndarray, dtype: int, tensor_scale: float | None = None, block: int = 16):
+    """(codes [R, L/2] u8, scales [R, L/block] u8, tensor_scale f32) of a 2-D tensor T[R, L];
+    block 16 is NVFP4, block 32 the activation form of the sparse FP4 MMA."""
     t = _bits(t, dtype)
     if t.ndim != 2:
         raise ValueError("nvfp4_encode wants a 2-D tensor")
     R, L = t.shape
     codes = np.zeros((R, L // 2), dtype=np.uint8)
-    scales = np.zeros((R, L // 16), dtype=np.uint8)
+    scales = np.zeros((R, L // block), dtype=np.uint8)
     ts_out = np.zeros(1, dtype=np.float32)
     ts_in = None if tensor_scale is None else np.array([tensor_scale], dtype=np.float32)
-    _check(lib().sp24o_nvfp4_encode(_ptr(t), dtype, R, L, _ptr(ts_in), _ptr(codes), _ptr(scales),
-                                    _ptr(ts_out)), "nvfp4_encode")
+    _check(lib().sp24o_nvfp4_encode_blk(_ptr(t), dtype, R, L, block, _ptr(ts_in), _ptr(codes), _ptr(scales),
+                                        _ptr(ts_out)), "nvfp4_encode")
     return codes, scales, np.float32(ts_out[0])
 
 
-def nvfp4_decode(codes: np.ndarray, scales: np.ndarray, tensor_scale) -> np.ndarray:
+def nvfp4_decode(codes: np.ndarray, scales: np.ndarray, tensor_scale, block: int = 16) -> np.ndarray:
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     R, L2 = codes.shape
     out = np.empty((R, 2 * L2), dtype=np.float64)
-    _check(lib().sp24o_nvfp4_decode(_ptr(codes), _ptr(scales), float(np.float32(tensor_scale)),
-                                    R, 2 * L2, _ptr(out)), "nvfp4_decode")
+    _check(lib().sp24o_nvfp4_decode_blk(_ptr(codes), _ptr(scales), float(np.float32(tensor_scale)),
+                                        R, 2 * L2, block, _ptr(out)), "nvfp4_decode")
     return out
 
 

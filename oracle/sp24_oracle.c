@@ -429,22 +429,25 @@ float sp24o_nvfp4_tensor_scale(const void* t, int dtype, int64_t n) {
 }
 
 /* NVFP4 encode of T[rows, cols] ([P5] "Convert BF16 to NVFP4 yourself": 4-bit E2M1 values,
- * one FP8 E4M3 scale per 16 values, one FP32 global scale), per reading R4.
- * codes: [rows, cols/2] bytes, element 2i in the low nibble; scales: [rows, cols/16] E4M3
+ * one FP8 E4M3 scale per block of consecutive values, one FP32 global scale), per reading R4.
+ * The pages' block is 16 values; block 32 is the activation form the sparse FP4 MMA reads
+ * (one scale per 32 K, reading R22), computed by the same steps over 32 values.
+ * codes: [rows, cols/2] bytes, element 2i in the low nibble; scales: [rows, cols/block] E4M3
  * bytes.  ts_in: NULL to derive the tensor scale from amax, else the shared scale to use
  * ([P5] "The shared global scale").  *ts_out receives the scale used. */
-int sp24o_nvfp4_encode(const void* t, int dtype, int64_t rows, int64_t cols, const float* ts_in,
-                       uint8_t* codes, uint8_t* scales, float* ts_out) {
+int sp24o_nvfp4_encode_blk(const void* t, int dtype, int64_t rows, int64_t cols, int block, const float* ts_in,
+                           uint8_t* codes, uint8_t* scales, float* ts_out) {
   if (!elem_bytes(dtype)) return O_EDTYPE;
-  if (rows < 0 || cols < 0 || cols % 16) return O_ESHAPE;
+  if (block != 16 && block != 32) return O_EARG;
+  if (rows < 0 || cols < 0 || cols % block) return O_ESHAPE;
   volatile float s_t = ts_in ? *ts_in : sp24o_nvfp4_tensor_scale(t, dtype, rows * cols);
   if (ts_out) *ts_out = s_t;
   volatile float d = s_t * 6.0f;
   for (int64_t r = 0; r < rows; ++r) {
-    for (int64_t b = 0; b < cols / 16; ++b) {
-      int64_t base = r * cols + b * 16;
+    for (int64_t b = 0; b < cols / block; ++b) {
+      int64_t base = r * cols + b * block;
       float bmax = 0.0f;
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < block; ++i) {
         float a = fabsf(elem_f32(t, dtype, base + i));
         if (a > bmax) bmax = a;
       }
@@ -453,9 +456,9 @@ int sp24o_nvfp4_encode(const void* t, int dtype, int64_t rows, int64_t cols, con
         volatile float q = bmax / d;
         sb = sp24o_e4m3_round((double)q);
       }
-      scales[r * (cols / 16) + b] = (uint8_t)sb;
+      scales[r * (cols / block) + b] = (uint8_t)sb;
       volatile float sc = (float)sp24o_e4m3_value(sb) * s_t;
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < block; ++i) {
         float v = elem_f32(t, dtype, base + i);
         int mag = 0;
         if (sc != 0.0f) {
@@ -473,18 +476,29 @@ int sp24o_nvfp4_encode(const void* t, int dtype, int64_t rows, int64_t cols, con
   return O_OK;
 }
 
-/* NVFP4 decode: E2M1(code) * E4M3(scale) * s_t, evaluated in fp64. */
-int sp24o_nvfp4_decode(const uint8_t* codes, const uint8_t* scales, float s_t, int64_t rows,
-                       int64_t cols, double* out) {
-  if (rows < 0 || cols < 0 || cols % 16) return O_ESHAPE;
+int sp24o_nvfp4_encode(const void* t, int dtype, int64_t rows, int64_t cols, const float* ts_in,
+                       uint8_t* codes, uint8_t* scales, float* ts_out) {
+  return sp24o_nvfp4_encode_blk(t, dtype, rows, cols, 16, ts_in, codes, scales, ts_out);
+}
+
+/* NVFP4 decode: E2M1(code) * E4M3(scale of the element's block) * s_t, evaluated in fp64. */
+int sp24o_nvfp4_decode_blk(const uint8_t* codes, const uint8_t* scales, float s_t, int64_t rows,
+                           int64_t cols, int block, double* out) {
+  if (block != 16 && block != 32) return O_EARG;
+  if (rows < 0 || cols < 0 || cols % block) return O_ESHAPE;
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       int64_t e = r * cols + c;
       int code = (codes[e / 2] >> ((e % 2) * 4)) & 0xf;
-      double sb = sp24o_e4m3_value(scales[r * (cols / 16) + c / 16]);
+      double sb = sp24o_e4m3_value(scales[r * (cols / block) + c / block]);
       out[e] = sp24o_e2m1_value(code) * sb * (double)s_t;
     }
   return O_OK;
+}
+
+int sp24o_nvfp4_decode(const uint8_t* codes, const uint8_t* scales, float s_t, int64_t rows,
+                       int64_t cols, double* out) {
+  return sp24o_nvfp4_decode_blk(codes, scales, s_t, rows, cols, 16, out);
 }
 
 /* Element values of a real tensor in fp64 (exact). */

@@ -637,3 +637,51 @@ def test_pairwise48_odd_chunk_count_and_illegal_nibble(oracle):
     assert meta.tolist() == [0xE] and vals.astype(np.float64).tolist() == [[5, 6, 7, 8]]
     with pytest.raises(oracle.OracleError):
         oracle.decompress_48(vals, np.array([0x6], np.uint8), oracle.F16, (1, 8))
+
+
+# ----------------------------------------------------------------------------- NVFP4, 32-entry blocks
+
+def test_block32_against_ml_dtypes(oracle):
+    """The 32-entry block form (the activation operand of the sparse FP4 MMA) written out with
+    numpy and ml_dtypes' RNE casts: block scale = E4M3(fp32(bmax32 / fp32(6 s_t))), code =
+    E2M1(fp32(|t| / fp32(dec(sb) s_t))) with the sign bit, every step in fp32."""
+    g = synth.rng(44)
+    x = synth.normal(g, (12, 256)) * np.exp(synth.normal(g, (12, 1)))
+    t = synth.as_storage(x, "bf16")
+    codes, scales, ts = oracle.nvfp4_encode(t, oracle.BF16, block=32)
+    assert codes.shape == (12, 128) and scales.shape == (12, 8)
+    tf = synth.bf16_bits_to_f32(t).astype(np.float32)
+    s_t = np.float32(np.abs(tf).max()) / np.float32(2688)
+    assert np.float32(ts) == s_t
+    d = np.float32(s_t * np.float32(6))
+    bmax = np.abs(tf).reshape(12, 8, 32).max(-1)
+    sb = (bmax / d).astype(np.float32).astype(ml_dtypes.float8_e4m3fn)
+    assert np.array_equal(scales, sb.view(np.uint8))
+    sc = (sb.astype(np.float32) * s_t).astype(np.float32)
+    q = (np.abs(tf).reshape(12, 8, 32) / sc[..., None]).astype(np.float32)
+    mag = np.minimum(q, np.float32(6)).astype(ml_dtypes.float4_e2m1fn).view(np.uint8).reshape(12, 256)
+    want = mag | (np.signbit(tf).astype(np.uint8) << 3)
+    assert np.array_equal(_codes_nibbles(codes), want)
+
+
+def test_block32_equals_block16_when_halves_share_their_max(oracle):
+    """When both 16-halves of every 32-block have the same largest magnitude, the two block
+    sizes give the same codes, and each block-32 scale is the shared scale of its two halves."""
+    g = synth.rng(45)
+    x = synth.normal(g, (6, 128))
+    x.reshape(6, 4, 2, 16)[..., 1, 3] = np.abs(x.reshape(6, 4, 2, 16)).max(axis=(2, 3)) * 1.5
+    x.reshape(6, 4, 2, 16)[..., 0, 7] = -x.reshape(6, 4, 2, 16)[..., 1, 3]
+    t = x.astype(np.float32)
+    c16, s16, ts16 = oracle.nvfp4_encode(t, oracle.F32)
+    c32, s32, ts32 = oracle.nvfp4_encode(t, oracle.F32, block=32)
+    assert ts16 == ts32 and np.array_equal(c16, c32)
+    assert np.array_equal(s16[:, 0::2], s32) and np.array_equal(s16[:, 1::2], s32)
+    d32 = oracle.nvfp4_decode(c32, s32, ts32, block=32)
+    assert np.array_equal(d32, oracle.nvfp4_decode(c16, s16, ts16))
+
+
+def test_block32_shape_rules(oracle):
+    with pytest.raises(oracle.OracleError):
+        oracle.nvfp4_encode(np.zeros((1, 48), np.float32), oracle.F32, block=32)
+    with pytest.raises(oracle.OracleError):
+        oracle.nvfp4_encode(np.zeros((1, 64), np.float32), oracle.F32, block=8)
