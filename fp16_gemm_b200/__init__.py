@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libsp24.so")
 # status codes (include/sp24.h)
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT, ERR_WORKSPACE = range(9)
-F16, BF16, F32, NVFP4 = 0, 1, 2, 3
+F16, BF16, F32, NVFP4, NVFP4_B32 = 0, 1, 2, 3, 4
 OP_MATMUL, OP_CONV = 0, 1
 ALGO_AUTO, ALGO_SKINNY, ALGO_TILED = 0, 1, 2
 
@@ -38,7 +38,8 @@ EXPORTS = ("sp24_status_string", "sp24_abi_version", "sp24_sizes", "sp24_check_2
            "sp24_quantize_nvfp4_pair", "sp24_nvfp4_group_tensor_scale_workspace_size",
            "sp24_nvfp4_group_tensor_scale", "sp24_gemm_select", "sp24_gemm_choice", "sp24_gemm_auto",
            "sp24_gemm_choice_reset", "sp24_moe_block_workspace_size", "sp24_moe_block",
-           "sp24_interleave_rows", "sp24_check_48", "sp24_prune_compress_48", "sp24_decompress_48")
+           "sp24_interleave_rows", "sp24_check_48", "sp24_prune_compress_48", "sp24_decompress_48",
+           "sp24_quantize_nvfp4_block32", "sp24_gemm_sparse48")
 
 _lock = threading.Lock()
 _lib = None
@@ -112,6 +113,9 @@ def lib() -> ctypes.CDLL:
             L.sp24_check_48.argtypes = [P, I, I64, I64, P, P, P]
             L.sp24_prune_compress_48.argtypes = [P, I, I64, I64, P, P, P]
             L.sp24_decompress_48.argtypes = [P, P, I, I64, I64, P, P]
+            L.sp24_quantize_nvfp4_block32.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, P]
+            L.sp24_gemm_sparse48.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_SparseOperand), I64, I64,
+                                             I64, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -312,6 +316,26 @@ def quantize_nvfp4(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None,
     return out
 
 
+def quantize_nvfp4_block32(t: torch.Tensor, tensor_scale: Optional[torch.Tensor] = None, out=None,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> NVFP4Tensor:
+    """E2M1 codes with one E4M3 scale per 32 entries (scales [R, L/32]): the activation form of
+    the pairwise-4:8 FP4 GEMM (gemm_sparse48)."""
+    _cuda(t, "t")
+    if t.dim() != 2:
+        raise ValueError("quantize_nvfp4_block32 wants a 2-D tensor")
+    R, L = t.shape
+    if out is None:
+        out = NVFP4Tensor(torch.empty((R, L // 2), dtype=torch.uint8, device=t.device),
+                          torch.empty((R, L // 32), dtype=torch.uint8, device=t.device),
+                          torch.empty(1, dtype=torch.float32, device=t.device))
+    if workspace is None and tensor_scale is None:
+        workspace = torch.empty(quantize_workspace_bytes(R, L), dtype=torch.uint8, device=t.device)
+    _call("sp24_quantize_nvfp4_block32", _ptr(t), _dtype_code(t), R, L, _ptr(tensor_scale),
+          _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), _ptr(workspace),
+          0 if workspace is None else workspace.numel(), _stream(stream))
+    return out
+
+
 def nvfp4_group_tensor_scale(tensors, out: Optional[torch.Tensor] = None,
                              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """One NVFP4 tensor scale (fp32 [1], device) shared by a group of tensors of one dtype:
@@ -502,6 +526,29 @@ def gemm_sparse24(x, w: Sparse24, K: int, out=None, algo: int = ALGO_AUTO, works
     xo = _operand(x)
     _call("sp24_gemm_sparse24", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out),
           _ptr(workspace), 0 if workspace is None else workspace.numel(), algo, _stream(stream))
+    return out
+
+
+class Sparse48(NamedTuple):
+    """A pairwise-4:8 weight [N, K] for the sparse FP4 MMA: the kept values [N, K/2] as NVFP4
+    (16-value blocks: codes [N, K/4], scales [N, K/32]) + the nibble stream of prune_compress_48."""
+    values: NVFP4Tensor
+    meta: torch.Tensor
+
+
+def gemm_sparse48(x: NVFP4Tensor, w: Sparse48, K: int, out=None, stream=None) -> torch.Tensor:
+    """y[M, N] = x w^T on the sparse FP4 MMA: x from quantize_nvfp4_block32 ([M, K]), w a
+    pairwise-4:8 weight; K % 512 == 0."""
+    M = x.codes.shape[0]
+    if x.codes.shape[1] * 2 != K:
+        raise ValueError(f"K mismatch: {x.codes.shape[1] * 2} vs {K}")
+    v = w.values
+    N = v.codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=w.meta.device)
+    xo = _Operand(NVFP4_B32, x.codes.data_ptr(), x.scales.data_ptr(), x.tensor_scale.data_ptr())
+    wo = _SparseOperand(NVFP4, v.codes.data_ptr(), v.scales.data_ptr(), v.tensor_scale.data_ptr(), w.meta.data_ptr())
+    _call("sp24_gemm_sparse48", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out), _stream(stream))
     return out
 
 

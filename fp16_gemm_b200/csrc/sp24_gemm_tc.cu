@@ -567,6 +567,220 @@ int launch_nvfp4(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
   return launch_status();
 }
 
+
+// ------------------------------------------------------------------ W4A4 with a pairwise 4:8 weight
+//
+// The sparse FP4 MMA (tcgen05.mma.sp kind::mxf4nvf4.block_scale, K = 128 logical per
+// instruction).  A = the kept values of a pairwise-4:8 weight as packed E2M1 (64 stored per row
+// per instruction, the pairs in ascending order) with their 16-value E4M3 scales (one per 32
+// logical K) and the metadata nibbles; B = the activations as E2M1 with one E4M3 scale per 32 K.
+// Per stage (512 logical K): A one 128-byte swizzled box, B two; 16 scale bytes per row of each
+// operand, rewritten by warp 6 into the same TMEM tiles as the dense kernel (4 per instruction);
+// the metadata as two boxes of 128 rows x 16 bytes, copied into TMEM with tcgen05.cp.128x128b
+// (row m on lane m, 16 bytes = 256 logical K = 4 columns, chunk 2c in the low nibble of byte
+// c).  Rows beyond N arrive as zeros, which is not a legal nibble; warp 6 writes the legal 0x4
+// (pairs 0 and 1) there before the copy, and those rows' outputs are never stored.
+template <int BN>
+struct SCfg {
+  static constexpr int S = BN == 256 ? 2 : 3;
+  static constexpr uint32_t A = kBM * 128;  // 128 rows x 256 stored FP4 = 512 logical K
+  static constexpr uint32_t B = BN * 256;   // BN rows x 512 FP4, two 128-byte boxes
+  static constexpr uint32_t SFA = kBM * 16;
+  static constexpr uint32_t SFB = BN * 16;
+  static constexpr uint32_t E = kBM * 32;   // two boxes of 128 rows x 16 bytes
+  static constexpr uint32_t STAGE = A + B + 2 * SFA + 2 * SFB + E;
+  static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
+  static constexpr int E_COLS = 8;
+  static constexpr int SFA_COLS = 16;             // 4 MMAs x 4 columns
+  static constexpr int SFB_COLS = 4 * (BN / 32);  // 4 MMAs x BN/32 columns
+  static constexpr int STAGE_COLS = E_COLS + SFA_COLS + SFB_COLS;
+  static constexpr int COLS = BN + S * STAGE_COLS <= 256 ? 256 : 512;
+  static_assert(STAGE % 1024 == 0 && SMEM <= 232448, "stage layout");
+  static_assert(BN + S * STAGE_COLS <= 512, "TMEM columns");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(224, 1)
+    gemm_nvfp4sp_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                           const __grid_constant__ CUtensorMap tmE, const TcParams p) {
+  using C = SCfg<BN>;
+  constexpr int S = C::S;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = tc::align1024(smem_raw);
+  auto sA = [&](int s) { return smem + s * C::STAGE; };
+  auto sB = [&](int s) { return sA(s) + C::A; };
+  auto sSAr = [&](int s) { return sB(s) + C::B; };
+  auto sSAt = [&](int s) { return sSAr(s) + C::SFA; };
+  auto sSBr = [&](int s) { return sSAt(s) + C::SFA; };
+  auto sSBt = [&](int s) { return sSBr(s) + C::SFB; };
+  auto sE = [&](int s) { return sSBt(s) + C::SFB; };
+  __shared__ uint64_t full_bar[S], sf_bar[S], empty_bar[S], tfull_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int aborted;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;  // weight rows
+  const int n0 = blockIdx.y * BN;   // activation rows
+  const int KB = p.K / 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&sf_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&tfull_bar, 1);
+    aborted = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSA);
+    prefetch_tmap(&tmSB);
+    prefetch_tmap(&tmE);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base, C::COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], C::A + C::B + C::SFA + C::SFB + C::E);
+        tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 128, m0);  // 128 bytes = 256 stored codes
+        tma_load_2d(sB(s), &tmB, &full_bar[s], kb * 256, n0);  // 2 x 128 bytes = 512 codes
+        tma_load_2d(sB(s) + BN * 128, &tmB, &full_bar[s], kb * 256 + 128, n0);
+        tma_load_2d(sSAr(s), &tmSA, &full_bar[s], kb * 16, m0);  // 16 scales per row
+        tma_load_2d(sSBr(s), &tmSB, &full_bar[s], kb * 16, n0);
+        tma_load_2d(sE(s), &tmE, &full_bar[s], kb * 32, m0);  // 2 x 16 bytes of nibbles per row
+        tma_load_2d(sE(s) + 2048, &tmE, &full_bar[s], kb * 32 + 16, m0);
+        ++issued;
+      }
+      for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
+        mbar_wait(&full_bar[kb % S], (kb / S) & 1);
+    }
+  } else if (warp == 6) {
+    const int valid = p.N - m0;  // rows of this weight tile that exist (>= 1)
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (kb / S) & 1;
+      if (!mbar_wait(&full_bar[s], ph) || *(volatile int*)&aborted) {
+        aborted = 1;
+        break;
+      }
+      // tile (j, g) = MMA j, rows 128 g .. 128 g + 127: word of row r at index 4 * (r % 32) + r / 32
+      auto rewrite = [&](const uint8_t* raw, uint8_t* tiles, int groups) {
+        for (int g = 0; g < groups; ++g) {
+          uint4 w[4];
+#pragma unroll
+          for (int rq = 0; rq < 4; ++rq) w[rq] = *reinterpret_cast<const uint4*>(raw + 16 * (128 * g + 32 * rq + lane));
+          const uint32_t col[4][4] = {{w[0].x, w[1].x, w[2].x, w[3].x}, {w[0].y, w[1].y, w[2].y, w[3].y},
+                                      {w[0].z, w[1].z, w[2].z, w[3].z}, {w[0].w, w[1].w, w[2].w, w[3].w}};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(tiles + 512 * (j * groups + g) + 16 * lane) =
+                make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
+        }
+      };
+      rewrite(sSAr(s), sSAt(s), 1);
+      rewrite(sSBr(s), sSBt(s), BN / 128);
+      for (int r = valid + lane; r < kBM; r += 32) {
+        const uint4 legal = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+        *reinterpret_cast<uint4*>(sE(s) + 16 * r) = legal;
+        *reinterpret_cast<uint4*>(sE(s) + 2048 + 16 * r) = legal;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sf_bar[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_nvfp4(kBM, BN, true);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&full_bar[s], ph) || !mbar_wait(&sf_bar[s], ph) || *(volatile int*)&aborted) {
+          aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t e0 = tmem + BN + s * C::STAGE_COLS;
+        const uint32_t sfa0 = e0 + C::E_COLS;
+        const uint32_t sfb0 = sfa0 + C::SFA_COLS;
+        tmem_cp_128x128b(e0, desc_rows16_noswizzle(smem_u32(sE(s))));
+        tmem_cp_128x128b(e0 + 4, desc_rows16_noswizzle(smem_u32(sE(s) + 2048)));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSAt(s) + 512 * j)));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+            tmem_cp_32x128b_x4(sfb0 + (BN / 32) * j + 4 * g,
+                               desc_rows16_noswizzle(smem_u32(sSBt(s) + 512 * (j * (BN / 128) + g))));
+        }
+        const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
+        const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB(s)));
+        const uint64_t b1 = desc_kmajor_sw128(smem_u32(sB(s) + BN * 128));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)  // A: 32 bytes (2 descriptor units) per MMA; B: 64 bytes (4)
+          umma_nvfp4_sp(tmem, a0 + 2 * j, (j < 2 ? b0 : b1) + 4 * (j & 1), e0 + 2 * j, idesc, sfa0 + 4 * j,
+                        sfb0 + (BN / 32) * j, (kb | j) != 0);
+        umma_commit(&empty_bar[s]);
+      }
+      umma_commit(&tfull_bar);
+    }
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const int row = m0 + 32 * q + lane;
+    if (!mbar_wait(&tfull_bar, 0)) {
+      aborted = 1;
+    } else {
+      tc_fence_after();
+      float scale = 1.0f;
+      if (p.scale_a) scale *= *p.scale_a;
+      if (p.scale_b) scale *= *p.scale_b;
+#pragma unroll 1
+      for (int j = 0; j < BN / 32; ++j) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * j, v);
+        if (row < p.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = n0 + 32 * j + i;
+            if (tok < p.M) p.y[(int64_t)tok * p.N + row] = v[i] * scale;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && aborted) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::COLS);
+  }
+}
+
+template <int BN>
+int launch_nvfp4sp(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa, const CUtensorMap& sb,
+                   const CUtensorMap& e, const TcParams& p, cudaStream_t s) {
+  auto kern = gemm_nvfp4sp_tc_kernel<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCfg<BN>::SMEM) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  dim3 grid((unsigned)((p.N + kBM - 1) / kBM), (unsigned)((p.M + BN - 1) / BN));
+  kern<<<grid, 224, SCfg<BN>::SMEM, s>>>(a, b, sa, sb, e, p);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ weight expansion to 16-bit
 
 // Dense NVFP4 ([rows, K/2] codes, [rows, K/16] scales) or 2:4-compressed weights (16-bit values
@@ -663,6 +877,33 @@ int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const
   return BN == 256 ? launch_nvfp4<256>(ta, tb, tsa, tsb, p, s) : launch_nvfp4<128>(ta, tb, tsa, tsb, p, s);
 }
 
+// W4A4 GEMM on the sparse FP4 MMA: y = s_w s_x sum_k dec(x) dec(w) with w a pairwise-4:8 weight
+// (values codes [N, K/4], their scales [N, K/32], meta [N, K/16]) and x packed E2M1 with one
+// scale per 32 K ([M, K/2] codes, [M, K/32] scales); K % 512 == 0 (whole stages, and 16-byte
+// scale-row pitches for the tensor maps).
+int tc_gemm_nvfp4_sp48(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* vc,
+                       const uint8_t* vs, const uint8_t* meta, const float* w_ts, int64_t M, int64_t N, int64_t K,
+                       float* y, cudaStream_t s) {
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 512) return SP24_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return SP24_OK;
+  if (K == 0)
+    return cudaMemsetAsync(y, 0, (size_t)(M * N) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  const int BN = M > 128 ? 256 : 128;
+  CUtensorMap ta, tb, tsa, tsb, te;
+  int st = make_tmap_2d(&ta, vc, 1, N, K / 4, K / 4, 128, kBM);
+  if (st) return st;
+  st = make_tmap_2d(&tb, xc, 1, M, K / 2, K / 2, 128, BN);
+  if (st) return st;
+  st = make_tmap_2d_plain(&tsa, vs, N, K / 32, K / 32, 16, kBM);
+  if (st) return st;
+  st = make_tmap_2d_plain(&tsb, xs, M, K / 32, K / 32, 16, BN);
+  if (st) return st;
+  st = make_tmap_2d_plain(&te, meta, N, K / 16, K / 16, 16, kBM);
+  if (st) return st;
+  TcParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts};
+  return BN == 256 ? launch_nvfp4sp<256>(ta, tb, tsa, tsb, te, p, s) : launch_nvfp4sp<128>(ta, tb, tsa, tsb, te, p, s);
+}
+
 // Expands an NVFP4 / 2:4 operand of `rows` rows into 16-bit [rows, K] at `out` (workspace).
 int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta, int64_t rows,
                int64_t K, uint16_t* out, cudaStream_t s) {
@@ -702,3 +943,24 @@ int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, b
 }
 
 }  // namespace sp24
+
+using namespace sp24;
+
+extern "C" int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
+                                  int64_t K, float* y, void* stream) {
+  if (!x || !w) return SP24_ERR_INVALID_ARG;
+  if (x->format != SP24_NVFP4_B32 || w->format != SP24_NVFP4) return SP24_ERR_DTYPE;
+  if (M < 0 || N < 0 || K < 0 || K % 512) return SP24_ERR_SHAPE;
+  if (M == 0 || N == 0) return SP24_OK;
+  if (!y) return SP24_ERR_INVALID_ARG;
+  if (K > 0) {
+    if (!x->data || !x->scales || !x->tensor_scale || !w->values || !w->scales || !w->tensor_scale || !w->meta)
+      return SP24_ERR_INVALID_ARG;
+    if (!aligned(x->data, 16) || !aligned(x->scales, 16) || !aligned(w->values, 16) || !aligned(w->scales, 16) ||
+        !aligned(w->meta, 16))
+      return SP24_ERR_ALIGN;
+  }
+  return tc_gemm_nvfp4_sp48(static_cast<const uint8_t*>(x->data), x->scales, x->tensor_scale,
+                            static_cast<const uint8_t*>(w->values), w->scales, w->meta, w->tensor_scale, M, N, K, y,
+                            as_stream(stream));
+}

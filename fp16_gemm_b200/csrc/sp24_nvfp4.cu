@@ -423,6 +423,46 @@ int ring_grid(Kern k, int64_t bytes) {
   return full_wave_grid(k, kThreads, (bytes + kChunk - 1) / kChunk, kRingBytes);
 }
 
+// ---- 32-entry blocks: the activation form the sparse FP4 MMA reads (one scale per 32 K).
+// The same steps as the 16-entry encoder over 32 entries: bmax, sb = E4M3(bmax / (6 s_t)),
+// code = E2M1(|t| / (E4M3(sb) s_t)), every step an IEEE fp32 operation (the per-entry division
+// is __fdiv_rn, then the hardware's RNE + satfinite conversion).  One thread per block, grid-
+// stride; the tensor is an activation (small next to the weights), so the plain division is
+// affordable here.
+template <int DT>
+__global__ void __launch_bounds__(kThreads) encode32_kernel(const void* __restrict__ t, int64_t nblk,
+                                                            const float* __restrict__ ts_in,
+                                                            const unsigned int* __restrict__ amax_bits,
+                                                            uint4* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                            float* __restrict__ ts_out) {
+  const float s_t = ts_in ? *ts_in : __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
+  const float d = __fmul_rn(s_t, 6.0f);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+    float v[32];
+    load_block<DT>(t, 2 * b, *reinterpret_cast<float(*)[16]>(&v[0]));
+    load_block<DT>(t, 2 * b + 1, *reinterpret_cast<float(*)[16]>(&v[16]));
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+    const uint32_t sb = d != 0.0f ? e4m3_rne_satfinite(__fdiv_rn(bmax, d)) : 0u;
+    const float sc = __fmul_rn(e4m3_value(sb), s_t);
+    uint32_t packed[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float q0 = sc != 0.0f ? __fdiv_rn(fabsf(v[i]), sc) : 0.0f;
+      const float q1 = sc != 0.0f ? __fdiv_rn(fabsf(v[i + 1]), sc) : 0.0f;
+      uint32_t byte = e2m1x2_rne_satfinite(q0, q1);
+      byte |= (__float_as_uint(v[i]) >> 31) << 3;
+      byte |= (__float_as_uint(v[i + 1]) >> 31) << 7;
+      packed[i / 8] |= byte << (8 * ((i % 8) / 2));
+    }
+    codes[b] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    scales[b] = (uint8_t)sb;
+  }
+}
+
 constexpr int64_t kQuantWorkspace = 256;
 
 }  // namespace
@@ -483,6 +523,51 @@ extern "C" int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64
   }
   return quantize_nvfp4_launch(t, dtype, rows, cols, tensor_scale_in, codes, scales,
                                tensor_scale_out, amax_word, as_stream(stream));
+}
+
+extern "C" int sp24_quantize_nvfp4_block32(const void* t, int dtype, int64_t rows, int64_t cols,
+                                           const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                           float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
+                                           void* stream) {
+  const int eb = elem_bytes(dtype);
+  if (!eb) return SP24_ERR_DTYPE;
+  if (rows < 0 || cols < 0 || cols % 32) return SP24_ERR_SHAPE;
+  if (!tensor_scale_out) return SP24_ERR_INVALID_ARG;
+  const int64_t nblk = rows * cols / 32;
+  if (nblk > 0 && (!t || !codes || !scales)) return SP24_ERR_INVALID_ARG;
+  if (nblk > 0 && (!aligned(t, 16) || !aligned(codes, 16))) return SP24_ERR_ALIGN;
+  unsigned int* amax_word = nullptr;
+  if (!tensor_scale_in) {
+    if (!workspace || workspace_bytes < kQuantWorkspace) return SP24_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return SP24_ERR_ALIGN;
+    amax_word = reinterpret_cast<unsigned int*>(workspace);
+  }
+  cudaStream_t s = as_stream(stream);
+  int nl = 1;
+  if (!tensor_scale_in) {
+    if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return SP24_ERR_CUDA;
+    if (nblk > 0) {
+      const int64_t n16 = 2 * nblk, bytes = n16 * (dtype == SP24_F32 ? 64 : 32);
+      if (dtype == SP24_F32)
+        amax_kernel<SP24_F32><<<ring_grid(amax_kernel<SP24_F32>, bytes), kThreads, kRingBytes, s>>>(t, n16, amax_word);
+      else if (dtype == SP24_BF16)
+        amax_kernel<SP24_BF16><<<ring_grid(amax_kernel<SP24_BF16>, bytes), kThreads, kRingBytes, s>>>(t, n16, amax_word);
+      else
+        amax_kernel<SP24_F16><<<ring_grid(amax_kernel<SP24_F16>, bytes), kThreads, kRingBytes, s>>>(t, n16, amax_word);
+      ++nl;
+    }
+  }
+  // launched even when nblk == 0 so that tensor_scale_out is written
+  if (dtype == SP24_F32)
+    encode32_kernel<SP24_F32><<<full_wave_grid(encode32_kernel<SP24_F32>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(
+        t, nblk, tensor_scale_in, amax_word, (uint4*)codes, scales, tensor_scale_out);
+  else if (dtype == SP24_BF16)
+    encode32_kernel<SP24_BF16><<<full_wave_grid(encode32_kernel<SP24_BF16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(
+        t, nblk, tensor_scale_in, amax_word, (uint4*)codes, scales, tensor_scale_out);
+  else
+    encode32_kernel<SP24_F16><<<full_wave_grid(encode32_kernel<SP24_F16>, kThreads, blocks_for(nblk)), kThreads, 0, s>>>(
+        t, nblk, tensor_scale_in, amax_word, (uint4*)codes, scales, tensor_scale_out);
+  return launch_status(nl);
 }
 
 extern "C" int sp24_quantize_nvfp4_pair(const void* t0, int dtype, int64_t rows0, int64_t cols0,

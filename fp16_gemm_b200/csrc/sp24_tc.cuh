@@ -217,9 +217,26 @@ __device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// Sparse block-scaled FP4 MMA (kind::mxf4nvf4 with a pairwise 4:8 A operand): K = 128 logical
+// per instruction, A holds 64 stored E2M1 per row (32 bytes), B 128 E2M1 per row; the metadata
+// (4 bits per 8 logical K, row m on TMEM lane m) at `e_tmem`; one E4M3 scale per 32 logical K
+// for both operands at `sfa` / `sfb`.
+__device__ __forceinline__ void umma_nvfp4_sp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                              uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %7, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%3], %4, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor of kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 scales, K = 64), K-major.
-__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// Bit 2 marks a sparse A operand (K = 128 logical per instruction, metadata selector 0).
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N, bool sparse = false) {
+  return (sparse ? 1u << 2 : 0u) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Copies 32 rows x 128 bits from shared memory into TMEM lanes 0-31 of 4 columns and repeats

@@ -43,7 +43,7 @@ enum {
 
 /* ----------------------------------------------------------------------- enums */
 /* element types */
-enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3 };
+enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3, SP24_NVFP4_B32 = 4 };
 
 /* The operation a weight belongs to decides which four entries form a group ([P2] "The
  * operation determines which four entries belong together"). */
@@ -63,6 +63,8 @@ enum { SP24_ALGO_AUTO = 0, SP24_ALGO_SKINNY = 1, SP24_ALGO_TILED = 2 };
  *   scale per 16 values, one fp32 tensor scale):
  *       data -> [rows, K/2] bytes of packed E2M1 codes (entry 2i in the low nibble),
  *       scales -> [rows, K/16] E4M3 block scales, tensor_scale -> one fp32 (device).
+ *   format SP24_NVFP4_B32: the same encoding with one E4M3 scale per 32 values, scales ->
+ *       [rows, K/32] (the activation form read by sp24_gemm_sparse48 only).
  * Decoded value = E2M1(code) * E4M3(scale) * tensor_scale. */
 typedef struct {
   int32_t format;
@@ -153,6 +155,21 @@ int sp24_prune_compress_48(const void* w, int dtype, int64_t rows, int64_t K, vo
 int sp24_decompress_48(const void* values, const uint8_t* meta, int dtype, int64_t rows, int64_t K,
                        void* w_out, void* stream);
 
+/* W4A4 GEMM on the sparse FP4 MMA (tcgen05.mma.sp kind::mxf4nvf4, K = 128 logical per
+ * instruction): y[M, N] = s_x s_w sum_k dec(x[m, k]) dec(w[n, k]), fp32 accumulation, the
+ * product of the pages' 2:4-sparse W4A4 path ([P1] "NVFP4 vs 2:4 sparse: where the other half
+ * of the petaflop went") in the pattern that MMA reads.
+ *   x  format SP24_NVFP4_B32: data [M, K/2] codes, scales [M, K/32] (sp24_quantize_nvfp4_block32).
+ *   w  format SP24_NVFP4: a pairwise-4:8 weight W[N, K]: values -> [N, K/4] codes of the kept
+ *      values [N, K/2] quantised with sp24_quantize_nvfp4 (scales -> [N, K/32], one per 16
+ *      stored = 32 logical K), meta -> [N, K/16] from sp24_prune_compress_48 (every nibble
+ *      legal; other metadata gives undefined results for its rows).
+ *   y  device fp32 [M, N], written (not accumulated).
+ * K % 512 == 0 (SP24_ERR_SHAPE otherwise); every operand pointer 16-byte aligned; M, N, K up to
+ * 2^31 - 1.  Wrong formats: SP24_ERR_DTYPE.  One launch; nothing is allocated. */
+int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
+                       int64_t K, float* y, void* stream);
+
 /* ----------------------------------------------------------------------- a3: NVFP4 */
 /* [P5] "Convert BF16 to NVFP4 yourself", "The shared global scale": quantise T[rows, cols]
  * (cols % 16 == 0) to NVFP4.
@@ -188,6 +205,18 @@ int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
 int sp24_quantize_nvfp4_noalloc(const void* t, int dtype, int64_t rows, int64_t cols,
                                 const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
                                 float* tensor_scale_out, void* stream);
+
+/* NVFP4 encoding with 32-value blocks: the activation operand of the sparse FP4 MMA, which
+ * reads one scale per 32 K (sp24_gemm_sparse48).  The steps of sp24_quantize_nvfp4 over
+ * 32 consecutive entries of a row:  s_t = tensor_scale_in ? *tensor_scale_in : amax / 2688;
+ * sb = E4M3_rne_satfinite(bmax32 / (s_t * 6));  code = sign << 3 | E2M1_rne_satfinite(|t| /
+ * (E4M3(sb) * s_t)), every step IEEE fp32.  cols % 32 == 0; codes [rows, cols/2] (16-byte
+ * aligned), scales [rows, cols/32]; workspace as sp24_quantize_nvfp4 (used only when no scale
+ * is supplied).  Errors as sp24_quantize_nvfp4. */
+int sp24_quantize_nvfp4_block32(const void* t, int dtype, int64_t rows, int64_t cols,
+                                const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
+                                void* stream);
 
 /* Two quantisations in one launch (a weight and its 2:4 values, with the tensor scales that
  * sp24_prepare_24 derived, say): the results equal those of sp24_quantize_nvfp4(t0, ts0) and

@@ -1,0 +1,117 @@
+"""GPU parity of the W4A4 GEMM on the sparse FP4 MMA: a pairwise-4:8 weight (kept values as
+NVFP4) times activations in 32-value blocks, against the oracle's fp64 product of the decoded
+operands, plus the bit-exact 32-value-block activation quantiser."""
+import numpy as np
+import pytest
+import torch
+
+import fp16_gemm_b200 as sp
+import oracle
+import synth
+from helpers import ORACLE_DT, assert_gemm_close, bits, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits32(x) -> int:
+    return int(np.float32(x).view(np.uint32))
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 32), (7, 96), (130, 512), (33, 2048)], ids=lambda s: "x".join(map(str, s)))
+def test_block32_quantiser_bit_exact(dtype, shape):
+    g = synth.rng(500 + shape[0])
+    x = synth.normal(g, shape) * np.exp(synth.normal(g, (shape[0], 1)))
+    t = synth.as_storage(x, dtype)
+    c_ref, s_ref, ts_ref = oracle.nvfp4_encode(t, ORACLE_DT[dtype], block=32)
+    q = sp.quantize_nvfp4_block32(to_dev(t, dtype))
+    torch.cuda.synchronize()
+    assert _bits32(q.tensor_scale.item()) == _bits32(ts_ref)
+    assert np.array_equal(to_host(q.scales), s_ref)
+    assert np.array_equal(to_host(q.codes), c_ref)
+    # with a supplied (shared) scale
+    ts = torch.tensor([float(ts_ref) * 3], dtype=torch.float32, device="cuda")
+    q2 = sp.quantize_nvfp4_block32(to_dev(t, dtype), tensor_scale=ts)
+    c2, s2, _ = oracle.nvfp4_encode(t, ORACLE_DT[dtype], tensor_scale=float(ts_ref) * 3, block=32)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(q2.scales), s2) and np.array_equal(to_host(q2.codes), c2)
+    assert sp.last_device_error() == sp.OK
+
+
+def test_block32_quantiser_zero_and_rejects():
+    z = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    q = sp.quantize_nvfp4_block32(z)
+    torch.cuda.synchronize()
+    assert q.tensor_scale.item() == 0 and not q.scales.any() and not q.codes.any()
+    with pytest.raises(sp.SP24Error) as e:
+        sp.quantize_nvfp4_block32(torch.zeros((2, 48), dtype=torch.bfloat16, device="cuda"))
+    assert e.value.status == sp.ERR_SHAPE
+
+
+def _decompress48_f64(vals: np.ndarray, meta: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Dense fp64 [N, K] from decoded kept values [N, K/2] and the nibble stream."""
+    nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()[: N * K // 8].reshape(N, K // 8)
+    out = np.zeros((N, K // 8, 4, 2))
+    v = vals.reshape(N, K // 8, 2, 2)
+    rows = np.arange(N)[:, None]
+    ch = np.arange(K // 8)[None, :]
+    out[rows, ch, nib & 3] = v[:, :, 0]
+    out[rows, ch, nib >> 2] = v[:, :, 1]
+    return out.reshape(N, K)
+
+
+def _case(M, N, K, seed):
+    g = synth.rng(seed)
+    X = synth.draw(g, (M, K), "bf16")
+    W = synth.draw(g, (N, K), "bf16", 0.02)
+    return X, W
+
+
+def _run(M, N, K, seed):
+    X, W = _case(M, N, K, seed)
+    # oracle
+    v_ref, m_ref = oracle.compress_48(W, oracle.BF16)
+    vc, vs, vts = oracle.nvfp4_encode(v_ref, oracle.BF16)
+    Wd = _decompress48_f64(oracle.nvfp4_decode(vc, vs, vts), m_ref, N, K)
+    xc, xs, xts = oracle.nvfp4_encode(X, oracle.BF16, block=32)
+    Xd = oracle.nvfp4_decode(xc, xs, xts, block=32)
+    Y, S = oracle.gemm(Xd, Wd)
+    # CUDA path
+    v, m = sp.prune_compress_48(to_dev(W, "bf16"))
+    vq = sp.quantize_nvfp4(v)
+    xq = sp.quantize_nvfp4_block32(to_dev(X, "bf16"))
+    y = sp.gemm_sparse48(xq, sp.Sparse48(vq, m), K)
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
+    # the operands are the oracle's, byte for byte
+    assert np.array_equal(bits(to_host(v)), bits(v_ref)) and np.array_equal(to_host(m), m_ref)
+    assert np.array_equal(to_host(vq.codes), vc) and np.array_equal(to_host(vq.scales), vs)
+    assert np.array_equal(to_host(xq.codes), xc) and np.array_equal(to_host(xq.scales), xs)
+    assert_gemm_close(y, Y, S)
+
+
+@pytest.mark.parametrize("mnk", [(1, 128, 512), (96, 200, 1024), (128, 256, 512), (300, 384, 1536),
+                                 (129, 129, 2048), (512, 130, 1024)], ids=lambda t: "x".join(map(str, t)))
+def test_gemm_sparse48(mnk):
+    """Every output, at sizes spanning several 128-row weight tiles, both activation tile widths
+    (128 for M <= 128, 256 above), ragged M and N, and several 512-wide K stages."""
+    _run(*mnk, seed=510 + sum(mnk))
+
+
+def test_gemm_sparse48_rejects():
+    X, W = _case(4, 128, 512, 520)
+    v, m = sp.prune_compress_48(to_dev(W, "bf16"))
+    vq = sp.quantize_nvfp4(v)
+    xq16 = sp.quantize_nvfp4(to_dev(X, "bf16"))
+    xo = sp._Operand(sp.NVFP4, xq16.codes.data_ptr(), xq16.scales.data_ptr(), xq16.tensor_scale.data_ptr())
+    wo = sp._SparseOperand(sp.NVFP4, vq.codes.data_ptr(), vq.scales.data_ptr(), vq.tensor_scale.data_ptr(),
+                           m.data_ptr())
+    y = torch.empty((4, 128), dtype=torch.float32, device="cuda")
+    L = sp.lib()
+    import ctypes
+    assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 4, 128, 512, y.data_ptr(), None) == sp.ERR_DTYPE
+    xo.format = sp.NVFP4_B32
+    assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 4, 128, 256, y.data_ptr(), None) == sp.ERR_SHAPE
+    assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 0, 128, 512, y.data_ptr(), None) == sp.OK
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
