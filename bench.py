@@ -447,7 +447,7 @@ def run_sweep(args) -> None:
         peak_bf16 = 1590.0
     # tensor peaks per pipe: measured bf16 dense; FP4 dense = bf16 x 4 (nominal 9 / 2.25 PF);
     # 2:4 sparse pipes count dense-equivalent FLOPs at twice the dense rate
-    tensor_peak = {"f16": peak_bf16, "f16.sp": 2 * peak_bf16, "nvfp4": 4 * peak_bf16}
+    tensor_peak = {"f16": peak_bf16, "f16.sp": 2 * peak_bf16, "nvfp4": 4 * peak_bf16, "nvfp4.sp": 8 * peak_bf16}
     dev = torch.device("cuda", 0)
     t16 = lambda a, d: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if d == "bf16"
                         else torch.from_numpy(a)).to(dev)
@@ -557,6 +557,37 @@ def run_sweep(args) -> None:
         Xb = synth.draw(synth.rng(Mv), (Mv, 5120), "bf16")
         case("msweep_nvfp4_w4a16", Mv, 5120, 5120, "bf16", "nvfp4", Xb, Wb)
         case("msweep_nvfp4_w4a4", Mv, 5120, 5120, "nvfp4", "nvfp4", Xb, Wb)
+    def case48(workload, M, N, K, X, W):
+        """W4A4 on the sparse FP4 MMA (pairwise 4:8 weight, activations in 32-value blocks)
+        against the dense W4A4 GEMM of the same weight (NVFP4, 16-value blocks)."""
+        xb, wb16 = t16(X, "bf16"), t16(W, "bf16")
+        x16, x32 = sp.quantize_nvfp4(xb), sp.quantize_nvfp4_block32(xb)
+        v, m = sp.prune_compress_48(wb16)
+        dense, sparse = sp.quantize_nvfp4(wb16), sp.Sparse48(sp.quantize_nvfp4(v), m)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        flops = 2.0 * M * N * K
+        line = {"sweep": workload, "M": M, "N": N, "K": K, "x": "nvfp4", "w": "nvfp4"}
+        for name, wop, xop, pipe in (("dense", dense, x16, "nvfp4"), ("sparse48", sparse, x32, "nvfp4.sp")):
+            wbytes = op_bytes(wop.values) + wop.meta.numel() if name == "sparse48" else op_bytes(wop)
+            copies = max(1, min(8, int(256e6 // max(wbytes, 1))))
+            wops = [wop] + [clone_op(wop) for _ in range(copies - 1)]
+            if name == "dense":
+                fn = lambda r: sp.gemm_dense(xop, wops[r % copies], out=y)
+            else:
+                fn = lambda r: sp.gemm_sparse48(xop, wops[r % copies], K, out=y)
+            us = timeit(fn)
+            byts = xop.codes.numel() + xop.scales.numel() + wbytes + M * N * 4
+            tflops = flops / (us * 1e-6) / 1e12
+            line[name] = {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(byts / us / 1e3, 1),
+                          "bytes": byts, "pipe": pipe, "frac_tensor": round(tflops / tensor_peak[pipe], 3)}
+        line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse48"]["us"], 3)
+        print(json.dumps(line), flush=True)
+
+    d = synth.prefill_w4a4()
+    case48("w4a4_pairwise48", 4096, 4096, 4096, d["X"], d["W"])
+    for Mv in (128, 1024, 4096, 16384):
+        case48("msweep_w4a4_pairwise48", Mv, 5120, 5120, synth.draw(synth.rng(Mv), (Mv, 5120), "bf16"), Wb)
+
     agree = sum(c["rule"] == c["faster"] for c in selections)
     print(json.dumps({"sweep": "dense_sparse_selection", "shapes": len(selections), "rule_picks_faster": agree,
                       "worst_loss": max(c["loss"] for c in selections), "cases": selections}), flush=True)
@@ -690,7 +721,7 @@ def run_sweep(args) -> None:
 def run_ncu_target() -> None:
     """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode
     pipeline on the decode workload: prepare_vec, encode_pair_kernel, decode_tile_kernel dense
-    and 2:4 per pass; W4A4 dense / 2:4 at 4096^3, FP16 dense / 2:4 at M = 4096; then the
+    and 2:4 per pass; W4A4 dense / 2:4 / pairwise 4:8 at 4096^3, FP16 dense / 2:4 at M = 4096; then the
     routed-expert workload once, NVFP4 experts dense and 2:4)."""
     import torch
 
@@ -709,9 +740,12 @@ def run_ncu_target() -> None:
     xq, w = sp.quantize_nvfp4(bf(d["X"])), bf(d["W"])
     v, m = sp.prune_compress_24(w)
     wq, vq = sp.quantize_nvfp4(w), sp.quantize_nvfp4(v)
+    v48, m48 = sp.prune_compress_48(w)
+    s48, x32 = sp.Sparse48(sp.quantize_nvfp4(v48), m48), sp.quantize_nvfp4_block32(bf(d["X"]))
     for _ in range(2):
         sp.gemm_dense(xq, wq)
         sp.gemm_sparse24(xq, sp.Sparse24(vq, m), 4096)
+        sp.gemm_sparse48(x32, s48, 4096)
     g = synth.rng(0)
     w16 = torch.from_numpy(synth.draw(g, (5120, 5120), "f16")).cuda()
     x16 = torch.from_numpy(synth.draw(g, (4096, 5120), "f16")).cuda()

@@ -94,7 +94,7 @@ def _run(M, N, K, seed):
                                  (129, 129, 2048), (512, 130, 1024)], ids=lambda t: "x".join(map(str, t)))
 def test_gemm_sparse48(mnk):
     """Every output, at sizes spanning several 128-row weight tiles, both activation tile widths
-    (128 for M <= 128, 256 above), ragged M and N, and several 512-wide K stages."""
+    (128 for M <= 256, 256 above), ragged M and N, and several 512-wide K stages."""
     _run(*mnk, seed=510 + sum(mnk))
 
 
