@@ -382,24 +382,48 @@ __global__ void __launch_bounds__(224, 1)
 // cubed is the pages' kernel ceiling.  Here both operands stay packed E2M1 in shared memory
 // (TMA, 128-byte swizzle: 256 K per row) and the tensor core applies the E4M3 block scales from
 // TMEM (tcgen05.mma kind::mxf4nvf4.block_scale.block16, K = 64 per instruction).  Per stage
-// (256 K) the producer also loads each row's 16 scale bytes; warp 6 rewrites them into 128-row x
-// 4-scale tiles (row r at byte 16*(r%32) + 4*(r/32)), one tile per MMA and per 128 rows, which
+// (256 K) the producer also loads each row's 16 scale bytes; warp 6 rewrites them in place into
+// 128-row x 4-scale tiles (row r at byte 16*(r%32) + 4*(r/32)), one tile per MMA and per 128
+// rows (in place, so four 54 KB stages fit at BN = 256), which
 // the MMA thread copies into TMEM with tcgen05.cp.32x128b.warpx4 (lanes 0-31, repeated in every
 // lane quarter).  The tensor scales s_w * s_x multiply the accumulator in the epilogue.
-constexpr int kQStages = 3;
-
 template <int BN>
 struct QCfg {
+  static constexpr int S = BN == 256 ? 4 : 6;     // stages (the scale tiles are rewritten in place)
   static constexpr uint32_t A = kBM * 128;        // 128 rows x 256 FP4
   static constexpr uint32_t B = BN * 128;
-  static constexpr uint32_t SFA = kBM * 16;       // raw scale rows (16 per 256 K)
+  static constexpr uint32_t SFA = kBM * 16;       // scale rows (16 per 256 K), then tiles
   static constexpr uint32_t SFB = BN * 16;
-  static constexpr uint32_t STAGE = A + B + 2 * SFA + 2 * SFB;
-  static constexpr size_t SMEM = (size_t)kQStages * STAGE + 1024;
+  static constexpr uint32_t STAGE = A + B + SFA + SFB;
+  static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
   static constexpr int SFA_COLS = 16;             // 4 MMAs x 4 columns
   static constexpr int SFB_COLS = 4 * (BN / 32);  // 4 MMAs x BN/32 columns
-  static constexpr int COLS = BN + kQStages * (SFA_COLS + SFB_COLS) <= 256 ? 256 : 512;
+  static constexpr int COLS = BN + S * (SFA_COLS + SFB_COLS) <= 256 ? 256 : 512;
+  static_assert(STAGE % 1024 == 0 && SMEM <= 232448, "stage layout");
+  static_assert(BN + S * (SFA_COLS + SFB_COLS) <= 512, "TMEM columns");
 };
+
+// Rewrites, in place, the scale rows of `groups` 128-row groups (16 bytes per row: 4 MMAs x 4
+// scales) into the tiles tcgen05.cp reads: tile (j, g) = MMA j, rows 128 g .. 128 g + 127, the
+// word of row r at index 4 * (r % 32) + r / 32.  One warp; every lane loads all it needs before
+// any lane stores.
+template <int GROUPS>
+__device__ __forceinline__ void scale_tiles_in_place(uint8_t* buf, int lane) {
+  uint4 w[GROUPS][4];
+#pragma unroll
+  for (int g = 0; g < GROUPS; ++g)
+#pragma unroll
+    for (int rq = 0; rq < 4; ++rq) w[g][rq] = *reinterpret_cast<const uint4*>(buf + 16 * (128 * g + 32 * rq + lane));
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < GROUPS; ++g) {
+    const uint32_t col[4][4] = {{w[g][0].x, w[g][1].x, w[g][2].x, w[g][3].x}, {w[g][0].y, w[g][1].y, w[g][2].y, w[g][3].y},
+                                {w[g][0].z, w[g][1].z, w[g][2].z, w[g][3].z}, {w[g][0].w, w[g][1].w, w[g][2].w, w[g][3].w}};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(buf + 512 * (j * GROUPS + g) + 16 * lane) = make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
+  }
+}
 
 template <int BN>
 __global__ void __launch_bounds__(224, 1)
@@ -407,15 +431,13 @@ __global__ void __launch_bounds__(224, 1)
                          const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                          const TcParams p) {
   using C = QCfg<BN>;
-  constexpr int S = kQStages;
+  constexpr int S = C::S;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = tc::align1024(smem_raw);
   auto sA = [&](int s) { return smem + s * C::STAGE; };
   auto sB = [&](int s) { return smem + s * C::STAGE + C::A; };
-  auto sSAr = [&](int s) { return smem + s * C::STAGE + C::A + C::B; };
-  auto sSAt = [&](int s) { return smem + s * C::STAGE + C::A + C::B + C::SFA; };
-  auto sSBr = [&](int s) { return smem + s * C::STAGE + C::A + C::B + 2 * C::SFA; };
-  auto sSBt = [&](int s) { return smem + s * C::STAGE + C::A + C::B + 2 * C::SFA + C::SFB; };
+  auto sSA = [&](int s) { return smem + s * C::STAGE + C::A + C::B; };
+  auto sSB = [&](int s) { return smem + s * C::STAGE + C::A + C::B + C::SFA; };
   __shared__ uint64_t full_bar[S], sf_bar[S], empty_bar[S], tfull_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int aborted;
@@ -458,8 +480,8 @@ __global__ void __launch_bounds__(224, 1)
         mbar_arrive_expect_tx(&full_bar[s], C::A + C::B + C::SFA + C::SFB);
         tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 128, m0);   // 128 bytes = 256 codes
         tma_load_2d(sB(s), &tmB, &full_bar[s], kb * 128, n0);
-        tma_load_2d(sSAr(s), &tmSA, &full_bar[s], kb * 16, m0); // 16 scales per row
-        tma_load_2d(sSBr(s), &tmSB, &full_bar[s], kb * 16, n0);
+        tma_load_2d(sSA(s), &tmSA, &full_bar[s], kb * 16, m0);  // 16 scales per row
+        tma_load_2d(sSB(s), &tmSB, &full_bar[s], kb * 16, n0);
         ++issued;
       }
       for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
@@ -473,22 +495,8 @@ __global__ void __launch_bounds__(224, 1)
         aborted = 1;
         break;
       }
-      // tile (j, g) = MMA j, rows 128 g .. 128 g + 127: word of row r at index 4 * (r % 32) + r / 32
-      auto rewrite = [&](const uint8_t* raw, uint8_t* tiles, int groups) {
-        for (int g = 0; g < groups; ++g) {
-          uint4 w[4];
-#pragma unroll
-          for (int rq = 0; rq < 4; ++rq) w[rq] = *reinterpret_cast<const uint4*>(raw + 16 * (128 * g + 32 * rq + lane));
-          const uint32_t col[4][4] = {{w[0].x, w[1].x, w[2].x, w[3].x}, {w[0].y, w[1].y, w[2].y, w[3].y},
-                                      {w[0].z, w[1].z, w[2].z, w[3].z}, {w[0].w, w[1].w, w[2].w, w[3].w}};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(tiles + 512 * (j * groups + g) + 16 * lane) =
-                make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
-        }
-      };
-      rewrite(sSAr(s), sSAt(s), 1);
-      rewrite(sSBr(s), sSBt(s), BN / 128);
+      scale_tiles_in_place<1>(sSA(s), lane);
+      scale_tiles_in_place<BN / 128>(sSB(s), lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sf_bar[s]);
@@ -508,11 +516,11 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t sfb0 = sfa0 + C::SFA_COLS;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSAt(s) + 512 * j)));
+          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSA(s) + 512 * j)));
 #pragma unroll
           for (int g = 0; g < BN / 128; ++g)
             tmem_cp_32x128b_x4(sfb0 + (BN / 32) * j + 4 * g,
-                               desc_rows16_noswizzle(smem_u32(sSBt(s) + 512 * (j * (BN / 128) + g))));
+                               desc_rows16_noswizzle(smem_u32(sSB(s) + 512 * (j * (BN / 128) + g))));
         }
         const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
         const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB(s)));
@@ -575,20 +583,21 @@ int launch_nvfp4(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
 // per instruction, the pairs in ascending order) with their 16-value E4M3 scales (one per 32
 // logical K) and the metadata nibbles; B = the activations as E2M1 with one E4M3 scale per 32 K.
 // Per stage (512 logical K): A one 128-byte swizzled box, B two; 16 scale bytes per row of each
-// operand, rewritten by warp 6 into the same TMEM tiles as the dense kernel (4 per instruction);
+// operand, rewritten in place by warp 6 into the same TMEM tiles as the dense kernel (4 per
+// instruction);
 // the metadata as two boxes of 128 rows x 16 bytes, copied into TMEM with tcgen05.cp.128x128b
 // (row m on lane m, 16 bytes = 256 logical K = 4 columns, chunk 2c in the low nibble of byte
 // c).  Rows beyond N arrive as zeros, which is not a legal nibble; warp 6 writes the legal 0x4
 // (pairs 0 and 1) there before the copy, and those rows' outputs are never stored.
 template <int BN>
 struct SCfg {
-  static constexpr int S = BN == 256 ? 2 : 3;
+  static constexpr int S = BN == 256 ? 2 : 4;
   static constexpr uint32_t A = kBM * 128;  // 128 rows x 256 stored FP4 = 512 logical K
   static constexpr uint32_t B = BN * 256;   // BN rows x 512 FP4, two 128-byte boxes
-  static constexpr uint32_t SFA = kBM * 16;
+  static constexpr uint32_t SFA = kBM * 16; // scale rows, rewritten in place into tiles
   static constexpr uint32_t SFB = BN * 16;
   static constexpr uint32_t E = kBM * 32;   // two boxes of 128 rows x 16 bytes
-  static constexpr uint32_t STAGE = A + B + 2 * SFA + 2 * SFB + E;
+  static constexpr uint32_t STAGE = A + B + SFA + SFB + E;
   static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
   static constexpr int E_COLS = 8;
   static constexpr int SFA_COLS = 16;             // 4 MMAs x 4 columns
@@ -610,11 +619,9 @@ __global__ void __launch_bounds__(224, 1)
   uint8_t* smem = tc::align1024(smem_raw);
   auto sA = [&](int s) { return smem + s * C::STAGE; };
   auto sB = [&](int s) { return sA(s) + C::A; };
-  auto sSAr = [&](int s) { return sB(s) + C::B; };
-  auto sSAt = [&](int s) { return sSAr(s) + C::SFA; };
-  auto sSBr = [&](int s) { return sSAt(s) + C::SFA; };
-  auto sSBt = [&](int s) { return sSBr(s) + C::SFB; };
-  auto sE = [&](int s) { return sSBt(s) + C::SFB; };
+  auto sSA = [&](int s) { return sB(s) + C::B; };
+  auto sSB = [&](int s) { return sSA(s) + C::SFA; };
+  auto sE = [&](int s) { return sSB(s) + C::SFB; };
   __shared__ uint64_t full_bar[S], sf_bar[S], empty_bar[S], tfull_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int aborted;
@@ -659,8 +666,8 @@ __global__ void __launch_bounds__(224, 1)
         tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 128, m0);  // 128 bytes = 256 stored codes
         tma_load_2d(sB(s), &tmB, &full_bar[s], kb * 256, n0);  // 2 x 128 bytes = 512 codes
         tma_load_2d(sB(s) + BN * 128, &tmB, &full_bar[s], kb * 256 + 128, n0);
-        tma_load_2d(sSAr(s), &tmSA, &full_bar[s], kb * 16, m0);  // 16 scales per row
-        tma_load_2d(sSBr(s), &tmSB, &full_bar[s], kb * 16, n0);
+        tma_load_2d(sSA(s), &tmSA, &full_bar[s], kb * 16, m0);  // 16 scales per row
+        tma_load_2d(sSB(s), &tmSB, &full_bar[s], kb * 16, n0);
         tma_load_2d(sE(s), &tmE, &full_bar[s], kb * 32, m0);  // 2 x 16 bytes of nibbles per row
         tma_load_2d(sE(s) + 2048, &tmE, &full_bar[s], kb * 32 + 16, m0);
         ++issued;
@@ -677,22 +684,8 @@ __global__ void __launch_bounds__(224, 1)
         aborted = 1;
         break;
       }
-      // tile (j, g) = MMA j, rows 128 g .. 128 g + 127: word of row r at index 4 * (r % 32) + r / 32
-      auto rewrite = [&](const uint8_t* raw, uint8_t* tiles, int groups) {
-        for (int g = 0; g < groups; ++g) {
-          uint4 w[4];
-#pragma unroll
-          for (int rq = 0; rq < 4; ++rq) w[rq] = *reinterpret_cast<const uint4*>(raw + 16 * (128 * g + 32 * rq + lane));
-          const uint32_t col[4][4] = {{w[0].x, w[1].x, w[2].x, w[3].x}, {w[0].y, w[1].y, w[2].y, w[3].y},
-                                      {w[0].z, w[1].z, w[2].z, w[3].z}, {w[0].w, w[1].w, w[2].w, w[3].w}};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(tiles + 512 * (j * groups + g) + 16 * lane) =
-                make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
-        }
-      };
-      rewrite(sSAr(s), sSAt(s), 1);
-      rewrite(sSBr(s), sSBt(s), BN / 128);
+      scale_tiles_in_place<1>(sSA(s), lane);
+      scale_tiles_in_place<BN / 128>(sSB(s), lane);
       for (int r = valid + lane; r < kBM; r += 32) {
         const uint4 legal = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
         *reinterpret_cast<uint4*>(sE(s) + 16 * r) = legal;
@@ -720,11 +713,11 @@ __global__ void __launch_bounds__(224, 1)
         tmem_cp_128x128b(e0 + 4, desc_rows16_noswizzle(smem_u32(sE(s) + 2048)));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSAt(s) + 512 * j)));
+          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSA(s) + 512 * j)));
 #pragma unroll
           for (int g = 0; g < BN / 128; ++g)
             tmem_cp_32x128b_x4(sfb0 + (BN / 32) * j + 4 * g,
-                               desc_rows16_noswizzle(smem_u32(sSBt(s) + 512 * (j * (BN / 128) + g))));
+                               desc_rows16_noswizzle(smem_u32(sSB(s) + 512 * (j * (BN / 128) + g))));
         }
         const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
         const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB(s)));

@@ -115,3 +115,36 @@ def test_gemm_sparse48_rejects():
     assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 0, 128, 512, y.data_ptr(), None) == sp.OK
     torch.cuda.synchronize()
     assert sp.last_device_error() == sp.OK
+
+
+def _sampled48(M, N, K, rows, d):
+    X, W = d["X"], d["W"]
+    v_ref, m_ref = oracle.compress_48(W, oracle.BF16)
+    vc, vs, vts = oracle.nvfp4_encode(v_ref, oracle.BF16)
+    Wd = _decompress48_f64(oracle.nvfp4_decode(vc, vs, vts), m_ref, N, K)
+    # the tensor scale of x is the whole tensor's; the sampled rows are encoded with it
+    _, _, xts = oracle.nvfp4_encode(X, oracle.BF16, block=32)
+    Xs = np.ascontiguousarray(X[rows])
+    xc, xs, _ = oracle.nvfp4_encode(Xs, oracle.BF16, tensor_scale=float(xts), block=32)
+    Y, S = oracle.gemm(oracle.nvfp4_decode(xc, xs, xts, block=32), Wd)
+    v, m = sp.prune_compress_48(to_dev(W, "bf16"))
+    xq = sp.quantize_nvfp4_block32(to_dev(X, "bf16"))
+    y = sp.gemm_sparse48(xq, sp.Sparse48(sp.quantize_nvfp4(v), m), K)
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
+    assert _bits32(xq.tensor_scale.item()) == _bits32(xts)
+    assert_gemm_close(y[torch.as_tensor(rows, device=y.device)], Y, S)
+
+
+def test_prefill_4096_sampled():
+    """The W4A4 prefill shape M = N = K = 4096 in the configuration the sweep times (256-wide
+    activation tiles): 24 sampled token rows x all 4096 outputs against the oracle."""
+    rows = np.sort(synth.rng(78).choice(4096, 24, replace=False))
+    _sampled48(4096, 4096, 4096, rows, synth.prefill_w4a4())
+
+
+def test_msweep_16384_sampled():
+    """The largest M of the sweep's W4A4 lines: x [16384, 5120], w [5120, 5120], 8 sampled rows."""
+    rows = np.sort(synth.rng(79).choice(16384, 8, replace=False))
+    d = {"X": synth.draw(synth.rng(16384), (16384, 5120), "bf16"), "W": synth.draw(synth.rng(0), (5120, 5120), "bf16")}
+    _sampled48(16384, 5120, 5120, rows, d)
