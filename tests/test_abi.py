@@ -110,3 +110,37 @@ def test_binding_refuses_cpu_tensors():
         sp.check_24(torch.zeros(4, 8, dtype=torch.float16))
     with pytest.raises(ValueError):
         sp.quantize_nvfp4(torch.zeros(4, 16))
+
+
+def test_pairwise48_host_validation():
+    """Pairwise 4:8 entry points reject bad arguments before any CUDA call."""
+    assert _raw("sp24_check_48", None, 7, 2, 16, None, None, None) == sp.ERR_DTYPE
+    assert _raw("sp24_check_48", None, sp.F16, 2, 12, None, None, None) == sp.ERR_SHAPE
+    assert _raw("sp24_check_48", None, sp.F16, -1, 16, None, None, None) == sp.ERR_SHAPE
+    assert _raw("sp24_check_48", None, sp.F16, 2, 16, None, None, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_check_48", 1, sp.F16, 2, 16, 16, None, None) == sp.ERR_ALIGN
+    assert _raw("sp24_prune_compress_48", None, sp.BF16, 2, 16, None, None, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_prune_compress_48", 16, sp.F32, 2, 16, 18, 16, None) == sp.ERR_ALIGN
+    assert _raw("sp24_prune_compress_48", None, sp.F16, 0, 16, None, None, None) == sp.OK  # empty: no-op
+    assert _raw("sp24_decompress_48", 16, None, sp.F16, 2, 16, 16, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_decompress_48", 16, 16, sp.F16, 2, 20, 16, None) == sp.ERR_SHAPE
+
+
+def test_block32_quantiser_and_sparse48_gemm_host_validation():
+    assert _raw("sp24_quantize_nvfp4_block32", None, sp.F16, 4, 48, None, None, None, 16, None, 0, None) == sp.ERR_SHAPE
+    assert _raw("sp24_quantize_nvfp4_block32", None, 7, 4, 64, None, None, None, 16, None, 0, None) == sp.ERR_DTYPE
+    assert _raw("sp24_quantize_nvfp4_block32", None, sp.F16, 4, 64, None, None, None, None, None, 0, None) == sp.ERR_INVALID_ARG
+    assert _raw("sp24_quantize_nvfp4_block32", 16, sp.F16, 4, 64, None, 16, 16, 16, None, 0, None) == sp.ERR_WORKSPACE
+    assert _raw("sp24_quantize_nvfp4_block32", 16, sp.F16, 4, 64, None, 24, 16, 16, 16, 256, None) == sp.ERR_ALIGN
+    L = sp.lib()
+    x = sp._Operand(sp.NVFP4_B32, 16, 16, 16)
+    w = sp._SparseOperand(sp.NVFP4, 16, 16, 16, 16)
+    call = lambda xo, wo, M, N, K, y=16: L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), M, N, K, y, None)
+    assert call(sp._Operand(sp.NVFP4, 16, 16, 16), w, 8, 128, 512) == sp.ERR_DTYPE
+    assert call(x, sp._SparseOperand(sp.BF16, 16, None, None, 16), 8, 128, 512) == sp.ERR_DTYPE
+    assert call(x, w, 8, 128, 256) == sp.ERR_SHAPE
+    assert call(x, w, -1, 128, 512) == sp.ERR_SHAPE
+    assert call(x, w, 0, 128, 512) == sp.OK  # empty: no-op
+    assert call(x, sp._SparseOperand(sp.NVFP4, 16, 16, 16, None), 8, 128, 512) == sp.ERR_INVALID_ARG
+    assert call(x, sp._SparseOperand(sp.NVFP4, 16, 16, 16, 8), 8, 128, 512) == sp.ERR_ALIGN
+    assert call(x, w, 8, 128, 512, y=None) == sp.ERR_INVALID_ARG
