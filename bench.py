@@ -165,6 +165,21 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ our arm
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: every rank takes part and every rank gets the maximum."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(world: int, step_bytes: int, ms_step: float) -> float:
+    """Whole-job algorithmic GB/s: each of the `world` replicas moves `step_bytes` per step."""
+    return world * step_bytes / (ms_step * 1e-3) / 1e9
+
+
 def run_ours(args, rank: int, world: int, dist) -> dict | None:
     import torch
 
@@ -285,14 +300,11 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     total_ms = t_start.elapsed_time(t_end)
     dom_ms = sum(ev[0].elapsed_time(ev[1]) for _, ev in windows) / len(windows)
 
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_step = total_ms / args.steps
     bytes_ = stage_bytes()
     step_bytes = sum(bytes_.values())
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = replica_value(world, step_bytes, ms_step)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     s0 = sets[0]
@@ -326,10 +338,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     # results are still correct after all the replays (cheap sanity, outside timing)
     assert sp.last_device_error() == sp.OK
     assert int(hnf.item()) == N * K // 4  # raw normal weights: every group fails the check
@@ -380,7 +389,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict | None:
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 3),
                      "launch_us": round(dom_ms * 1e3, 3), "launches_timed": len(windows),
                      "traffic": None if rec is None else rec["traffic_bytes_per_launch"]},
-        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(replica_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "steps": args.e2e_steps,
                 "h2d_bytes_per_step": hx.numel() * 2 + hw.numel() * 2,
                 "d2h_bytes_per_step": hyd.numel() * 4 + hys.numel() * 4 + 4},
