@@ -233,6 +233,7 @@ extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int
   }
   if (M == 0 || N == 0) return SP24_OK;
   if (!y) return SP24_ERR_INVALID_ARG;
+  if (!aligned(y, 4)) return SP24_ERR_ALIGN;
   if (K > 0 && !w->data) return SP24_ERR_INVALID_ARG;
   if (!aligned(w->data, 16)) return SP24_ERR_ALIGN;
   p.w = reinterpret_cast<const uint8_t*>(w->data);
@@ -275,6 +276,7 @@ extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_opera
   p.meta_row_bytes = K / 8;
   if (M == 0 || N == 0) return SP24_OK;
   if (!y) return SP24_ERR_INVALID_ARG;
+  if (!aligned(y, 4)) return SP24_ERR_ALIGN;
   if (K > 0 && (!w->values || !w->meta)) return SP24_ERR_INVALID_ARG;
   if (!aligned(w->values, 16) || !aligned(w->meta, 8)) return SP24_ERR_ALIGN;
   p.w = reinterpret_cast<const uint8_t*>(w->values);

@@ -950,6 +950,7 @@ extern "C" int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_opera
   if (M < 0 || N < 0 || K < 0 || K % 512) return SP24_ERR_SHAPE;
   if (M == 0 || N == 0) return SP24_OK;
   if (!y) return SP24_ERR_INVALID_ARG;
+  if (!aligned(y, 4)) return SP24_ERR_ALIGN;
   if (K > 0) {
     if (!x->data || !x->scales || !x->tensor_scale || !w->values || !w->scales || !w->tensor_scale || !w->meta)
       return SP24_ERR_INVALID_ARG;

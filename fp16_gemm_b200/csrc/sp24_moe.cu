@@ -167,6 +167,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   const int64_t n = T * topk;
   if (n == 0 || N == 0) return SP24_OK;
   if (!routing || !y) return SP24_ERR_INVALID_ARG;
+  if (!aligned(y, 4)) return SP24_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   if (K == 0) return cudaMemsetAsync(y, 0, (size_t)(n * N) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
 
@@ -369,6 +370,7 @@ extern "C" int sp24_moe_block(const sp24_operand* x, const int32_t* routing, con
   cudaStream_t s = as_stream(stream);
   if (H == 0 || T == 0) return SP24_OK;
   if (!y) return SP24_ERR_INVALID_ARG;
+  if (!aligned(y, 16)) return SP24_ERR_ALIGN;  // the combine writes y as float4 rows (H % 4 == 0)
   if (n == 0 || F == 0) return cudaMemsetAsync(y, 0, (size_t)(T * H) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
   if (!routing || !router_w || !x->data) return SP24_ERR_INVALID_ARG;
   if (!aligned(x->data, 16)) return SP24_ERR_ALIGN;

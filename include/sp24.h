@@ -164,7 +164,7 @@ int sp24_decompress_48(const void* values, const uint8_t* meta, int dtype, int64
  *      values [N, K/2] quantised with sp24_quantize_nvfp4 (scales -> [N, K/32], one per 16
  *      stored = 32 logical K), meta -> [N, K/16] from sp24_prune_compress_48 (every nibble
  *      legal; other metadata gives undefined results for its rows).
- *   y  device fp32 [M, N], written (not accumulated).
+ *   y  device fp32 [M, N], written (not accumulated), 4-byte aligned.
  * K % 512 == 0 (SP24_ERR_SHAPE otherwise); every operand pointer 16-byte aligned; M, N, K up to
  * 2^31 - 1.  Wrong formats: SP24_ERR_DTYPE.  One launch; nothing is allocated. */
 int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
@@ -279,7 +279,8 @@ int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* 
  * x: M rows (F16, BF16 or NVFP4); w: N rows (F16, BF16 or NVFP4).  16-bit x and 16-bit w
  * must have the same type; NVFP4 w is decoded in-kernel to x's type (bf16 when x is NVFP4).
  * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
- * aligned.  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
+ * aligned, y 4-byte aligned (SP24_ERR_ALIGN otherwise; the same holds for every GEMM entry
+ * point below).  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
  * workspace: device scratch of sp24_gemm_workspace_size() bytes (may be NULL when 0).
  * Kernels that split K across CTAs or warps combine partial sums with fp32 atomics, so two
  * identical calls may differ in the last bits of an output. */
@@ -358,7 +359,7 @@ int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, int64_t T, 
  *              gate and up share one tensor scale (sp24_nvfp4_group_tensor_scale); exactly one
  *              of w_gate_up (dense) or w_gate_up_sparse (2:4 values + nibbles, same packing)
  *   w_down     [E * H, F], NVFP4 dense or 2:4 (w_down_sparse), one of the two
- *   y          device fp32 [T, H], overwritten
+ *   y          device fp32 [T, H], overwritten, 16-byte aligned (written as 4-float vectors)
  *   Shapes: F % 64 and H % 128; dense K (H for gate/up, F for down) % 256, 2:4 K % 512;
  *   SP24_ERR_UNSUPPORTED otherwise.  Each routed row's down output is stored once and a token's
  *   slots are summed in slot order in fp32 (deterministic).

@@ -144,3 +144,18 @@ def test_block32_quantiser_and_sparse48_gemm_host_validation():
     assert call(x, sp._SparseOperand(sp.NVFP4, 16, 16, 16, None), 8, 128, 512) == sp.ERR_INVALID_ARG
     assert call(x, sp._SparseOperand(sp.NVFP4, 16, 16, 16, 8), 8, 128, 512) == sp.ERR_ALIGN
     assert call(x, w, 8, 128, 512, y=None) == sp.ERR_INVALID_ARG
+
+
+def test_output_alignment_checked_on_the_host():
+    """A y pointer that cannot hold fp32 stores (or, for the expert block, 4-float vectors) is
+    refused before any launch."""
+    L = sp.lib()
+    x = sp._Operand(sp.F16, 16, None, None)
+    w = sp._Operand(sp.F16, 16, None, None)
+    assert L.sp24_gemm_dense(ctypes.byref(x), ctypes.byref(w), 8, 8, 64, 18, None, 0, sp.ALGO_AUTO, None) == sp.ERR_ALIGN
+    sw = sp._SparseOperand(sp.F16, 16, None, None, 16)
+    assert L.sp24_gemm_sparse24(ctypes.byref(x), ctypes.byref(sw), 8, 8, 64, 2, None, 0, sp.ALGO_AUTO, None) == sp.ERR_ALIGN
+    xq = sp._Operand(sp.NVFP4_B32, 16, 16, 16)
+    wq = sp._SparseOperand(sp.NVFP4, 16, 16, 16, 16)
+    assert L.sp24_gemm_sparse48(ctypes.byref(xq), ctypes.byref(wq), 8, 128, 512, 6, None) == sp.ERR_ALIGN
+
