@@ -604,6 +604,7 @@ extern "C" int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales
   int64_t nbytes = rows * cols / 2;
   if (nbytes == 0) return SP24_OK;
   if (!codes || !scales || !tensor_scale || !out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(out, elem_bytes(out_dtype))) return SP24_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   if (out_dtype == SP24_F32)
     decode_kernel<SP24_F32><<<full_wave_grid(decode_kernel<SP24_F32>, kThreads, blocks_for(nbytes)), kThreads, 0, s>>>(codes, scales, tensor_scale, nbytes, out);

@@ -558,6 +558,7 @@ extern "C" int sp24_check_24(const void* w, int dtype, int op, const int64_t* sh
   int st = parse_shape(op, shape, ndim, &G, &L);
   if (st) return st;
   if (G > 0 && (!w || !pass)) return SP24_ERR_INVALID_ARG;
+  if (G > 0 && !aligned(w, eb)) return SP24_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   if (n_fail && cudaMemsetAsync(n_fail, 0, sizeof(int32_t), s) != cudaSuccess) return SP24_ERR_CUDA;
   if (G == 0) return launch_status(0);
@@ -602,6 +603,7 @@ extern "C" int sp24_prune_compress_24(const void* w, int dtype, int op, const in
   if (st) return st;
   if (G == 0) return SP24_OK;
   if (!w || !values || !meta) return SP24_ERR_INVALID_ARG;
+  if (!aligned(w, eb) || !aligned(values, eb)) return SP24_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   int nl = 0;
   int64_t p_done = 0;  // meta bytes (group pairs) already written
@@ -646,6 +648,7 @@ extern "C" int sp24_decompress_24(const void* values, const uint8_t* meta, int d
   if (st) return st;
   if (G == 0) return SP24_OK;
   if (!values || !meta || !w_out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(values, eb) || !aligned(w_out, eb)) return SP24_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   int nl = 0;
   int64_t g_done = 0;

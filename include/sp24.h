@@ -11,7 +11,9 @@
  *   - Pointers named as device pointers must point to memory of the current CUDA device;
  *     `shape` arrays and the operand structs are host memory and are read before the call
  *     returns.  The caller owns every buffer; the library never allocates device memory.
- *   - Tensors are dense and row-major (C order).  GEMM operands are K-contiguous.
+ *   - Tensors are dense and row-major (C order).  GEMM operands are K-contiguous.  Every
+ *     element pointer needs at least the alignment of its element type (SP24_ERR_ALIGN
+ *     otherwise); calls that need more say so.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream) and returns a status.  Argument errors are detected on the host and return a
  *     status without launching anything.  SP24_ERR_CUDA reports a failed launch.  Kernels

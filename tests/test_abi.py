@@ -159,3 +159,12 @@ def test_output_alignment_checked_on_the_host():
     wq = sp._SparseOperand(sp.NVFP4, 16, 16, 16, 16)
     assert L.sp24_gemm_sparse48(ctypes.byref(xq), ctypes.byref(wq), 8, 128, 512, 6, None) == sp.ERR_ALIGN
 
+
+def test_element_alignment_checked_on_the_host():
+    """An element pointer without its type's natural alignment is refused before any launch."""
+    shp = (ctypes.c_int64 * 4)(4, 8)
+    assert _raw("sp24_check_24", 17, sp.F16, sp.OP_MATMUL, shp, 2, 16, None, None) == sp.ERR_ALIGN
+    assert _raw("sp24_prune_compress_24", 16, sp.F32, sp.OP_MATMUL, shp, 2, 18, 16, None) == sp.ERR_ALIGN
+    assert _raw("sp24_decompress_24", 16, 16, sp.BF16, sp.OP_MATMUL, shp, 2, 19, None) == sp.ERR_ALIGN
+    assert _raw("sp24_dequantize_nvfp4", 16, 16, 16, 4, 32, sp.F32, 18, None) == sp.ERR_ALIGN
+
