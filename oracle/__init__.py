@@ -16,6 +16,11 @@ ctypes over numpy arrays.  Pages followed, by title:
 * "NVFP4 Without FP4 Hardware" -- "Convert BF16 to NVFP4 yourself", "The shared global
   scale", "Bit-exact check against lyf's ModelOpt output".
 
+Pairwise 4:8 (``check_48`` / ``compress_48`` / ``decompress_48``) and the 32-value NVFP4 block
+(``nvfp4_encode(..., block=32)``) follow readings R21 / R22 of the same pages ("What 2:4
+actually is", carried over to pairs; the block size the sparse FP4 MMA reads); they are pinned
+against brute force over the six pair choices and against ml_dtypes' roundings.
+
 Parity unpinned: the NVFP4 scale and rounding formulae (tensor scale = amax / 2688, block
 scale = E4M3(bmax / (6 s_t)), code = E2M1(|t| / (dec(sb) s_t)), all RNE) are a reading; the
 pages state the format but print no worked example, so only their properties (sizes,

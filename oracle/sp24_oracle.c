@@ -31,6 +31,12 @@
  *       magnitude code is 0.  Packing: element 2i in the low nibble.
  *   R5  A sparse NVFP4 operand quantises the compressed values [N, K/2]: one block scale per
  *       16 stored values.
+ *   R21 Pairwise 4:8 (the sparse unit of the tensor cores' packed-FP4 MMA is a pair of
+ *       entries): chunks of 8 along K; a chunk passes when at most two of its four pairs hold
+ *       a nonzero; pruning keeps the two pairs of largest fp32 |a| + |b| (NaN highest, ties to
+ *       the lower pair); nibble i0 | i1 << 2 per chunk, stored as in R3.
+ *   R22 The activations of the pairwise-4:8 FP4 GEMM use the R4 steps over 32-value blocks
+ *       (that MMA reads one scale per 32 K for both operands).
  */
 #include <math.h>
 #include <stdint.h>
