@@ -37,7 +37,7 @@ enum {
   SP24_ERR_SHAPE = 2,         /* shape violates the operation's rule (e.g. C % 4 != 0) */
   SP24_ERR_DTYPE = 3,         /* element type not accepted by this call */
   SP24_ERR_ALIGN = 4,         /* a pointer is not aligned as the call requires */
-  SP24_ERR_UNSUPPORTED = 5,   /* valid request that no kernel of this build serves */
+  SP24_ERR_UNSUPPORTED = 5,   /* valid request that no kernel of the library serves */
   SP24_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
   SP24_ERR_DEVICE_TIMEOUT = 7,/* a bounded device-side wait gave up */
   SP24_ERR_WORKSPACE = 8      /* workspace missing or smaller than the size query says */
