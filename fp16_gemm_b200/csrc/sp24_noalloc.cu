@@ -1,16 +1,20 @@
 // NVFP4 quantisation for callers that cannot allocate device memory.
 //
 // sp24_quantize_nvfp4 needs a few bytes of scratch (the running amax of |T|), which the caller
-// normally passes as `workspace`.  Some callers have no way to get one: code that runs while a
-// CUDA graph is being captured in relaxed or global mode (cudaMalloc is illegal there), runtimes
-// that hand out only a fixed arena of operand buffers and no general-purpose allocator, and
-// plugins whose host code must not touch the device allocator at all.  For them this entry
-// point keeps its scratch in a file-scope __device__ array instead.
+// normally passes as `workspace`.  Some callers have no way to get one: runtimes that hand out
+// only a fixed arena of operand buffers and no general-purpose allocator, plugins hosted by a
+// framework whose own caching allocator owns the device memory (a direct cudaMalloc would bypass
+// its budget), and latency-bound host loops that must not call cudaMalloc at all because it can
+// synchronise the device.  For them this entry point keeps its scratch in a file-scope
+// __device__ array instead.
 //
 // The array exists once per device that loads the library and lives until the process exits.
 // Every call on a device shares it and it keeps the last call's contents, so the amax word is
 // cleared (cudaMemsetAsync, which allocates nothing) at the start of every call, and two calls
 // whose work overlaps on the GPU (different streams, no ordering between them) race on it.
+// The array's device address is looked up once per device and cached; a cudaDeviceReset in the
+// same process invalidates that address, so a process that resets a device must not call this
+// entry point on that device afterwards.
 #include <mutex>
 
 #include "sp24_internal.cuh"

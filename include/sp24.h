@@ -192,15 +192,17 @@ int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
                         float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
                         void* stream);
 
-/* The same quantisation for callers that cannot allocate device memory (code running inside a
- * CUDA graph capture where cudaMalloc is not allowed, runtimes that only hand out fixed operand
- * buffers, plugins that must not touch the allocator).  No counterpart on the source pages: it
- * is a property of this library, not of the method.
+/* The same quantisation for callers that cannot allocate device memory: runtimes that only hand
+ * out a fixed arena of operand buffers, plugins whose host framework owns the device allocator,
+ * and host loops that must not call cudaMalloc (it can synchronise the device).  No counterpart
+ * on the source pages: it is a property of this library, not of the method.
  *   Arguments as sp24_quantize_nvfp4, without the workspace.  The scratch is a 256-byte
  *   __device__ array inside the library, one per device, kept until the process exits; the
  *   quantiser needs 4 bytes of it (the amax word) for every tensor shape, and a request needing
  *   more than 256 bytes returns SP24_ERR_WORKSPACE.  The first call on each device looks up the
- *   array's device address; make that first call before any stream capture begins.  The call
+ *   array's device address (cudaGetSymbolAddress) and caches it; make that first call before
+ *   any stream capture begins, and do not call this entry point on a device after a
+ *   cudaDeviceReset of it in the same process (the cached address is then stale).  The call
  *   allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).  All calls on a
  *   device share the array: each call clears the amax word first, and calls whose GPU work can
  *   overlap (different streams without ordering) race on it. */
@@ -277,9 +279,13 @@ int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* 
                     void* stream);
 
 /* ----------------------------------------------------------------------- a4-a6: GEMM */
-/* Y[m, n] = sum_k x[m, k] * w[n, k] with fp32 accumulation, Y fp32 [M, N] row-major (device).
+/* [P1] "The roofline is the whole argument" and [P5] "Why NVFP4 helps without FP4 hardware":
+ * the dense product whose bytes (decode) or FLOPs (prefill) the sparse form is compared with.
+ * Y[m, n] = sum_k x[m, k] * w[n, k] with fp32 accumulation, Y fp32 [M, N] row-major (device).
  * x: M rows (F16, BF16 or NVFP4); w: N rows (F16, BF16 or NVFP4).  16-bit x and 16-bit w
- * must have the same type; NVFP4 w is decoded in-kernel to x's type (bf16 when x is NVFP4).
+ * must have the same type.  Where NVFP4 meets NVFP4 (W4A4) both stay 4-bit and the tensor core
+ * applies the block scales.  NVFP4 w with 16-bit x is decoded inside the kernel to x's type at
+ * M <= 64; at larger M it is first expanded to x's type in the workspace (exact values).
  * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
  * aligned, y 4-byte aligned (SP24_ERR_ALIGN otherwise; the same holds for every GEMM entry
  * point below).  M == 0 or N == 0 is a no-op; K == 0 writes zeros.

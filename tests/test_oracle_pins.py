@@ -685,3 +685,39 @@ def test_block32_shape_rules(oracle):
         oracle.nvfp4_encode(np.zeros((1, 48), np.float32), oracle.F32, block=32)
     with pytest.raises(oracle.OracleError):
         oracle.nvfp4_encode(np.zeros((1, 64), np.float32), oracle.F32, block=8)
+
+
+# ----------------------------------------------------------------------------- input decoding
+
+def _same_doubles(got, want):
+    """Equal as numbers, NaN where the other is NaN, and the sign of zero kept."""
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+
+
+def test_to_double_f16_every_pattern(oracle):
+    """Every GEMM parity check decodes its inputs through to_double.  For IEEE binary16 the
+    value of each of the 65,536 patterns is fixed by the format (subnormals f * 2^-24, inf,
+    NaN, signed zero); numpy's own half -> double cast is the independent check."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    _same_doubles(oracle.to_double(bits.view(np.float16), oracle.F16),
+                  bits.view(np.float16).astype(np.float64))
+
+
+def test_to_double_bf16_every_pattern(oracle):
+    """bfloat16 is the upper half of a binary32; ml_dtypes' bfloat16 -> double cast (its own
+    implementation, not the oracle's) must agree on all 65,536 patterns."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    _same_doubles(oracle.to_double(bits, oracle.BF16),
+                  bits.view(ml_dtypes.bfloat16).astype(np.float64))
+
+
+def test_to_double_f32_passthrough(oracle):
+    """fp32 entries widen exactly (a sample of patterns across every exponent)."""
+    g = np.random.default_rng(7)
+    bits = g.integers(0, 1 << 32, size=1 << 16, dtype=np.uint64).astype(np.uint32)
+    with np.errstate(invalid="ignore"):
+        want = bits.view(np.float32).astype(np.float64)
+    _same_doubles(oracle.to_double(bits.view(np.float32), oracle.F32), want)

@@ -1,8 +1,9 @@
 """The allocation-free quantisation entry point, called through the C ABI.
 
-sp24_quantize_nvfp4_noalloc serves callers that cannot allocate device memory (for example code
-running under CUDA graph capture, or runtimes with a fixed buffer arena): it keeps its scratch
-in a __device__ array inside the library instead of a caller workspace.  Its results must equal
+sp24_quantize_nvfp4_noalloc serves callers that cannot allocate device memory (runtimes with a
+fixed buffer arena, plugins whose host framework owns the allocator, host loops that must not
+call cudaMalloc): it keeps its scratch in a __device__ array inside the library instead of a
+caller workspace.  Its results must equal
 those of sp24_quantize_nvfp4 (bit for bit: codes, block scales and tensor scale are exact),
 including on consecutive calls that reuse the shared scratch.  This file sorts last so that a
 run stopping at the first failure has already run every other test."""
@@ -13,6 +14,7 @@ import pytest
 import torch
 
 import fp16_gemm_b200 as sp
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -51,6 +53,14 @@ def _assert_same(a, b):
         assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
 
 
+def _assert_oracle(t_np: np.ndarray, dtype_code: int, got, ts_in=None):
+    """The no-alloc result against the CPU oracle's encoder (bit for bit)."""
+    codes, scales, ts = oracle.nvfp4_encode(t_np, dtype_code, tensor_scale=ts_in)
+    assert np.array_equal(got[0].cpu().numpy(), codes)
+    assert np.array_equal(got[1].cpu().numpy(), scales)
+    assert np.float32(got[2].item()) == np.float32(ts)
+
+
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     g = synth.rng(1234)
     # two calls in a row on different tensors: the second must not see the first's amax
@@ -61,6 +71,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         ref, got = _quantize_both(t, sp.BF16)
         _assert_same(ref, got)
         assert got[2].item() > 0
+        _assert_oracle(arr, oracle.BF16, got)
 
 
 def test_noalloc_decode_weight_and_shared_scale():
@@ -68,6 +79,8 @@ def test_noalloc_decode_weight_and_shared_scale():
     t = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).cuda()
     ref, got = _quantize_both(t, sp.BF16)
     _assert_same(ref, got)
+    _assert_oracle(np.ascontiguousarray(w[:512]), oracle.BF16,
+                   (got[0][:512], got[1][:512], got[2]), ts_in=float(got[2].item()))
     shared = torch.tensor([float(ref[2].item()) * 4], dtype=torch.float32, device="cuda")
     ref2, got2 = _quantize_both(t, sp.BF16, ts_in=shared)
     _assert_same(ref2, got2)
