@@ -25,7 +25,17 @@ launch duration (for `roofline`) is measured inside the timed region.  The per-s
 `value` is the whole step's algorithmic HBM traffic divided by the step time (GB/s); the GEMV
 comparison (dense vs 2:4 sparse: TFLOP/s, GB/s, speedup) is in `gemv`.
 
+After the timed step (N = 1 only) the line gains `per_config`: every config of the workload
+list at full size, each GEMM timed on prepared operands from CUDA-graph replays over operand
+sets whose inputs exceed twice the L2 -- config 1 (FP16 toy), 2 (decode W4A16 GEMV), 3 (W4A4
+4096^3: dense, element 2:4, pairwise 4:8 on the sparse FP4 MMA), 4 (routed experts), 5a / 5b
+(M sweep, FP16 and NVFP4) and 5c (conv check + compress) -- each with dense and sparse time,
+dense-equivalent TFLOP/s, algorithmic GB/s, arithmetic intensity, the binding roofline's
+fraction and the sparse/dense speedup; `roofline_compute` is config 3's dense FP4 GEMM against
+the dense FP4 tensor peak.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--sweep] [--no-per-config]
 
 With --impl reference the CPU oracle (oracle/, plain scalar C) is timed on the host cores on
 a bounded row sample of the same workload: that arm is a reported baseline, not the target.
@@ -437,33 +447,64 @@ def cpu_baseline(budget_s: float, steps: int = 1):
 
 # ------------------------------------------------------------------------------ per-shape sweep
 
-def run_sweep(args) -> None:
-    """One JSON line per (workload, shape, dense|sparse24): GEMM time on prepared operands, with
-    enough rotating weight copies that each launch reads its operands from DRAM."""
+L2_BYTES = 126e6
+
+
+def tensor_peaks():
+    """Roofline denominators: (HBM GB/s, {pipe: TFLOP/s}, {pipe: where it came from}).
+
+    HBM copy and dense bf16 GEMM are the measured figures of MEASURED_PEAKS.json (the
+    profiling recipe's fallback when absent).  The FP4 pipes come from this repository's own MMA
+    microbenchmark (`bench.py --peaks`, written to profiles/peaks.json) when it is present, else
+    from the measured bf16 figure x 4 (dense, the nominal 9 / 2.25 PF ratio) and x 8 (2:4,
+    dense-equivalent); 16-bit 2:4 counts dense-equivalent FLOPs at twice the measured bf16 rate."""
+    hbm, kind = peaks()
+    bf16, bkind = 1590.0, "fallback"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16, bkind = float(json.load(f)["bf16_tflops"]), "measured bf16 GEMM"
+    except Exception:
+        pass
+    tp = {"f16": bf16, "f16.sp": 2 * bf16, "nvfp4": 4 * bf16, "nvfp4.sp": 8 * bf16}
+    src = {"hbm": kind, "f16": bkind, "f16.sp": bkind + " x 2", "nvfp4": bkind + " x 4",
+           "nvfp4.sp": bkind + " x 8"}
+    try:
+        with open(os.path.join(ROOT, "profiles", "peaks.json")) as f:
+            mb = json.load(f)["mma_tflops"]
+        for pipe in ("nvfp4", "nvfp4.sp"):
+            if pipe in mb:
+                tp[pipe] = float(mb[pipe])
+                src[pipe] = "MMA microbenchmark (profiles/peaks.json)"
+    except Exception:
+        pass
+    return hbm, tp, src
+
+
+def _copies(set_bytes: float, lo: int = 2, hi: int = 64) -> int:
+    """Operand sets to rotate over so the inputs of consecutive launches exceed twice the L2."""
+    return int(max(lo, min(hi, -(-2 * L2_BYTES // max(set_bytes, 1)))))
+
+
+def sweep(emit, full: bool) -> None:
+    """One record per (config, shape) with dense and sparse forms side by side: GEMM time on
+    prepared operands from CUDA-graph replays over rotating operand copies whose inputs total
+    more than twice the L2, TFLOP/s (dense-equivalent), algorithmic GB/s, arithmetic intensity,
+    the binding roofline and its fraction, and the sparse/dense speedup.  `full` adds the rows
+    beyond the five configs (expert block, output-head quantisation, pairwise 4:8 on it)."""
     import torch
 
     import fp16_gemm_b200 as sp
     import synth
 
-    torch.cuda.set_device(0)
-    peak_hbm, kind = peaks()
-    peak_bf16 = 1717.8
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak_bf16 = float(json.load(f)["bf16_tflops"])
-    except Exception:
-        kind = "fallback"
-        peak_bf16 = 1590.0
-    # tensor peaks per pipe: measured bf16 dense; FP4 dense = bf16 x 4 (nominal 9 / 2.25 PF);
-    # 2:4 sparse pipes count dense-equivalent FLOPs at twice the dense rate
-    tensor_peak = {"f16": peak_bf16, "f16.sp": 2 * peak_bf16, "nvfp4": 4 * peak_bf16, "nvfp4.sp": 8 * peak_bf16}
-    dev = torch.device("cuda", 0)
+    peak_hbm, tensor_peak, peak_src = tensor_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
     t16 = lambda a, d: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if d == "bf16"
-                        else torch.from_numpy(a)).to(dev)
+                        else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
 
-    def timeit(fn, reps=20):
-        """Median over 5 replays of a CUDA graph of `reps` back-to-back launches (rotating
-        operand copies), per launch in microseconds: no host time between launches."""
+    def timeit(fn, n_sets, reps=20):
+        """Median over 5 replays of a CUDA graph of back-to-back launches cycling through the
+        operand sets (at least `reps` launches and every set once), per launch in us."""
+        reps = max(reps, n_sets)
         for r in range(3):
             fn(r)
         torch.cuda.synchronize()
@@ -481,6 +522,7 @@ def run_sweep(args) -> None:
             b.record()
             torch.cuda.synchronize()
             times.append(a.elapsed_time(b) * 1e3 / reps)
+        del g
         return statistics.median(times)
 
     def clone_op(o):
@@ -491,14 +533,26 @@ def run_sweep(args) -> None:
     def op_bytes(t):
         if isinstance(t, sp.NVFP4Tensor):
             return t.codes.numel() + t.scales.numel() + 4
-        if isinstance(t, sp.Sparse24):
+        if isinstance(t, (sp.Sparse24, sp.Sparse48)):
             return op_bytes(t.values) + t.meta.numel()
         return t.numel() * t.element_size()
 
+    def record(us, flops, byts, pipe):
+        ai = flops / byts
+        ridge = tensor_peak[pipe] * 1e12 / (peak_hbm * 1e9)
+        tflops = flops / (us * 1e-6) / 1e12
+        gbs = byts / (us * 1e-6) / 1e9
+        bound = "hbm" if ai < ridge else "tensor"
+        frac = gbs / peak_hbm if bound == "hbm" else tflops / tensor_peak[pipe]
+        return {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(gbs, 1), "bytes": int(byts),
+                "AI": round(ai, 1), "bound": bound, "pipe": pipe, "frac": round(frac, 3),
+                "frac_tensor": round(tflops / tensor_peak[pipe], 3), "frac_hbm": round(gbs / peak_hbm, 3)}
+
     selections = []
 
-    def case(workload, M, N, K, xdt, wdt, X, W):
-        """X, W numpy storage; xdt in {f16,bf16,nvfp4}; wdt in {f16,bf16,nvfp4}."""
+    def case(config, workload, M, N, K, xdt, wdt, X, W):
+        """X, W numpy storage; xdt in {f16, bf16, nvfp4}; wdt in {f16, bf16, nvfp4}: the dense
+        GEMM on the pruned weight against the 2:4 GEMM on its compressed form."""
         x = t16(X, "f16" if xdt == "f16" else "bf16")
         if xdt == "nvfp4":
             x = sp.quantize_nvfp4(x)
@@ -507,34 +561,27 @@ def run_sweep(args) -> None:
         wd = sp.decompress_24(v, m, w16.shape) if wdt != "nvfp4" else w16  # dense on pruned W
         dense = sp.quantize_nvfp4(w16) if wdt == "nvfp4" else wd
         sparse = sp.Sparse24(sp.quantize_nvfp4(v) if wdt == "nvfp4" else v, m)
+        del w16, wd, v
         res = {}
+        flops = 2.0 * M * N * K
         for name, wop in (("dense", dense), ("sparse24", sparse)):
-            wb = op_bytes(wop)
-            copies = max(1, min(8, int(256e6 // max(wb, 1))))
-            wops = [wop] + [clone_op(wop) for _ in range(copies - 1)]
+            wb, xb = op_bytes(wop), op_bytes(x)
+            n = _copies(wb + xb)
+            sets = [(x, wop)] + [(clone_op(x), clone_op(wop)) for _ in range(n - 1)]
             y = torch.empty((M, N), dtype=torch.float32, device=dev)
-            if name == "dense":
-                ws_b = sp.gemm_workspace_bytes(x, wop, False, M, N, K)
-                ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev)
-                fn = lambda r: sp.gemm_dense(x, wops[r % copies], out=y, workspace=ws if ws_b else None)
+            sparse_ = name == "sparse24"
+            ws_b = sp.gemm_workspace_bytes(x, wop, sparse_, M, N, K)
+            ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev) if ws_b else None
+            if sparse_:
+                fn = lambda r: sp.gemm_sparse24(sets[r % n][0], sets[r % n][1], K, out=y, workspace=ws)
             else:
-                ws_b = sp.gemm_workspace_bytes(x, wop, True, M, N, K)
-                ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev)
-                fn = lambda r: sp.gemm_sparse24(x, wops[r % copies], K, out=y, workspace=ws if ws_b else None)
-            us = timeit(fn)
-            byts = op_bytes(x) + wb + M * N * 4
-            flops = 2.0 * M * N * K
-            ai = flops / byts
-            pipe = ("nvfp4" if xdt == "nvfp4" and wdt == "nvfp4" and name == "dense" else
-                    "f16.sp" if name == "sparse24" else "f16")
-            ridge = tensor_peak[pipe] * 1e12 / (peak_hbm * 1e9)
-            tflops = flops / (us * 1e-6) / 1e12
-            gbs = byts / (us * 1e-6) / 1e9
-            bound = "hbm" if ai < ridge else "tensor"
-            frac = gbs / peak_hbm if bound == "hbm" else tflops / tensor_peak[pipe]
-            res[name] = {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(gbs, 1),
-                         "bytes": byts, "AI": round(ai, 1), "bound": bound, "pipe": pipe,
-                         "frac": round(frac, 3)}
+                fn = lambda r: sp.gemm_dense(sets[r % n][0], sets[r % n][1], out=y, workspace=ws)
+            us = timeit(fn, n)
+            pipe = ("nvfp4" if xdt == "nvfp4" and wdt == "nvfp4" and not sparse_ else
+                    "f16.sp" if sparse_ else "f16")
+            res[name] = record(us, flops, xb + wb + M * N * 4, pipe)
+            res[name]["input_sets"] = n
+            del sets, y, ws
         # the dense / 2:4 choice the library makes for this shape without measuring (its rule
         # of measured crossovers) against the faster of the two just timed
         fmt = {"f16": sp.F16, "bf16": sp.BF16, "nvfp4": sp.NVFP4}
@@ -545,78 +592,121 @@ def run_sweep(args) -> None:
         selections.append({"workload": workload, "M": M, "rule": "sparse24" if rule_sparse else "dense",
                            "faster": "sparse24" if faster_sparse else "dense",
                            "loss": round(chosen / min(res["dense"]["us"], res["sparse24"]["us"]) - 1.0, 3)})
-        line = {"sweep": workload, "M": M, "N": N, "K": K, "x": xdt, "w": wdt, **res,
-                "sparse_dense_speedup": round(res["dense"]["us"] / res["sparse24"]["us"], 3),
-                "selected": "sparse24" if rule_sparse else "dense",
-                "peaks": {"hbm_gbs": peak_hbm, "tensor_tflops": tensor_peak, "kind": kind}}
-        print(json.dumps(line), flush=True)
+        emit({"config": config, "sweep": workload, "M": M, "N": N, "K": K, "x": xdt, "w": wdt, **res,
+              "sparse_dense_speedup": round(res["dense"]["us"] / res["sparse24"]["us"], 3),
+              "selected": "sparse24" if rule_sparse else "dense"})
 
-    d = synth.fp16_toy()
-    case("fp16_toy", 16, 256, 512, "f16", "f16", d["X"], d["W"])
-    d = synth.decode_nvfp4()
-    case("decode_w4a16", 8, 5120, 5120, "bf16", "nvfp4", d["X"], d["W"])
-    d = synth.prefill_w4a4()
-    case("prefill_w4a4", 4096, 4096, 4096, "nvfp4", "nvfp4", d["X"], d["W"])
-    g = synth.rng(0)
-    W16 = synth.draw(g, (5120, 5120), "f16")
-    Wb = synth.draw(synth.rng(0), (5120, 5120), "bf16")
-    for Mv in (1, 16, 128, 1024, 4096, 16384):
-        X16 = synth.draw(synth.rng(Mv), (Mv, 5120), "f16")
-        case("msweep_fp16", Mv, 5120, 5120, "f16", "f16", X16, W16)
-        Xb = synth.draw(synth.rng(Mv), (Mv, 5120), "bf16")
-        case("msweep_nvfp4_w4a16", Mv, 5120, 5120, "bf16", "nvfp4", Xb, Wb)
-        case("msweep_nvfp4_w4a4", Mv, 5120, 5120, "nvfp4", "nvfp4", Xb, Wb)
-    def case48(workload, M, N, K, X, W):
+    def case48(config, workload, M, N, K, X, W):
         """W4A4 on the sparse FP4 MMA (pairwise 4:8 weight, activations in 32-value blocks)
         against the dense W4A4 GEMM of the same weight (NVFP4, 16-value blocks)."""
         xb, wb16 = t16(X, "bf16"), t16(W, "bf16")
         x16, x32 = sp.quantize_nvfp4(xb), sp.quantize_nvfp4_block32(xb)
         v, m = sp.prune_compress_48(wb16)
         dense, sparse = sp.quantize_nvfp4(wb16), sp.Sparse48(sp.quantize_nvfp4(v), m)
+        del xb, wb16, v
         y = torch.empty((M, N), dtype=torch.float32, device=dev)
         flops = 2.0 * M * N * K
-        line = {"sweep": workload, "M": M, "N": N, "K": K, "x": "nvfp4", "w": "nvfp4"}
+        line = {"config": config, "sweep": workload, "M": M, "N": N, "K": K, "x": "nvfp4", "w": "nvfp4"}
         for name, wop, xop, pipe in (("dense", dense, x16, "nvfp4"), ("sparse48", sparse, x32, "nvfp4.sp")):
-            wbytes = op_bytes(wop.values) + wop.meta.numel() if name == "sparse48" else op_bytes(wop)
-            copies = max(1, min(8, int(256e6 // max(wbytes, 1))))
-            wops = [wop] + [clone_op(wop) for _ in range(copies - 1)]
+            wbytes, xbytes = op_bytes(wop), op_bytes(xop)
+            n = _copies(wbytes + xbytes)
+            sets = [(xop, wop)] + [(clone_op(xop), clone_op(wop)) for _ in range(n - 1)]
             if name == "dense":
-                fn = lambda r: sp.gemm_dense(xop, wops[r % copies], out=y)
+                fn = lambda r: sp.gemm_dense(sets[r % n][0], sets[r % n][1], out=y)
             else:
-                fn = lambda r: sp.gemm_sparse48(xop, wops[r % copies], K, out=y)
-            us = timeit(fn)
-            byts = xop.codes.numel() + xop.scales.numel() + wbytes + M * N * 4
-            tflops = flops / (us * 1e-6) / 1e12
-            line[name] = {"us": round(us, 3), "TFLOP/s": round(tflops, 2), "GB/s": round(byts / us / 1e3, 1),
-                          "bytes": byts, "pipe": pipe, "frac_tensor": round(tflops / tensor_peak[pipe], 3)}
+                fn = lambda r: sp.gemm_sparse48(sets[r % n][0], sets[r % n][1], K, out=y)
+            us = timeit(fn, n)
+            line[name] = record(us, flops, xbytes + wbytes + M * N * 4, pipe)
+            line[name]["input_sets"] = n
+            del sets
         line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse48"]["us"], 3)
-        print(json.dumps(line), flush=True)
+        emit(line)
 
+    # config 1: FP16 2:4 toy (L2-resident by size: a correctness configuration)
+    d = synth.fp16_toy()
+    case("1", "fp16_toy", 16, 256, 512, "f16", "f16", d["X"], d["W"])
+    # config 2: decode-shaped W4A16 GEMV
+    d = synth.decode_nvfp4()
+    case("2", "decode_w4a16", 8, 5120, 5120, "bf16", "nvfp4", d["X"], d["W"])
+    # config 3: prefill W4A4 4096^3, dense vs element 2:4 vs pairwise 4:8 (sparse FP4 MMA)
     d = synth.prefill_w4a4()
-    case48("w4a4_pairwise48", 4096, 4096, 4096, d["X"], d["W"])
-    for Mv in (128, 1024, 4096, 16384):
-        case48("msweep_w4a4_pairwise48", Mv, 5120, 5120, synth.draw(synth.rng(Mv), (Mv, 5120), "bf16"), Wb)
-
+    case("3", "prefill_w4a4", 4096, 4096, 4096, "nvfp4", "nvfp4", d["X"], d["W"])
+    case48("3", "prefill_w4a4_pairwise48", 4096, 4096, 4096, d["X"], d["W"])
+    del d
+    # config 4: routed experts, 4096 tokens x top-10 of 512 experts [512, 2048], bf16 x, NVFP4
+    # experts dense and 2:4 (every expert is touched: each call reads all of them once, 302 MB
+    # dense / 218 MB 2:4, beyond the L2)
+    d = synth.moe()
+    E, Ne, Ke = d["W"].shape
+    xm = t16(d["X"], "bf16")
+    rt = torch.from_numpy(d["routing"]).to(dev)
+    wm = t16(d["W"].reshape(E * Ne, Ke), "bf16")
+    del d
+    _, wq, sw = sp.prepare_nvfp4_24(wm)
+    del wm
+    ym = torch.empty((rt.shape[0], rt.shape[1], Ne), dtype=torch.float32, device=dev)
+    T, topk = rt.shape
+    fl = 2.0 * T * topk * Ne * Ke
+    xy = T * Ke * 2 + T * topk * Ne * 4 + T * topk * 4
+    line = {"config": "4", "sweep": "moe_grouped", "experts": E, "expert_shape": [Ne, Ke], "tokens": T,
+            "topk": topk, "x": "bf16", "w": "nvfp4"}
+    for name, wop in (("dense", wq), ("sparse24", sw)):
+        us = timeit(lambda r: sp.gemm_grouped(xm, rt, wop, E, Ne, Ke, out=ym), 1, reps=5)
+        line[name] = record(us, fl, op_bytes(wop) + xy, "f16.sp" if name == "sparse24" else "f16")
+    line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse24"]["us"], 3)
+    emit(line)
+    del xm, rt, wq, sw, ym
+    # config 5a / 5b: M sweep at N = K = 5120, FP16 and NVFP4 (W4A16; W4A4 as an extra row)
+    W16 = synth.draw(synth.rng(0), (5120, 5120), "f16")
+    Wb = synth.draw(synth.rng(0), (5120, 5120), "bf16")
+    for Mv in (1, 16, 128, 1024, 4096, 16384):
+        X16 = synth.draw(synth.rng(Mv), (Mv, 5120), "f16")
+        case("5a", "msweep_fp16", Mv, 5120, 5120, "f16", "f16", X16, W16)
+        del X16
+        Xb = synth.draw(synth.rng(Mv), (Mv, 5120), "bf16")
+        case("5b", "msweep_nvfp4_w4a16", Mv, 5120, 5120, "bf16", "nvfp4", Xb, Wb)
+        case("5b", "msweep_nvfp4_w4a4", Mv, 5120, 5120, "nvfp4", "nvfp4", Xb, Wb)
+        if Mv >= 128:
+            case48("5b", "msweep_w4a4_pairwise48", Mv, 5120, 5120, Xb, Wb)
+        del Xb
+        torch.cuda.empty_cache()
     agree = sum(c["rule"] == c["faster"] for c in selections)
-    print(json.dumps({"sweep": "dense_sparse_selection", "shapes": len(selections), "rule_picks_faster": agree,
-                      "worst_loss": max(c["loss"] for c in selections), "cases": selections}), flush=True)
-    # conv eligibility check + compression (fp16 [256, 256, 3, 3], 5% failing groups), one
-    # tensor and a batch of 512 such tensors as one [512*256, 256, 3, 3] launch
+    emit({"config": "selection", "sweep": "dense_sparse_selection", "shapes": len(selections),
+          "rule_picks_faster": agree, "worst_loss": max(c["loss"] for c in selections), "cases": selections})
+    # config 5c: conv eligibility check + compression (fp16 [256, 256, 3, 3], 5% failing groups),
+    # one tensor and a batch of 512 such tensors as one [512*256, 256, 3, 3] launch
     c = synth.conv_fail5()
     for batch in (1, 512):
         wc = t16(np.ascontiguousarray(np.broadcast_to(c["W"], (batch,) + c["W"].shape)).reshape(
             (batch * 256, 256, 3, 3)), "f16")
+        nb = wc.numel() * 2
+        n = _copies(nb)
+        wcs = [wc] + [wc.clone() for _ in range(n - 1)]
         pass_ = torch.empty((batch * 256, 64, 3, 3), dtype=torch.uint8, device=dev)
         nf = torch.empty(1, dtype=torch.int32, device=dev)
         vals = torch.empty((batch * 256, 128, 3, 3), dtype=torch.float16, device=dev)
         meta = torch.empty(batch * 256 * 64 * 9 // 2, dtype=torch.uint8, device=dev)
-        us_c = timeit(lambda r: sp.check_24(wc, sp.OP_CONV, pass_out=pass_, n_fail_out=nf))
-        us_p = timeit(lambda r: sp.prune_compress_24(wc, sp.OP_CONV, values_out=vals, meta_out=meta))
-        nb = wc.numel() * 2
-        print(json.dumps({"sweep": "conv_check_compress", "tensors": batch, "shape": [batch * 256, 256, 3, 3],
-                          "check": {"us": round(us_c, 3), "GB/s": round((nb + pass_.numel()) / us_c / 1e3, 1)},
-                          "compress": {"us": round(us_p, 3), "GB/s": round((nb + vals.numel() * 2 + meta.numel()) / us_p / 1e3, 1)},
-                          "n_fail": int(nf.item())}), flush=True)
+        us_c = timeit(lambda r: sp.check_24(wcs[r % n], sp.OP_CONV, pass_out=pass_, n_fail_out=nf), n)
+        us_p = timeit(lambda r: sp.prune_compress_24(wcs[r % n], sp.OP_CONV, values_out=vals, meta_out=meta), n)
+        bc, bp = nb + pass_.numel(), nb + vals.numel() * 2 + meta.numel()
+        emit({"config": "5c", "sweep": "conv_check_compress", "tensors": batch, "shape": [batch * 256, 256, 3, 3],
+              "input_sets": n,
+              "check": {"us": round(us_c, 3), "GB/s": round(bc / us_c / 1e3, 1),
+                        "frac_hbm": round(bc / us_c / 1e3 / peak_hbm, 3)},
+              "compress": {"us": round(us_p, 3), "GB/s": round(bp / us_p / 1e3, 1),
+                           "frac_hbm": round(bp / us_p / 1e3 / peak_hbm, 3)},
+              "n_fail": int(nf.item())})
+        del wc, wcs, pass_, vals, meta
+    torch.cuda.empty_cache()
+    if full:
+        sweep_next_rows(emit, sp, synth, dev, t16, timeit, op_bytes, peak_hbm, tensor_peak)
+    emit({"config": "peaks", "hbm_gbs": peak_hbm, "tensor_tflops": tensor_peak, "source": peak_src})
+
+
+def sweep_next_rows(emit, sp, synth, dev, t16, timeit, op_bytes, peak_hbm, tensor_peak) -> None:
+    """Rows beyond the five configs: the fused expert block, a large single-tensor quantisation
+    and pairwise 4:8 check / prune on the same tensor."""
+    import torch
 
     # routed expert block: 512 experts (gate/up [1024, 2048] packed, down [2048, 512]), 4096 bf16
     # tokens top-10, NVFP4 experts dense or 2:4; FLOPs 6 T topk H F; bytes: weights once, x, y,
@@ -646,16 +736,16 @@ def run_sweep(args) -> None:
     wsb = torch.empty(sp.moe_block_workspace_bytes(Tb, kb, E, H, F), dtype=torch.uint8, device=dev)
     flb = 6.0 * Tb * kb * H * F
     xyh = Tb * H * 2 + Tb * H * 4 + 2 * Tb * kb * F * 2 + 2 * Tb * kb * H * 4
-    line = {"sweep": "moe_block", "experts": E, "hidden": H, "inter": F, "tokens": Tb, "topk": kb, "x": "bf16",
-            "w": "nvfp4", "flop": flb}
+    line = {"config": "next", "sweep": "moe_block", "experts": E, "hidden": H, "inter": F, "tokens": Tb,
+            "topk": kb, "x": "bf16", "w": "nvfp4", "flop": flb}
     for name, (gop, dop) in (("dense", (gu_d, dn_d)), ("sparse24", (gu_s, dn_s))):
-        us = timeit(lambda r: sp.moe_block(xb, rtb, rwb, gop, dop, E, H, F, out=yb, workspace=wsb), reps=3)
+        us = timeit(lambda r: sp.moe_block(xb, rtb, rwb, gop, dop, E, H, F, out=yb, workspace=wsb), 1, reps=3)
         byt = op_bytes(gop) + op_bytes(dop) + xyh
         line[name] = {"us": round(us, 1), "TFLOP/s": round(flb / us / 1e6, 1), "GB/s": round(byt / us / 1e3, 1),
                       "bytes": byt, "frac_hbm": round(byt / us / 1e3 / peak_hbm, 3),
                       "frac_tensor": round(flb / us / 1e6 / tensor_peak["f16"], 3)}
     line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse24"]["us"], 3)
-    print(json.dumps(line), flush=True)
+    emit(line)
     del gu_d, dn_d, gu_s, dn_s, xb, yb, wsb
 
     # large single-tensor quantisation: a [151936, 4096] bf16 output head (~1.16 GiB -> 0.33 GiB
@@ -665,66 +755,73 @@ def run_sweep(args) -> None:
     R, L = Wh.shape
     qh = sp.quantize_nvfp4(Wh)
     nb_in, nb_out = Wh.numel() * 2, R * L // 2 + R * L // 16 + 4
-    us_full = timeit(lambda r: sp.quantize_nvfp4(Wh, out=qh), reps=5)
+    us_full = timeit(lambda r: sp.quantize_nvfp4(Wh, out=qh), 1, reps=5)
     ts_h = qh.tensor_scale.clone()
-    us_one = timeit(lambda r: sp.quantize_nvfp4(Wh, tensor_scale=ts_h, out=qh), reps=5)
+    us_one = timeit(lambda r: sp.quantize_nvfp4(Wh, tensor_scale=ts_h, out=qh), 1, reps=5)
     gs_out = torch.empty(1, dtype=torch.float32, device=dev)
-    us_gs = timeit(lambda r: sp.nvfp4_group_tensor_scale([Wh], out=gs_out), reps=5)
+    us_gs = timeit(lambda r: sp.nvfp4_group_tensor_scale([Wh], out=gs_out), 1, reps=5)
     alg = nb_in + nb_out
-    print(json.dumps({"sweep": "quantize_large", "shape": [R, L], "dtype": "bf16",
-                      "in_bytes": nb_in, "out_bytes": nb_out,
-                      "derived_scale": {"us": round(us_full, 1), "GB/s": round(alg / us_full / 1e3, 1),
-                                        "frac_hbm": round(alg / us_full / 1e3 / peak_hbm, 3),
-                                        "traffic_GB/s": round((2 * nb_in + nb_out) / us_full / 1e3, 1),
-                                        "note": "two reads of the tensor (amax, then encode)"},
-                      "supplied_scale": {"us": round(us_one, 1), "GB/s": round(alg / us_one / 1e3, 1),
-                                         "frac_hbm": round(alg / us_one / 1e3 / peak_hbm, 3)},
-                      "group_scale_only": {"us": round(us_gs, 1), "GB/s": round(nb_in / us_gs / 1e3, 1),
-                                           "frac_hbm": round(nb_in / us_gs / 1e3 / peak_hbm, 3)}}), flush=True)
+    emit({"config": "next", "sweep": "quantize_large", "shape": [R, L], "dtype": "bf16",
+          "in_bytes": nb_in, "out_bytes": nb_out,
+          "derived_scale": {"us": round(us_full, 1), "GB/s": round(alg / us_full / 1e3, 1),
+                            "frac_hbm": round(alg / us_full / 1e3 / peak_hbm, 3),
+                            "traffic_GB/s": round((2 * nb_in + nb_out) / us_full / 1e3, 1),
+                            "note": "two reads of the tensor (amax, then encode)"},
+          "supplied_scale": {"us": round(us_one, 1), "GB/s": round(alg / us_one / 1e3, 1),
+                             "frac_hbm": round(alg / us_one / 1e3 / peak_hbm, 3)},
+          "group_scale_only": {"us": round(us_gs, 1), "GB/s": round(nb_in / us_gs / 1e3, 1),
+                               "frac_hbm": round(nb_in / us_gs / 1e3 / peak_hbm, 3)}})
     # pairwise 4:8 on the same tensor (check; prune + compress), 2:4 prune + compress beside it
     pass48 = torch.empty((R, L // 8), dtype=torch.uint8, device=dev)
     nf48 = torch.empty(1, dtype=torch.int32, device=dev)
     vals = torch.empty((R, L // 2), dtype=torch.bfloat16, device=dev)
     meta48 = torch.empty(R * L // 16, dtype=torch.uint8, device=dev)
     meta24 = torch.empty(R * L // 8, dtype=torch.uint8, device=dev)
-    us_c48 = timeit(lambda r: sp.check_48(Wh, pass_out=pass48, n_fail_out=nf48), reps=5)
-    us_p48 = timeit(lambda r: sp.prune_compress_48(Wh, values_out=vals, meta_out=meta48), reps=5)
-    us_p24 = timeit(lambda r: sp.prune_compress_24(Wh, values_out=vals, meta_out=meta24), reps=5)
+    us_c48 = timeit(lambda r: sp.check_48(Wh, pass_out=pass48, n_fail_out=nf48), 1, reps=5)
+    us_p48 = timeit(lambda r: sp.prune_compress_48(Wh, values_out=vals, meta_out=meta48), 1, reps=5)
+    us_p24 = timeit(lambda r: sp.prune_compress_24(Wh, values_out=vals, meta_out=meta24), 1, reps=5)
     b_c48 = nb_in + pass48.numel()
     b_p48, b_p24 = nb_in + nb_in // 2 + meta48.numel(), nb_in + nb_in // 2 + meta24.numel()
-    print(json.dumps({"sweep": "pairwise48", "shape": [R, L], "dtype": "bf16",
-                      "check_48": {"us": round(us_c48, 1), "GB/s": round(b_c48 / us_c48 / 1e3, 1),
-                                   "frac_hbm": round(b_c48 / us_c48 / 1e3 / peak_hbm, 3)},
-                      "prune_compress_48": {"us": round(us_p48, 1), "GB/s": round(b_p48 / us_p48 / 1e3, 1),
-                                            "frac_hbm": round(b_p48 / us_p48 / 1e3 / peak_hbm, 3)},
-                      "prune_compress_24": {"us": round(us_p24, 1), "GB/s": round(b_p24 / us_p24 / 1e3, 1),
-                                            "frac_hbm": round(b_p24 / us_p24 / 1e3 / peak_hbm, 3)}}), flush=True)
+    emit({"config": "next", "sweep": "pairwise48", "shape": [R, L], "dtype": "bf16",
+          "check_48": {"us": round(us_c48, 1), "GB/s": round(b_c48 / us_c48 / 1e3, 1),
+                       "frac_hbm": round(b_c48 / us_c48 / 1e3 / peak_hbm, 3)},
+          "prune_compress_48": {"us": round(us_p48, 1), "GB/s": round(b_p48 / us_p48 / 1e3, 1),
+                                "frac_hbm": round(b_p48 / us_p48 / 1e3 / peak_hbm, 3)},
+          "prune_compress_24": {"us": round(us_p24, 1), "GB/s": round(b_p24 / us_p24 / 1e3, 1),
+                                "frac_hbm": round(b_p24 / us_p24 / 1e3 / peak_hbm, 3)}})
     del Wh, qh, pass48, vals, meta48, meta24
+    torch.cuda.empty_cache()
 
-    # routed experts: 4096 tokens x top-10 of 512 experts [512, 2048], bf16 x, NVFP4 experts
-    # (dense, and 2:4 of the same experts); every expert is touched, so each call reads all of
-    # them once (one copy: 302 MB dense / 218 MB 2:4, well beyond L2)
-    d = synth.moe()
-    E, Ne, Ke = d["W"].shape
-    xm = t16(d["X"], "bf16")
-    rt = torch.from_numpy(d["routing"]).to(dev)
-    wm = t16(d["W"].reshape(E * Ne, Ke), "bf16")
-    del d
-    _, wq, sw = sp.prepare_nvfp4_24(wm)
-    del wm
-    ym = torch.empty((rt.shape[0], rt.shape[1], Ne), dtype=torch.float32, device=dev)
-    T, topk = rt.shape
-    fl = 2.0 * T * topk * Ne * Ke
-    xy = T * Ke * 2 + T * topk * Ne * 4 + T * topk * 4
-    line = {"sweep": "moe_grouped", "experts": E, "expert_shape": [Ne, Ke], "tokens": T, "topk": topk,
-            "x": "bf16", "w": "nvfp4"}
-    for name, wop in (("dense", wq), ("sparse24", sw)):
-        us = timeit(lambda r: sp.gemm_grouped(xm, rt, wop, E, Ne, Ke, out=ym), reps=5)
-        byt = op_bytes(wop) + xy
-        line[name] = {"us": round(us, 2), "TFLOP/s": round(fl / us / 1e6, 2), "GB/s": round(byt / us / 1e3, 1),
-                      "bytes": byt, "frac_hbm": round(byt / us / 1e3 / peak_hbm, 3)}
-    line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse24"]["us"], 3)
-    print(json.dumps(line), flush=True)
+
+def per_config(lines: list) -> dict:
+    """The sweep records grouped by config, for the default JSON line."""
+    out: dict = {}
+    for ln in lines:
+        c = ln.get("config")
+        if c in ("peaks", "selection"):
+            out[c] = {k: v for k, v in ln.items() if k not in ("config", "cases")}
+            continue
+        out.setdefault(c, []).append({k: v for k, v in ln.items() if k != "config"})
+    return out
+
+
+def compute_roofline(lines: list):
+    """The config-3 dense W4A4 GEMM (4096^3) against the dense FP4 tensor peak."""
+    for ln in lines:
+        if ln.get("sweep") == "prefill_w4a4":
+            d = ln["dense"]
+            _, tp, src = tensor_peaks()
+            return {"bound": "tensor", "kernel": "gemm_dense W4A4 4096^3 (tcgen05 kind::mxf4nvf4)",
+                    "achieved": d["TFLOP/s"], "peak": round(tp["nvfp4"], 1), "peak_kind": src["nvfp4"],
+                    "unit": "TFLOP/s", "frac": round(d["TFLOP/s"] / tp["nvfp4"], 3), "launch_us": d["us"],
+                    "traffic": None}
+    return None
+
+
+def run_sweep(args) -> None:
+    import torch
+    torch.cuda.set_device(0)
+    sweep(lambda ln: print(json.dumps(ln), flush=True), full=True)
 
 
 def run_ncu_target() -> None:
@@ -789,6 +886,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
     ap.add_argument("--ncu-target", action="store_true", help="run each kernel once, untimed")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-config GEMM table that follows the timed step")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
@@ -843,6 +942,17 @@ def main():
     line = run_ours(args, rank, world, dist)
     if line is not None:
         line["cpu_baseline"] = cpu
+        if world == 1 and not args.no_per_config:
+            # every config at full size, each GEMM on prepared operands (CUDA-graph timing over
+            # operand sets larger than the L2), after the timed step so it cannot disturb it
+            lines = []
+            t0 = time.perf_counter()
+            with ClockSampler(torch.cuda.current_device()) as clk:
+                sweep(lines.append, full=False)
+            line["per_config"] = per_config(lines)
+            line["per_config_clocks"] = clk.summary()
+            line["per_config_seconds"] = round(time.perf_counter() - t0, 1)
+            line["roofline_compute"] = compute_roofline(lines)
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
