@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libsp24.so")
 # status codes (include/sp24.h)
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT, ERR_WORKSPACE = range(9)
-F16, BF16, F32, NVFP4, NVFP4_B32 = 0, 1, 2, 3, 4
+F16, BF16, F32, NVFP4, NVFP4_B32, NVFP4_MMA = 0, 1, 2, 3, 4, 5
 OP_MATMUL, OP_CONV = 0, 1
 ALGO_AUTO, ALGO_SKINNY, ALGO_TILED = 0, 1, 2
 
@@ -116,6 +116,8 @@ def lib() -> ctypes.CDLL:
             L.sp24_quantize_nvfp4_block32.argtypes = [P, I, I64, I64, P, P, P, P, P, I64, P]
             L.sp24_gemm_sparse48.argtypes = [ctypes.POINTER(_Operand), ctypes.POINTER(_SparseOperand), I64, I64,
                                              I64, P, P]
+            L.sp24_nvfp4_mma_size.argtypes = [I64, I64, P, P]
+            L.sp24_nvfp4_to_mma.argtypes = [P, P, I64, I64, P, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L
@@ -197,6 +199,17 @@ class NVFP4Tensor(NamedTuple):
     codes: torch.Tensor
     scales: torch.Tensor
     tensor_scale: torch.Tensor
+
+
+class NVFP4MMA(NamedTuple):
+    """An NVFP4 tensor as the W4A4 GEMM's tile images (see to_mma): codes and scales are flat
+    uint8 tensors (rows padded to a multiple of 128), tensor_scale fp32 [1]; rows, cols the
+    logical shape."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tensor_scale: torch.Tensor
+    rows: int
+    cols: int
 
 
 class Sparse24(NamedTuple):
@@ -462,23 +475,40 @@ def prepare_nvfp4_24(w: torch.Tensor, stream=None):
 
 # ---------------------------------------------------------------------------- a4 .. a6
 
+def to_mma(q: NVFP4Tensor, stream=None) -> NVFP4MMA:
+    """The same NVFP4 tensor rewritten as the tile images the W4A4 GEMM loads whole
+    (sp24_nvfp4_to_mma; cols % 256 == 0); the tensor scale is shared, not copied."""
+    rows, cols = q.codes.shape[0], 2 * q.codes.shape[1]
+    nc, ns = ctypes.c_int64(0), ctypes.c_int64(0)
+    _call("sp24_nvfp4_mma_size", rows, cols, ctypes.byref(nc), ctypes.byref(ns))
+    codes = torch.empty(nc.value, dtype=torch.uint8, device=q.codes.device)
+    scales = torch.empty(ns.value, dtype=torch.uint8, device=q.codes.device)
+    _call("sp24_nvfp4_to_mma", _ptr(q.codes), _ptr(q.scales), rows, cols, _ptr(codes), _ptr(scales),
+          _stream(stream))
+    return NVFP4MMA(codes, scales, q.tensor_scale, rows, cols)
+
+
 def _operand(t) -> _Operand:
     if isinstance(t, NVFP4Tensor):
         return _Operand(NVFP4, t.codes.data_ptr(), t.scales.data_ptr(), t.tensor_scale.data_ptr())
+    if isinstance(t, NVFP4MMA):
+        return _Operand(NVFP4_MMA, t.codes.data_ptr(), t.scales.data_ptr(), t.tensor_scale.data_ptr())
     _cuda(t, "operand")
     return _Operand(_dtype_code(t), t.data_ptr(), None, None)
 
 
 def _rows_k(t) -> tuple:
+    if isinstance(t, NVFP4MMA):
+        return t.rows, t.cols
     if isinstance(t, NVFP4Tensor):
         return t.codes.shape[0], 2 * t.codes.shape[1]
     return t.shape[0], t.shape[1]
 
 
 def gemm_workspace_bytes(x, w, sparse: bool, M: int, N: int, K: int, algo: int = ALGO_AUTO) -> int:
-    xf = NVFP4 if isinstance(x, NVFP4Tensor) else _DT[x.dtype]
-    wv = w.values if sparse else w
-    wf = NVFP4 if isinstance(wv, NVFP4Tensor) else _DT[wv.dtype]
+    fmt = lambda t: NVFP4 if isinstance(t, NVFP4Tensor) else NVFP4_MMA if isinstance(t, NVFP4MMA) else _DT[t.dtype]
+    xf = fmt(x)
+    wf = fmt(w.values if sparse else w)
     n = ctypes.c_int64(0)
     _call("sp24_gemm_workspace_size", xf, wf, int(sparse), M, N, K, algo, ctypes.byref(n))
     return n.value
@@ -490,7 +520,7 @@ def gemm_dense(x, w, out=None, algo: int = ALGO_AUTO, workspace=None, stream=Non
     N, Kw = _rows_k(w)
     if K != Kw:
         raise ValueError(f"K mismatch: {K} vs {Kw}")
-    dev = (x.codes if isinstance(x, NVFP4Tensor) else x).device
+    dev = (x.codes if isinstance(x, (NVFP4Tensor, NVFP4MMA)) else x).device
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=dev)
     ws_bytes = gemm_workspace_bytes(x, w, False, M, N, K, algo)

@@ -80,11 +80,20 @@ bool native_nvfp4(int x_fmt, int wf, const SkinnyParams& p) {
          aligned(p.x_scales, 16) && aligned(p.w_scales, 16);
 }
 
+// Workspace of the W4A4 pair kernel: the tile images (codes and scales) of each operand given
+// in row order (x_mma / w_mma: that operand already is an image).
+int64_t w4a4_image_bytes(int64_t rows, int64_t K) {
+  return round256(nvfp4_mma_codes_bytes(rows, K)) + round256(nvfp4_mma_scales_bytes(rows, K));
+}
+int64_t w4a4_workspace(bool x_mma, bool w_mma, int64_t M, int64_t N, int64_t K) {
+  return (x_mma ? 0 : w4a4_image_bytes(M, K)) + (w_mma ? 0 : w4a4_image_bytes(N, K));
+}
+
 // Workspace of the tiled path: 16-bit copies of the operands that are not 16-bit already
 // (NVFP4 2:4 values decoded to 16 bits for the native sparse kernel; otherwise the weight
-// expanded to a dense 16-bit matrix).
+// expanded to a dense 16-bit matrix); for W4A4, the relaid block scales.
 int64_t tiled_workspace(int x_fmt, int wf, int64_t M, int64_t N, int64_t K) {
-  if (x_fmt == X_Q4 && wf == W_DQ4 && K % 256 == 0) return 0;  // native NVFP4 kernel
+  if (x_fmt == X_Q4 && wf == W_DQ4 && K % 256 == 0) return w4a4_workspace(false, false, M, N, K);
   int64_t b = 0;
   if (native_sparse(wf, K)) {
     if (wf == W_SQ4) b += round256(N * K);  // N x K/2 values of 2 bytes
@@ -95,12 +104,41 @@ int64_t tiled_workspace(int x_fmt, int wf, int64_t M, int64_t N, int64_t K) {
   return b;
 }
 
+// W4A4 on the CTA-pair kernel: an operand given in row order (x_mma / w_mma false) is first
+// rewritten as its tile images in the workspace.
+int run_w4a4_pair(const uint8_t* xc, const uint8_t* xs, bool x_mma, const float* x_ts, const uint8_t* wc,
+                  const uint8_t* wsc, bool w_mma, const float* w_ts, int64_t M, int64_t N, int64_t K, float* y,
+                  void* ws, int64_t ws_bytes, cudaStream_t s) {
+  const int64_t need = w4a4_workspace(x_mma, w_mma, M, N, K);
+  if (need > 0 && (!ws || ws_bytes < need)) return SP24_ERR_WORKSPACE;
+  if (need > 0 && !aligned(ws, 256)) return SP24_ERR_ALIGN;
+  uint8_t* cur = reinterpret_cast<uint8_t*>(ws);
+  auto image = [&](const uint8_t** codes, const uint8_t** scales, int64_t rows) {
+    uint8_t* c = cur;
+    uint8_t* sc = cur + round256(nvfp4_mma_codes_bytes(rows, K));
+    cur += w4a4_image_bytes(rows, K);
+    int st = nvfp4_to_mma(*codes, *scales, rows, K, c, sc, s);
+    *codes = c;
+    *scales = sc;
+    return st;
+  };
+  if (!x_mma) {
+    int st = image(&xc, &xs, M);
+    if (st) return st;
+  }
+  if (!w_mma) {
+    int st = image(&wc, &wsc, N);
+    if (st) return st;
+  }
+  return tc_gemm_nvfp4_pair(xc, xs, x_ts, wc, wsc, w_ts, M, N, K, y, s, 0);
+}
+
 // Tiled (tcgen05) path: decode what is not plain 16-bit into the workspace, then one GEMM.
 int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes, cudaStream_t s) {
   // NVFP4 x with NVFP4 w: both stay 4-bit, the tensor core applies the block scales
   if (native_nvfp4(p.x_fmt, wf, p))
-    return tc_gemm_nvfp4(reinterpret_cast<const uint8_t*>(p.x), p.x_scales, p.x_ts, p.w, p.w_scales, p.w_ts,
-                         p.M, p.N, p.K, p.y, s);
+    return run_w4a4_pair(reinterpret_cast<const uint8_t*>(p.x), p.x_scales, false, p.x_ts, p.w, p.w_scales, false,
+                         p.w_ts, p.M, p.N, p.K, p.y, ws, ws_bytes, s);
   const int64_t need = tiled_workspace(p.x_fmt, wf, p.M, p.N, p.K);
   if (need > 0 && (!ws || ws_bytes < need)) return SP24_ERR_WORKSPACE;
   if (need > 0 && !aligned(ws, 256)) return SP24_ERR_ALIGN;
@@ -196,6 +234,13 @@ extern "C" int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, 
   if (!bytes) return SP24_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
   if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
+  if (x_format == SP24_NVFP4_MMA || w_format == SP24_NVFP4_MMA) {
+    const bool q4 = (x_format == SP24_NVFP4 || x_format == SP24_NVFP4_MMA) &&
+                    (w_format == SP24_NVFP4 || w_format == SP24_NVFP4_MMA);
+    if (!q4 || sparse) return SP24_ERR_DTYPE;
+    *bytes = w4a4_workspace(x_format == SP24_NVFP4_MMA, w_format == SP24_NVFP4_MMA, M, N, K);
+    return SP24_OK;
+  }
   if (!(is16(x_format) || x_format == SP24_NVFP4) || !(is16(w_format) || w_format == SP24_NVFP4))
     return SP24_ERR_DTYPE;
   const int wf = sparse ? (is16(w_format) ? W_S16 : W_SQ4) : (is16(w_format) ? W_D16 : W_DQ4);
@@ -211,6 +256,27 @@ extern "C" int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int
   if (!x || !w) return SP24_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return SP24_ERR_SHAPE;
   if (algo < SP24_ALGO_AUTO || algo > SP24_ALGO_TILED) return SP24_ERR_INVALID_ARG;
+  if (x->format == SP24_NVFP4_MMA || w->format == SP24_NVFP4_MMA) {
+    // W4A4 with scales in the tensor cores' tile order: only the CTA-pair kernel reads them
+    const bool xq = x->format == SP24_NVFP4 || x->format == SP24_NVFP4_MMA;
+    const bool wq = w->format == SP24_NVFP4 || w->format == SP24_NVFP4_MMA;
+    if (!xq || !wq) return SP24_ERR_DTYPE;
+    if (K % 256) return SP24_ERR_SHAPE;
+    if (algo == SP24_ALGO_SKINNY) return SP24_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return SP24_OK;
+    if (!y) return SP24_ERR_INVALID_ARG;
+    if (!aligned(y, 4)) return SP24_ERR_ALIGN;
+    if (K > 0) {
+      if (!x->data || !x->scales || !x->tensor_scale || !w->data || !w->scales || !w->tensor_scale)
+        return SP24_ERR_INVALID_ARG;
+      if (!aligned(x->data, 16) || !aligned(x->scales, 16) || !aligned(w->data, 16) || !aligned(w->scales, 16))
+        return SP24_ERR_ALIGN;
+    }
+    return run_w4a4_pair(static_cast<const uint8_t*>(x->data), x->scales, x->format == SP24_NVFP4_MMA,
+                         x->tensor_scale, static_cast<const uint8_t*>(w->data), w->scales,
+                         w->format == SP24_NVFP4_MMA, w->tensor_scale, M, N, K, y, workspace, workspace_bytes,
+                         as_stream(stream));
+  }
   SkinnyParams p;
   memset(&p, 0, sizeof(p));
   int st = prep_x(x, M, K, &p);
@@ -288,6 +354,23 @@ extern "C" int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_opera
   p.K = K;
   p.y = y;
   return dispatch(wf, t16, p, algo, workspace, workspace_bytes, as_stream(stream));
+}
+
+extern "C" int sp24_nvfp4_mma_size(int64_t rows, int64_t cols, int64_t* codes_bytes, int64_t* scales_bytes) {
+  if (rows < 0 || cols < 0 || cols % 256) return SP24_ERR_SHAPE;
+  if (codes_bytes) *codes_bytes = nvfp4_mma_codes_bytes(rows, cols);
+  if (scales_bytes) *scales_bytes = nvfp4_mma_scales_bytes(rows, cols);
+  return SP24_OK;
+}
+
+extern "C" int sp24_nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                 uint8_t* codes_out, uint8_t* scales_out, void* stream) {
+  if (rows < 0 || cols < 0 || cols % 256) return SP24_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return SP24_OK;
+  if (!codes || !scales || !codes_out || !scales_out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || !aligned(codes_out, 16) || !aligned(scales_out, 16))
+    return SP24_ERR_ALIGN;
+  return nvfp4_to_mma(codes, scales, rows, cols, codes_out, scales_out, as_stream(stream));
 }
 
 extern "C" int64_t sp24_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -154,6 +154,20 @@ int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, i
 int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* wc, const uint8_t* wsc,
                   const float* w_ts, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t s);
 
+// NVFP4 operand images for the W4A4 kernel (K % 256 == 0): codes [rows, K/2] -> 16 KB tiles of
+// 128 rows x 256 K in the 128-byte-swizzled shared-memory order; scales [rows, K/16] -> 512-byte
+// tiles of 128 rows x 4 scales in tcgen05.cp order.  Either output may be null (skipped).
+int64_t nvfp4_mma_codes_bytes(int64_t rows, int64_t K);
+int64_t nvfp4_mma_scales_bytes(int64_t rows, int64_t K);
+int nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
+                 uint8_t* scales_out, cudaStream_t s);
+
+// W4A4 GEMM on the persistent CTA-pair kernel (both operands as images above).  wait_ns bounds
+// every device-side wait (0: the library's default).
+int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float* x_ts, const uint8_t* wc_mma,
+                       const uint8_t* ws_mma, const float* w_ts, int64_t M, int64_t N, int64_t K, float* y,
+                       cudaStream_t s, uint64_t wait_ns);
+
 // Expands an NVFP4 (W_DQ4) or 2:4-compressed (W_S16 / W_SQ4) operand into exact 16-bit values.
 int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta,
                int64_t rows, int64_t K, uint16_t* out, cudaStream_t s);

@@ -45,7 +45,7 @@ enum {
 
 /* ----------------------------------------------------------------------- enums */
 /* element types */
-enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3, SP24_NVFP4_B32 = 4 };
+enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3, SP24_NVFP4_B32 = 4, SP24_NVFP4_MMA = 5 };
 
 /* The operation a weight belongs to decides which four entries form a group ([P2] "The
  * operation determines which four entries belong together"). */
@@ -67,6 +67,9 @@ enum { SP24_ALGO_AUTO = 0, SP24_ALGO_SKINNY = 1, SP24_ALGO_TILED = 2 };
  *       scales -> [rows, K/16] E4M3 block scales, tensor_scale -> one fp32 (device).
  *   format SP24_NVFP4_B32: the same encoding with one E4M3 scale per 32 values, scales ->
  *       [rows, K/32] (the activation form read by sp24_gemm_sparse48 only).
+ *   format SP24_NVFP4_MMA: SP24_NVFP4 rewritten as tile images (sp24_nvfp4_to_mma): data ->
+ *       code tiles, scales -> scale tiles; accepted by sp24_gemm_dense when both operands are
+ *       NVFP4 (either layout), K % 256 == 0. 
  * Decoded value = E2M1(code) * E4M3(scale) * tensor_scale. */
 typedef struct {
   int32_t format;
@@ -192,6 +195,23 @@ int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
                         float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
                         void* stream);
 
+/* An NVFP4 tensor [rows, cols] (cols % 256 == 0) rewritten as the tile images the W4A4 GEMM
+ * loads whole (format SP24_NVFP4_MMA): each tile lands in shared memory with one copy.  Not on
+ * the source pages: a layout of this library's W4A4 kernel; the values are unchanged.
+ *   codes_out:  per 128-row block rb and 256-column chunk kc a 16 KB tile at byte
+ *               16384 * (rb * cols/256 + kc); row r of the block at byte 128 * r, its 16-byte
+ *               piece c (columns 32c .. 32c+31 of the chunk) at 16 * (c ^ (r % 8)).
+ *   scales_out: per 128-row block rb and 64-column chunk kc a 512-byte tile at byte
+ *               512 * (rb * cols/64 + kc); row r's four scales of the chunk at byte
+ *               16 * (r % 32) + 4 * (r / 32).
+ *   Rows are padded to a multiple of 128 with zero codes and zero scales; sizes from
+ *   sp24_nvfp4_mma_size.  codes: device [rows, cols/2] (16-byte aligned); scales: device
+ *   [rows, cols/16] (4-byte aligned); outputs device, 16-byte aligned.  Two launches;
+ *   SP24_ERR_SHAPE when cols % 256 != 0. */
+int sp24_nvfp4_mma_size(int64_t rows, int64_t cols, int64_t* codes_bytes, int64_t* scales_bytes);
+int sp24_nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                      uint8_t* codes_out, uint8_t* scales_out, void* stream);
+
 /* The same quantisation for callers that cannot allocate device memory: runtimes that only hand
  * out a fixed arena of operand buffers, plugins whose host framework owns the device allocator,
  * and host loops that must not call cudaMalloc (it can synchronise the device).  No counterpart
@@ -284,7 +304,9 @@ int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* 
  * Y[m, n] = sum_k x[m, k] * w[n, k] with fp32 accumulation, Y fp32 [M, N] row-major (device).
  * x: M rows (F16, BF16 or NVFP4); w: N rows (F16, BF16 or NVFP4).  16-bit x and 16-bit w
  * must have the same type.  Where NVFP4 meets NVFP4 (W4A4) both stay 4-bit and the tensor core
- * applies the block scales.  NVFP4 w with 16-bit x is decoded inside the kernel to x's type at
+ * applies the block scales (K % 256 == 0 and M > 64, or either operand SP24_NVFP4_MMA: a
+ * persistent kernel on pairs of SMs; the workspace then holds the tile images of each operand
+ * given as SP24_NVFP4).  NVFP4 w with 16-bit x is decoded inside the kernel to x's type at
  * M <= 64; at larger M it is first expanded to x's type in the workspace (exact values).
  * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
  * aligned, y 4-byte aligned (SP24_ERR_ALIGN otherwise; the same holds for every GEMM entry

@@ -168,3 +168,32 @@ def test_element_alignment_checked_on_the_host():
     assert _raw("sp24_decompress_24", 16, 16, sp.BF16, sp.OP_MATMUL, shp, 2, 19, None) == sp.ERR_ALIGN
     assert _raw("sp24_dequantize_nvfp4", 16, 16, 16, 4, 32, sp.F32, 18, None) == sp.ERR_ALIGN
 
+
+
+def test_w4a4_tile_layout_host_validation():
+    """The scale-tile rearrangement and the tile-order operand format, checked on the host."""
+    L = sp.lib()
+    n, m = ctypes.c_int64(-1), ctypes.c_int64(-1)
+    assert L.sp24_nvfp4_mma_size(200, 512, ctypes.byref(n), ctypes.byref(m)) == sp.OK
+    assert (n.value, m.value) == (256 * 256, 256 * 32)
+    assert L.sp24_nvfp4_mma_size(1, 256, ctypes.byref(n), None) == sp.OK and n.value == 128 * 128
+    assert L.sp24_nvfp4_mma_size(8, 384, ctypes.byref(n), None) == sp.ERR_SHAPE
+    assert L.sp24_nvfp4_to_mma(None, None, 8, 384, None, None, None) == sp.ERR_SHAPE
+    assert L.sp24_nvfp4_to_mma(None, None, 0, 256, None, None, None) == sp.OK
+    assert L.sp24_nvfp4_to_mma(None, None, 4, 256, None, None, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_nvfp4_to_mma(8, 4, 4, 256, 16, 16, None) == sp.ERR_ALIGN
+    mma = sp._Operand(sp.NVFP4_MMA, 16, 16, 16)
+    f16 = sp._Operand(sp.F16, 16, None, None)
+    y = ctypes.c_void_p(256)
+    # a tile-order operand only meets NVFP4; K % 256; never the skinny kernels
+    assert L.sp24_gemm_dense(ctypes.byref(f16), ctypes.byref(mma), 8, 8, 256, y, None, 0, 0, None) == sp.ERR_DTYPE
+    assert L.sp24_gemm_dense(ctypes.byref(mma), ctypes.byref(mma), 8, 8, 128, y, None, 0, 0, None) == sp.ERR_SHAPE
+    assert L.sp24_gemm_dense(ctypes.byref(mma), ctypes.byref(mma), 8, 8, 256, y, None, 0,
+                             sp.ALGO_SKINNY, None) == sp.ERR_UNSUPPORTED
+    q = sp._Operand(sp.NVFP4, 16, 16, 16)
+    assert L.sp24_gemm_dense(ctypes.byref(q), ctypes.byref(mma), 8, 8, 256, y, None, 0, 0, None) == sp.ERR_WORKSPACE
+    assert L.sp24_gemm_workspace_size(sp.NVFP4_MMA, sp.NVFP4_MMA, 0, 300, 520, 768, 0, ctypes.byref(n)) == sp.OK
+    assert n.value == 0
+    assert L.sp24_gemm_workspace_size(sp.NVFP4, sp.NVFP4_MMA, 0, 300, 520, 768, 0, ctypes.byref(n)) == sp.OK
+    assert n.value == 384 * 384 + 384 * 48
+    assert L.sp24_gemm_workspace_size(sp.NVFP4_MMA, sp.BF16, 0, 300, 520, 768, 0, ctypes.byref(n)) == sp.ERR_DTYPE
