@@ -112,22 +112,27 @@ int run_w4a4_pair(const uint8_t* xc, const uint8_t* xs, bool x_mma, const float*
   const int64_t need = w4a4_workspace(x_mma, w_mma, M, N, K);
   if (need > 0 && (!ws || ws_bytes < need)) return SP24_ERR_WORKSPACE;
   if (need > 0 && !aligned(ws, 256)) return SP24_ERR_ALIGN;
+  // one launch rewrites whichever operands are in row order
   uint8_t* cur = reinterpret_cast<uint8_t*>(ws);
-  auto image = [&](const uint8_t** codes, const uint8_t** scales, int64_t rows) {
-    uint8_t* c = cur;
-    uint8_t* sc = cur + round256(nvfp4_mma_codes_bytes(rows, K));
-    cur += w4a4_image_bytes(rows, K);
-    int st = nvfp4_to_mma(*codes, *scales, rows, K, c, sc, s);
-    *codes = c;
-    *scales = sc;
-    return st;
+  const uint8_t *c[2] = {nullptr, nullptr}, *sc[2] = {nullptr, nullptr};
+  uint8_t *co[2] = {nullptr, nullptr}, *so[2] = {nullptr, nullptr};
+  int64_t rows[2] = {0, 0};
+  int n = 0;
+  auto add = [&](const uint8_t** codes, const uint8_t** scales, int64_t r) {
+    c[n] = *codes;
+    sc[n] = *scales;
+    rows[n] = r;
+    co[n] = cur;
+    so[n] = cur + round256(nvfp4_mma_codes_bytes(r, K));
+    cur += w4a4_image_bytes(r, K);
+    *codes = co[n];
+    *scales = so[n];
+    ++n;
   };
-  if (!x_mma) {
-    int st = image(&xc, &xs, M);
-    if (st) return st;
-  }
-  if (!w_mma) {
-    int st = image(&wc, &wsc, N);
+  if (!x_mma) add(&xc, &xs, M);
+  if (!w_mma) add(&wc, &wsc, N);
+  if (n > 0) {
+    int st = nvfp4_to_mma2(c[0], sc[0], rows[0], co[0], so[0], c[1], sc[1], rows[1], co[1], so[1], K, s);
     if (st) return st;
   }
   return tc_gemm_nvfp4_pair(xc, xs, x_ts, wc, wsc, w_ts, M, N, K, y, s, 0);

@@ -9,19 +9,26 @@
 //     N = BN tokens, and each CTA loads only half of the tokens' B tile (the pair's tensor cores
 //     share their B halves), so an SM brings in 128 weight rows + BN/2 token rows per K step for
 //     128 x BN outputs;
-//   * block scales arrive already in the tensor cores' 128-row x 4-scale tile order
-//     (sp24_nvfp4_scales_to_mma), so one TMA box per operand per stage lands them ready for
-//     tcgen05.cp, with no rewrite on chip;
+//   * operands arrive as tile images (sp24_nvfp4_to_mma): codes already in the 128-byte
+//     swizzled shared-memory order, one TMA box of eight 2 KB rows per 16 KB tile (boxes of
+//     128-byte rows cost the TMA unit one request per row and capped an SM near 48 GB/s), block
+//     scales already in the 128-row x 4-scale order that tcgen05.cp moves into TMEM;
+//   * scale copies off the MMA thread: a tcgen05 instruction costs its issuing thread tens of
+//     nanoseconds, and the twelve scale copies of a 256-K stage (4 SFA + 8 SFB tiles) issued by
+//     the MMA thread took longer than the stage's four MMAs (measured: 0.80 us per stage against
+//     0.42 us without copies); two warps issue them, six each, into two TMEM slots that
+//     alternate between stages (0.51 us per stage);
 //   * persistent: one CTA per SM, tiles assigned round-robin to the pairs; two TMEM
-//     accumulators, so a tile's epilogue (TMEM -> registers -> fp32 Y) overlaps the next tile's
-//     main loop.  For BN = 256 the two accumulators overlap in 64 columns (0-255 and 192-447,
-//     scale factors in 448-495): the epilogue drains the shared 64 columns first and releases
-//     the accumulator, then drains the rest while the next tile's MMAs run.
+//     accumulators, so a tile's epilogue (TMEM -> registers -> shared memory -> TMA store of
+//     32-token x 128-row fp32 boxes) overlaps the next tile's main loop.  For BN = 256 the two
+//     accumulators overlap in 96 columns (0-255 and 160-415, scale slots in 416-511): the
+//     epilogue reads the shared columns first and releases the accumulator, then drains the rest
+//     while the next tile's MMAs run.
 //
-// Warp roles (192 threads per CTA): warp 0 = TMA producer (one lane, both CTAs load their own
+// Warp roles (256 threads per CTA): warp 0 = TMA producer (one lane; both CTAs load their own
 // halves and count the bytes on the even CTA's barrier); warp 1 = TMEM allocation (both CTAs)
 // and, in the even CTA, the MMA issuer (one lane); warps 2-5 = epilogue (TMEM lane quarter =
-// warp % 4), each thread one weight row, storing 32 consecutive tokens' outputs per TMEM load.
+// warp % 4), each thread one weight row; warps 6-7 = scale copies (even CTA, one lane each).
 // Every wait is bounded: when one runs out the kernel records SP24_ERR_DEVICE_TIMEOUT and
 // unwinds.  No TMA load uses cluster multicast.
 #include <cudaTypedefs.h>
@@ -47,38 +54,47 @@ namespace sp24 {
 
 namespace {
 
-// One thread per 16-byte piece of the codes (reads coalesced along the row, writes whole
-// 128-byte rows of a tile).
-__global__ void __launch_bounds__(256) codes_to_mma_kernel(const uint4* __restrict__ in, int64_t rows,
-                                                           int64_t pieces_per_row, int64_t total,
-                                                           uint4* __restrict__ out) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t r = t / pieces_per_row, j = t - r * pieces_per_row;
-    const uint4 v = r < rows ? in[t] : make_uint4(0u, 0u, 0u, 0u);
-    const int64_t kc = j >> 3, c = j & 7;
-    const int rr = (int)(r & 127);
-    out[((r >> 7) * (pieces_per_row >> 3) + kc) * 1024 + rr * 8 + (c ^ (rr & 7))] = v;
+struct ImageJob {
+  const uint4* codes;        // [rows, K/2] bytes as 16-byte pieces
+  const uint32_t* scales;    // [rows, K/16] bytes as words
+  uint4* codes_out;
+  uint32_t* scales_out;
+  int rows, K, tiles;        // tiles = row blocks x K/256
+};
+
+// One CTA per code tile (128 rows x 256 K): its 16 KB of codes (8 threads per 128-byte row
+// segment, reads coalesced, each 128-byte row written whole) and the four scale tiles of the
+// same rows and K range.  Up to two operands per launch (job b may be empty).
+__global__ void __launch_bounds__(256) to_mma_kernel(ImageJob ja, ImageJob jb) {
+  int t = blockIdx.x;
+  const bool second = t >= ja.tiles;
+  const ImageJob& j = second ? jb : ja;
+  if (second) t -= ja.tiles;
+  const int kc256 = j.K / 256, rb = t / kc256, kc = t - rb * kc256;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < 1024; i += 256) {
+    const int rr = i >> 3, c = i & 7, r = rb * 128 + rr;
+    const uint4 v = r < j.rows ? j.codes[(int64_t)r * (j.K / 32) + kc * 8 + c] : zero;
+    j.codes_out[(int64_t)t * 1024 + rr * 8 + (c ^ (rr & 7))] = v;
+  }
+  for (int i = threadIdx.x; i < 512; i += 256) {
+    const int rr = i >> 2, w = i & 3, r = rb * 128 + rr;
+    const uint32_t v = r < j.rows ? j.scales[(int64_t)r * (j.K / 64) + kc * 4 + w] : 0u;
+    j.scales_out[((int64_t)rb * (j.K / 64) + kc * 4 + w) * 128 + 4 * (rr & 31) + (rr >> 5)] = v;
   }
 }
 
-// One CTA per (128-row block, 16 chunks of 64 K): the rows' 16 scale words come in coalesced
-// (64 bytes per row) through shared memory and leave as 16 whole 512-byte tiles.
-__global__ void __launch_bounds__(256) scales_to_mma_kernel(const uint32_t* __restrict__ in, int64_t rows,
-                                                            int64_t kc, uint32_t* __restrict__ out) {
-  __shared__ uint32_t tile[128][17];
-  const int64_t rb = blockIdx.x, c0 = (int64_t)blockIdx.y * 16;
-  const int nc = (int)(kc - c0 < 16 ? kc - c0 : 16);
-  for (int i = threadIdx.x; i < 128 * 16; i += 256) {
-    const int rr = i >> 4, c = i & 15;
-    const int64_t r = rb * 128 + rr;
-    tile[rr][c] = (c < nc && r < rows) ? in[r * kc + c0 + c] : 0u;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nc * 128; i += 256) {
-    const int c = i >> 7, w = i & 127;          // word w of tile c: row 32 (w % 4) + w / 4
-    out[(rb * kc + c0 + c) * 128 + w] = tile[32 * (w & 3) + (w >> 2)][c];
-  }
+ImageJob image_job(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
+                   uint8_t* scales_out) {
+  ImageJob j;
+  j.codes = reinterpret_cast<const uint4*>(codes);
+  j.scales = reinterpret_cast<const uint32_t*>(scales);
+  j.codes_out = reinterpret_cast<uint4*>(codes_out);
+  j.scales_out = reinterpret_cast<uint32_t*>(scales_out);
+  j.rows = (int)rows;
+  j.K = (int)K;
+  j.tiles = (int)((rows + 127) / 128 * (K / 256));
+  return j;
 }
 
 }  // namespace
@@ -86,28 +102,23 @@ __global__ void __launch_bounds__(256) scales_to_mma_kernel(const uint32_t* __re
 int64_t nvfp4_mma_codes_bytes(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * (K / 2); }
 int64_t nvfp4_mma_scales_bytes(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * (K / 16); }
 
+// Tile images of one or two NVFP4 operands (rows1 == 0: only the first), one launch.
+int nvfp4_to_mma2(const uint8_t* c0, const uint8_t* s0, int64_t rows0, uint8_t* co0, uint8_t* so0,
+                  const uint8_t* c1, const uint8_t* s1, int64_t rows1, uint8_t* co1, uint8_t* so1, int64_t K,
+                  cudaStream_t s) {
+  if (K % 256 || rows0 > INT32_MAX || rows1 > INT32_MAX || K > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  const ImageJob ja = image_job(c0, s0, rows0, K, co0, so0);
+  const ImageJob jb = image_job(c1, s1, rows1, K, co1, so1);
+  const int64_t blocks = (int64_t)ja.tiles + jb.tiles;
+  if (blocks == 0) return SP24_OK;
+  if (blocks > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  to_mma_kernel<<<(unsigned)blocks, 256, 0, s>>>(ja, jb);
+  return launch_status();
+}
+
 int nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
                  uint8_t* scales_out, cudaStream_t s) {
-  const int64_t rb = (rows + 127) / 128;
-  if (rb == 0 || K == 0) return SP24_OK;
-  if (codes_out) {
-    const int64_t ppr = K / 32, total = rb * 128 * ppr;
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > (int64_t)sm_count() * 16) blocks = (int64_t)sm_count() * 16;
-    codes_to_mma_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(codes), rows, ppr, total,
-                                                         reinterpret_cast<uint4*>(codes_out));
-    int st = launch_status();
-    if (st) return st;
-  }
-  if (scales_out) {
-    const int64_t kc = K / 64;
-    if (rb > INT32_MAX || (kc + 15) / 16 > 65535) return SP24_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)rb, (unsigned)((kc + 15) / 16));
-    scales_to_mma_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(scales), rows, kc,
-                                              reinterpret_cast<uint32_t*>(scales_out));
-    return launch_status();
-  }
-  return SP24_OK;
+  return nvfp4_to_mma2(codes, scales, rows, codes_out, scales_out, nullptr, nullptr, 0, nullptr, nullptr, K, s);
 }
 
 // ------------------------------------------------------------------ the pair GEMM

@@ -156,11 +156,15 @@ int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const
 
 // NVFP4 operand images for the W4A4 kernel (K % 256 == 0): codes [rows, K/2] -> 16 KB tiles of
 // 128 rows x 256 K in the 128-byte-swizzled shared-memory order; scales [rows, K/16] -> 512-byte
-// tiles of 128 rows x 4 scales in tcgen05.cp order.  Either output may be null (skipped).
+// tiles of 128 rows x 4 scales in tcgen05.cp order.
 int64_t nvfp4_mma_codes_bytes(int64_t rows, int64_t K);
 int64_t nvfp4_mma_scales_bytes(int64_t rows, int64_t K);
 int nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
                  uint8_t* scales_out, cudaStream_t s);
+// The same for two operands in one launch (rows1 == 0: the first only).
+int nvfp4_to_mma2(const uint8_t* c0, const uint8_t* s0, int64_t rows0, uint8_t* co0, uint8_t* so0,
+                  const uint8_t* c1, const uint8_t* s1, int64_t rows1, uint8_t* co1, uint8_t* so1, int64_t K,
+                  cudaStream_t s);
 
 // W4A4 GEMM on the persistent CTA-pair kernel (both operands as images above).  wait_ns bounds
 // every device-side wait (0: the library's default).
