@@ -118,6 +118,9 @@ def lib() -> ctypes.CDLL:
                                              I64, P, P]
             L.sp24_nvfp4_mma_size.argtypes = [I64, I64, P, P]
             L.sp24_nvfp4_to_mma.argtypes = [P, P, I64, I64, P, P, P]
+            L.sp24_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+            L.sp24_get_wait_limit.argtypes = [P]
+            L.sp24_selftest_wait_timeout.argtypes = [P, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L

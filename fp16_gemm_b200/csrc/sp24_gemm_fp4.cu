@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(256, 1)
   const int pair = (int)cluster_id_x(), pairs = (int)cluster_count_x();
   const int KB = p.K / 256;
   const int tiles = p.tiles_w * p.tiles_n;
+  const uint64_t wait_ns = p.wait_ns ? p.wait_ns : wait_limit();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(256, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
-          if (!mbar_wait_for(&empty_bar[s], ph ^ 1, p.wait_ns) || *(volatile int*)&aborted) {
+          if (!mbar_wait_for(&empty_bar[s], ph ^ 1, wait_ns) || *(volatile int*)&aborted) {
             aborted = 1;
             ok = false;
             break;
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(256, 1)
       // the even CTA's producer armed every stage it counted: wait (bounded) until those copies
       // (its own and the odd CTA's) have landed before the pair may exit
       if (leader)
-        for (int i = it - S > 0 ? it - S : 0; i < it; ++i) mbar_wait_for(&full_bar[i % S], (i / S) & 1, p.wait_ns);
+        for (int i = it - S > 0 ? it - S : 0; i < it; ++i) mbar_wait_for(&full_bar[i % S], (i / S) & 1, wait_ns);
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += pairs, ++j) {
         const uint32_t d = tmem + ((j & 1) ? C::ACC1 : 0u);
-        if (j >= 1 && !mbar_wait_cluster(&tempty_bar, (j - 1) & 1, p.wait_ns)) {
+        if (j >= 1 && !mbar_wait_cluster(&tempty_bar, (j - 1) & 1, wait_ns)) {
           aborted = 1;
           break;
         }
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(256, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
-          if (!mbar_wait_for(&full_bar[s], ph, p.wait_ns) || *(volatile int*)&aborted) {
+          if (!mbar_wait_for(&full_bar[s], ph, wait_ns) || *(volatile int*)&aborted) {
             aborted = 1;
             ok = false;
             break;
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(256, 1)
           const uint32_t sf0 = tmem + C::SF + (uint32_t)(it & 1) * C::SF_STAGE;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {  // the scale copies of MMAs 2h, 2h + 1 (warp 6 + h)
-            if (!mbar_wait_for(&sf_bar[h * S + s], ph, p.wait_ns)) {
+            if (!mbar_wait_for(&sf_bar[h * S + s], ph, wait_ns)) {
               aborted = 1;
               ok = false;
               break;
@@ -303,8 +304,8 @@ __global__ void __launch_bounds__(256, 1)
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
           const int prev = it - 2;  // the stage whose MMAs last read this slot
-          if (!mbar_wait_for(&full_bar[s], ph, p.wait_ns) ||
-              (prev >= 0 && !mbar_wait_for(&empty_bar[prev % S], (prev / S) & 1, p.wait_ns)) ||
+          if (!mbar_wait_for(&full_bar[s], ph, wait_ns) ||
+              (prev >= 0 && !mbar_wait_for(&empty_bar[prev % S], (prev / S) & 1, wait_ns)) ||
               *(volatile int*)&aborted) {
             aborted = 1;
             ok = false;
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(256, 1)
       const int n0 = (t / p.tiles_w) * BN;
       // the four epilogue warps agree on the outcome of the wait, so that none of them leaves
       // while the others wait for it at a named barrier
-      const bool got = mbar_wait_for(&tfull_bar, j & 1, p.wait_ns);
+      const bool got = mbar_wait_for(&tfull_bar, j & 1, wait_ns);
       if (lane == 0) epi_ok[q] = got;
       named_bar_sync(1, 128);
       const bool all = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
@@ -508,8 +509,7 @@ int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float
   const bool tma_y = N % 4 == 0 && aligned(y, 16);
   memset(&ty, 0, sizeof(ty));
   if (tma_y && (st = make_tmap_y(&ty, y, M, N))) return st;
-  PairParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts, (int)((N + 255) / 256), (int)((M + BN - 1) / BN),
-               wait_ns ? wait_ns : tc::kWaitLimitNs};
+  PairParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts, (int)((N + 255) / 256), (int)((M + BN - 1) / BN), wait_ns};
   if (BN == 256)
     return tma_y ? launch_pair<256, true>(ta, tb, tsa, tsb, ty, p, s) : launch_pair<256, false>(ta, tb, tsa, tsb, ty, p, s);
   return tma_y ? launch_pair<128, true>(ta, tb, tsa, tsb, ty, p, s) : launch_pair<128, false>(ta, tb, tsa, tsb, ty, p, s);

@@ -18,6 +18,10 @@ extern __device__ int g_dev_error;
 
 __device__ __forceinline__ void set_dev_error(int code) { atomicCAS(&g_dev_error, 0, code); }
 
+// Time limit of every bounded device-side wait of this library, in nanoseconds of %globaltimer
+// (one per device; default 2 s; sp24_set_wait_limit changes it for later launches).
+extern __device__ unsigned long long g_wait_limit_ns;
+
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // Host-side count of kernels this library has launched (diagnostics: sp24_kernel_launches).

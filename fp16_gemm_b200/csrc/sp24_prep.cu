@@ -18,6 +18,7 @@
 namespace sp24 {
 
 __device__ int g_dev_error = 0;
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 namespace {
 

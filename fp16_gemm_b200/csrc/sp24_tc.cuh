@@ -11,9 +11,10 @@
 namespace sp24 {
 namespace tc {
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer (the kernel then sets the
-// device error word and unwinds instead of hanging the GPU).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// A bounded wait gives up after the library's wait limit (g_wait_limit_ns, 2 s unless changed
+// with sp24_set_wait_limit) of %globaltimer; the kernel then sets the device error word and
+// unwinds instead of hanging the GPU.
+__device__ __forceinline__ uint64_t wait_limit() { return *(const volatile unsigned long long*)&g_wait_limit_ns; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -57,9 +58,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase of `parity` to complete; false when the time limit ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t lim = wait_limit();
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > lim) return false;
   }
   return true;
 }
@@ -96,9 +98,10 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // barrier instead of spinning, so it takes no issue slots from them.  Same time limit.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+  const uint64_t lim = wait_limit();
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > lim) return false;
   }
   return true;
 }

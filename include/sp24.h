@@ -212,6 +212,25 @@ int sp24_nvfp4_mma_size(int64_t rows, int64_t cols, int64_t* codes_bytes, int64_
 int sp24_nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
                       uint8_t* codes_out, uint8_t* scales_out, void* stream);
 
+/* ----------------------------------------------------------------------- bounded waits */
+/* Every device-side wait of this library (mbarrier phases, TMA and bulk-copy completions) gives
+ * up after a time limit: the kernel then records SP24_ERR_DEVICE_TIMEOUT in the device error
+ * word (read with sp24_last_device_error), waits (bounded) for its own copies in flight, frees
+ * the tensor memory it holds and returns; nothing traps.  Not on the source pages.
+ *   sp24_set_wait_limit   the limit in nanoseconds (> 0; default 2e9) for the current device,
+ *                         used by kernels launched afterwards.  Synchronous.
+ *   sp24_get_wait_limit   reads it back.
+ *   sp24_selftest_wait_timeout  runs that unwind on purpose: one CTA allocates TMEM, starts a
+ *                         1 KB bulk copy from `src` (device, 16-byte aligned), waits on an
+ *                         mbarrier phase that nothing completes until the limit runs out, sets
+ *                         SP24_ERR_DEVICE_TIMEOUT, lets the copy land, frees TMEM.  out (device
+ *                         int[2]): out[0] = 2 when the wait ran out (1 if it completed),
+ *                         out[1] = 1 + the copy's last byte once it landed (0 if not).
+ *                         Takes about one wait limit; for tests. */
+int sp24_set_wait_limit(unsigned long long ns);
+int sp24_get_wait_limit(unsigned long long* ns);
+int sp24_selftest_wait_timeout(const void* src, int* out, void* stream);
+
 /* The same quantisation for callers that cannot allocate device memory: runtimes that only hand
  * out a fixed arena of operand buffers, plugins whose host framework owns the device allocator,
  * and host loops that must not call cudaMalloc (it can synchronise the device).  No counterpart

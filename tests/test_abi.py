@@ -197,3 +197,11 @@ def test_w4a4_tile_layout_host_validation():
     assert L.sp24_gemm_workspace_size(sp.NVFP4, sp.NVFP4_MMA, 0, 300, 520, 768, 0, ctypes.byref(n)) == sp.OK
     assert n.value == 384 * 384 + 384 * 48
     assert L.sp24_gemm_workspace_size(sp.NVFP4_MMA, sp.BF16, 0, 300, 520, 768, 0, ctypes.byref(n)) == sp.ERR_DTYPE
+
+
+def test_wait_limit_and_selftest_host_validation():
+    L = sp.lib()
+    assert L.sp24_set_wait_limit(0) == sp.ERR_INVALID_ARG
+    assert L.sp24_get_wait_limit(None) == sp.ERR_INVALID_ARG
+    assert L.sp24_selftest_wait_timeout(None, None, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_selftest_wait_timeout(ctypes.c_void_p(8), ctypes.c_void_p(16), None) == sp.ERR_ALIGN
