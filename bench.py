@@ -454,10 +454,9 @@ def tensor_peaks():
     """Roofline denominators: (HBM GB/s, {pipe: TFLOP/s}, {pipe: where it came from}).
 
     HBM copy and dense bf16 GEMM are the measured figures of MEASURED_PEAKS.json (the
-    profiling recipe's fallback when absent).  The FP4 pipes come from this repository's own MMA
-    microbenchmark (`bench.py --peaks`, written to profiles/peaks.json) when it is present, else
-    from the measured bf16 figure x 4 (dense, the nominal 9 / 2.25 PF ratio) and x 8 (2:4,
-    dense-equivalent); 16-bit 2:4 counts dense-equivalent FLOPs at twice the measured bf16 rate."""
+    profiling recipe's fallback when absent); the other pipes take the measured bf16 figure
+    times the nominal ratio (FP4 dense x 4, i.e. 9 / 2.25 PF; 2:4 pipes count dense-equivalent
+    FLOPs at twice their dense rate)."""
     hbm, kind = peaks()
     bf16, bkind = 1590.0, "fallback"
     try:
@@ -468,16 +467,17 @@ def tensor_peaks():
     tp = {"f16": bf16, "f16.sp": 2 * bf16, "nvfp4": 4 * bf16, "nvfp4.sp": 8 * bf16}
     src = {"hbm": kind, "f16": bkind, "f16.sp": bkind + " x 2", "nvfp4": bkind + " x 4",
            "nvfp4.sp": bkind + " x 8"}
+    return hbm, tp, src
+
+
+def mma_microbench():
+    """{pipe: TFLOP/s} of back-to-back MMAs measured by `bench.py --peaks` (profiles/peaks.json),
+    or {} when that file is absent."""
     try:
         with open(os.path.join(ROOT, "profiles", "peaks.json")) as f:
-            mb = json.load(f)["mma_tflops"]
-        for pipe in ("nvfp4", "nvfp4.sp"):
-            if pipe in mb:
-                tp[pipe] = float(mb[pipe])
-                src[pipe] = "MMA microbenchmark (profiles/peaks.json)"
+            return json.load(f)["mma_tflops"]
     except Exception:
-        pass
-    return hbm, tp, src
+        return {}
 
 
 def _copies(set_bytes: float, lo: int = 2, hi: int = 64) -> int:
@@ -824,7 +824,9 @@ def compute_roofline(lines: list):
                               "cta_group::2 kind::mxf4nvf4)",
                     "achieved": d["TFLOP/s"], "peak": round(tp["nvfp4"], 1), "peak_kind": src["nvfp4"],
                     "unit": "TFLOP/s", "frac": round(d["TFLOP/s"] / tp["nvfp4"], 3), "launch_us": d["us"],
-                    "row_order_operands_us": ln["dense"]["us"], "traffic": None}
+                    "row_order_operands_us": ln["dense"]["us"],
+                    "mma_loop_tflops": {k: v for k, v in mma_microbench().items() if k.startswith("nvfp4")},
+                    "traffic": None}
     return None
 
 
@@ -832,6 +834,72 @@ def run_sweep(args) -> None:
     import torch
     torch.cuda.set_device(0)
     sweep(lambda ln: print(json.dumps(ln), flush=True), full=True)
+
+
+PEAK_KINDS = (  # kind, name, FLOPs per MMA (2 M N K, K logical), rounds of four MMAs
+    (0, "f16", 2 * 128 * 256 * 16, 8000),
+    (1, "f16.sp", 2 * 128 * 256 * 32, 8000),
+    (2, "nvfp4", 2 * 128 * 256 * 64, 8000),
+    (3, "nvfp4.sp", 2 * 128 * 256 * 128, 8000),
+    (4, "nvfp4.pair", 2 * 256 * 256 * 64, 8000),
+)
+
+
+def run_peaks(args) -> None:
+    """The tensor-pipe and HBM rates this device reaches with this library's own instructions
+    (back-to-back tcgen05 MMA loops on non-zero operands; a 16-byte load stream), written to
+    profiles/peaks.json.  Reported beside the recipe's denominators (the driver's measured bf16
+    GEMM x the nominal dtype ratio, and its measured copy bandwidth), not in their place."""
+    import ctypes
+
+    import torch
+
+    import fp16_gemm_b200 as sp
+
+    torch.cuda.set_device(0)
+    L = sp.lib()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    res, per = {}, {}
+    with ClockSampler(0) as clk:
+        for kind, name, flops, rounds in PEAK_KINDS:
+            n = L.sp24_peak_ctas(kind)
+            out = torch.zeros(n, dtype=torch.int64, device="cuda")
+            best = None
+            for _ in range(4):  # the first launch warms up; keep the fastest of the rest
+                rc = L.sp24_peak_mma(kind, rounds, ctypes.c_void_p(out.data_ptr()), st)
+                assert rc == sp.OK, sp.lib().sp24_status_string(rc)
+                torch.cuda.synchronize()
+                ns = out.cpu().numpy()
+                issuers = int((ns > 0).sum())
+                t = float(ns.max()) * 1e-9
+                tf = issuers * 4 * rounds * flops / t / 1e12
+                best = tf if best is None or tf > best else best
+            assert sp.last_device_error() == sp.OK
+            res[name] = round(best, 1)
+            per[name] = {"issuing_ctas": issuers, "mma_per_cta": 4 * rounds, "flop_per_mma": flops}
+        nbytes = 4 << 30
+        buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+        times = []
+        for i in range(6):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            assert L.sp24_peak_read(ctypes.c_void_p(buf.data_ptr()), nbytes, ctypes.c_void_p(acc.data_ptr()), st) == sp.OK
+            b.record()
+            torch.cuda.synchronize()
+            if i:
+                times.append(a.elapsed_time(b) * 1e-3)
+        hbm_read = nbytes / min(times) / 1e9
+        del buf
+    hbm, tp, src = tensor_peaks()
+    line = {"mma_tflops": res, "mma_detail": per, "hbm_read_gbs": round(hbm_read, 1),
+            "recipe_denominators": {"hbm_gbs": hbm, "tensor_tflops": tp, "source": src},
+            "clocks": clk.summary(), "device": torch.cuda.get_device_name(0),
+            "command": "python bench.py --peaks"}
+    os.makedirs(os.path.join(ROOT, "profiles"), exist_ok=True)
+    with open(os.path.join(ROOT, "profiles", "peaks.json"), "w") as f:
+        json.dump(line, f, indent=1)
+    print(json.dumps(line), flush=True)
 
 
 def run_ncu_target() -> None:
@@ -896,6 +964,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
     ap.add_argument("--ncu-target", action="store_true", help="run each kernel once, untimed")
+    ap.add_argument("--peaks", action="store_true", help="measure MMA and HBM peaks into profiles/peaks.json")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-config GEMM table that follows the timed step")
     args = ap.parse_args()
@@ -904,6 +973,9 @@ def main():
         return
     if args.ncu_target:
         run_ncu_target()
+        return
+    if args.peaks:
+        run_peaks(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

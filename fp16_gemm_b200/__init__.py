@@ -121,6 +121,9 @@ def lib() -> ctypes.CDLL:
             L.sp24_set_wait_limit.argtypes = [ctypes.c_ulonglong]
             L.sp24_get_wait_limit.argtypes = [P]
             L.sp24_selftest_wait_timeout.argtypes = [P, P, P]
+            L.sp24_peak_mma.argtypes = [I, I, P, P]
+            L.sp24_peak_ctas.argtypes = [I]
+            L.sp24_peak_read.argtypes = [P, I64, P, P]
             L.sp24_kernel_launches.restype = I64
             L.sp24_kernel_launches.argtypes = []
             _lib = L

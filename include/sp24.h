@@ -231,6 +231,23 @@ int sp24_set_wait_limit(unsigned long long ns);
 int sp24_get_wait_limit(unsigned long long* ns);
 int sp24_selftest_wait_timeout(const void* src, int* out, void* stream);
 
+/* ----------------------------------------------------------------------- roofline peaks */
+/* The denominators of the roofline fractions, measured with this library's own instructions
+ * (not on the source pages).
+ *   sp24_peak_mma   one CTA per SM (kind 4: per CTA pair) issues 4 * (rounds + 1) back-to-back
+ *                   tcgen05 MMAs of N = 256 from shared-memory operands holding non-zero data,
+ *                   accumulating in TMEM; out_ns[cta] = nanoseconds of the last 4 * rounds (0 for
+ *                   the odd CTA of a pair).  kind 0: kind::f16 bf16, M 128, K 16; 1: .sp
+ *                   kind::f16, K 32 logical; 2: kind::mxf4nvf4 block16, K 64; 3: .sp
+ *                   kind::mxf4nvf4, K 128 logical (pairwise 4:8 metadata); 4: kind::mxf4nvf4 on
+ *                   a CTA pair (cta_group::2), M 256, K 64.  FLOPs per MMA: 2 M N K (logical K).
+ *   sp24_peak_ctas  CTAs the launch uses (entries of out_ns) for a kind.
+ *   sp24_peak_read  a grid-stride stream of 16-byte loads over src (bytes % 16 == 0, 16-byte
+ *                   aligned), reduced into *out (device word) so nothing is optimised away. */
+int sp24_peak_mma(int kind, int rounds, unsigned long long* out_ns, void* stream);
+int sp24_peak_ctas(int kind);
+int sp24_peak_read(const void* src, int64_t bytes, unsigned int* out, void* stream);
+
 /* The same quantisation for callers that cannot allocate device memory: runtimes that only hand
  * out a fixed arena of operand buffers, plugins whose host framework owns the device allocator,
  * and host loops that must not call cudaMalloc (it can synchronise the device).  No counterpart

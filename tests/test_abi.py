@@ -205,3 +205,13 @@ def test_wait_limit_and_selftest_host_validation():
     assert L.sp24_get_wait_limit(None) == sp.ERR_INVALID_ARG
     assert L.sp24_selftest_wait_timeout(None, None, None) == sp.ERR_INVALID_ARG
     assert L.sp24_selftest_wait_timeout(ctypes.c_void_p(8), ctypes.c_void_p(16), None) == sp.ERR_ALIGN
+
+
+def test_peak_microbenchmark_host_validation():
+    L = sp.lib()
+    assert L.sp24_peak_ctas(5) == 0 and L.sp24_peak_ctas(-1) == 0
+    assert L.sp24_peak_mma(5, 10, ctypes.c_void_p(64), None) == sp.ERR_INVALID_ARG
+    assert L.sp24_peak_mma(0, 0, ctypes.c_void_p(64), None) == sp.ERR_INVALID_ARG
+    assert L.sp24_peak_mma(0, 10, ctypes.c_void_p(4), None) == sp.ERR_ALIGN
+    assert L.sp24_peak_read(None, 1024, None, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_peak_read(ctypes.c_void_p(16), 24, ctypes.c_void_p(16), None) == sp.ERR_INVALID_ARG
