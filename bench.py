@@ -902,11 +902,13 @@ def run_peaks(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-def run_ncu_target() -> None:
-    """Untimed: each kernel family once after a warm-up call, for an ncu capture (decode
-    pipeline on the decode workload: prepare_vec, encode_pair_kernel, decode_tile_kernel dense
-    and 2:4 per pass; W4A4 dense / 2:4 / pairwise 4:8 at 4096^3, FP16 dense / 2:4 at M = 4096; then the
-    routed-expert workload once, NVFP4 experts dense and 2:4)."""
+def run_ncu_target(which: str) -> None:
+    """Untimed: kernels run once each after a warm-up call, for an ncu capture of one family.
+      decode  the decode step on its workload (prepare_vec, encode_pair_kernel, decode_tile_kernel
+              dense and 2:4), twice;
+      w4a4    the W4A4 GEMM at 4096^3 on tile images (gemm_nvfp4_pair_kernel), three times;
+      all     both, then the 2:4 and pairwise-4:8 W4A4 GEMMs, the FP16 M = 4096 GEMMs and the
+              routed-expert workload once (several GB on the device)."""
     import torch
 
     import fp16_gemm_b200 as sp
@@ -914,39 +916,45 @@ def run_ncu_target() -> None:
 
     torch.cuda.set_device(0)
     bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
-    d = synth.decode_nvfp4()
-    x, w = bf(d["X"]), bf(d["W"])
-    for _ in range(2):
-        _, wq, sw = sp.prepare_nvfp4_24(w)
-        sp.gemm_dense(x, wq)
-        sp.gemm_sparse24(x, sw, K)
-    d = synth.prefill_w4a4()
-    xq, w = sp.quantize_nvfp4(bf(d["X"])), bf(d["W"])
-    v, m = sp.prune_compress_24(w)
-    wq, vq = sp.quantize_nvfp4(w), sp.quantize_nvfp4(v)
-    v48, m48 = sp.prune_compress_48(w)
-    s48, x32 = sp.Sparse48(sp.quantize_nvfp4(v48), m48), sp.quantize_nvfp4_block32(bf(d["X"]))
-    for _ in range(2):
-        sp.gemm_dense(xq, wq)
-        sp.gemm_sparse24(xq, sp.Sparse24(vq, m), 4096)
-        sp.gemm_sparse48(x32, s48, 4096)
-    g = synth.rng(0)
-    w16 = torch.from_numpy(synth.draw(g, (5120, 5120), "f16")).cuda()
-    x16 = torch.from_numpy(synth.draw(g, (4096, 5120), "f16")).cuda()
-    v, m = sp.prune_compress_24(w16)
-    for _ in range(2):
-        sp.gemm_dense(x16, w16)
-        sp.gemm_sparse24(x16, sp.Sparse24(v, m), 5120)
-    del w16, x16, v, m
-    d = synth.moe()
-    E, Ne, Ke = d["W"].shape
-    xm, rt = bf(d["X"]), torch.from_numpy(d["routing"]).cuda()
-    wm = bf(d["W"].reshape(E * Ne, Ke))
-    del d
-    _, wq, sw = sp.prepare_nvfp4_24(wm)
-    del wm
-    sp.gemm_grouped(xm, rt, wq, E, Ne, Ke)
-    sp.gemm_grouped(xm, rt, sw, E, Ne, Ke)
+    if which in ("decode", "all"):
+        d = synth.decode_nvfp4()
+        x, w = bf(d["X"]), bf(d["W"])
+        for _ in range(2):
+            _, wq, sw = sp.prepare_nvfp4_24(w)
+            sp.gemm_dense(x, wq)
+            sp.gemm_sparse24(x, sw, K)
+    if which in ("w4a4", "all"):
+        d = synth.prefill_w4a4()
+        xq, w = sp.quantize_nvfp4(bf(d["X"])), bf(d["W"])
+        wq = sp.quantize_nvfp4(w)
+        xi, wi = sp.to_mma(xq), sp.to_mma(wq)
+        for _ in range(3):
+            sp.gemm_dense(xi, wi)
+    if which == "all":
+        v, m = sp.prune_compress_24(w)
+        vq = sp.quantize_nvfp4(v)
+        v48, m48 = sp.prune_compress_48(w)
+        s48, x32 = sp.Sparse48(sp.quantize_nvfp4(v48), m48), sp.quantize_nvfp4_block32(bf(d["X"]))
+        for _ in range(2):
+            sp.gemm_sparse24(xq, sp.Sparse24(vq, m), 4096)
+            sp.gemm_sparse48(x32, s48, 4096)
+        g = synth.rng(0)
+        w16 = torch.from_numpy(synth.draw(g, (5120, 5120), "f16")).cuda()
+        x16 = torch.from_numpy(synth.draw(g, (4096, 5120), "f16")).cuda()
+        v, m = sp.prune_compress_24(w16)
+        for _ in range(2):
+            sp.gemm_dense(x16, w16)
+            sp.gemm_sparse24(x16, sp.Sparse24(v, m), 5120)
+        del w16, x16, v, m
+        d = synth.moe()
+        E, Ne, Ke = d["W"].shape
+        xm, rt = bf(d["X"]), torch.from_numpy(d["routing"]).cuda()
+        wm = bf(d["W"].reshape(E * Ne, Ke))
+        del d
+        _, wq, sw = sp.prepare_nvfp4_24(wm)
+        del wm
+        sp.gemm_grouped(xm, rt, wq, E, Ne, Ke)
+        sp.gemm_grouped(xm, rt, sw, E, Ne, Ke)
     torch.cuda.synchronize()
     assert sp.last_device_error() == sp.OK
     print("ncu target done")
@@ -963,7 +971,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
-    ap.add_argument("--ncu-target", action="store_true", help="run each kernel once, untimed")
+    ap.add_argument("--ncu-target", nargs="?", const="all", choices=["decode", "w4a4", "all"], default=None,
+                    help="run one kernel family once, untimed (for an ncu capture); no value: all")
     ap.add_argument("--peaks", action="store_true", help="measure MMA and HBM peaks into profiles/peaks.json")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-config GEMM table that follows the timed step")
@@ -972,7 +981,7 @@ def main():
         run_sweep(args)
         return
     if args.ncu_target:
-        run_ncu_target()
+        run_ncu_target(args.ncu_target)
         return
     if args.peaks:
         run_peaks(args)

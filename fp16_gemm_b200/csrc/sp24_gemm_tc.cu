@@ -376,32 +376,7 @@ __global__ void __launch_bounds__(224, 1)
   }
 }
 
-// ------------------------------------------------------------------ W4A4: native NVFP4 GEMM
-//
-// [P1] "NVFP4 vs 2:4 sparse", "The ladder, top to bottom": the measured dense NVFP4 GEMM at 4096
-// cubed is the pages' kernel ceiling.  Here both operands stay packed E2M1 in shared memory
-// (TMA, 128-byte swizzle: 256 K per row) and the tensor core applies the E4M3 block scales from
-// TMEM (tcgen05.mma kind::mxf4nvf4.block_scale.block16, K = 64 per instruction).  Per stage
-// (256 K) the producer also loads each row's 16 scale bytes; warp 6 rewrites them in place into
-// 128-row x 4-scale tiles (row r at byte 16*(r%32) + 4*(r/32)), one tile per MMA and per 128
-// rows (in place, so four 54 KB stages fit at BN = 256), which
-// the MMA thread copies into TMEM with tcgen05.cp.32x128b.warpx4 (lanes 0-31, repeated in every
-// lane quarter).  The tensor scales s_w * s_x multiply the accumulator in the epilogue.
-template <int BN>
-struct QCfg {
-  static constexpr int S = BN == 256 ? 4 : 6;     // stages (the scale tiles are rewritten in place)
-  static constexpr uint32_t A = kBM * 128;        // 128 rows x 256 FP4
-  static constexpr uint32_t B = BN * 128;
-  static constexpr uint32_t SFA = kBM * 16;       // scale rows (16 per 256 K), then tiles
-  static constexpr uint32_t SFB = BN * 16;
-  static constexpr uint32_t STAGE = A + B + SFA + SFB;
-  static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
-  static constexpr int SFA_COLS = 16;             // 4 MMAs x 4 columns
-  static constexpr int SFB_COLS = 4 * (BN / 32);  // 4 MMAs x BN/32 columns
-  static constexpr int COLS = BN + S * (SFA_COLS + SFB_COLS) <= 256 ? 256 : 512;
-  static_assert(STAGE % 1024 == 0 && SMEM <= 232448, "stage layout");
-  static_assert(BN + S * (SFA_COLS + SFB_COLS) <= 512, "TMEM columns");
-};
+// ------------------------------------------------------------------ scale tiles for the sparse FP4 MMA
 
 // Rewrites, in place, the scale rows of `groups` 128-row groups (16 bytes per row: 4 MMAs x 4
 // scales) into the tiles tcgen05.cp reads: tile (j, g) = MMA j, rows 128 g .. 128 g + 127, the
@@ -424,157 +399,6 @@ __device__ __forceinline__ void scale_tiles_in_place(uint8_t* buf, int lane) {
       *reinterpret_cast<uint4*>(buf + 512 * (j * GROUPS + g) + 16 * lane) = make_uint4(col[j][0], col[j][1], col[j][2], col[j][3]);
   }
 }
-
-template <int BN>
-__global__ void __launch_bounds__(224, 1)
-    gemm_nvfp4_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                         const TcParams p) {
-  using C = QCfg<BN>;
-  constexpr int S = C::S;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = tc::align1024(smem_raw);
-  auto sA = [&](int s) { return smem + s * C::STAGE; };
-  auto sB = [&](int s) { return smem + s * C::STAGE + C::A; };
-  auto sSA = [&](int s) { return smem + s * C::STAGE + C::A + C::B; };
-  auto sSB = [&](int s) { return smem + s * C::STAGE + C::A + C::B + C::SFA; };
-  __shared__ uint64_t full_bar[S], sf_bar[S], empty_bar[S], tfull_bar;
-  __shared__ uint32_t tmem_base;
-  __shared__ int aborted;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int n0 = blockIdx.y * BN;
-  const int KB = (p.K + 255) / 256;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&sf_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    mbar_init(&tfull_bar, 1);
-    aborted = 0;
-    fence_mbar_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmSA);
-    prefetch_tmap(&tmSB);
-  }
-  if (warp == 1) tmem_alloc(&tmem_base, C::COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1) || *(volatile int*)&aborted) {
-          aborted = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full_bar[s], C::A + C::B + C::SFA + C::SFB);
-        tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 128, m0);   // 128 bytes = 256 codes
-        tma_load_2d(sB(s), &tmB, &full_bar[s], kb * 128, n0);
-        tma_load_2d(sSA(s), &tmSA, &full_bar[s], kb * 16, m0);  // 16 scales per row
-        tma_load_2d(sSB(s), &tmSB, &full_bar[s], kb * 16, n0);
-        ++issued;
-      }
-      for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
-        mbar_wait(&full_bar[kb % S], (kb / S) & 1);
-    }
-  } else if (warp == 6) {
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % S;
-      const uint32_t ph = (kb / S) & 1;
-      if (!mbar_wait(&full_bar[s], ph) || *(volatile int*)&aborted) {
-        aborted = 1;
-        break;
-      }
-      scale_tiles_in_place<1>(sSA(s), lane);
-      scale_tiles_in_place<BN / 128>(sSB(s), lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sf_bar[s]);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_nvfp4(kBM, BN);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&full_bar[s], ph) || !mbar_wait(&sf_bar[s], ph) || *(volatile int*)&aborted) {
-          aborted = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sfa0 = tmem + BN + s * (C::SFA_COLS + C::SFB_COLS);
-        const uint32_t sfb0 = sfa0 + C::SFA_COLS;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tmem_cp_32x128b_x4(sfa0 + 4 * j, desc_rows16_noswizzle(smem_u32(sSA(s) + 512 * j)));
-#pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-            tmem_cp_32x128b_x4(sfb0 + (BN / 32) * j + 4 * g,
-                               desc_rows16_noswizzle(smem_u32(sSB(s) + 512 * (j * (BN / 128) + g))));
-        }
-        const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
-        const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB(s)));
-#pragma unroll
-        for (int j = 0; j < 4; ++j)  // K = 64 codes = 32 bytes = 2 descriptor units
-          umma_nvfp4(tmem, a0 + 2 * j, b0 + 2 * j, idesc, sfa0 + 4 * j, sfb0 + (BN / 32) * j, (kb | j) != 0);
-        umma_commit(&empty_bar[s]);
-      }
-      umma_commit(&tfull_bar);
-    }
-  } else {
-    const int q = warp & 3;
-    const int row = m0 + 32 * q + lane;
-    if (!mbar_wait(&tfull_bar, 0)) {
-      aborted = 1;
-    } else {
-      tc_fence_after();
-      float scale = 1.0f;
-      if (p.scale_a) scale *= *p.scale_a;
-      if (p.scale_b) scale *= *p.scale_b;
-#pragma unroll 1
-      for (int j = 0; j < BN / 32; ++j) {
-        float v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * j, v);
-        if (row < p.N) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int tok = n0 + 32 * j + i;
-            if (tok < p.M) p.y[(int64_t)tok * p.N + row] = v[i] * scale;
-          }
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0 && aborted) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::COLS);
-  }
-}
-
-template <int BN>
-int launch_nvfp4(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa, const CUtensorMap& sb,
-                 const TcParams& p, cudaStream_t s) {
-  auto kern = gemm_nvfp4_tc_kernel<BN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QCfg<BN>::SMEM) != cudaSuccess)
-    return SP24_ERR_CUDA;
-  dim3 grid((unsigned)((p.N + kBM - 1) / kBM), (unsigned)((p.M + BN - 1) / BN));
-  kern<<<grid, 224, QCfg<BN>::SMEM, s>>>(a, b, sa, sb, p);
-  return launch_status();
-}
-
 
 // ------------------------------------------------------------------ W4A4 with a pairwise 4:8 weight
 //
@@ -849,27 +673,6 @@ int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, i
   dim3 grid((unsigned)((N + kBM - 1) / kBM), (unsigned)((M + kSpBN - 1) / kSpBN));
   kern<<<grid, 224, kSpSmem, s>>>(ta, tb, te, p);
   return launch_status();
-}
-
-// Native NVFP4 x NVFP4 GEMM: y = s_w s_x sum_k dec(x) dec(w) with both operands packed E2M1 +
-// E4M3 scales per 16 (K % 256 == 0, so every 256-wide stage holds 16 whole scale bytes per row).
-int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* wc, const uint8_t* wsc,
-                  const float* w_ts, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t s) {
-  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 256) return SP24_ERR_UNSUPPORTED;
-  // 128-wide activation tiles up to M = 256 (twice the CTAs; 16.2 vs 20.8 us at M = 256,
-  // N = K = 4096), 256-wide above (22.1 vs 32.1 us at M = 1024)
-  const int BN = M > 256 ? 256 : 128;
-  CUtensorMap ta, tb, tsa, tsb;
-  int st = make_tmap_2d(&ta, wc, 1, N, K / 2, K / 2, 128, kBM);
-  if (st) return st;
-  st = make_tmap_2d(&tb, xc, 1, M, K / 2, K / 2, 128, BN);
-  if (st) return st;
-  st = make_tmap_2d_plain(&tsa, wsc, N, K / 16, K / 16, 16, kBM);
-  if (st) return st;
-  st = make_tmap_2d_plain(&tsb, xs, M, K / 16, K / 16, 16, BN);
-  if (st) return st;
-  TcParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts};
-  return BN == 256 ? launch_nvfp4<256>(ta, tb, tsa, tsb, p, s) : launch_nvfp4<128>(ta, tb, tsa, tsb, p, s);
 }
 
 // W4A4 GEMM on the sparse FP4 MMA: y = s_w s_x sum_k dec(x) dec(w) with w a pairwise-4:8 weight

@@ -154,10 +154,6 @@ int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, i
                        int64_t K, bool bf16, float* y, const float* scale_a, const float* scale_b,
                        cudaStream_t s);
 
-// Native NVFP4 x NVFP4 tensor-core GEMM (tcgen05 kind::mxf4nvf4, block16 E4M3 scales); K % 256.
-int tc_gemm_nvfp4(const uint8_t* xc, const uint8_t* xs, const float* x_ts, const uint8_t* wc, const uint8_t* wsc,
-                  const float* w_ts, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t s);
-
 // NVFP4 operand images for the W4A4 kernel (K % 256 == 0): codes [rows, K/2] -> 16 KB tiles of
 // 128 rows x 256 K in the 128-byte-swizzled shared-memory order; scales [rows, K/16] -> 512-byte
 // tiles of 128 rows x 4 scales in tcgen05.cp order.
