@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libsp24.so")
 # status codes (include/sp24.h)
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT, ERR_WORKSPACE = range(9)
-F16, BF16, F32, NVFP4, NVFP4_B32, NVFP4_MMA = 0, 1, 2, 3, 4, 5
+F16, BF16, F32, NVFP4, NVFP4_B32, NVFP4_MMA, NVFP4_B32_MMA = 0, 1, 2, 3, 4, 5, 6
 OP_MATMUL, OP_CONV = 0, 1
 ALGO_AUTO, ALGO_SKINNY, ALGO_TILED = 0, 1, 2
 
@@ -121,6 +121,10 @@ def lib() -> ctypes.CDLL:
             L.sp24_set_wait_limit.argtypes = [ctypes.c_ulonglong]
             L.sp24_get_wait_limit.argtypes = [P]
             L.sp24_selftest_wait_timeout.argtypes = [P, P, P]
+            L.sp24_nvfp4_b32_mma_size.argtypes = [I64, I64, P, P]
+            L.sp24_nvfp4_b32_to_mma.argtypes = [P, P, I64, I64, P, P, P]
+            L.sp24_sparse48_mma_size.argtypes = [I64, I64, P, P, P]
+            L.sp24_sparse48_to_mma.argtypes = [P, P, P, I64, I64, P, P, P, P]
             L.sp24_peak_mma.argtypes = [I, I, P, P]
             L.sp24_peak_ctas.argtypes = [I]
             L.sp24_peak_read.argtypes = [P, I64, P, P]
@@ -572,9 +576,61 @@ class Sparse48(NamedTuple):
     meta: torch.Tensor
 
 
-def gemm_sparse48(x: NVFP4Tensor, w: Sparse48, K: int, out=None, stream=None) -> torch.Tensor:
+class Sparse48MMA(NamedTuple):
+    """A pairwise-4:8 weight [rows, K] as the sparse FP4 pair kernel's tile images (flat uint8:
+    values, scales, metadata; rows padded to 256), with its tensor scale."""
+    values: torch.Tensor
+    scales: torch.Tensor
+    meta: torch.Tensor
+    tensor_scale: torch.Tensor
+    rows: int
+    K: int
+
+
+def sparse48_to_mma(w: Sparse48, K: int, stream=None) -> Sparse48MMA:
+    """The weight rewritten as tile images (sp24_sparse48_to_mma), once per weight."""
+    v = w.values
+    rows = v.codes.shape[0]
+    nv, ns, nm = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+    _call("sp24_sparse48_mma_size", rows, K, ctypes.byref(nv), ctypes.byref(ns), ctypes.byref(nm))
+    dev = v.codes.device
+    vo = torch.empty(nv.value, dtype=torch.uint8, device=dev)
+    so = torch.empty(ns.value, dtype=torch.uint8, device=dev)
+    mo = torch.empty(nm.value, dtype=torch.uint8, device=dev)
+    _call("sp24_sparse48_to_mma", _ptr(v.codes), _ptr(v.scales), _ptr(w.meta), rows, K, _ptr(vo), _ptr(so), _ptr(mo),
+          _stream(stream))
+    return Sparse48MMA(vo, so, mo, v.tensor_scale, rows, K)
+
+
+def b32_to_mma(q: NVFP4Tensor, stream=None) -> NVFP4MMA:
+    """Activations from quantize_nvfp4_block32 rewritten as tile images (sp24_nvfp4_b32_to_mma)."""
+    rows, cols = q.codes.shape[0], 2 * q.codes.shape[1]
+    nc, ns = ctypes.c_int64(0), ctypes.c_int64(0)
+    _call("sp24_nvfp4_b32_mma_size", rows, cols, ctypes.byref(nc), ctypes.byref(ns))
+    codes = torch.empty(nc.value, dtype=torch.uint8, device=q.codes.device)
+    scales = torch.empty(ns.value, dtype=torch.uint8, device=q.codes.device)
+    _call("sp24_nvfp4_b32_to_mma", _ptr(q.codes), _ptr(q.scales), rows, cols, _ptr(codes), _ptr(scales),
+          _stream(stream))
+    return NVFP4MMA(codes, scales, q.tensor_scale, rows, cols)
+
+
+def gemm_sparse48(x, w, K: int, out=None, stream=None) -> torch.Tensor:
     """y[M, N] = x w^T on the sparse FP4 MMA: x from quantize_nvfp4_block32 ([M, K]), w a
-    pairwise-4:8 weight; K % 512 == 0."""
+    pairwise-4:8 weight; K % 512 == 0.  With both operands as tile images (b32_to_mma,
+    sparse48_to_mma) the persistent CTA-pair kernel runs."""
+    if isinstance(x, NVFP4MMA) or isinstance(w, Sparse48MMA):
+        if not (isinstance(x, NVFP4MMA) and isinstance(w, Sparse48MMA)):
+            raise ValueError("tile images are taken for both operands or neither")
+        M, N = x.rows, w.rows
+        if x.cols != K or w.K != K:
+            raise ValueError(f"K mismatch: {x.cols}, {w.K} vs {K}")
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.float32, device=w.meta.device)
+        xo = _Operand(NVFP4_B32_MMA, x.codes.data_ptr(), x.scales.data_ptr(), x.tensor_scale.data_ptr())
+        wo = _SparseOperand(NVFP4_MMA, w.values.data_ptr(), w.scales.data_ptr(), w.tensor_scale.data_ptr(),
+                            w.meta.data_ptr())
+        _call("sp24_gemm_sparse48", ctypes.byref(xo), ctypes.byref(wo), M, N, K, _ptr(out), _stream(stream))
+        return out
     M = x.codes.shape[0]
     if x.codes.shape[1] * 2 != K:
         raise ValueError(f"K mismatch: {x.codes.shape[1] * 2} vs {K}")

@@ -55,16 +55,20 @@ namespace sp24 {
 namespace {
 
 struct ImageJob {
-  const uint4* codes;        // [rows, K/2] bytes as 16-byte pieces
-  const uint32_t* scales;    // [rows, K/16] bytes as words
+  const uint4* codes;        // [rows, K/2] bytes as 16-byte pieces (K = FP4 entries per row)
+  const uint32_t* scales;    // [rows, K/16] (sw = 4) or [rows, K/32] (sw = 2) bytes, as words
+  const uint4* meta;         // pairwise-4:8 nibbles [rows, K/8] bytes (K stored = K/8 bytes), or null
   uint4* codes_out;
   uint32_t* scales_out;
-  int rows, K, tiles;        // tiles = row blocks x K/256
+  uint4* meta_out;
+  int rows, K, sw, tiles;    // sw: scale words per row per 256-entry tile; tiles = row blocks x K/256
 };
 
-// One CTA per code tile (128 rows x 256 K): its 16 KB of codes (8 threads per 128-byte row
-// segment, reads coalesced, each 128-byte row written whole) and the four scale tiles of the
-// same rows and K range.  Up to two operands per launch (job b may be empty).
+// One CTA per code tile (128 rows x 256 entries): its 16 KB of codes (8 threads per 128-byte row
+// segment, reads coalesced, each 128-byte row written whole), the scale tiles of the same rows
+// and range (sw of them) and, for a pairwise-4:8 weight, its two 2 KB metadata tiles (row r's
+// 16 bytes at 16 r; padding rows get 0x44, the legal index pair 0, 1).  Row blocks past `rows`
+// are padding.  Up to two operands per launch (job b may be empty).
 __global__ void __launch_bounds__(256) to_mma_kernel(ImageJob ja, ImageJob jb) {
   int t = blockIdx.x;
   const bool second = t >= ja.tiles;
@@ -77,23 +81,34 @@ __global__ void __launch_bounds__(256) to_mma_kernel(ImageJob ja, ImageJob jb) {
     const uint4 v = r < j.rows ? j.codes[(int64_t)r * (j.K / 32) + kc * 8 + c] : zero;
     j.codes_out[(int64_t)t * 1024 + rr * 8 + (c ^ (rr & 7))] = v;
   }
-  for (int i = threadIdx.x; i < 512; i += 256) {
-    const int rr = i >> 2, w = i & 3, r = rb * 128 + rr;
-    const uint32_t v = r < j.rows ? j.scales[(int64_t)r * (j.K / 64) + kc * 4 + w] : 0u;
-    j.scales_out[((int64_t)rb * (j.K / 64) + kc * 4 + w) * 128 + 4 * (rr & 31) + (rr >> 5)] = v;
+  const int spr = kc256 * j.sw;  // scale words per row
+  for (int i = threadIdx.x; i < 128 * j.sw; i += 256) {
+    const int rr = i / j.sw, w = i - rr * j.sw, r = rb * 128 + rr;
+    const uint32_t v = r < j.rows ? j.scales[(int64_t)r * spr + kc * j.sw + w] : 0u;
+    j.scales_out[((int64_t)rb * spr + kc * j.sw + w) * 128 + 4 * (rr & 31) + (rr >> 5)] = v;
+  }
+  if (j.meta) {  // K entries stored = 2K logical; K/8 meta bytes per row, 32 per code tile
+    const int rr = threadIdx.x >> 1, h = threadIdx.x & 1, r = rb * 128 + rr;
+    const uint4 v = r < j.rows ? j.meta[(int64_t)r * (j.K / 128) + kc * 2 + h]
+                               : make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    j.meta_out[((int64_t)rb * kc256 * 2 + kc * 2 + h) * 128 + rr] = v;
   }
 }
 
 ImageJob image_job(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
-                   uint8_t* scales_out) {
+                   uint8_t* scales_out, int sw = 4, int64_t row_blocks = -1, const uint8_t* meta = nullptr,
+                   uint8_t* meta_out = nullptr) {
   ImageJob j;
   j.codes = reinterpret_cast<const uint4*>(codes);
   j.scales = reinterpret_cast<const uint32_t*>(scales);
+  j.meta = reinterpret_cast<const uint4*>(meta);
   j.codes_out = reinterpret_cast<uint4*>(codes_out);
   j.scales_out = reinterpret_cast<uint32_t*>(scales_out);
+  j.meta_out = reinterpret_cast<uint4*>(meta_out);
   j.rows = (int)rows;
   j.K = (int)K;
-  j.tiles = (int)((rows + 127) / 128 * (K / 256));
+  j.sw = sw;
+  j.tiles = (int)((row_blocks >= 0 ? row_blocks : (rows + 127) / 128) * (K / 256));
   return j;
 }
 
@@ -121,34 +136,70 @@ int nvfp4_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int6
   return nvfp4_to_mma2(codes, scales, rows, codes_out, scales_out, nullptr, nullptr, 0, nullptr, nullptr, K, s);
 }
 
+// Images for the sparse FP4 pair kernel: activations with one scale per 32 K (scale tiles of
+// 128 K), and a pairwise-4:8 weight (kept values [rows, K/2] as codes with one scale per 16
+// stored, metadata tiles), rows padded to whole 256-row pair tiles.
+int64_t b32_mma_scales_bytes(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * (K / 32); }
+int64_t sp48_rows_padded(int64_t rows) { return (rows + 255) / 256 * 256; }
+int64_t sp48_mma_values_bytes(int64_t rows, int64_t K) { return sp48_rows_padded(rows) * (K / 4); }
+int64_t sp48_mma_scales_bytes(int64_t rows, int64_t K) { return sp48_rows_padded(rows) * (K / 32); }
+int64_t sp48_mma_meta_bytes(int64_t rows, int64_t K) { return sp48_rows_padded(rows) * (K / 16); }
+
+int nvfp4_b32_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
+                     uint8_t* scales_out, cudaStream_t s) {
+  if (K % 256 || rows > INT32_MAX || K > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  const ImageJob j = image_job(codes, scales, rows, K, codes_out, scales_out, 2);
+  if (j.tiles == 0) return SP24_OK;
+  to_mma_kernel<<<(unsigned)j.tiles, 256, 0, s>>>(j, image_job(nullptr, nullptr, 0, 256, nullptr, nullptr));
+  return launch_status();
+}
+
+int sp48_to_mma(const uint8_t* values, const uint8_t* scales, const uint8_t* meta, int64_t rows, int64_t K,
+                uint8_t* values_out, uint8_t* scales_out, uint8_t* meta_out, cudaStream_t s) {
+  if (K % 512 || rows > INT32_MAX || K > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  const ImageJob j = image_job(values, scales, rows, K / 2, values_out, scales_out, 4, sp48_rows_padded(rows) / 128,
+                               meta, meta_out);
+  if (j.tiles == 0) return SP24_OK;
+  to_mma_kernel<<<(unsigned)j.tiles, 256, 0, s>>>(j, image_job(nullptr, nullptr, 0, 256, nullptr, nullptr));
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ the pair GEMM
 
 namespace {
 
 using namespace tc;
 
-template <int BN>
+// SP: the pairwise-4:8 sparse FP4 MMA (tcgen05.mma.sp kind::mxf4nvf4, K = 128 logical per
+// instruction): a stage is 512 logical K (A 256 stored codes per row, B two 256-entry tiles),
+// plus two 2 KB metadata tiles per CTA; dense: a stage is 256 K.
+template <int BN, bool SP = false>
 struct PairCfg {
   static constexpr uint32_t A = 16384;                 // 128 weight rows x 256 FP4: one tile
-  static constexpr uint32_t B = (BN / 2) * 128;        // this CTA's half of the tokens
+  static constexpr uint32_t B = (SP ? 2 : 1) * (BN / 2) * 128;  // this CTA's half of the tokens
   static constexpr uint32_t SFA = 2048;                // 4 scale tiles (128 rows x 4 scales)
   static constexpr uint32_t SFB = (BN / 128) * 2048;   // all BN tokens' scale tiles
-  static constexpr uint32_t STAGE = A + B + SFA + SFB;
-  static constexpr int S = BN == 256 ? 5 : 6;
+  static constexpr uint32_t META = SP ? 4096 : 0;      // two metadata tiles (128 rows x 16 bytes)
+  static constexpr uint32_t STAGE = A + B + SFA + SFB + META;
+  static constexpr int S = SP ? (BN == 256 ? 3 : 4) : (BN == 256 ? 5 : 6);
   static constexpr uint32_t EPI = 32 * 128 * 4;        // one 32-token x 128-row fp32 chunk
   static constexpr size_t SMEM = (size_t)S * STAGE + 2 * EPI + 1024;
-  // TMEM columns: two accumulators (overlapping in 96 columns at BN = 256), then two stages of
-  // scale factors (per MMA: SFA 4 columns + SFB BN/32), so the copies for stage i + 1 run while
-  // the MMAs of stage i read theirs
-  static constexpr uint32_t ACC1 = BN == 256 ? 160 : BN;
+  static constexpr int KSTAGE = SP ? 512 : 256;        // logical K per stage
+  // TMEM columns: two accumulators (overlapping at BN = 256), then two stages of scale factors
+  // (per MMA: SFA 4 columns + SFB BN/32; SP: then 8 metadata columns), so the copies for stage
+  // i + 1 run while the MMAs of stage i read theirs
+  static constexpr uint32_t ACC1 = BN == 256 ? (SP ? 128 : 160) : BN;
   static constexpr uint32_t SF = ACC1 + BN;
   static constexpr uint32_t SLOT = 4 + BN / 32;     // one MMA's scale columns
-  static constexpr uint32_t SF_STAGE = 4 * SLOT;    // one 256-K stage
+  static constexpr uint32_t META_COL = 4 * SLOT;    // SP: metadata columns after the scales
+  static constexpr uint32_t SF_STAGE = 4 * SLOT + (SP ? 8 : 0);
   static constexpr uint32_t COLS = 512;
   static constexpr int CHUNKS = BN / 32;
-  static constexpr int OVERLAP_CHUNKS = BN == 256 ? 3 : 0;  // read before the accumulator is released
+  static constexpr int OVERLAP_CHUNKS = BN == 256 ? (int)((256 - ACC1) / 32) : 0;
+  static constexpr int EARLY = OVERLAP_CHUNKS > 3 ? OVERLAP_CHUNKS : 3;  // chunks read before the release
   static_assert(STAGE % 1024 == 0 && SMEM <= 232448, "shared memory layout");
   static_assert(SF + 2 * SF_STAGE <= COLS, "TMEM columns");
+  static_assert(EARLY <= CHUNKS, "epilogue buffers");
 };
 
 struct PairParams {
@@ -162,12 +213,13 @@ struct PairParams {
 
 // TMA_Y: the epilogue stages each 32-token chunk in shared memory and writes it with one TMA
 // store (needs N % 4 == 0 and a 16-byte aligned y); otherwise each warp stores its rows directly.
-template <int BN, bool TMA_Y>
+template <int BN, bool TMA_Y, bool SP>
 __global__ void __launch_bounds__(256, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                           const __grid_constant__ CUtensorMap tmY, const PairParams p) {
-  using C = PairCfg<BN>;
+                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                           const PairParams p) {
+  using C = PairCfg<BN, SP>;
   constexpr int S = C::S;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = tc::align1024(smem_raw);
@@ -175,6 +227,7 @@ __global__ void __launch_bounds__(256, 1)
   auto sB = [&](int s) { return sA(s) + C::A; };
   auto sSA = [&](int s) { return sB(s) + C::B; };
   auto sSB = [&](int s) { return sSA(s) + C::SFA; };
+  auto sE = [&](int s) { return sSB(s) + C::SFB; };  // SP: metadata tiles
   float* sY = reinterpret_cast<float*>(smem + S * C::STAGE);  // two epilogue chunks
   __shared__ uint64_t full_bar[S], empty_bar[S], sf_bar[2 * S], tfull_bar, tempty_bar;
   __shared__ uint32_t tmem_base;
@@ -185,7 +238,7 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = (int)cluster_id_x(), pairs = (int)cluster_count_x();
-  const int KB = p.K / 256;
+  const int KB = p.K / C::KSTAGE;
   const int tiles = p.tiles_w * p.tiles_n;
   const uint64_t wait_ns = p.wait_ns ? p.wait_ns : wait_limit();
 
@@ -205,6 +258,7 @@ __global__ void __launch_bounds__(256, 1)
     prefetch_tmap(&tmSA);
     prefetch_tmap(&tmSB);
     if (TMA_Y) prefetch_tmap(&tmY);
+    if (SP) prefetch_tmap(&tmE);
   }
   if (warp == 1) tmem_alloc_pair(&tmem_base, C::COLS);
   tc_fence_before();
@@ -231,16 +285,26 @@ __global__ void __launch_bounds__(256, 1)
           }
           const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
           if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * C::STAGE);
-          // code tiles: 8 rows of 2 KB each; a 64-token half tile is 4 of them
+          // code tiles: 8 rows of 2 KB each; a 64-token half tile is 4 of them.  SP: A holds the
+          // kept values (K/2 stored per row, one tile per stage), B two consecutive tiles
+          constexpr int TB = SP ? 2 : 1;          // token tiles per stage
+          const int kcx = p.K / 256;              // token tiles per row block
           tma_load_2d_pair(sA(s), &tmA, fb, 0, (wb * KB + kb) * 8);
-          if (BN == 256)
-            tma_load_2d_pair(sB(s), &tmB, fb, 0, ((n0 / 128 + (int)rank) * KB + kb) * 8);
-          else
-            tma_load_2d_pair(sB(s), &tmB, fb, 0, ((n0 / 128) * KB + kb) * 8 + 4 * (int)rank);
-          tma_load_2d_pair(sSA(s), &tmSA, fb, 0, wb * (p.K / 64) + kb * 4);  // 4 scale tiles
+          if (BN == 256) {
+            tma_load_2d_pair(sB(s), &tmB, fb, 0, ((n0 / 128 + (int)rank) * kcx + TB * kb) * 8);
+          } else {
+#pragma unroll
+            for (int u = 0; u < TB; ++u)
+              tma_load_2d_pair(sB(s) + u * (BN / 2) * 128, &tmB, fb, 0,
+                               ((n0 / 128) * kcx + TB * kb + u) * 8 + 4 * (int)rank);
+          }
+          // four scale tiles per stage (dense: 64 K each; SP: 128 logical K each)
+          const int kst = p.K / (SP ? 128 : 64);  // scale tiles per row block
+          tma_load_2d_pair(sSA(s), &tmSA, fb, 0, wb * kst + kb * 4);
 #pragma unroll
           for (int g = 0; g < BN / 128; ++g)
-            tma_load_2d_pair(sSB(s) + 2048 * g, &tmSB, fb, 0, (n0 / 128 + g) * (p.K / 64) + kb * 4);
+            tma_load_2d_pair(sSB(s) + 2048 * g, &tmSB, fb, 0, (n0 / 128 + g) * kst + kb * 4);
+          if (SP) tma_load_2d_pair(sE(s), &tmE, fb, 0, wb * (p.K / 256) + kb * 2);  // 2 metadata tiles
         }
       }
       // the even CTA's producer armed every stage it counted: wait (bounded) until those copies
@@ -250,7 +314,7 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_nvfp4(256, BN);
+      const uint32_t idesc = idesc_nvfp4(256, BN, SP);
       int it = 0, j = 0;
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += pairs, ++j) {
@@ -280,9 +344,15 @@ __global__ void __launch_bounds__(256, 1)
             }
             tc_fence_after();
 #pragma unroll
-            for (int q = 2 * h; q < 2 * h + 2; ++q)  // K = 64 codes = 32 bytes = 2 descriptor units
-              umma_nvfp4_pair(d, a0 + 2 * q, b0 + 2 * q, idesc, sf0 + C::SLOT * q, sf0 + C::SLOT * q + 4,
-                              (kb | q) != 0);
+            for (int q = 2 * h; q < 2 * h + 2; ++q) {
+              if (SP)  // A: 64 stored = 32 bytes; B: 128 entries = 64 bytes of token tile q / 2
+                umma_nvfp4_sp_pair(d, a0 + 2 * q, b0 + (uint64_t)((q >> 1) * (BN / 2) * 128 / 16) + 4 * (q & 1),
+                                   sf0 + C::META_COL + 2 * q, idesc, sf0 + C::SLOT * q, sf0 + C::SLOT * q + 4,
+                                   (kb | q) != 0);
+              else  // K = 64 codes = 32 bytes = 2 descriptor units
+                umma_nvfp4_pair(d, a0 + 2 * q, b0 + 2 * q, idesc, sf0 + C::SLOT * q, sf0 + C::SLOT * q + 4,
+                                (kb | q) != 0);
+            }
           }
           if (!ok) break;
           umma_commit_pair(&empty_bar[s], 0x3);
@@ -321,6 +391,8 @@ __global__ void __launch_bounds__(256, 1)
               tmem_cp_32x128b_x4_pair(sf0 + C::SLOT * q + 4 + 4 * g,
                                       desc_rows16_noswizzle(smem_u32(sSB(s) + 2048 * g + 512 * q)));
           }
+          // SP: metadata tile h (256 logical K, MMAs 2h and 2h + 1) -> row m on lane m, 4 columns
+          if (SP) tmem_cp_128x128b_pair(sf0 + C::META_COL + 4 * h, desc_rows16_noswizzle(smem_u32(sE(s) + 2048 * h)));
           umma_commit_pair(&sf_bar[h * S + s], 0x1);
         }
       }
@@ -452,11 +524,11 @@ int make_tmap_y(CUtensorMap* map, float* y, int64_t M, int64_t N) {
   return r == CUDA_SUCCESS ? SP24_OK : SP24_ERR_CUDA;
 }
 
-template <int BN, bool TMA_Y>
+template <int BN, bool TMA_Y, bool SP>
 int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa, const CUtensorMap& sb,
-                const CUtensorMap& ty, const PairParams& p, cudaStream_t s) {
-  auto kern = gemm_nvfp4_pair_kernel<BN, TMA_Y>;
-  const size_t smem = PairCfg<BN>::SMEM;
+                const CUtensorMap& te, const CUtensorMap& ty, const PairParams& p, cudaStream_t s) {
+  auto kern = gemm_nvfp4_pair_kernel<BN, TMA_Y, SP>;
+  const size_t smem = PairCfg<BN, SP>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
   const int tiles = p.tiles_w * p.tiles_n;
@@ -475,7 +547,7 @@ int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& s
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, a, b, sa, sb, ty, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, a, b, sa, sb, te, ty, p) != cudaSuccess) {
     cudaGetLastError();
     return SP24_ERR_CUDA;
   }
@@ -497,7 +569,7 @@ int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float
   const int BN = M > 128 ? 256 : 128;
   const uint64_t tiles_w = (uint64_t)(N + 127) / 128 * (K / 256), tiles_x = (uint64_t)(M + 127) / 128 * (K / 256);
   if (tiles_w * 8 > INT32_MAX || tiles_x * 8 > INT32_MAX) return SP24_ERR_UNSUPPORTED;
-  CUtensorMap ta, tb, tsa, tsb, ty;
+  CUtensorMap ta, tb, tsa, tsb, ty, te;
   int st = make_tmap_rows(&ta, wc_mma, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 2048, tiles_w * 8, 8);
   if (st) return st;
   st = make_tmap_rows(&tb, xc_mma, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 2048, tiles_x * 8, BN == 256 ? 8 : 4);
@@ -508,11 +580,50 @@ int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float
   if (st) return st;
   const bool tma_y = N % 4 == 0 && aligned(y, 16);
   memset(&ty, 0, sizeof(ty));
+  memset(&te, 0, sizeof(te));
   if (tma_y && (st = make_tmap_y(&ty, y, M, N))) return st;
   PairParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts, (int)((N + 255) / 256), (int)((M + BN - 1) / BN), wait_ns};
   if (BN == 256)
-    return tma_y ? launch_pair<256, true>(ta, tb, tsa, tsb, ty, p, s) : launch_pair<256, false>(ta, tb, tsa, tsb, ty, p, s);
-  return tma_y ? launch_pair<128, true>(ta, tb, tsa, tsb, ty, p, s) : launch_pair<128, false>(ta, tb, tsa, tsb, ty, p, s);
+    return tma_y ? launch_pair<256, true, false>(ta, tb, tsa, tsb, te, ty, p, s)
+                 : launch_pair<256, false, false>(ta, tb, tsa, tsb, te, ty, p, s);
+  return tma_y ? launch_pair<128, true, false>(ta, tb, tsa, tsb, te, ty, p, s)
+               : launch_pair<128, false, false>(ta, tb, tsa, tsb, te, ty, p, s);
+}
+
+// W4A4 on the sparse FP4 MMA with a pairwise-4:8 weight, CTA-pair kernel: x as images with one
+// scale per 32 K (nvfp4_b32_to_mma), the weight as images (sp48_to_mma: kept values, their
+// scales, metadata; rows padded to 256); K % 512 == 0.
+int tc_gemm_nvfp4_sp48_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float* x_ts, const uint8_t* vc_mma,
+                            const uint8_t* vs_mma, const uint8_t* meta_mma, const float* w_ts, int64_t M, int64_t N,
+                            int64_t K, float* y, cudaStream_t s, uint64_t wait_ns) {
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 512) return SP24_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return SP24_OK;
+  if (K == 0)
+    return cudaMemsetAsync(y, 0, (size_t)(M * N) * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  const int BN = M > 128 ? 256 : 128;
+  const uint64_t wblocks = (uint64_t)sp48_rows_padded(N) / 128, xblocks = (uint64_t)(M + 127) / 128;
+  if (wblocks * (K / 512) * 8 > INT32_MAX || xblocks * (K / 256) * 8 > INT32_MAX) return SP24_ERR_UNSUPPORTED;
+  CUtensorMap ta, tb, tsa, tsb, ty, te;
+  int st = make_tmap_rows(&ta, vc_mma, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 2048, wblocks * (K / 512) * 8, 8);
+  if (st) return st;
+  st = make_tmap_rows(&tb, xc_mma, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 2048, xblocks * (K / 256) * 8,
+                      BN == 256 ? 16 : 4);
+  if (st) return st;
+  st = make_tmap_rows(&tsa, vs_mma, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 512, wblocks * (K / 128), 4);
+  if (st) return st;
+  st = make_tmap_rows(&tsb, xs_mma, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 512, xblocks * (K / 128), 4);
+  if (st) return st;
+  st = make_tmap_rows(&te, meta_mma, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 2048, wblocks * (K / 256), 2);
+  if (st) return st;
+  const bool tma_y = N % 4 == 0 && aligned(y, 16);
+  memset(&ty, 0, sizeof(ty));
+  if (tma_y && (st = make_tmap_y(&ty, y, M, N))) return st;
+  PairParams p{(int)M, (int)N, (int)K, y, w_ts, x_ts, (int)((N + 255) / 256), (int)((M + BN - 1) / BN), wait_ns};
+  if (BN == 256)
+    return tma_y ? launch_pair<256, true, true>(ta, tb, tsa, tsb, te, ty, p, s)
+                 : launch_pair<256, false, true>(ta, tb, tsa, tsb, te, ty, p, s);
+  return tma_y ? launch_pair<128, true, true>(ta, tb, tsa, tsb, te, ty, p, s)
+               : launch_pair<128, false, true>(ta, tb, tsa, tsb, te, ty, p, s);
 }
 
 }  // namespace sp24

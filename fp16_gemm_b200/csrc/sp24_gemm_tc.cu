@@ -749,7 +749,8 @@ using namespace sp24;
 extern "C" int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
                                   int64_t K, float* y, void* stream) {
   if (!x || !w) return SP24_ERR_INVALID_ARG;
-  if (x->format != SP24_NVFP4_B32 || w->format != SP24_NVFP4) return SP24_ERR_DTYPE;
+  const bool images = x->format == SP24_NVFP4_B32_MMA && w->format == SP24_NVFP4_MMA;
+  if (!images && (x->format != SP24_NVFP4_B32 || w->format != SP24_NVFP4)) return SP24_ERR_DTYPE;
   if (M < 0 || N < 0 || K < 0 || K % 512) return SP24_ERR_SHAPE;
   if (M == 0 || N == 0) return SP24_OK;
   if (!y) return SP24_ERR_INVALID_ARG;
@@ -761,7 +762,49 @@ extern "C" int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_opera
         !aligned(w->meta, 16))
       return SP24_ERR_ALIGN;
   }
+  if (images)
+    return tc_gemm_nvfp4_sp48_pair(static_cast<const uint8_t*>(x->data), x->scales, x->tensor_scale,
+                                   static_cast<const uint8_t*>(w->values), w->scales, w->meta, w->tensor_scale, M, N,
+                                   K, y, as_stream(stream), 0);
   return tc_gemm_nvfp4_sp48(static_cast<const uint8_t*>(x->data), x->scales, x->tensor_scale,
                             static_cast<const uint8_t*>(w->values), w->scales, w->meta, w->tensor_scale, M, N, K, y,
                             as_stream(stream));
+}
+
+extern "C" int sp24_nvfp4_b32_mma_size(int64_t rows, int64_t cols, int64_t* codes_bytes, int64_t* scales_bytes) {
+  if (rows < 0 || cols < 0 || cols % 256) return SP24_ERR_SHAPE;
+  if (codes_bytes) *codes_bytes = nvfp4_mma_codes_bytes(rows, cols);
+  if (scales_bytes) *scales_bytes = b32_mma_scales_bytes(rows, cols);
+  return SP24_OK;
+}
+
+extern "C" int sp24_nvfp4_b32_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                     uint8_t* codes_out, uint8_t* scales_out, void* stream) {
+  if (rows < 0 || cols < 0 || cols % 256) return SP24_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return SP24_OK;
+  if (!codes || !scales || !codes_out || !scales_out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || !aligned(codes_out, 16) || !aligned(scales_out, 16))
+    return SP24_ERR_ALIGN;
+  return nvfp4_b32_to_mma(codes, scales, rows, cols, codes_out, scales_out, as_stream(stream));
+}
+
+extern "C" int sp24_sparse48_mma_size(int64_t rows, int64_t K, int64_t* values_bytes, int64_t* scales_bytes,
+                                      int64_t* meta_bytes) {
+  if (rows < 0 || K < 0 || K % 512) return SP24_ERR_SHAPE;
+  if (values_bytes) *values_bytes = sp48_mma_values_bytes(rows, K);
+  if (scales_bytes) *scales_bytes = sp48_mma_scales_bytes(rows, K);
+  if (meta_bytes) *meta_bytes = sp48_mma_meta_bytes(rows, K);
+  return SP24_OK;
+}
+
+extern "C" int sp24_sparse48_to_mma(const uint8_t* values, const uint8_t* scales, const uint8_t* meta,
+                                    int64_t rows, int64_t K, uint8_t* values_out, uint8_t* scales_out,
+                                    uint8_t* meta_out, void* stream) {
+  if (rows < 0 || K < 0 || K % 512) return SP24_ERR_SHAPE;
+  if (rows == 0 || K == 0) return SP24_OK;
+  if (!values || !scales || !meta || !values_out || !scales_out || !meta_out) return SP24_ERR_INVALID_ARG;
+  if (!aligned(values, 16) || !aligned(scales, 4) || !aligned(meta, 16) || !aligned(values_out, 16) ||
+      !aligned(scales_out, 16) || !aligned(meta_out, 16))
+    return SP24_ERR_ALIGN;
+  return sp48_to_mma(values, scales, meta, rows, K, values_out, scales_out, meta_out, as_stream(stream));
 }

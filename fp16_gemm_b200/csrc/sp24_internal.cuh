@@ -166,6 +166,20 @@ int nvfp4_to_mma2(const uint8_t* c0, const uint8_t* s0, int64_t rows0, uint8_t* 
                   const uint8_t* c1, const uint8_t* s1, int64_t rows1, uint8_t* co1, uint8_t* so1, int64_t K,
                   cudaStream_t s);
 
+// Images for the sparse FP4 pair kernel: activations with one scale per 32 K; a pairwise-4:8
+// weight (kept values, their scales, metadata tiles), rows padded to 256.
+int64_t b32_mma_scales_bytes(int64_t rows, int64_t K);
+int64_t sp48_mma_values_bytes(int64_t rows, int64_t K);
+int64_t sp48_mma_scales_bytes(int64_t rows, int64_t K);
+int64_t sp48_mma_meta_bytes(int64_t rows, int64_t K);
+int nvfp4_b32_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, uint8_t* codes_out,
+                     uint8_t* scales_out, cudaStream_t s);
+int sp48_to_mma(const uint8_t* values, const uint8_t* scales, const uint8_t* meta, int64_t rows, int64_t K,
+                uint8_t* values_out, uint8_t* scales_out, uint8_t* meta_out, cudaStream_t s);
+int tc_gemm_nvfp4_sp48_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float* x_ts, const uint8_t* vc_mma,
+                            const uint8_t* vs_mma, const uint8_t* meta_mma, const float* w_ts, int64_t M, int64_t N,
+                            int64_t K, float* y, cudaStream_t s, uint64_t wait_ns);
+
 // W4A4 GEMM on the persistent CTA-pair kernel (both operands as images above).  wait_ns bounds
 // every device-side wait (0: the library's default).
 int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float* x_ts, const uint8_t* wc_mma,

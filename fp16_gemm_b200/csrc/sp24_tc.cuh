@@ -421,6 +421,25 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
       : "memory");
 }
 
+// Sparse block-scaled FP4 MMA over the CTA pair (pairwise 4:8 A, K = 128 logical per
+// instruction), metadata at `e_tmem` in each CTA's TMEM.
+__device__ __forceinline__ void umma_nvfp4_sp_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                                   uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %7, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%3], %4, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+// 128 TMEM lanes x 128 bits (4 columns) in both CTAs of the pair, each from its own shared
+// memory (the source form of desc_rows16_noswizzle).
+__device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Scale-factor copy (32 rows x 128 bits, repeated in the four lane quarters) in both CTAs of
 // the pair, each from its own shared memory at the same address into its own TMEM.
 __device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {

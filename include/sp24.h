@@ -45,7 +45,8 @@ enum {
 
 /* ----------------------------------------------------------------------- enums */
 /* element types */
-enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3, SP24_NVFP4_B32 = 4, SP24_NVFP4_MMA = 5 };
+enum { SP24_F16 = 0, SP24_BF16 = 1, SP24_F32 = 2, SP24_NVFP4 = 3, SP24_NVFP4_B32 = 4, SP24_NVFP4_MMA = 5,
+       SP24_NVFP4_B32_MMA = 6 };
 
 /* The operation a weight belongs to decides which four entries form a group ([P2] "The
  * operation determines which four entries belong together"). */
@@ -69,7 +70,9 @@ enum { SP24_ALGO_AUTO = 0, SP24_ALGO_SKINNY = 1, SP24_ALGO_TILED = 2 };
  *       [rows, K/32] (the activation form read by sp24_gemm_sparse48 only).
  *   format SP24_NVFP4_MMA: SP24_NVFP4 rewritten as tile images (sp24_nvfp4_to_mma): data ->
  *       code tiles, scales -> scale tiles; accepted by sp24_gemm_dense when both operands are
- *       NVFP4 (either layout), K % 256 == 0. 
+ *       NVFP4 (either layout), K % 256 == 0.
+ *   format SP24_NVFP4_B32_MMA: SP24_NVFP4_B32 rewritten as tile images
+ *       (sp24_nvfp4_b32_to_mma), the activation form of sp24_gemm_sparse48's pair kernel. 
  * Decoded value = E2M1(code) * E4M3(scale) * tensor_scale. */
 typedef struct {
   int32_t format;
@@ -174,6 +177,31 @@ int sp24_decompress_48(const void* values, const uint8_t* meta, int dtype, int64
  * 2^31 - 1.  Wrong formats: SP24_ERR_DTYPE.  One launch; nothing is allocated. */
 int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
                        int64_t K, float* y, void* stream);
+
+/* The same GEMM on tile images (x format SP24_NVFP4_B32_MMA, w format SP24_NVFP4_MMA; both or
+ * neither) runs a persistent kernel on pairs of SMs (tcgen05.mma.sp.cta_group::2, 256 weight
+ * rows x 256 tokens per pair tile, 512 logical K per stage).  Not on the source pages: layouts
+ * of this library's kernel.
+ *   sp24_nvfp4_b32_mma_size / sp24_nvfp4_b32_to_mma: activations [rows, cols] (cols % 256 == 0)
+ *       with one scale per 32 entries -> code tiles as sp24_nvfp4_to_mma, scale tiles of 128 rows
+ *       x 4 scales (128 entries) at byte 512 * (rb * cols/128 + t), row r at 16 (r % 32) +
+ *       4 (r / 32); rows padded to 128.
+ *   sp24_sparse48_mma_size / sp24_sparse48_to_mma: a pairwise-4:8 weight [rows, K] (K % 512):
+ *       the kept values' codes [rows, K/4] and scales [rows, K/32] as the code and scale tiles of
+ *       a [rows, K/2] NVFP4 tensor (scale tiles of 64 stored = 128 logical K), the metadata
+ *       [rows, K/16] as 2 KB tiles per 128 rows and 256 logical K (row r's 16 bytes at 16 r);
+ *       rows padded to a multiple of 256 with zero codes and scales and metadata 0x44 (a legal
+ *       pattern), so every tile the kernel loads exists.
+ * Inputs device, codes and metadata 16-byte aligned, scales 4-byte aligned; outputs 16-byte
+ * aligned, of the sizes the queries give.  One launch each. */
+int sp24_nvfp4_b32_mma_size(int64_t rows, int64_t cols, int64_t* codes_bytes, int64_t* scales_bytes);
+int sp24_nvfp4_b32_to_mma(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                          uint8_t* codes_out, uint8_t* scales_out, void* stream);
+int sp24_sparse48_mma_size(int64_t rows, int64_t K, int64_t* values_bytes, int64_t* scales_bytes,
+                           int64_t* meta_bytes);
+int sp24_sparse48_to_mma(const uint8_t* values, const uint8_t* scales, const uint8_t* meta, int64_t rows,
+                         int64_t K, uint8_t* values_out, uint8_t* scales_out, uint8_t* meta_out,
+                         void* stream);
 
 /* ----------------------------------------------------------------------- a3: NVFP4 */
 /* [P5] "Convert BF16 to NVFP4 yourself", "The shared global scale": quantise T[rows, cols]

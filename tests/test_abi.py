@@ -215,3 +215,19 @@ def test_peak_microbenchmark_host_validation():
     assert L.sp24_peak_mma(0, 10, ctypes.c_void_p(4), None) == sp.ERR_ALIGN
     assert L.sp24_peak_read(None, 1024, None, None) == sp.ERR_INVALID_ARG
     assert L.sp24_peak_read(ctypes.c_void_p(16), 24, ctypes.c_void_p(16), None) == sp.ERR_INVALID_ARG
+
+
+def test_sparse_pair_images_host_validation():
+    L = sp.lib()
+    a, b, c = ctypes.c_int64(-1), ctypes.c_int64(-1), ctypes.c_int64(-1)
+    assert L.sp24_sparse48_mma_size(300, 1024, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == sp.OK
+    assert (a.value, b.value, c.value) == (512 * 256, 512 * 32, 512 * 64)
+    assert L.sp24_sparse48_mma_size(8, 768, None, None, None) == sp.ERR_SHAPE
+    assert L.sp24_nvfp4_b32_mma_size(200, 512, ctypes.byref(a), ctypes.byref(b)) == sp.OK
+    assert (a.value, b.value) == (256 * 256, 256 * 16)
+    assert L.sp24_sparse48_to_mma(None, None, None, 4, 512, None, None, None, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_nvfp4_b32_to_mma(None, None, 4, 256, None, None, None) == sp.ERR_INVALID_ARG
+    # images are taken for both operands or neither
+    xo = sp._Operand(sp.NVFP4_B32_MMA, 16, 16, 16)
+    wo = sp._SparseOperand(sp.NVFP4, 16, 16, 16, 16)
+    assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 4, 128, 512, ctypes.c_void_p(256), None) == sp.ERR_DTYPE

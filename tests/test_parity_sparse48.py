@@ -88,13 +88,20 @@ def _run(M, N, K, seed):
     assert np.array_equal(to_host(vq.codes), vc) and np.array_equal(to_host(vq.scales), vs)
     assert np.array_equal(to_host(xq.codes), xc) and np.array_equal(to_host(xq.scales), xs)
     assert_gemm_close(y, Y, S)
+    # the same product on the CTA-pair kernel from tile images of the same operands
+    y2 = sp.gemm_sparse48(sp.b32_to_mma(xq), sp.sparse48_to_mma(sp.Sparse48(vq, m), K), K)
+    torch.cuda.synchronize()
+    assert sp.last_device_error() == sp.OK
+    assert_gemm_close(y2, Y, S)
 
 
 @pytest.mark.parametrize("mnk", [(1, 128, 512), (96, 200, 1024), (128, 256, 512), (300, 384, 1536),
-                                 (129, 129, 2048), (512, 130, 1024)], ids=lambda t: "x".join(map(str, t)))
+                                 (129, 129, 2048), (512, 130, 1024), (1280, 4096, 512)],
+                         ids=lambda t: "x".join(map(str, t)))
 def test_gemm_sparse48(mnk):
     """Every output, at sizes spanning several 128-row weight tiles, both activation tile widths
-    (128 for M <= 256, 256 above), ragged M and N, and several 512-wide K stages."""
+    (128 for M <= 256, 256 above), ragged M and N, and several 512-wide K stages; on tile images
+    also more pair tiles (80) than CTA pairs, so pairs reuse both TMEM accumulators."""
     _run(*mnk, seed=510 + sum(mnk))
 
 
@@ -129,11 +136,15 @@ def _sampled48(M, N, K, rows, d):
     Y, S = oracle.gemm(oracle.nvfp4_decode(xc, xs, xts, block=32), Wd)
     v, m = sp.prune_compress_48(to_dev(W, "bf16"))
     xq = sp.quantize_nvfp4_block32(to_dev(X, "bf16"))
-    y = sp.gemm_sparse48(xq, sp.Sparse48(sp.quantize_nvfp4(v), m), K)
+    w48 = sp.Sparse48(sp.quantize_nvfp4(v), m)
+    y = sp.gemm_sparse48(xq, w48, K)
+    y2 = sp.gemm_sparse48(sp.b32_to_mma(xq), sp.sparse48_to_mma(w48, K), K)
     torch.cuda.synchronize()
     assert sp.last_device_error() == sp.OK
     assert _bits32(xq.tensor_scale.item()) == _bits32(xts)
-    assert_gemm_close(y[torch.as_tensor(rows, device=y.device)], Y, S)
+    sel = torch.as_tensor(rows, device=y.device)
+    assert_gemm_close(y[sel], Y, S)
+    assert_gemm_close(y2[sel], Y, S)
 
 
 def test_prefill_4096_sampled():
@@ -148,3 +159,59 @@ def test_msweep_16384_sampled():
     rows = np.sort(synth.rng(79).choice(16384, 8, replace=False))
     d = {"X": synth.draw(synth.rng(16384), (16384, 5120), "bf16"), "W": synth.draw(synth.rng(0), (5120, 5120), "bf16")}
     _sampled48(16384, 5120, 5120, rows, d)
+
+
+def _tiles(a: np.ndarray, rows_pad: int, words: int) -> np.ndarray:
+    """Scale tiles from their definition: per 128-row block, `words` 4-byte groups per row, tile
+    (rb, w) holding row r's group w at byte 16 (r % 32) + 4 (r / 32)."""
+    rows = a.shape[0]
+    out = np.zeros(rows_pad // 128 * words * 512, dtype=np.uint8)
+    for r in range(rows):
+        rb, rr = divmod(r, 128)
+        for w in range(words):
+            base = (rb * words + w) * 512 + 16 * (rr % 32) + 4 * (rr // 32)
+            out[base:base + 4] = a[r, 4 * w:4 * w + 4]
+    return out
+
+
+def _code_image(c: np.ndarray, rows_pad: int) -> np.ndarray:
+    rows, half = c.shape
+    kc = half // 128
+    out = np.zeros(rows_pad // 128 * kc * 16384, dtype=np.uint8)
+    for r in range(rows):
+        rb, rr = divmod(r, 128)
+        for k in range(kc):
+            for p in range(8):
+                dst = (rb * kc + k) * 16384 + 128 * rr + 16 * (p ^ (rr % 8))
+                out[dst:dst + 16] = c[r, 128 * k + 16 * p:128 * k + 16 * p + 16]
+    return out
+
+
+@pytest.mark.parametrize("rows,K", [(1, 512), (130, 1024), (300, 512)])
+def test_pair_images_match_their_definition(rows, K):
+    """Tile images of a pairwise-4:8 weight (rows padded to 256, metadata padding 0x44) and of
+    block-32 activations, byte for byte against their definitions."""
+    g = synth.rng(rows + K)
+    vc = g.integers(0, 256, size=(rows, K // 4), dtype=np.uint8)
+    vs = g.integers(0, 256, size=(rows, K // 32), dtype=np.uint8)
+    mt = g.integers(0, 256, size=(rows, K // 16), dtype=np.uint8)
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    w = sp.Sparse48(sp.NVFP4Tensor(to_dev(vc, "u8"), to_dev(vs, "u8"), one), to_dev(mt.reshape(-1), "u8"))
+    im = sp.sparse48_to_mma(w, K)
+    rp = -(-rows // 256) * 256
+    meta_ref = np.full(rp // 128 * (K // 256) * 2048, 0x44, dtype=np.uint8)
+    for r in range(rows):
+        rb, rr = divmod(r, 128)
+        for t in range(K // 256):
+            dst = (rb * (K // 256) + t) * 2048 + 16 * rr
+            meta_ref[dst:dst + 16] = mt[r, 16 * t:16 * t + 16]
+    xc = g.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    xs = g.integers(0, 256, size=(rows, K // 32), dtype=np.uint8)
+    xi = sp.b32_to_mma(sp.NVFP4Tensor(to_dev(xc, "u8"), to_dev(xs, "u8"), one))
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(im.values), _code_image(vc, rp))
+    assert np.array_equal(to_host(im.scales), _tiles(vs, rp, K // 128))
+    assert np.array_equal(to_host(im.meta), meta_ref)
+    xp = -(-rows // 128) * 128
+    assert np.array_equal(to_host(xi.codes), _code_image(xc, xp))
+    assert np.array_equal(to_host(xi.scales), _tiles(xs, xp, K // 128))
