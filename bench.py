@@ -626,8 +626,19 @@ def sweep(emit, full: bool) -> None:
             us = timeit(fn, n)
             line[name] = record(us, flops, xbytes + wbytes + M * N * 4, pipe)
             line[name]["input_sets"] = n
-            del sets
+            # both forms again on the kernels' tile images (the CTA-pair kernels): the weight is
+            # rewritten once, the activations as a quantiser emitting images would leave them
+            if name == "dense":
+                isets = [(sp.to_mma(a), sp.to_mma(b)) for a, b in sets]
+                fn_i = lambda r: sp.gemm_dense(isets[r % n][0], isets[r % n][1], out=y)
+            else:
+                isets = [(sp.b32_to_mma(a), sp.sparse48_to_mma(b, K)) for a, b in sets]
+                fn_i = lambda r: sp.gemm_sparse48(isets[r % n][0], isets[r % n][1], K, out=y)
+            line[name + "_tile_images"] = record(timeit(fn_i, n), flops, xbytes + wbytes + M * N * 4, pipe)
+            del sets, isets
         line["sparse_dense_speedup"] = round(line["dense"]["us"] / line["sparse48"]["us"], 3)
+        line["sparse_dense_speedup_tile_images"] = round(
+            line["dense_tile_images"]["us"] / line["sparse48_tile_images"]["us"], 3)
         emit(line)
 
     # config 1: FP16 2:4 toy (L2-resident by size: a correctness configuration)
@@ -814,7 +825,17 @@ def per_config(lines: list) -> dict:
 
 
 def compute_roofline(lines: list):
-    """The config-3 dense W4A4 GEMM (4096^3) against the dense FP4 tensor peak."""
+    """The config-3 dense W4A4 GEMM (4096^3) against the dense FP4 tensor peak, with the
+    pairwise-4:8 sparse FP4 GEMM of the same shape against the sparse (dense-equivalent) peak."""
+    sparse = None
+    for ln in lines:
+        if ln.get("sweep") == "prefill_w4a4_pairwise48" and "sparse48_tile_images" in ln:
+            _, tp, src = tensor_peaks()
+            d = ln["sparse48_tile_images"]
+            sparse = {"kernel": "gemm_nvfp4_pair_kernel (sparse): tcgen05.mma.sp cta_group::2 kind::mxf4nvf4",
+                      "achieved": d["TFLOP/s"], "peak": round(tp["nvfp4.sp"], 1), "peak_kind": src["nvfp4.sp"],
+                      "frac": round(d["TFLOP/s"] / tp["nvfp4.sp"], 3), "launch_us": d["us"],
+                      "sparse_dense_speedup": ln.get("sparse_dense_speedup_tile_images")}
     for ln in lines:
         if ln.get("sweep") == "prefill_w4a4":
             d = ln.get("dense_tile_images", ln["dense"])
@@ -826,7 +847,7 @@ def compute_roofline(lines: list):
                     "unit": "TFLOP/s", "frac": round(d["TFLOP/s"] / tp["nvfp4"], 3), "launch_us": d["us"],
                     "row_order_operands_us": ln["dense"]["us"],
                     "mma_loop_tflops": {k: v for k, v in mma_microbench().items() if k.startswith("nvfp4")},
-                    "traffic": None}
+                    "sparse_pairwise48": sparse, "traffic": None}
     return None
 
 
