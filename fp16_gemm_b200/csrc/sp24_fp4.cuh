@@ -41,13 +41,17 @@ __device__ __forceinline__ uint32_t fp4_pair_i4(uint32_t w, int i) {
   return (shl2(w, P2<T>::MAGPOS - 4 * i) & P2<T>::MAG) | (shl2(w, 12 - 4 * i) & 0x80008000u);
 }
 
-// The byte at bits [8bb, 8bb+8) of w (two consecutive codes) -> 16-bit pair (lo, hi).
+// The byte at bits [8bb, 8bb+8) of w (two consecutive codes) -> 16-bit pair (lo, hi).  With the
+// byte alone in x, x * (2^P + 2^(P+12)) is x << P plus x << (P + 12), two copies whose bits do
+// not overlap, so the product places the low code's magnitude bits at P and the high code's at
+// P + 16 at once; x * (2^12 + 2^24) likewise moves the two sign bits (3, 7) to 15 and 31.  Two
+// integer multiplies and two masks instead of four shift-and-mask terms.
 template <typename T>
 __device__ __forceinline__ uint32_t fp4_pair_byte(uint32_t w, int bb) {
-  const uint32_t x = w >> (8 * bb);
+  const uint32_t x = __byte_perm(w, 0u, 0x4440u | (uint32_t)bb);  // byte bb, upper bytes zero
   constexpr int P = P2<T>::MAGPOS;
-  return ((x << P) & (7u << P)) | ((x << 12) & 0x8000u) | ((x << (P + 12)) & (7u << (P + 16))) |
-         ((x << 24) & 0x80000000u);
+  const uint32_t mag = (x * ((1u << P) | (1u << (P + 12)))) & P2<T>::MAG;
+  return mag | ((x * 0x01001000u) & 0x80008000u);
 }
 
 template <typename T>

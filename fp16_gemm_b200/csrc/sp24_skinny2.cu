@@ -917,12 +917,13 @@ __global__ void __launch_bounds__(kTileThreads, 1) decode_tile_kernel(const Skin
           const uint2 m1 = *reinterpret_cast<const uint2*>(me + r1 * tg.mb + 8 * v);
           const uint32_t sc0 = *reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 2 * v);
           const uint32_t sc1 = *reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 2 * v);
+          uint32_t s0w[2], s1w[2];  // both windows' scales of each row in one conversion
+          scale_pair<T>(sc0, s0w[0], s0w[1]);
+          scale_pair<T>(sc1, s1w[0], s1w[1]);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const uint32_t e = __byte_perm(u ? m0.y : m0.x, u ? m1.y : m1.x, (c & 1) ? 0x7632 : 0x5410);
-            uint32_t s0, s1, unused;
-            scale_pair<T>((sc0 >> (8 * u)) & 0xffu, s0, unused);
-            scale_pair<T>((sc1 >> (8 * u)) & 0xffu, s1, unused);
+            const uint32_t s0 = s0w[u], s1 = s1w[u];
             const uint32_t b0 = __byte_perm(u ? c0.z : c0.x, u ? c0.w : c0.y, c | ((c + 4) << 4));
             const uint32_t b1 = __byte_perm(u ? c1.z : c1.x, u ? c1.w : c1.y, c | ((c + 4) << 4));
             const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
