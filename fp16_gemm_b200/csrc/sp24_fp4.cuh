@@ -54,6 +54,37 @@ __device__ __forceinline__ uint32_t fp4_pair_byte(uint32_t w, int bb) {
   return mag | ((x * 0x01001000u) & 0x80008000u);
 }
 
+// Four bytes of E2M1 codes -> four f16 pairs (byte i -> ri; the low code of a byte in the low
+// half), by the sm_100a conversion instruction: every E2M1 value is exact in f16.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(w));
+}
+
+// The two low bytes of w -> two f16 pairs (byte 0 -> r0, byte 1 -> r1).
+__device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t& r0, uint32_t& r1) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t}"
+      : "=r"(r0), "=r"(r1)
+      : "r"(w));
+}
+
+// Two E4M3 codes (low bytes of code2) -> f16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t code2) {
+  uint32_t h2;
+  const uint16_t c = (uint16_t)code2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+  return h2;
+}
+
 template <typename T>
 __device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {

@@ -766,17 +766,33 @@ int launch_decode(const SkinnyParams& p, cudaStream_t s) {
 //
 // When there are at least as many 16-row tiles as SMs, each CTA owns a contiguous range of whole
 // tiles.  A tile's codes (and block scales, and 2:4 nibbles) over the full K are one contiguous
-// block of memory, so a producer thread fetches each with a single bulk copy into a ring of
-// tile buffers (bulk copies move data efficiently only in large requests), and x arrives as 8
-// bulk-copied rows padded by 16 bytes (so B-fragment reads of different tokens fall in
-// different banks).  16 consumer warps split each tile's K chunks round-robin, add their partial
-// sums into the tile's shared buffer, and release the buffer; at the end the CTA writes its
-// tiles' outputs with plain stores: every output has exactly one writer, so y needs no zeroing
-// and no atomics.  Rows sit unswizzled at a pitch that is a multiple of 128 bytes, so an A read
-// meets a 2-way bank conflict per 8-lane phase.
-constexpr int kTileWarps = 16;
-constexpr int kTileThreads = (kTileWarps + 1) * 32;  // + producer warp
+// block of memory, so thread 0 fetches each with a single bulk copy into a ring of tile slots
+// (bulk copies cost ~30 ns each to issue and move large requests at full speed; tensor copies of
+// narrow boxes do not), and x arrives first with one bulk copy of its M rows; the tile copies are
+// issued once x has landed, so x does not share the SM's inbound bandwidth with them.
+//
+// Warp w owns the K range [256 w, 256 w + 256) of every tile (K / 256 warps): its x fragments for
+// that range are loaded once, into registers, as f16.  bf16 x is converted as is when the warp's
+// largest |x| lies in [2^-8, 2^15) (f16 keeps bf16's 8 significant bits there; values below 2^-14
+// round to f16 subnormals, an error under 2^-25 against a maximum of at least 2^-8); otherwise it
+// is first multiplied by a power of two 2^S that brings the maximum into [2^14, 2^15), and the
+// warp's partial sums are multiplied back by 2^-S.  NVFP4 codes become f16 pairs by the sm_100a
+// conversion instruction (E2M1 exact in f16) times their E4M3 block scale (exact: at most five
+// significant bits, magnitudes at most 2688), and feed mma.m16n8k16 (dense) or mma.sp m16n8k32
+// (2:4) with fp32 accumulation; a measured loop of conversions, scale multiplies and MMAs runs as
+// fast as the MMAs alone.  Every warp adds its partial sums into the tile's shared buffer and
+// releases the slot; the CTA writes its tiles' outputs at the end with plain stores: every output
+// has exactly one writer, so y needs no zeroing and no atomics.
+//
+// Dense fragments: chunk j (128 entries at k0 = 256 w + 128 j): lane (g, c) holds the 32 codes
+// k0 + 32c .. +31 (two E4M3 blocks) of rows g and g + 8 in one 16-byte load each; MMA m of the
+// chunk takes codes k0 + 32c + 4m .. +3 (bytes 2m, 2m+1) and x[g][the same four entries].  2:4
+// fragments: window pair q = 4w + j: lane (g, c) supplies the kept pair of groups c and c+4 of each
+// 32-wide window, B = x[g][32v + 2c + 8i .. +1] for i = 0..3, and the nibbles as in the skinny
+// kernel above.
 constexpr int kTileMaxLocal = 32;
+constexpr int kTileMaxBuf = 4;
+constexpr int kTileKW = 256;  // K entries per warp
 
 template <int WF>
 struct TileGeom {
@@ -786,191 +802,262 @@ struct TileGeom {
   __host__ __device__ int64_t bytes() const { return 16 * (cb + sb + mb); }
 };
 
-// Dynamic shared memory: x (8 rows of 2K + 16 bytes), nbuf tile buffers, per-tile sums.
+// x row pitch in shared memory: 2K bytes plus 32 (dense) or 16 (2:4), so that the fragment loads
+// below are bank-conflict free.
 template <int WF>
-size_t tile_smem(int64_t K, int nbuf, int64_t local_tiles) {
-  return 8 * (size_t)(2 * K + 16) + (size_t)nbuf * TileGeom<WF>(K).bytes() + (size_t)local_tiles * 512;
+__host__ __device__ int64_t x_pitch(int64_t K) { return 2 * K + (WF == W_DQ4 ? 32 : 16); }
+
+// Dynamic shared memory: nbuf tile buffers, x (M padded rows), per-tile sums.
+template <int WF>
+size_t tile_smem(int64_t M, int64_t K, int nbuf, int64_t local_tiles) {
+  return (size_t)nbuf * TileGeom<WF>(K).bytes() + (size_t)M * (size_t)x_pitch<WF>(K) + (size_t)local_tiles * 512;
 }
 
-template <int WF, typename T, int NBUF>
-__global__ void __launch_bounds__(kTileThreads, 1) decode_tile_kernel(const SkinnyParams p) {
+// f16 pair <- bf16 pair times sf (a power of two), through f32 (the rounding only touches values
+// below f16's normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float sf) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16) * sf, __uint_as_float(w & 0xffff0000u) * sf);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Scale exponent S for a warp whose largest |x| has the bf16 magnitude bits m: 0 when m is 0,
+// infinite, NaN or in [2^-8, 2^15); else the S with max|x| 2^S in [2^14, 2^15).
+__device__ __forceinline__ int x_scale_exp(uint32_t m) {
+  if (m == 0 || m >= 0x7f80u || (m >= 0x3B80u && m < 0x4700u)) return 0;
+  const int e = (int)(m >> 7) - 127;  // subnormal: -127
+  const int s = 14 - e;
+  return s > 126 ? 126 : s;
+}
+
+template <int WF, typename T, int XI>
+__global__ void __launch_bounds__(640, 1) decode_tile_kernel(const SkinnyParams p, int nbuf) {
   extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ uint64_t full_bar[NBUF], empty_bar[NBUF], x_bar;
+  __shared__ uint64_t full_bar[kTileMaxBuf], empty_bar[kTileMaxBuf], x_bar;
   __shared__ int issued, abort_flag;
   const TileGeom<WF> tg(p.K);
-  const int64_t xp = 2 * p.K + 16;                       // padded x row
-  uint8_t* xs = dsm;
-  uint8_t* bufs = dsm + 8 * xp;
-  float* tbuf = reinterpret_cast<float*>(bufs + NBUF * tg.bytes());  // [local tile][16 rows][8 tokens]
+  uint8_t* bufs = dsm;
+  const int64_t xp = x_pitch<WF>(p.K);
+  const uint8_t* xs = bufs + nbuf * tg.bytes();                                 // x rows [M][xp]
+  float* tbuf = reinterpret_cast<float*>(bufs + nbuf * tg.bytes() + p.M * xp);  // [tile][16][8]
+  const int W = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT16 = (int)(p.N / 16);
   const int t0 = (int)((int64_t)NT16 * blockIdx.x / gridDim.x), t1 = (int)((int64_t)NT16 * (blockIdx.x + 1) / gridDim.x);
-  const int ntiles = t1 - t0;                             // >= 1 (host: T >= grid), <= kTileMaxLocal
+  const int ntiles = t1 - t0;  // >= 1 (host: tiles >= grid), <= kTileMaxLocal
+  // ---- copies: x (one row per copy, into padded rows), then each tile's codes / scales /
+  // nibbles, one bulk copy apiece, all issued by thread 0 as its first work; tile i goes to slot
+  // i % nbuf once the tile that held it has been released by every warp
+  auto issue_tile = [&](int i) {
+    const int sl = i % nbuf;
+    uint8_t* d = bufs + sl * tg.bytes();
+    const int64_t row = (int64_t)(t0 + i) * 16;
+    tc::mbar_arrive_expect_tx(&full_bar[sl], (uint32_t)tg.bytes());
+    stream::bulk_g2s(d, p.w + row * tg.cb, (uint32_t)(16 * tg.cb), &full_bar[sl]);
+    stream::bulk_g2s(d + 16 * tg.cb, p.w_scales + row * tg.sb, (uint32_t)(16 * tg.sb), &full_bar[sl]);
+    if (WF == W_SQ4) stream::bulk_g2s(d + 16 * (tg.cb + tg.sb), p.meta + row * tg.mb, (uint32_t)(16 * tg.mb), &full_bar[sl]);
+    issued = i + 1;
+  };
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBUF; ++i) {
-      tc::mbar_init(&full_bar[i], 1);
-      tc::mbar_init(&empty_bar[i], kTileWarps);
-    }
     tc::mbar_init(&x_bar, 1);
-    issued = 0;
+    for (int i = 0; i < nbuf; ++i) {
+      tc::mbar_init(&full_bar[i], 1);
+      tc::mbar_init(&empty_bar[i], W);
+    }
     abort_flag = 0;
+    issued = 0;
     tc::fence_mbar_init();
+    tc::mbar_arrive_expect_tx(&x_bar, (uint32_t)(p.M * 2 * p.K));
+    const uint8_t* xg = reinterpret_cast<const uint8_t*>(p.x);
+    for (int r = 0; r < p.M; ++r)
+      stream::bulk_g2s(const_cast<uint8_t*>(xs) + r * xp, xg + (int64_t)r * 2 * p.K, (uint32_t)(2 * p.K), &x_bar);
+    for (int i = 0; i < ntiles && i < nbuf; ++i) issue_tile(i);
   }
   for (int i = threadIdx.x; i < ntiles * 128; i += blockDim.x) tbuf[i] = 0.f;
-  // token rows past M: zeros
-  for (int i = threadIdx.x; i < (8 - p.M) * (int)(xp / 16); i += blockDim.x) {
-    const int r = p.M + i / (int)(xp / 16), j = i % (int)(xp / 16);
-    *reinterpret_cast<uint4*>(xs + r * xp + 16 * j) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  __syncthreads();
+  __syncthreads();  // barriers initialised, sums zeroed
 
-  if (warp == kTileWarps) {
-    // ---- producer: x rows, then each tile's codes / scales / nibbles, one bulk copy apiece
-    if (lane == 0) {
-      const uint8_t* xg = reinterpret_cast<const uint8_t*>(p.x);
-      tc::mbar_arrive_expect_tx(&x_bar, (uint32_t)(p.M * 2 * p.K));
-      for (int g = 0; g < p.M; ++g) stream::bulk_g2s(xs + g * xp, xg + (int64_t)g * 2 * p.K, (uint32_t)(2 * p.K), &x_bar);
-      int i = 0;
-      for (; i < ntiles; ++i) {
-        const int sl = i % NBUF;
-        if (!mbar_wait(&empty_bar[sl], ((i / NBUF) & 1) ^ 1)) {
-          set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-          abort_flag = 1;
-          break;
+  const int g = lane >> 2, c = lane & 3;
+  // every wait is decided warp-uniformly (the MMAs need the whole warp)
+  bool ok = __all_sync(0xffffffffu, mbar_wait(&x_bar, 0));
+  if (!ok && lane == 0) {
+    set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+    abort_flag = 1;
+  }
+  // x fragments of this warp's K range (token rows past M: zeros)
+  const int k0 = kTileKW * warp;
+  uint32_t xf[XI][16];
+  {
+    const uint8_t* xg = xs + (int64_t)g * xp;
+    const bool live = ok && g < p.M;
+#pragma unroll
+    for (int j = 0; j < XI; ++j) {
+      if constexpr (WF == W_DQ4) {
+        // load h takes piece (h + c / 2) % 4 of the lane's four 16-byte pieces: with the row
+        // pitch 32 bytes past a multiple of 128, the 8 lanes of each quarter-warp then read 8
+        // different bank groups; the pieces are put back in order after
+        uint4 v[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          v[h] = live ? *reinterpret_cast<const uint4*>(xg + 2 * (k0 + 128 * j + 32 * c) + 16 * ((h + (c >> 1)) & 3))
+                      : make_uint4(0u, 0u, 0u, 0u);
+        const bool rot = c >= 2;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint4 u = rot ? v[(h + 3) & 3] : v[h];
+          xf[j][4 * h] = u.x; xf[j][4 * h + 1] = u.y; xf[j][4 * h + 2] = u.z; xf[j][4 * h + 3] = u.w;
         }
-        uint8_t* d = bufs + sl * tg.bytes();
-        const int64_t row = (int64_t)(t0 + i) * 16;
-        tc::mbar_arrive_expect_tx(&full_bar[sl], (uint32_t)tg.bytes());
-        stream::bulk_g2s(d, p.w + row * tg.cb, (uint32_t)(16 * tg.cb), &full_bar[sl]);
-        stream::bulk_g2s(d + 16 * tg.cb, p.w_scales + row * tg.sb, (uint32_t)(16 * tg.sb), &full_bar[sl]);
-        if (WF == W_SQ4) stream::bulk_g2s(d + 16 * (tg.cb + tg.sb), p.meta + row * tg.mb, (uint32_t)(16 * tg.mb), &full_bar[sl]);
+      } else {
+        // window pairs 2j, 2j + 1 of the warp (windows 4j .. 4j + 3)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            xf[j][4 * u + t] = live ? *reinterpret_cast<const uint32_t*>(xg + 2 * (k0 + 32 * (4 * j + u) + 2 * c + 8 * t)) : 0u;
       }
-      issued = i;
     }
-  } else {
-    // ---- consumers: chunks (128 k dense, 32-k windows 2:4) of each tile, round-robin over warps
-    const int g = lane >> 2, c = lane & 3;
-    const int r0 = prow(g), r1 = prow(g + 8);
-    const uint8_t* x0 = xs + g * xp;  // this lane's token row
-    const int nq = WF == W_DQ4 ? (int)(p.K / 128) : (int)(p.K / 32);
-    bool ok = mbar_wait(&x_bar, 0);
-    if (!ok) {
-      set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-      abort_flag = 1;
-    }
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const int sl = i % NBUF;
-      if (!mbar_wait(&full_bar[sl], (i / NBUF) & 1)) {
+  }
+  float descale = 1.0f;  // 2^-S of x
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    __nv_bfloat162 mx = __floats2bfloat162_rn(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < XI; ++j)
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const uint32_t a = xf[j][t] & 0x7fff7fffu;
+        mx = __hmax2(mx, *reinterpret_cast<const __nv_bfloat162*>(&a));
+      }
+    const uint32_t mb2 = *reinterpret_cast<const uint32_t*>(&mx);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, max(mb2 & 0xffffu, mb2 >> 16));
+    const int S = x_scale_exp(m);
+    const float sf = __int_as_float((127 + S) << 23);
+    descale = __int_as_float((127 - S) << 23);
+#pragma unroll
+    for (int j = 0; j < XI; ++j)
+#pragma unroll
+      for (int t = 0; t < 16; ++t) xf[j][t] = bf16x2_to_f16x2(xf[j][t], sf);
+  }
+  const int r0 = g, r1 = g + 8;
+  for (int i = 0; ok && i < ntiles; ++i) {
+    const int sl = i % nbuf;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[sl], (i / nbuf) & 1))) {
+      if (lane == 0) {
         set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
         abort_flag = 1;
-        break;
       }
-      const uint8_t* d = bufs + sl * tg.bytes();
-      const uint8_t* sc = d + 16 * tg.cb;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+      break;
+    }
+    const uint8_t* d = bufs + sl * tg.bytes();
+    const uint8_t* sc = d + 16 * tg.cb;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < XI; ++j) {
+      float(&a)[4] = (j & 1) ? acc2 : acc;
       if constexpr (WF == W_DQ4) {
-        // chunks q and q + 16 of a warp are decoded step by step into two accumulator chains
-        for (int q = warp; q < nq; q += 2 * kTileWarps) {
-          const bool two = q + kTileWarps < nq;
-          uint32_t w0[2][4], w1[2][4], sa[2][2], sb[2][2];
+        const int kb = (k0 + 128 * j + 32 * c) / 2;  // byte of the lane's codes in a row
+        const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + kb);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + kb);
+        const int sbk = (k0 + 128 * j + 32 * c) / 16;
+        const uint32_t h0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + sbk));
+        const uint32_t h1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + sbk));
+        const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qc = u && two ? q + kTileWarps : q;  // a missing second chunk repeats the first, unused
-            const uint4 v0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 64 * qc + 16 * c);
-            const uint4 v1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 64 * qc + 16 * c);
-            w0[u][0] = v0.x; w0[u][1] = v0.y; w0[u][2] = v0.z; w0[u][3] = v0.w;
-            w1[u][0] = v1.x; w1[u][1] = v1.y; w1[u][2] = v1.z; w1[u][3] = v1.w;
-            scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 8 * qc + 2 * c), sa[u][0], sa[u][1]);
-            scale_pair<T>(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 8 * qc + 2 * c), sb[u][0], sb[u][1]);
-          }
+        for (int hb = 0; hb < 2; ++hb) {  // E4M3 block hb: MMAs 4 hb .. 4 hb + 3
+          const uint32_t s0 = __byte_perm(h0, 0u, hb ? 0x3232 : 0x1010), s1 = __byte_perm(h1, 0u, hb ? 0x3232 : 0x1010);
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
+          for (int ww = 0; ww < 2; ++ww) {  // word 2 hb + ww: MMAs 4 hb + 2 ww, +1
+            uint32_t c0[4], c1[4];
+            e2m1x8_to_f16x2(w0[2 * hb + ww], c0[0], c0[1], c0[2], c0[3]);
+            e2m1x8_to_f16x2(w1[2 * hb + ww], c1[0], c1[1], c1[2], c1[3]);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              if (u && !two) continue;
-              const int qc = u ? q + kTileWarps : q;
-              // x[g][P .. P+8), P = 128 qc + 32c + 8qq: codes at nibbles (i, i+4) of word qq pair
-              // with x entries (i, i+4)
-              const uint4 xv = *reinterpret_cast<const uint4*>(x0 + 2 * (128 * qc + 32 * c + 8 * qq));
-              const uint32_t s0 = sa[u][qq >> 1], s1 = sb[u][qq >> 1];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const uint32_t xa = h ? xv.y : xv.x, xb = h ? xv.w : xv.z;
-                const uint2 bx = make_uint2(__byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632));
-                const uint32_t a0 = hmul2u<T>(fp4_pair_i4<T>(w0[u][qq], 2 * h), s0);
-                const uint32_t a2 = hmul2u<T>(fp4_pair_i4<T>(w0[u][qq], 2 * h + 1), s0);
-                const uint32_t a1 = hmul2u<T>(fp4_pair_i4<T>(w1[u][qq], 2 * h), s1);
-                const uint32_t a3 = hmul2u<T>(fp4_pair_i4<T>(w1[u][qq], 2 * h + 1), s1);
-                mma_k16<T>(u ? acc2 : acc, a0, a1, a2, a3, bx);
-              }
+            for (int mm = 0; mm < 2; ++mm) {
+              const int m = 4 * hb + 2 * ww + mm;
+              mma_k16<__half>(a, hmul2u<__half>(c0[2 * mm], s0), hmul2u<__half>(c1[2 * mm], s1),
+                              hmul2u<__half>(c0[2 * mm + 1], s0), hmul2u<__half>(c1[2 * mm + 1], s1),
+                              make_uint2(xf[j][2 * m], xf[j][2 * m + 1]));
             }
           }
         }
       } else {
-        // window pairs (2v, 2v + 1): 16 bytes of codes and 8 of nibbles per row in one load each,
-        // the two windows into two accumulator chains
         const uint8_t* me = sc + 16 * tg.sb;
-        for (int v = warp; 2 * v < nq; v += kTileWarps) {
-          const uint4 c0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 16 * v);
-          const uint4 c1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 16 * v);
-          const uint2 m0 = *reinterpret_cast<const uint2*>(me + r0 * tg.mb + 8 * v);
-          const uint2 m1 = *reinterpret_cast<const uint2*>(me + r1 * tg.mb + 8 * v);
-          const uint32_t sc0 = *reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 2 * v);
-          const uint32_t sc1 = *reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 2 * v);
-          uint32_t s0w[2], s1w[2];  // both windows' scales of each row in one conversion
-          scale_pair<T>(sc0, s0w[0], s0w[1]);
-          scale_pair<T>(sc1, s1w[0], s1w[1]);
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {  // window pair q = 4w + 2j + pp
+          const int q = 4 * warp + 2 * j + pp;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 16 * q);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 16 * q);
+          const uint2 m0 = *reinterpret_cast<const uint2*>(me + r0 * tg.mb + 8 * q);
+          const uint2 m1 = *reinterpret_cast<const uint2*>(me + r1 * tg.mb + 8 * q);
+          const uint32_t h0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 2 * q));
+          const uint32_t h1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 2 * q));
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const uint32_t e = __byte_perm(u ? m0.y : m0.x, u ? m1.y : m1.x, (c & 1) ? 0x7632 : 0x5410);
-            const uint32_t s0 = s0w[u], s1 = s1w[u];
+            const uint32_t s0 = __byte_perm(h0, 0u, u ? 0x3232 : 0x1010), s1 = __byte_perm(h1, 0u, u ? 0x3232 : 0x1010);
             const uint32_t b0 = __byte_perm(u ? c0.z : c0.x, u ? c0.w : c0.y, c | ((c + 4) << 4));
             const uint32_t b1 = __byte_perm(u ? c1.z : c1.x, u ? c1.w : c1.y, c | ((c + 4) << 4));
-            const uint32_t a0 = hmul2u<T>(fp4_pair_byte<T>(b0, 0), s0);
-            const uint32_t a2 = hmul2u<T>(fp4_pair_byte<T>(b0, 1), s0);
-            const uint32_t a1 = hmul2u<T>(fp4_pair_byte<T>(b1, 0), s1);
-            const uint32_t a3 = hmul2u<T>(fp4_pair_byte<T>(b1, 1), s1);
-            // x[g][32w + 2c + 8i + {0, 1}], i = 0..3, w = 2v + u
-            const uint8_t* xr = x0 + 2 * (32 * (2 * v + u)) + 4 * c;
-            const uint4 bx = make_uint4(*reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 16),
-                                        *reinterpret_cast<const uint32_t*>(xr + 32), *reinterpret_cast<const uint32_t*>(xr + 48));
-            mma_sp_k32<T>(u ? acc2 : acc, a0, a1, a2, a3, bx, e);
+            uint32_t a0, a2, a1, a3;
+            e2m1x4_to_f16x2(b0, a0, a2);
+            e2m1x4_to_f16x2(b1, a1, a3);
+            const int v = 2 * pp + u;  // window of the j-th group of four
+            mma_sp_k32<__half>(a, hmul2u<__half>(a0, s0), hmul2u<__half>(a1, s1), hmul2u<__half>(a2, s0),
+                               hmul2u<__half>(a3, s1),
+                               make_uint4(xf[j][4 * v], xf[j][4 * v + 1], xf[j][4 * v + 2], xf[j][4 * v + 3]), e);
           }
         }
       }
-      float* b = tbuf + i * 128;
-      atomicAdd(b + r0 * 8 + 2 * c, acc[0] + acc2[0]);
-      atomicAdd(b + r0 * 8 + 2 * c + 1, acc[1] + acc2[1]);
-      atomicAdd(b + r1 * 8 + 2 * c, acc[2] + acc2[2]);
-      atomicAdd(b + r1 * 8 + 2 * c + 1, acc[3] + acc2[3]);
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
+    }
+    float* bt = tbuf + i * 128;
+    atomicAdd(bt + r0 * 8 + 2 * c, (acc[0] + acc2[0]) * descale);
+    atomicAdd(bt + r0 * 8 + 2 * c + 1, (acc[1] + acc2[1]) * descale);
+    atomicAdd(bt + r1 * 8 + 2 * c, (acc[2] + acc2[2]) * descale);
+    atomicAdd(bt + r1 * 8 + 2 * c + 1, (acc[3] + acc2[3]) * descale);
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&empty_bar[sl]);
+    if (warp == 0 && i + nbuf < ntiles) {
+      int released = 1;
+      if (lane == 0) {
+        released = mbar_wait(&empty_bar[sl], (i / nbuf) & 1) ? 1 : 0;
+        if (released) {
+          issue_tile(i + nbuf);
+        } else {
+          set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
+          abort_flag = 1;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, released, 0)) break;
     }
   }
   __syncthreads();
   // a gave-up wait may leave copies in flight: let them land before the CTA's memory goes away
-  if (abort_flag && threadIdx.x == kTileWarps * 32) {
+  if (abort_flag && threadIdx.x == 0) {
     tc::mbar_wait(&x_bar, 0);
-    for (int i = issued > NBUF ? issued - NBUF : 0; i < issued; ++i) tc::mbar_wait(&full_bar[i % NBUF], (i / NBUF) & 1);
+    for (int i = issued > nbuf ? issued - nbuf : 0; i < issued; ++i) tc::mbar_wait(&full_bar[i % nbuf], (i / nbuf) & 1);
   }
   // ---- the CTA's tiles into y, one writer per output
-  const float scale = 256.0f * *p.w_ts;
+  const float scale = *p.w_ts;
   for (int e = threadIdx.x; e < ntiles * 128; e += blockDim.x) {
     const int lt = e >> 7, row = (e >> 3) & 15, tok = e & 7;
     if (tok < p.M) p.y[(int64_t)tok * p.N + (int64_t)(t0 + lt) * 16 + row] = tbuf[e] * scale;
   }
 }
 
+// Tile slots: as many as fit beside x and the per-tile sums, up to kTileMaxBuf.
+template <int WF>
+int tile_buffers(int64_t M, int64_t K, int64_t local) {
+  int nbuf = kTileMaxBuf;
+  while (nbuf >= 2 && tile_smem<WF>(M, K, nbuf, local) > 227 * 1024 - 1024) --nbuf;
+  return nbuf;
+}
+
 template <int WF, typename T>
 int launch_tile(const SkinnyParams& p, cudaStream_t s) {
   const int grid = sm_count();
   const int64_t T16 = p.N / 16, local = (T16 + grid - 1) / grid;
-  const bool three = tile_smem<WF>(p.K, 3, local) <= 227 * 1024 - 256;
-  const size_t smem = tile_smem<WF>(p.K, three ? 3 : 2, local);
-  auto kern = three ? decode_tile_kernel<WF, T, 3> : decode_tile_kernel<WF, T, 2>;
+  const int nbuf = tile_buffers<WF>(p.M, p.K, local);
+  const size_t smem = tile_smem<WF>(p.M, p.K, nbuf, local);
+  const int warps = (int)(p.K / kTileKW);
+  auto kern = decode_tile_kernel<WF, T, 2>;  // two 128-entry chunks (dense) / two window-pair groups (2:4)
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SP24_ERR_CUDA;
-  kern<<<grid, kTileThreads, smem, s>>>(p);
+  kern<<<grid, warps * 32, smem, s>>>(p, nbuf);
   return launch_status();
 }
 
@@ -1009,17 +1096,16 @@ bool decode_supported(int wf, const SkinnyParams& p) {
 }
 
 // True when the whole-tile decode kernel takes the problem: 16-bit x of at most 8 tokens,
-// NVFP4 weights (dense: K % 128; 2:4: K % 64) with at least one 16-row tile per SM and at most
-// kTileMaxLocal tiles per CTA, 16-byte aligned operands, and x plus two tile buffers in shared
-// memory.
+// NVFP4 weights (dense or 2:4) with K a multiple of 256 up to 5120 (one warp per 256 entries of
+// K, at most 20 warps), at least one 16-row tile per SM and at most kTileMaxLocal tiles per CTA,
+// 16-byte aligned operands, and x plus two tile buffers in shared memory.
 bool decode_tile_supported(int wf, const SkinnyParams& p) {
-  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0) return false;
+  if (p.x_fmt != X_16 || p.M > 8 || p.M < 1 || p.N % 16 || p.K == 0 || p.K % kTileKW || p.K > 20 * kTileKW) return false;
   if (!aligned(p.x, 16) || !aligned(p.w, 16) || !aligned(p.w_scales, 16) || !aligned(p.y, 4)) return false;
   const int64_t T16 = p.N / 16, grid = sm_count(), local = (T16 + grid - 1) / grid;
   if (T16 < grid || local > kTileMaxLocal) return false;
-  if (wf == W_DQ4) return p.K % 128 == 0 && tile_smem<W_DQ4>(p.K, 2, local) <= 227 * 1024 - 256;
-  if (wf == W_SQ4)
-    return p.K % 64 == 0 && aligned(p.meta, 16) && tile_smem<W_SQ4>(p.K, 2, local) <= 227 * 1024 - 256;
+  if (wf == W_DQ4) return tile_smem<W_DQ4>(p.M, p.K, 2, local) <= 227 * 1024 - 1024;
+  if (wf == W_SQ4) return aligned(p.meta, 16) && tile_smem<W_SQ4>(p.M, p.K, 2, local) <= 227 * 1024 - 1024;
   return false;
 }
 

@@ -3,6 +3,7 @@ or 2:4) against the oracle's fp64 GEMM, on shapes that stress how it splits work
 weight units shared between neighbouring CTAs, many tiles per CTA (short K), fewer than 8
 tokens (the missing token rows of x read as zeros), K at the kernel's limit (8192), and fewer
 units than SMs.  Also checks that the skinny and decode paths agree with each other."""
+import numpy as np
 import pytest
 import torch
 
@@ -19,6 +20,8 @@ DECODE_SHAPES = [
     (8, 48, 8192),     # largest K: x fills 128 KB of shared memory; fewer units than SMs
     (5, 16, 512),      # a single tile
     (8, 4096, 4608),   # 18 / 9 units per tile
+    (3, 2560, 2048),   # 3 tokens on the whole-tile kernel (160 tiles)
+    (8, 4736, 7168),   # K above the whole-tile kernel's 5120: the k-group decode kernel
 ]
 
 
@@ -30,6 +33,22 @@ def test_decode_gemv_parity(shape, xdt, sparse):
     X, xs, W, ws = make_case(xdt, "nvfp4", M, N, K, seed=M * 7919 + N * 31 + K, w_sigma=0.02)
     Y, S = oracle_side(X, xs, xdt, W, ws, "nvfp4", sparse)
     y = gpu_side(X, xs, xdt, W, ws, "nvfp4", sparse)
+    assert_gemm_close(y, Y, S)
+    assert sp.last_device_error() == sp.OK
+
+
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse24"])
+@pytest.mark.parametrize("shift", [-100, 60])
+def test_decode_tile_bf16_far_from_unit_range(shift, sparse):
+    """bf16 x times 2^shift (every value still a normal bf16 number, far outside f16's range):
+    the whole-tile kernel runs its MMAs in f16 on x times a power of two that each warp picks
+    for its K range, so the result still meets the oracle's tolerance at both ends."""
+    M, N, K = 8, 2560, 1024
+    X, xs, W, ws = make_case("bf16", "nvfp4", M, N, K, seed=4242 + shift, w_sigma=0.02)
+    f = (X.astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** shift)
+    X = (f.view(np.uint32) >> 16).astype(np.uint16)
+    Y, S = oracle_side(X, xs, "bf16", W, ws, "nvfp4", sparse)
+    y = gpu_side(X, xs, "bf16", W, ws, "nvfp4", sparse)
     assert_gemm_close(y, Y, S)
     assert sp.last_device_error() == sp.OK
 
