@@ -79,7 +79,7 @@ __device__ __forceinline__ uint32_t e2m1x2_rne_satfinite(float x_lo, float x_hi)
 }
 
 // Streaming ring: 3 stages of 16 KB per CTA (512 blocks of 16 16-bit entries, or 256 fp32).
-constexpr int kChunk = 16384, kStages = 3;  // 48 KB per CTA: four CTAs per SM
+constexpr int kChunk = 16384, kStages = 2;  // 32 KB per CTA (+ 8 KB of threshold tables): four CTAs per SM
 constexpr size_t kRingBytes = (size_t)kChunk * kStages;
 
 // 16 entries of a block from shared memory as fp32.
@@ -219,7 +219,7 @@ template <int DT>
 struct Pack16;
 template <>
 struct Pack16<SP24_BF16> {
-  static constexpr uint32_t BIAS = 0x43004300u;  // 128.0 twice: 128 + k has k in its low bits
+  static constexpr uint32_t BIAS = 0x43004300u;  // 128.0 twice: 128 + k has k in its low byte
   static constexpr uint32_t QNAN = 0x7FC07FC0u;
 };
 template <>
@@ -291,15 +291,24 @@ __device__ __forceinline__ void encode_block16(const uint8_t* p, const uint32_t*
   const uint4 t0 = reinterpret_cast<const uint4*>(tab + 8 * sb)[0];
   const uint4 t1 = reinterpret_cast<const uint4*>(tab + 8 * sb)[1];
   const uint32_t th[7] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z};
-  uint32_t packed[2] = {0u, 0u};
+  // per pair of entries: the count starts at BIAS plus 8 for a negative entry, so the low byte of
+  // each half ends as the entry's 4-bit code (sign << 3 | magnitude code)
+  uint32_t nib[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    uint32_t acc = Pack16<DT>::BIAS;
+    uint32_t acc = ((w[i] >> 12) & 0x00080008u) | Pack16<DT>::BIAS;
 #pragma unroll
     for (int j = 0; j < 7; ++j) acc = add2<DT>(acc, ge2<DT>(a[i], th[j]));
-    // codes in bits 0-2 and 16-18, signs of the two entries to bits 3 and 19
-    const uint32_t x = (acc & 0x00070007u) | ((w[i] >> 12) & 0x00080008u);
-    packed[i >> 2] |= ((x | (x >> 12)) & 0xffu) << (8 * (i & 3));
+    nib[i] = acc;
+  }
+  // four pairs per code word: gather the low bytes of both halves, fold each byte pair into one
+  // byte (high entry in the high nibble), gather again
+  uint32_t packed[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t p0 = __byte_perm(nib[4 * k], nib[4 * k + 1], 0x6420);
+    const uint32_t p1 = __byte_perm(nib[4 * k + 2], nib[4 * k + 3], 0x6420);
+    packed[k] = __byte_perm(p0 | (p0 >> 4), p1 | (p1 >> 4), 0x6420);
   }
   codes[b] = make_uint2(packed[0], packed[1]);
   scales[b] = (uint8_t)sb;
