@@ -124,6 +124,8 @@ def lib() -> ctypes.CDLL:
             L.sp24_nvfp4_b32_mma_size.argtypes = [I64, I64, P, P]
             L.sp24_nvfp4_b32_to_mma.argtypes = [P, P, I64, I64, P, P, P]
             L.sp24_sparse48_mma_size.argtypes = [I64, I64, P, P, P]
+            L.sp24_prepare_sparse_size.argtypes = [I64, I64, P]
+            L.sp24_prepare_sparse.argtypes = [P, I64, I64, P, P]
             L.sp24_sparse48_to_mma.argtypes = [P, P, P, I64, I64, P, P, P, P]
             L.sp24_peak_mma.argtypes = [I, I, P, P]
             L.sp24_peak_ctas.argtypes = [I]
@@ -600,6 +602,16 @@ def sparse48_to_mma(w: Sparse48, K: int, stream=None) -> Sparse48MMA:
     _call("sp24_sparse48_to_mma", _ptr(v.codes), _ptr(v.scales), _ptr(w.meta), rows, K, _ptr(vo), _ptr(so), _ptr(mo),
           _stream(stream))
     return Sparse48MMA(vo, so, mo, v.tensor_scale, rows, K)
+
+
+def prepare_sparse(meta: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:
+    """The 2:4 nibble stream of a [rows, K] weight in the tensor cores' metadata layout
+    (sp24_prepare_sparse): uint8 tiles of 2 KB per 128 rows and 128 K, rows padded to 256."""
+    n = ctypes.c_int64(0)
+    _call("sp24_prepare_sparse_size", rows, K, ctypes.byref(n))
+    out = torch.empty(n.value, dtype=torch.uint8, device=meta.device)
+    _call("sp24_prepare_sparse", _ptr(meta), rows, K, _ptr(out), _stream(stream))
+    return out
 
 
 def b32_to_mma(q: NVFP4Tensor, stream=None) -> NVFP4MMA:

@@ -97,6 +97,7 @@ int64_t tiled_workspace(int x_fmt, int wf, int64_t M, int64_t N, int64_t K) {
   int64_t b = 0;
   if (native_sparse(wf, K)) {
     if (wf == W_SQ4) b += round256(N * K);  // N x K/2 values of 2 bytes
+    b += round256(meta_image_bytes(N, K));  // the metadata in the tcgen05 layout
   } else if (wf != W_D16) {
     b += round256(N * K * 2);
   }
@@ -169,10 +170,17 @@ int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes
                         reinterpret_cast<uint16_t*>(cur), s);
     if (st) return st;
     x16 = cur;
+    cur += round256(p.M * p.K * 2);
   }
   const float* sa = (wf == W_DQ4 || wf == W_SQ4) ? p.w_ts : nullptr;
   const float* sb = p.x_fmt == X_Q4 ? p.x_ts : nullptr;
-  if (sp_native) return tc_gemm_f16_sparse(x16, w16, p.meta, p.M, p.N, p.K, bf, p.y, sa, sb, s);
+  if (sp_native) {
+    // the nibble stream rewritten as tcgen05 metadata tiles, then the CTA-pair 2:4 kernel
+    int st = meta_to_image(p.meta, p.N, p.K, cur, s);
+    if (st) return st;
+    return tc_gemm_f16_pair(x16, w16, cur, p.M, p.N, p.K, bf, p.y, sa, sb, s, 0);
+  }
+  if (p.K % 64 == 0) return tc_gemm_f16_pair(x16, w16, nullptr, p.M, p.N, p.K, bf, p.y, sa, sb, s, 0);
   return tc_gemm_f16(x16, w16, p.M, p.N, p.K, bf, p.y, sa, sb, s);
 }
 

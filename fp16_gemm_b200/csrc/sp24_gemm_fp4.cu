@@ -475,6 +475,8 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+}  // namespace
+
 using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
 
 int tmap_encoder(EncodeFn* out) {
@@ -523,6 +525,8 @@ int make_tmap_y(CUtensorMap* map, float* y, int64_t M, int64_t N) {
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SP24_OK : SP24_ERR_CUDA;
 }
+
+namespace {
 
 template <int BN, bool TMA_Y, bool SP>
 int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa, const CUtensorMap& sb,

@@ -1,4 +1,7 @@
-// a4 / a5 at prefill-sized M: tensor-core GEMM on tcgen05 (kind::f16), TMA-fed, TMEM accumulator.
+// a4 at prefill-sized M, single-CTA form: tensor-core GEMM on tcgen05 (kind::f16), TMA-fed, TMEM
+// accumulator, for K that is not a multiple of 64 (the CTA-pair kernel of sp24_gemm_f16pair.cu
+// takes every other 16-bit shape, dense and 2:4); also the tensor-map helpers, the sparse FP4
+// kernel for pairwise-4:8 weights and the NVFP4 -> 16-bit expansion.
 //
 // [P1] "NVFP4 vs 2:4 sparse: where the other half of the petaflop went", "The roofline is the
 // whole argument": past the ridge point the product is bound by the tensor pipe, so this path
@@ -16,9 +19,9 @@
 // MMA warp frees a stage with tcgen05.commit.  Every wait is bounded: when one runs out the
 // kernel records SP24_ERR_DEVICE_TIMEOUT and unwinds.
 //
-// NVFP4 and 2:4-compressed weights reach this path through an expansion kernel that writes the
-// exact 16-bit values E2M1 * E4M3 (and zeros for pruned entries) into a workspace; the tensor
-// scales are applied in the epilogue.
+// NVFP4 and 2:4-compressed NVFP4 weights reach the 16-bit kernels through an expansion kernel
+// that writes the exact 16-bit values E2M1 * E4M3 (and, for a dense expansion, zeros for pruned
+// entries) into a workspace; the tensor scales are applied in the epilogue.
 #include <cudaTypedefs.h>
 
 #include "sp24_tc.cuh"
@@ -209,171 +212,6 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, c
   dim3 grid((p.N + kBM - 1) / kBM, (p.M + BN - 1) / BN);
   kern<<<grid, 192, smem, s>>>(ta, tb, p);
   return launch_status();
-}
-
-// ------------------------------------------------------------------ 2:4 sparse tcgen05 GEMM
-//
-// [P2] "The mechanism needs both values and their positions": the kept values are the A operand
-// (128 rows x 64 stored values = 128 logical K per stage) and the positions travel as metadata
-// in TMEM.  Per stage the producer also loads the 16 nibble-stream bytes of each of the 128
-// rows; warp 6 rewrites them into the tcgen05 metadata layout (TMEM lane l holds, for rows
-// m = 16*(l/16) + l%8 and m + 8, the nibbles of groups 4*((l/8)%2) .. +3 of each 32-wide K
-// window, one 32-bit column per window: the low half for row m, the high half for row m + 8),
-// the MMA thread moves that 2 KB tile into 4 TMEM columns with tcgen05.cp and issues four
-// tcgen05.mma.sp (K = 32 logical each) on it.
-constexpr int kSpBN = 128, kSpStages = 4;
-constexpr uint32_t kSpA = kBM * 128;           // 128 rows x 64 stored 16-bit values
-constexpr uint32_t kSpB = kSpBN * 128;         // one 64-wide K half of B (two per stage)
-constexpr uint32_t kSpM = kBM * 16;            // raw nibble rows (16 B each)
-constexpr uint32_t kSpStage = kSpA + 2 * kSpB + 2 * kSpM;
-constexpr size_t kSpSmem = (size_t)kSpStages * kSpStage + 1024;
-constexpr int kSpCols = 256;                   // TMEM: 128 accumulator + 16 metadata columns
-
-template <bool BF16>
-__global__ void __launch_bounds__(224, 1)
-    gemm_f16sp_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmE, const TcParams p) {
-  constexpr int S = kSpStages, BN = kSpBN;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = tc::align1024(smem_raw);
-  // stage s: [A 16 KB][B0 16 KB][B1 16 KB][raw nibbles 2 KB][tcgen05 metadata 2 KB]
-  auto sA = [&](int s) { return smem + s * kSpStage; };
-  auto sB = [&](int s, int h) { return smem + s * kSpStage + kSpA + h * kSpB; };
-  auto sMr = [&](int s) { return smem + s * kSpStage + kSpA + 2 * kSpB; };
-  auto sMe = [&](int s) { return smem + s * kSpStage + kSpA + 2 * kSpB + kSpM; };
-  __shared__ uint64_t full_bar[S], meta_bar[S], empty_bar[S], tfull_bar;
-  __shared__ uint32_t tmem_base;
-  __shared__ int aborted;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int n0 = blockIdx.y * BN;
-  const int KB = (p.K + 127) / 128;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&meta_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    mbar_init(&tfull_bar, 1);
-    aborted = 0;
-    fence_mbar_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmE);
-  }
-  if (warp == 1) tmem_alloc(&tmem_base, kSpCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1) || *(volatile int*)&aborted) {
-          aborted = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full_bar[s], kSpA + 2 * kSpB + kSpM);
-        tma_load_2d(sA(s), &tmA, &full_bar[s], kb * 64, m0);        // stored values
-        tma_load_2d(sB(s, 0), &tmB, &full_bar[s], kb * 128, n0);     // logical K [0, 64)
-        tma_load_2d(sB(s, 1), &tmB, &full_bar[s], kb * 128 + 64, n0);
-        tma_load_2d(sMr(s), &tmE, &full_bar[s], kb * 16, m0);        // 16 nibble bytes per row
-        ++issued;
-      }
-      for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
-        mbar_wait(&full_bar[kb % S], (kb / S) & 1);
-    }
-  } else if (warp == 6) {
-    // metadata rewrite: lane handles TMEM lanes l = lane + 32 i
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % S;
-      const uint32_t ph = (kb / S) & 1;
-      if (!mbar_wait(&full_bar[s], ph) || *(volatile int*)&aborted) {
-        aborted = 1;
-        break;
-      }
-      const uint8_t* raw = sMr(s);
-      uint8_t* out = sMe(s);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int l = lane + 32 * i;
-        const int m = 16 * (l / 16) + (l % 8), half = (l / 8) % 2;
-        const uint4 lo = *reinterpret_cast<const uint4*>(raw + 16 * m);        // row m, 16 bytes
-        const uint4 hi = *reinterpret_cast<const uint4*>(raw + 16 * (m + 8));  // row m + 8
-        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)  // window t: bytes 4t + 2*half (+1) of each row
-          o[t] = __byte_perm(wl[t], wh[t], half ? 0x7632 : 0x5410);
-        *reinterpret_cast<uint4*>(out + 16 * l) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&meta_bar[s]);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16(kBM, BN, BF16, true);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&full_bar[s], ph) || !mbar_wait(&meta_bar[s], ph) || *(volatile int*)&aborted) {
-          aborted = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t ecol = tmem + BN + 4 * s;
-        tmem_cp_128x128b(ecol, desc_rows16_noswizzle(smem_u32(sMe(s))));
-        const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA(s)));
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {  // K window t: A + 32 B, B half t/2 + 64 B * (t%2)
-          const uint64_t b = desc_kmajor_sw128(smem_u32(sB(s, t >> 1))) + 4 * (t & 1);
-          // the metadata address must be even: an odd column is named by the even one below
-          // it plus the descriptor's sparse-id2 field
-          const uint32_t e = ecol + t;
-          umma_f16_sp(tmem, a0 + 2 * t, b, e & ~1u, idesc | (e & 1u), (kb | t) != 0);
-        }
-        umma_commit(&empty_bar[s]);
-      }
-      umma_commit(&tfull_bar);
-    }
-  } else {
-    const int q = warp & 3;
-    const int row = m0 + 32 * q + lane;
-    if (!mbar_wait(&tfull_bar, 0)) {
-      aborted = 1;
-    } else {
-      tc_fence_after();
-      float scale = 1.0f;
-      if (p.scale_a) scale *= *p.scale_a;
-      if (p.scale_b) scale *= *p.scale_b;
-#pragma unroll 1
-      for (int j = 0; j < BN / 32; ++j) {
-        float v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * j, v);
-        if (row < p.N) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int tok = n0 + 32 * j + i;
-            if (tok < p.M) p.y[(int64_t)tok * p.N + row] = v[i] * scale;
-          }
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0 && aborted) set_dev_error(SP24_ERR_DEVICE_TIMEOUT);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kSpCols);
-  }
 }
 
 // ------------------------------------------------------------------ scale tiles for the sparse FP4 MMA
@@ -652,28 +490,6 @@ __global__ void __launch_bounds__(256) expand_w16_kernel(const uint8_t* __restri
 }
 
 }  // namespace
-
-// Native 2:4 tensor-core GEMM on 16-bit kept values: y = (*sa)(*sb) x w^T with w given by
-// values [N, K/2] and its nibble stream [N, K/8].  Needs K % 128 == 0 (16-byte nibble rows).
-int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, int64_t M, int64_t N,
-                       int64_t K, bool bf16, float* y, const float* scale_a, const float* scale_b,
-                       cudaStream_t s) {
-  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || K % 128) return SP24_ERR_UNSUPPORTED;
-  CUtensorMap ta, tb, te;
-  int st = make_tmap_2d(&ta, values, 2, N, K / 2, K, 64, kBM);
-  if (st) return st;
-  st = make_tmap_2d(&tb, x, 2, M, K, K * 2, 64, kSpBN);
-  if (st) return st;
-  st = make_tmap_2d_plain(&te, meta, N, K / 8, K / 8, 16, kBM);
-  if (st) return st;
-  TcParams p{(int)M, (int)N, (int)K, y, scale_a, scale_b};
-  auto kern = bf16 ? gemm_f16sp_tc_kernel<true> : gemm_f16sp_tc_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpSmem) != cudaSuccess)
-    return SP24_ERR_CUDA;
-  dim3 grid((unsigned)((N + kBM - 1) / kBM), (unsigned)((M + kSpBN - 1) / kSpBN));
-  kern<<<grid, 224, kSpSmem, s>>>(ta, tb, te, p);
-  return launch_status();
-}
 
 // W4A4 GEMM on the sparse FP4 MMA: y = s_w s_x sum_k dec(x) dec(w) with w a pairwise-4:8 weight
 // (values codes [N, K/4], their scales [N, K/32], meta [N, K/16]) and x packed E2M1 with one

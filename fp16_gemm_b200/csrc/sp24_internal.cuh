@@ -149,11 +149,6 @@ int moe_tc_block_gemm(int epi, int wf, int t16, const MoeBlockGemm& g, cudaStrea
 int tc_gemm_f16(const void* x, const void* w, int64_t M, int64_t N, int64_t K, bool bf16, float* y,
                 const float* scale_a, const float* scale_b, cudaStream_t s);
 
-// Native 2:4 tensor-core GEMM (tcgen05.mma.sp) on 16-bit kept values + nibble stream; K % 128.
-int tc_gemm_f16_sparse(const void* x, const void* values, const uint8_t* meta, int64_t M, int64_t N,
-                       int64_t K, bool bf16, float* y, const float* scale_a, const float* scale_b,
-                       cudaStream_t s);
-
 // NVFP4 operand images for the W4A4 kernel (K % 256 == 0): codes [rows, K/2] -> 16 KB tiles of
 // 128 rows x 256 K in the 128-byte-swizzled shared-memory order; scales [rows, K/16] -> 512-byte
 // tiles of 128 rows x 4 scales in tcgen05.cp order.
@@ -180,11 +175,27 @@ int tc_gemm_nvfp4_sp48_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const 
                             const uint8_t* vs_mma, const uint8_t* meta_mma, const float* w_ts, int64_t M, int64_t N,
                             int64_t K, float* y, cudaStream_t s, uint64_t wait_ns);
 
+// A 2-D map over rows of row_bytes bytes (elements of elem bytes), box box_rows whole rows, no
+// swizzle; and the fp32 output Y [M, N] with box 128 rows of N x 32 tokens.
+int make_tmap_rows(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem, uint64_t row_bytes,
+                   uint64_t rows, uint32_t box_rows);
+int make_tmap_y(CUtensorMap* map, float* y, int64_t M, int64_t N);
+
 // W4A4 GEMM on the persistent CTA-pair kernel (both operands as images above).  wait_ns bounds
 // every device-side wait (0: the library's default).
 int tc_gemm_nvfp4_pair(const uint8_t* xc_mma, const uint8_t* xs_mma, const float* x_ts, const uint8_t* wc_mma,
                        const uint8_t* ws_mma, const float* w_ts, int64_t M, int64_t N, int64_t K, float* y,
                        cudaStream_t s, uint64_t wait_ns);
+
+// 16-bit GEMM on the persistent CTA-pair kernel (tcgen05 cta_group::2): dense (meta_img null,
+// K % 64) or 2:4 with values [N, K/2] and the metadata image of meta_to_image (K % 128).
+int tc_gemm_f16_pair(const void* x, const void* w, const uint8_t* meta_img, int64_t M, int64_t N, int64_t K,
+                     bool bf16, float* y, const float* scale_a, const float* scale_b, cudaStream_t s,
+                     uint64_t wait_ns);
+// The 2:4 metadata image of the pair kernel (tcgen05 metadata tiles of 128 rows x 128 K, rows
+// padded to 256) and its size in bytes.
+int64_t meta_image_bytes(int64_t rows, int64_t K);
+int meta_to_image(const uint8_t* meta, int64_t rows, int64_t K, uint8_t* out, cudaStream_t s);
 
 // Expands an NVFP4 (W_DQ4) or 2:4-compressed (W_S16 / W_SQ4) operand into exact 16-bit values.
 int expand_w16(int wf, bool bf16, const uint8_t* w, const uint8_t* scales, const uint8_t* meta,

@@ -434,6 +434,29 @@ __device__ __forceinline__ void umma_nvfp4_sp_pair(uint32_t d_tmem, uint64_t a_d
       : "memory");
 }
 
+// kind::f16 MMA over the CTA pair (M = 256: 128 A rows from each CTA's shared memory).
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 2:4 sparse kind::f16 MMA over the CTA pair (K = 32 logical), metadata at `e_tmem` in each
+// CTA's TMEM.
+__device__ __forceinline__ void umma_f16_sp_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // 128 TMEM lanes x 128 bits (4 columns) in both CTAs of the pair, each from its own shared
 // memory (the source form of desc_rows16_noswizzle).
 __device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {

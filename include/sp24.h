@@ -137,6 +137,23 @@ int sp24_prune_compress_24(const void* w, int dtype, int op, const int64_t* shap
 int sp24_decompress_24(const void* values, const uint8_t* meta, int dtype, int op,
                        const int64_t* shape, int ndim, void* w_out, void* stream);
 
+/* The nibble stream of a 2:4 weight [rows, K] (matmul layout, K % 128 == 0) rewritten in the
+ * layout the sparse tensor-core MMA reads its metadata in ([P1] "What 2:4 actually is": the
+ * positions travel with the kept values), so that a GEMM moves it into tensor memory without
+ * touching it.  Not on the source pages: the layout of this library's kernel.
+ *   meta_img: for each 128-row block rb and 128-K chunk kc a 2 KB tile at byte
+ *             2048 (rb * K/128 + kc); its 16-byte row l (l = 0..127) is TMEM lane l: rows
+ *             m = 128 rb + 16 (l / 16) + l % 8 and m + 8, half h = (l / 8) % 2; 32-bit word t
+ *             (the 32-wide K window t) = the two nibble bytes 16 kc + 4 t + 2 h, +1 of row m in
+ *             the low half and of row m + 8 in the high half.  Rows are padded to a multiple of
+ *             256 with bytes 0x44 (index pair 0, 1 in every group).
+ *   sp24_prepare_sparse_size gives the bytes (rows rounded up to 256, times K/128 x 2 KB / 128).
+ *   meta: device, [rows, K/8] as from sp24_prune_compress_24; meta_img: device, 16-byte aligned,
+ *   owned by the caller.  K % 128 != 0 or negative sizes: SP24_ERR_SHAPE.  One launch.
+ * sp24_gemm_sparse24 with 16-bit values at M > 64 builds this image in its workspace itself. */
+int sp24_prepare_sparse_size(int64_t rows, int64_t K, int64_t* bytes);
+int sp24_prepare_sparse(const uint8_t* meta, int64_t rows, int64_t K, uint8_t* meta_img, void* stream);
+
 /* ----------------------------------------------------------------------- pairwise 4:8 */
 /* The sparse pattern of the tensor cores' packed-FP4 MMA kind, whose sparse unit is a pair of
  * consecutive entries.  [P1] "What 2:4 actually is" (the largest magnitudes survive), carried

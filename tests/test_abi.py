@@ -231,3 +231,19 @@ def test_sparse_pair_images_host_validation():
     xo = sp._Operand(sp.NVFP4_B32_MMA, 16, 16, 16)
     wo = sp._SparseOperand(sp.NVFP4, 16, 16, 16, 16)
     assert L.sp24_gemm_sparse48(ctypes.byref(xo), ctypes.byref(wo), 4, 128, 512, ctypes.c_void_p(256), None) == sp.ERR_DTYPE
+
+
+def test_prepare_sparse_host_validation():
+    """The metadata image of the 16-bit 2:4 pair kernel: rows padded to 256, 2 KB per 128 rows and
+    128 K; K must be a multiple of 128."""
+    L = sp.lib()
+    n = ctypes.c_int64(-1)
+    assert L.sp24_prepare_sparse_size(300, 256, ctypes.byref(n)) == sp.OK
+    assert n.value == 4 * 2 * 2048
+    assert L.sp24_prepare_sparse_size(256, 128, ctypes.byref(n)) == sp.OK and n.value == 2 * 1 * 2048
+    assert L.sp24_prepare_sparse_size(8, 192, ctypes.byref(n)) == sp.ERR_SHAPE
+    assert L.sp24_prepare_sparse_size(8, 128, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_prepare_sparse(None, 8, 256, None, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_prepare_sparse(None, 8, 96, None, None) == sp.ERR_SHAPE
+    assert L.sp24_prepare_sparse(None, 0, 256, None, None) == sp.OK
+    assert L.sp24_prepare_sparse(ctypes.c_void_p(16), 8, 256, ctypes.c_void_p(8), None) == sp.ERR_ALIGN
