@@ -928,6 +928,8 @@ def run_ncu_target(which: str) -> None:
       decode  the decode step on its workload (prepare_vec, encode_pair_kernel, decode_tile_kernel
               dense and 2:4), twice;
       w4a4    the W4A4 GEMM at 4096^3 on tile images (gemm_nvfp4_pair_kernel), three times;
+      f16     the FP16 M-sweep GEMMs at M = 4096, N = K = 5120 (gemm_f16_pair_kernel dense, then
+              2:4 after its metadata image), twice;
       all     both, then the 2:4 and pairwise-4:8 W4A4 GEMMs, the FP16 M = 4096 GEMMs and the
               routed-expert workload once (several GB on the device)."""
     import torch
@@ -951,6 +953,14 @@ def run_ncu_target(which: str) -> None:
         xi, wi = sp.to_mma(xq), sp.to_mma(wq)
         for _ in range(3):
             sp.gemm_dense(xi, wi)
+    if which == "f16":
+        g = synth.rng(0)
+        w16 = torch.from_numpy(synth.draw(g, (5120, 5120), "f16")).cuda()
+        x16 = torch.from_numpy(synth.draw(g, (4096, 5120), "f16")).cuda()
+        v16, m16 = sp.prune_compress_24(w16)
+        for _ in range(2):
+            sp.gemm_dense(x16, w16)
+            sp.gemm_sparse24(x16, sp.Sparse24(v16, m16), 5120)
     if which == "all":
         v, m = sp.prune_compress_24(w)
         vq = sp.quantize_nvfp4(v)
@@ -992,7 +1002,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-shape GEMM table instead of the step")
-    ap.add_argument("--ncu-target", nargs="?", const="all", choices=["decode", "w4a4", "all"], default=None,
+    ap.add_argument("--ncu-target", nargs="?", const="all", choices=["decode", "w4a4", "f16", "all"], default=None,
                     help="run one kernel family once, untimed (for an ncu capture); no value: all")
     ap.add_argument("--peaks", action="store_true", help="measure MMA and HBM peaks into profiles/peaks.json")
     ap.add_argument("--no-per-config", action="store_true",
