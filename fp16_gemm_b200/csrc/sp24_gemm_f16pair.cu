@@ -19,8 +19,9 @@
 //     4-column TMEM slot of that stage, issued by the MMA thread before the stage's MMAs, so no
 //     warp rewrites nibbles on the way;
 //   * persistent, tiles round-robin over the pairs, two TMEM accumulators so that a tile's
-//     epilogue (TMEM -> registers -> shared memory -> TMA store of 32-token x 128-row fp32 boxes)
-//     overlaps the next tile's main loop (2:4 at BN = 256: the accumulators overlap in 32
+//     epilogue (TMEM -> registers -> shared memory -> TMA store of 32-token x 128-row fp32 boxes,
+//     marked evict-first in L2 so the output does not push the operands out) overlaps the next
+//     tile's main loop (2:4 at BN = 256: the accumulators overlap in 32
 //     columns, read first and released, as in the FP4 pair kernel).
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer (one lane; both CTAs load their own
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(192, 1)
     const bool epi_leader = warp == 2 && lane == 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
+    const uint64_t y_policy = l2_evict_first_policy();
     float scale = 1.0f;
     if (p.scale_a) scale *= *p.scale_a;
     if (p.scale_b) scale *= *p.scale_b;
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(192, 1)
           fence_proxy_async_smem();
           named_bar_sync(1, 128);
           if (epi_leader && row0 < p.N && n0 + 32 * c < p.M) {  // boxes wholly outside Y are skipped
-            tma_store_2d(&tmY, st, row0, n0 + 32 * c);
+            tma_store_2d_evict_first(&tmY, st, row0, n0 + 32 * c, y_policy);
             bulk_commit();
           }
           ++chunk;

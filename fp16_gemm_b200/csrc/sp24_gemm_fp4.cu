@@ -20,7 +20,7 @@
 //     alternate between stages (0.51 us per stage);
 //   * persistent: one CTA per SM, tiles assigned round-robin to the pairs; two TMEM
 //     accumulators, so a tile's epilogue (TMEM -> registers -> shared memory -> TMA store of
-//     32-token x 128-row fp32 boxes) overlaps the next tile's main loop.  For BN = 256 the two
+//     32-token x 128-row fp32 boxes, marked evict-first in L2) overlaps the next tile's main loop.  For BN = 256 the two
 //     accumulators overlap in 96 columns (0-255 and 160-415, scale slots in 416-511): the
 //     epilogue reads the shared columns first and releases the accumulator, then drains the rest
 //     while the next tile's MMAs run.
@@ -403,6 +403,7 @@ __global__ void __launch_bounds__(256, 1)
     const bool epi_leader = warp == 2 && lane == 0;
     const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty_bar), 0);
     const float scale = __fmul_rn(*p.ts_w, *p.ts_x);
+    const uint64_t y_policy = l2_evict_first_policy();
     int j = 0, chunk = 0;
     for (int t = pair; t < tiles; t += pairs, ++j) {
       const int row0 = (t % p.tiles_w) * 256 + (int)rank * 128;
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(256, 1)
           fence_proxy_async_smem();
           named_bar_sync(1, 128);
           if (epi_leader && row0 < p.N && n0 + 32 * c < p.M) {  // boxes wholly outside Y are skipped
-            tma_store_2d(&tmY, st, row0, n0 + 32 * c);
+            tma_store_2d_evict_first(&tmY, st, row0, n0 + 32 * c, y_policy);
             bulk_commit();
           }
           ++chunk;

@@ -519,6 +519,20 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                "r"(y), "r"(smem_u32(src))
                : "memory");
 }
+// The same store marked evict-first in L2: an output written once and not read again here
+// should not push the GEMM's operands out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_store_2d_evict_first(const CUtensorMap* map, const void* src, int x, int y,
+                                                         uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
+                   map),
+               "r"(x), "r"(y), "r"(smem_u32(src)), "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Returns once at most N of this thread's bulk groups still read shared memory.
 template <int N>
