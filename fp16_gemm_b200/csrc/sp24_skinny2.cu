@@ -948,6 +948,13 @@ __global__ void __launch_bounds__(640, 1) decode_tile_kernel(const SkinnyParams 
     const uint8_t* d = bufs + sl * tg.bytes();
     const uint8_t* sc = d + 16 * tg.cb;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+    // 2:4: the block scales of the warp's four window pairs in one 8-byte load per row, and below
+    // the nibbles of two pairs in one 16-byte load per row, instead of narrow loads per pair
+    uint2 sw0, sw1;
+    if constexpr (WF == W_SQ4) {
+      sw0 = *reinterpret_cast<const uint2*>(sc + r0 * tg.sb + 8 * warp);
+      sw1 = *reinterpret_cast<const uint2*>(sc + r1 * tg.sb + 8 * warp);
+    }
 #pragma unroll
     for (int j = 0; j < XI; ++j) {
       float(&a)[4] = (j & 1) ? acc2 : acc;
@@ -978,15 +985,17 @@ __global__ void __launch_bounds__(640, 1) decode_tile_kernel(const SkinnyParams 
         }
       } else {
         const uint8_t* me = sc + 16 * tg.sb;
+        const uint4 mq0 = *reinterpret_cast<const uint4*>(me + r0 * tg.mb + 8 * (4 * warp + 2 * j));
+        const uint4 mq1 = *reinterpret_cast<const uint4*>(me + r1 * tg.mb + 8 * (4 * warp + 2 * j));
 #pragma unroll
-        for (int pp = 0; pp < 2; ++pp) {  // window pair q = 4w + 2j + pp
-          const int q = 4 * warp + 2 * j + pp;
+        for (int pp = 0; pp < 2; ++pp) {  // window pair q = 4w + p, p = 2j + pp
+          const int p = 2 * j + pp, q = 4 * warp + p;
           const uint4 c0 = *reinterpret_cast<const uint4*>(d + r0 * tg.cb + 16 * q);
           const uint4 c1 = *reinterpret_cast<const uint4*>(d + r1 * tg.cb + 16 * q);
-          const uint2 m0 = *reinterpret_cast<const uint2*>(me + r0 * tg.mb + 8 * q);
-          const uint2 m1 = *reinterpret_cast<const uint2*>(me + r1 * tg.mb + 8 * q);
-          const uint32_t h0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r0 * tg.sb + 2 * q));
-          const uint32_t h1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sc + r1 * tg.sb + 2 * q));
+          const uint2 m0 = pp ? make_uint2(mq0.z, mq0.w) : make_uint2(mq0.x, mq0.y);
+          const uint2 m1 = pp ? make_uint2(mq1.z, mq1.w) : make_uint2(mq1.x, mq1.y);
+          const uint32_t h0 = e4m3x2_to_f16x2(((p >> 1) ? sw0.y : sw0.x) >> (16 * (p & 1)));
+          const uint32_t h1 = e4m3x2_to_f16x2(((p >> 1) ? sw1.y : sw1.x) >> (16 * (p & 1)));
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const uint32_t e = __byte_perm(u ? m0.y : m0.x, u ? m1.y : m1.x, (c & 1) ? 0x7632 : 0x5410);
