@@ -247,3 +247,20 @@ def test_prepare_sparse_host_validation():
     assert L.sp24_prepare_sparse(None, 8, 96, None, None) == sp.ERR_SHAPE
     assert L.sp24_prepare_sparse(None, 0, 256, None, None) == sp.OK
     assert L.sp24_prepare_sparse(ctypes.c_void_p(16), 8, 256, ctypes.c_void_p(8), None) == sp.ERR_ALIGN
+
+
+def test_gemm_workspace_holds_the_metadata_image():
+    """At M > 64 a 2:4 product runs on the 16-bit CTA-pair kernel, whose workspace holds the
+    metadata image (2 KB per 128 rows padded to 256 and 128 K) beside any 16-bit expansion of
+    NVFP4 kept values (N x K/2 entries of 2 bytes); dense 16-bit needs none, nor the skinny path."""
+    L = sp.lib()
+    n = ctypes.c_int64(-1)
+    image = 4 * 2 * 2048  # N = 300 -> 512 rows, K = 256 -> 2 chunks
+    assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 1, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == image
+    assert L.sp24_gemm_workspace_size(sp.BF16, sp.NVFP4, 1, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 300 * 256 + image
+    assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 0, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 0
+    assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 1, 8, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 0
