@@ -403,7 +403,10 @@ int sp24_gemm_dense(const sp24_operand* x, const sp24_operand* w, int64_t M, int
 
 /* [P2] "The mechanism needs both values and their positions": the same product with w in
  * 2:4-compressed form; only kept entries are multiplied.  K alignment: 16-bit values K % 16,
- * NVFP4 values K % 64. */
+ * NVFP4 values K % 64.  At M > 64 with K % 128 == 0 the product runs on the sparse tensor-core
+ * MMA of a persistent CTA-pair kernel (NVFP4 kept values first expanded to x's 16-bit type, exact),
+ * which reads the metadata in the layout of sp24_prepare_sparse: the call builds it in the
+ * workspace (sp24_gemm_workspace_size counts it). */
 int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M,
                        int64_t N, int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                        int algo, void* stream);
