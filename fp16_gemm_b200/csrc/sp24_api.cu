@@ -184,8 +184,18 @@ int run_tiled(int wf, int t16, const SkinnyParams& p, void* ws, int64_t ws_bytes
   return tc_gemm_f16(x16, w16, p.M, p.N, p.K, bf, p.y, sa, sb, s);
 }
 
+// ALGO_AUTO: the skinny kernels (FP4 decoded in registers, one launch per 64 rows of x) up to
+// M = 64, and up to M = 128 for dense NVFP4 weights with 16-bit x, where the tiled path first
+// expands the whole weight to 16 bits in HBM (measured at N = K = 5120: 47 / 52 / 67 us against
+// 70 / 71 / 71 us at M = 80 / 96 / 128; at M = 192 tiled wins).  2:4 NVFP4 weights go tiled
+// above 64 rows: the skinny 2:4 kernel took 72-120 us there against 50 us tiled.
+bool auto_skinny(int x_fmt, int wf, int64_t M) {
+  return M <= 64 || (M <= 128 && x_fmt == X_16 && wf == W_DQ4);
+}
+
 int dispatch(int wf, int t16, const SkinnyParams& p, int algo, void* ws, int64_t ws_bytes, cudaStream_t s) {
-  if (algo == SP24_ALGO_SKINNY || (algo == SP24_ALGO_AUTO && p.M <= 64)) return run_skinny(wf, t16, p, s);
+  if (algo == SP24_ALGO_SKINNY || (algo == SP24_ALGO_AUTO && auto_skinny(p.x_fmt, wf, p.M)))
+    return run_skinny(wf, t16, p, s);
   return run_tiled(wf, t16, p, ws, ws_bytes, s);
 }
 
@@ -258,7 +268,7 @@ extern "C" int sp24_gemm_workspace_size(int x_format, int w_format, int sparse, 
     return SP24_ERR_DTYPE;
   const int wf = sparse ? (is16(w_format) ? W_S16 : W_SQ4) : (is16(w_format) ? W_D16 : W_DQ4);
   const int xf = x_format == SP24_NVFP4 ? X_Q4 : X_16;
-  const bool tiled = algo == SP24_ALGO_TILED || (algo == SP24_ALGO_AUTO && M > 64);
+  const bool tiled = algo == SP24_ALGO_TILED || (algo == SP24_ALGO_AUTO && !auto_skinny(xf, wf, M));
   *bytes = tiled ? tiled_workspace(xf, wf, M, N, K) : 0;
   return SP24_OK;
 }

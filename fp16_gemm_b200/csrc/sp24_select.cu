@@ -7,12 +7,14 @@
 //     `reps` back-to-back launches after one warm-up launch each) and records the faster one
 //     for (device, x format, weight format, M, N, K);
 //   * sp24_gemm_choice answers from that record, else from a rule of measured crossovers on
-//     B200 (the repository's benchmark sweep at N = K = 5120): FP16 weights go 2:4 up to
-//     M = 2048 (measured 1.04-1.30x at M <= 1024, 0.94-0.99x at M >= 4096); NVFP4 weights with
-//     16-bit activations go 2:4 at every M (1.00-1.56x); NVFP4 weights with NVFP4 activations
-//     stay dense (the dense FP4 MMA against the 16-bit sparse MMA: 0.42-0.79x, 1.03x only at
-//     M = 16); weights of fewer than 2^20 entries stay dense (launch-bound: 5.0 vs 5.7 us
-//     for a [256, 512] weight at M = 16, the dense kernel starts sooner);
+//     B200 (the repository's benchmark at N = K = 5120): 16-bit weights go 2:4 from M = 128
+//     (the CTA-pair tensor-core kernels: 1.10x at M = 128, 1.18-1.49x from M = 1024; 0.97-1.01x
+//     at M = 1 and 16); NVFP4 weights with 16-bit activations go 2:4 from M = 128 (1.34-1.61x),
+//     below it the dense decode and skinny kernels win (0.87-0.92x, and dense 47 against 50 us
+//     at M = 80); NVFP4 weights with NVFP4 activations stay dense (the dense FP4 MMA against
+//     the 16-bit sparse MMA: 0.45-0.49x, 1.05x only at M = 16); weights of fewer than 2^20
+//     entries stay dense (launch-bound: 5.1 vs 5.6 us for a [256, 512] weight at M = 16, the
+//     dense kernel starts sooner);
 //   * sp24_gemm_auto runs the chosen GEMM (asynchronous; usable under graph capture).
 // Host code only: the GEMMs are the library's own entry points.
 #include "sp24_internal.cuh"
@@ -39,8 +41,7 @@ int rule_choice(int x_format, int w_format, int64_t M, int64_t N, int64_t K) {
   const bool pair16 = is16(x_format) && is16(w_format), w4a16 = is16(x_format) && w_format == SP24_NVFP4;
   if (!pair16 && !w4a16 && !(x_format == SP24_NVFP4 && w_format == SP24_NVFP4)) return -1;
   if (N * K < (int64_t)1 << 20) return 0;  // launch-bound: the dense kernel starts sooner
-  if (pair16) return M <= 2048 ? 1 : 0;
-  if (w4a16) return 1;
+  if (pair16 || w4a16) return M >= 128 ? 1 : 0;
   return 0;
 }
 

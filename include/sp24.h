@@ -388,7 +388,8 @@ int sp24_prepare_24(const void* w, int dtype, int64_t rows, int64_t K, uint8_t* 
  * applies the block scales (K % 256 == 0 and M > 64, or either operand SP24_NVFP4_MMA: a
  * persistent kernel on pairs of SMs; the workspace then holds the tile images of each operand
  * given as SP24_NVFP4).  NVFP4 w with 16-bit x is decoded inside the kernel to x's type at
- * M <= 64; at larger M it is first expanded to x's type in the workspace (exact values).
+ * M <= 64 (dense w with algo auto: M <= 128, one launch per 64 rows of x); at larger M it is
+ * first expanded to x's type in the workspace (exact values).
  * K alignment: 16-bit w K % 8, NVFP4 w K % 32, NVFP4 x K % 32.  Operand pointers 16-byte
  * aligned, y 4-byte aligned (SP24_ERR_ALIGN otherwise; the same holds for every GEMM entry
  * point below).  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
@@ -422,8 +423,8 @@ int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int6
  *                     not for use during graph capture.  y receives a result of either form.
  *   sp24_gemm_choice  (host only) the recorded decision, else a rule of crossovers measured on
  *                     B200: weights of fewer than 2^20 entries dense (launch-bound); else
- *                     16-bit weights 2:4 for M <= 2048, NVFP4 weights with 16-bit x 2:4,
- *                     NVFP4 weights with NVFP4 x dense.  *measured (may be NULL): 1 if recorded.
+ *                     16-bit weights, and NVFP4 weights with 16-bit x, 2:4 for M >= 128
+ *                     and dense below; NVFP4 weights with NVFP4 x dense.  *measured (may be NULL): 1 if recorded.
  *                     SP24_ERR_DTYPE for format pairs without a 2:4 path.
  *   sp24_gemm_auto    runs the GEMM sp24_gemm_choice names; *used_sparse (may be NULL) says
  *                     which.  Asynchronous.

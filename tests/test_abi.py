@@ -250,16 +250,23 @@ def test_prepare_sparse_host_validation():
 
 
 def test_gemm_workspace_holds_the_metadata_image():
-    """At M > 64 a 2:4 product runs on the 16-bit CTA-pair kernel, whose workspace holds the
-    metadata image (2 KB per 128 rows padded to 256 and 128 K) beside any 16-bit expansion of
-    NVFP4 kept values (N x K/2 entries of 2 bytes); dense 16-bit needs none, nor the skinny path."""
+    """A tiled 2:4 product runs on the 16-bit CTA-pair kernel, whose workspace holds the metadata
+    image (2 KB per 128 rows padded to 256 and 128 K) beside any 16-bit expansion of NVFP4 kept
+    values (N x K/2 entries of 2 bytes); dense 16-bit needs none, nor the skinny path."""
     L = sp.lib()
     n = ctypes.c_int64(-1)
     image = 4 * 2 * 2048  # N = 300 -> 512 rows, K = 256 -> 2 chunks
     assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 1, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
     assert n.value == image
+    assert L.sp24_gemm_workspace_size(sp.BF16, sp.NVFP4, 1, 256, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 300 * 256 + image
     assert L.sp24_gemm_workspace_size(sp.BF16, sp.NVFP4, 1, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
     assert n.value == 300 * 256 + image
+    # dense NVFP4 weights with 16-bit x stay on the skinny kernels up to M = 128 (no expansion)
+    assert L.sp24_gemm_workspace_size(sp.BF16, sp.NVFP4, 0, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 0
+    assert L.sp24_gemm_workspace_size(sp.BF16, sp.NVFP4, 0, 129, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
+    assert n.value == 300 * 256 * 2
     assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 0, 128, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
     assert n.value == 0
     assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 1, 8, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK

@@ -59,12 +59,13 @@ def test_select_records_the_faster_and_auto_matches_oracle(wfmt, M):
     assert sp.gemm_choice(sp.BF16, wf, M, N, K)[1] is False
 
 
-def test_auto_without_record_follows_the_rule():
-    M, N, K = 16, 1024, 1024
+@pytest.mark.parametrize("M,expect", [(16, False), (128, True)])
+def test_auto_without_record_follows_the_rule(M, expect):
+    N, K = 1024, 1024
     X, W, wd, ws = _forms(M, N, K, "nvfp4", 210)
     sp.gemm_choice_reset()
     y, used = sp.gemm_auto(to_dev(X, "bf16"), wd, ws)
     torch.cuda.synchronize()
-    assert used is True  # NVFP4 weights with 16-bit x: the rule says 2:4
-    Y, S = _oracle(X, W, "nvfp4", True)
+    assert used is expect  # NVFP4 weights with 16-bit x: dense below M = 128, 2:4 from it
+    Y, S = _oracle(X, W, "nvfp4", expect)
     assert_gemm_close(y, Y, S)

@@ -6,9 +6,10 @@ import fp16_gemm_b200 as sp
 
 
 @pytest.mark.parametrize("xf,wf,M,expect", [
-    (sp.F16, sp.F16, 1, True), (sp.F16, sp.F16, 1024, True), (sp.F16, sp.F16, 2048, True),
-    (sp.F16, sp.F16, 2049, False), (sp.BF16, sp.BF16, 16384, False),
-    (sp.BF16, sp.NVFP4, 1, True), (sp.F16, sp.NVFP4, 16384, True),
+    (sp.F16, sp.F16, 1, False), (sp.F16, sp.F16, 127, False), (sp.F16, sp.F16, 128, True),
+    (sp.F16, sp.F16, 4096, True), (sp.BF16, sp.BF16, 16384, True),
+    (sp.BF16, sp.NVFP4, 1, False), (sp.BF16, sp.NVFP4, 8, False), (sp.F16, sp.NVFP4, 128, True),
+    (sp.F16, sp.NVFP4, 16384, True),
     (sp.NVFP4, sp.NVFP4, 16, False), (sp.NVFP4, sp.NVFP4, 4096, False),
 ])
 def test_rule(xf, wf, M, expect):
@@ -19,7 +20,7 @@ def test_rule(xf, wf, M, expect):
 @pytest.mark.parametrize("N,K,expect", [(256, 512, False), (1024, 1023, False), (1024, 1024, True)])
 def test_rule_small_weights_stay_dense(N, K, expect):
     sp.gemm_choice_reset()
-    assert sp.gemm_choice(sp.F16, sp.F16, 16, N, K) == (expect, False)
+    assert sp.gemm_choice(sp.F16, sp.F16, 256, N, K) == (expect, False)
 
 
 @pytest.mark.parametrize("xf,wf", [(sp.NVFP4, sp.F16), (sp.F32, sp.F16), (sp.F16, sp.F32)])
