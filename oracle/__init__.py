@@ -21,10 +21,12 @@ Pairwise 4:8 (``check_48`` / ``compress_48`` / ``decompress_48``) and the 32-val
 actually is", carried over to pairs; the block size the sparse FP4 MMA reads); they are pinned
 against brute force over the six pair choices and against ml_dtypes' roundings.
 
-Parity unpinned: the NVFP4 scale and rounding formulae (tensor scale = amax / 2688, block
-scale = E4M3(bmax / (6 s_t)), code = E2M1(|t| / (dec(sb) s_t)), all RNE) are a reading; the
-pages state the format but print no worked example, so only their properties (sizes,
-re-quantisation stability, negative zero, exhaustive rounding) are pinned.
+The NVFP4 scale and rounding formulae (tensor scale = amax / 2688, block scale =
+E4M3(bmax / (6 s_t)), code = E2M1(|t| / (dec(sb) s_t)), all RNE) are a reading: the pages
+state the format but print no worked example.  They are pinned to the recipe the pages'
+converter reproduces bit for bit (ModelOpt's), as compressed-tensors (global scale) and vLLM
+(reference quantiser) implement it, up to one rounding step next to a rounding boundary, and
+by their properties (sizes, re-quantisation stability, negative zero, exhaustive rounding).
 """
 from __future__ import annotations
 
