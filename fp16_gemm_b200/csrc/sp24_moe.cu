@@ -257,7 +257,7 @@ extern "C" int sp24_gemm_grouped(const sp24_operand* x, const int32_t* routing, 
   return skinny2_grouped(wf, t16, p, n_tiles, s);
 }
 
-// ------------------------------------------------------------------ expert block (NEXT-3)
+// ------------------------------------------------------------------ expert block
 //
 // y[t] = sum_s r[t, s] * (SiLU(x_t Wg_e^T) * (x_t Wu_e^T)) Wd_e^T,  e = routing[t, s]
 // ([P1] "Concurrency, not sparsity, is the lever": the routed experts of a decode step).

@@ -80,32 +80,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// As mbar_try_wait, but the thread may be suspended (not polling, issuing nothing) until the
-// phase completes or about `hint_ns` nanoseconds pass.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
-// mbar_wait for waiters that share the SM with busy warps: the waiting thread sleeps in the
-// barrier instead of spinning, so it takes no issue slots from them.  Same time limit.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
-  const uint64_t lim = wait_limit();
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
-    if (globaltimer() - t0 > lim) return false;
-  }
-  return true;
-}
-
 // 16-byte asynchronous global -> shared copy on the load/store path (not the TMA engine), cached
 // in L2 only.  Copies complete in commit-group order: cp_async_wait<N>() returns once at most N
 // of the calling thread's groups are still in flight; other threads see the data after a barrier.
@@ -133,19 +107,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Row gather: four rows (y0 .. y3, any order, out-of-range rows read as zeros) of `cols_box`
-// elements at column x from a 2-D tensor map whose box is one row high, written as four
-// consecutive box rows at dst (with the map's swizzle), completing their bytes on `bar`.
-// No cluster multicast.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
-                                            int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -329,8 +290,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
-
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)
 //
 // Two CTAs of a cluster of two run one MMA of M = 256 rows: each holds 128 rows of A and half
@@ -512,15 +471,9 @@ __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 2-D TMA tile store from this CTA's shared memory (elements outside the tensor are skipped),
-// tracked as one bulk async-group per commit.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
-               "r"(y), "r"(smem_u32(src))
-               : "memory");
-}
-// The same store marked evict-first in L2: an output written once and not read again here
-// should not push the GEMM's operands out of L2.
+// 2-D TMA tile stores from this CTA's shared memory (elements outside the tensor are skipped),
+// tracked as one bulk async-group per commit, marked evict-first in L2: an output written once
+// and not read again here should not push the GEMM's operands out of L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
