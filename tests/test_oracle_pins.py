@@ -199,6 +199,32 @@ def test_conv_roundtrip(oracle):
     assert np.array_equal(back.view(np.uint16), np.ascontiguousarray(pr_mm).view(np.uint16))
 
 
+def test_conv_values_layout_brute_force(oracle):
+    """The compressed conv tensor is [K, C/2, R, S]: group (k, j, r, s) runs over w[k, 4j..4j+3,
+    r, s] ("The operation determines which four entries belong together": groups along C) and
+    its kept entries, the two largest magnitudes in ascending index order, sit at
+    values[k, 2j], values[k, 2j + 1] of the same (r, s); found here by sorting each group."""
+    g = synth.rng(9)
+    K, C, R, S = 3, 12, 2, 3
+    w = f16(synth.normal(g, (K, C, R, S)))
+    vals, meta = oracle.compress_24(w, oracle.F16, oracle.CONV)
+    assert vals.shape == (K, C // 2, R, S)
+    want = np.zeros((K, C // 2, R, S), dtype=np.float16)
+    nib = []
+    for k in range(K):
+        for j in range(C // 4):
+            for r in range(R):
+                for s_ in range(S):
+                    grp = w[k, 4 * j:4 * j + 4, r, s_]
+                    order = sorted(range(4), key=lambda i: (-abs(float(grp[i])), i))
+                    i0, i1 = sorted(order[:2])
+                    want[k, 2 * j, r, s_], want[k, 2 * j + 1, r, s_] = grp[i0], grp[i1]
+                    nib.append(i0 | i1 << 2)
+    assert np.array_equal(vals.view(np.uint16), want.view(np.uint16))
+    got_nib = np.stack([meta & 0xF, meta >> 4], 1).ravel()[:len(nib)]
+    assert got_nib.tolist() == nib
+
+
 def test_decompress_rejects_illegal_nibble(oracle):
     with pytest.raises(oracle.OracleError):
         oracle.decompress_24(np.zeros(2, np.float16), np.array([0x5], np.uint8), oracle.F16, (4,))
@@ -496,6 +522,11 @@ def test_moe_block_hand_example(oracle):
     # in f16 h keeps 11 bits: 1.4619140625 (1 + 473/1024)
     Y16, _ = oracle.moe_block(X, np.array([[0]]), np.array([[1.0]]), Wg, Wu, Wd, oracle.F16)
     assert Y16.tolist() == [[3 * 1.4619140625, -1.4619140625]]
+    # a negative h: gate row [-1, 0] gives g = -1, h = 2 SiLU(-1) = -2 / (1 + e) = -0.53788284...,
+    # in bf16 -0.5390625 (1 + 10/128 times 2^-1); the tolerance scale takes |h|
+    Yn, Sn = oracle.moe_block(X, np.array([[0]]), np.array([[0.5]]), -Wg, Wu, Wd, oracle.BF16)
+    assert Yn.tolist() == [[-0.80859375, 0.26953125]]
+    assert Sn.tolist() == [[0.80859375, 0.26953125]]
 
 
 def test_moe_block_silu_zero_and_linearity(oracle):
@@ -524,9 +555,15 @@ def test_moe_block_silu_zero_and_linearity(oracle):
 def test_round_to_16_against_ml_dtypes(oracle):
     """The block's 16-bit hold of h: round to nearest even, checked against ml_dtypes' casts."""
     x = synth.normal(synth.rng(44), 4096) * np.exp(3 * synth.normal(synth.rng(45), 4096))
+    # exact ties between neighbours, which random draws almost never hit: to the even neighbour
+    # (1 + 2^-8 -> 1, 1 + 3 2^-8 -> 1 + 2^-6 in bf16; 1 + 2^-11 -> 1, 1 + 3 2^-11 -> 1 + 2^-9 in f16)
+    ties = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11])
+    x = np.concatenate([x, ties, -ties, ties * 2.0 ** -20])
     bf = np.asarray(x.astype(np.float32).astype(ml_dtypes.bfloat16), dtype=np.float64)
     assert np.array_equal(oracle.round_to_16(x, oracle.BF16), bf)
     assert np.array_equal(oracle.round_to_16(x, oracle.F16), x.astype(np.float16).astype(np.float64))
+    assert oracle.round_to_16(ties[:2], oracle.BF16).tolist() == [1.0, 1 + 2.0 ** -6]
+    assert oracle.round_to_16(ties[2:], oracle.F16).tolist() == [1.0, 1 + 2.0 ** -9]
 
 
 
