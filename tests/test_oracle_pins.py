@@ -302,6 +302,39 @@ def _codes_nibbles(codes):
     return np.stack([codes & 0xF, codes >> 4], -1).reshape(codes.shape[0], -1)
 
 
+def test_nvfp4_exact_ties(oracle):
+    """Block maxima and entries placed exactly on E4M3 / E2M1 rounding midpoints and one fp32
+    step either side, with supplied tensor scales that make the divisors exact ("Convert BF16
+    to NVFP4 yourself": E4M3 block scales, E2M1 codes; round to nearest even): the decisions
+    there are those of ml_dtypes' RNE casts, saturating at 448 and 6.  Random data never lands
+    this close to a boundary, so a slightly wrong quotient or tie rule shows only here."""
+    up, dn = (lambda v: np.nextafter(np.float32(v), np.float32(np.inf))), \
+             (lambda v: np.nextafter(np.float32(v), np.float32(0)))
+    # block scales: s_t = fp32(1/6) makes d = fl32(6 s_t) = 1, so the scale is E4M3(bmax)
+    e4 = np.arange(0, 127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    mids = (e4[1:] + e4[:-1]) / 2
+    q = [m for m in mids[[1, 2, 9, 10, 40, 41, 120, 124, 125]]]
+    q = np.array(q + [up(v) for v in q] + [dn(v) for v in q] + [448.0, 460.0, 464.0, 1e4], dtype=np.float32)
+    t = np.zeros((q.size, 16), dtype=np.float32)
+    t[:, 5] = q
+    t[::2, 5] *= -1
+    s_t = np.float32(1 / 6)
+    _, scales, _ = oracle.nvfp4_encode(t, oracle.F32, tensor_scale=float(s_t))
+    want = np.minimum(q, np.float32(448)).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert scales[:, 0].tolist() == want.tolist()
+    # codes: s_t = 1 and a block maximum of 6 give sb = 1 and divisor 1, so the code is E2M1(t)
+    e2 = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    v = np.concatenate([e2, [up(x) for x in e2], [dn(x) for x in e2], [6.0, 0.0]]).astype(np.float32)
+    v = np.concatenate([v, -v])
+    v = np.concatenate([v, np.zeros((-v.size) % 15, np.float32)]).reshape(-1, 15)
+    t = np.concatenate([np.full((v.shape[0], 1), 6.0, np.float32), v], axis=1)
+    codes, scales, _ = oracle.nvfp4_encode(t, oracle.F32, tensor_scale=1.0)
+    assert np.all(scales == 0x38)  # E4M3 1.0
+    mag = np.minimum(np.abs(t), np.float32(6)).astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    want = mag | (np.signbit(t).astype(np.uint8) << 3)
+    assert np.array_equal(_codes_nibbles(codes), want)
+
+
 def test_nvfp4_error_bound(oracle):
     """Every code is the nearest E2M1 point to |t| / (dec(sb) s_t) (the format's rounding
     bound: at most half a grid step away), and the block scale maps the block maximum close to
