@@ -149,3 +149,37 @@ def test_16bit_entries_on_rounding_boundaries(dtype, ts):
     g = synth.rng(41)
     t = synth.as_storage(np.round(synth.normal(g, (64, 256)) * 8) / 4, dtype)
     _compare(t, dtype, ts)
+
+
+def _neighbours(q, dtype):
+    """q (exact in the storage type) and the storage type's next values below and above it."""
+    q = np.asarray(q, dtype=np.float64)
+    if dtype == "f32":
+        v = q.astype(np.float32)
+        return np.concatenate([v, np.nextafter(v, np.float32(0)), np.nextafter(v, np.float32(np.inf))]).astype(np.float64)
+    if dtype == "f16":
+        v = q.astype(np.float16)
+        return np.concatenate([v, np.nextafter(v, np.float16(0)), np.nextafter(v, np.float16(np.inf))]).astype(np.float64)
+    b = synth.f32_to_bf16_bits(q.astype(np.float32)).astype(np.int64)
+    bits = np.concatenate([b, b - 1, b + 1]).astype(np.uint16)
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+def test_block_scales_at_e4m3_midpoints(dtype):
+    """Block maxima exactly on E4M3 rounding midpoints (ties to the even code) and one step of
+    the storage type either side, with the tensor scale fp32(1/6), which makes the block divisor
+    6 s_t exactly 1: the block scale is E4M3(bmax) rounded at the tie itself.  Normal,
+    subnormal and saturating (above 448) maxima; the other entries of each block are fractions of
+    its maximum with mixed signs, so their codes are checked under the same scale."""
+    e4 = np.array([oracle.e4m3_value(c) for c in range(127)])
+    mids = (e4[1:] + e4[:-1]) / 2
+    pick = mids[[1, 2, 5, 9, 10, 17, 40, 41, 64, 90, 110, 120, 124, 125]]
+    q = _neighbours(np.concatenate([pick, [448.0, 464.0, 4096.0]]), dtype)
+    g = synth.rng(52)
+    frac = np.array([0.5, -0.25, 0.125, 0.75, -0.0625, 0.875, -0.375, 0.3, 0.6, -0.9, 0.05, 0.2, -0.45, 0.65, 0.95])
+    t = np.zeros((q.size, 16))
+    t[:, 0] = np.where(g.random(q.size) < 0.5, -q, q)
+    t[:, 1:] = q[:, None] * frac[None, :]
+    _compare(synth.as_storage(t, dtype), dtype, float(np.float32(1 / 6)))
+
