@@ -271,3 +271,95 @@ def test_gemm_workspace_holds_the_metadata_image():
     assert n.value == 0
     assert L.sp24_gemm_workspace_size(sp.F16, sp.F16, 1, 8, 300, 256, sp.ALGO_AUTO, ctypes.byref(n)) == sp.OK
     assert n.value == 0
+
+
+def test_expert_and_step_entry_points_host_validation():
+    """The routed-expert, expert-block, paired-quantiser, prepare, group-scale, interleave and
+    selection entry points reject bad arguments on the host, before any CUDA call."""
+    L = sp.lib()
+    P = ctypes.c_void_p
+    n = ctypes.c_int64(-1)
+    # routed experts
+    assert L.sp24_gemm_grouped_workspace_size(8, 2, 0, ctypes.byref(n)) == sp.ERR_SHAPE
+    assert L.sp24_gemm_grouped_workspace_size(8, 2, 4, None) == sp.ERR_INVALID_ARG
+    x16 = sp._Operand(sp.F16, 16, None, None)
+    x32 = sp._Operand(sp.F32, 16, None, None)
+    wd = sp._Operand(sp.F16, 16, None, None)
+    ws = sp._SparseOperand(sp.F16, 16, None, None, 16)
+    g = lambda x, d, s, E=4, N=8, K=64, rt=16, y=16: L.sp24_gemm_grouped(
+        x, rt, 8, 2, d, s, E, N, K, y, None, 0, None)
+    assert g(None, ctypes.byref(wd), None) == sp.ERR_INVALID_ARG
+    assert g(ctypes.byref(x16), ctypes.byref(wd), ctypes.byref(ws)) == sp.ERR_INVALID_ARG  # both forms
+    assert g(ctypes.byref(x16), None, None) == sp.ERR_INVALID_ARG                           # neither
+    assert g(ctypes.byref(x16), ctypes.byref(wd), None, E=0) == sp.ERR_SHAPE
+    assert g(ctypes.byref(x16), ctypes.byref(wd), None, N=0) == sp.OK                       # nothing to do
+    assert g(ctypes.byref(x16), ctypes.byref(wd), None, rt=None) == sp.ERR_INVALID_ARG
+    assert g(ctypes.byref(x16), ctypes.byref(wd), None, y=18) == sp.ERR_ALIGN
+    assert g(ctypes.byref(x32), ctypes.byref(wd), None) == sp.ERR_DTYPE
+    # expert block: NVFP4 experts, 16-bit tokens
+    assert L.sp24_moe_block_workspace_size(8, 2, 4, -1, 16, ctypes.byref(n)) == sp.ERR_SHAPE
+    q = sp._Operand(sp.NVFP4, 16, 16, 16)
+    qs_nometa = sp._SparseOperand(sp.NVFP4, 16, 16, 16, None)
+    b = lambda x, gu, gus, dn, dns, E=4, H=64, y=16: L.sp24_moe_block(
+        x, 16, 16, 8, 2, gu, gus, dn, dns, E, H, 32, y, None, 0, None)
+    assert b(None, ctypes.byref(q), None, ctypes.byref(q), None) == sp.ERR_INVALID_ARG
+    assert b(ctypes.byref(x16), ctypes.byref(q), None, ctypes.byref(q), None, E=0) == sp.ERR_SHAPE
+    assert b(ctypes.byref(x32), ctypes.byref(q), None, ctypes.byref(q), None) == sp.ERR_DTYPE
+    assert b(ctypes.byref(x16), ctypes.byref(wd), None, ctypes.byref(q), None) == sp.ERR_DTYPE  # 16-bit experts
+    assert b(ctypes.byref(x16), None, ctypes.byref(qs_nometa), ctypes.byref(q), None) == sp.ERR_INVALID_ARG
+    assert b(ctypes.byref(x16), ctypes.byref(q), None, None, None) == sp.ERR_INVALID_ARG
+    assert b(ctypes.byref(x16), ctypes.byref(q), None, ctypes.byref(q), None, H=0) == sp.OK
+    assert b(ctypes.byref(x16), ctypes.byref(q), None, ctypes.byref(q), None, y=None) == sp.ERR_INVALID_ARG
+    assert b(ctypes.byref(x16), ctypes.byref(q), None, ctypes.byref(q), None, y=20) == sp.ERR_ALIGN
+    # gate / up row interleave
+    assert L.sp24_interleave_rows(16, 16, 8, 64, 0, 16, None) == sp.ERR_SHAPE
+    assert L.sp24_interleave_rows(16, 16, 8, 64, 3, 16, None) == sp.ERR_SHAPE    # rows % block_rows
+    assert L.sp24_interleave_rows(16, 16, 8, 40, 4, 16, None) == sp.ERR_SHAPE    # row bytes % 16
+    assert L.sp24_interleave_rows(None, None, 0, 64, 4, None, None) == sp.OK
+    assert L.sp24_interleave_rows(None, 16, 8, 64, 4, 16, None) == sp.ERR_INVALID_ARG
+    assert L.sp24_interleave_rows(16, 24, 8, 64, 4, 16, None) == sp.ERR_ALIGN
+    # one-pass prepare (check + prune / compress + both tensor scales)
+    assert L.sp24_prepare_24_workspace_size(4, 24, ctypes.byref(n)) == sp.ERR_SHAPE
+    pr = lambda dt=sp.BF16, K=64, w=16, wsp=256, wsb=256: L.sp24_prepare_24(
+        w, dt, 4, K, None, None, 16, 16, 16, 16, wsp, wsb, None)
+    assert pr(dt=9) == sp.ERR_DTYPE
+    assert pr(K=24) == sp.ERR_SHAPE
+    assert pr(w=None) == sp.ERR_INVALID_ARG
+    assert pr(wsp=None) == sp.ERR_WORKSPACE
+    assert pr(wsb=128) == sp.ERR_WORKSPACE
+    assert pr(wsp=264) == sp.ERR_ALIGN
+    assert pr(w=24) == sp.ERR_ALIGN
+    # paired NVFP4 encode (a weight and its kept values, each with a supplied scale)
+    qp = lambda dt=sp.BF16, c0=64, ts=16, t0=16: L.sp24_quantize_nvfp4_pair(
+        t0, dt, 4, c0, ts, 16, 16, 16, 16, 4, 32, 16, 16, 16, 16, None)
+    assert qp(dt=9) == sp.ERR_DTYPE
+    assert qp(c0=24) == sp.ERR_SHAPE
+    assert qp(ts=None) == sp.ERR_INVALID_ARG
+    assert qp(t0=None) == sp.ERR_INVALID_ARG
+    assert qp(t0=8) == sp.ERR_ALIGN
+    # group-shared tensor scale
+    assert L.sp24_nvfp4_group_tensor_scale_workspace_size(ctypes.byref(n)) == sp.OK and n.value == 16
+    ptrs = (P * 2)(16, 32)
+    gs = lambda nums, dt=sp.BF16, out=16, wsp=256, p=ptrs: L.sp24_nvfp4_group_tensor_scale(
+        p, (ctypes.c_int64 * 2)(*nums), 2, dt, out, wsp, 16, None)
+    assert gs((64, 64), out=None) == sp.ERR_INVALID_ARG
+    assert gs((64, 64), dt=9) == sp.ERR_DTYPE
+    assert gs((64, 12)) == sp.ERR_SHAPE                                         # 24 bytes
+    assert gs((64, 64), p=(P * 2)(16, None)) == sp.ERR_INVALID_ARG
+    assert gs((64, 64), p=(P * 2)(16, 40)) == sp.ERR_ALIGN
+    assert gs((64, 64), wsp=None) == sp.ERR_WORKSPACE
+    assert L.sp24_nvfp4_group_tensor_scale(None, None, -1, sp.BF16, 16, 256, 16, None) == sp.ERR_INVALID_ARG
+    # measured selection and the auto GEMM
+    use = ctypes.c_int(-1)
+    wq = sp._Operand(sp.NVFP4, 16, 16, 16)
+    assert L.sp24_gemm_select(ctypes.byref(x16), ctypes.byref(wd), ctypes.byref(ws), 8, 8, 64, 16, None, 0, 0,
+                              ctypes.byref(use), None, None, None) == sp.ERR_INVALID_ARG   # reps < 1
+    assert L.sp24_gemm_select(ctypes.byref(x16), ctypes.byref(wq), ctypes.byref(ws), 8, 8, 64, 16, None, 0, 3,
+                              ctypes.byref(use), None, None, None) == sp.ERR_DTYPE         # forms disagree
+    assert L.sp24_gemm_select(ctypes.byref(x32), ctypes.byref(wd), ctypes.byref(ws), 8, 8, 64, 16, None, 0, 3,
+                              ctypes.byref(use), None, None, None) == sp.ERR_DTYPE         # no such pair
+    assert L.sp24_gemm_auto(ctypes.byref(x16), ctypes.byref(wd), None, 8, 8, 64, 16, None, 0, None,
+                            None) == sp.ERR_INVALID_ARG
+    assert L.sp24_gemm_auto(ctypes.byref(x16), ctypes.byref(wq), ctypes.byref(ws), 8, 8, 64, 16, None, 0, None,
+                            None) == sp.ERR_DTYPE
+    assert use.value == -1
