@@ -101,7 +101,9 @@ typedef struct {
 const char* sp24_status_string(int status);
 int sp24_abi_version(void);
 
-/* Sizes of what the pipeline produces for a tensor (host only, no device access).
+/* [P1] "The byte saving is about a quarter, not a half"; [P5] "Bit-exact check against lyf's
+ * ModelOpt output" (packed and scale bytes of real tensors).
+ * Sizes of what the pipeline produces for a tensor (host only, no device access).
  * groups: groups of four along the reduction axis; values_bytes / meta_bytes: compressed
  * form; nvfp4_codes_bytes / nvfp4_scales_bytes: dense NVFP4 of the tensor viewed as
  * [numel / L, L] with L its last axis (matmul only; 0 for conv).  Any output may be NULL. */
@@ -131,7 +133,8 @@ int sp24_check_24(const void* w, int dtype, int op, const int64_t* shape, int nd
 int sp24_prune_compress_24(const void* w, int dtype, int op, const int64_t* shape, int ndim,
                            void* values, uint8_t* meta, void* stream);
 
-/* Inverse of compression: w_out (device, dtype, `shape`) receives the kept values at their
+/* [P2] "The mechanism needs both values and their positions".
+ * Inverse of compression: w_out (device, dtype, `shape`) receives the kept values at their
  * indices and +0 elsewhere.  Nibbles must be legal (i0 < i1); an illegal nibble yields +0 in
  * its group and sets the device error word (SP24_ERR_INVALID_ARG). */
 int sp24_decompress_24(const void* values, const uint8_t* meta, int dtype, int op,
@@ -195,7 +198,8 @@ int sp24_decompress_48(const void* values, const uint8_t* meta, int dtype, int64
 int sp24_gemm_sparse48(const sp24_operand* x, const sp24_sparse_operand* w, int64_t M, int64_t N,
                        int64_t K, float* y, void* stream);
 
-/* The same GEMM on tile images (x format SP24_NVFP4_B32_MMA, w format SP24_NVFP4_MMA; both or
+/* [P1] "The ladder, top to bottom" (the sparse FP4 rate of the tensor cores).
+ * The same GEMM on tile images (x format SP24_NVFP4_B32_MMA, w format SP24_NVFP4_MMA; both or
  * neither) runs a persistent kernel on pairs of SMs (tcgen05.mma.sp.cta_group::2, 256 weight
  * rows x 256 tokens per pair tile, 512 logical K per stage).  Not on the source pages: layouts
  * of this library's kernel.
@@ -240,7 +244,8 @@ int sp24_quantize_nvfp4(const void* t, int dtype, int64_t rows, int64_t cols,
                         float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
                         void* stream);
 
-/* An NVFP4 tensor [rows, cols] (cols % 256 == 0) rewritten as the tile images the W4A4 GEMM
+/* [P1] "The ladder, top to bottom" (the dense NVFP4 GEMM at 4096^3).
+ * An NVFP4 tensor [rows, cols] (cols % 256 == 0) rewritten as the tile images the W4A4 GEMM
  * loads whole (format SP24_NVFP4_MMA): each tile lands in shared memory with one copy.  Not on
  * the source pages: a layout of this library's W4A4 kernel; the values are unchanged.
  *   codes_out:  per 128-row block rb and 256-column chunk kc a 16 KB tile at byte
@@ -277,7 +282,8 @@ int sp24_get_wait_limit(unsigned long long* ns);
 int sp24_selftest_wait_timeout(const void* src, int* out, void* stream);
 
 /* ----------------------------------------------------------------------- roofline peaks */
-/* The denominators of the roofline fractions, measured with this library's own instructions
+/* [P1] "The roofline is the whole argument".
+ * The denominators of the roofline fractions, measured with this library's own instructions
  * (not on the source pages).
  *   sp24_peak_mma   one CTA per SM (kind 4: per CTA pair) issues 4 * (rounds + 1) back-to-back
  *                   tcgen05 MMAs of N = 256 from shared-memory operands holding non-zero data,
@@ -293,7 +299,8 @@ int sp24_peak_mma(int kind, int rounds, unsigned long long* out_ns, void* stream
 int sp24_peak_ctas(int kind);
 int sp24_peak_read(const void* src, int64_t bytes, unsigned int* out, void* stream);
 
-/* The same quantisation for callers that cannot allocate device memory: runtimes that only hand
+/* [P5] "Convert BF16 to NVFP4 yourself".
+ * The same quantisation for callers that cannot allocate device memory: runtimes that only hand
  * out a fixed arena of operand buffers, plugins whose host framework owns the device allocator,
  * and host loops that must not call cudaMalloc (it can synchronise the device).  No counterpart
  * on the source pages: it is a property of this library, not of the method.
@@ -311,7 +318,8 @@ int sp24_quantize_nvfp4_noalloc(const void* t, int dtype, int64_t rows, int64_t 
                                 const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
                                 float* tensor_scale_out, void* stream);
 
-/* NVFP4 encoding with 32-value blocks: the activation operand of the sparse FP4 MMA, which
+/* [P5] "Convert BF16 to NVFP4 yourself" (the steps; its blocks hold 16 values).
+ * NVFP4 encoding with 32-value blocks: the activation operand of the sparse FP4 MMA, which
  * reads one scale per 32 K (sp24_gemm_sparse48).  The steps of sp24_quantize_nvfp4 over
  * 32 consecutive entries of a row:  s_t = tensor_scale_in ? *tensor_scale_in : amax / 2688;
  * sb = E4M3_rne_satfinite(bmax32 / (s_t * 6));  code = sign << 3 | E2M1_rne_satfinite(|t| /
@@ -323,7 +331,8 @@ int sp24_quantize_nvfp4_block32(const void* t, int dtype, int64_t rows, int64_t 
                                 float* tensor_scale_out, void* workspace, int64_t workspace_bytes,
                                 void* stream);
 
-/* Two quantisations in one launch (a weight and its 2:4 values, with the tensor scales that
+/* [P5] "Convert BF16 to NVFP4 yourself"; [P1] "The byte saving is about a quarter, not a half".
+ * Two quantisations in one launch (a weight and its 2:4 values, with the tensor scales that
  * sp24_prepare_24 derived, say): the results equal those of sp24_quantize_nvfp4(t0, ts0) and
  * sp24_quantize_nvfp4(t1, ts1).  Both tensors have type `dtype`; each tensor scale is required
  * (device fp32) and is copied to its ts_out (which may be the same pointer).  Shapes, layouts
@@ -349,7 +358,8 @@ int sp24_nvfp4_group_tensor_scale(const void* const* tensors, const int64_t* num
                                   int dtype, float* tensor_scale_out, void* workspace,
                                   int64_t workspace_bytes, void* stream);
 
-/* Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
+/* [P5] "Convert BF16 to NVFP4 yourself" (the format decoded).
+ * Decode: out[r, c] = E2M1(code) * E4M3(scale) * tensor_scale, rounded once to out_dtype
  * (F16/BF16/F32). */
 int sp24_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales,
                           const float* tensor_scale, int64_t rows, int64_t cols, int out_dtype,
@@ -424,7 +434,8 @@ int sp24_gemm_sparse24(const sp24_operand* x, const sp24_sparse_operand* w, int6
  *   sp24_gemm_choice  (host only) the recorded decision, else a rule of crossovers measured on
  *                     B200: weights of fewer than 2^20 entries dense (launch-bound); else
  *                     16-bit weights, and NVFP4 weights with 16-bit x, 2:4 for M >= 128
- *                     and dense below; NVFP4 weights with NVFP4 x dense.  *measured (may be NULL): 1 if recorded.
+ *                     and dense below; NVFP4 weights with NVFP4 x dense.
+ *                     *measured (may be NULL): 1 if recorded.
  *                     SP24_ERR_DTYPE for format pairs without a 2:4 path.
  *   sp24_gemm_auto    runs the GEMM sp24_gemm_choice names; *used_sparse (may be NULL) says
  *                     which.  Asynchronous.
@@ -488,7 +499,8 @@ int sp24_moe_block(const sp24_operand* x, const int32_t* routing, const float* r
                    const sp24_sparse_operand* w_down_sparse, int64_t E, int64_t H, int64_t F,
                    float* y, void* workspace, int64_t workspace_bytes, void* stream);
 
-/* Row interleave: out[2 * rows, row_bytes] takes block_rows rows of a, then block_rows rows of
+/* [P5] "The shared global scale" (gate and up are read together).
+ * Row interleave: out[2 * rows, row_bytes] takes block_rows rows of a, then block_rows rows of
  * b, and so on (the gate / up packing of sp24_moe_block).  rows % block_rows == 0, row_bytes % 16
  * == 0, all pointers device and 16-byte aligned. */
 int sp24_interleave_rows(const void* a, const void* b, int64_t rows, int64_t row_bytes,
